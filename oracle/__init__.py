@@ -1,0 +1,221 @@
+"""ctypes shim over the plain-C NVFP4 oracle (oracle/nvfp4_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the package smoke check and the
+benchmark's CPU-baseline leg may use this module; the product (the CUDA
+library and its binding) never imports it.  Arrays are numpy; bf16 tensors
+are passed as their uint16 bit patterns.  The oracle's arithmetic lives in
+the C file; this module only marshals arguments.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        _lib = ctypes.CDLL(path)
+        L = _lib
+        i64, f32, f64, i32 = ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_int
+        vp = ctypes.c_void_p
+        L.oracle_e2m1_value.restype = f64
+        L.oracle_e2m1_value.argtypes = [i32]
+        L.oracle_e4m3_value.restype = f64
+        L.oracle_e4m3_value.argtypes = [i32]
+        L.oracle_e2m1_encode.restype = i32
+        L.oracle_e2m1_encode.argtypes = [f64, f64]
+        L.oracle_e4m3_round_quotient.restype = i32
+        L.oracle_e4m3_round_quotient.argtypes = [f64, f64]
+        L.oracle_effective_scale.restype = f32
+        L.oracle_effective_scale.argtypes = [f32, i32]
+        L.oracle_float_to_bf16.restype = ctypes.c_uint16
+        L.oracle_float_to_bf16.argtypes = [f32]
+        L.oracle_global_scale.argtypes = [vp, i64, vp]
+        L.oracle_max_rule_code.argtypes = [vp, f32]
+        L.oracle_scale_search_max.argtypes = [vp, i64, i64, f32, vp]
+        L.oracle_block_mse.restype = f64
+        L.oracle_block_mse.argtypes = [vp, f32, i32]
+        L.oracle_block_lh.restype = f64
+        L.oracle_block_lh.argtypes = [vp, f32, i32, vp]
+        L.oracle_block_objectives.argtypes = [vp, f32, vp, vp]
+        L.oracle_scale_search_mse.argtypes = [vp, i64, i64, f32, vp, vp]
+        L.oracle_scale_search_lh.argtypes = [vp, i64, i64, f32, vp, vp, vp]
+        L.oracle_scale_search_sampled.argtypes = [vp, i64, f32, vp, vp, vp, i64, vp, vp]
+        L.oracle_gram_accumulate.argtypes = [vp, i64, i64, vp]
+        L.oracle_gram_accumulate_grouped.argtypes = [vp, vp, i64, i64, vp]
+        L.oracle_quantize_pack.argtypes = [vp, i64, i64, f32, vp, vp]
+        L.oracle_dequantize.argtypes = [vp, vp, f32, i64, i64, vp]
+        L.oracle_fake_quant.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+        L.oracle_max_threads.restype = i32
+    return _lib
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("bf16 data must be passed as uint16 bit patterns")
+    return a
+
+
+def _check(st):
+    if st != 0:
+        raise OracleError("oracle status %d" % st)
+
+
+def max_threads():
+    return lib().oracle_max_threads()
+
+
+# ------------------------------------------------------------ scalar helpers
+def e2m1_value(code):
+    return lib().oracle_e2m1_value(int(code))
+
+
+def e4m3_value(code):
+    return lib().oracle_e4m3_value(int(code))
+
+
+def e2m1_encode(x, s):
+    return lib().oracle_e2m1_encode(float(x), float(s))
+
+
+def e4m3_round_quotient(num, den):
+    return lib().oracle_e4m3_round_quotient(float(num), float(den))
+
+
+def effective_scale(s_g, code):
+    return lib().oracle_effective_scale(float(s_g), int(code))
+
+
+def float_to_bf16(f):
+    return lib().oracle_float_to_bf16(float(f))
+
+
+# ------------------------------------------------------------ tensor ops
+def global_scale(x_u16):
+    x = _u16(x_u16)
+    out = ctypes.c_float()
+    _check(lib().oracle_global_scale(_ptr(x), x.size, ctypes.byref(out)))
+    return np.float32(out.value)
+
+
+def scale_search_max(w_u16, s_g):
+    w = _u16(w_u16)
+    R, C = w.shape
+    codes = np.zeros((R, C // 16), np.uint8)
+    _check(lib().oracle_scale_search_max(_ptr(w), R, C, float(s_g), _ptr(codes)))
+    return codes
+
+
+def scale_search_mse(w_u16, s_g):
+    w = _u16(w_u16)
+    R, C = w.shape
+    codes = np.zeros((R, C // 16), np.uint8)
+    best = np.zeros((R, C // 16), np.float64)
+    _check(lib().oracle_scale_search_mse(_ptr(w), R, C, float(s_g), _ptr(codes), _ptr(best)))
+    return codes, best
+
+
+def scale_search_lh(w_u16, s_g, H):
+    w = _u16(w_u16)
+    R, C = w.shape
+    H = np.ascontiguousarray(H, dtype=np.float64).reshape(C // 16, 16, 16)
+    codes = np.zeros((R, C // 16), np.uint8)
+    best = np.zeros((R, C // 16), np.float64)
+    _check(lib().oracle_scale_search_lh(_ptr(w), R, C, float(s_g), _ptr(H), _ptr(codes),
+                                        _ptr(best)))
+    return codes, best
+
+
+def scale_search_sampled(w_u16, s_g, H, rows, blocks):
+    """Search only the blocks (rows[i], blocks[i]); H=None selects MSE."""
+    w = _u16(w_u16)
+    C = w.shape[-1]
+    rows = np.ascontiguousarray(rows, np.int64)
+    blocks = np.ascontiguousarray(blocks, np.int64)
+    if H is not None:
+        H = np.ascontiguousarray(H, dtype=np.float64).reshape(C // 16, 16, 16)
+    codes = np.zeros(rows.size, np.uint8)
+    best = np.zeros(rows.size, np.float64)
+    _check(lib().oracle_scale_search_sampled(_ptr(w), C, float(s_g), _ptr(H), _ptr(rows),
+                                             _ptr(blocks), rows.size, _ptr(codes), _ptr(best)))
+    return codes, best
+
+
+def block_objectives(blk_u16, s_g, Hb=None):
+    """All 126 objectives of one 16-element block (index c-1)."""
+    b = _u16(blk_u16).reshape(16)
+    out = np.zeros(126, np.float64)
+    if Hb is not None:
+        Hb = np.ascontiguousarray(Hb, dtype=np.float64).reshape(16, 16)
+    lib().oracle_block_objectives(_ptr(b), float(s_g), _ptr(Hb), _ptr(out))
+    return out
+
+
+def max_rule_code(blk_u16, s_g):
+    b = _u16(blk_u16).reshape(16)
+    return lib().oracle_max_rule_code(_ptr(b), ctypes.c_float(float(s_g)))
+
+
+def gram(x_u16, H=None):
+    x = _u16(x_u16)
+    N, C = x.shape
+    if H is None:
+        H = np.zeros((C // 16, 16, 16), np.float64)
+    else:
+        H = np.ascontiguousarray(H, np.float64).copy()
+    _check(lib().oracle_gram_accumulate(_ptr(x), N, C, _ptr(H)))
+    return H
+
+
+def gram_grouped(x_u16, offsets, G):
+    x = _u16(x_u16)
+    C = x.shape[-1]
+    offsets = np.ascontiguousarray(offsets, np.int64)
+    H = np.zeros((G, C // 16, 16, 16), np.float64)
+    _check(lib().oracle_gram_accumulate_grouped(_ptr(x), _ptr(offsets), G, C, _ptr(H)))
+    return H
+
+
+def quantize_pack(w_u16, s_g, codes):
+    w = _u16(w_u16)
+    R, C = w.shape
+    codes = np.ascontiguousarray(codes, np.uint8)
+    packed = np.zeros((R, C // 2), np.uint8)
+    _check(lib().oracle_quantize_pack(_ptr(w), R, C, float(s_g), _ptr(codes), _ptr(packed)))
+    return packed
+
+
+def dequantize(packed, codes, s_g):
+    packed = np.ascontiguousarray(packed, np.uint8)
+    codes = np.ascontiguousarray(codes, np.uint8)
+    R, C = packed.shape[0], packed.shape[1] * 2
+    out = np.zeros((R, C), np.uint16)
+    _check(lib().oracle_dequantize(_ptr(packed), _ptr(codes), float(s_g), R, C, _ptr(out)))
+    return out
+
+
+def fake_quant(x_u16, want_packed=True):
+    x = _u16(x_u16)
+    R, C = x.shape
+    out = np.zeros((R, C), np.uint16)
+    packed = np.zeros((R, C // 2), np.uint8) if want_packed else None
+    codes = np.zeros((R, C // 16), np.uint8) if want_packed else None
+    s_g = ctypes.c_float()
+    _check(lib().oracle_fake_quant(_ptr(x), R, C, _ptr(out), _ptr(packed), _ptr(codes),
+                                   ctypes.byref(s_g)))
+    return out, packed, codes, np.float32(s_g.value)

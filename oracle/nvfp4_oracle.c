@@ -1,0 +1,475 @@
+/*
+ * NVFP4 scale-calibration ORACLE — plain, slow, scalar CPU reference.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product (the CUDA library and its
+ * Python binding) may include, link, load or call this file.  Only the test
+ * suite, the smoke check of the package entry point and the CPU-baseline leg of
+ * the benchmark use it.  It shares no code, header, table or helper with the
+ * CUDA path: every table below is written out here from the format
+ * definitions, independently.
+ *
+ * Arithmetic: fp64 throughout (bf16 inputs are exact in double), except where
+ * the method itself fixes an fp32 quantity (the tensor scale s_g, the
+ * effective block scale s_eff and the dequantised value before its bf16
+ * rounding); those are formed with single IEEE float operations.
+ *
+ * Sources (cited by page title and section):
+ *   [QAD]   "為什么NVFP4推理精度會掉以及QAD到底在修什么" (czchanglian.com),
+ *           sections 2.1, 2.3, 3.2, 4.2.
+ *   [BT]    Baseten engineering blog, "What makes high-quality NVFP4"
+ *           (Chinese copy on attain.fans), sections "Why do we need scales?",
+ *           "Block scaling: one scale per 16 values", "Why blocks?",
+ *           "Calibration".
+ *   [LH]    "4 比特量化到底让模型笨了多少？" (2kiu.com), a write-up of NVIDIA
+ *           Model Optimizer's "Improving NVFP4 Accuracy with Local-Hessian
+ *           Weight Scales"; sections "The NVFP4 structure" and "A different
+ *           objective: output error as the ruler".
+ *
+ * Readings where the pages are silent (each is also listed in the design
+ * notes): the tensor scale s_g = fl32(amax / (6*448)) (1 when amax = 0);
+ * round-to-nearest-even and saturation for both E2M1 and E4M3; the sign of
+ * a value that rounds to zero is kept (code 0x8 for negative inputs); ties
+ * in a scale search keep the smallest code; element 2j of a row goes into the
+ * low nibble of byte j; dequantisation rounds v*s_eff to fp32 and then to
+ * bf16, both to nearest even.
+ *
+ * Parity pins: every exported function is pinned by a test that does not go
+ * through this file's arithmetic (brute-force enumeration with exact
+ * rationals, the worked example of [BT], the trace identity of [LH], the
+ * H = I and C = 16 special cases, library Gram products on tiny inputs).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_SHAPE 2
+#define ORACLE_ERR_NONFINITE 4
+
+/* ---------------------------------------------------------------- formats */
+
+/* E2M1 magnitudes by 3-bit magnitude index k = code & 7 ([BT] "Why do we
+ * need scales?" lists the 16 representable values; [LH] "The NVFP4
+ * structure" gives the 1 sign / 2 exponent / 1 mantissa split). */
+static const double E2M1_MAGNITUDE[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double oracle_e2m1_value(int code)
+{
+    double m = E2M1_MAGNITUDE[code & 7];
+    return (code & 8) ? -m : m;
+}
+
+/* E4M3 (the FN variant: no infinities, 0x7F is NaN): 1 sign, 4 exponent bits
+ * with bias 7, 3 mantissa bits; exponent field 0 is subnormal, m * 2^-9.
+ * [LH] "The NVFP4 structure": each block carries one FP8 scale.  126 of the
+ * codes (0x01..0x7E) are positive, finite and non-zero, which is the
+ * candidate count of the MSE search in [LH]. */
+double oracle_e4m3_value(int code)
+{
+    int e = (code >> 3) & 0xF;
+    int m = code & 7;
+    double v;
+    if ((code & 0x7F) == 0x7F)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+    return (code & 0x80) ? -v : v;
+}
+
+double oracle_bf16_to_double(uint16_t h)
+{
+    uint32_t bits = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &bits, 4);
+    return (double)f;
+}
+
+/* fp32 -> bf16, round to nearest even (finite inputs). */
+uint16_t oracle_float_to_bf16(float f)
+{
+    uint32_t bits;
+    memcpy(&bits, &f, 4);
+    if ((bits & 0x7F800000u) == 0x7F800000u) /* inf / nan: truncate, keep nan quiet */
+        return (uint16_t)((bits >> 16) | ((bits & 0xFFFF) ? 0x40 : 0));
+    uint32_t lsb = (bits >> 16) & 1u;
+    bits += 0x7FFFu + lsb;
+    return (uint16_t)(bits >> 16);
+}
+
+/* Effective block scale: the FP8 block scale times the FP32 tensor scale,
+ * formed as one fp32 multiply ([BT] "Why do we need scales?": NVFP4 has a
+ * tensor-level FP32 scale on top of the block scale). */
+float oracle_effective_scale(float s_g, int code)
+{
+    float e = (float)oracle_e4m3_value(code); /* exact: <= 4 significant bits */
+    return s_g * e;
+}
+
+/* --------------------------------------------------------- E2M1 rounding */
+
+/* Round x / s onto the E2M1 grid: nearest magnitude, ties to the even
+ * magnitude index (round-to-nearest-even on the 1-bit mantissa), saturating
+ * at 6; s = 0 gives magnitude 0.  The decision compares |x| with each
+ * midpoint times s; both products are exact in double (the midpoints have at
+ * most 3 significant bits and s has 24), so the exact quotient is rounded,
+ * not an fp32 approximation of it.  [QAD] section 2.1: a value between two
+ * representable values goes to the nearer one.  [BT] "Why blocks?": with
+ * scale 14, everything below 3.5 becomes 0. */
+int oracle_e2m1_encode(double x, double s)
+{
+    int sign = signbit(x) ? 8 : 0;
+    double a = fabs(x);
+    int k = 0;
+    if (s > 0.0) {
+        for (int i = 0; i < 7; i++) {
+            double mid = 0.5 * (E2M1_MAGNITUDE[i] + E2M1_MAGNITUDE[i + 1]);
+            double thr = mid * s;
+            /* between index i and i+1 a tie goes to the even index */
+            int up = (i % 2 == 0) ? (a > thr) : (a >= thr);
+            if (up)
+                k = i + 1;
+        }
+    }
+    return sign | k;
+}
+
+/* ------------------------------------------------------- E4M3 rounding */
+
+/* Round the exact quotient num/den (num >= 0, den > 0) to E4M3 with
+ * round-to-nearest-even and saturation to the largest finite value 448
+ * (code 0x7E).  Ties between codes c and c+1 go to the even code.  The
+ * caller guarantees that midpoint*den is exact in double (midpoints have at
+ * most 5 significant bits). */
+int oracle_e4m3_round_quotient(double num, double den)
+{
+    int code = 0;
+    for (int c = 0; c < 126; c++) {
+        double mid = 0.5 * (oracle_e4m3_value(c) + oracle_e4m3_value(c + 1));
+        double thr = mid * den;
+        int up = (c % 2 == 0) ? (num > thr) : (num >= thr);
+        if (up)
+            code = c + 1;
+    }
+    return code;
+}
+
+/* --------------------------------------------------------- global scale */
+
+/* Tensor amax -> FP32 tensor scale s_g = fl32(amax / 2688), 2688 = 6 * 448,
+ * so that the largest E4M3 block scale (448) maps the tensor's largest
+ * value onto the largest E2M1 magnitude (6).  amax = 0 gives s_g = 1.
+ * [BT] "Why do we need scales?" (the FP32 tensor scale exists; its formula
+ * is this reading).  Non-finite input is an error. */
+int oracle_global_scale(const uint16_t *x, int64_t n, float *s_g)
+{
+    double amax = 0.0;
+    for (int64_t i = 0; i < n; i++) {
+        double v = oracle_bf16_to_double(x[i]);
+        if (!isfinite(v))
+            return ORACLE_ERR_NONFINITE;
+        if (fabs(v) > amax)
+            amax = fabs(v);
+    }
+    if (amax == 0.0) {
+        *s_g = 1.0f;
+    } else {
+        float a = (float)amax;        /* exact: a bf16 value */
+        *s_g = a / 2688.0f;           /* one IEEE fp32 division */
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------ max rule */
+
+/* Max scaling: block scale = block amax / 6 relative to s_g, rounded to
+ * E4M3 (RNE, saturating at 448, which is the clamp to the FP8 maximum of
+ * [QAD] section 4.2).  An all-zero block gets code 0.  [QAD] section 2.3
+ * (step M/6); [BT] "Why blocks?" (84 / 6 = 14) and "Calibration"
+ * (activations use the block max); [LH] "The NVFP4 structure" (max scaling
+ * is the default). */
+int oracle_max_rule_code(const uint16_t *blk, float s_g)
+{
+    double amax = 0.0;
+    for (int i = 0; i < 16; i++) {
+        double v = fabs(oracle_bf16_to_double(blk[i]));
+        if (v > amax)
+            amax = v;
+    }
+    if (amax == 0.0)
+        return 0;
+    return oracle_e4m3_round_quotient(amax, 6.0 * (double)s_g);
+}
+
+int oracle_scale_search_max(const uint16_t *w, int64_t R, int64_t C, float s_g,
+                            uint8_t *codes)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    int64_t nb = C / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t b = 0; b < nb; b++)
+            codes[r * nb + b] = (uint8_t)oracle_max_rule_code(w + r * C + b * 16, s_g);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------- objectives and searches */
+
+/* Quantisation error of one block for candidate code c:
+ * delta_i = w_i - v(q_i) * s_eff(c), with q_i the E2M1 code of w_i / s_eff. */
+static void block_delta(const uint16_t *blk, float s_g, int c, double delta[16])
+{
+    double s = (double)oracle_effective_scale(s_g, c);
+    for (int i = 0; i < 16; i++) {
+        double w = oracle_bf16_to_double(blk[i]);
+        int q = oracle_e2m1_encode(w, s);
+        delta[i] = w - oracle_e2m1_value(q) * s;
+    }
+}
+
+/* MSE objective: sum of squared weight errors ([LH] "The NVFP4 structure":
+ * the MSE method tries all 126 positive non-zero FP8 scales and keeps the
+ * one with the smallest weight error). */
+double oracle_block_mse(const uint16_t *blk, float s_g, int c)
+{
+    double d[16], e = 0.0;
+    block_delta(blk, s_g, c, d);
+    for (int i = 0; i < 16; i++)
+        e += d[i] * d[i];
+    return e;
+}
+
+/* Local-Hessian objective E = delta H_b delta^T with the 16x16 diagonal block
+ * H_b of the calibration Gram matrix ([LH] "A different objective":
+ * E(s) = ||delta X||^2 = tr(delta X X^T delta^T), block-diagonal
+ * approximation, exhaustive over the 126 candidates per block). */
+double oracle_block_lh(const uint16_t *blk, float s_g, int c, const double *Hb)
+{
+    double d[16], e = 0.0;
+    block_delta(blk, s_g, c, d);
+    for (int j = 0; j < 16; j++)
+        for (int k = 0; k < 16; k++)
+            e += d[j] * Hb[j * 16 + k] * d[k];
+    return e;
+}
+
+/* Exhaustive search over codes 1..126; the first (smallest) code reaching
+ * the minimum wins.  Hb == NULL selects the MSE objective. */
+static int search_block(const uint16_t *blk, float s_g, const double *Hb, double *best)
+{
+    int best_c = 1;
+    double best_e = INFINITY;
+    for (int c = 1; c <= 126; c++) {
+        double e = Hb ? oracle_block_lh(blk, s_g, c, Hb) : oracle_block_mse(blk, s_g, c);
+        if (e < best_e) {
+            best_e = e;
+            best_c = c;
+        }
+    }
+    if (best)
+        *best = best_e;
+    return best_c;
+}
+
+/* Objectives of all 126 candidates of one block (index c-1), for tie
+ * analysis in the tests. */
+void oracle_block_objectives(const uint16_t *blk, float s_g, const double *Hb, double *out126)
+{
+    for (int c = 1; c <= 126; c++)
+        out126[c - 1] = Hb ? oracle_block_lh(blk, s_g, c, Hb) : oracle_block_mse(blk, s_g, c);
+}
+
+int oracle_scale_search_mse(const uint16_t *w, int64_t R, int64_t C, float s_g,
+                            uint8_t *codes, double *best_obj)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    int64_t nb = C / 16;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t b = 0; b < nb; b++) {
+            double e;
+            codes[r * nb + b] = (uint8_t)search_block(w + r * C + b * 16, s_g, NULL, &e);
+            if (best_obj)
+                best_obj[r * nb + b] = e;
+        }
+    return ORACLE_OK;
+}
+
+/* H: [C/16][16][16] (row-major 16x16 per column block), shared by all rows. */
+int oracle_scale_search_lh(const uint16_t *w, int64_t R, int64_t C, float s_g,
+                           const double *H, uint8_t *codes, double *best_obj)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    int64_t nb = C / 16;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t b = 0; b < nb; b++) {
+            double e;
+            codes[r * nb + b] = (uint8_t)search_block(w + r * C + b * 16, s_g, H + b * 256, &e);
+            if (best_obj)
+                best_obj[r * nb + b] = e;
+        }
+    return ORACLE_OK;
+}
+
+/* Same search restricted to a list of (row, column-block) pairs, for parity
+ * on samples of large layers. */
+int oracle_scale_search_sampled(const uint16_t *w, int64_t C, float s_g, const double *H,
+                                const int64_t *rows, const int64_t *blocks, int64_t n,
+                                uint8_t *codes, double *best_obj)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t i = 0; i < n; i++) {
+        double e;
+        const double *Hb = H ? H + blocks[i] * 256 : NULL;
+        codes[i] = (uint8_t)search_block(w + rows[i] * C + blocks[i] * 16, s_g, Hb, &e);
+        if (best_obj)
+            best_obj[i] = e;
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------- Gram */
+
+/* Block-diagonal Gram accumulation: for every column block j,
+ * H[j] += sum_t x[t, 16j:16j+16]^T x[t, 16j:16j+16], in fp64.  x is
+ * tokens-by-channels ([LH] writes Y = W X with X channels-by-tokens; this is
+ * the same product with X transposed).  [LH] "A different objective": only
+ * the 16x16 diagonal blocks of X X^T are kept. */
+int oracle_gram_accumulate(const uint16_t *x, int64_t n_tok, int64_t C, double *H)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    int64_t nb = C / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < nb; j++) {
+        double *Hj = H + j * 256;
+        for (int64_t t = 0; t < n_tok; t++) {
+            const uint16_t *row = x + t * C + j * 16;
+            double v[16];
+            for (int a = 0; a < 16; a++)
+                v[a] = oracle_bf16_to_double(row[a]);
+            for (int a = 0; a < 16; a++)
+                for (int b = 0; b < 16; b++)
+                    Hj[a * 16 + b] += v[a] * v[b];
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Grouped form (experts): tokens offsets[g]..offsets[g+1] accumulate into
+ * H[g]. */
+int oracle_gram_accumulate_grouped(const uint16_t *x, const int64_t *offsets, int64_t G,
+                                   int64_t C, double *H)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    for (int64_t g = 0; g < G; g++) {
+        int64_t n = offsets[g + 1] - offsets[g];
+        int st = oracle_gram_accumulate(x + offsets[g] * C, n, C, H + g * (C / 16) * 256);
+        if (st)
+            return st;
+    }
+    return ORACLE_OK;
+}
+
+/* ----------------------------------------------------- pack / dequant */
+
+/* E2M1 codes of a row-major [R, C] tensor given block codes, two codes per
+ * byte: element 2j in the low nibble of byte j, element 2j+1 in the high
+ * nibble ([BT] "Where quantisation helps": FP4 takes half a byte per value;
+ * the nibble order is this reading). */
+int oracle_quantize_pack(const uint16_t *w, int64_t R, int64_t C, float s_g,
+                         const uint8_t *codes, uint8_t *packed)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    int64_t nb = C / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t i = 0; i < C; i += 2) {
+            double s = (double)oracle_effective_scale(s_g, codes[r * nb + i / 16]);
+            int q0 = oracle_e2m1_encode(oracle_bf16_to_double(w[r * C + i]), s);
+            int q1 = oracle_e2m1_encode(oracle_bf16_to_double(w[r * C + i + 1]), s);
+            packed[r * (C / 2) + i / 2] = (uint8_t)(q0 | (q1 << 4));
+        }
+    return ORACLE_OK;
+}
+
+/* y = bf16_rn(fl32(v(q) * s_eff)) ([QAD] section 3.2: the dequantised value
+ * is the E2M1 value times the scale). */
+int oracle_dequantize(const uint8_t *packed, const uint8_t *codes, float s_g, int64_t R,
+                      int64_t C, uint16_t *out)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    int64_t nb = C / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t i = 0; i < C; i++) {
+            uint8_t byte = packed[r * (C / 2) + i / 2];
+            int q = (i & 1) ? (byte >> 4) : (byte & 0xF);
+            float s = oracle_effective_scale(s_g, codes[r * nb + i / 16]);
+            float y = (float)oracle_e2m1_value(q) * s; /* one fp32 multiply */
+            out[r * C + i] = oracle_float_to_bf16(y);
+        }
+    return ORACLE_OK;
+}
+
+/* Dynamic activation fake-quant (W4A4): tensor scale from the whole
+ * activation, then per 16 consecutive channels of each token the max rule,
+ * E2M1 encode and dequantise ([BT] "Calibration": activation blocks of 16
+ * use their absolute maximum; [QAD] section 3.2: reshape into blocks of 16,
+ * scale by the block max over 6, quantise, dequantise).  packed and codes
+ * may be NULL. */
+int oracle_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16_t *out,
+                      uint8_t *packed, uint8_t *codes, float *s_g_out)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    float s_g;
+    int st = oracle_global_scale(x, rows * C, &s_g);
+    if (st)
+        return st;
+    *s_g_out = s_g;
+    int64_t nb = C / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t b = 0; b < nb; b++) {
+            const uint16_t *blk = x + r * C + b * 16;
+            int c = oracle_max_rule_code(blk, s_g);
+            float s = oracle_effective_scale(s_g, c);
+            if (codes)
+                codes[r * nb + b] = (uint8_t)c;
+            for (int i = 0; i < 16; i++) {
+                int q = oracle_e2m1_encode(oracle_bf16_to_double(blk[i]), (double)s);
+                float y = (float)oracle_e2m1_value(q) * s;
+                out[r * C + b * 16 + i] = oracle_float_to_bf16(y);
+                if (packed) {
+                    int64_t idx = r * (C / 2) + (b * 16 + i) / 2;
+                    if (i & 1)
+                        packed[idx] = (uint8_t)(packed[idx] | (q << 4));
+                    else
+                        packed[idx] = (uint8_t)q;
+                }
+            }
+        }
+    return ORACLE_OK;
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

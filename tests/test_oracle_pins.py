@@ -1,0 +1,362 @@
+"""Pins for the CPU oracle: each check compares the oracle with something other
+than its own arithmetic — values printed on the source pages (tests/golden),
+exact-rational brute force, an independent library decode, the trace identity
+of the Local-Hessian objective, and its special cases (H = I, one block).
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import bf16_bits, bits_to_f64, f32_to_bf16_bits
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def read_golden(name):
+    rows = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            rows.setdefault(key, []).append(vals)
+    return rows
+
+
+# ------------------------------------------------------------ value sets
+def test_e2m1_value_set_matches_page(oracle_mod):
+    g = read_golden("e2m1_values.txt")
+    mags = [float(v) for v in g["magnitudes"][0]]
+    vals = [oracle_mod.e2m1_value(c) for c in range(16)]
+    assert len(vals) == int(g["codes"][0][0])
+    assert sorted({abs(v) for v in vals}) == sorted(mags)
+    assert sorted(set(vals)) == sorted(set(mags) | {-m for m in mags})
+    # the sign bit is bit 3 and the magnitude code orders the values
+    for c in range(8):
+        assert oracle_mod.e2m1_value(c) == mags[c]
+        assert oracle_mod.e2m1_value(c | 8) == -mags[c]
+        assert math.copysign(1.0, oracle_mod.e2m1_value(8)) == -1.0
+
+
+def test_e4m3_decode_matches_torch_float8(oracle_mod):
+    # independent decode: torch's float8_e4m3fn dtype
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for c in range(256):
+        o = oracle_mod.e4m3_value(c)
+        if math.isnan(ref[c]):
+            assert math.isnan(o)
+        else:
+            assert o == ref[c], c
+
+
+def test_candidate_count_126(oracle_mod):
+    g = read_golden("candidates.txt")
+    vals = [oracle_mod.e4m3_value(c) for c in range(256)]
+    pos = [v for v in vals if math.isfinite(v) and v > 0]
+    assert len(pos) == int(g["candidates"][0][0]) == 126
+    cand = [oracle_mod.e4m3_value(c) for c in range(1, 127)]
+    assert cand == sorted(pos)
+    assert all(b > a for a, b in zip(cand, cand[1:]))
+    assert cand[0] == 2.0 ** -9 and cand[-1] == 448.0
+    assert oracle_mod.e4m3_value(0x56) == 14.0
+
+
+# ------------------------------------------------------------ E2M1 rounding
+E2M1_MAG = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2),
+            Fraction(3), Fraction(4), Fraction(6)]
+
+
+def brute_e2m1(x: float, s: float) -> int:
+    """Nearest E2M1 magnitude to |x|/s by enumeration with exact rationals;
+    ties to the even magnitude index; s = 0 gives 0; sign kept."""
+    sign = 8 if math.copysign(1.0, x) < 0 else 0
+    if s == 0:
+        return sign
+    q = abs(Fraction(x)) / Fraction(s)
+    best, best_d = None, None
+    for k, v in enumerate(E2M1_MAG):
+        d = abs(q - v)
+        if best is None or d < best_d or (d == best_d and k % 2 == 0):
+            best, best_d = k, d
+    return sign | best
+
+
+def all_finite_bf16():
+    u = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    f = bits_to_f64(u)
+    return f[np.isfinite(f)]
+
+
+@pytest.mark.parametrize("s", [1.0, 14.0, 2.0 ** -5, 0.0078125 * 3, 1.1920929e-07 * 1.5,
+                               float(np.float32(0.0123456)), float(np.float32(3.3e-3))])
+def test_e2m1_encode_brute_force_all_bf16(oracle_mod, s):
+    s = float(np.float32(s))
+    xs = all_finite_bf16()
+    # every finite bf16 at this scale; exact rationals make this the slow reference
+    step = 1 if s in (1.0, 14.0) else 7
+    for x in xs[::step]:
+        assert oracle_mod.e2m1_encode(x, s) == brute_e2m1(float(x), s), (x, s)
+
+
+def test_e2m1_encode_exact_midpoints_and_saturation(oracle_mod):
+    s = float(np.float32(0.75))
+    for k in range(7):
+        mid = (E2M1_MAG[k] + E2M1_MAG[k + 1]) / 2
+        x = float(mid * Fraction(s))
+        expect = k if k % 2 == 0 else k + 1
+        assert oracle_mod.e2m1_encode(x, s) == expect
+        assert oracle_mod.e2m1_encode(-x, s) == 8 | expect
+    assert oracle_mod.e2m1_encode(1e30, s) == 7
+    assert oracle_mod.e2m1_encode(-0.0, s) == 8
+    assert oracle_mod.e2m1_encode(0.0, s) == 0
+    assert oracle_mod.e2m1_encode(5.0, 0.0) == 0
+
+
+# ------------------------------------------------------------ E4M3 rounding
+def e4m3_table():
+    codes = torch.arange(127, dtype=torch.int32).to(torch.uint8)
+    return [Fraction(float(v)) for v in codes.view(torch.float8_e4m3fn).to(torch.float64)]
+
+
+def brute_e4m3(q: Fraction, table) -> int:
+    """Nearest of the 127 non-negative finite E4M3 values (code 0..126),
+    ties to the even code, anything above 448 saturates to 448."""
+    best, best_d = None, None
+    for c, v in enumerate(table):
+        d = abs(q - v)
+        if best is None or d < best_d or (d == best_d and c % 2 == 0):
+            best, best_d = c, d
+    return best
+
+
+def test_e4m3_rounding_brute_force(oracle_mod):
+    table = e4m3_table()
+    rng = np.random.default_rng(7)
+    nums = []
+    # every midpoint, exactly, and just around it
+    for c in range(126):
+        mid = (table[c] + table[c + 1]) / 2
+        nums += [mid, mid * (1 + Fraction(1, 2 ** 40)), mid * (1 - Fraction(1, 2 ** 40))]
+    nums += [Fraction(float(v)) for v in np.exp2(rng.uniform(-14, 10, 3000))]
+    nums += [Fraction(0), Fraction(1, 2 ** 11), Fraction(448), Fraction(464), Fraction(10 ** 6)]
+    for q in nums:
+        den = 1.0
+        num = float(q)
+        if Fraction(num) != q:  # keep the quotient exact: scale the denominator instead
+            den = float(Fraction(1, 2 ** 50))
+            num = float(q * Fraction(1, 2 ** 50))
+            assert Fraction(num) / Fraction(den) == q
+        assert oracle_mod.e4m3_round_quotient(num, den) == brute_e4m3(q, table), float(q)
+
+
+# ------------------------------------------------------------ worked example
+def test_worked_example_84(oracle_mod):
+    g = read_golden("worked_example_84.txt")
+    amax = float(g["amax"][0][0])
+    scale = float(g["scale"][0][0])
+    levels = [float(v) for v in g["levels"][0]]
+    zero_below = float(g["zero_below"][0][0])
+    blk = np.array([amax, 1, 2, 1.5, 1, 2, 1, 1.25, 2, 1, 1.5, 2, 1, 2, 1, 2], np.float32)
+    u = f32_to_bf16_bits(blk)
+    s_g = oracle_mod.global_scale(u)
+    assert s_g == np.float32(amax / 2688.0) == np.float32(2.0 ** -5)
+    code = oracle_mod.max_rule_code(u, s_g)
+    assert code == 0x7E
+    s_eff = oracle_mod.effective_scale(s_g, code)
+    assert s_eff == scale
+    # every level is reachable and reproduces itself
+    for lv in levels:
+        q = oracle_mod.e2m1_encode(lv, s_eff)
+        assert oracle_mod.e2m1_value(q) * s_eff == lv
+    got = sorted({abs(oracle_mod.e2m1_value(q)) * s_eff for q in range(16)})
+    assert got == levels
+    # the small values of the example all become 0; 3.5 is the boundary
+    for v in [1.0, 1.5, 2.0, zero_below]:
+        assert oracle_mod.e2m1_encode(v, s_eff) == 0
+    assert oracle_mod.e2m1_encode(float(np.nextafter(np.float32(zero_below), 9)), s_eff) == 1
+    # with a unit tensor scale the same block gets FP8 code 0x56 (= 14)
+    assert oracle_mod.max_rule_code(u, 1.0) == 0x56
+    # dequantised block: 84 stays 84, the rest are 0
+    codes = np.array([[code]], np.uint8)
+    packed = oracle_mod.quantize_pack(u.reshape(1, 16), s_g, codes)
+    deq = bits_to_f64(oracle_mod.dequantize(packed, codes, s_g)).ravel()
+    assert deq[0] == amax and np.all(deq[1:] == 0)
+
+
+def test_global_scale_reading(oracle_mod):
+    assert oracle_mod.global_scale(np.zeros(32, np.uint16)) == np.float32(1.0)
+    x = f32_to_bf16_bits(np.array([0.5, -3.0, 2.0], np.float32))
+    assert oracle_mod.global_scale(x) == np.float32(3.0) / np.float32(2688.0)
+    bad = f32_to_bf16_bits(np.array([1.0, np.inf], np.float32))
+    with pytest.raises(Exception):
+        oracle_mod.global_scale(bad)
+
+
+def test_effective_scale_is_fp32_product(oracle_mod):
+    rng = np.random.default_rng(1)
+    for s_g in rng.uniform(1e-4, 1e-1, 20).astype(np.float32):
+        for c in (1, 7, 8, 0x38, 0x56, 0x7E):
+            e = np.float32(float(torch.tensor([c], dtype=torch.uint8)
+                                 .view(torch.float8_e4m3fn).float()))
+            assert oracle_mod.effective_scale(s_g, c) == np.float32(s_g * e)
+
+
+# ------------------------------------------------------------ Local-Hessian
+def _tiny_layer(R, C, N, seed):
+    g = torch.Generator().manual_seed(seed)
+    W = (torch.randn(R, C, generator=g) * 0.02).to(torch.bfloat16)
+    X = torch.randn(N, C, generator=g)
+    X[:, 3] *= 20.0
+    X = X.to(torch.bfloat16)
+    return bf16_bits(W), bf16_bits(X)
+
+
+def test_gram_matches_library_product(oracle_mod):
+    W, X = _tiny_layer(8, 48, 40, 3)
+    H = oracle_mod.gram(X)
+    Xf = bits_to_f64(X)
+    for j in range(3):
+        Xb = Xf[:, 16 * j:16 * j + 16]
+        np.testing.assert_allclose(H[j], Xb.T @ Xb, rtol=1e-15, atol=0)
+    # accumulation: two halves add up to the whole
+    H2 = oracle_mod.gram(X[20:], oracle_mod.gram(X[:20]))
+    np.testing.assert_allclose(H2, H, rtol=1e-15)
+
+
+def test_lh_objective_equals_output_error_norm(oracle_mod):
+    """E(s) = delta H delta^T equals ||X_b delta^T||^2 computed straight from X."""
+    W, X = _tiny_layer(6, 64, 48, 5)
+    Xf = bits_to_f64(X)
+    Wf = bits_to_f64(W)
+    H = oracle_mod.gram(X)
+    s_g = oracle_mod.global_scale(W)
+    for r in range(W.shape[0]):
+        for b in range(4):
+            blk = W[r, 16 * b:16 * b + 16]
+            E = oracle_mod.block_objectives(blk, s_g, H[b])
+            for c in (1, 30, 60, 90, 100, 110, 118, 126):
+                s = float(oracle_mod.effective_scale(s_g, c))
+                q = [oracle_mod.e2m1_encode(w, s) for w in Wf[r, 16 * b:16 * b + 16]]
+                delta = Wf[r, 16 * b:16 * b + 16] - np.array([oracle_mod.e2m1_value(k) for k in q]) * s
+                direct = float(np.sum((Xf[:, 16 * b:16 * b + 16] @ delta) ** 2))
+                assert E[c - 1] == pytest.approx(direct, rel=1e-11, abs=1e-300)
+
+
+def test_lh_with_identity_hessian_equals_mse(oracle_mod):
+    W, _ = _tiny_layer(64, 128, 16, 11)
+    s_g = oracle_mod.global_scale(W)
+    c_mse, e_mse = oracle_mod.scale_search_mse(W, s_g)
+    for alpha in (1.0, 3.7, 1e-3):
+        H = np.tile(np.eye(16) * alpha, (8, 1, 1))
+        c_lh, e_lh = oracle_mod.scale_search_lh(W, s_g, H)
+        assert np.array_equal(c_lh, c_mse)
+        np.testing.assert_allclose(e_lh, e_mse * alpha, rtol=1e-12)
+
+
+def test_lh_single_block_is_exact_full_search(oracle_mod):
+    """With C = 16 the block-diagonal approximation is exact: brute force over
+    all 126 scales with the full ||delta X||^2 must pick the same scale."""
+    W, X = _tiny_layer(40, 16, 64, 13)
+    Xf, Wf = bits_to_f64(X), bits_to_f64(W)
+    s_g = oracle_mod.global_scale(W)
+    codes, _ = oracle_mod.scale_search_lh(W, s_g, oracle_mod.gram(X))
+    for r in range(W.shape[0]):
+        errs = []
+        for c in range(1, 127):
+            s = float(oracle_mod.effective_scale(s_g, c))
+            v = np.array([oracle_mod.e2m1_value(oracle_mod.e2m1_encode(w, s)) for w in Wf[r]])
+            errs.append(float(np.sum((Xf @ (Wf[r] - v * s)) ** 2)))
+        errs = np.array(errs)
+        best = int(np.argmin(errs)) + 1
+        if codes[r, 0] != best:  # only a tie at fp64 resolution may differ
+            assert errs[codes[r, 0] - 1] <= errs.min() * (1 + 1e-12)
+
+
+def test_search_invariants(oracle_mod):
+    W, X = _tiny_layer(32, 64, 64, 17)
+    s_g = oracle_mod.global_scale(W)
+    H = oracle_mod.gram(X)
+    c_max = oracle_mod.scale_search_max(W, s_g)
+    c_mse, _ = oracle_mod.scale_search_mse(W, s_g)
+    c_lh, _ = oracle_mod.scale_search_lh(W, s_g, H)
+    for r in range(W.shape[0]):
+        for b in range(4):
+            blk = W[r, 16 * b:16 * b + 16]
+            e_mse = oracle_mod.block_objectives(blk, s_g)
+            e_lh = oracle_mod.block_objectives(blk, s_g, H[b])
+            assert e_mse[c_mse[r, b] - 1] == e_mse.min()
+            assert e_lh[c_lh[r, b] - 1] == e_lh.min()
+            # first minimum: no smaller code reaches the minimum
+            assert np.all(e_lh[:c_lh[r, b] - 1] > e_lh.min())
+            if c_max[r, b]:
+                assert e_mse[c_mse[r, b] - 1] <= e_mse[c_max[r, b] - 1]
+                assert e_lh[c_lh[r, b] - 1] <= e_lh[c_max[r, b] - 1]
+            assert e_lh[c_lh[r, b] - 1] <= e_lh[c_mse[r, b] - 1]
+
+
+def test_zero_block_and_zero_hessian(oracle_mod):
+    W = np.zeros((2, 32), np.uint16)
+    W[1, 16:] = f32_to_bf16_bits(np.linspace(-1, 1, 16, dtype=np.float32))
+    s_g = oracle_mod.global_scale(W)
+    c_max = oracle_mod.scale_search_max(W, s_g)
+    assert c_max[0, 0] == 0 and c_max[1, 0] == 0 and c_max[1, 1] != 0
+    c_mse, e = oracle_mod.scale_search_mse(W, s_g)
+    assert c_mse[0, 0] == 1 and e[0, 0] == 0
+    c_lh, e = oracle_mod.scale_search_lh(W, s_g, np.zeros((2, 16, 16)))
+    assert np.all(c_lh == 1) and np.all(e == 0)
+
+
+# ------------------------------------------------------------ pack / dequant
+def test_pack_nibble_order_and_dequant(oracle_mod):
+    s_g = np.float32(1.0)
+    code = 0x38  # E4M3 value 1.0
+    vals = np.array([0.5, -1, 1.5, 6, -6, 0, 2, 3, 4, -0.5, 1, -1.5, 2, -3, -4, 6], np.float32)
+    u = f32_to_bf16_bits(vals).reshape(1, 16)
+    codes = np.array([[code]], np.uint8)
+    packed = oracle_mod.quantize_pack(u, s_g, codes)
+    assert packed[0, 0] == (1 | (0xA << 4))      # 0.5 low nibble, -1 high nibble
+    assert packed[0, 1] == (3 | (7 << 4))
+    assert packed[0, 2] == (0xF | (0 << 4))
+    deq = bits_to_f64(oracle_mod.dequantize(packed, codes, s_g))
+    np.testing.assert_array_equal(deq.ravel(), vals.astype(np.float64))
+
+
+def test_quantize_dequantize_idempotent(oracle_mod):
+    W, _ = _tiny_layer(16, 64, 1, 19)
+    s_g = oracle_mod.global_scale(W)
+    codes = oracle_mod.scale_search_max(W, s_g)
+    p1 = oracle_mod.quantize_pack(W, s_g, codes)
+    y1 = oracle_mod.dequantize(p1, codes, s_g)
+    p2 = oracle_mod.quantize_pack(y1, s_g, codes)
+    assert np.array_equal(p1, p2)
+    # |y| <= 6 s_eff blockwise
+    yf = bits_to_f64(y1).reshape(16, 4, 16)
+    for r in range(16):
+        for b in range(4):
+            s = oracle_mod.effective_scale(s_g, codes[r, b])
+            assert np.all(np.abs(yf[r, b]) <= 6 * s * (1 + 2 ** -8))
+
+
+def test_fake_quant_composes_pinned_steps(oracle_mod):
+    g = torch.Generator().manual_seed(23)
+    X = torch.randn(24, 96, generator=g)
+    X[:, 5] *= 40
+    Xu = bf16_bits(X.to(torch.bfloat16))
+    y, packed, codes, s_g = oracle_mod.fake_quant(Xu)
+    assert s_g == oracle_mod.global_scale(Xu)
+    assert np.array_equal(codes, oracle_mod.scale_search_max(Xu, s_g))
+    assert np.array_equal(packed, oracle_mod.quantize_pack(Xu, s_g, codes))
+    assert np.array_equal(y, oracle_mod.dequantize(packed, codes, s_g))
+
+
+def test_snr_closed_form_arithmetic():
+    g = read_golden("snr_closed_form.txt")
+    for ratio, _, db in g["m_over_sigma"]:
+        est = 20 * math.log10(1.0 / (float(ratio) / 6.0))
+        assert est == pytest.approx(float(db), abs=0.06)

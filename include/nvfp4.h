@@ -1,0 +1,207 @@
+/*
+ * nvfp4.h — C ABI of libnvfp4.so: NVFP4 scale calibration on B200 (sm_100a).
+ *
+ * NVFP4 stores a tensor as 4-bit E2M1 codes in blocks of 16 consecutive
+ * values of a row, one FP8 E4M3 scale per block and one FP32 scale per
+ * tensor.  This library computes, on the GPU:
+ *   - the FP32 tensor scale,
+ *   - the block-diagonal Gram matrix of calibration activations,
+ *   - the per-block FP8 scale by the max, MSE or Local-Hessian rule,
+ *   - E2M1 quantisation with packing, dequantisation,
+ *   - dynamic (per call) activation fake-quantisation for W4A4.
+ *
+ * Sources (page title, section):
+ *   [BT]  Baseten engineering blog, "What makes high-quality NVFP4":
+ *         "Why do we need scales?" (E2M1 value set, FP32 tensor scale),
+ *         "Block scaling: one scale per 16 values", "Why blocks?" (worked
+ *         example, max / 6), "Calibration" (activation block scales).
+ *   [LH]  "4 比特量化到底让模型笨了多少？" (write-up of NVIDIA Model
+ *         Optimizer's "Improving NVFP4 Accuracy with Local-Hessian Weight
+ *         Scales"): "The NVFP4 structure" (FP8 block scale, max scaling,
+ *         MSE over 126 candidates), "A different objective" (E(s) =
+ *         ||delta X||^2 = tr(delta X X^T delta^T), 16x16 block-diagonal
+ *         approximation, exhaustive candidate search).
+ *   [QAD] "為什么NVFP4推理精度會掉以及QAD到底在修什么": 2.1 (round to the
+ *         nearest E2M1 value), 2.3 (step = block max / 6), 3.2 (fake-quant
+ *         forward: block max / 6, quantise, multiply back), 4.2 (clamp the
+ *         scale to the FP8 maximum).
+ *
+ * Conventions shared by every entry point:
+ *   - bf16 tensors are passed as uint16_t bit patterns; every pointer is a
+ *     DEVICE pointer owned by the caller unless stated otherwise; nothing is
+ *     freed or retained by the library.
+ *   - Matrices are row-major.  A weight W is [R, C] (C = input channels);
+ *     activations X are [tokens, C].  Blocks are 16 consecutive elements of
+ *     a row, so C must be a multiple of 16 (else NVFP4_ERR_SHAPE).
+ *   - bf16 and packed-code pointers must be 16-byte aligned, float pointers
+ *     4-byte aligned (else NVFP4_ERR_MISALIGNED).  Block-code (uint8) arrays
+ *     have no alignment requirement.
+ *   - `batch` >= 1 stacks independent tensors (e.g. MoE experts) with a
+ *     contiguous batch stride; each has its own FP32 scale s_g[batch].
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work on it and return without synchronising, except
+ *     nvfp4_get_device_status.  Argument errors are detected on the host
+ *     before anything is enqueued; a failed launch returns NVFP4_ERR_CUDA.
+ *   - A CUDA device must be current; all pointers must belong to it.
+ *
+ * Block-scale codes are E4M3 (FN variant) bit patterns, 0x00..0x7E.  The
+ * effective scale of a block is s_eff = fl32(s_g * e4m3(code)).  E2M1 codes
+ * are sign<<3 | k with magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}[k]; element 2j
+ * of a row is the low nibble of byte j of its packed row.  Rounding is to
+ * nearest, ties to even, decided on the exact quotient |x| / s_eff, and
+ * saturates at 6; a negative input that rounds to zero keeps its sign.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum nvfp4_status {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,     /* null pointer, negative size, batch or group count < 1 */
+    NVFP4_ERR_SHAPE = 2,           /* C not a multiple of 16, or sizes overflow */
+    NVFP4_ERR_MISALIGNED = 3,      /* pointer alignment rule above violated */
+    NVFP4_ERR_NONFINITE = 4,       /* NaN or Inf met in an input (device-side report) */
+    NVFP4_ERR_CUDA = 5,            /* a CUDA runtime call or launch failed */
+    NVFP4_ERR_NOT_IMPLEMENTED = 6,
+    NVFP4_ERR_TOO_LARGE = 7        /* request beyond a documented maximum */
+} nvfp4_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *nvfp4_status_string(nvfp4_status st);
+
+/*
+ * FP32 tensor scale per batch element ([BT] "Why do we need scales?": NVFP4
+ * has a tensor-level FP32 scale besides the block scales; the formula is
+ * this library's reading): s_g[i] = fl32(amax_i / 2688) with amax_i the
+ * largest |x| of batch element i and 2688 = 6 * 448, so that the largest
+ * E4M3 scale maps the tensor maximum onto E2M1's 6.  amax = 0 gives 1.
+ *   x        [batch, n_per_batch] bf16, n_per_batch a multiple of 8.
+ *   s_g      [batch] float, written.  If an element is NaN/Inf, its s_g is
+ *            set to NaN and the device status becomes NVFP4_ERR_NONFINITE
+ *            (see nvfp4_get_device_status).
+ */
+nvfp4_status nvfp4_global_scale(const uint16_t *x, int64_t batch, int64_t n_per_batch,
+                                float *s_g, void *stream);
+
+/*
+ * Block-diagonal Gram accumulation over calibration tokens ([LH] "A
+ * different objective": H = X X^T restricted to its 16x16 diagonal blocks):
+ *   H[j] += sum_t x[t, 16j:16j+16]^T x[t, 16j:16j+16],  j = 0..C/16-1.
+ *   x   [n_tok, C] bf16 (n_tok >= 0; 0 is a no-op).
+ *   H   [C/16, 16, 16] float, read and written (accumulated in place, so a
+ *       calibration set can be streamed in chunks).
+ * Products of bf16 values are exact in fp32 and accumulate in fp32 on the
+ * tensor cores; partial sums over token ranges are combined in a fixed
+ * order, so the result is bitwise reproducible for a given shape.  Uses a
+ * stream-ordered scratch buffer from a library-owned memory pool.
+ */
+nvfp4_status nvfp4_hessian_accumulate(const uint16_t *x, int64_t n_tok, int64_t C, float *H,
+                                      void *stream);
+
+/*
+ * Grouped form for experts: tokens are sorted by group; group g owns rows
+ * offsets[g] .. offsets[g+1]-1 of x and accumulates into H[g].
+ *   x         [n_tok_total, C] bf16
+ *   offsets   DEVICE int64 [G+1], non-decreasing, offsets[0] = 0,
+ *             offsets[G] = n_tok_total (the host passes n_tok_total so that no
+ *             device value has to be read back).  Offsets outside
+ *             [0, n_tok_total] are clamped on the device.
+ *   H         [G, C/16, 16, 16] float, accumulated.
+ */
+nvfp4_status nvfp4_hessian_accumulate_grouped(const uint16_t *x, const int64_t *offsets,
+                                              int64_t G, int64_t n_tok_total, int64_t C,
+                                              float *H, void *stream);
+
+/*
+ * Max rule ([QAD] 2.3 and 4.2, [BT] "Why blocks?", [LH] "The NVFP4
+ * structure"): code = E4M3 round-to-nearest-even, saturating at 448, of the
+ * exact quotient amax_b / (6 * s_g); an all-zero block gets code 0.
+ *   w            [batch, R, C] bf16
+ *   s_g          DEVICE [batch] float, positive and finite
+ *   scale_codes  [batch, R, C/16] uint8, written
+ */
+nvfp4_status nvfp4_scale_search_max(const uint16_t *w, int64_t batch, int64_t R, int64_t C,
+                                    const float *s_g, uint8_t *scale_codes, void *stream);
+
+/*
+ * MSE rule ([LH] "The NVFP4 structure"): for every block, the code in
+ * 1..126 minimising sum_i (w_i - v(q_i) s_eff)^2, q_i the E2M1 code of w_i at
+ * s_eff; the smallest code wins a tie.  Candidates are screened in fp32 and
+ * near-ties (best two within 2^-12 relative) are re-scored in fp64.
+ *   best_obj     optional [batch, R, C/16] float, the winning objective.
+ */
+nvfp4_status nvfp4_scale_search_mse(const uint16_t *w, int64_t batch, int64_t R, int64_t C,
+                                    const float *s_g, uint8_t *scale_codes, float *best_obj,
+                                    void *stream);
+
+/*
+ * Local-Hessian rule ([LH] "A different objective"): for every block b of
+ * every row, the code in 1..126 minimising E = delta H_b delta^T, with
+ * delta_i = w_i - v(q_i) s_eff and H_b the 16x16 Gram block of the block's
+ * columns (shared by all rows); the smallest code wins a tie.  H_b is
+ * factored once per column block (fp64 Cholesky, semidefinite pivots
+ * dropped) and candidates are screened in fp32 as ||L^T delta||^2;
+ * near-ties (best two within 2^-12 relative) are re-scored in fp64 from H.
+ *   H            [batch, C/16, 16, 16] float (e.g. from
+ *                nvfp4_hessian_accumulate), symmetric positive semidefinite
+ *   best_obj     optional [batch, R, C/16] float, the winning objective.
+ */
+nvfp4_status nvfp4_scale_search_local_hessian(const uint16_t *w, int64_t batch, int64_t R,
+                                              int64_t C, const float *s_g, const float *H,
+                                              uint8_t *scale_codes, float *best_obj,
+                                              void *stream);
+
+/*
+ * E2M1 quantisation and packing given block codes ([BT] "Why do we need
+ * scales?", "Block scaling"; [QAD] 2.1).  Two codes per byte, element 2j in
+ * the low nibble.  A block with code 0 has s_eff = 0 and encodes as
+ * (signed) zeros.
+ *   packed  [batch, R, C/2] uint8, written (16-byte aligned)
+ */
+nvfp4_status nvfp4_quantize_pack(const uint16_t *w, int64_t batch, int64_t R, int64_t C,
+                                 const float *s_g, const uint8_t *scale_codes, uint8_t *packed,
+                                 void *stream);
+
+/*
+ * Dequantisation ([QAD] 3.2: the quantised value times its scale):
+ * out = bf16_rn(fl32(v(q) * s_eff)).
+ *   out   [batch, R, C] bf16, written
+ */
+nvfp4_status nvfp4_dequantize(const uint8_t *packed, const uint8_t *scale_codes,
+                              const float *s_g, int64_t batch, int64_t R, int64_t C,
+                              uint16_t *out, void *stream);
+
+/*
+ * Dynamic W4A4 activation fake-quant ([BT] "Calibration"; [QAD] 3.2):
+ * s_g from the whole x (as nvfp4_global_scale), then per block the max rule,
+ * E2M1 encode and dequantise, fused in one pass over x.
+ *   x       [rows, C] bf16
+ *   out     [rows, C] bf16, written (may not alias x)
+ *   packed  optional [rows, C/2] uint8 (NULL to skip)
+ *   scale_codes optional [rows, C/16] uint8 (NULL to skip)
+ *   s_g     DEVICE float [1], written
+ */
+nvfp4_status nvfp4_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16_t *out,
+                              uint8_t *packed, uint8_t *scale_codes, float *s_g, void *stream);
+
+/*
+ * Reads and clears the device-side status of the current device after
+ * synchronising `stream` (the only call that blocks the host).  *out is
+ * NVFP4_OK or NVFP4_ERR_NONFINITE.
+ */
+nvfp4_status nvfp4_get_device_status(void *stream, nvfp4_status *out);
+
+/* Releases the library's memory pool on every device it touched.  No call
+ * may be in flight. */
+void nvfp4_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

@@ -5,15 +5,13 @@ The compute path is the C-ABI library ``libnvfp4.so`` built from ``csrc/``;
 the package itself loads nothing, so the seeded input module ``workloads``
 can be used without the CUDA library.
 """
-__all__ = ["nvfp4", "workloads"]
+import importlib
+
+__all__ = ["nvfp4", "workloads", "build"]
 __version__ = "0.1.0"
 
 
 def __getattr__(name):
-    if name == "nvfp4":
-        from . import nvfp4 as _m
-        return _m
-    if name == "workloads":
-        from . import workloads as _w
-        return _w
+    if name in __all__:
+        return importlib.import_module("." + name, __name__)
     raise AttributeError(name)

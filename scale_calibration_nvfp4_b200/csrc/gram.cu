@@ -1,0 +1,313 @@
+// Block-diagonal Gram accumulation H[j] += X_j^T X_j over calibration tokens
+// (the Local-Hessian write-up "4 比特量化到底让模型笨了多少？", section "A
+// different objective": H = X X^T is the (half) Hessian of the output error;
+// the block-diagonal approximation keeps only its 16x16 diagonal blocks).
+//
+// Data path: a CTA owns a group of up to 8 column blocks (128 channels) and a
+// range of tokens.  Token tiles [64 tokens x 128 channels] of bf16 stream from
+// HBM into shared memory through a 4-stage cp.async pipeline; rows are padded
+// to 272 bytes so the transposing ldmatrix reads are bank-conflict free.
+// Warp w owns column block w of the group: per 16 tokens one ldmatrix.x4.trans
+// yields X_j^T as the A fragment of a 16x8x16 bf16 MMA, and the same four
+// registers are the B fragments of the two 8-channel halves, so the 16x16
+// block comes from two MMAs with no wasted product (bf16 x bf16 products are
+// exact in fp32, sums are fp32).  Each CTA writes its fp32 partial block to a
+// stream-ordered scratch buffer; a second kernel adds the partials of a group
+// to H in a fixed order, so the result does not depend on scheduling.
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int kGramThreads = 256;             // 8 warps
+constexpr int kGroupBlocks = 8;               // column blocks per CTA
+constexpr int kTileTok = 64;                  // tokens per pipeline stage
+constexpr int kStages = 4;
+constexpr int kRowBytes = 128 * 2 + 16;       // padded smem row
+constexpr int kStageBytes = kTileTok * kRowBytes;
+constexpr int kGramSmem = kStages * kStageBytes;  // 69,632 bytes
+constexpr int64_t kGroupedItemTokens = 2048;  // tokens per work item, grouped form
+
+struct ItemRange {
+  int64_t group, t_begin, t_end;
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t r[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Work item -> (group, token range).  Uniform split of one group when
+// `items` == nullptr, else the device table built by build_items_kernel.
+__device__ __forceinline__ bool item_range(int64_t item, const ItemRange *items,
+                                           const int64_t *n_items_dev, int64_t n_tok,
+                                           int64_t per_item, ItemRange &out) {
+  if (items) {
+    if (item >= *n_items_dev) return false;
+    out = items[item];
+    return true;
+  }
+  out.group = 0;
+  out.t_begin = item * per_item;
+  out.t_end = min(n_tok, out.t_begin + per_item);
+  return out.t_begin < out.t_end;
+}
+
+__global__ void __launch_bounds__(kGramThreads)
+    gram_partial_kernel(const uint16_t *__restrict__ x, int64_t C, const ItemRange *items,
+                        const int64_t *n_items_dev, int64_t n_tok, int64_t per_item,
+                        float *__restrict__ partial) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int64_t nb = C / kBlock;
+  const int64_t item = blockIdx.x;
+  const int64_t cg = blockIdx.y;
+  ItemRange ir;
+  if (!item_range(item, items, n_items_dev, n_tok, per_item, ir)) return;
+  const int width = (int)min((int64_t)kGroupBlocks, nb - cg * kGroupBlocks);  // column blocks
+  const int chunks_per_row = width * 2;                                        // 16 B chunks
+  const int64_t ntiles = (ir.t_end - ir.t_begin + kTileTok - 1) / kTileTok;
+  const uint16_t *xbase = x + cg * kGroupBlocks * kBlock;
+  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+
+  auto load_tile = [&](int64_t tile, int stage) {
+    const int64_t t0 = ir.t_begin + tile * kTileTok;
+    const int total = kTileTok * chunks_per_row;
+    for (int i = threadIdx.x; i < total; i += kGramThreads) {
+      const int row = i / chunks_per_row;
+      const int ch = i - row * chunks_per_row;
+      const int64_t t = t0 + row;
+      const bool valid = t < ir.t_end;
+      const uint16_t *src = valid ? xbase + t * C + ch * 8 : xbase;
+      cp_async16(sbase + stage * kStageBytes + row * kRowBytes + ch * 16, src, valid ? 16u : 0u);
+    }
+  };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+  // ldmatrix row address of this lane inside a 16-token step
+  const int lrow = (lane & 7) + ((lane >> 4) & 1) * 8;
+  const int lcol = warp * 32 + ((lane >> 3) & 1) * 16;
+
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (s < ntiles) load_tile(s, s);
+    cp_async_commit();
+  }
+  for (int64_t tile = 0; tile < ntiles; ++tile) {
+    cp_async_wait<kStages - 2>();
+    __syncthreads();
+    const int64_t next = tile + kStages - 1;
+    if (next < ntiles) load_tile(next, (int)(next % kStages));
+    cp_async_commit();
+    if (warp < width) {
+      const uint32_t st = sbase + (uint32_t)(tile % kStages) * kStageBytes;
+#pragma unroll
+      for (int k = 0; k < kTileTok / 16; ++k) {
+        uint32_t a[4];
+        ldmatrix_x4_trans(st + (k * 16 + lrow) * kRowBytes + lcol, a);
+        mma_bf16_16816(d0, a, a[0], a[2]);
+        mma_bf16_16816(d1, a, a[1], a[3]);
+      }
+    }
+  }
+  cp_async_wait<0>();
+
+  if (warp < width) {
+    const int64_t j = cg * kGroupBlocks + warp;
+    float *P = partial + (item * nb + j) * 256;
+    const int g = lane >> 2, t = lane & 3;
+    P[g * 16 + 2 * t] = d0[0];
+    P[g * 16 + 2 * t + 1] = d0[1];
+    P[(g + 8) * 16 + 2 * t] = d0[2];
+    P[(g + 8) * 16 + 2 * t + 1] = d0[3];
+    P[g * 16 + 8 + 2 * t] = d1[0];
+    P[g * 16 + 8 + 2 * t + 1] = d1[1];
+    P[(g + 8) * 16 + 8 + 2 * t] = d1[2];
+    P[(g + 8) * 16 + 8 + 2 * t + 1] = d1[3];
+  }
+}
+
+// H[g][j][e] += sum of the partials of group g's items, in item order.
+__global__ void gram_reduce_kernel(const float *__restrict__ partial, int64_t nb, int64_t G,
+                                   const int64_t *__restrict__ item_start, int64_t n_items_uniform,
+                                   float *__restrict__ H) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over G * nb * 256
+  const int64_t per_group = nb * 256;
+  if (idx >= G * per_group) return;
+  const int64_t g = idx / per_group;
+  const int64_t je = idx - g * per_group;
+  int64_t i0 = 0, i1 = n_items_uniform;
+  if (item_start) {
+    i0 = item_start[g];
+    i1 = item_start[g + 1];
+  }
+  float acc = 0.0f;
+  for (int64_t i = i0; i < i1; ++i) acc += partial[i * per_group + je];
+  H[idx] += acc;
+}
+
+// Grouped form: per-group item counts, an exclusive scan (one CTA) and the
+// item table.  Offsets are clamped to [0, n_tok] and made non-decreasing.
+__global__ void build_items_kernel(const int64_t *__restrict__ offsets, int64_t G, int64_t n_tok,
+                                   int64_t per_item, int64_t max_items,
+                                   int64_t *__restrict__ item_start, ItemRange *__restrict__ items,
+                                   int64_t *__restrict__ n_items) {
+  __shared__ int64_t warp_sums[32];
+  __shared__ int64_t carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  auto clamp_off = [&](int64_t g) {
+    int64_t o = offsets[g];
+    return o < 0 ? (int64_t)0 : (o > n_tok ? n_tok : o);
+  };
+  for (int64_t base = 0; base < G; base += blockDim.x) {
+    const int64_t g = base + threadIdx.x;
+    int64_t cnt = 0, lo = 0, hi = 0;
+    if (g < G) {
+      lo = clamp_off(g);
+      hi = clamp_off(g + 1);
+      if (hi < lo) hi = lo;
+      cnt = (hi - lo + per_item - 1) / per_item;
+    }
+    // block-wide inclusive scan of cnt
+    int64_t v = cnt;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int64_t n = __shfl_up_sync(0xFFFFFFFFu, v, o);
+      if (lane >= o) v += n;
+    }
+    if (lane == 31) warp_sums[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+      int64_t s = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int64_t n = __shfl_up_sync(0xFFFFFFFFu, s, o);
+        if (lane >= o) s += n;
+      }
+      warp_sums[lane] = s;
+    }
+    __syncthreads();
+    const int64_t excl = carry + (warp ? warp_sums[warp - 1] : 0) + v - cnt;
+    if (g < G) {
+      item_start[g] = excl;
+      for (int64_t c = 0; c < cnt && excl + c < max_items; ++c) {
+        ItemRange r;
+        r.group = g;
+        r.t_begin = lo + c * per_item;
+        r.t_end = min(hi, r.t_begin + per_item);
+        items[excl + c] = r;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = excl + cnt;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    item_start[G] = carry;
+    *n_items = carry < max_items ? carry : max_items;
+  }
+}
+
+bool g_smem_attr_set = false;
+
+}  // namespace
+
+cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, int64_t n_tok,
+                        int64_t C, float *H, cudaStream_t st) {
+  if (n_tok == 0 || C == 0 || G == 0) return cudaSuccess;
+  cudaError_t e;
+  if (!g_smem_attr_set) {
+    e = cudaFuncSetAttribute(gram_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kGramSmem);
+    if (e != cudaSuccess) return e;
+    g_smem_attr_set = true;
+  }
+  const int64_t nb = C / kBlock;
+  const int64_t ngroups = (nb + kGroupBlocks - 1) / kGroupBlocks;
+  const int64_t per_group = nb * 256;
+
+  if (!offsets) {
+    // uniform split of the tokens into items, enough CTAs for ~3 waves of
+    // 3 resident CTAs per SM, at least 4 tiles per item
+    const int64_t target = (int64_t)sm_count() * 3 * 2;
+    int64_t items = (target + ngroups - 1) / ngroups;
+    const int64_t max_items = (n_tok + 4 * kTileTok - 1) / (4 * kTileTok);
+    if (items > max_items) items = max_items;
+    if (items < 1) items = 1;
+    int64_t per_item = (n_tok + items - 1) / items;
+    per_item = (per_item + kTileTok - 1) / kTileTok * kTileTok;
+    items = (n_tok + per_item - 1) / per_item;
+    float *partial = nullptr;
+    e = scratch_alloc((void **)&partial, sizeof(float) * items * per_group, st);
+    if (e != cudaSuccess) return e;
+    gram_partial_kernel<<<dim3((unsigned)items, (unsigned)ngroups), kGramThreads, kGramSmem, st>>>(
+        x, C, nullptr, nullptr, n_tok, per_item, partial);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) {
+      const int64_t n = per_group;
+      gram_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, nb, 1, nullptr,
+                                                                      items, H);
+      e = cudaGetLastError();
+    }
+    cudaError_t e2 = scratch_free(partial, st);
+    return e != cudaSuccess ? e : e2;
+  }
+
+  const int64_t per_item = kGroupedItemTokens;
+  const int64_t max_items = n_tok / per_item + G;
+  // scratch layout: item_start [G+1] | n_items [1] | items [max_items] | partials
+  const size_t off_items = (sizeof(int64_t) * (G + 2) + 255) / 256 * 256;
+  const size_t off_part = (off_items + sizeof(ItemRange) * max_items + 255) / 256 * 256;
+  const size_t bytes = off_part + sizeof(float) * max_items * per_group;
+  unsigned char *ws = nullptr;
+  e = scratch_alloc((void **)&ws, bytes, st);
+  if (e != cudaSuccess) return e;
+  int64_t *item_start = reinterpret_cast<int64_t *>(ws);
+  int64_t *n_items = item_start + G + 1;
+  ItemRange *items = reinterpret_cast<ItemRange *>(ws + off_items);
+  float *partial = reinterpret_cast<float *>(ws + off_part);
+  build_items_kernel<<<1, 1024, 0, st>>>(offsets, G, n_tok, per_item, max_items, item_start,
+                                         items, n_items);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    gram_partial_kernel<<<dim3((unsigned)max_items, (unsigned)ngroups), kGramThreads, kGramSmem,
+                          st>>>(x, C, items, n_items, n_tok, per_item, partial);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) {
+    const int64_t n = G * per_group;
+    gram_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, nb, G, item_start,
+                                                                    0, H);
+    e = cudaGetLastError();
+  }
+  cudaError_t e2 = scratch_free(ws, st);
+  return e != cudaSuccess ? e : e2;
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,36 @@
+// Launchers behind the C ABI (arguments already validated by api.cu).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+int sm_count();
+
+cudaError_t launch_global_scale(const uint16_t *x, int64_t batch, int64_t n_per_batch,
+                                float *s_g, cudaStream_t st);
+cudaError_t launch_scale_max(const uint16_t *w, int64_t batch, int64_t nblk, const float *s_g,
+                             uint8_t *codes, cudaStream_t st);
+cudaError_t launch_pack(const uint16_t *w, int64_t batch, int64_t nblk, const float *s_g,
+                        const uint8_t *codes, uint8_t *packed, cudaStream_t st);
+cudaError_t launch_dequant(const uint8_t *packed, const uint8_t *codes, const float *s_g,
+                           int64_t batch, int64_t nblk, uint16_t *out, cudaStream_t st);
+cudaError_t launch_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16_t *out,
+                              uint8_t *packed, uint8_t *codes, float *s_g, cudaStream_t st);
+cudaError_t read_and_clear_device_status(cudaStream_t st, int *out);
+
+// Scale search: objective 0 = MSE, 1 = Local-Hessian (H required).
+cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int64_t C,
+                                const float *s_g, const float *H, uint8_t *codes,
+                                float *best_obj, int local_hessian, cudaStream_t st);
+
+// Gram accumulation.  `offsets` == nullptr: one group of n_tok tokens.
+cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, int64_t n_tok,
+                        int64_t C, float *H, cudaStream_t st);
+
+// Stream-ordered scratch from the library's pool on the current device.
+cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t st);
+cudaError_t scratch_free(void *p, cudaStream_t st);
+void scratch_release_all();
+
+}  // namespace nvfp4

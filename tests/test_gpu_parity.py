@@ -1,0 +1,398 @@
+"""GPU parity: every C-ABI entry point against the CPU oracle, element by
+element, on seeded inputs (small cases that span many tiles with ragged
+tails, edge cases, and samples of the full-size workloads)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import bf16_bits, bits_to_f64, f32_to_bf16_bits
+from parity_util import GRAM_REL, check_search_codes, rel_frobenius
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from scale_calibration_nvfp4_b200 import build, nvfp4
+    build.build()
+    nvfp4.lib()
+    oracle.lib()
+    return nvfp4
+
+
+def dev_bf16(u16):
+    t = torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16)
+    return t.cuda()
+
+
+def rand_bf16(shape, seed, std=1.0, outlier_frac=0.0, factor=1.0):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(*shape, generator=g) * std
+    n = int(outlier_frac * x.numel())
+    if n:
+        idx = torch.randperm(x.numel(), generator=g)[:n]
+        x.view(-1)[idx] *= factor
+    return x.to(torch.bfloat16)
+
+
+# ------------------------------------------------------------ global scale
+def test_global_scale_bitexact(nv):
+    x = rand_bf16((5, 4104), 1, 0.02, 0.01, 30.0)
+    s = nv.global_scale(x.cuda(), batch=5).cpu().numpy()
+    xu = bf16_bits(x)
+    for b in range(5):
+        assert s[b] == oracle.global_scale(xu[b]), b
+    z = torch.zeros(3, 64, dtype=torch.bfloat16, device="cuda")
+    assert torch.equal(nv.global_scale(z, batch=3).cpu(), torch.ones(3))
+    # one element only, and a subnormal-range maximum
+    t = torch.zeros(16, dtype=torch.bfloat16)
+    t[7] = -2.0 ** -130
+    assert nv.global_scale(t.cuda()).item() == oracle.global_scale(bf16_bits(t))
+    assert nv.get_device_status() == "NVFP4_OK"
+
+
+def test_global_scale_nonfinite_reports(nv):
+    x = torch.ones(2, 32, dtype=torch.bfloat16)
+    x[1, 5] = float("nan")
+    s = nv.global_scale(x.cuda(), batch=2).cpu()
+    assert s[0].item() == oracle.global_scale(bf16_bits(x[0]))
+    assert torch.isnan(s[1])
+    assert nv.get_device_status() == "NVFP4_ERR_NONFINITE"
+    assert nv.get_device_status() == "NVFP4_OK"  # cleared by the read
+
+
+# ------------------------------------------------------------ max rule
+def test_max_rule_bitexact_with_edge_blocks(nv):
+    x = rand_bf16((67, 176), 2, 0.02, 0.01, 20.0)
+    x[3, :16] = 0                               # all-zero block
+    x[4, 16:32] = 1e-3 * x[4, 16:32]            # small block
+    x[5, 32:48] = 0
+    x[5, 40] = -1e-7                            # single tiny non-zero: subnormal / zero code
+    x[6, 48:64] = x.abs().max()                 # saturating block
+    s_g = nv.global_scale(x.cuda())
+    codes = nv.scale_search_max(x.cuda(), s_g).cpu().numpy()
+    ref = oracle.scale_search_max(bf16_bits(x), s_g.item())
+    np.testing.assert_array_equal(codes, ref)
+    assert codes[3, 0] == 0 and codes[6, 3] == 0x7E
+
+
+def test_max_rule_exact_midpoint_ties(nv):
+    # block maxima exactly on E4M3 midpoints times 6 s_g (s_g = 2^-5 keeps every
+    # product a bf16 value): ties go to the even code
+    s_g = np.float32(2.0 ** -5)
+    vals = [0.5 * (oracle.e4m3_value(c) + oracle.e4m3_value(c + 1)) * 6 * float(s_g)
+            for c in range(0, 126)]
+    blocks = np.zeros((len(vals), 16), np.float32)
+    blocks[:, 0] = vals
+    u = f32_to_bf16_bits(blocks)
+    assert np.array_equal(bits_to_f64(u)[:, 0], np.array(vals))
+    sg = torch.tensor([s_g], device="cuda")
+    codes = nv.scale_search_max(dev_bf16(u), sg).cpu().numpy()
+    ref = oracle.scale_search_max(u, s_g)
+    np.testing.assert_array_equal(codes, ref)
+    assert np.all(ref[:, 0] % 2 == 0)
+
+
+# ------------------------------------------------------------ E2M1 encode
+@pytest.mark.parametrize("s_g,code", [(1.0, 0x38), (1.0, 0x56), (2.0 ** -5, 0x7E),
+                                      (0.0123456, 0x31), (3.3e-3, 0x01), (7.1e-4, 0x77),
+                                      (1.0, 0x07), (0.5, 0x00)])
+def test_encode_every_bf16_pattern(nv, s_g, code):
+    """All 65,536 bf16 bit patterns (NaN/Inf replaced by 0) through the
+    packed encode at one block scale: bit-exact against the oracle."""
+    u = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    exp = (u >> 7) & 0xFF
+    u[exp == 0xFF] = 0
+    W = u.reshape(256, 256)
+    s_g = np.float32(s_g)
+    codes = np.full((256, 16), code, np.uint8)
+    packed = nv.quantize_pack(dev_bf16(W), torch.tensor([s_g], device="cuda"),
+                              torch.from_numpy(codes).cuda()).cpu().numpy()
+    ref = oracle.quantize_pack(W, s_g, codes)
+    np.testing.assert_array_equal(packed, ref)
+
+
+def test_encode_exact_midpoints(nv):
+    # values exactly on E2M1 midpoints at scale s_eff: the tie rule decides
+    s_g = np.float32(1.0)
+    codes = np.array([[0x30, 0x38, 0x3A, 0x44]], np.uint8)  # 0.5, 1, 1.25, 2.5
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5]
+    rows = []
+    for c in codes[0]:
+        s = oracle.effective_scale(s_g, int(c))
+        rows += [m * s for m in mids] + [-m * s for m in mids]
+    u = f32_to_bf16_bits(np.array(rows, np.float32)).reshape(1, 64)
+    assert np.array_equal(bits_to_f64(u).ravel(), np.array(rows))
+    packed = nv.quantize_pack(dev_bf16(u), torch.tensor([s_g], device="cuda"),
+                              torch.from_numpy(codes).cuda()).cpu().numpy()
+    np.testing.assert_array_equal(packed, oracle.quantize_pack(u, s_g, codes))
+
+
+# ------------------------------------------------------------ pack / dequant
+@pytest.mark.parametrize("shape", [(1, 16), (37, 80), (3, 4096), (129, 272)])
+def test_pack_dequant_bitexact(nv, shape):
+    R, C = shape
+    x = rand_bf16(shape, R * 7 + C, 0.02, 0.02, 25.0)
+    xu = bf16_bits(x)
+    s_g = nv.global_scale(x.cuda())
+    assert s_g.item() == oracle.global_scale(xu)
+    g = torch.Generator().manual_seed(R + C)
+    codes = torch.randint(0, 127, (R, C // 16), generator=g, dtype=torch.int32).to(torch.uint8)
+    codes.view(-1)[:4] = torch.tensor([0, 1, 8, 126], dtype=torch.uint8)[: codes.numel()]
+    packed = nv.quantize_pack(x.cuda(), s_g, codes.cuda())
+    ref_p = oracle.quantize_pack(xu, s_g.item(), codes.numpy())
+    np.testing.assert_array_equal(packed.cpu().numpy(), ref_p)
+    y = nv.dequantize(packed, codes.cuda(), s_g)
+    ref_y = oracle.dequantize(ref_p, codes.numpy(), s_g.item())
+    np.testing.assert_array_equal(bf16_bits(y), ref_y)
+
+
+def test_batched_pack_dequant_per_expert_scale(nv):
+    x = rand_bf16((4, 24, 64), 31, 0.02)
+    s_g = nv.global_scale(x.cuda(), batch=4)
+    codes = nv.scale_search_max(x.cuda(), s_g)
+    packed = nv.quantize_pack(x.cuda(), s_g, codes)
+    y = nv.dequantize(packed, codes, s_g)
+    xu = bf16_bits(x)
+    for b in range(4):
+        sg = s_g[b].item()
+        assert sg == oracle.global_scale(xu[b])
+        rc = oracle.scale_search_max(xu[b], sg)
+        np.testing.assert_array_equal(codes[b].cpu().numpy(), rc)
+        rp = oracle.quantize_pack(xu[b], sg, rc)
+        np.testing.assert_array_equal(packed[b].cpu().numpy(), rp)
+        np.testing.assert_array_equal(bf16_bits(y[b]), oracle.dequantize(rp, rc, sg))
+
+
+# ------------------------------------------------------------ fake-quant
+@pytest.mark.parametrize("shape", [(333, 96), (1, 16), (64, 8192)])
+def test_fake_quant_bitexact(nv, shape):
+    x = rand_bf16(shape, shape[0] + shape[1], 1.0)
+    if shape[1] > 16:
+        x[:, 5] *= 40
+    y, packed, codes, s_g = nv.fake_quant(x.cuda(), want_packed=True)
+    ry, rp, rc, rs = oracle.fake_quant(bf16_bits(x))
+    assert s_g.item() == rs
+    np.testing.assert_array_equal(codes.cpu().numpy(), rc)
+    np.testing.assert_array_equal(packed.cpu().numpy(), rp)
+    np.testing.assert_array_equal(bf16_bits(y), ry)
+    y2, p2, c2, _ = nv.fake_quant(x.cuda(), want_packed=False)
+    assert p2 is None and torch.equal(y2, y)
+
+
+def test_fake_quant_w4a4_full_size_sampled(nv):
+    """Dynamic W4A4 workload at full size (32768 x 8192): the tensor scale over
+    all of it, and 48 sampled token rows element by element."""
+    from scale_calibration_nvfp4_b200 import workloads
+    X = workloads.w4a4_inputs("cuda")
+    y, packed, codes, s_g = nv.fake_quant(X, want_packed=True)
+    torch.cuda.synchronize()
+    xu_all = bf16_bits(X)
+    assert s_g.item() == oracle.global_scale(xu_all)
+    rows = np.random.default_rng(5).choice(X.shape[0], 48, replace=False)
+    rows[0], rows[1] = 0, X.shape[0] - 1
+    xu = xu_all[rows]
+    sg = s_g.item()
+    rc = oracle.scale_search_max(xu, sg)
+    rp = oracle.quantize_pack(xu, sg, rc)
+    ry = oracle.dequantize(rp, rc, sg)
+    idx = torch.from_numpy(rows).cuda()
+    np.testing.assert_array_equal(codes[idx].cpu().numpy(), rc)
+    np.testing.assert_array_equal(packed[idx].cpu().numpy(), rp)
+    np.testing.assert_array_equal(bf16_bits(y[idx]), ry)
+
+
+# ------------------------------------------------------------ Gram
+@pytest.mark.parametrize("N,C", [(512, 512), (1000, 48), (1, 16), (65, 144), (3000, 1040)])
+def test_gram_matches_fp64(nv, N, C):
+    x = rand_bf16((N, C), N + C)
+    if C > 32:
+        x[:, 3] *= 30
+    H = torch.zeros(C // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate(x.cuda(), H)
+    ref = oracle.gram(bf16_bits(x))
+    Hc = H.cpu().numpy()
+    assert rel_frobenius(Hc, ref) <= GRAM_REL
+    for j in range(C // 16):
+        assert rel_frobenius(Hc[j], ref[j]) <= GRAM_REL
+    np.testing.assert_allclose(Hc, np.transpose(Hc, (0, 2, 1)), rtol=1e-6, atol=1e-6)
+
+
+def test_gram_accumulates_and_is_deterministic(nv):
+    x = rand_bf16((4096, 256), 77).cuda()
+    H1 = torch.zeros(16, 16, 16, device="cuda")
+    nv.hessian_accumulate(x, H1)
+    H2 = torch.zeros(16, 16, 16, device="cuda")
+    nv.hessian_accumulate(x, H2)
+    assert torch.equal(H1, H2)
+    H3 = torch.zeros(16, 16, 16, device="cuda")
+    nv.hessian_accumulate(x[:1500], H3)
+    nv.hessian_accumulate(x[1500:], H3)
+    assert rel_frobenius(H3.cpu().numpy(), H1.cpu().numpy()) <= 1e-6
+    H4 = H1.clone()
+    nv.hessian_accumulate(x[:0], H4)  # zero tokens: no-op
+    assert torch.equal(H4, H1)
+
+
+def test_gram_grouped(nv):
+    C = 96
+    counts = [0, 1, 700, 2049, 0, 35, 4100, 17]
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    x = rand_bf16((int(offs[-1]), C), 99)
+    H = torch.zeros(len(counts), C // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate_grouped(x.cuda(), torch.from_numpy(offs).cuda(), H)
+    ref = oracle.gram_grouped(bf16_bits(x), offs, len(counts))
+    Hc = H.cpu().numpy()
+    for g, n in enumerate(counts):
+        if n == 0:
+            assert np.all(Hc[g] == 0)
+        else:
+            assert rel_frobenius(Hc[g], ref[g]) <= GRAM_REL, g
+
+
+# ------------------------------------------------------------ scale search
+def _layer(name):
+    from scale_calibration_nvfp4_b200 import workloads
+    W, X = workloads.layer_inputs(name, "cuda")
+    return W, X
+
+
+def test_tiny_layer_all_rules(nv):
+    """Tiny-layer workload, every block: max, MSE and Local-Hessian codes."""
+    W, X = _layer("tiny")
+    wu = bf16_bits(W)
+    s_g = nv.global_scale(W)
+    sg = s_g.item()
+    assert sg == oracle.global_scale(wu)
+    H = torch.zeros(W.shape[1] // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate(X, H)
+    H64 = H.cpu().numpy().astype(np.float64)
+    assert rel_frobenius(H64, oracle.gram(bf16_bits(X))) <= GRAM_REL
+
+    cmax = nv.scale_search_max(W, s_g).cpu().numpy()
+    np.testing.assert_array_equal(cmax, oracle.scale_search_max(wu, sg))
+
+    cmse, omse = nv.scale_search_mse(W, s_g, return_objective=True)
+    rc, ro = oracle.scale_search_mse(wu, sg)
+    n_tie_mse = check_search_codes(cmse.cpu().numpy(), rc, wu, sg)
+    np.testing.assert_allclose(omse.cpu().numpy(), ro, rtol=1e-4, atol=1e-30)
+
+    clh, olh = nv.scale_search_local_hessian(W, s_g, H, return_objective=True)
+    rc, ro = oracle.scale_search_lh(wu, sg, H64)
+    n_tie_lh = check_search_codes(clh.cpu().numpy(), rc, wu, sg, H64)
+    np.testing.assert_allclose(olh.cpu().numpy(), ro, rtol=1e-4, atol=1e-30)
+    assert n_tie_mse + n_tie_lh < 10
+
+
+def test_identity_hessian_gives_mse_on_gpu(nv):
+    W, _ = _layer("tiny")
+    s_g = nv.global_scale(W)
+    nb = W.shape[1] // 16
+    H = torch.eye(16, device="cuda").repeat(nb, 1, 1) * 2.5
+    clh = nv.scale_search_local_hessian(W, s_g, H)
+    cmse = nv.scale_search_mse(W, s_g)
+    wu = bf16_bits(W)
+    rc, _ = oracle.scale_search_mse(wu, s_g.item())
+    check_search_codes(clh.cpu().numpy(), rc, wu, s_g.item())
+    check_search_codes(cmse.cpu().numpy(), rc, wu, s_g.item())
+
+
+def test_search_degenerate_blocks(nv):
+    """Zero blocks, a zero Hessian block, a rank-deficient Hessian (dead
+    channels) and blocks already on the NVFP4 grid (exact-zero ties)."""
+    x = rand_bf16((48, 64), 5, 0.02)
+    x[0, :16] = 0
+    s_g = nv.global_scale(x.cuda())
+    codes = nv.scale_search_max(x.cuda(), s_g)
+    packed = nv.quantize_pack(x.cuda(), s_g, codes)
+    y = nv.dequantize(packed, codes, s_g)
+    y[10:20] = x[10:20].cuda()      # half the rows back off the grid
+    W = y.contiguous()
+    wu = bf16_bits(W)
+    sg = s_g.item()
+    X = rand_bf16((200, 64), 6)
+    X[:, 20:23] = 0                 # dead channels in block 1
+    H = torch.zeros(4, 16, 16, device="cuda")
+    nv.hessian_accumulate(X.cuda(), H)
+    H[3] = 0                        # no calibration signal at all for block 3
+    H64 = H.cpu().numpy().astype(np.float64)
+    clh = nv.scale_search_local_hessian(W, s_g, H).cpu().numpy()
+    rc, _ = oracle.scale_search_lh(wu, sg, H64)
+    check_search_codes(clh, rc, wu, sg, H64)
+    assert np.all(clh[:, 3] == 1)   # every candidate ties at zero: smallest code
+    cm = nv.scale_search_mse(W, s_g).cpu().numpy()
+    rc, _ = oracle.scale_search_mse(wu, sg)
+    check_search_codes(cm, rc, wu, sg)
+    assert cm[0, 0] == 1
+
+
+def test_dense_layer_sampled(nv):
+    """Dense 4096x4096 workload (the benchmarked configuration): full GPU
+    search, 3000 sampled blocks per rule checked against the oracle."""
+    W, X = _layer("dense")
+    s_g = nv.global_scale(W)
+    sg = s_g.item()
+    wu = bf16_bits(W)
+    assert sg == oracle.global_scale(wu)
+    H = torch.zeros(W.shape[1] // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate(X, H)
+    H64 = H.cpu().numpy().astype(np.float64)
+    xu = bf16_bits(X)
+    cols = np.array([0, 17, 255])
+    ref_H = oracle.gram(np.ascontiguousarray(
+        np.concatenate([xu[:, 16 * j:16 * j + 16] for j in cols], axis=1)))
+    for i, j in enumerate(cols):
+        assert rel_frobenius(H64[j], ref_H[i]) <= GRAM_REL
+    rng = np.random.default_rng(11)
+    n = 3000
+    rows = rng.integers(0, W.shape[0], n)
+    blocks = rng.integers(0, W.shape[1] // 16, n)
+    cmax = nv.scale_search_max(W, s_g).cpu().numpy()
+    np.testing.assert_array_equal(cmax, oracle.scale_search_max(wu, sg))
+    cmse = nv.scale_search_mse(W, s_g).cpu().numpy()
+    rc, _ = oracle.scale_search_sampled(wu, sg, None, rows, blocks)
+    check_search_codes(cmse[rows, blocks], rc, wu, sg, None, rows, blocks)
+    clh = nv.scale_search_local_hessian(W, s_g, H).cpu().numpy()
+    rc, _ = oracle.scale_search_sampled(wu, sg, H64, rows, blocks)
+    check_search_codes(clh[rows, blocks], rc, wu, sg, H64, rows, blocks)
+    packed = nv.quantize_pack(W, s_g, torch.from_numpy(clh).cuda())
+    sub = np.unique(rows[:64])
+    rp = oracle.quantize_pack(wu[sub], sg, clh[sub])
+    np.testing.assert_array_equal(packed.cpu().numpy()[sub], rp)
+    y = nv.dequantize(packed, torch.from_numpy(clh).cuda(), s_g)
+    np.testing.assert_array_equal(bf16_bits(y)[sub], oracle.dequantize(rp, clh[sub], sg))
+
+
+def test_moe_experts_sampled(nv):
+    """MoE workload at full size: grouped Gram over 262,144 routed tokens,
+    per-expert tensor scales and batched Local-Hessian search; experts with
+    many and few tokens checked against the oracle."""
+    from scale_calibration_nvfp4_b200 import workloads
+    W, X, offsets = workloads.moe_inputs("cuda")
+    G, R, C = W.shape
+    nb = C // 16
+    s_g = nv.global_scale(W, batch=G)
+    H = torch.zeros(G, nb, 16, 16, device="cuda")
+    nv.hessian_accumulate_grouped(X, offsets.cuda(), H)
+    codes = nv.scale_search_local_hessian(W, s_g, H).cpu().numpy()
+    Hc = H.cpu().numpy().astype(np.float64)
+    wu_all = bf16_bits(W)
+    xu = bf16_bits(X)
+    rng = np.random.default_rng(3)
+    for e in (0, 1, 63, 127):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        assert hi > lo
+        sg = s_g[e].item()
+        assert sg == oracle.global_scale(wu_all[e])
+        cb = rng.integers(0, nb, 4)
+        ref_H = oracle.gram(np.ascontiguousarray(
+            np.concatenate([xu[lo:hi, 16 * j:16 * j + 16] for j in cb], axis=1)))
+        for i, j in enumerate(cb):
+            assert rel_frobenius(Hc[e, j], ref_H[i]) <= GRAM_REL
+        rows = rng.integers(0, R, 400)
+        blocks = rng.integers(0, nb, 400)
+        rc, _ = oracle.scale_search_sampled(wu_all[e], sg, Hc[e], rows, blocks)
+        check_search_codes(codes[e][rows, blocks], rc, wu_all[e], sg, Hc[e], rows, blocks)

@@ -132,11 +132,10 @@ class Path:
         }
 
 
-# LH search arithmetic per block (the form the kernel evaluates): per
-# candidate 16 FMA for delta, 136 FMA for L^T delta, 16 FMA for ||.||^2.
-LH_FLOP_PER_BLOCK = 126 * 2 * (16 + 136 + 16)
-# the same objective written as delta H delta^T (16 + 256 + 16 FMA)
-LH_FLOP_PER_BLOCK_FULL_FORM = 126 * 2 * (16 + 256 + 16)
+# Local-Hessian search work per block, counted on the definition E = delta
+# H_b delta^T: per candidate 256 FMA for H_b delta and 16 FMA for the dot
+# product, 2 flop each (the E2M1 encodes are not counted as flops).
+LH_FLOP_PER_BLOCK = 126 * 2 * (256 + 16)
 
 
 # ------------------------------------------------------------------ clocks
@@ -324,8 +323,7 @@ def run_gpu(args):
             "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 flop x %.0f MHz (%s clocks)"
                          % (sm_mhz_peak, pk_kind),
             "flop_per_block": LH_FLOP_PER_BLOCK,
-            "full_form_equivalent_TFLOP/s": round(
-                LH_FLOP_PER_BLOCK_FULL_FORM * blocks / (lh_ms / 1e3) / 1e12, 2),
+            "flop_basis": "definition delta H delta^T: 126 x (256 + 16) FMA per block",
         }
         hbm = float(pk.get("hbm_gbs", FALLBACK_HBM_GBS))
         streaming = {n: {"GB/s": kernels[n]["GB/s"], "frac_of_%s_hbm" % pk_kind:

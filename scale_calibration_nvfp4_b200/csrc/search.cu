@@ -7,43 +7,118 @@
 // the smallest weight error) and section "A different objective" (E(s) =
 // ||delta X||^2 = tr(delta X X^T delta^T); the block-diagonal approximation
 // solves each 16-value block alone against its 16x16 H_b, still trying all
-// 126 candidates).
+// 126 candidates).  MSE is the same search with H_b = I.
 //
-// Mapping: one CTA owns one column block b of one batch element and a run
-// of rows; one thread owns one row's block.  All threads of a CTA share H_b,
-// so its factor L (H_b = L L^T, fp64 Cholesky by one warp, semidefinite
-// pivots dropped) lives in every thread's registers as warp-uniform values
-// and E = ||L^T delta||^2 costs 136 + 16 FMA per candidate instead of 272.
-// Candidate scales and their reciprocal bracket sit in shared memory
-// (broadcast reads).  Each candidate's E2M1 codes come from the hardware
-// fp32 -> e2m1x2 conversion at both ends of the bracket t_lo <= |w|/s <= t_hi;
-// a disagreement (|w|/s within ~2^-23 of a rounding midpoint) falls back to
-// the exact fp64 midpoint test.
+// Work mapping.  A CTA owns one column block b of one batch element and a run
+// of rows; a warp takes 16 rows at a time, laid out like the A operand of a
+// 16x8x16 tensor-core MMA: lane (g, t) holds elements {2t, 2t+1, 2t+8, 2t+9}
+// of rows g and g+8.
 //
-// Exactness of the winner: the fp32 screen tracks the best two objectives.
-// If they are within 2^-12 relative, the row's block is re-scored in a second
-// pass: candidates whose fp32 objective lies inside that band are evaluated
-// in fp64 straight from H_b (delta H_b delta^T), and the first minimum in
-// ascending code order wins, as in the plain definition.
+// Per candidate scale s the objective is rewritten with H_b = L L^T (fp64
+// Cholesky once per CTA, semidefinite pivots dropped):
+//     E = ||L^T delta||^2,  delta = w - s v,   so   L^T delta = p - s u,
+// with p = L^T w fixed per row and u = L^T v.  The signed E2M1 values v are
+// exact in f16, so u comes from two f16 MMAs per 8 outputs against L split
+// into an f16 high and low part (22 significant bits), accumulated in fp32;
+// for MSE the B operand is the identity and u = v exactly.  The CUDA cores
+// only form z = p - s u and sum z^2.
+//
+// Exact E2M1 codes without a fallback branch.  Candidate values are o * 2^p
+// with odd o in {1, 3, ..., 15}, and s(c) = fl(s_g o) 2^p exactly, so for each
+// element and each odd part o the quotient q = |w| / fl(s_g o) is formed once:
+// t from a double-float reciprocal (within one ulp of q), and t_alt, the
+// neighbouring float on the other side of q, chosen by the exact sign of the
+// residual |w| - t fl(s_g o) (one fma).  Candidates of class o scale both by
+// 2^-p exactly.  Round-to-nearest-even of t and of t_alt (hardware e2m1x2
+// conversion) can only disagree when one of them is a rounding midpoint; q
+// then lies strictly on the other one's side and the correct code is the odd
+// one of the two (the tie went to the even one).
+//
+// Winner: fp32 screen keeping the best three objectives; when the best two
+// are within 2^-12 (relative) or the best is numerically zero, the candidates
+// in the band are re-scored in fp64 straight from the definition
+// (delta H_b delta^T with exact E2M1 codes) and the first minimum in
+// ascending code order wins.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace nvfp4 {
 namespace {
 
-constexpr int kSearchThreads = 128;
-constexpr int kRowIters = 4;
+constexpr int kThreads = 128;  // 4 warps
+constexpr int kWarps = kThreads / 32;
+constexpr int kTileRows = 16;
+constexpr int kTilesPerWarp = 4;
+constexpr int kRowsPerCta = kWarps * kTileRows * kTilesPerWarp;  // 256
 constexpr float kTieBand = 1.0f / 4096.0f;
-constexpr int kTriangle = 136;  // 16 * 17 / 2
+constexpr float kZeroFloor = 0x1p-40f;  // relative to ||p||^2
+constexpr int kMaxClasses = kCandidates;
 
-// Offset of column k in the packed lower triangle (column-major, rows j >= k).
-__host__ __device__ constexpr int tri_col(int k) { return 16 * k - (k * (k - 1)) / 2; }
+// Candidate classes by odd part o of the E4M3 value o * 2^p (p >= -9):
+// start of each class (o = 1, 3, ..., 15) in candidate order.
+__constant__ int kClassBegin[9] = {0, 18, 35, 51, 67, 82, 97, 112, 126};
 
-// Cooperative Cholesky of the 16x16 block in Hs (fp32, row-major) by warp 0,
-// lanes 0..15 owning one row each.  A pivot at or below 1e-12 of the largest
-// diagonal (or non-finite) drops its column, which keeps a positive
-// semidefinite H usable.  Writes the packed factor to Ls.
-__device__ void cholesky16(const float *Hs, float *Ls) {
+struct ClassInfo {
+  float S, r_hi, r_lo;  // S = fl(s_g o), 1/S = r_hi + r_lo
+  int end;              // one past its last candidate
+};
+struct CandInfo {
+  float f;      // 2^-p, scales the class quotient to this candidate
+  float s_mma;  // s / sigma_L (the MMA's B operand is L * sigma_L)
+  float s;      // effective scale fl(s_g e4m3(c))
+  int c;        // E4M3 code
+};
+
+// ----------------------------------------------------------------- helpers
+// Four e2m1x2 conversions packed into one word: byte i holds
+// (code(hi_i) << 4) | code(lo_i).
+__device__ __forceinline__ uint32_t cvt4_e2m1x2(float h0, float l0, float h1, float l1,
+                                                float h2, float l2, float h3, float l3) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %1, %2;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %3, %4;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %5, %6;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %7, %8;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(r)
+      : "f"(h0), "f"(l0), "f"(h1), "f"(l1), "f"(h2), "f"(l2), "f"(h3), "f"(l3));
+  return r;
+}
+
+// Four code bytes -> four f16x2 registers (low nibble -> low half).
+__device__ __forceinline__ void cvt4_f16x2(uint32_t codes, uint32_t a[4]) {
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "mov.b32 {q0, q1, q2, q3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, q2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, q3;\n\t}"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+      : "r"(codes));
+}
+
+__device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4], uint32_t b0,
+                                              uint32_t b1, const float c[4]) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]),
+        "f"(c[2]), "f"(c[3]));
+}
+
+__device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
+  return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+}
+
+// Cooperative Cholesky of the 16x16 block in Hs (fp32, row-major) by one
+// warp, lanes 0..15 owning one row each.  A pivot at or below 1e-12 of the
+// largest diagonal (or non-finite) drops its column, which keeps a positive
+// semidefinite H usable.  Writes the full lower-triangular factor (zeros above
+// the diagonal) to Lf.
+__device__ void cholesky16(const float *Hs, float *Lf) {
   const int lane = threadIdx.x & 31;
   const bool own = lane < 16;
   double a[16];
@@ -55,7 +130,8 @@ __device__ void cholesky16(const float *Hs, float *Ls) {
     if (j == lane) diag = a[j];
   double maxdiag = diag;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) maxdiag = fmax(maxdiag, __shfl_xor_sync(0xFFFFFFFFu, maxdiag, o));
+  for (int o = 16; o > 0; o >>= 1)
+    maxdiag = fmax(maxdiag, __shfl_xor_sync(0xFFFFFFFFu, maxdiag, o));
   const double tol = 1e-12 * maxdiag;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
@@ -65,7 +141,7 @@ __device__ void cholesky16(const float *Hs, float *Ls) {
     double lik = 0.0;
     if (lane == k) lik = piv;
     else if (own && lane > k && ok) lik = a[k] / piv;
-    if (own && lane >= k) Ls[tri_col(k) + (lane - k)] = (float)lik;
+    if (own) Lf[lane * 16 + k] = (float)lik;  // zero above the diagonal
 #pragma unroll
     for (int j = k + 1; j < 16; ++j) {
       const double ljk = __shfl_sync(0xFFFFFFFFu, lik, j);
@@ -74,187 +150,355 @@ __device__ void cholesky16(const float *Hs, float *Ls) {
   }
 }
 
-// fp32 objective of candidate c for one block, and the signed E2M1 values
-// v[] it uses.  `Lf` is the packed factor (registers in the screen, shared
-// memory in the re-score: both hold the same fp32 values and the arithmetic
-// below is a fixed sequence of fmaf, so both paths give identical results).
-template <bool kLH, typename LT>
-__device__ __forceinline__ float candidate_objective(const float x[16], const uint32_t sgn[8],
-                                                     const float4 t, const LT &Lf,
-                                                     float v[16]) {
-  const ScaleRecip rr = {t.x, t.y, t.z};
-  uint32_t bytes[8], mismatch = 0;
+// fp64 objective of candidate c for one block, from the definition: exact
+// E2M1 codes, delta_i = w_i - v_i s, E = delta H delta^T (MSE: H = I).
+__device__ double objective64(const float x[16], float s_g, int c, const float *Hs) {
+  const float s = effective_scale(s_g, (uint32_t)c);
+  double d[16];
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    bytes[j] = e2m1_pair_bracket(fabsf(x[2 * j]), fabsf(x[2 * j + 1]), rr, mismatch);
-  if (mismatch) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      bytes[j] = e2m1_mag_exact(fabsf(x[2 * j]), t.x) |
-                 (e2m1_mag_exact(fabsf(x[2 * j + 1]), t.x) << 4);
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t k = e2m1_mag_exact(fabsf(x[j]), s);
+    const double v = k < 2 ? 0.5 * k : (1.0 + 0.5 * (double)(k & 1)) * (double)(1 << ((k >> 1) - 1));
+    d[j] = (double)x[j] - copysign(v, (double)x[j]) * (double)s;
   }
-  float d[16];
+  double e = 0.0;
+  if (Hs) {
+    for (int j = 0; j < 16; ++j) {
+      double row = 0.0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t h2 = cvt_f16x2_from_e2m1x2(bytes[j] | sgn[j]);
-    v[2 * j] = f16_lo_to_float(h2);
-    v[2 * j + 1] = f16_hi_to_float(h2);
-    d[2 * j] = fmaf(-v[2 * j], t.x, x[2 * j]);
-    d[2 * j + 1] = fmaf(-v[2 * j + 1], t.x, x[2 * j + 1]);
-  }
-  float e = 0.0f;
-  if (kLH) {
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      float z = 0.0f;
-#pragma unroll
-      for (int j = k; j < 16; ++j) z = fmaf(Lf[tri_col(k) + (j - k)], d[j], z);
-      e = fmaf(z, z, e);
+      for (int k = 0; k < 16; ++k) row = fma((double)Hs[j * 16 + k], d[k], row);
+      e = fma(d[j], row, e);
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) e = fmaf(d[j], d[j], e);
+    for (int j = 0; j < 16; ++j) e = fma(d[j], d[j], e);
   }
   return e;
 }
 
-__device__ __forceinline__ void unpack_block(const uint32_t wv[8], float x[16], uint32_t sgn[8]) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    x[2 * j] = bf16_lo(wv[j]);
-    x[2 * j + 1] = bf16_hi(wv[j]);
-    sgn[j] = ((wv[j] >> 12) & 0x8u) | ((wv[j] >> 24) & 0x80u);
-  }
-}
-
-// Packed factor from shared memory with non-hoistable loads, so the compiler
-// keeps it out of registers outside the candidate loop that uses it.
-__device__ __forceinline__ void load_factor(const float *Ls, float L[kTriangle]) {
-  const uint32_t base = (uint32_t)__cvta_generic_to_shared(Ls);
-#pragma unroll
-  for (int i = 0; i < kTriangle; i += 4) {
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(L[i]), "=f"(L[i + 1]), "=f"(L[i + 2]), "=f"(L[i + 3])
-                 : "r"(base + 4 * i));
-  }
-}
-
-// Near-tie re-score of one block: every candidate whose fp32 objective is
-// within `band` is evaluated in fp64 from the definition (delta H delta^T, or
-// delta delta^T for MSE); the first minimum in ascending code order wins.
-template <bool kLH>
-__device__ __noinline__ int rescore_block(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
-                                          uint32_t w4, uint32_t w5, uint32_t w6, uint32_t w7,
-                                          const float4 *tab, const float *Ls, const float *Hs,
-                                          float band, double *best_out) {
-  const uint32_t wv[8] = {w0, w1, w2, w3, w4, w5, w6, w7};
+// Near-tie resolution for one block: fp64 scores of {c1, c2}, or of every
+// candidate when more than two may lie in the band; first minimum wins.
+__device__ __noinline__ int refine_block(const uint16_t *wrow, float s_g, const float *Hs,
+                                         int c1, int c2, bool full, float *obj) {
   float x[16];
-  uint32_t sgn[8];
-  unpack_block(wv, x, sgn);
+  {
+    const uint4 *q = reinterpret_cast<const uint4 *>(wrow);
+    const uint4 v0 = q[0], v1 = q[1];
+    const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      x[2 * j] = bf16_lo(wv[j]);
+      x[2 * j + 1] = bf16_hi(wv[j]);
+    }
+  }
   double best = __longlong_as_double(0x7FF0000000000000LL);
   int best_c = 1;
-  for (int c = 1; c <= kCandidates; ++c) {
-    const float4 t = tab[c - 1];
-    float v[16];
-    float L[kLH ? kTriangle : 4];
-    if (kLH) load_factor(Ls, L);
-    const float e = candidate_objective<kLH>(x, sgn, t, L, v);
-    if (!(e <= band)) continue;
-    double dd[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) dd[j] = (double)x[j] - (double)v[j] * (double)t.x;
-    double e64 = 0.0;
-    if (kLH) {
-      for (int j = 0; j < 16; ++j) {
-        double row = 0.0;
-        for (int k = 0; k < 16; ++k) row = fma((double)Hs[j * 16 + k], dd[k], row);
-        e64 = fma(dd[j], row, e64);
+  if (full) {
+    for (int c = 1; c <= kCandidates; ++c) {
+      const double e = objective64(x, s_g, c, Hs);
+      if (e < best) {
+        best = e;
+        best_c = c;
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) e64 = fma(dd[j], dd[j], e64);
     }
-    if (e64 < best) {
-      best = e64;
-      best_c = c;
+  } else {
+    const int lo = min(c1, c2), hi = max(c1, c2);
+    const double el = objective64(x, s_g, lo, Hs);
+    const double eh = objective64(x, s_g, hi, Hs);
+    best = el;
+    best_c = lo;
+    if (eh < el) {
+      best = eh;
+      best_c = hi;
     }
   }
-  *best_out = best;
+  *obj = (float)best;
   return best_c;
 }
 
+// Keep the three smallest objectives (codes of the best two).
+__device__ __forceinline__ void track3(float e, int c, float &b1, int &c1, float &b2, int &c2,
+                                       float &b3) {
+  const bool lt1 = e < b1, lt2 = e < b2;
+  b3 = fminf(b3, fmaxf(b2, e));
+  c2 = lt1 ? c1 : (lt2 ? c : c2);
+  b2 = fminf(b2, fmaxf(b1, e));
+  c1 = lt1 ? c : c1;
+  b1 = fminf(b1, e);
+}
+
+// Select word t (0..3) of four without local memory.
+__device__ __forceinline__ uint32_t pick4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                          int t) {
+  return t == 0 ? w0 : (t == 1 ? w1 : (t == 2 ? w2 : w3));
+}
+
 template <bool kLH>
-__global__ void __launch_bounds__(kSearchThreads)
+__global__ void __launch_bounds__(kThreads)
     search_kernel(const uint16_t *__restrict__ w, int64_t R, int64_t C,
-                  const float *__restrict__ s_g, const float *__restrict__ H,
+                  const float *__restrict__ s_g_arr, const float *__restrict__ H,
                   uint8_t *__restrict__ codes, float *__restrict__ best_obj) {
   const int64_t nb = C / kBlock;
   const int64_t b = blockIdx.y;
   const int64_t batch = blockIdx.z;
-  const int64_t row0 = (int64_t)blockIdx.x * kSearchThreads * kRowIters;
+  const int64_t row_base = (int64_t)blockIdx.x * kRowsPerCta;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
 
-  __shared__ float4 tab[kCandidates];
+  __shared__ ClassInfo cls[kMaxClasses];
+  __shared__ CandInfo cand[kCandidates];
   __shared__ float Hs[kLH ? 256 : 1];
-  __shared__ __align__(16) float Ls[kLH ? kTriangle : 4];
+  __shared__ float Lf[kLH ? 256 : 1];
+  __shared__ float sigma_sh;
+  __shared__ int ncls_sh, zero_h_sh;
 
-  const float sg = s_g[batch];
-  for (int c = threadIdx.x; c < kCandidates; c += kSearchThreads) {
-    const float s = effective_scale(sg, (uint32_t)(c + 1));
-    const ScaleRecip r = make_recip(s);
-    tab[c] = make_float4(s, r.r_lo, r.r_hi, 0.0f);
-  }
-  if (kLH) {
-    const float *Hb = H + (batch * nb + b) * 256;
-    for (int i = threadIdx.x; i < 256; i += kSearchThreads) Hs[i] = Hb[i];
-    __syncthreads();
-    if (threadIdx.x < 32) cholesky16(Hs, Ls);
-  }
-  __syncthreads();
-
+  const float s_g = s_g_arr[batch];
   const uint16_t *wb = w + batch * R * C + b * kBlock;
   uint8_t *cb = codes + batch * R * nb + b;
   float *ob = best_obj ? best_obj + batch * R * nb + b : nullptr;
 
-  for (int it = 0; it < kRowIters; ++it) {
-    const int64_t r = row0 + it * kSearchThreads + threadIdx.x;
-    if (r >= R) break;
-    uint32_t wv[8];
-    {
-      const uint4 *q = reinterpret_cast<const uint4 *>(wb + r * C);
-      const uint4 v0 = ld_stream_v4(q), v1 = ld_stream_v4(q + 1);
-      wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w;
-      wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
-    }
-    float x[16];
-    uint32_t sgn[8];
-    unpack_block(wv, x, sgn);
-    // the factor is reloaded per row so that it is not live across the
-    // (rare) re-score call
-    float L[kLH ? kTriangle : 4];
-    if (kLH) load_factor(Ls, L);
-
-    float best1 = __int_as_float(0x7F800000), best2 = __int_as_float(0x7F800000);
-    int c1 = 1;
-    for (int c = 1; c <= kCandidates; ++c) {
-      float v[16];
-      const float e = candidate_objective<kLH>(x, sgn, tab[c - 1], L, v);
-      if (e < best1) {
-        best2 = best1;
-        best1 = e;
-        c1 = c;
-      } else {
-        best2 = fminf(best2, e);
+  // ---- factor of H_b, its scale for f16, and the zero-H shortcut
+  if (kLH) {
+    const float *Hb = H + (batch * nb + b) * 256;
+    for (int i = threadIdx.x; i < 256; i += kThreads) Hs[i] = Hb[i];
+    __syncthreads();
+    if (warp == 0) {
+      cholesky16(Hs, Lf);
+      __syncwarp();
+      float m = 0.0f;
+      for (int i = lane; i < 256; i += 32) m = fmaxf(m, fabsf(Lf[i]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      if (lane == 0) {
+        int e = 0;
+        frexpf(m, &e);  // m < 2^e
+        sigma_sh = m > 0.0f ? ldexpf(1.0f, 15 - e) : 1.0f;
+        zero_h_sh = !(m > 0.0f);
       }
     }
-    float obj = best1;
-    if (best2 - best1 <= kTieBand * best2) {
-      double e64;
-      c1 = rescore_block<kLH>(wv[0], wv[1], wv[2], wv[3], wv[4], wv[5], wv[6], wv[7], tab, Ls,
-                              Hs, best1 + kTieBand * best2, &e64);
-      obj = (float)e64;
+  } else if (threadIdx.x == 0) {
+    sigma_sh = 1.0f;
+    zero_h_sh = 0;
+  }
+  __syncthreads();
+  const float sigma = sigma_sh;
+
+  if (kLH && zero_h_sh) {  // every candidate scores 0: the smallest code wins
+    const int64_t r_end = min(R, row_base + kRowsPerCta);
+    for (int64_t r = row_base + threadIdx.x; r < r_end; r += kThreads) {
+      cb[r * nb] = 1;
+      if (ob) ob[r * nb] = 0.0f;
     }
-    cb[r * nb] = (uint8_t)c1;
-    if (ob) ob[r * nb] = obj;
+    return;
+  }
+
+  // ---- candidate tables (per CTA, from this batch element's s_g)
+  const bool by_class = s_g >= 0x1p-100f && s_g < 0x1p100f;
+  if (threadIdx.x < kCandidates) {
+    const int c = threadIdx.x + 1;
+    const int M = c < 8 ? c : 8 + (c & 7);
+    const int E = c < 8 ? -9 : (c >> 3) - 10;
+    const int tz = __ffs(M) - 1;
+    const int o = M >> tz, p = E + tz;
+    const int k = (o - 1) >> 1;
+    const float s = effective_scale(s_g, (uint32_t)c);
+    const int pos = by_class ? kClassBegin[k] + (p + 9) : c - 1;
+    CandInfo ci;
+    ci.f = by_class ? ldexpf(1.0f, -p) : 1.0f;
+    ci.s = s;
+    ci.s_mma = s / sigma;  // sigma is a power of two: exact
+    ci.c = c;
+    cand[pos] = ci;
+    const int ncls = by_class ? 8 : kCandidates;
+    if (threadIdx.x < ncls) {
+      const float S = by_class ? __fmul_rn(s_g, (float)(2 * threadIdx.x + 1)) : s;
+      const double rr = 1.0 / (double)S;
+      ClassInfo k2;
+      k2.S = S;
+      k2.r_hi = (float)rr;
+      k2.r_lo = (float)(rr - (double)k2.r_hi);
+      k2.end = by_class ? kClassBegin[threadIdx.x + 1] : (int)threadIdx.x + 1;
+      cls[threadIdx.x] = k2;
+    }
+    if (threadIdx.x == 0) ncls_sh = ncls;
+  }
+  __syncthreads();
+  const int ncls = ncls_sh;
+
+  // ---- B operand fragments: L * sigma split in f16 hi + lo (LH) or I (MSE)
+  uint32_t bh[2][2], bl[2][2];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    const int n = nt * 8 + g;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int k0 = 2 * t + 8 * half;
+      if (kLH) {
+        const float x0 = Lf[k0 * 16 + n] * sigma, x1 = Lf[(k0 + 1) * 16 + n] * sigma;
+        const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+        const __half l0 = __float2half_rn(x0 - __half2float(h0));
+        const __half l1 = __float2half_rn(x1 - __half2float(h1));
+        bh[nt][half] = pack_half2(h0, h1);
+        bl[nt][half] = pack_half2(l0, l1);
+      } else {
+        bh[nt][half] = pack_half2(__float2half_rn(k0 == n ? 1.0f : 0.0f),
+                                  __float2half_rn(k0 + 1 == n ? 1.0f : 0.0f));
+        bl[nt][half] = 0u;
+      }
+    }
+  }
+
+  for (int tile = 0; tile < kTilesPerWarp; ++tile) {
+    const int64_t r0 = row_base + (int64_t)(tile * kWarps + warp) * kTileRows;
+    if (r0 >= R) break;
+    const int64_t rg = r0 + g, rg8 = r0 + g + 8;
+    // full rows g and g+8 (zeros past the end)
+    uint32_t W0[8], W1[8];
+    {
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      const uint4 *q0 = reinterpret_cast<const uint4 *>(wb + rg * C);
+      const uint4 *q1 = reinterpret_cast<const uint4 *>(wb + rg8 * C);
+      const uint4 a0 = rg < R ? ld_stream_v4(q0) : z, a1 = rg < R ? ld_stream_v4(q0 + 1) : z;
+      const uint4 c0 = rg8 < R ? ld_stream_v4(q1) : z, c1 = rg8 < R ? ld_stream_v4(q1 + 1) : z;
+      W0[0] = a0.x; W0[1] = a0.y; W0[2] = a0.z; W0[3] = a0.w;
+      W0[4] = a1.x; W0[5] = a1.y; W0[6] = a1.z; W0[7] = a1.w;
+      W1[0] = c0.x; W1[1] = c0.y; W1[2] = c0.z; W1[3] = c0.w;
+      W1[4] = c1.x; W1[5] = c1.y; W1[6] = c1.z; W1[7] = c1.w;
+    }
+    // this lane's four pairs in MMA order: (g,2t) (g+8,2t) (g,2t+8) (g+8,2t+8)
+    const uint32_t pw[4] = {pick4(W0[0], W0[1], W0[2], W0[3], t),
+                            pick4(W1[0], W1[1], W1[2], W1[3], t),
+                            pick4(W0[4], W0[5], W0[6], W0[7], t),
+                            pick4(W1[4], W1[5], W1[6], W1[7], t)};
+    // element k of the lane in C order: 2i, 2i+1 = low, high half of pair i
+    float xs[8], a[8];
+    uint32_t sgn = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      xs[2 * i] = bf16_lo(pw[i]);
+      xs[2 * i + 1] = bf16_hi(pw[i]);
+      a[2 * i] = fabsf(xs[2 * i]);
+      a[2 * i + 1] = fabsf(xs[2 * i + 1]);
+      sgn |= (((pw[i] >> 12) & 0x8u) | ((pw[i] >> 24) & 0x80u)) << (8 * i);
+    }
+    // p = L^T w at the C positions: pz[nt][0..1] row g, n = 8nt + 2t + {0,1};
+    // pz[nt][2..3] row g+8, same n
+    float pz[2][4];
+    if (kLH) {
+      float xr0[16], xr1[16];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        xr0[2 * j] = bf16_lo(W0[j]);
+        xr0[2 * j + 1] = bf16_hi(W0[j]);
+        xr1[2 * j] = bf16_lo(W1[j]);
+        xr1[2 * j + 1] = bf16_hi(W1[j]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int n = nt * 8 + 2 * t + e;
+          float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float l = Lf[j * 16 + n];
+            s0 = fmaf(l, xr0[j], s0);
+            s1 = fmaf(l, xr1[j], s1);
+          }
+          pz[nt][e] = s0;
+          pz[nt][2 + e] = s1;
+        }
+      }
+    } else {
+      pz[0][0] = xs[0]; pz[0][1] = xs[1]; pz[0][2] = xs[2]; pz[0][3] = xs[3];
+      pz[1][0] = xs[4]; pz[1][1] = xs[5]; pz[1][2] = xs[6]; pz[1][3] = xs[7];
+    }
+    float pp0 = pz[0][0] * pz[0][0] + pz[0][1] * pz[0][1] + pz[1][0] * pz[1][0] +
+                pz[1][1] * pz[1][1];
+    float pp1 = pz[0][2] * pz[0][2] + pz[0][3] * pz[0][3] + pz[1][2] * pz[1][2] +
+                pz[1][3] * pz[1][3];
+    pp0 += __shfl_xor_sync(0xFFFFFFFFu, pp0, 1);
+    pp0 += __shfl_xor_sync(0xFFFFFFFFu, pp0, 2);
+    pp1 += __shfl_xor_sync(0xFFFFFFFFu, pp1, 1);
+    pp1 += __shfl_xor_sync(0xFFFFFFFFu, pp1, 2);
+
+    const float inf = __int_as_float(0x7F800000);
+    float b1[2] = {inf, inf}, b2[2] = {inf, inf}, b3[2] = {inf, inf};
+    int c1[2] = {1, 1}, c2[2] = {1, 1};
+    const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+
+    int j = 0;
+    for (int k = 0; k < ncls; ++k) {
+      const ClassInfo ci = cls[k];
+      // class quotient t and its neighbour across q, per element
+      float tq[8], ta[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float tt = fmaf(a[e], ci.r_hi, a[e] * ci.r_lo);
+        const float rho = fmaf(-tt, ci.S, a[e]);
+        const int step = (rho > 0.0f) - (rho < 0.0f);
+        tq[e] = tt;
+        ta[e] = __int_as_float(__float_as_int(tt) + step);
+      }
+      for (; j < ci.end; ++j) {
+        const CandInfo cd = cand[j];
+        const float f = cd.f;
+        const uint32_t ct = cvt4_e2m1x2(tq[1] * f, tq[0] * f, tq[3] * f, tq[2] * f,
+                                        tq[5] * f, tq[4] * f, tq[7] * f, tq[6] * f);
+        const uint32_t ca = cvt4_e2m1x2(ta[1] * f, ta[0] * f, ta[3] * f, ta[2] * f,
+                                        ta[5] * f, ta[4] * f, ta[7] * f, ta[6] * f);
+        const uint32_t odd = (ct & 0x11111111u) * 15u;
+        const uint32_t code = ((ct & odd) | (ca & ~odd)) | sgn;
+        uint32_t A[4];
+        cvt4_f16x2(code, A);
+        float u0[4], u1[4];
+        mma_f16_16816(u0, A, bh[0][0], bh[0][1], zero4);
+        mma_f16_16816(u1, A, bh[1][0], bh[1][1], zero4);
+        if (kLH) {
+          mma_f16_16816(u0, A, bl[0][0], bl[0][1], u0);
+          mma_f16_16816(u1, A, bl[1][0], bl[1][1], u1);
+        }
+        const float sm = cd.s_mma;
+        const float z00 = fmaf(-sm, u0[0], pz[0][0]), z01 = fmaf(-sm, u0[1], pz[0][1]);
+        const float z02 = fmaf(-sm, u0[2], pz[0][2]), z03 = fmaf(-sm, u0[3], pz[0][3]);
+        const float z10 = fmaf(-sm, u1[0], pz[1][0]), z11 = fmaf(-sm, u1[1], pz[1][1]);
+        const float z12 = fmaf(-sm, u1[2], pz[1][2]), z13 = fmaf(-sm, u1[3], pz[1][3]);
+        float e0 = fmaf(z00, z00, fmaf(z01, z01, fmaf(z10, z10, z11 * z11)));
+        float e1 = fmaf(z02, z02, fmaf(z03, z03, fmaf(z12, z12, z13 * z13)));
+        e0 += __shfl_xor_sync(0xFFFFFFFFu, e0, 1);
+        e1 += __shfl_xor_sync(0xFFFFFFFFu, e1, 1);
+        e0 += __shfl_xor_sync(0xFFFFFFFFu, e0, 2);
+        e1 += __shfl_xor_sync(0xFFFFFFFFu, e1, 2);
+        track3(e0, cd.c, b1[0], c1[0], b2[0], c2[0], b3[0]);
+        track3(e1, cd.c, b1[1], c1[1], b2[1], c2[1], b3[1]);
+      }
+    }
+
+    // lane t = 0 finishes row g, lane t = 1 row g + 8
+    if (t < 2) {
+      const int h = t;
+      const int64_t r = h ? rg8 : rg;
+      if (r < R) {
+        bool zero_blk = true;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) zero_blk = zero_blk && (((h ? W1[i] : W0[i]) & 0x7FFF7FFFu) == 0u);
+        const float pp = h ? pp1 : pp0;
+        const float fl = kZeroFloor * pp;
+        int code = h ? c1[1] : c1[0];
+        float obj = h ? b1[1] : b1[0];
+        const float e1b = h ? b1[1] : b1[0], e2b = h ? b2[1] : b2[0], e3b = h ? b3[1] : b3[0];
+        if (zero_blk) {  // every candidate scores exactly 0
+          code = 1;
+          obj = 0.0f;
+        } else if (e2b - e1b <= kTieBand * e2b || e1b <= fl) {
+          const bool full = !(e3b - e1b > kTieBand * e3b + fl);
+          code = refine_block(wb + r * C, s_g, kLH ? Hs : nullptr, h ? c1[1] : c1[0],
+                              h ? c2[1] : c2[0], full, &obj);
+        }
+        cb[r * nb] = (uint8_t)code;
+        if (ob) ob[r * nb] = obj;
+      }
+    }
   }
 }
 
@@ -264,14 +508,12 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
                                 const float *s_g, const float *H, uint8_t *codes,
                                 float *best_obj, int local_hessian, cudaStream_t st) {
   if (R == 0 || C == 0) return cudaSuccess;
-  const int64_t rows_per_cta = (int64_t)kSearchThreads * kRowIters;
-  dim3 grid((unsigned)((R + rows_per_cta - 1) / rows_per_cta), (unsigned)(C / kBlock),
+  dim3 grid((unsigned)((R + kRowsPerCta - 1) / kRowsPerCta), (unsigned)(C / kBlock),
             (unsigned)batch);
   if (local_hessian)
-    search_kernel<true><<<grid, kSearchThreads, 0, st>>>(w, R, C, s_g, H, codes, best_obj);
+    search_kernel<true><<<grid, kThreads, 0, st>>>(w, R, C, s_g, H, codes, best_obj);
   else
-    search_kernel<false><<<grid, kSearchThreads, 0, st>>>(w, R, C, s_g, nullptr, codes,
-                                                          best_obj);
+    search_kernel<false><<<grid, kThreads, 0, st>>>(w, R, C, s_g, nullptr, codes, best_obj);
   return cudaGetLastError();
 }
 

@@ -66,7 +66,7 @@ struct ClassInfo {
 };
 struct CandInfo {
   float f;      // 2^-p, scales the class quotient to this candidate
-  float s_mma;  // s / sigma_L (the MMA's B operand is L * sigma_L)
+  float pad;
   float s;      // effective scale fl(s_g e4m3(c))
   int c;        // E4M3 code
 };
@@ -151,11 +151,13 @@ __device__ void cholesky16(const float *Hs, float *Lf) {
 }
 
 // fp64 objective of candidate c for one block, from the definition: exact
-// E2M1 codes, delta_i = w_i - v_i s, E = delta H delta^T (MSE: H = I).
-__device__ double objective64(const float x[16], float s_g, int c, const float *Hs) {
+// E2M1 codes, delta_i = w_i - v_i s, E = delta H delta^T (MSE: H = I).  Rare
+// path: loops are kept rolled so that the caller's register budget is not
+// raised by it.
+__device__ __noinline__ double objective64(const float *x, float s_g, int c, const float *Hs) {
   const float s = effective_scale(s_g, (uint32_t)c);
   double d[16];
-#pragma unroll
+#pragma unroll 1
   for (int j = 0; j < 16; ++j) {
     const uint32_t k = e2m1_mag_exact(fabsf(x[j]), s);
     const double v = k < 2 ? 0.5 * k : (1.0 + 0.5 * (double)(k & 1)) * (double)(1 << ((k >> 1) - 1));
@@ -163,14 +165,15 @@ __device__ double objective64(const float x[16], float s_g, int c, const float *
   }
   double e = 0.0;
   if (Hs) {
+#pragma unroll 1
     for (int j = 0; j < 16; ++j) {
       double row = 0.0;
-#pragma unroll
+#pragma unroll 4
       for (int k = 0; k < 16; ++k) row = fma((double)Hs[j * 16 + k], d[k], row);
       e = fma(d[j], row, e);
     }
   } else {
-#pragma unroll
+#pragma unroll 1
     for (int j = 0; j < 16; ++j) e = fma(d[j], d[j], e);
   }
   return e;
@@ -181,19 +184,12 @@ __device__ double objective64(const float x[16], float s_g, int c, const float *
 __device__ __noinline__ int refine_block(const uint16_t *wrow, float s_g, const float *Hs,
                                          int c1, int c2, bool full, float *obj) {
   float x[16];
-  {
-    const uint4 *q = reinterpret_cast<const uint4 *>(wrow);
-    const uint4 v0 = q[0], v1 = q[1];
-    const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      x[2 * j] = bf16_lo(wv[j]);
-      x[2 * j + 1] = bf16_hi(wv[j]);
-    }
-  }
+#pragma unroll 1
+  for (int j = 0; j < 16; ++j) x[j] = __uint_as_float((uint32_t)wrow[j] << 16);
   double best = __longlong_as_double(0x7FF0000000000000LL);
   int best_c = 1;
   if (full) {
+#pragma unroll 1
     for (int c = 1; c <= kCandidates; ++c) {
       const double e = objective64(x, s_g, c, Hs);
       if (e < best) {
@@ -216,15 +212,19 @@ __device__ __noinline__ int refine_block(const uint16_t *wrow, float s_g, const 
   return best_c;
 }
 
-// Keep the three smallest objectives (codes of the best two).
-__device__ __forceinline__ void track3(float e, int c, float &b1, int &c1, float &b2, int &c2,
-                                       float &b3) {
-  const bool lt1 = e < b1, lt2 = e < b2;
-  b3 = fminf(b3, fmaxf(b2, e));
-  c2 = lt1 ? c1 : (lt2 ? c : c2);
-  b2 = fminf(b2, fmaxf(b1, e));
-  c1 = lt1 ? c : c1;
-  b1 = fminf(b1, e);
+// Objective and code in one sortable value: a non-negative float whose seven
+// lowest mantissa bits are replaced by the code (relative change below
+// 2^-16, far inside the re-score band); equal objectives order by code.
+__device__ __forceinline__ float key_of(float e, int c) {
+  return __int_as_float((__float_as_int(e) & ~0x7F) | c);
+}
+__device__ __forceinline__ int code_of(float key) { return __float_as_int(key) & 0x7F; }
+
+// Keep the three smallest keys.
+__device__ __forceinline__ void track3(float key, float &b1, float &b2, float &b3) {
+  b3 = fminf(b3, fmaxf(b2, key));
+  b2 = fminf(b2, fmaxf(b1, key));
+  b1 = fminf(b1, key);
 }
 
 // Select word t (0..3) of four without local memory.
@@ -244,6 +244,7 @@ __global__ void __launch_bounds__(kThreads)
   const int64_t row_base = (int64_t)blockIdx.x * kRowsPerCta;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
+  const bool upper = t >= 2;  // which of the lane's two rows it finishes
 
   __shared__ ClassInfo cls[kMaxClasses];
   __shared__ CandInfo cand[kCandidates];
@@ -304,9 +305,9 @@ __global__ void __launch_bounds__(kThreads)
     const float s = effective_scale(s_g, (uint32_t)c);
     const int pos = by_class ? kClassBegin[k] + (p + 9) : c - 1;
     CandInfo ci;
+    ci.pad = 0.0f;
     ci.f = by_class ? ldexpf(1.0f, -p) : 1.0f;
     ci.s = s;
-    ci.s_mma = s / sigma;  // sigma is a power of two: exact
     ci.c = c;
     cand[pos] = ci;
     const int ncls = by_class ? 8 : kCandidates;
@@ -365,6 +366,12 @@ __global__ void __launch_bounds__(kThreads)
       W1[0] = c0.x; W1[1] = c0.y; W1[2] = c0.z; W1[3] = c0.w;
       W1[4] = c1.x; W1[5] = c1.y; W1[6] = c1.z; W1[7] = c1.w;
     }
+    bool zero0 = true, zero1 = true;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      zero0 = zero0 && ((W0[i] & 0x7FFF7FFFu) == 0u);
+      zero1 = zero1 && ((W1[i] & 0x7FFF7FFFu) == 0u);
+    }
     // this lane's four pairs in MMA order: (g,2t) (g+8,2t) (g,2t+8) (g+8,2t+8)
     const uint32_t pw[4] = {pick4(W0[0], W0[1], W0[2], W0[3], t),
                             pick4(W1[0], W1[1], W1[2], W1[3], t),
@@ -382,37 +389,37 @@ __global__ void __launch_bounds__(kThreads)
       sgn |= (((pw[i] >> 12) & 0x8u) | ((pw[i] >> 24) & 0x80u)) << (8 * i);
     }
     // p = L^T w at the C positions: pz[nt][0..1] row g, n = 8nt + 2t + {0,1};
-    // pz[nt][2..3] row g+8, same n
+    // pz[nt][2..3] row g+8, same n.  Local-Hessian: from the tensor cores
+    // with w scaled by 2^kw (exact; the tile maximum lands in [2^14, 2^15) in
+    // f16), so pz and every z below carry the factor sigma_L 2^kw, removed
+    // from the reported objective at the end.  MSE: p = w.
     float pz[2][4];
+    float zscale = 1.0f;  // objectives carry zscale^2
     if (kLH) {
-      float xr0[16], xr1[16];
+      uint32_t m = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        xr0[2 * j] = bf16_lo(W0[j]);
-        xr0[2 * j + 1] = bf16_hi(W0[j]);
-        xr1[2 * j] = bf16_lo(W1[j]);
-        xr1[2 * j + 1] = bf16_hi(W1[j]);
-      }
+      for (int i = 0; i < 8; ++i) m = __vmaxu2(m, __vmaxu2(W0[i] & 0x7FFF7FFFu, W1[i] & 0x7FFF7FFFu));
+      m = max(m & 0xFFFFu, m >> 16);
+      m = __reduce_max_sync(0xFFFFFFFFu, m);
+      const int emax = (int)(m >> 7) - 127;  // exponent of the tile's largest |w|
+      const int kw = m ? 14 - emax : 0;
+      const float wsc = ldexpf(1.0f, kw);
+      zscale = sigma * wsc;
+      uint32_t Aw[4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int n = nt * 8 + 2 * t + e;
-          float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float l = Lf[j * 16 + n];
-            s0 = fmaf(l, xr0[j], s0);
-            s1 = fmaf(l, xr1[j], s1);
-          }
-          pz[nt][e] = s0;
-          pz[nt][2 + e] = s1;
-        }
-      }
+      for (int i = 0; i < 4; ++i)
+        Aw[i] = pack_half2(__float2half_rn(xs[2 * i] * wsc), __float2half_rn(xs[2 * i + 1] * wsc));
+      const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      mma_f16_16816(pz[0], Aw, bh[0][0], bh[0][1], zero4);
+      mma_f16_16816(pz[1], Aw, bh[1][0], bh[1][1], zero4);
+      mma_f16_16816(pz[0], Aw, bl[0][0], bl[0][1], pz[0]);
+      mma_f16_16816(pz[1], Aw, bl[1][0], bl[1][1], pz[1]);
     } else {
       pz[0][0] = xs[0]; pz[0][1] = xs[1]; pz[0][2] = xs[2]; pz[0][3] = xs[3];
       pz[1][0] = xs[4]; pz[1][1] = xs[5]; pz[1][2] = xs[6]; pz[1][3] = xs[7];
     }
+    // multiplier of u in z: s for MSE; s 2^kw for Local-Hessian (u carries sigma_L)
+    const float umul = kLH ? zscale / sigma : 1.0f;
     float pp0 = pz[0][0] * pz[0][0] + pz[0][1] * pz[0][1] + pz[1][0] * pz[1][0] +
                 pz[1][1] * pz[1][1];
     float pp1 = pz[0][2] * pz[0][2] + pz[0][3] * pz[0][3] + pz[1][2] * pz[1][2] +
@@ -421,10 +428,8 @@ __global__ void __launch_bounds__(kThreads)
     pp0 += __shfl_xor_sync(0xFFFFFFFFu, pp0, 2);
     pp1 += __shfl_xor_sync(0xFFFFFFFFu, pp1, 1);
     pp1 += __shfl_xor_sync(0xFFFFFFFFu, pp1, 2);
-
     const float inf = __int_as_float(0x7F800000);
-    float b1[2] = {inf, inf}, b2[2] = {inf, inf}, b3[2] = {inf, inf};
-    int c1[2] = {1, 1}, c2[2] = {1, 1};
+    float b1 = inf, b2 = inf, b3 = inf;
     const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 
     int j = 0;
@@ -458,42 +463,37 @@ __global__ void __launch_bounds__(kThreads)
           mma_f16_16816(u0, A, bl[0][0], bl[0][1], u0);
           mma_f16_16816(u1, A, bl[1][0], bl[1][1], u1);
         }
-        const float sm = cd.s_mma;
+        const float sm = cd.s * umul;
         const float z00 = fmaf(-sm, u0[0], pz[0][0]), z01 = fmaf(-sm, u0[1], pz[0][1]);
         const float z02 = fmaf(-sm, u0[2], pz[0][2]), z03 = fmaf(-sm, u0[3], pz[0][3]);
         const float z10 = fmaf(-sm, u1[0], pz[1][0]), z11 = fmaf(-sm, u1[1], pz[1][1]);
         const float z12 = fmaf(-sm, u1[2], pz[1][2]), z13 = fmaf(-sm, u1[3], pz[1][3]);
-        float e0 = fmaf(z00, z00, fmaf(z01, z01, fmaf(z10, z10, z11 * z11)));
-        float e1 = fmaf(z02, z02, fmaf(z03, z03, fmaf(z12, z12, z13 * z13)));
-        e0 += __shfl_xor_sync(0xFFFFFFFFu, e0, 1);
-        e1 += __shfl_xor_sync(0xFFFFFFFFu, e1, 1);
-        e0 += __shfl_xor_sync(0xFFFFFFFFu, e0, 2);
-        e1 += __shfl_xor_sync(0xFFFFFFFFu, e1, 2);
-        track3(e0, cd.c, b1[0], c1[0], b2[0], c2[0], b3[0]);
-        track3(e1, cd.c, b1[1], c1[1], b2[1], c2[1], b3[1]);
+        const float e0 = fmaf(z00, z00, fmaf(z01, z01, fmaf(z10, z10, z11 * z11)));
+        const float e1 = fmaf(z02, z02, fmaf(z03, z03, fmaf(z12, z12, z13 * z13)));
+        // reduce-scatter over the quad: lanes t < 2 end with row g, t >= 2 with
+        // row g + 8 (sums in the same order on every lane of a pair)
+        float mine = upper ? e1 : e0;
+        const float other = upper ? e0 : e1;
+        mine += __shfl_xor_sync(0xFFFFFFFFu, other, 2);
+        mine += __shfl_xor_sync(0xFFFFFFFFu, mine, 1);
+        track3(key_of(mine, cd.c), b1, b2, b3);
       }
     }
 
-    // lane t = 0 finishes row g, lane t = 1 row g + 8
-    if (t < 2) {
-      const int h = t;
-      const int64_t r = h ? rg8 : rg;
+    // lane t = 0 finishes row g, lane t = 2 row g + 8
+    if ((t & 1) == 0) {
+      const int64_t r = upper ? rg8 : rg;
       if (r < R) {
-        bool zero_blk = true;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) zero_blk = zero_blk && (((h ? W1[i] : W0[i]) & 0x7FFF7FFFu) == 0u);
-        const float pp = h ? pp1 : pp0;
-        const float fl = kZeroFloor * pp;
-        int code = h ? c1[1] : c1[0];
-        float obj = h ? b1[1] : b1[0];
-        const float e1b = h ? b1[1] : b1[0], e2b = h ? b2[1] : b2[0], e3b = h ? b3[1] : b3[0];
-        if (zero_blk) {  // every candidate scores exactly 0
+        const float fl = kZeroFloor * (upper ? pp1 : pp0);
+        int code = code_of(b1);
+        float obj = b1 / (zscale * zscale);
+        if (upper ? zero1 : zero0) {  // every candidate scores exactly 0
           code = 1;
           obj = 0.0f;
-        } else if (e2b - e1b <= kTieBand * e2b || e1b <= fl) {
-          const bool full = !(e3b - e1b > kTieBand * e3b + fl);
-          code = refine_block(wb + r * C, s_g, kLH ? Hs : nullptr, h ? c1[1] : c1[0],
-                              h ? c2[1] : c2[0], full, &obj);
+        } else if (b2 - b1 <= kTieBand * b2 || b1 <= fl) {
+          const bool full = !(b3 - b1 > kTieBand * b3 + fl);
+          code = refine_block(wb + r * C, s_g, kLH ? Hs : nullptr, code_of(b1), code_of(b2), full,
+                              &obj);
         }
         cb[r * nb] = (uint8_t)code;
         if (ob) ob[r * nb] = obj;

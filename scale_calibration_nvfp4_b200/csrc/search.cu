@@ -50,7 +50,18 @@ namespace {
 constexpr int kThreads = 128;  // 4 warps
 constexpr int kWarps = kThreads / 32;
 constexpr int kTileRows = 16;
-constexpr int kTilesPerWarp = 4;
+#ifndef NVFP4_SEARCH_TILES
+#define NVFP4_SEARCH_TILES 4
+#endif
+#ifndef NVFP4_SEARCH_UNROLL
+#define NVFP4_SEARCH_UNROLL 2
+#endif
+#ifndef NVFP4_SEARCH_ALT_SKIP
+#define NVFP4_SEARCH_ALT_SKIP 1
+#endif
+constexpr int kTilesPerWarp = NVFP4_SEARCH_TILES;
+constexpr bool kAltSkip = NVFP4_SEARCH_ALT_SKIP;
+constexpr int kUnroll = NVFP4_SEARCH_UNROLL;
 constexpr int kRowsPerCta = kWarps * kTileRows * kTilesPerWarp;  // 256
 constexpr float kTieBand = 1.0f / 4096.0f;
 constexpr float kZeroFloor = 0x1p-40f;  // relative to ||p||^2
@@ -231,6 +242,50 @@ __device__ __forceinline__ void track3(float key, float &b1, float &b2, float &b
 __device__ __forceinline__ uint32_t pick4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
                                           int t) {
   return t == 0 ? w0 : (t == 1 ? w1 : (t == 2 ? w2 : w3));
+}
+
+// One candidate: codes (with or without the neighbouring-float correction),
+// the tensor-core product u, z = p - s u, and the row objective after a quad
+// reduce-scatter (lanes t < 2: row g, t >= 2: row g + 8).
+template <bool kLH, bool kAlt>
+__device__ __forceinline__ float candidate_objective(const float tq[8], const float ta[8],
+                                                     float f, float sm, uint32_t sgn,
+                                                     const uint32_t bh[2][2],
+                                                     const uint32_t bl[2][2],
+                                                     const float pz[2][4], bool upper) {
+  const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  uint32_t code;
+  const uint32_t ct = cvt4_e2m1x2(tq[1] * f, tq[0] * f, tq[3] * f, tq[2] * f, tq[5] * f,
+                                  tq[4] * f, tq[7] * f, tq[6] * f);
+  if (kAlt) {
+    const uint32_t ca = cvt4_e2m1x2(ta[1] * f, ta[0] * f, ta[3] * f, ta[2] * f, ta[5] * f,
+                                    ta[4] * f, ta[7] * f, ta[6] * f);
+    const uint32_t odd = (ct & 0x11111111u) * 15u;
+    code = ((ct & odd) | (ca & ~odd)) | sgn;
+  } else {
+    code = ct | sgn;
+  }
+  uint32_t A[4];
+  cvt4_f16x2(code, A);
+  float u0[4], u1[4];
+  mma_f16_16816(u0, A, bh[0][0], bh[0][1], zero4);
+  mma_f16_16816(u1, A, bh[1][0], bh[1][1], zero4);
+  if (kLH) {
+    mma_f16_16816(u0, A, bl[0][0], bl[0][1], u0);
+    mma_f16_16816(u1, A, bl[1][0], bl[1][1], u1);
+  }
+  const float z00 = fmaf(-sm, u0[0], pz[0][0]), z01 = fmaf(-sm, u0[1], pz[0][1]);
+  const float z02 = fmaf(-sm, u0[2], pz[0][2]), z03 = fmaf(-sm, u0[3], pz[0][3]);
+  const float z10 = fmaf(-sm, u1[0], pz[1][0]), z11 = fmaf(-sm, u1[1], pz[1][1]);
+  const float z12 = fmaf(-sm, u1[2], pz[1][2]), z13 = fmaf(-sm, u1[3], pz[1][3]);
+  const float e0 = fmaf(z00, z00, fmaf(z01, z01, fmaf(z10, z10, z11 * z11)));
+  const float e1 = fmaf(z02, z02, fmaf(z03, z03, fmaf(z12, z12, z13 * z13)));
+  // the same sums in the same order on both lanes of a pair
+  float mine = upper ? e1 : e0;
+  const float other = upper ? e0 : e1;
+  mine += __shfl_xor_sync(0xFFFFFFFFu, other, 2);
+  mine += __shfl_xor_sync(0xFFFFFFFFu, mine, 1);
+  return mine;
 }
 
 template <bool kLH>
@@ -437,6 +492,7 @@ __global__ void __launch_bounds__(kThreads)
       const ClassInfo ci = cls[k];
       // class quotient t and its neighbour across q, per element
       float tq[8], ta[8];
+      bool near = false;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float tt = fmaf(a[e], ci.r_hi, a[e] * ci.r_lo);
@@ -444,39 +500,26 @@ __global__ void __launch_bounds__(kThreads)
         const int step = (rho > 0.0f) - (rho < 0.0f);
         tq[e] = tt;
         ta[e] = __int_as_float(__float_as_int(tt) + step);
+        // t within two floats of a value whose low 21 mantissa bits are zero
+        // (every rounding midpoint times a power of two is one), and not exact
+        near = near || (step != 0 && ((__float_as_uint(tt) + 2u) & 0x1FFFFFu) <= 4u);
       }
-      for (; j < ci.end; ++j) {
-        const CandInfo cd = cand[j];
-        const float f = cd.f;
-        const uint32_t ct = cvt4_e2m1x2(tq[1] * f, tq[0] * f, tq[3] * f, tq[2] * f,
-                                        tq[5] * f, tq[4] * f, tq[7] * f, tq[6] * f);
-        const uint32_t ca = cvt4_e2m1x2(ta[1] * f, ta[0] * f, ta[3] * f, ta[2] * f,
-                                        ta[5] * f, ta[4] * f, ta[7] * f, ta[6] * f);
-        const uint32_t odd = (ct & 0x11111111u) * 15u;
-        const uint32_t code = ((ct & odd) | (ca & ~odd)) | sgn;
-        uint32_t A[4];
-        cvt4_f16x2(code, A);
-        float u0[4], u1[4];
-        mma_f16_16816(u0, A, bh[0][0], bh[0][1], zero4);
-        mma_f16_16816(u1, A, bh[1][0], bh[1][1], zero4);
-        if (kLH) {
-          mma_f16_16816(u0, A, bl[0][0], bl[0][1], u0);
-          mma_f16_16816(u1, A, bl[1][0], bl[1][1], u1);
+      if (!kAltSkip || __any_sync(0xFFFFFFFFu, near)) {
+#pragma unroll kUnroll
+        for (; j < ci.end; ++j) {
+          const CandInfo cd = cand[j];
+          const float e = candidate_objective<kLH, true>(tq, ta, cd.f, cd.s * umul, sgn, bh, bl,
+                                                         pz, upper);
+          track3(key_of(e, cd.c), b1, b2, b3);
         }
-        const float sm = cd.s * umul;
-        const float z00 = fmaf(-sm, u0[0], pz[0][0]), z01 = fmaf(-sm, u0[1], pz[0][1]);
-        const float z02 = fmaf(-sm, u0[2], pz[0][2]), z03 = fmaf(-sm, u0[3], pz[0][3]);
-        const float z10 = fmaf(-sm, u1[0], pz[1][0]), z11 = fmaf(-sm, u1[1], pz[1][1]);
-        const float z12 = fmaf(-sm, u1[2], pz[1][2]), z13 = fmaf(-sm, u1[3], pz[1][3]);
-        const float e0 = fmaf(z00, z00, fmaf(z01, z01, fmaf(z10, z10, z11 * z11)));
-        const float e1 = fmaf(z02, z02, fmaf(z03, z03, fmaf(z12, z12, z13 * z13)));
-        // reduce-scatter over the quad: lanes t < 2 end with row g, t >= 2 with
-        // row g + 8 (sums in the same order on every lane of a pair)
-        float mine = upper ? e1 : e0;
-        const float other = upper ? e0 : e1;
-        mine += __shfl_xor_sync(0xFFFFFFFFu, other, 2);
-        mine += __shfl_xor_sync(0xFFFFFFFFu, mine, 1);
-        track3(key_of(mine, cd.c), b1, b2, b3);
+      } else {  // no quotient near a midpoint: t alone rounds exactly
+#pragma unroll kUnroll
+        for (; j < ci.end; ++j) {
+          const CandInfo cd = cand[j];
+          const float e = candidate_objective<kLH, false>(tq, ta, cd.f, cd.s * umul, sgn, bh,
+                                                          bl, pz, upper);
+          track3(key_of(e, cd.c), b1, b2, b3);
+        }
       }
     }
 

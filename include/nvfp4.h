@@ -104,6 +104,24 @@ nvfp4_status nvfp4_hessian_accumulate(const uint16_t *x, int64_t n_tok, int64_t 
                                       void *stream);
 
 /*
+ * The same accumulation as nvfp4_hessian_accumulate, for callers that may not
+ * allocate device memory: applications that give all of HBM to their own
+ * allocator or work under a fixed memory budget, and loops that cannot take an
+ * allocation's latency or implicit synchronisation.  The pages have no
+ * counterpart to this call; it is a property of this library only.
+ * Partial sums go to one 16 MiB device array inside the library (held by each
+ * device that loads it until exit) instead of the memory pool, so nothing is
+ * allocated.  C must not exceed 262,144 (else NVFP4_ERR_TOO_LARGE, nothing
+ * launched).  All calls on a device share that array: calls that overlap on
+ * the GPU race and must be serialised by the caller.  The first call on a
+ * device looks up the array's address with that device current; make it
+ * before any stream capture.  Results agree with nvfp4_hessian_accumulate up
+ * to fp32 summation order.
+ */
+nvfp4_status nvfp4_hessian_accumulate_noalloc(const uint16_t *x, int64_t n_tok, int64_t C,
+                                              float *H, void *stream);
+
+/*
  * Grouped form for experts: tokens are sorted by group; group g owns rows
  * offsets[g] .. offsets[g+1]-1 of x and accumulates into H[g].
  *   x         [n_tok_total, C] bf16

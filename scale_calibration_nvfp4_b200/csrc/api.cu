@@ -134,6 +134,15 @@ nvfp4_status nvfp4_hessian_accumulate(const uint16_t *x, int64_t n_tok, int64_t 
   return map_cuda(nvfp4::launch_gram(x, nullptr, 1, n_tok, C, H, as_stream(stream)));
 }
 
+nvfp4_status nvfp4_hessian_accumulate_noalloc(const uint16_t *x, int64_t n_tok, int64_t C,
+                                              float *H, void *stream) {
+  if (n_tok < 0 || C < 0 || !H || (n_tok > 0 && !x)) return NVFP4_ERR_INVALID_ARG;
+  if (C % 16 || !fits(n_tok, C)) return NVFP4_ERR_SHAPE;
+  if (C > nvfp4::gram_noalloc_max_channels()) return NVFP4_ERR_TOO_LARGE;
+  if ((x && !aligned(x, 16)) || !aligned(H, 4)) return NVFP4_ERR_MISALIGNED;
+  return map_cuda(nvfp4::launch_gram_noalloc(x, n_tok, C, H, as_stream(stream)));
+}
+
 nvfp4_status nvfp4_hessian_accumulate_grouped(const uint16_t *x, const int64_t *offsets,
                                               int64_t G, int64_t n_tok_total, int64_t C,
                                               float *H, void *stream) {

@@ -14,6 +14,8 @@
 // exact in fp32, sums are fp32).  Each CTA writes its fp32 partial block to a
 // stream-ordered scratch buffer; a second kernel adds the partials of a group
 // to H in a fixed order, so the result does not depend on scheduling.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -234,35 +236,53 @@ __global__ void build_items_kernel(const int64_t *__restrict__ offsets, int64_t 
   }
 }
 
-bool g_smem_attr_set = false;
+constexpr int kMaxDevices = 64;
+bool g_smem_attr_set[kMaxDevices] = {};
+
+cudaError_t ensure_smem_attr() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!g_smem_attr_set[dev]) {
+    e = cudaFuncSetAttribute(gram_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kGramSmem);
+    if (e != cudaSuccess) return e;
+    g_smem_attr_set[dev] = true;
+  }
+  return cudaSuccess;
+}
+
+// Token items of the uniform split: enough CTAs for a few waves of 3 resident
+// CTAs per SM, at least 4 tiles per item, at most `cap` items.
+void uniform_items(int64_t n_tok, int64_t ngroups, int64_t cap, int64_t *items_out,
+                   int64_t *per_item_out) {
+  const int64_t target = (int64_t)sm_count() * 3 * 2;
+  int64_t items = (target + ngroups - 1) / ngroups;
+  const int64_t max_items = (n_tok + 4 * kTileTok - 1) / (4 * kTileTok);
+  if (items > max_items) items = max_items;
+  if (items > cap) items = cap;
+  if (items < 1) items = 1;
+  int64_t per_item = (n_tok + items - 1) / items;
+  per_item = (per_item + kTileTok - 1) / kTileTok * kTileTok;
+  *items_out = (n_tok + per_item - 1) / per_item;
+  *per_item_out = per_item;
+}
 
 }  // namespace
 
 cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, int64_t n_tok,
                         int64_t C, float *H, cudaStream_t st) {
   if (n_tok == 0 || C == 0 || G == 0) return cudaSuccess;
-  cudaError_t e;
-  if (!g_smem_attr_set) {
-    e = cudaFuncSetAttribute(gram_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kGramSmem);
-    if (e != cudaSuccess) return e;
-    g_smem_attr_set = true;
-  }
+  cudaError_t e = ensure_smem_attr();
+  if (e != cudaSuccess) return e;
   const int64_t nb = C / kBlock;
   const int64_t ngroups = (nb + kGroupBlocks - 1) / kGroupBlocks;
   const int64_t per_group = nb * 256;
 
   if (!offsets) {
-    // uniform split of the tokens into items, enough CTAs for ~3 waves of
-    // 3 resident CTAs per SM, at least 4 tiles per item
-    const int64_t target = (int64_t)sm_count() * 3 * 2;
-    int64_t items = (target + ngroups - 1) / ngroups;
-    const int64_t max_items = (n_tok + 4 * kTileTok - 1) / (4 * kTileTok);
-    if (items > max_items) items = max_items;
-    if (items < 1) items = 1;
-    int64_t per_item = (n_tok + items - 1) / items;
-    per_item = (per_item + kTileTok - 1) / kTileTok * kTileTok;
-    items = (n_tok + per_item - 1) / per_item;
+    int64_t items, per_item;
+    uniform_items(n_tok, ngroups, INT64_MAX, &items, &per_item);
     float *partial = nullptr;
     e = scratch_alloc((void **)&partial, sizeof(float) * items * per_group, st);
     if (e != cudaSuccess) return e;
@@ -308,6 +328,79 @@ cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, in
   }
   cudaError_t e2 = scratch_free(ws, st);
   return e != cudaSuccess ? e : e2;
+}
+
+// ---------------------------------------------------------------------------
+// Gram accumulation without any allocation.
+//
+// The per-item partial sums of this entry point live in one fixed array of
+// this file, so the call never allocates.  It exists for callers that may not
+// allocate device memory themselves: code that hands all of HBM to its own
+// allocator or runs under a fixed memory budget (a library-side allocation
+// could fail there or take memory the caller has planned for something else),
+// and code that cannot afford an allocation's latency or implicit device
+// synchronisation in the middle of a calibration loop.
+//
+// The array is 16 MiB (kNoAllocPartialFloats floats) and is held by every
+// device that loads the library until the process exits.  A call needs
+// C/16 * 1 KiB per token range, so C is limited to 262,144 channels; fewer
+// token ranges are used when C is large.  All calls on a device share the
+// array: calls that overlap on the GPU (different streams, or graphs replayed
+// concurrently) race on it and must be serialised by the caller.  Every
+// partial is written before it is read, so nothing needs clearing between
+// calls.  The first call on each device looks up the array's device address
+// (cudaGetSymbolAddress, with that device current) and caches it; make that
+// first call before any stream capture.
+constexpr size_t kNoAllocPartialFloats = (size_t)4 << 20;  // 16 MiB
+static __device__ __align__(256) float g_noalloc_partials[kNoAllocPartialFloats];
+
+namespace {
+std::mutex g_noalloc_mu;
+float *g_noalloc_ptr[kMaxDevices] = {};
+
+cudaError_t noalloc_partials(float **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = static_cast<float *>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+int64_t gram_noalloc_max_channels() {
+  return (int64_t)(kNoAllocPartialFloats / 256) * kBlock;
+}
+
+cudaError_t launch_gram_noalloc(const uint16_t *x, int64_t n_tok, int64_t C, float *H,
+                                cudaStream_t st) {
+  if (n_tok == 0 || C == 0) return cudaSuccess;
+  const int64_t nb = C / kBlock;
+  const int64_t per_group = nb * 256;
+  const int64_t cap = (int64_t)(kNoAllocPartialFloats / (size_t)per_group);
+  if (cap < 1) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_attr();
+  if (e != cudaSuccess) return e;
+  float *partial = nullptr;
+  e = noalloc_partials(&partial);
+  if (e != cudaSuccess) return e;
+  const int64_t ngroups = (nb + kGroupBlocks - 1) / kGroupBlocks;
+  int64_t items, per_item;
+  uniform_items(n_tok, ngroups, cap, &items, &per_item);
+  gram_partial_kernel<<<dim3((unsigned)items, (unsigned)ngroups), kGramThreads, kGramSmem, st>>>(
+      x, C, nullptr, nullptr, n_tok, per_item, partial);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  gram_reduce_kernel<<<(unsigned)((per_group + 255) / 256), 256, 0, st>>>(partial, nb, 1, nullptr,
+                                                                          items, H);
+  return cudaGetLastError();
 }
 
 }  // namespace nvfp4

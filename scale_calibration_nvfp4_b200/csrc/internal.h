@@ -28,6 +28,12 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
 cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, int64_t n_tok,
                         int64_t C, float *H, cudaStream_t st);
 
+// Gram accumulation with its partial sums in a fixed device array (no
+// allocation); C up to gram_noalloc_max_channels().
+cudaError_t launch_gram_noalloc(const uint16_t *x, int64_t n_tok, int64_t C, float *H,
+                                cudaStream_t st);
+int64_t gram_noalloc_max_channels();
+
 // Stream-ordered scratch from the library's pool on the current device.
 cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t st);
 cudaError_t scratch_free(void *p, cudaStream_t st);

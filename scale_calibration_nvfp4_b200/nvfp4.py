@@ -26,6 +26,7 @@ _vp, _i64 = ctypes.c_void_p, ctypes.c_int64
 SIGNATURES = {
     "nvfp4_global_scale": [_vp, _i64, _i64, _vp, _vp],
     "nvfp4_hessian_accumulate": [_vp, _i64, _i64, _vp, _vp],
+    "nvfp4_hessian_accumulate_noalloc": [_vp, _i64, _i64, _vp, _vp],
     "nvfp4_hessian_accumulate_grouped": [_vp, _vp, _i64, _i64, _i64, _vp, _vp],
     "nvfp4_scale_search_max": [_vp, _i64, _i64, _i64, _vp, _vp, _vp],
     "nvfp4_scale_search_mse": [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp],
@@ -123,6 +124,20 @@ def hessian_accumulate(x, H, stream=None):
     if H.numel() != (C // 16) * 256:
         raise ValueError("H must hold C/16 x 16 x 16 floats")
     _call("nvfp4_hessian_accumulate", _p(x), N, C, _p(H), _stream(stream))
+    return H
+
+
+def hessian_accumulate_noalloc(x, H, stream=None):
+    """As hessian_accumulate, for callers that may not allocate device memory:
+    the library keeps the partial sums in its own fixed 16 MiB device array
+    (C <= 262,144).  Calls that overlap on the GPU share that array and race;
+    make the first call on a device outside stream capture."""
+    _need(x, torch.bfloat16, "x")
+    _need(H, torch.float32, "H")
+    N, C = x.shape
+    if H.numel() != (C // 16) * 256:
+        raise ValueError("H must hold C/16 x 16 x 16 floats")
+    _call("nvfp4_hessian_accumulate_noalloc", _p(x), N, C, _p(H), _stream(stream))
     return H
 
 

@@ -1,24 +1,32 @@
 """Benchmark of the NVFP4 calibration path on B200.
 
-One step = one pass of the whole path over one layer of the chosen workload
-(default: dense projection, W 4096x4096, X 2048x4096):
+One step = one pass of the whole path over one workload's inputs, which are
+resident in HBM when the timed region starts.  Default workload: the dense
+projection (W 4096x4096, X 2048x4096), whose step is
 
     global scale(W) -> Gram(X) -> max rule -> MSE search -> Local-Hessian
     search -> quantise+pack (Local-Hessian codes) -> dequantise ->
     W4A4 fake-quant(X)
 
-Metric: NVFP4 weight blocks per second through the whole path (the
-Local-Hessian search dominates).  Inputs are resident in HBM; the L2 cache is
-flushed (a 256 MiB write) before every timed step, outside the step's CUDA
-events.  Per-row kernel times are CUDA events on the launching stream.
+Other workloads (--workload): tiny, moe (128 experts, grouped Gram over 262,144
+routed tokens, per-expert scales, Local-Hessian search, pack, dequantise),
+mlp_pair (up and down projections with the 16 calibration chunks of 65,536
+tokens each kept resident), w4a4 (activation fake-quant of 32768x8192 with
+packed outputs).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dense|tiny|moe|mlp_pair]
+Metric: NVFP4 blocks per second through the step (weight blocks; activation
+blocks for w4a4).  The L2 cache is flushed (a 256 MiB write) before every
+timed step, outside the step's CUDA events.  Per-row times are CUDA events on
+the launching stream.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle on a bounded sample
 
 Multi-GPU (torchrun): every rank runs its own replica of the workload (the
 path has no cross-GPU exchange); timing is the max over ranks.
 """
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -41,42 +49,31 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
+WORKLOAD_NAMES = ["dense", "tiny", "moe", "mlp_pair", "w4a4"]
 
-ROWS = ["global_scale", "gram", "search_max", "search_mse", "search_lh", "quantize_pack",
-        "dequantize", "fake_quant"]
-# kernels of this library launched by each row (memsets are not kernels)
-LAUNCHES = {"global_scale": 2, "gram": 2, "search_max": 1, "search_mse": 1, "search_lh": 1,
-            "quantize_pack": 1, "dequantize": 1, "fake_quant": 3}
+# Local-Hessian search work per block, counted on the definition E = delta
+# H_b delta^T: per candidate 256 FMA for H_b delta and 16 FMA for the dot
+# product, 2 flop each (the E2M1 encodes are not counted as flops).
+LH_FLOP_PER_BLOCK = 126 * 2 * (256 + 16)
+# bytes per activation element of the fused fake-quant with packed outputs:
+# amax pass 2, fused pass 2 read + 2 write + 0.5 packed + 1/16 block codes
+FAKE_QUANT_BYTES_PER_ELEM = 2 + 2 + 2 + 0.5 + 1 / 16
 
 
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
-# ------------------------------------------------------------------ inputs
-def make_inputs(workload, device):
-    from scale_calibration_nvfp4_b200 import workloads
-    if workload in ("tiny", "dense"):
-        W, X = workloads.layer_inputs(workload, device)
-        return dict(W=W.unsqueeze(0), X=X, offsets=None, desc=workloads.BY_NAME[workload].description)
-    if workload == "moe":
-        W, X, offsets = workloads.moe_inputs(device)
-        return dict(W=W, X=X, offsets=offsets.to(device), desc=workloads.BY_NAME["moe"].description)
-    if workload == "mlp_pair":
-        up, _ = workloads.mlp_weights(device)
-        X = workloads.mlp_chunk("up", 0, device)
-        return dict(W=up.unsqueeze(0), X=X, offsets=None,
-                    desc="up projection 12288x4096 with one 65,536-token Student-t chunk")
-    raise ValueError(workload)
+# ------------------------------------------------------------------ workloads
+class Layer:
+    """One weight tensor (optionally batched) with its calibration input."""
 
-
-class Path:
-    """Preallocated outputs and the per-row calls of one step."""
-
-    def __init__(self, inp):
-        from scale_calibration_nvfp4_b200 import nvfp4
-        self.nv = nvfp4
-        self.W, self.X, self.offsets = inp["W"], inp["X"], inp["offsets"]
+    def __init__(self, name, W, X=None, offsets=None, chunks=None):
+        self.name = name
+        self.W = W if W.dim() == 3 else W.unsqueeze(0)
+        self.X = X
+        self.offsets = offsets
+        self.chunks = chunks  # list of resident calibration chunks
         B, R, C = self.W.shape
         dev = self.W.device
         self.B, self.R, self.C = B, R, C
@@ -87,55 +84,146 @@ class Path:
         self.c_lh = torch.empty_like(self.c_max)
         self.packed = torch.empty(B, R, C // 2, dtype=torch.uint8, device=dev)
         self.deq = torch.empty(B, R, C, dtype=torch.bfloat16, device=dev)
-        self.fq = torch.empty_like(self.X)
-
-    def row(self, name):
-        nv = self.nv
-        if name == "global_scale":
-            nv.global_scale(self.W, batch=self.B, out=self.s_g)
-        elif name == "gram":
-            if self.offsets is None:
-                nv.hessian_accumulate(self.X, self.H[0])
-            else:
-                nv.hessian_accumulate_grouped(self.X, self.offsets, self.H)
-        elif name == "search_max":
-            nv.scale_search_max(self.W, self.s_g, out=self.c_max)
-        elif name == "search_mse":
-            nv.scale_search_mse(self.W, self.s_g, out=self.c_mse)
-        elif name == "search_lh":
-            nv.scale_search_local_hessian(self.W, self.s_g, self.H, out=self.c_lh)
-        elif name == "quantize_pack":
-            nv.quantize_pack(self.W, self.s_g, self.c_lh, out=self.packed)
-        elif name == "dequantize":
-            nv.dequantize(self.packed, self.c_lh, self.s_g, out=self.deq)
-        elif name == "fake_quant":
-            nv.fake_quant(self.X, want_packed=False, out=self.fq)
 
     def blocks(self):
         return self.B * self.R * self.C // 16
 
-    def algorithmic_bytes(self):
-        """Bytes each row must move at least (read + write), per step."""
-        n_w = self.B * self.R * self.C
-        n_x = self.X.numel()
-        nb = n_w // 16
-        h = self.H.numel() * 4
-        return {
-            "global_scale": 2 * n_w,
-            "gram": 2 * n_x + 2 * h,
-            "search_max": 2 * n_w + nb,
-            "search_mse": 2 * n_w + nb,
-            "search_lh": 2 * n_w + nb + h,
-            "quantize_pack": 2 * n_w + nb + n_w // 2,
-            "dequantize": n_w // 2 + nb + 2 * n_w,
-            "fake_quant": 6 * n_x,
-        }
+    def tokens(self):
+        if self.chunks is not None:
+            return sum(c.shape[0] for c in self.chunks)
+        return 0 if self.X is None else self.X.shape[0]
 
 
-# Local-Hessian search work per block, counted on the definition E = delta
-# H_b delta^T: per candidate 256 FMA for H_b delta and 16 FMA for the dot
-# product, 2 flop each (the E2M1 encodes are not counted as flops).
-LH_FLOP_PER_BLOCK = 126 * 2 * (256 + 16)
+class Runner:
+    """Rows of one workload: (name, callable, algorithmic bytes, launches)."""
+
+    def __init__(self, workload, device):
+        from scale_calibration_nvfp4_b200 import nvfp4, workloads
+        self.nv = nvfp4
+        self.workload = workload
+        wl = workloads
+        if workload in ("tiny", "dense"):
+            W, X = wl.layer_inputs(workload, device)
+            self.layers = [Layer(workload, W, X)]
+            self.desc = wl.BY_NAME[workload].description
+            self.rules = ["max", "mse", "lh"]
+            self.fq_input = X
+        elif workload == "moe":
+            W, X, offsets = wl.moe_inputs(device)
+            self.layers = [Layer("experts", W, X, offsets=offsets.to(device))]
+            self.desc = wl.BY_NAME["moe"].description
+            self.rules = ["lh"]
+            self.fq_input = None
+        elif workload == "mlp_pair":
+            up, down = wl.mlp_weights(device)
+            p = wl.BY_NAME["mlp_pair"].params
+            ch_up = [wl.mlp_chunk("up", k, device) for k in range(p["chunks"])]
+            ch_dn = [wl.mlp_chunk("down", k, device) for k in range(p["chunks"])]
+            self.layers = [Layer("up", up, chunks=ch_up), Layer("down", down, chunks=ch_dn)]
+            self.desc = wl.BY_NAME["mlp_pair"].description
+            self.rules = ["lh"]
+            self.fq_input = None
+        elif workload == "w4a4":
+            X = wl.w4a4_inputs(device)
+            self.layers = []
+            self.desc = wl.BY_NAME["w4a4"].description
+            self.rules = []
+            self.fq_input = X
+        else:
+            raise ValueError(workload)
+        if self.fq_input is not None:
+            X = self.fq_input
+            self.fq_out = torch.empty_like(X)
+            self.fq_packed = torch.empty(X.shape[0], X.shape[1] // 2, dtype=torch.uint8,
+                                         device=X.device)
+            self.fq_codes = torch.empty(X.shape[0], X.shape[1] // 16, dtype=torch.uint8,
+                                        device=X.device)
+            self.fq_sg = torch.empty(1, dtype=torch.float32, device=X.device)
+        self.rows = self._rows()
+
+    def _rows(self):
+        nv = self.nv
+        rows = []
+        for L in self.layers:
+            n_w = L.B * L.R * L.C
+            nb = n_w // 16
+            h = L.H.numel() * 4
+            pre = L.name + "." if len(self.layers) > 1 else ""
+            rows.append((pre + "global_scale",
+                         lambda L=L: nv.global_scale(L.W, batch=L.B, out=L.s_g), 2 * n_w, 2))
+            if L.chunks is not None:
+                def gram(L=L):
+                    for ch in L.chunks:
+                        nv.hessian_accumulate(ch, L.H[0])
+                rows.append((pre + "gram", gram,
+                             2 * L.tokens() * L.C + 2 * h * len(L.chunks), 2 * len(L.chunks)))
+            elif L.offsets is not None:
+                rows.append((pre + "gram",
+                             lambda L=L: nv.hessian_accumulate_grouped(L.X, L.offsets, L.H),
+                             2 * L.X.numel() + 2 * h, 3))
+            else:
+                rows.append((pre + "gram", lambda L=L: nv.hessian_accumulate(L.X, L.H[0]),
+                             2 * L.X.numel() + 2 * h, 2))
+            if "max" in self.rules:
+                rows.append((pre + "search_max",
+                             lambda L=L: nv.scale_search_max(L.W, L.s_g, out=L.c_max),
+                             2 * n_w + nb, 1))
+            if "mse" in self.rules:
+                rows.append((pre + "search_mse",
+                             lambda L=L: nv.scale_search_mse(L.W, L.s_g, out=L.c_mse),
+                             2 * n_w + nb, 1))
+            rows.append((pre + "search_lh",
+                         lambda L=L: nv.scale_search_local_hessian(L.W, L.s_g, L.H, out=L.c_lh),
+                         2 * n_w + nb + h, 1))
+            rows.append((pre + "quantize_pack",
+                         lambda L=L: nv.quantize_pack(L.W, L.s_g, L.c_lh, out=L.packed),
+                         2 * n_w + nb + n_w // 2, 1))
+            rows.append((pre + "dequantize",
+                         lambda L=L: nv.dequantize(L.packed, L.c_lh, L.s_g, out=L.deq),
+                         n_w // 2 + nb + 2 * n_w, 1))
+        if self.fq_input is not None:
+            n_x = self.fq_input.numel()
+            if self.workload == "w4a4":
+                rows.append(("fake_quant", lambda: self._fq(True),
+                             FAKE_QUANT_BYTES_PER_ELEM * n_x, 3))
+            else:
+                rows.append(("fake_quant", lambda: self._fq(False), 6 * n_x, 3))
+        return rows
+
+    def _fq(self, packed):
+        nv = self.nv
+        X = self.fq_input
+        nv._call("nvfp4_fake_quant", nv._p(X), X.shape[0], X.shape[1], nv._p(self.fq_out),
+                 nv._p(self.fq_packed) if packed else None,
+                 nv._p(self.fq_codes) if packed else None, nv._p(self.fq_sg), nv._stream())
+
+    def blocks(self):
+        if self.layers:
+            return sum(L.blocks() for L in self.layers)
+        return self.fq_input.numel() // 16
+
+    def launches(self):
+        return sum(r[3] for r in self.rows)
+
+    def inputs(self):
+        t = []
+        for L in self.layers:
+            t.append(L.W)
+            if L.X is not None:
+                t.append(L.X)
+            if L.chunks is not None:
+                t.extend(L.chunks)
+        if self.fq_input is not None and not any(x is self.fq_input for x in t):
+            t.append(self.fq_input)
+        return t
+
+    def results(self):
+        out = []
+        for L in self.layers:
+            out += [L.c_lh, L.packed]
+        if self.workload == "w4a4":
+            out += [self.fq_packed, self.fq_codes]
+        return out
 
 
 # ------------------------------------------------------------------ clocks
@@ -233,13 +321,20 @@ def dist_env():
     return 0, 1, 0
 
 
+def max_over_ranks(pg, value):
+    if pg is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return t.item()
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_gpu(args):
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     pg = None
     if world > 1:
-        import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
         pg = dist
@@ -250,16 +345,16 @@ def run_gpu(args):
         pg.barrier()
     nvfp4.lib()
 
-    inp = make_inputs(args.workload, "cuda")
-    path = Path(inp)
+    run = Runner(args.workload, "cuda")
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    rows = run.rows
 
     def step(events=None):
-        for i, name in enumerate(ROWS):
+        for i, r in enumerate(rows):
             if events is not None:
                 events[i].record(stream)
-            path.row(name)
+            r[1]()
         if events is not None:
             events[-1].record(stream)
 
@@ -268,7 +363,7 @@ def run_gpu(args):
         step()
     torch.cuda.synchronize()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ROWS) + 1)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(rows) + 1)]
           for _ in range(args.steps)]
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
@@ -285,92 +380,94 @@ def run_gpu(args):
         pg.barrier()
     clk = clocks.stop() if clocks else None
 
-    per_row = {n: [] for n in ROWS}
+    per_row = {r[0]: [] for r in rows}
     step_ms = []
     for k in range(args.steps):
-        for i, n in enumerate(ROWS):
-            per_row[n].append(ev[k][i].elapsed_time(ev[k][i + 1]))
+        for i, r in enumerate(rows):
+            per_row[r[0]].append(ev[k][i].elapsed_time(ev[k][i + 1]))
         step_ms.append(ev[k][0].elapsed_time(ev[k][-1]))
-    ms_total = sum(step_ms)
-    if pg:
-        t = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_total = t.item()
-    ms_per_step = ms_total / args.steps
-    blocks = path.blocks()
+    ms_per_step = max_over_ranks(pg, sum(step_ms)) / args.steps
+    blocks = run.blocks()
     value = world * blocks / (ms_per_step / 1e3)
 
-    # end to end through the C ABI with host buffers
-    e2e = run_e2e(path, inp, args, pg, world) if not args.no_e2e else None
+    e2e = None if args.no_e2e else run_e2e(run, args, pg, world)
 
     if rank == 0:
         pk, pk_kind = peaks()
-        rows_ms = {n: statistics.mean(v) for n, v in per_row.items()}
-        alg = path.algorithmic_bytes()
-        kernels = {}
-        for n in ROWS:
-            kernels[n] = {"ms": round(rows_ms[n], 5),
-                          "GB/s": round(alg[n] / (rows_ms[n] / 1e3) / 1e9, 1)}
-        lh_ms = rows_ms["search_lh"]
-        sm_mhz_peak = float(pk.get("sm_max_mhz", 1965.0))
-        fp32_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * sm_mhz_peak * 1e6 / 1e12
-        achieved = LH_FLOP_PER_BLOCK * blocks / (lh_ms / 1e3) / 1e12
-        roofline = {
-            "kernel": "search_kernel<Local-Hessian>",
-            "bound": "alu", "achieved": round(achieved, 2), "peak": round(fp32_peak, 2),
-            "unit": "TFLOP/s", "frac": round(achieved / fp32_peak, 4),
-            "traffic": recorded_traffic("search_lh", args.workload),
-            "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 flop x %.0f MHz (%s clocks)"
-                         % (sm_mhz_peak, pk_kind),
-            "flop_per_block": LH_FLOP_PER_BLOCK,
-            "flop_basis": "definition delta H delta^T: 126 x (256 + 16) FMA per block",
-        }
         hbm = float(pk.get("hbm_gbs", FALLBACK_HBM_GBS))
-        streaming = {n: {"GB/s": kernels[n]["GB/s"], "frac_of_%s_hbm" % pk_kind:
-                         round(kernels[n]["GB/s"] / hbm, 3)}
-                     for n in ("gram", "quantize_pack", "dequantize", "fake_quant",
-                               "global_scale", "search_max")}
+        kernels = {}
+        for r in rows:
+            ms = statistics.mean(per_row[r[0]])
+            gbs = r[2] / (ms / 1e3) / 1e9
+            kernels[r[0]] = {"ms": round(ms, 5), "GB/s": round(gbs, 1),
+                             "frac_of_%s_hbm" % pk_kind: round(gbs / hbm, 3)}
         out = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; no dataset or trained weights)",
-            "config": {"workload": args.workload, "desc": inp["desc"],
-                       "blocks_per_step": blocks, "rows": ROWS,
-                       "parallelism": "replicas" if world > 1 else "single GPU",
+            "config": {"workload": args.workload, "desc": run.desc, "blocks_per_step": blocks,
+                       "rows": [r[0] for r in rows],
+                       "parallelism": "replicas (one per GPU)" if world > 1 else "single GPU",
                        "cache": "L2 flushed (256 MiB write) before every timed step"},
-            "roofline": roofline,
-            "hbm_kernels": streaming,
+            "roofline": make_roofline(run, kernels, pk, pk_kind, args.workload),
             "kernels": kernels,
-            "gpu_launches": args.steps * sum(LAUNCHES.values()),
+            "gpu_launches": args.steps * run.launches(),
             "clocks": clk,
             "e2e": e2e,
         }
         if not args.no_cpu_baseline and world == 1:
-            out["cpu_baseline"] = cpu_baseline(args.workload, inp, budget_s=args.cpu_seconds)
+            out["cpu_baseline"] = cpu_baseline(run, budget_s=args.cpu_seconds)
         print(json.dumps(out), flush=True)
     if pg:
         pg.barrier()
         pg.destroy_process_group()
 
 
-def run_e2e(path, inp, args, pg, world):
+def make_roofline(run, kernels, pk, pk_kind, workload):
+    lh_rows = [k for k in kernels if k.endswith("search_lh")]
+    if lh_rows:
+        lh_ms = sum(kernels[k]["ms"] for k in lh_rows)
+        sm_mhz = float(pk.get("sm_max_mhz", 1965.0))
+        fp32_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+        achieved = LH_FLOP_PER_BLOCK * run.blocks() / (lh_ms / 1e3) / 1e12
+        return {
+            "kernel": "search_kernel<Local-Hessian>",
+            "bound": "alu", "achieved": round(achieved, 2), "peak": round(fp32_peak, 2),
+            "unit": "TFLOP/s", "frac": round(achieved / fp32_peak, 4),
+            "traffic": recorded_traffic("search_lh", workload),
+            "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 flop x %.0f MHz (%s clocks)"
+                         % (sm_mhz, pk_kind),
+            "flop_basis": "definition delta H_b delta^T: 126 x (256 + 16) FMA per block",
+            "flop_per_block": LH_FLOP_PER_BLOCK,
+        }
+    ms = kernels["fake_quant"]["ms"]
+    n = run.fq_input.numel()
+    achieved = FAKE_QUANT_BYTES_PER_ELEM * n / (ms / 1e3) / 1e9
+    hbm = float(pk.get("hbm_gbs", FALLBACK_HBM_GBS))
+    return {"kernel": "fake_quant (amax pass + fused pass)", "bound": "hbm",
+            "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4),
+            "traffic": recorded_traffic("fake_quant", workload),
+            "peak_kind": "%s HBM copy bandwidth" % pk_kind,
+            "bytes_per_element": FAKE_QUANT_BYTES_PER_ELEM}
+
+
+def run_e2e(run, args, pg, world):
     """Same metric through the public API with host buffers: every step copies
-    W and X from pinned host memory to the device, runs the path and reads
-    the Local-Hessian codes and packed weights back."""
-    W_h = path.W.cpu().pin_memory()
-    X_h = path.X.cpu().pin_memory()
-    codes_h = torch.empty(path.c_lh.shape, dtype=torch.uint8).pin_memory()
-    packed_h = torch.empty(path.packed.shape, dtype=torch.uint8).pin_memory()
+    the inputs from pinned host memory to the device, runs the path and reads
+    the results (codes and packed weights, or packed activations) back."""
+    ins = [(t, t.cpu().pin_memory()) for t in run.inputs()]
+    outs = [(t, torch.empty(t.shape, dtype=t.dtype).pin_memory()) for t in run.results()]
     stream = torch.cuda.current_stream()
 
     def step():
-        path.W.copy_(W_h, non_blocking=True)
-        path.X.copy_(X_h, non_blocking=True)
-        for name in ROWS:
-            path.row(name)
-        codes_h.copy_(path.c_lh, non_blocking=True)
-        packed_h.copy_(path.packed, non_blocking=True)
+        for d, h in ins:
+            d.copy_(h, non_blocking=True)
+        for r in run.rows:
+            r[1]()
+        for d, h in outs:
+            h.copy_(d, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
         step()
@@ -383,83 +480,107 @@ def run_e2e(path, inp, args, pg, world):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if pg:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = t.item()
-    ms_step = ms / args.steps
-    h2d = W_h.numel() * 2 + X_h.numel() * 2
-    d2h = codes_h.numel() + packed_h.numel()
-    return {"value": round(world * path.blocks() / (ms_step / 1e3), 1), "unit": UNIT,
+    ms_step = max_over_ranks(pg, e0.elapsed_time(e1)) / args.steps
+    h2d = sum(h.numel() * h.element_size() for _, h in ins)
+    d2h = sum(h.numel() * h.element_size() for _, h in outs)
+    return {"value": round(world * run.blocks() / (ms_step / 1e3), 1), "unit": UNIT,
             "ms_per_step": round(ms_step, 5), "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h}
 
 
 # ------------------------------------------------------------------ CPU arm
-def cpu_baseline(workload, inp, budget_s=15.0):
+def _bits(t):
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def cpu_baseline(run, budget_s=15.0):
     """The oracle, as it stands, on a bounded sample of the same workload: the
-    whole path on the first rows of the (first) weight, the Gram on a
-    proportional share of the tokens; blocks/s extrapolated from the sample."""
+    step's rows on the first weight rows, the Gram on the same fraction of the
+    calibration tokens (fake-quant on the same fraction of activation rows);
+    blocks/s over the sample."""
     import oracle
     oracle.lib()
-
-    def bits(t):
-        return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
-
-    W = inp["W"][0]
-    X = inp["X"]
+    if not run.layers:  # activation-only workload: fake-quant on leading rows
+        X = run.fq_input
+        t0 = time.perf_counter()
+        oracle.fake_quant(_bits(X[:64]))
+        per_row = (time.perf_counter() - t0) / 64
+        n = int(max(1, min(X.shape[0], budget_s / max(per_row, 1e-6))))
+        xu = _bits(X[:n])
+        t0 = time.perf_counter()
+        oracle.fake_quant(xu)
+        t = time.perf_counter() - t0
+        blocks = n * X.shape[1] // 16
+        return {"value": round(blocks / t, 2), "unit": UNIT, "cores": oracle.max_threads(),
+                "kind": "oracle", "seconds": round(t, 3),
+                "sample": "fake-quant of %d of %d token rows (%d blocks)"
+                          % (n, X.shape[0], blocks)}
+    L = run.layers[0]
+    W = L.W[0]
     R, C = W.shape
-    wu_all = bits(W)
-    # calibrate the sample size with a short probe, then run ~budget_s
-    probe_rows = max(1, min(R, 8))
-    t_probe = _oracle_path(wu_all, bits(X[: max(16, X.shape[0] * probe_rows // R)]), probe_rows)
-    rows = int(max(1, min(R, probe_rows * budget_s / max(t_probe, 1e-3))))
-    x_rows = max(16, X.shape[0] * rows // R)
-    t = _oracle_path(wu_all, bits(X[:x_rows]), rows)
+    wu_all = _bits(W)
+    if L.chunks is not None:
+        X = L.chunks[0]
+    elif L.offsets is not None:
+        X = L.X[int(L.offsets[0]):int(L.offsets[1])]
+    else:
+        X = L.X
+    n_tok_total = L.tokens() if L.offsets is None else X.shape[0]
+
+    def path(rows):
+        frac = rows / R
+        x_rows = min(X.shape[0], max(16, int(n_tok_total * frac)))
+        xu = _bits(X[:x_rows])
+        fq = None
+        if run.fq_input is not None:
+            fq = _bits(run.fq_input[:max(1, int(run.fq_input.shape[0] * frac))])
+        t0 = time.perf_counter()
+        sg = oracle.global_scale(wu_all)
+        H = oracle.gram(xu)
+        wu = np.ascontiguousarray(wu_all[:rows])
+        if "max" in run.rules:
+            oracle.scale_search_max(wu, sg)
+        if "mse" in run.rules:
+            oracle.scale_search_mse(wu, sg)
+        codes, _ = oracle.scale_search_lh(wu, sg, H)
+        packed = oracle.quantize_pack(wu, sg, codes)
+        oracle.dequantize(packed, codes, sg)
+        if fq is not None:
+            oracle.fake_quant(fq)
+        return time.perf_counter() - t0, x_rows
+
+    probe = min(R, 32)
+    t_probe, _ = path(probe)
+    rows = int(max(1, min(R, probe * budget_s / max(t_probe, 1e-3))))
+    t, x_rows = path(rows)
     blocks = rows * C // 16
     return {"value": round(blocks / t, 2), "unit": UNIT, "cores": oracle.max_threads(),
             "kind": "oracle", "seconds": round(t, 3),
-            "sample": "whole path on %d of %d weight rows (%d blocks) with %d of %d "
-                      "calibration tokens; blocks/s over the sample" % (rows, R, blocks, x_rows,
-                                                                       X.shape[0])}
-
-
-def _oracle_path(wu_all, xu, rows):
-    import oracle
-    t0 = time.perf_counter()
-    sg = oracle.global_scale(wu_all)
-    H = oracle.gram(xu)
-    wu = np.ascontiguousarray(wu_all[:rows])
-    oracle.scale_search_max(wu, sg)
-    oracle.scale_search_mse(wu, sg)
-    codes, _ = oracle.scale_search_lh(wu, sg, H)
-    packed = oracle.quantize_pack(wu, sg, codes)
-    oracle.dequantize(packed, codes, sg)
-    oracle.fake_quant(xu, want_packed=False)
-    return time.perf_counter() - t0
+            "sample": "the step's rows on %d of %d weight rows (%d blocks) of %s with %d "
+                      "calibration tokens (the same fraction); blocks/s over the sample"
+                      % (rows, R, blocks, L.name, x_rows)}
 
 
 def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
         return
-    inp = make_inputs(args.workload, "cpu")
-    steps = []
-    cb = None
-    for k in range(args.warmup + args.steps):
-        cb = cpu_baseline(args.workload, inp, budget_s=args.cpu_seconds / max(1, args.steps))
-        if k >= args.warmup:
-            steps.append(cb)
+    small = args.workload in ("tiny", "dense", "w4a4")
+    dev = "cpu" if small or not torch.cuda.is_available() else "cuda"
+    run = Runner(args.workload, dev)
+    budget = args.cpu_seconds / max(1, args.steps)
+    for _ in range(args.warmup):
+        cpu_baseline(run, budget_s=min(budget, 2.0))
+    steps = [cpu_baseline(run, budget_s=budget) for _ in range(args.steps)]
     v = statistics.mean(s["value"] for s in steps)
     ms = statistics.mean(s["seconds"] for s in steps) * 1e3
     out = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": UNIT,
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-           "config": {"workload": args.workload, "desc": inp["desc"]},
-           "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": cb["cores"],
-                            "kind": "oracle", "sample": cb["sample"]},
+           "config": {"workload": args.workload, "desc": run.desc},
+           "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": steps[-1]["cores"],
+                            "kind": "oracle", "sample": steps[-1]["sample"]},
            "e2e": {"value": round(v, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -470,7 +591,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="dense", choices=["dense", "tiny", "moe", "mlp_pair"])
+    ap.add_argument("--workload", default="dense", choices=WORKLOAD_NAMES)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -93,32 +93,129 @@ __device__ __forceinline__ void load_block(const uint16_t *p, uint32_t w[8]) {
   w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
 }
 
-// Eight packed bytes (two signed E2M1 codes each) of one block at scale s.
-// s = 0 (code 0) encodes every value as a signed zero.
-__device__ __forceinline__ void encode_block(const uint32_t w[8], float s, uint32_t bytes[8]) {
-  if (s > 0.0f) {
-    const ScaleRecip r = make_recip(s);
-    uint32_t mismatch = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      bytes[j] = e2m1_pair_bracket(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j])), r, mismatch);
-    if (mismatch) {  // some |x|/s within rounding distance of a midpoint
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        bytes[j] = e2m1_mag_exact(fabsf(bf16_lo(w[j])), s) |
-                   (e2m1_mag_exact(fabsf(bf16_hi(w[j])), s) << 4);
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) bytes[j] = 0u;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) bytes[j] |= ((w[j] >> 12) & 0x8u) | ((w[j] >> 24) & 0x80u);
+// ------------------------------------------------------- exact block encode
+//
+// Rounding rule used below (both for E2M1 codes and for the E4M3 max-rule
+// code): t, an fp32 value within one ulp of the exact quotient q, and t_alt,
+// the neighbouring float on the other side of q (chosen by the exact sign of
+// a residual), are rounded to nearest-even by the hardware conversion.  They
+// can only disagree when one of them is a rounding midpoint; q then lies
+// strictly on the other one's side, so the correct code is the odd one of the
+// two (the tie went to the even one).  When neither t is within two floats of
+// a value with 21 zero low mantissa bits (every E2M1 midpoint times a power of
+// two is such a value), t alone rounds exactly.
+
+// Four e2m1x2 conversions into one word: byte i = (code(h_i) << 4) | code(l_i),
+// signed inputs give signed codes (a negative value rounding to 0 gives -0).
+__device__ __forceinline__ uint32_t cvt4_e2m1(float h0, float l0, float h1, float l1, float h2,
+                                              float l2, float h3, float l3) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %1, %2;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %3, %4;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %5, %6;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %7, %8;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(r)
+      : "f"(h0), "f"(l0), "f"(h1), "f"(l1), "f"(h2), "f"(l2), "f"(h3), "f"(l3));
+  return r;
 }
 
-__device__ __forceinline__ uint2 pack8(const uint32_t bytes[8]) {
+// Adjacent float of t towards the side given by the residual (same sign as
+// q - t); t itself when the residual is zero (q == t exactly).
+__device__ __forceinline__ float toward(float t, float rho) {
+  const int rb = __float_as_int(rho);
+  const int dir = ((rb ^ __float_as_int(t)) >> 31) | 1;  // +1 away from 0, -1 towards
+  return __int_as_float(__float_as_int(t) + (rb != 0 ? dir : 0));
+}
+
+// Low 21 mantissa bits of t within two floats of zero (a superset test).
+__device__ __forceinline__ uint32_t near_key(float t) {
+  return (__float_as_uint(t) + 2u) & 0x1FFFF8u;
+}
+
+// Packed signed E2M1 codes of one block (two words, 16 codes) at scale s > 0
+// with r_hi + r_lo = 1/s (r_lo >= 0).
+__device__ __forceinline__ uint2 encode_block(const uint32_t w[8], float s, float r_hi,
+                                              float r_lo) {
+  float t[16];
+  uint32_t nk = 0xFFFFFFFFu;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
+    t[e] = fmaf(x, r_hi, x * r_lo);
+    nk = min(nk, near_key(t[e]));
+  }
+  uint2 c;
+  c.x = cvt4_e2m1(t[1], t[0], t[3], t[2], t[5], t[4], t[7], t[6]);
+  c.y = cvt4_e2m1(t[9], t[8], t[11], t[10], t[13], t[12], t[15], t[14]);
+  if (__any_sync(__activemask(), nk == 0u)) {
+    float ta[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
+      ta[e] = toward(t[e], fmaf(-t[e], s, x));
+    }
+    const uint32_t ax = cvt4_e2m1(ta[1], ta[0], ta[3], ta[2], ta[5], ta[4], ta[7], ta[6]);
+    const uint32_t ay = cvt4_e2m1(ta[9], ta[8], ta[11], ta[10], ta[13], ta[12], ta[15], ta[14]);
+    const uint32_t ox = (c.x & 0x11111111u) * 15u, oy = (c.y & 0x11111111u) * 15u;
+    c.x = (c.x & ox) | (ax & ~ox);
+    c.y = (c.y & oy) | (ay & ~oy);
+  }
+  return c;
+}
+
+// Same codes for any s >= 0 (s = 0: signed zeros; s below 2^-100, where the
+// reciprocal may overflow: the exact fp64 midpoint test).  r_hi is the
+// reciprocal rounded down, so r_lo >= 0 and x = -0 keeps its sign in t.
+__device__ __forceinline__ uint2 encode_block_any(const uint32_t w[8], float s) {
+  if (s >= 0x1p-100f) {
+    const float r_hi = __frcp_rd(s);
+    return encode_block(w, s, r_hi, fmaf(-s, r_hi, 1.0f) * r_hi);
+  }
+  uint32_t bytes[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    bytes[j] = (s > 0.0f ? (e2m1_mag_exact(fabsf(bf16_lo(w[j])), s) |
+                            (e2m1_mag_exact(fabsf(bf16_hi(w[j])), s) << 4))
+                         : 0u) |
+               ((w[j] >> 12) & 0x8u) | ((w[j] >> 24) & 0x80u);
+  }
   return make_uint2(bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24),
                     bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24));
+}
+
+// E4M3 code of amax / (6 s_g), exact (nearest even, saturating at 448), from
+// D = 6 s_g (exact in fp64) and R = 1/D split as r_hi + r_lo: t = amax R, the
+// residual amax - t D is exact in one fp64 fma, and the same odd-code rule
+// picks between the two e4m3x2 conversions.
+struct MaxRule {
+  double D;
+  float r_hi, r_lo;
+};
+__device__ __forceinline__ MaxRule make_max_rule(float s_g) {
+  MaxRule m;
+  m.D = 6.0 * (double)s_g;
+  const double R = 1.0 / m.D;
+  m.r_hi = (float)R;
+  m.r_lo = (float)(R - (double)m.r_hi);
+  return m;
+}
+__device__ __forceinline__ uint32_t max_rule_code_fast(float amax, const MaxRule &m) {
+  const float t = fmaf(amax, m.r_hi, amax * m.r_lo);
+  const double rho = fma(-(double)t, m.D, (double)amax);
+  const float ta = __int_as_float(__float_as_int(t) + (rho > 0.0 ? 1 : (rho < 0.0 ? -1 : 0)));
+  unsigned short pair;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(ta), "f"(t));
+  const uint32_t ct = pair & 0xFFu, ca = pair >> 8;
+  return (ct & 1u) ? ct : ca;  // equal, or the odd one of two neighbours
+}
+
+// E4M3 code (0..0x7E) -> fp32 value, branch-free.
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const float sub = (float)c * 0x1p-9f;
+  const float nor = __uint_as_float((c << 20) + (120u << 23));
+  return c < 8u ? sub : nor;
 }
 
 // bf16 pair of v(q) * s for one packed byte: fp32 product, then bf16 RN.
@@ -148,7 +245,7 @@ __global__ void __launch_bounds__(kThreads) max_rule_kernel(const uint16_t *__re
                                                             const float *__restrict__ s_g,
                                                             uint8_t *__restrict__ codes) {
   const int64_t b = blockIdx.y;
-  const float sg = s_g[b];
+  const MaxRule mr = make_max_rule(s_g[b]);
   w += b * nblk * kBlock;
   codes += b * nblk;
   for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nblk;
@@ -156,7 +253,7 @@ __global__ void __launch_bounds__(kThreads) max_rule_kernel(const uint16_t *__re
     uint32_t v[8];
     load_block(w + i * kBlock, v);
     const float amax = __uint_as_float(amax_bits8(v) << 16);
-    codes[i] = (uint8_t)max_rule_code(amax, sg);
+    codes[i] = (uint8_t)max_rule_code_fast(amax, mr);
   }
 }
 
@@ -170,13 +267,27 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const uint16_t *__restri
   w += b * nblk * kBlock;
   codes += b * nblk;
   packed += b * nblk * (kBlock / 2);
-  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nblk;
-       i += (int64_t)gridDim.x * kThreads) {
-    uint32_t v[8], bytes[8];
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  uint32_t v[8];
+  uint32_t code = 0;
+  if (i < nblk) {
     load_block(w + i * kBlock, v);
-    const float s = effective_scale(sg, codes[i]);
-    encode_block(v, s, bytes);
-    st_stream_v2(packed + i * 8, pack8(bytes));
+    code = codes[i];
+  }
+  for (; i < nblk; i += stride) {
+    // issue the next block's loads before this block's arithmetic
+    uint32_t nv[8];
+    uint32_t ncode = 0;
+    const int64_t n = i + stride;
+    if (n < nblk) {
+      load_block(w + n * kBlock, nv);
+      ncode = codes[n];
+    }
+    st_stream_v2(packed + i * 8, encode_block_any(v, __fmul_rn(sg, e4m3_value(code))));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = nv[j];
+    code = ncode;
   }
 }
 
@@ -209,17 +320,27 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__
                                                               uint8_t *__restrict__ packed,
                                                               uint8_t *__restrict__ codes) {
   const float sg = *s_g;
-  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nblk;
-       i += (int64_t)gridDim.x * kThreads) {
-    uint32_t v[8], bytes[8];
-    load_block(x + i * kBlock, v);
+  const MaxRule mr = make_max_rule(sg);
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  uint32_t v[8];
+  if (i < nblk) load_block(x + i * kBlock, v);
+  for (; i < nblk; i += stride) {
+    // issue the next block's loads before this block's arithmetic
+    uint32_t nv[8];
+    const int64_t n = i + stride;
+    if (n < nblk) load_block(x + n * kBlock, nv);
     const float amax = __uint_as_float(amax_bits8(v) << 16);
-    const uint32_t code = max_rule_code(amax, sg);
-    const float s = effective_scale(sg, code);
-    encode_block(v, s, bytes);
+    const uint32_t code = max_rule_code_fast(amax, mr);
+    const float s = __fmul_rn(sg, e4m3_value(code));
+    const uint2 q = encode_block_any(v, s);
+    const uint32_t bytes[8] = {q.x & 0xFFu, (q.x >> 8) & 0xFFu, (q.x >> 16) & 0xFFu, q.x >> 24,
+                               q.y & 0xFFu, (q.y >> 8) & 0xFFu, (q.y >> 16) & 0xFFu, q.y >> 24};
     store_dequant(out + i * kBlock, bytes, s);
-    if (packed) st_stream_v2(packed + i * 8, pack8(bytes));
+    if (packed) st_stream_v2(packed + i * 8, q);
     if (codes) codes[i] = (uint8_t)code;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = nv[j];
   }
 }
 

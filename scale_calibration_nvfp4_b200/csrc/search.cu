@@ -485,7 +485,6 @@ __global__ void __launch_bounds__(kThreads)
     pp1 += __shfl_xor_sync(0xFFFFFFFFu, pp1, 2);
     const float inf = __int_as_float(0x7F800000);
     float b1 = inf, b2 = inf, b3 = inf;
-    const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 
     int j = 0;
     for (int k = 0; k < ncls; ++k) {

@@ -321,12 +321,20 @@ def dist_env():
     return 0, 1, 0
 
 
-def max_over_ranks(pg, value):
+def max_over_ranks(pg, value, device="cuda"):
+    """Max of a per-rank value over all ranks (the job's time is the slowest
+    rank's)."""
     if pg is None:
         return value
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return t.item()
+
+
+def job_value(world, blocks_per_rank, ms_per_step):
+    """Whole-job throughput: every rank processes its own replica of the
+    workload (weak scaling), timed by the slowest rank."""
+    return world * blocks_per_rank / (ms_per_step / 1e3)
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -388,7 +396,7 @@ def run_gpu(args):
         step_ms.append(ev[k][0].elapsed_time(ev[k][-1]))
     ms_per_step = max_over_ranks(pg, sum(step_ms)) / args.steps
     blocks = run.blocks()
-    value = world * blocks / (ms_per_step / 1e3)
+    value = job_value(world, blocks, ms_per_step)
 
     e2e = None if args.no_e2e else run_e2e(run, args, pg, world)
 
@@ -483,7 +491,7 @@ def run_e2e(run, args, pg, world):
     ms_step = max_over_ranks(pg, e0.elapsed_time(e1)) / args.steps
     h2d = sum(h.numel() * h.element_size() for _, h in ins)
     d2h = sum(h.numel() * h.element_size() for _, h in outs)
-    return {"value": round(world * run.blocks() / (ms_step / 1e3), 1), "unit": UNIT,
+    return {"value": round(job_value(world, run.blocks(), ms_step), 1), "unit": UNIT,
             "ms_per_step": round(ms_step, 5), "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h}
 

@@ -360,3 +360,31 @@ def test_snr_closed_form_arithmetic():
     for ratio, _, db in g["m_over_sigma"]:
         est = 20 * math.log10(1.0 / (float(ratio) / 6.0))
         assert est == pytest.approx(float(db), abs=0.06)
+
+
+def test_grouped_gram_is_per_group_product(oracle_mod):
+    g = torch.Generator().manual_seed(29)
+    X = torch.randn(50, 32, generator=g).to(torch.bfloat16)
+    Xu = bf16_bits(X)
+    Xf = bits_to_f64(Xu)
+    offsets = np.array([0, 0, 7, 30, 30, 50], np.int64)
+    H = oracle_mod.gram_grouped(Xu, offsets, 5)
+    for gi in range(5):
+        lo, hi = offsets[gi], offsets[gi + 1]
+        for j in range(2):
+            Xb = Xf[lo:hi, 16 * j:16 * j + 16]
+            np.testing.assert_allclose(H[gi, j], Xb.T @ Xb, rtol=1e-15, atol=0)
+
+
+def test_sampled_search_equals_full_search(oracle_mod):
+    W, X = _tiny_layer(20, 64, 32, 31)
+    s_g = oracle_mod.global_scale(W)
+    H = oracle_mod.gram(X)
+    full, fobj = oracle_mod.scale_search_lh(W, s_g, H)
+    mfull, mobj = oracle_mod.scale_search_mse(W, s_g)
+    rows = np.array([0, 3, 19, 7, 7])
+    blocks = np.array([0, 3, 2, 1, 0])
+    c, o = oracle_mod.scale_search_sampled(W, s_g, H, rows, blocks)
+    assert np.array_equal(c, full[rows, blocks]) and np.array_equal(o, fobj[rows, blocks])
+    c, o = oracle_mod.scale_search_sampled(W, s_g, None, rows, blocks)
+    assert np.array_equal(c, mfull[rows, blocks]) and np.array_equal(o, mobj[rows, blocks])

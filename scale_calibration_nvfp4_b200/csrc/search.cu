@@ -161,6 +161,45 @@ __device__ void cholesky16(const float *Hs, float *Lf) {
   }
 }
 
+// Lower bound of the smallest eigenvalue of L L^T, computed by one warp and
+// returned to every lane: 0.98 / ||(L L^T)^-1||_1.  For a symmetric matrix the
+// column-sum norm bounds the 2-norm from above, so this bounds lambda_min from
+// below (with 2% to spare for rounding).  Lane i < 16 forms column i of the
+// inverse by a forward and a backward triangular solve in fp64.  A dropped
+// pivot (zero diagonal in L) makes the matrix singular: the bound is 0.
+__device__ __noinline__ float lambda_lower_bound(const float *Lf) {
+  const int lane = threadIdx.x & 31;
+  double colsum = 0.0;
+  int singular = 0;
+  if (lane < 16) {
+    // once per CTA: kept rolled (y in local memory) so that it does not raise
+    // the kernel's register budget
+    double y[16];
+#pragma unroll 1
+    for (int k = 0; k < 16; ++k) {
+      double acc = (k == lane) ? 1.0 : 0.0;
+#pragma unroll 1
+      for (int m = 0; m < k; ++m) acc = fma(-(double)Lf[k * 16 + m], y[m], acc);
+      const double d = (double)Lf[k * 16 + k];
+      singular |= (d == 0.0);
+      y[k] = acc / d;
+    }
+#pragma unroll 1
+    for (int k = 15; k >= 0; --k) {
+      double acc = y[k];
+#pragma unroll 1
+      for (int m = k + 1; m < 16; ++m) acc = fma(-(double)Lf[m * 16 + k], y[m], acc);
+      y[k] = acc / (double)Lf[k * 16 + k];
+      colsum += fabs(y[k]);
+    }
+  }
+  singular = __any_sync(0xFFFFFFFFu, singular);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) colsum = fmax(colsum, __shfl_xor_sync(0xFFFFFFFFu, colsum, o));
+  if (singular || !(colsum > 0.0) || !(colsum < 1e300)) return 0.0f;
+  return (float)(0.98 / colsum);
+}
+
 // fp64 objective of candidate c for one block, from the definition: exact
 // E2M1 codes, delta_i = w_i - v_i s, E = delta H delta^T (MSE: H = I).  Rare
 // path: loops are kept rolled so that the caller's register budget is not
@@ -305,7 +344,7 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ CandInfo cand[kCandidates];
   __shared__ float Hs[kLH ? 256 : 1];
   __shared__ float Lf[kLH ? 256 : 1];
-  __shared__ float sigma_sh;
+  __shared__ float sigma_sh, lambda_sh;
   __shared__ int ncls_sh, zero_h_sh;
 
   const float s_g = s_g_arr[batch];
@@ -325,19 +364,23 @@ __global__ void __launch_bounds__(kThreads)
       for (int i = lane; i < 256; i += 32) m = fmaxf(m, fabsf(Lf[i]));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      const float lam = lambda_lower_bound(Lf);
       if (lane == 0) {
         int e = 0;
         frexpf(m, &e);  // m < 2^e
         sigma_sh = m > 0.0f ? ldexpf(1.0f, 15 - e) : 1.0f;
         zero_h_sh = !(m > 0.0f);
+        lambda_sh = lam;
       }
     }
   } else if (threadIdx.x == 0) {
     sigma_sh = 1.0f;
     zero_h_sh = 0;
+    lambda_sh = 1.0f;  // H = I
   }
   __syncthreads();
   const float sigma = sigma_sh;
+  const float sqrt_lambda = sqrtf(lambda_sh);
 
   if (kLH && zero_h_sh) {  // every candidate scores 0: the smallest code wins
     const int64_t r_end = min(R, row_base + kRowsPerCta);
@@ -485,8 +528,21 @@ __global__ void __launch_bounds__(kThreads)
     pp1 += __shfl_xor_sync(0xFFFFFFFFu, pp1, 2);
     const float inf = __int_as_float(0x7F800000);
     float b1 = inf, b2 = inf, b3 = inf;
+    // Pruning small scales.  For s < amax_row / 6 the row's largest value
+    // saturates, so |delta| >= amax_row - 6 s and E >= lambda_min (amax_row -
+    // 6 s)^2; within a class candidates run from the largest scale down, so
+    // once this bound (in the objective's units) exceeds the best objective
+    // beyond the tie band for every row of the warp, the rest of the class is
+    // skipped.  Rows past the end and all-zero rows never hold the warp back.
+    uint32_t am = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) am = __vmaxu2(am, (upper ? W1[i] : W0[i]) & 0x7FFF7FFFu);
+    am = max(am & 0xFFFFu, am >> 16);
+    const float amax_row = __uint_as_float(am << 16);
+    const float zl = zscale * sqrt_lambda;
+    const float row_floor = kZeroFloor * (upper ? pp1 : pp0);
 
-    int j = 0;
+    int jbegin = 0;
     for (int k = 0; k < ncls; ++k) {
       const ClassInfo ci = cls[k];
       // class quotient t and its neighbour across q, per element
@@ -503,23 +559,29 @@ __global__ void __launch_bounds__(kThreads)
         // (every rounding midpoint times a power of two is one), and not exact
         near = near || (step != 0 && ((__float_as_uint(tt) + 2u) & 0x1FFFFFu) <= 4u);
       }
-      if (!kAltSkip || __any_sync(0xFFFFFFFFu, near)) {
-#pragma unroll kUnroll
-        for (; j < ci.end; ++j) {
-          const CandInfo cd = cand[j];
-          const float e = candidate_objective<kLH, true>(tq, ta, cd.f, cd.s * umul, sgn, bh, bl,
-                                                         pz, upper);
-          track3(key_of(e, cd.c), b1, b2, b3);
+      const bool alt = !kAltSkip || __any_sync(0xFFFFFFFFu, near);
+      // two candidates per step (independent chains), largest scale first
+      for (int j = ci.end - 1; j >= jbegin; j -= 2) {
+        const CandInfo c0 = cand[j];
+        const bool two = j - 1 >= jbegin;
+        const CandInfo c1 = cand[two ? j - 1 : j];
+        float e0, e1;
+        if (alt) {
+          e0 = candidate_objective<kLH, true>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
+          e1 = candidate_objective<kLH, true>(tq, ta, c1.f, c1.s * umul, sgn, bh, bl, pz, upper);
+        } else {
+          e0 = candidate_objective<kLH, false>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
+          e1 = candidate_objective<kLH, false>(tq, ta, c1.f, c1.s * umul, sgn, bh, bl, pz, upper);
         }
-      } else {  // no quotient near a midpoint: t alone rounds exactly
-#pragma unroll kUnroll
-        for (; j < ci.end; ++j) {
-          const CandInfo cd = cand[j];
-          const float e = candidate_objective<kLH, false>(tq, ta, cd.f, cd.s * umul, sgn, bh,
-                                                          bl, pz, upper);
-          track3(key_of(e, cd.c), b1, b2, b3);
-        }
+        track3(key_of(e0, c0.c), b1, b2, b3);
+        if (two) track3(key_of(e1, c1.c), b1, b2, b3);
+        // lower bound at the smaller of the two scales (all later ones are smaller)
+        const float d = zl * fmaf(-6.0f, c1.s, amax_row);
+        const bool done = amax_row == 0.0f ||
+                          (d > 0.0f && d * d * (1.0f - 2.0f * kTieBand) > b1 + row_floor);
+        if (__all_sync(0xFFFFFFFFu, done)) break;
       }
+      jbegin = ci.end;
     }
 
     // lane t = 0 finishes row g, lane t = 2 row g + 8

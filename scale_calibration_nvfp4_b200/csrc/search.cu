@@ -37,8 +37,9 @@
 // Winner: fp32 screen keeping the best three objectives; when the best two
 // are within 2^-12 (relative) or the best is numerically zero, the candidates
 // in the band are re-scored in fp64 straight from the definition
-// (delta H_b delta^T with exact E2M1 codes) and the first minimum in
-// ascending code order wins.
+// (delta H_b delta^T with exact E2M1 codes, one element per lane, two
+// candidates per warp pass) and the first minimum in ascending code order
+// wins.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -53,15 +54,11 @@ constexpr int kTileRows = 16;
 #ifndef NVFP4_SEARCH_TILES
 #define NVFP4_SEARCH_TILES 4
 #endif
-#ifndef NVFP4_SEARCH_UNROLL
-#define NVFP4_SEARCH_UNROLL 2
-#endif
 #ifndef NVFP4_SEARCH_ALT_SKIP
 #define NVFP4_SEARCH_ALT_SKIP 1
 #endif
 constexpr int kTilesPerWarp = NVFP4_SEARCH_TILES;
 constexpr bool kAltSkip = NVFP4_SEARCH_ALT_SKIP;
-constexpr int kUnroll = NVFP4_SEARCH_UNROLL;
 constexpr int kRowsPerCta = kWarps * kTileRows * kTilesPerWarp;  // 256
 constexpr float kTieBand = 1.0f / 4096.0f;
 constexpr float kZeroFloor = 0x1p-40f;  // relative to ||p||^2
@@ -200,57 +197,58 @@ __device__ __noinline__ float lambda_lower_bound(const float *Lf) {
   return (float)(0.98 / colsum);
 }
 
-// fp64 objective of candidate c for one block, from the definition: exact
-// E2M1 codes, delta_i = w_i - v_i s, E = delta H delta^T (MSE: H = I).  Rare
-// path: loops are kept rolled so that the caller's register budget is not
-// raised by it.
-__device__ __noinline__ double objective64(const float *x, float s_g, int c, const float *Hs) {
+// fp64 objective of one candidate from the definition, computed by a
+// half-warp: lane l holds element j = l & 15 of the block (value x) and the
+// lanes of each half score their own candidate c.  Exact E2M1 codes,
+// delta_j = x_j - v_j s, row_j = sum_k H_jk delta_k, E = sum_j delta_j row_j
+// (MSE: H = I); every lane of the half returns the same E.
+__device__ __noinline__ double objective64_half(float x, float s_g, int c, const float *Hs) {
+  const int lane = threadIdx.x & 31, j = lane & 15, half = lane & 16;
   const float s = effective_scale(s_g, (uint32_t)c);
-  double d[16];
-#pragma unroll 1
-  for (int j = 0; j < 16; ++j) {
-    const uint32_t k = e2m1_mag_exact(fabsf(x[j]), s);
-    const double v = k < 2 ? 0.5 * k : (1.0 + 0.5 * (double)(k & 1)) * (double)(1 << ((k >> 1) - 1));
-    d[j] = (double)x[j] - copysign(v, (double)x[j]) * (double)s;
-  }
-  double e = 0.0;
+  const uint32_t k = e2m1_mag_exact(fabsf(x), s);
+  const double v = k < 2 ? 0.5 * k : (1.0 + 0.5 * (double)(k & 1)) * (double)(1 << ((k >> 1) - 1));
+  const double d = (double)x - copysign(v, (double)x) * (double)s;
+  double row = d;
   if (Hs) {
-#pragma unroll 1
-    for (int j = 0; j < 16; ++j) {
-      double row = 0.0;
+    row = 0.0;
 #pragma unroll 4
-      for (int k = 0; k < 16; ++k) row = fma((double)Hs[j * 16 + k], d[k], row);
-      e = fma(d[j], row, e);
-    }
-  } else {
-#pragma unroll 1
-    for (int j = 0; j < 16; ++j) e = fma(d[j], d[j], e);
+    for (int m = 0; m < 16; ++m)
+      row = fma((double)Hs[j * 16 + m], __shfl_sync(0xFFFFFFFFu, d, half | m), row);
   }
+  double e = d * row;
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) e += __shfl_xor_sync(0xFFFFFFFFu, e, o);
   return e;
 }
 
-// Near-tie resolution for one block: fp64 scores of {c1, c2}, or of every
-// candidate when more than two may lie in the band; first minimum wins.
+// Near-tie resolution for one block by the whole warp: fp64 scores of
+// {c1, c2}, or of every candidate (two per pass) when more than two may lie
+// in the band; the first minimum in ascending code order wins.  Every lane
+// returns the result.
 __device__ __noinline__ int refine_block(const uint16_t *wrow, float s_g, const float *Hs,
                                          int c1, int c2, bool full, float *obj) {
-  float x[16];
-#pragma unroll 1
-  for (int j = 0; j < 16; ++j) x[j] = __uint_as_float((uint32_t)wrow[j] << 16);
+  const int lane = threadIdx.x & 31;
+  const float x = __uint_as_float((uint32_t)wrow[lane & 15] << 16);
   double best = __longlong_as_double(0x7FF0000000000000LL);
   int best_c = 1;
   if (full) {
 #pragma unroll 1
-    for (int c = 1; c <= kCandidates; ++c) {
-      const double e = objective64(x, s_g, c, Hs);
-      if (e < best) {
-        best = e;
+    for (int c = 1; c < kCandidates; c += 2) {
+      const double e = objective64_half(x, s_g, c + (lane >> 4), Hs);
+      const double ea = __shfl_sync(0xFFFFFFFFu, e, 0), eb = __shfl_sync(0xFFFFFFFFu, e, 16);
+      if (ea < best) {
+        best = ea;
         best_c = c;
+      }
+      if (eb < best) {
+        best = eb;
+        best_c = c + 1;
       }
     }
   } else {
     const int lo = min(c1, c2), hi = max(c1, c2);
-    const double el = objective64(x, s_g, lo, Hs);
-    const double eh = objective64(x, s_g, hi, Hs);
+    const double e = objective64_half(x, s_g, lane < 16 ? lo : hi, Hs);
+    const double el = __shfl_sync(0xFFFFFFFFu, e, 0), eh = __shfl_sync(0xFFFFFFFFu, e, 16);
     best = el;
     best_c = lo;
     if (eh < el) {
@@ -327,10 +325,72 @@ __device__ __forceinline__ float candidate_objective(const float tq[8], const fl
   return mine;
 }
 
+// Per column block (and batch element) of H: the f16 high/low B-operand
+// fragments of sigma L for every lane, sigma, the eigenvalue bound and the
+// zero-H flag.  One warp per block; the search kernel then starts straight on
+// its rows.
+struct Factor {
+  float sigma;   // power of two putting max |L| in [2^14, 2^15)
+  float lambda;  // lower bound of lambda_min(L L^T), 0 when unknown
+  int zero;      // H_b == 0 (every candidate scores 0)
+  int pad;
+};
+
+__global__ void __launch_bounds__(kThreads)
+    factor_kernel(const float *__restrict__ H, int64_t nblocks, uint4 *__restrict__ frag,
+                  Factor *__restrict__ fac) {
+  __shared__ float Hs[kWarps][256];
+  __shared__ float Lf[kWarps][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t blk = (int64_t)blockIdx.x * kWarps + warp;
+  if (blk >= nblocks) return;  // whole warps only
+  const float *Hb = H + blk * 256;
+  for (int i = lane; i < 256; i += 32) Hs[warp][i] = Hb[i];
+  __syncwarp();
+  cholesky16(Hs[warp], Lf[warp]);
+  __syncwarp();
+  float m = 0.0f;
+  for (int i = lane; i < 256; i += 32) m = fmaxf(m, fabsf(Lf[warp][i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  const float lam = lambda_lower_bound(Lf[warp]);
+  int e = 0;
+  frexpf(m, &e);  // m < 2^e
+  const float sigma = m > 0.0f ? ldexpf(1.0f, 15 - e) : 1.0f;
+  // this lane's fragments: B[k][n] = sigma L[k][n], n = 8 nt + g, k = 2t + 8 half + {0, 1}
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    const int n = nt * 8 + g;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int k0 = 2 * t + 8 * half;
+      const float x0 = Lf[warp][k0 * 16 + n] * sigma, x1 = Lf[warp][(k0 + 1) * 16 + n] * sigma;
+      const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+      const __half l0 = __float2half_rn(x0 - __half2float(h0));
+      const __half l1 = __float2half_rn(x1 - __half2float(h1));
+      hi[nt * 2 + half] = pack_half2(h0, h1);
+      lo[nt * 2 + half] = pack_half2(l0, l1);
+    }
+  }
+  frag[(blk * 32 + lane) * 2] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  frag[(blk * 32 + lane) * 2 + 1] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  if (lane == 0) {
+    Factor f;
+    f.sigma = sigma;
+    f.lambda = lam;
+    f.zero = !(m > 0.0f);
+    f.pad = 0;
+    fac[blk] = f;
+  }
+}
+
 template <bool kLH>
 __global__ void __launch_bounds__(kThreads)
     search_kernel(const uint16_t *__restrict__ w, int64_t R, int64_t C,
                   const float *__restrict__ s_g_arr, const float *__restrict__ H,
+                  const uint4 *__restrict__ frag, const Factor *__restrict__ fac,
                   uint8_t *__restrict__ codes, float *__restrict__ best_obj) {
   const int64_t nb = C / kBlock;
   const int64_t b = blockIdx.y;
@@ -342,54 +402,46 @@ __global__ void __launch_bounds__(kThreads)
 
   __shared__ ClassInfo cls[kMaxClasses];
   __shared__ CandInfo cand[kCandidates];
-  __shared__ float Hs[kLH ? 256 : 1];
-  __shared__ float Lf[kLH ? 256 : 1];
-  __shared__ float sigma_sh, lambda_sh;
-  __shared__ int ncls_sh, zero_h_sh;
+  __shared__ int ncls_sh;
 
   const float s_g = s_g_arr[batch];
   const uint16_t *wb = w + batch * R * C + b * kBlock;
   uint8_t *cb = codes + batch * R * nb + b;
   float *ob = best_obj ? best_obj + batch * R * nb + b : nullptr;
 
-  // ---- factor of H_b, its scale for f16, and the zero-H shortcut
+  // ---- factor of H_b (from factor_kernel) and the zero-H shortcut
+  const int64_t blk = batch * nb + b;
+  const float *Hb = kLH ? H + blk * 256 : nullptr;  // the definition, for re-scoring
+  float sigma = 1.0f, lambda = 1.0f;  // MSE: H = I
+  uint32_t bh[2][2], bl[2][2];
   if (kLH) {
-    const float *Hb = H + (batch * nb + b) * 256;
-    for (int i = threadIdx.x; i < 256; i += kThreads) Hs[i] = Hb[i];
-    __syncthreads();
-    if (warp == 0) {
-      cholesky16(Hs, Lf);
-      __syncwarp();
-      float m = 0.0f;
-      for (int i = lane; i < 256; i += 32) m = fmaxf(m, fabsf(Lf[i]));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-      const float lam = lambda_lower_bound(Lf);
-      if (lane == 0) {
-        int e = 0;
-        frexpf(m, &e);  // m < 2^e
-        sigma_sh = m > 0.0f ? ldexpf(1.0f, 15 - e) : 1.0f;
-        zero_h_sh = !(m > 0.0f);
-        lambda_sh = lam;
+    const Factor f = fac[blk];
+    if (f.zero) {  // every candidate scores 0: the smallest code wins
+      const int64_t r_end = min(R, row_base + kRowsPerCta);
+      for (int64_t r = row_base + threadIdx.x; r < r_end; r += kThreads) {
+        cb[r * nb] = 1;
+        if (ob) ob[r * nb] = 0.0f;
       }
+      return;
     }
-  } else if (threadIdx.x == 0) {
-    sigma_sh = 1.0f;
-    zero_h_sh = 0;
-    lambda_sh = 1.0f;  // H = I
+    sigma = f.sigma;
+    lambda = f.lambda;
+    const uint4 h = frag[(blk * 32 + lane) * 2], l = frag[(blk * 32 + lane) * 2 + 1];
+    bh[0][0] = h.x; bh[0][1] = h.y; bh[1][0] = h.z; bh[1][1] = h.w;
+    bl[0][0] = l.x; bl[0][1] = l.y; bl[1][0] = l.z; bl[1][1] = l.w;
+  } else {
+    // B = I: u = v exactly
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int n = nt * 8 + g, k0 = 2 * t + 8 * half;
+        bh[nt][half] = pack_half2(__float2half_rn(k0 == n ? 1.0f : 0.0f),
+                                  __float2half_rn(k0 + 1 == n ? 1.0f : 0.0f));
+        bl[nt][half] = 0u;
+      }
   }
-  __syncthreads();
-  const float sigma = sigma_sh;
-  const float sqrt_lambda = sqrtf(lambda_sh);
-
-  if (kLH && zero_h_sh) {  // every candidate scores 0: the smallest code wins
-    const int64_t r_end = min(R, row_base + kRowsPerCta);
-    for (int64_t r = row_base + threadIdx.x; r < r_end; r += kThreads) {
-      cb[r * nb] = 1;
-      if (ob) ob[r * nb] = 0.0f;
-    }
-    return;
-  }
+  const float sqrt_lambda = sqrtf(lambda);
 
   // ---- candidate tables (per CTA, from this batch element's s_g)
   const bool by_class = s_g >= 0x1p-100f && s_g < 0x1p100f;
@@ -423,29 +475,6 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   const int ncls = ncls_sh;
-
-  // ---- B operand fragments: L * sigma split in f16 hi + lo (LH) or I (MSE)
-  uint32_t bh[2][2], bl[2][2];
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    const int n = nt * 8 + g;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int k0 = 2 * t + 8 * half;
-      if (kLH) {
-        const float x0 = Lf[k0 * 16 + n] * sigma, x1 = Lf[(k0 + 1) * 16 + n] * sigma;
-        const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
-        const __half l0 = __float2half_rn(x0 - __half2float(h0));
-        const __half l1 = __float2half_rn(x1 - __half2float(h1));
-        bh[nt][half] = pack_half2(h0, h1);
-        bl[nt][half] = pack_half2(l0, l1);
-      } else {
-        bh[nt][half] = pack_half2(__float2half_rn(k0 == n ? 1.0f : 0.0f),
-                                  __float2half_rn(k0 + 1 == n ? 1.0f : 0.0f));
-        bl[nt][half] = 0u;
-      }
-    }
-  }
 
   for (int tile = 0; tile < kTilesPerWarp; ++tile) {
     const int64_t r0 = row_base + (int64_t)(tile * kWarps + warp) * kTileRows;
@@ -584,24 +613,38 @@ __global__ void __launch_bounds__(kThreads)
       jbegin = ci.end;
     }
 
-    // lane t = 0 finishes row g, lane t = 2 row g + 8
-    if ((t & 1) == 0) {
-      const int64_t r = upper ? rg8 : rg;
-      if (r < R) {
-        const float fl = kZeroFloor * (upper ? pp1 : pp0);
-        int code = code_of(b1);
-        float obj = b1 / (zscale * zscale);
-        if (upper ? zero1 : zero0) {  // every candidate scores exactly 0
-          code = 1;
-          obj = 0.0f;
-        } else if (b2 - b1 <= kTieBand * b2 || b1 <= fl) {
-          const bool full = !(b3 - b1 > kTieBand * b3 + fl);
-          code = refine_block(wb + r * C, s_g, kLH ? Hs : nullptr, code_of(b1), code_of(b2), full,
-                              &obj);
-        }
-        cb[r * nb] = (uint8_t)code;
-        if (ob) ob[r * nb] = obj;
+    // lane t = 0 finishes row g, lane t = 2 row g + 8; near ties are
+    // re-scored by the whole warp, one row at a time
+    const int64_t r = upper ? rg8 : rg;
+    const bool owner = (t & 1) == 0 && r < R;
+    int code = code_of(b1);
+    float obj = b1 / (zscale * zscale);
+    int need = 0;  // 1: re-score the best two, 2: re-score every candidate
+    if (owner) {
+      const float fl = kZeroFloor * (upper ? pp1 : pp0);
+      if (upper ? zero1 : zero0) {  // every candidate scores exactly 0
+        code = 1;
+        obj = 0.0f;
+      } else if (b2 - b1 <= kTieBand * b2 || b1 <= fl) {
+        need = (b3 - b1 > kTieBand * b3 + fl) ? 1 : 2;
       }
+    }
+    for (uint32_t pend = __ballot_sync(0xFFFFFFFFu, need != 0); pend; pend &= pend - 1) {
+      const int src = __ffs(pend) - 1;
+      const int64_t rr = __shfl_sync(0xFFFFFFFFu, (long long)r, src);
+      const int n = __shfl_sync(0xFFFFFFFFu, need, src);
+      const int k1 = __shfl_sync(0xFFFFFFFFu, code_of(b1), src);
+      const int k2 = __shfl_sync(0xFFFFFFFFu, code_of(b2), src);
+      float o;
+      const int c = refine_block(wb + rr * C, s_g, Hb, k1, k2, n == 2, &o);
+      if (lane == src) {
+        code = c;
+        obj = o;
+      }
+    }
+    if (owner) {
+      cb[r * nb] = (uint8_t)code;
+      if (ob) ob[r * nb] = obj;
     }
   }
 }
@@ -614,11 +657,28 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
   if (R == 0 || C == 0) return cudaSuccess;
   dim3 grid((unsigned)((R + kRowsPerCta - 1) / kRowsPerCta), (unsigned)(C / kBlock),
             (unsigned)batch);
-  if (local_hessian)
-    search_kernel<true><<<grid, kThreads, 0, st>>>(w, R, C, s_g, H, codes, best_obj);
-  else
-    search_kernel<false><<<grid, kThreads, 0, st>>>(w, R, C, s_g, nullptr, codes, best_obj);
-  return cudaGetLastError();
+  if (!local_hessian) {
+    search_kernel<false><<<grid, kThreads, 0, st>>>(w, R, C, s_g, nullptr, nullptr, nullptr,
+                                                    codes, best_obj);
+    return cudaGetLastError();
+  }
+  // factors of every H_b first (stream-ordered scratch, freed after the search)
+  const int64_t nblocks = batch * (C / kBlock);
+  const size_t frag_bytes = (size_t)nblocks * 32 * 2 * sizeof(uint4);
+  void *scratch = nullptr;
+  cudaError_t e = scratch_alloc(&scratch, frag_bytes + (size_t)nblocks * sizeof(Factor), st);
+  if (e != cudaSuccess) return e;
+  uint4 *frag = static_cast<uint4 *>(scratch);
+  Factor *fac = reinterpret_cast<Factor *>(static_cast<char *>(scratch) + frag_bytes);
+  factor_kernel<<<(unsigned)((nblocks + kWarps - 1) / kWarps), kThreads, 0, st>>>(H, nblocks,
+                                                                                  frag, fac);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    search_kernel<true><<<grid, kThreads, 0, st>>>(w, R, C, s_g, H, frag, fac, codes, best_obj);
+    e = cudaGetLastError();
+  }
+  const cudaError_t ef = scratch_free(scratch, st);
+  return e != cudaSuccess ? e : ef;
 }
 
 }  // namespace nvfp4

@@ -403,6 +403,8 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ ClassInfo cls[kMaxClasses];
   __shared__ CandInfo cand[kCandidates];
   __shared__ int ncls_sh;
+  __shared__ uint4 Ws[kRowsPerCta][2];     // the CTA's 16-element row segments
+  __shared__ uint32_t keys[kRowsPerCta];  // amax << 16 | local row, sorted
 
   const float s_g = s_g_arr[batch];
   const uint16_t *wb = w + batch * R * C + b * kBlock;
@@ -476,35 +478,65 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
   const int ncls = ncls_sh;
 
-  for (int tile = 0; tile < kTilesPerWarp; ++tile) {
-    const int64_t r0 = row_base + (int64_t)(tile * kWarps + warp) * kTileRows;
-    if (r0 >= R) break;
-    const int64_t rg = r0 + g, rg8 = r0 + g + 8;
-    // full rows g and g+8 (zeros past the end)
+  // ---- the CTA's rows, staged in shared memory and ordered by amax so that
+  // every warp tile holds rows of similar magnitude: the pruning bounds below
+  // then stop the candidate walk at nearly the same point for all 16 rows.
+  // Sort key: amax (bf16 magnitude bits) above the local row index; rows past
+  // the end get magnitude 0xFFFF (zero data) and sort last.
+  for (int i = threadIdx.x; i < kRowsPerCta; i += kThreads) {
+    const int64_t r = row_base + i;
+    uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
+    uint32_t key = 0xFFFF0000u | (uint32_t)i;
+    if (r < R) {
+      const uint4 *q = reinterpret_cast<const uint4 *>(wb + r * C);
+      a0 = ld_stream_v4(q);
+      a1 = ld_stream_v4(q + 1);
+      const uint32_t w8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      key = (amax_bits8(w8) << 16) | (uint32_t)i;
+    }
+    Ws[i][0] = a0;
+    Ws[i][1] = a1;
+    keys[i] = key;
+  }
+  __syncthreads();
+  // bitonic sort of the 256 keys, ascending; one compare-exchange per thread
+  // and step
+  for (int size = 2; size <= kRowsPerCta; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const int i = 2 * threadIdx.x - (threadIdx.x & (stride - 1));
+      const int j = i + stride;
+      const uint32_t ki = keys[i], kj = keys[j];
+      if ((ki > kj) == ((i & size) == 0)) {
+        keys[i] = kj;
+        keys[j] = ki;
+      }
+      __syncthreads();
+    }
+  }
+
+  for (int tile = warp; tile < kRowsPerCta / kTileRows; tile += kWarps) {
+    const uint32_t kg = keys[tile * kTileRows + g], kg8 = keys[tile * kTileRows + g + 8];
+    const bool v0 = (kg >> 16) != 0xFFFFu, v1 = (kg8 >> 16) != 0xFFFFu;
+    if (!__any_sync(0xFFFFFFFFu, v0 || v1)) break;  // only padding from here on
+    const int i0 = (int)(kg & 0xFFFFu), i1 = (int)(kg8 & 0xFFFFu);
     uint32_t W0[8], W1[8];
     {
-      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-      const uint4 *q0 = reinterpret_cast<const uint4 *>(wb + rg * C);
-      const uint4 *q1 = reinterpret_cast<const uint4 *>(wb + rg8 * C);
-      const uint4 a0 = rg < R ? ld_stream_v4(q0) : z, a1 = rg < R ? ld_stream_v4(q0 + 1) : z;
-      const uint4 c0 = rg8 < R ? ld_stream_v4(q1) : z, c1 = rg8 < R ? ld_stream_v4(q1 + 1) : z;
+      const uint4 a0 = Ws[i0][0], a1 = Ws[i0][1], c0 = Ws[i1][0], c1 = Ws[i1][1];
       W0[0] = a0.x; W0[1] = a0.y; W0[2] = a0.z; W0[3] = a0.w;
       W0[4] = a1.x; W0[5] = a1.y; W0[6] = a1.z; W0[7] = a1.w;
       W1[0] = c0.x; W1[1] = c0.y; W1[2] = c0.z; W1[3] = c0.w;
       W1[4] = c1.x; W1[5] = c1.y; W1[6] = c1.z; W1[7] = c1.w;
     }
-    bool zero0 = true, zero1 = true;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      zero0 = zero0 && ((W0[i] & 0x7FFF7FFFu) == 0u);
-      zero1 = zero1 && ((W1[i] & 0x7FFF7FFFu) == 0u);
-    }
+    // row amax (bf16 magnitude bits; 0 for padding) and the tile's largest
+    const uint32_t am0 = v0 ? kg >> 16 : 0u, am1 = v1 ? kg8 >> 16 : 0u;
+    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(am0, am1));
     // this lane's four pairs in MMA order: (g,2t) (g+8,2t) (g,2t+8) (g+8,2t+8)
     const uint32_t pw[4] = {pick4(W0[0], W0[1], W0[2], W0[3], t),
                             pick4(W1[0], W1[1], W1[2], W1[3], t),
                             pick4(W0[4], W0[5], W0[6], W0[7], t),
                             pick4(W1[4], W1[5], W1[6], W1[7], t)};
     // element k of the lane in C order: 2i, 2i+1 = low, high half of pair i
+    // (row g: elements 0, 1, 4, 5; row g + 8: 2, 3, 6, 7)
     float xs[8], a[8];
     uint32_t sgn = 0;
 #pragma unroll
@@ -523,11 +555,6 @@ __global__ void __launch_bounds__(kThreads)
     float pz[2][4];
     float zscale = 1.0f;  // objectives carry zscale^2
     if (kLH) {
-      uint32_t m = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m = __vmaxu2(m, __vmaxu2(W0[i] & 0x7FFF7FFFu, W1[i] & 0x7FFF7FFFu));
-      m = max(m & 0xFFFFu, m >> 16);
-      m = __reduce_max_sync(0xFFFFFFFFu, m);
       const int emax = (int)(m >> 7) - 127;  // exponent of the tile's largest |w|
       const int kw = m ? 14 - emax : 0;
       const float wsc = ldexpf(1.0f, kw);
@@ -557,19 +584,24 @@ __global__ void __launch_bounds__(kThreads)
     pp1 += __shfl_xor_sync(0xFFFFFFFFu, pp1, 2);
     const float inf = __int_as_float(0x7F800000);
     float b1 = inf, b2 = inf, b3 = inf;
-    // Pruning small scales.  For s < amax_row / 6 the row's largest value
-    // saturates, so |delta| >= amax_row - 6 s and E >= lambda_min (amax_row -
-    // 6 s)^2; within a class candidates run from the largest scale down, so
-    // once this bound (in the objective's units) exceeds the best objective
-    // beyond the tie band for every row of the warp, the rest of the class is
-    // skipped.  Rows past the end and all-zero rows never hold the warp back.
-    uint32_t am = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) am = __vmaxu2(am, (upper ? W1[i] : W0[i]) & 0x7FFF7FFFu);
-    am = max(am & 0xFFFFu, am >> 16);
-    const float amax_row = __uint_as_float(am << 16);
-    const float zl = zscale * sqrt_lambda;
+    // Pruning, with lambda a lower bound of the smallest eigenvalue of H_b
+    // (1 for MSE); both bounds are in the objective's units (zl^2 = zscale^2
+    // lambda) and a candidate is skipped only when its bound exceeds the best
+    // objective beyond the tie band, for every row of the warp.
+    //  - small scales: for s < amax_row / 6 the row's largest value
+    //    saturates, |delta| >= amax_row - 6 s, so E >= lambda (amax_row -
+    //    6 s)^2, growing as s falls;
+    //  - large scales: every |w_i| <= s / 4 encodes to 0 (the tie at 1/4 goes
+    //    to the even code), so E >= lambda sum of those w_i^2, growing as s
+    //    rises.
+    // Each class is walked from its first scale at or above the tile's
+    // largest amax / 6 downwards, then from there upwards.  Rows past the end
+    // and all-zero rows never hold the warp back.
+    const float amax_row = __uint_as_float((upper ? am1 : am0) << 16);
+    const float zl = zscale * sqrtf(lambda);
+    const float zl2 = zl * zl;
     const float row_floor = kZeroFloor * (upper ? pp1 : pp0);
+    const float smax = __uint_as_float(m << 16) * (1.0f / 6.0f);
 
     int jbegin = 0;
     for (int k = 0; k < ncls; ++k) {
@@ -589,8 +621,13 @@ __global__ void __launch_bounds__(kThreads)
         near = near || (step != 0 && ((__float_as_uint(tt) + 2u) & 0x1FFFFFu) <= 4u);
       }
       const bool alt = !kAltSkip || __any_sync(0xFFFFFFFFu, near);
-      // two candidates per step (independent chains), largest scale first
-      for (int j = ci.end - 1; j >= jbegin; j -= 2) {
+      // first candidate of the class at or above smax (scales ascend within a
+      // class; a class has at most 18 candidates)
+      const int jl = jbegin + lane;
+      const uint32_t ge = __ballot_sync(0xFFFFFFFFu, jl < ci.end && cand[jl].s >= smax);
+      const int js = ge ? jbegin + __ffs(ge) - 1 : ci.end - 1;
+      // downwards from js, two candidates per step (independent chains)
+      for (int j = js; j >= jbegin; j -= 2) {
         const CandInfo c0 = cand[j];
         const bool two = j - 1 >= jbegin;
         const CandInfo c1 = cand[two ? j - 1 : j];
@@ -604,25 +641,57 @@ __global__ void __launch_bounds__(kThreads)
         }
         track3(key_of(e0, c0.c), b1, b2, b3);
         if (two) track3(key_of(e1, c1.c), b1, b2, b3);
-        // lower bound at the smaller of the two scales (all later ones are smaller)
-        const float d = zl * fmaf(-6.0f, c1.s, amax_row);
+        // saturation bound at the smaller of the two scales (every later one is smaller)
+        const float d = fmaf(-6.0f, c1.s, amax_row);
         const bool done = amax_row == 0.0f ||
-                          (d > 0.0f && d * d * (1.0f - 2.0f * kTieBand) > b1 + row_floor);
+                          (d > 0.0f && zl2 * d * d * (1.0f - 2.0f * kTieBand) > b1 + row_floor);
         if (__all_sync(0xFFFFFFFFu, done)) break;
+      }
+      // upwards from js + 1
+      for (int j = js + 1; j < ci.end; j += 2) {
+        const CandInfo c0 = cand[j];
+        // zero-code bound at the smaller of the two scales (every later one is larger)
+        const float q4 = 0.25f * c0.s;
+        float ug = 0.0f, ug8 = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float v = a[e] <= q4 ? a[e] : 0.0f;
+          if ((e & 2) == 0) ug = fmaf(v, v, ug);
+          else ug8 = fmaf(v, v, ug8);
+        }
+        ug += __shfl_xor_sync(0xFFFFFFFFu, ug, 1);
+        ug += __shfl_xor_sync(0xFFFFFFFFu, ug, 2);
+        ug8 += __shfl_xor_sync(0xFFFFFFFFu, ug8, 1);
+        ug8 += __shfl_xor_sync(0xFFFFFFFFu, ug8, 2);
+        const bool done = amax_row == 0.0f ||
+                          zl2 * (upper ? ug8 : ug) * (1.0f - 2.0f * kTieBand) > b1 + row_floor;
+        if (__all_sync(0xFFFFFFFFu, done)) break;
+        const bool two = j + 1 < ci.end;
+        const CandInfo c1 = cand[two ? j + 1 : j];
+        float e0, e1;
+        if (alt) {
+          e0 = candidate_objective<kLH, true>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
+          e1 = candidate_objective<kLH, true>(tq, ta, c1.f, c1.s * umul, sgn, bh, bl, pz, upper);
+        } else {
+          e0 = candidate_objective<kLH, false>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
+          e1 = candidate_objective<kLH, false>(tq, ta, c1.f, c1.s * umul, sgn, bh, bl, pz, upper);
+        }
+        track3(key_of(e0, c0.c), b1, b2, b3);
+        if (two) track3(key_of(e1, c1.c), b1, b2, b3);
       }
       jbegin = ci.end;
     }
 
     // lane t = 0 finishes row g, lane t = 2 row g + 8; near ties are
     // re-scored by the whole warp, one row at a time
-    const int64_t r = upper ? rg8 : rg;
-    const bool owner = (t & 1) == 0 && r < R;
+    const int64_t r = row_base + (upper ? i1 : i0);
+    const bool owner = (t & 1) == 0 && (upper ? v1 : v0);
     int code = code_of(b1);
     float obj = b1 / (zscale * zscale);
     int need = 0;  // 1: re-score the best two, 2: re-score every candidate
     if (owner) {
       const float fl = kZeroFloor * (upper ? pp1 : pp0);
-      if (upper ? zero1 : zero0) {  // every candidate scores exactly 0
+      if (amax_row == 0.0f) {  // all-zero row: every candidate scores exactly 0
         code = 1;
         obj = 0.0f;
       } else if (b2 - b1 <= kTieBand * b2 || b1 <= fl) {

@@ -329,6 +329,41 @@ def test_search_degenerate_blocks(nv):
     assert cm[0, 0] == 1
 
 
+def test_search_ragged_rows_mixed_magnitudes(nv):
+    """Every block of a ragged 600-row weight (three row groups, the last one
+    partly padding) whose rows differ in magnitude by up to 10^5, with zero
+    rows, single-spike rows and an outlier calibration channel: rows of very
+    different size share tiles, and the candidate walk must still return the
+    oracle's choice for each."""
+    R, C = 600, 96
+    g = torch.Generator().manual_seed(11)
+    W = torch.randn(R, C, generator=g) * 0.02
+    scale = torch.tensor([1e-3, 0.1, 1.0, 10.0, 100.0])[torch.randint(0, 5, (R,), generator=g)]
+    W = W * scale[:, None]
+    W[7] = 0
+    W[300:310] = 0
+    W[311, :] = 0
+    W[311, 5] = 0.75
+    W[599, 40] = -3.0
+    W = W.to(torch.bfloat16)
+    X = torch.randn(300, C, generator=g)
+    X[:, 17] *= 30.0
+    X = X.to(torch.bfloat16)
+    wu = bf16_bits(W)
+    s_g = nv.global_scale(W.cuda())
+    sg = s_g.item()
+    H = torch.zeros(C // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate(X.cuda(), H)
+    H64 = H.cpu().numpy().astype(np.float64)
+    clh = nv.scale_search_local_hessian(W.cuda(), s_g, H).cpu().numpy()
+    rc, _ = oracle.scale_search_lh(wu, sg, H64)
+    check_search_codes(clh, rc, wu, sg, H64)
+    cm = nv.scale_search_mse(W.cuda(), s_g).cpu().numpy()
+    rc, _ = oracle.scale_search_mse(wu, sg)
+    check_search_codes(cm, rc, wu, sg)
+    assert np.all(cm[7] == 1) and np.all(clh[300:310] == 1)
+
+
 def test_dense_layer_sampled(nv):
     """Dense 4096x4096 workload (the benchmarked configuration): full GPU
     search, 3000 sampled blocks per rule checked against the oracle."""

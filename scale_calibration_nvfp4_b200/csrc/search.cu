@@ -606,51 +606,51 @@ __global__ void __launch_bounds__(kThreads)
     int jbegin = 0;
     for (int k = 0; k < ncls; ++k) {
       const ClassInfo ci = cls[k];
-      // class quotient t and its neighbour across q, per element
+      // class quotient t per element (within one float of q)
       float tq[8], ta[8];
       bool near = false;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float tt = fmaf(a[e], ci.r_hi, a[e] * ci.r_lo);
-        const float rho = fmaf(-tt, ci.S, a[e]);
-        const int step = (rho > 0.0f) - (rho < 0.0f);
-        tq[e] = tt;
-        ta[e] = __int_as_float(__float_as_int(tt) + step);
+        tq[e] = fmaf(a[e], ci.r_hi, a[e] * ci.r_lo);
         // t within two floats of a value whose low 21 mantissa bits are zero
-        // (every rounding midpoint times a power of two is one), and not exact
-        near = near || (step != 0 && ((__float_as_uint(tt) + 2u) & 0x1FFFFFu) <= 4u);
+        // (every rounding midpoint times a power of two is one)
+        near = near || ((__float_as_uint(tq[e]) + 2u) & 0x1FFFFFu) <= 4u;
       }
       const bool alt = !kAltSkip || __any_sync(0xFFFFFFFFu, near);
+      if (alt) {
+        // the neighbouring float of t on the other side of q, by the exact
+        // sign of the residual |w| - t S (t itself when exact)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float rho = fmaf(-tq[e], ci.S, a[e]);
+          const int step = (rho > 0.0f) - (rho < 0.0f);
+          ta[e] = __int_as_float(__float_as_int(tq[e]) + step);
+        }
+      }
       // first candidate of the class at or above smax (scales ascend within a
       // class; a class has at most 18 candidates)
       const int jl = jbegin + lane;
       const uint32_t ge = __ballot_sync(0xFFFFFFFFu, jl < ci.end && cand[jl].s >= smax);
       const int js = ge ? jbegin + __ffs(ge) - 1 : ci.end - 1;
-      // downwards from js, two candidates per step (independent chains)
-      for (int j = js; j >= jbegin; j -= 2) {
+      // downwards from js (scales halve at every step of a class)
+      for (int j = js; j >= jbegin; --j) {
         const CandInfo c0 = cand[j];
-        const bool two = j - 1 >= jbegin;
-        const CandInfo c1 = cand[two ? j - 1 : j];
-        float e0, e1;
-        if (alt) {
-          e0 = candidate_objective<kLH, true>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
-          e1 = candidate_objective<kLH, true>(tq, ta, c1.f, c1.s * umul, sgn, bh, bl, pz, upper);
-        } else {
-          e0 = candidate_objective<kLH, false>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
-          e1 = candidate_objective<kLH, false>(tq, ta, c1.f, c1.s * umul, sgn, bh, bl, pz, upper);
+        if (j < js) {
+          // saturation bound at this scale (every later one is smaller)
+          const float d = fmaf(-6.0f, c0.s, amax_row);
+          const bool done = amax_row == 0.0f ||
+                            (d > 0.0f && zl2 * d * d * (1.0f - 2.0f * kTieBand) > b1 + row_floor);
+          if (__all_sync(0xFFFFFFFFu, done)) break;
         }
+        const float e0 =
+            alt ? candidate_objective<kLH, true>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper)
+                : candidate_objective<kLH, false>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
         track3(key_of(e0, c0.c), b1, b2, b3);
-        if (two) track3(key_of(e1, c1.c), b1, b2, b3);
-        // saturation bound at the smaller of the two scales (every later one is smaller)
-        const float d = fmaf(-6.0f, c1.s, amax_row);
-        const bool done = amax_row == 0.0f ||
-                          (d > 0.0f && zl2 * d * d * (1.0f - 2.0f * kTieBand) > b1 + row_floor);
-        if (__all_sync(0xFFFFFFFFu, done)) break;
       }
       // upwards from js + 1
-      for (int j = js + 1; j < ci.end; j += 2) {
+      for (int j = js + 1; j < ci.end; ++j) {
         const CandInfo c0 = cand[j];
-        // zero-code bound at the smaller of the two scales (every later one is larger)
+        // zero-code bound at this scale (every later one is larger)
         const float q4 = 0.25f * c0.s;
         float ug = 0.0f, ug8 = 0.0f;
 #pragma unroll
@@ -666,18 +666,10 @@ __global__ void __launch_bounds__(kThreads)
         const bool done = amax_row == 0.0f ||
                           zl2 * (upper ? ug8 : ug) * (1.0f - 2.0f * kTieBand) > b1 + row_floor;
         if (__all_sync(0xFFFFFFFFu, done)) break;
-        const bool two = j + 1 < ci.end;
-        const CandInfo c1 = cand[two ? j + 1 : j];
-        float e0, e1;
-        if (alt) {
-          e0 = candidate_objective<kLH, true>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
-          e1 = candidate_objective<kLH, true>(tq, ta, c1.f, c1.s * umul, sgn, bh, bl, pz, upper);
-        } else {
-          e0 = candidate_objective<kLH, false>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
-          e1 = candidate_objective<kLH, false>(tq, ta, c1.f, c1.s * umul, sgn, bh, bl, pz, upper);
-        }
+        const float e0 =
+            alt ? candidate_objective<kLH, true>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper)
+                : candidate_objective<kLH, false>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
         track3(key_of(e0, c0.c), b1, b2, b3);
-        if (two) track3(key_of(e1, c1.c), b1, b2, b3);
       }
       jbegin = ci.end;
     }

@@ -54,7 +54,7 @@ WORKLOAD_NAMES = ["dense", "tiny", "moe", "mlp_pair", "w4a4"]
 # Local-Hessian search work per block, counted on the definition E = delta
 # H_b delta^T: per candidate 256 FMA for H_b delta and 16 FMA for the dot
 # product, 2 flop each (the E2M1 encodes are not counted as flops).
-LH_FLOP_PER_BLOCK = 126 * 2 * (256 + 16)
+LH_FLOP_PER_EVAL = 2 * (256 + 16)  # delta H_b delta^T for one candidate
 # bytes per activation element of the fused fake-quant with packed outputs:
 # amax pass 2, fused pass 2 read + 2 write + 0.5 packed + 1/16 block codes
 FAKE_QUANT_BYTES_PER_ELEM = 2 + 2 + 2 + 0.5 + 1 / 16
@@ -174,7 +174,7 @@ class Runner:
                              2 * n_w + nb, 1))
             rows.append((pre + "search_lh",
                          lambda L=L: nv.scale_search_local_hessian(L.W, L.s_g, L.H, out=L.c_lh),
-                         2 * n_w + nb + h, 1))
+                         2 * n_w + nb + h, 2))  # factor_kernel + search_kernel
             rows.append((pre + "quantize_pack",
                          lambda L=L: nv.quantize_pack(L.W, L.s_g, L.c_lh, out=L.packed),
                          2 * n_w + nb + n_w // 2, 1))
@@ -290,10 +290,18 @@ def peaks():
     return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0}, "fallback"
 
 
-def kernel_source_hash():
+# source files each reported kernel is built from
+KERNEL_SOURCES = {
+    "search_lh": ("search.cu", "common.cuh"),
+    "fake_quant": ("quant.cu", "common.cuh"),
+    "gram": ("gram.cu", "common.cuh"),
+}
+
+
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "scale_calibration_nvfp4_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -302,14 +310,14 @@ def kernel_source_hash():
 
 def recorded_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources."""
+    the current sources of that kernel."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
     ent = t.get(kernel, {}).get(workload)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -379,7 +387,7 @@ def run_gpu(args):
         time.sleep(0.3)
     if pg:
         pg.barrier()
-    torch.cuda.synchronize()
+    nvfp4.search_evaluations(reset=True)  # synchronises
     for k in range(args.steps):
         flush.zero_()
         step(ev[k])
@@ -387,6 +395,8 @@ def run_gpu(args):
     if pg:
         pg.barrier()
     clk = clocks.stop() if clocks else None
+    # (block, candidate) evaluations the searches made per step
+    evals = [v / args.steps for v in nvfp4.search_evaluations(reset=True)]
 
     per_row = {r[0]: [] for r in rows}
     step_ms = []
@@ -418,7 +428,9 @@ def run_gpu(args):
                        "rows": [r[0] for r in rows],
                        "parallelism": "replicas (one per GPU)" if world > 1 else "single GPU",
                        "cache": "L2 flushed (256 MiB write) before every timed step"},
-            "roofline": make_roofline(run, kernels, pk, pk_kind, args.workload),
+            "roofline": make_roofline(run, kernels, pk, pk_kind, args.workload, evals[1]),
+            "search_evaluated_per_block": {"mse": round(evals[0] / blocks, 2),
+                                           "local_hessian": round(evals[1] / blocks, 2)},
             "kernels": kernels,
             "gpu_launches": args.steps * run.launches(),
             "clocks": clk,
@@ -432,13 +444,16 @@ def run_gpu(args):
         pg.destroy_process_group()
 
 
-def make_roofline(run, kernels, pk, pk_kind, workload):
+def make_roofline(run, kernels, pk, pk_kind, workload, lh_evals):
     lh_rows = [k for k in kernels if k.endswith("search_lh")]
     if lh_rows:
         lh_ms = sum(kernels[k]["ms"] for k in lh_rows)
         sm_mhz = float(pk.get("sm_max_mhz", 1965.0))
         fp32_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
-        achieved = LH_FLOP_PER_BLOCK * run.blocks() / (lh_ms / 1e3) / 1e12
+        # the definition's cost of every candidate the exact pruned walk
+        # evaluates (counted on the device); the skipped ones provably lose
+        achieved = LH_FLOP_PER_EVAL * lh_evals / (lh_ms / 1e3) / 1e12
+        brute = LH_FLOP_PER_EVAL * 126 * run.blocks() / (lh_ms / 1e3) / 1e12
         return {
             "kernel": "search_kernel<Local-Hessian>",
             "bound": "alu", "achieved": round(achieved, 2), "peak": round(fp32_peak, 2),
@@ -446,8 +461,10 @@ def make_roofline(run, kernels, pk, pk_kind, workload):
             "traffic": recorded_traffic("search_lh", workload),
             "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 flop x %.0f MHz (%s clocks)"
                          % (sm_mhz, pk_kind),
-            "flop_basis": "definition delta H_b delta^T: 126 x (256 + 16) FMA per block",
-            "flop_per_block": LH_FLOP_PER_BLOCK,
+            "flop_basis": "definition delta H_b delta^T, (256 + 16) FMA = 544 flop per "
+                          "(block, candidate) evaluated; evaluations counted on the device",
+            "evaluated_per_block": round(lh_evals / run.blocks(), 2),
+            "all_126_equivalent_TFLOP/s": round(brute, 2),
         }
     ms = kernels["fake_quant"]["ms"]
     n = run.fq_input.numel()

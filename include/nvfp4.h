@@ -40,7 +40,7 @@
  *     contiguous batch stride; each has its own FP32 scale s_g[batch].
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
  *     enqueue work on it and return without synchronising, except
- *     nvfp4_get_device_status.  Argument errors are detected on the host
+ *     nvfp4_get_device_status and nvfp4_search_evaluations.  Argument errors are detected on the host
  *     before anything is enqueued; a failed launch returns NVFP4_ERR_CUDA.
  *   - A CUDA device must be current; all pointers must belong to it.
  *
@@ -68,7 +68,10 @@ typedef enum nvfp4_status {
     NVFP4_ERR_NONFINITE = 4,       /* NaN or Inf met in an input (device-side report) */
     NVFP4_ERR_CUDA = 5,            /* a CUDA runtime call or launch failed */
     NVFP4_ERR_NOT_IMPLEMENTED = 6,
-    NVFP4_ERR_TOO_LARGE = 7        /* request beyond a documented maximum */
+    NVFP4_ERR_TOO_LARGE = 7,       /* request beyond a documented maximum */
+    NVFP4_ERR_DEVICE_TIMEOUT = 8   /* a kernel gave up waiting (one second) for its own
+                                      tile copies; its output was not written
+                                      (device-side report) */
 } nvfp4_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -130,6 +133,8 @@ nvfp4_status nvfp4_hessian_accumulate_noalloc(const uint16_t *x, int64_t n_tok, 
  *             device value has to be read back).  Offsets outside
  *             [0, n_tok_total] are clamped on the device.
  *   H         [G, C/16, 16, 16] float, accumulated.
+ * n_tok_total above 2^30 returns NVFP4_ERR_TOO_LARGE (tile row coordinates
+ * of the tile copies are 32-bit; split such a set into calls).
  */
 nvfp4_status nvfp4_hessian_accumulate_grouped(const uint16_t *x, const int64_t *offsets,
                                               int64_t G, int64_t n_tok_total, int64_t C,
@@ -209,10 +214,24 @@ nvfp4_status nvfp4_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16
 
 /*
  * Reads and clears the device-side status of the current device after
- * synchronising `stream` (the only call that blocks the host).  *out is
- * NVFP4_OK or NVFP4_ERR_NONFINITE.
+ * synchronising `stream`.  *out is NVFP4_OK, NVFP4_ERR_NONFINITE or
+ * NVFP4_ERR_DEVICE_TIMEOUT (the first one set, if several are).
  */
 nvfp4_status nvfp4_get_device_status(void *stream, nvfp4_status *out);
+
+/*
+ * Work statistic of the scale searches (the pages have no counterpart; it
+ * measures how much of the 126-candidate search the exact pruning leaves):
+ * out[0] and out[1] receive the number of (block, candidate) objective
+ * evaluations of the fp32 screen made by nvfp4_scale_search_mse and by
+ * nvfp4_scale_search_local_hessian on the current device since the last
+ * reset (the fp64 re-scores of near ties are not counted); between 1 and 126
+ * per block searched.  Synchronises `stream` first, so calls queued on it
+ * are included; calls still running on other streams may be partly
+ * included.  `reset` != 0 zeroes both counters afterwards.
+ *   out   [2] uint64, HOST, written
+ */
+nvfp4_status nvfp4_search_evaluations(void *stream, int reset, uint64_t *out);
 
 /* Releases the library's memory pool on every device it touched.  No call
  * may be in flight. */

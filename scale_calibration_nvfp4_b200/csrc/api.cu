@@ -111,6 +111,7 @@ const char *nvfp4_status_string(nvfp4_status st) {
     case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
     case NVFP4_ERR_NOT_IMPLEMENTED: return "NVFP4_ERR_NOT_IMPLEMENTED";
     case NVFP4_ERR_TOO_LARGE: return "NVFP4_ERR_TOO_LARGE";
+    case NVFP4_ERR_DEVICE_TIMEOUT: return "NVFP4_ERR_DEVICE_TIMEOUT";
   }
   return "NVFP4_ERR_UNKNOWN";
 }
@@ -149,7 +150,8 @@ nvfp4_status nvfp4_hessian_accumulate_grouped(const uint16_t *x, const int64_t *
   if (G < 1 || n_tok_total < 0 || C < 0 || !H || !offsets || (n_tok_total > 0 && !x))
     return NVFP4_ERR_INVALID_ARG;
   if (C % 16 || !fits(n_tok_total, C) || !fits(G, C, 16)) return NVFP4_ERR_SHAPE;
-  if (C / 16 > 8 * 65535 || n_tok_total / 2048 + G > INT32_MAX) return NVFP4_ERR_TOO_LARGE;
+  if (C / 16 > 8 * 65535 || n_tok_total > ((int64_t)1 << 30) || n_tok_total / 2048 + G > INT32_MAX)
+    return NVFP4_ERR_TOO_LARGE;
   if ((x && !aligned(x, 16)) || !aligned(H, 4) || !aligned(offsets, 8))
     return NVFP4_ERR_MISALIGNED;
   return map_cuda(nvfp4::launch_gram(x, offsets, G, n_tok_total, C, H, as_stream(stream)));
@@ -225,6 +227,16 @@ nvfp4_status nvfp4_get_device_status(void *stream, nvfp4_status *out) {
   cudaError_t e = nvfp4::read_and_clear_device_status(as_stream(stream), &v);
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   *out = (nvfp4_status)v;
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_search_evaluations(void *stream, int reset, uint64_t *out) {
+  if (!out) return NVFP4_ERR_INVALID_ARG;
+  unsigned long long v[2] = {0, 0};
+  cudaError_t e = nvfp4::read_search_evaluations(as_stream(stream), v, reset != 0);
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  out[0] = v[0];
+  out[1] = v[1];
   return NVFP4_OK;
 }
 

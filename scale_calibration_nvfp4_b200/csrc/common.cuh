@@ -31,17 +31,6 @@ __device__ __forceinline__ float e4m3_to_float(uint32_t c) {
 }
 
 // ---------------------------------------------------------- hardware cvt
-// Two fp32 -> two E2M1 codes in one byte (round to nearest even, saturating
-// at +-6).  `hi` lands in bits 7..4, `lo` in bits 3..0.
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q0, %1, %2;\n\t"
-      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
-      : "=r"(r) : "f"(hi), "f"(lo));
-  return r & 0xFFu;
-}
-
 // One byte of two E2M1 codes -> f16x2 (low nibble in the low half).
 __device__ __forceinline__ uint32_t cvt_f16x2_from_e2m1x2(uint32_t byte) {
   uint32_t r;
@@ -78,56 +67,28 @@ __device__ __forceinline__ uint32_t e2m1_mag_exact(float a, float s) {
   return k;
 }
 
-// Reciprocal bracket of a scale: r_lo <= 1/s <= r_hi.
-struct ScaleRecip {
-  float s, r_lo, r_hi;
-};
-
-__device__ __forceinline__ ScaleRecip make_recip(float s) {
-  ScaleRecip r;
-  r.s = s;
-  r.r_lo = __frcp_rd(s);
-  r.r_hi = __frcp_ru(s);
-  return r;
-}
-
-// Packed magnitude codes of 2 elements (a0 -> low nibble, a1 -> high) from
-// the reciprocal bracket: t_lo <= |x|/s <= t_hi elementwise, rounding is
-// monotone, so equal codes at both ends are the exact answer.  `mismatch`
-// accumulates any disagreement (then the caller redoes the block exactly).
-__device__ __forceinline__ uint32_t e2m1_pair_bracket(float a0, float a1, const ScaleRecip &r,
-                                                      uint32_t &mismatch) {
-  uint32_t lo = cvt_e2m1x2(__fmul_rd(a1, r.r_lo), __fmul_rd(a0, r.r_lo));
-  uint32_t hi = cvt_e2m1x2(__fmul_ru(a1, r.r_hi), __fmul_ru(a0, r.r_hi));
-  mismatch |= lo ^ hi;
-  return lo;
-}
-
-// ------------------------------------------------------ exact E4M3 round
-// E4M3 code (0..126) of num / den rounded to nearest even, saturating at 448,
-// for num >= 0, den > 0 given as fp64 values whose exact quotient is at
-// least 2^-32 (relative) away from every E4M3 midpoint unless equal to it
-// (true for num a bf16 value and den = 6 * s_g, s_g an fp32 value).  The
-// fp64 quotient then sits on the same side of every midpoint as the exact
-// one, and the rounding below is exact arithmetic on it.
-__device__ __forceinline__ uint32_t e4m3_round_quotient(double num, double den) {
-  double q = __ddiv_rn(num, den);
-  if (!(q < 448.0)) return 0x7Eu;            // saturate (also catches +inf)
-  if (q < 0.015625) {                        // below 2^-6: subnormal grid m * 2^-9
-    return (uint32_t)rint(q * 512.0);        // 0..8; 8 is the first normal code
+// Certificate that plain rounding of a quotient is exact.  For s >= 2^-100
+// finite and every bf16 value x, t = fl(x (r_hi + r_lo)) with r_hi + r_lo =
+// 1/s to about 2^-46 lies within one float of q = x / s.  Hardware
+// round-to-nearest-even of t can then differ from that of q only if an E2M1
+// rounding midpoint (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5: at most three
+// significant bits), times a power of two, lies within one float of q.  x
+// has at most 8 significant bits, so q = x / s sits within relative 2^-21 of
+// m 2^k (m = 1, 3, 5, 7) only if m s sits within relative 2^-21 of a number
+// with 8 significant bits.  Returns true when that holds for no m: no value
+// at scale s comes near a midpoint.  m s is exact in fp64; its significand
+// bits below the eighth must stay more than 2^-20 (in units of the leading
+// bit, i.e. 2^32 units of 2^-52) away from 0 and from 1.
+__device__ __forceinline__ bool quotients_far_from_midpoints(float s) {
+  bool far = true;
+#pragma unroll
+  for (int m = 1; m <= 7; m += 2) {
+    const double p = (double)s * (double)m;
+    const unsigned long long rem =
+        (unsigned long long)__double_as_longlong(p) & ((1ull << 45) - 1ull);
+    far = far && rem > (1ull << 32) && rem < (1ull << 45) - (1ull << 32);
   }
-  int e;
-  double m = frexp(q, &e);                   // q = m * 2^e, m in [0.5, 1)
-  // q = (1 + f/8) * 2^(e-1) with f = (2m - 1) * 8 in [0, 8); round f to even
-  double f = rint((2.0 * m - 1.0) * 8.0);    // 0..8, 8 carries into the exponent
-  uint32_t code = (uint32_t)(((e - 1 + 7) << 3) + (int)f);
-  return code > 0x7Eu ? 0x7Eu : code;
-}
-
-// Max rule: code of block amax a_max given s_g (exact decision).
-__device__ __forceinline__ uint32_t max_rule_code(float a_max, float s_g) {
-  if (a_max == 0.0f) return 0u;
-  return e4m3_round_quotient((double)a_max, 6.0 * (double)s_g);
+  return far;
 }
 
 __device__ __forceinline__ float effective_scale(float s_g, uint32_t code) {

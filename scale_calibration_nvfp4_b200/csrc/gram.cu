@@ -5,47 +5,101 @@
 //
 // Data path: a CTA owns a group of up to 8 column blocks (128 channels) and a
 // range of tokens.  Token tiles [64 tokens x 128 channels] of bf16 stream from
-// HBM into shared memory through a 4-stage cp.async pipeline; rows are padded
-// to 272 bytes so the transposing ldmatrix reads are bank-conflict free.
-// Warp w owns column block w of the group: per 16 tokens one ldmatrix.x4.trans
+// HBM into shared memory by the tensor-memory accelerator: one thread issues
+// two 2-D tile copies (64 x 64 bf16 each, 128-byte swizzle) per stage into a
+// 4-stage ring, completion is tracked by one mbarrier per stage, and no other
+// thread computes an address.  Warp w owns column block w of the group: per
+// 16 tokens one ldmatrix.x4.trans (through the swizzle, bank-conflict free)
 // yields X_j^T as the A fragment of a 16x8x16 bf16 MMA, and the same four
 // registers are the B fragments of the two 8-channel halves, so the 16x16
 // block comes from two MMAs with no wasted product (bf16 x bf16 products are
 // exact in fp32, sums are fp32).  Each CTA writes its fp32 partial block to a
-// stream-ordered scratch buffer; a second kernel adds the partials of a group
-// to H in a fixed order, so the result does not depend on scheduling.
+// scratch buffer; a second kernel adds the partials of a group to H in a
+// fixed order, so the result does not depend on scheduling.
+//
+// Every wait on an mbarrier is bounded (one second of %globaltimer): on
+// expiry the CTA records NVFP4_ERR_DEVICE_TIMEOUT in this file's device
+// status, waits (bounded again) for its own copies still in flight, writes
+// nothing and returns.
+#include <algorithm>
 #include <mutex>
+
+#include <cuda.h>
 
 #include "common.cuh"
 #include "internal.h"
+#include "../../include/nvfp4.h"
 
 namespace nvfp4 {
+
+// Sticky device status of the Gram kernels (NVFP4_OK or
+// NVFP4_ERR_DEVICE_TIMEOUT), read and cleared with the library status.
+__device__ int g_gram_status = 0;
+
 namespace {
 
 constexpr int kGramThreads = 256;             // 8 warps
 constexpr int kGroupBlocks = 8;               // column blocks per CTA
 constexpr int kTileTok = 64;                  // tokens per pipeline stage
 constexpr int kStages = 4;
-constexpr int kRowBytes = 128 * 2 + 16;       // padded smem row
-constexpr int kStageBytes = kTileTok * kRowBytes;
-constexpr int kGramSmem = kStages * kStageBytes;  // 69,632 bytes
+constexpr int kBoxCols = 64;                  // channels per tile copy (128 bytes)
+constexpr int kBoxBytes = kTileTok * kBoxCols * 2;  // 8 KiB
+constexpr int kStageBytes = 2 * kBoxBytes;          // 16 KiB
+constexpr int kGramSmem = kStages * kStageBytes + 1024;  // + alignment slack
 constexpr int64_t kGroupedItemTokens = 2048;  // tokens per work item, grouped form
+constexpr int64_t kMaxTokensPerLaunch = (int64_t)1 << 30;  // tile row coordinates fit int32
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 struct ItemRange {
   int64_t group, t_begin, t_end;
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
+
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
 }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+
+// Wait for phase `parity` of an mbarrier, for at most kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_test(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (!mbar_test(bar, parity)) {
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+// One 64 x 64 bf16 tile (channels x0.., tokens y0..) into shared memory,
+// completing on `bar`.  Rows past the tensor's end arrive as zeros.
+__device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap *tmap, int x0,
+                                              int y0, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x0), "r"(y0), "r"(bar)
+      : "memory");
 }
 
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t r[4]) {
@@ -61,6 +115,11 @@ __device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], 
       "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// bf16 pair of tokens (tok, tok + 1) kept only where the token is below n.
+__device__ __forceinline__ uint32_t keep_tokens(uint32_t pair, int tok, int n) {
+  return pair & ((tok < n ? 0x0000FFFFu : 0u) | (tok + 1 < n ? 0xFFFF0000u : 0u));
 }
 
 // Work item -> (group, token range).  Uniform split of one group when
@@ -79,69 +138,99 @@ __device__ __forceinline__ bool item_range(int64_t item, const ItemRange *items,
   return out.t_begin < out.t_end;
 }
 
+// `tmap`: X as a 2-D bf16 tensor [n_tok rows, C columns], 64 x 64 boxes,
+// 128-byte swizzle, zero fill past the end.
 __global__ void __launch_bounds__(kGramThreads)
-    gram_partial_kernel(const uint16_t *__restrict__ x, int64_t C, const ItemRange *items,
-                        const int64_t *n_items_dev, int64_t n_tok, int64_t per_item,
-                        float *__restrict__ partial) {
-  extern __shared__ __align__(128) unsigned char smem[];
+    gram_partial_kernel(const __grid_constant__ CUtensorMap tmap, int64_t C,
+                        const ItemRange *items, const int64_t *n_items_dev, int64_t n_tok,
+                        int64_t per_item, float *__restrict__ partial) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t full[kStages];
   const int64_t nb = C / kBlock;
   const int64_t item = blockIdx.x;
   const int64_t cg = blockIdx.y;
   ItemRange ir;
   if (!item_range(item, items, n_items_dev, n_tok, per_item, ir)) return;
   const int width = (int)min((int64_t)kGroupBlocks, nb - cg * kGroupBlocks);  // column blocks
-  const int chunks_per_row = width * 2;                                        // 16 B chunks
-  const int64_t ntiles = (ir.t_end - ir.t_begin + kTileTok - 1) / kTileTok;
-  const uint16_t *xbase = x + cg * kGroupBlocks * kBlock;
-  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+  const int ntiles = (int)((ir.t_end - ir.t_begin + kTileTok - 1) / kTileTok);
+  // 1024-byte aligned ring (the swizzle pattern repeats every 1024 bytes)
+  const uint32_t sraw = (uint32_t)__cvta_generic_to_shared(smem_raw);
+  const uint32_t sbase = (sraw + 1023u) & ~1023u;
+  const uint32_t bar0 = (uint32_t)__cvta_generic_to_shared(&full[0]);
+  const int x0 = (int)(cg * kGroupBlocks * kBlock);
 
-  auto load_tile = [&](int64_t tile, int stage) {
-    const int64_t t0 = ir.t_begin + tile * kTileTok;
-    const int total = kTileTok * chunks_per_row;
-    for (int i = threadIdx.x; i < total; i += kGramThreads) {
-      const int row = i / chunks_per_row;
-      const int ch = i - row * chunks_per_row;
-      const int64_t t = t0 + row;
-      const bool valid = t < ir.t_end;
-      const uint16_t *src = valid ? xbase + t * C + ch * 8 : xbase;
-      cp_async16(sbase + stage * kStageBytes + row * kRowBytes + ch * 16, src, valid ? 16u : 0u);
-    }
+  auto issue = [&](int tile, int stage) {
+    const uint32_t bar = bar0 + 8u * stage;
+    const int y0 = (int)(ir.t_begin + (int64_t)tile * kTileTok);
+    mbar_expect_tx(bar, kStageBytes);
+    tma_load_tile(sbase + stage * kStageBytes, &tmap, x0, y0, bar);
+    tma_load_tile(sbase + stage * kStageBytes + kBoxBytes, &tmap, x0 + kBoxCols, y0, bar);
   };
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-  // ldmatrix row address of this lane inside a 16-token step
-  const int lrow = (lane & 7) + ((lane >> 4) & 1) * 8;
-  const int lcol = warp * 32 + ((lane >> 3) & 1) * 16;
-
-#pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
-    if (s < ntiles) load_tile(s, s);
-    cp_async_commit();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8u * s, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  for (int64_t tile = 0; tile < ntiles; ++tile) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    const int64_t next = tile + kStages - 1;
-    if (next < ntiles) load_tile(next, (int)(next % kStages));
-    cp_async_commit();
-    if (warp < width) {
-      const uint32_t st = sbase + (uint32_t)(tile % kStages) * kStageBytes;
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int s = 0; s < kStages && s < ntiles; ++s) issue(s, s);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = lane & 3;
+  float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+  // ldmatrix rows of this lane inside a 16-token step, and its 16-byte chunk
+  // of the 128-byte row (channel block warp & 3 of box warp >> 2), swizzled
+  const int lrow = (lane & 7) + ((lane >> 4) & 1) * 8;
+  const uint32_t chunk = (uint32_t)(((warp & 3) * 2 + ((lane >> 3) & 1)) ^ (lane & 7));
+  const uint32_t lane_off = (uint32_t)(warp >> 2) * kBoxBytes + (uint32_t)lrow * 128u + chunk * 16u;
+
+  bool timed_out = false;
+  int tile = 0;
+  for (; tile < ntiles; ++tile) {
+    const int stage = tile % kStages;
+    const bool ok = mbar_wait_bounded(bar0 + 8u * stage, (uint32_t)(tile / kStages) & 1u);
+    if (ok && warp < width) {
+      const uint32_t st = sbase + (uint32_t)stage * kStageBytes + lane_off;
+      // tokens of this tile that belong to the item (the last tile of a
+      // grouped item may run into the next group)
+      const int nvalid = (int)min((int64_t)kTileTok, ir.t_end - ir.t_begin - (int64_t)tile * kTileTok);
 #pragma unroll
       for (int k = 0; k < kTileTok / 16; ++k) {
         uint32_t a[4];
-        ldmatrix_x4_trans(st + (k * 16 + lrow) * kRowBytes + lcol, a);
+        ldmatrix_x4_trans(st + k * 16 * 128, a);
+        if (nvalid < kTileTok) {
+          a[0] = keep_tokens(a[0], k * 16 + 2 * t, nvalid);
+          a[1] = keep_tokens(a[1], k * 16 + 2 * t, nvalid);
+          a[2] = keep_tokens(a[2], k * 16 + 8 + 2 * t, nvalid);
+          a[3] = keep_tokens(a[3], k * 16 + 8 + 2 * t, nvalid);
+        }
         mma_bf16_16816(d0, a, a[0], a[2]);
         mma_bf16_16816(d1, a, a[1], a[3]);
       }
     }
+    // every thread is done with the stage (and agrees on a timeout) before
+    // it is refilled
+    if (__syncthreads_or(!ok)) {
+      timed_out = true;
+      break;
+    }
+    if (threadIdx.x == 0 && tile + kStages < ntiles) issue(tile + kStages, stage);
   }
-  cp_async_wait<0>();
+
+  if (timed_out) {
+    if (threadIdx.x == 0) atomicExch(&g_gram_status, (int)NVFP4_ERR_DEVICE_TIMEOUT);
+    // copies still in flight land in this CTA's shared memory: wait for them
+    // (bounded) before leaving
+    for (int u = tile; u < ntiles && u < tile + kStages; ++u)
+      mbar_wait_bounded(bar0 + 8u * (u % kStages), (uint32_t)(u / kStages) & 1u);
+    return;
+  }
 
   if (warp < width) {
     const int64_t j = cg * kGroupBlocks + warp;
     float *P = partial + (item * nb + j) * 256;
-    const int g = lane >> 2, t = lane & 3;
+    const int g = lane >> 2;
     P[g * 16 + 2 * t] = d0[0];
     P[g * 16 + 2 * t + 1] = d0[1];
     P[(g + 8) * 16 + 2 * t] = d0[2];
@@ -239,6 +328,39 @@ __global__ void build_items_kernel(const int64_t *__restrict__ offsets, int64_t 
 constexpr int kMaxDevices = 64;
 bool g_smem_attr_set[kMaxDevices] = {};
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (no link-time dependency on the driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+// X [n_rows, C] bf16 (row stride C elements) as 64 x 64 tiles, 128-byte
+// swizzle, zeros past the end.  The caller has checked that x is 16-byte
+// aligned and C a multiple of 16 (so the row stride is a multiple of 32 bytes).
+cudaError_t make_x_tensor_map(const uint16_t *x, int64_t n_rows, int64_t C, CUtensorMap *out) {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (!g_encode) return cudaErrorNotSupported;
+  const cuuint64_t gdim[2] = {(cuuint64_t)C, (cuuint64_t)n_rows};
+  const cuuint64_t gstride[1] = {(cuuint64_t)C * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kBoxCols, (cuuint32_t)kTileTok};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = g_encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                             const_cast<uint16_t *>(x), gdim, gstride, box, estride,
+                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t ensure_smem_attr() {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -269,6 +391,25 @@ void uniform_items(int64_t n_tok, int64_t ngroups, int64_t cap, int64_t *items_o
   *per_item_out = per_item;
 }
 
+// One uniform split over n_tok tokens (fewer than 2^30): `items` partials of
+// `per_item` tokens into `partial`, then their fixed-order sum into H.
+cudaError_t gram_uniform(const uint16_t *x, int64_t n_tok, int64_t C, float *H, float *partial,
+                         int64_t items, int64_t per_item, cudaStream_t st) {
+  const int64_t nb = C / kBlock;
+  const int64_t ngroups = (nb + kGroupBlocks - 1) / kGroupBlocks;
+  const int64_t per_group = nb * 256;
+  CUtensorMap tmap;
+  cudaError_t e = make_x_tensor_map(x, n_tok, C, &tmap);
+  if (e != cudaSuccess) return e;
+  gram_partial_kernel<<<dim3((unsigned)items, (unsigned)ngroups), kGramThreads, kGramSmem, st>>>(
+      tmap, C, nullptr, nullptr, n_tok, per_item, partial);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  gram_reduce_kernel<<<(unsigned)((per_group + 255) / 256), 256, 0, st>>>(partial, nb, 1, nullptr,
+                                                                          items, H);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, int64_t n_tok,
@@ -281,24 +422,26 @@ cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, in
   const int64_t per_group = nb * 256;
 
   if (!offsets) {
-    int64_t items, per_item;
-    uniform_items(n_tok, ngroups, INT64_MAX, &items, &per_item);
-    float *partial = nullptr;
-    e = scratch_alloc((void **)&partial, sizeof(float) * items * per_group, st);
-    if (e != cudaSuccess) return e;
-    gram_partial_kernel<<<dim3((unsigned)items, (unsigned)ngroups), kGramThreads, kGramSmem, st>>>(
-        x, C, nullptr, nullptr, n_tok, per_item, partial);
-    e = cudaGetLastError();
-    if (e == cudaSuccess) {
-      const int64_t n = per_group;
-      gram_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, nb, 1, nullptr,
-                                                                      items, H);
-      e = cudaGetLastError();
+    // token chunks of at most 2^30 (tile row coordinates are 32-bit)
+    for (int64_t t0 = 0; t0 < n_tok; t0 += kMaxTokensPerLaunch) {
+      const int64_t n = std::min(kMaxTokensPerLaunch, n_tok - t0);
+      int64_t items, per_item;
+      uniform_items(n, ngroups, INT64_MAX, &items, &per_item);
+      float *partial = nullptr;
+      e = scratch_alloc((void **)&partial, sizeof(float) * items * per_group, st);
+      if (e != cudaSuccess) return e;
+      e = gram_uniform(x + t0 * C, n, C, H, partial, items, per_item, st);
+      const cudaError_t e2 = scratch_free(partial, st);
+      if (e == cudaSuccess) e = e2;
+      if (e != cudaSuccess) return e;
     }
-    cudaError_t e2 = scratch_free(partial, st);
-    return e != cudaSuccess ? e : e2;
+    return cudaSuccess;
   }
 
+  if (n_tok > kMaxTokensPerLaunch) return cudaErrorInvalidValue;
+  CUtensorMap tmap;
+  e = make_x_tensor_map(x, n_tok, C, &tmap);
+  if (e != cudaSuccess) return e;
   const int64_t per_item = kGroupedItemTokens;
   const int64_t max_items = n_tok / per_item + G;
   // scratch layout: item_start [G+1] | n_items [1] | items [max_items] | partials
@@ -317,7 +460,7 @@ cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, in
   e = cudaGetLastError();
   if (e == cudaSuccess) {
     gram_partial_kernel<<<dim3((unsigned)max_items, (unsigned)ngroups), kGramThreads, kGramSmem,
-                          st>>>(x, C, items, n_items, n_tok, per_item, partial);
+                          st>>>(tmap, C, items, n_items, n_tok, per_item, partial);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) {
@@ -328,6 +471,20 @@ cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, in
   }
   cudaError_t e2 = scratch_free(ws, st);
   return e != cudaSuccess ? e : e2;
+}
+
+cudaError_t read_and_clear_gram_status(cudaStream_t st, int *out) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_gram_status, sizeof(int), 0,
+                                            cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return e;
+  if (*out != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_gram_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  }
+  return e;
 }
 
 // ---------------------------------------------------------------------------
@@ -392,15 +549,14 @@ cudaError_t launch_gram_noalloc(const uint16_t *x, int64_t n_tok, int64_t C, flo
   e = noalloc_partials(&partial);
   if (e != cudaSuccess) return e;
   const int64_t ngroups = (nb + kGroupBlocks - 1) / kGroupBlocks;
-  int64_t items, per_item;
-  uniform_items(n_tok, ngroups, cap, &items, &per_item);
-  gram_partial_kernel<<<dim3((unsigned)items, (unsigned)ngroups), kGramThreads, kGramSmem, st>>>(
-      x, C, nullptr, nullptr, n_tok, per_item, partial);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  gram_reduce_kernel<<<(unsigned)((per_group + 255) / 256), 256, 0, st>>>(partial, nb, 1, nullptr,
-                                                                          items, H);
-  return cudaGetLastError();
+  for (int64_t t0 = 0; t0 < n_tok; t0 += kMaxTokensPerLaunch) {
+    const int64_t n = std::min(kMaxTokensPerLaunch, n_tok - t0);
+    int64_t items, per_item;
+    uniform_items(n, ngroups, cap, &items, &per_item);
+    e = gram_uniform(x + t0 * C, n, C, H, partial, items, per_item, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace nvfp4

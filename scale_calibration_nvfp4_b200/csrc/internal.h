@@ -24,6 +24,10 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
                                 const float *s_g, const float *H, uint8_t *codes,
                                 float *best_obj, int local_hessian, cudaStream_t st);
 
+// Copies the search's evaluation counters ([0] MSE, [1] Local-Hessian) to
+// the host after the work queued on `st`, optionally zeroing them.
+cudaError_t read_search_evaluations(cudaStream_t st, unsigned long long out[2], bool reset);
+
 // Gram accumulation.  `offsets` == nullptr: one group of n_tok tokens.
 cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, int64_t n_tok,
                         int64_t C, float *H, cudaStream_t st);
@@ -33,6 +37,10 @@ cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, in
 cudaError_t launch_gram_noalloc(const uint16_t *x, int64_t n_tok, int64_t C, float *H,
                                 cudaStream_t st);
 int64_t gram_noalloc_max_channels();
+
+// Copies the Gram kernels' device status to *out after the work queued on
+// `st`, and clears it.
+cudaError_t read_and_clear_gram_status(cudaStream_t st, int *out);
 
 // Stream-ordered scratch from the library's pool on the current device.
 cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t st);

@@ -7,14 +7,16 @@
 // Method sources: Baseten, "What makes high-quality NVFP4" ("Why do we need
 // scales?", "Block scaling", "Why blocks?", "Calibration"); the QAD article
 // "為什么NVFP4推理精度會掉以及QAD到底在修什么" (2.1, 2.3, 3.2, 4.2).
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "../../include/nvfp4.h"
 
 namespace nvfp4 {
 
-// Sticky device status (NVFP4_OK or NVFP4_ERR_NONFINITE), read and cleared
-// by nvfp4_get_device_status.
+// Sticky device status of the streaming kernels (NVFP4_OK or
+// NVFP4_ERR_NONFINITE), read and cleared by nvfp4_get_device_status.
 __device__ int g_device_status = 0;
 
 namespace {
@@ -165,14 +167,24 @@ __device__ __forceinline__ uint2 encode_block(const uint32_t w[8], float s, floa
   return c;
 }
 
-// Same codes for any s >= 0 (s = 0: signed zeros; s below 2^-100, where the
-// reciprocal may overflow: the exact fp64 midpoint test).  r_hi is the
-// reciprocal rounded down, so r_lo >= 0 and x = -0 keeps its sign in t.
-__device__ __forceinline__ uint2 encode_block_any(const uint32_t w[8], float s) {
-  if (s >= 0x1p-100f) {
-    const float r_hi = __frcp_rd(s);
-    return encode_block(w, s, r_hi, fmaf(-s, r_hi, 1.0f) * r_hi);
+// Packed codes with no midpoint test: only for scales certified by
+// quotients_far_from_midpoints.
+__device__ __forceinline__ uint2 encode_block_certified(const uint32_t w[8], float r_hi,
+                                                        float r_lo) {
+  float t[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
+    t[e] = fmaf(x, r_hi, x * r_lo);
   }
+  uint2 c;
+  c.x = cvt4_e2m1(t[1], t[0], t[3], t[2], t[5], t[4], t[7], t[6]);
+  c.y = cvt4_e2m1(t[9], t[8], t[11], t[10], t[13], t[12], t[15], t[14]);
+  return c;
+}
+
+// Packed codes by the exact fp64 midpoint test (s = 0: signed zeros).
+__device__ __forceinline__ uint2 encode_block_exact(const uint32_t w[8], float s) {
   uint32_t bytes[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -183,6 +195,50 @@ __device__ __forceinline__ uint2 encode_block_any(const uint32_t w[8], float s) 
   }
   return make_uint2(bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24),
                     bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24));
+}
+
+// E4M3 code (0..0x7E) -> fp32 value, branch-free.
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const float sub = (float)c * 0x1p-9f;
+  const float nor = __uint_as_float((c << 20) + (120u << 23));
+  return c < 8u ? sub : nor;
+}
+
+// Everything a block's encode needs from its scale, computed once per code
+// and CTA: s_eff, its reciprocal split (r_hi rounded down, so r_lo >= 0 and
+// x = -0 keeps its sign in t) and which encode is exact for it.
+constexpr uint32_t kCertified = 0;  // plain rounding of t
+constexpr uint32_t kChecked = 1;    // per-element midpoint test, odd-code rule
+constexpr uint32_t kExact = 2;      // s < 2^-100 (reciprocal may overflow), 0 or NaN
+struct ScaleEntry {
+  float s, r_hi, r_lo;
+  uint32_t mode;
+};
+__device__ __forceinline__ ScaleEntry make_scale_entry(float s) {
+  ScaleEntry e;
+  e.s = s;
+  e.r_hi = 0.0f;
+  e.r_lo = 0.0f;
+  e.mode = kExact;
+  if (s >= 0x1p-100f) {
+    e.r_hi = __frcp_rd(s);
+    e.r_lo = fmaf(-s, e.r_hi, 1.0f) * e.r_hi;
+    e.mode = quotients_far_from_midpoints(s) ? kCertified : kChecked;
+  }
+  return e;
+}
+__device__ __forceinline__ uint2 encode_block_entry(const uint32_t w[8], const ScaleEntry &e) {
+  if (e.mode == kCertified) return encode_block_certified(w, e.r_hi, e.r_lo);
+  if (e.mode == kChecked) return encode_block(w, e.s, e.r_hi, e.r_lo);
+  return encode_block_exact(w, e.s);
+}
+
+// Table of ScaleEntry for every code byte of one s_g, filled by the CTA's
+// 256 threads (one each; codes above 0x7E follow the same formula).
+__device__ __forceinline__ void fill_scale_table(ScaleEntry *tab, float sg) {
+  static_assert(kThreads == 256, "one table entry per thread");
+  tab[threadIdx.x] = make_scale_entry(__fmul_rn(sg, e4m3_value(threadIdx.x)));
+  __syncthreads();
 }
 
 // E4M3 code of amax / (6 s_g), exact (nearest even, saturating at 448), from
@@ -209,13 +265,6 @@ __device__ __forceinline__ uint32_t max_rule_code_fast(float amax, const MaxRule
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(ta), "f"(t));
   const uint32_t ct = pair & 0xFFu, ca = pair >> 8;
   return (ct & 1u) ? ct : ca;  // equal, or the odd one of two neighbours
-}
-
-// E4M3 code (0..0x7E) -> fp32 value, branch-free.
-__device__ __forceinline__ float e4m3_value(uint32_t c) {
-  const float sub = (float)c * 0x1p-9f;
-  const float nor = __uint_as_float((c << 20) + (120u << 23));
-  return c < 8u ? sub : nor;
 }
 
 // bf16 pair of v(q) * s for one packed byte: fp32 product, then bf16 RN.
@@ -263,7 +312,8 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const uint16_t *__restri
                                                         const uint8_t *__restrict__ codes,
                                                         uint8_t *__restrict__ packed) {
   const int64_t b = blockIdx.y;
-  const float sg = s_g[b];
+  __shared__ ScaleEntry tab[256];
+  fill_scale_table(tab, s_g[b]);
   w += b * nblk * kBlock;
   codes += b * nblk;
   packed += b * nblk * (kBlock / 2);
@@ -284,7 +334,7 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const uint16_t *__restri
       load_block(w + n * kBlock, nv);
       ncode = codes[n];
     }
-    st_stream_v2(packed + i * 8, encode_block_any(v, __fmul_rn(sg, e4m3_value(code))));
+    st_stream_v2(packed + i * 8, encode_block_entry(v, tab[code]));
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = nv[j];
     code = ncode;
@@ -321,6 +371,8 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__
                                                               uint8_t *__restrict__ codes) {
   const float sg = *s_g;
   const MaxRule mr = make_max_rule(sg);
+  __shared__ ScaleEntry tab[256];
+  fill_scale_table(tab, sg);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   uint32_t v[8];
@@ -332,8 +384,9 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__
     if (n < nblk) load_block(x + n * kBlock, nv);
     const float amax = __uint_as_float(amax_bits8(v) << 16);
     const uint32_t code = max_rule_code_fast(amax, mr);
-    const float s = __fmul_rn(sg, e4m3_value(code));
-    const uint2 q = encode_block_any(v, s);
+    const ScaleEntry se = tab[code];
+    const float s = se.s;
+    const uint2 q = encode_block_entry(v, se);
     const uint32_t bytes[8] = {q.x & 0xFFu, (q.x >> 8) & 0xFFu, (q.x >> 16) & 0xFFu, q.x >> 24,
                                q.y & 0xFFu, (q.y >> 8) & 0xFFu, (q.y >> 16) & 0xFFu, q.y >> 24};
     store_dequant(out + i * kBlock, bytes, s);
@@ -395,7 +448,13 @@ cudaError_t launch_scale_max(const uint16_t *w, int64_t batch, int64_t nblk, con
 cudaError_t launch_pack(const uint16_t *w, int64_t batch, int64_t nblk, const float *s_g,
                         const uint8_t *codes, uint8_t *packed, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
-  int gx = grid_for(nblk, 16);
+  // at least four blocks per thread where there is enough work, so that the
+  // CTA's scale table is amortised, but enough CTAs to fill every SM across
+  // the batch
+  const int64_t need = grid_for(nblk, 16);
+  const int64_t want = (nblk + 4 * kThreads - 1) / (4 * kThreads);
+  const int64_t fill = ((int64_t)sm_count() * 4 + batch - 1) / batch;
+  const int gx = (int)std::min(need, std::max(want, fill));
   pack_kernel<<<dim3(gx, (unsigned)batch), kThreads, 0, st>>>(w, nblk, s_g, codes, packed);
   return cudaGetLastError();
 }
@@ -426,7 +485,13 @@ cudaError_t read_and_clear_device_status(cudaStream_t st, int *out) {
   if (e != cudaSuccess) return e;
   e = cudaMemcpyFromSymbol(out, g_device_status, sizeof(int));
   if (e != cudaSuccess) return e;
-  return cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return e;
+  // the Gram kernels keep their own flag (a timed-out wait)
+  int gram = 0;
+  e = read_and_clear_gram_status(st, &gram);
+  if (*out == 0) *out = gram;
+  return e;
 }
 
 }  // namespace nvfp4

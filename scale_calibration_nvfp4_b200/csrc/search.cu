@@ -46,6 +46,12 @@
 #include "internal.h"
 
 namespace nvfp4 {
+
+// (block, candidate) objective evaluations of the fp32 screen since the last
+// reset: [0] MSE, [1] Local-Hessian.  A statistic of the work the pruned walk
+// does; nothing reads it on the device.
+__device__ unsigned long long g_search_evals[2];
+
 namespace {
 
 constexpr int kThreads = 128;  // 4 warps
@@ -71,6 +77,7 @@ __constant__ int kClassBegin[9] = {0, 18, 35, 51, 67, 82, 97, 112, 126};
 struct ClassInfo {
   float S, r_hi, r_lo;  // S = fl(s_g o), 1/S = r_hi + r_lo
   int end;              // one past its last candidate
+  int certified;        // no quotient |w| / S comes near a rounding midpoint
 };
 struct CandInfo {
   float f;      // 2^-p, scales the class quotient to this candidate
@@ -163,37 +170,50 @@ __device__ void cholesky16(const float *Hs, float *Lf) {
 // column-sum norm bounds the 2-norm from above, so this bounds lambda_min from
 // below (with 2% to spare for rounding).  Lane i < 16 forms column i of the
 // inverse by a forward and a backward triangular solve in fp64.  A dropped
-// pivot (zero diagonal in L) makes the matrix singular: the bound is 0.
-__device__ __noinline__ float lambda_lower_bound(const float *Lf) {
+// pivot (zero diagonal in L) makes the matrix singular: the bound is 0 (no
+// pruning).  So it is too when max diag(L L^T) ||(L L^T)^-1||_1 exceeds
+// 10^4: L L^T differs from H by at most 2^-23 trace(H) <= 2^-19 max diag(H)
+// (fp32 rounding of the factor), which then stays below 2% of lambda_min.
+__device__ __forceinline__ float lambda_lower_bound(const float *Lf, double *inv_d) {
   const int lane = threadIdx.x & 31;
-  double colsum = 0.0;
+  // 1 / L_kk and the largest diagonal entry of L L^T (lane k < 16: row k)
+  double maxdiag = 0.0;
   int singular = 0;
   if (lane < 16) {
-    // once per CTA: kept rolled (y in local memory) so that it does not raise
-    // the kernel's register budget
-    double y[16];
-#pragma unroll 1
-    for (int k = 0; k < 16; ++k) {
-      double acc = (k == lane) ? 1.0 : 0.0;
-#pragma unroll 1
-      for (int m = 0; m < k; ++m) acc = fma(-(double)Lf[k * 16 + m], y[m], acc);
-      const double d = (double)Lf[k * 16 + k];
-      singular |= (d == 0.0);
-      y[k] = acc / d;
-    }
-#pragma unroll 1
-    for (int k = 15; k >= 0; --k) {
-      double acc = y[k];
-#pragma unroll 1
-      for (int m = k + 1; m < 16; ++m) acc = fma(-(double)Lf[m * 16 + k], y[m], acc);
-      y[k] = acc / (double)Lf[k * 16 + k];
-      colsum += fabs(y[k]);
-    }
+    const double d = (double)Lf[lane * 16 + lane];
+    singular = d == 0.0;
+    inv_d[lane] = 1.0 / d;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) maxdiag = fma((double)Lf[lane * 16 + m], (double)Lf[lane * 16 + m], maxdiag);
   }
   singular = __any_sync(0xFFFFFFFFu, singular);
 #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) maxdiag = fmax(maxdiag, __shfl_xor_sync(0xFFFFFFFFu, maxdiag, o));
+  __syncwarp();
+  double colsum = 0.0;
+  if (lane < 16 && !singular) {
+    // column sweeps: acc = e_lane, then L y = acc, then L^T z = y (in place;
+    // outer loops rolled, acc in local memory: once per block of H)
+    double acc[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) acc[m] = (m == lane) ? 1.0 : 0.0;
+#pragma unroll 1
+    for (int k = 0; k < 16; ++k) {
+      acc[k] *= inv_d[k];
+#pragma unroll
+      for (int m = k + 1; m < 16; ++m) acc[m] = fma(-(double)Lf[m * 16 + k], acc[k], acc[m]);
+    }
+#pragma unroll 1
+    for (int k = 15; k >= 0; --k) {
+      acc[k] *= inv_d[k];
+      colsum += fabs(acc[k]);
+#pragma unroll
+      for (int m = 0; m < k; ++m) acc[m] = fma(-(double)Lf[k * 16 + m], acc[k], acc[m]);
+    }
+  }
+#pragma unroll
   for (int o = 16; o > 0; o >>= 1) colsum = fmax(colsum, __shfl_xor_sync(0xFFFFFFFFu, colsum, o));
-  if (singular || !(colsum > 0.0) || !(colsum < 1e300)) return 0.0f;
+  if (singular || !(colsum > 0.0) || !(colsum < 1e300) || maxdiag * colsum > 1e4) return 0.0f;
   return (float)(0.98 / colsum);
 }
 
@@ -336,24 +356,24 @@ struct Factor {
   int pad;
 };
 
-__global__ void __launch_bounds__(kThreads)
-    factor_kernel(const float *__restrict__ H, int64_t nblocks, uint4 *__restrict__ frag,
+__global__ void __launch_bounds__(32)
+    factor_kernel(const float *__restrict__ H, uint4 *__restrict__ frag,
                   Factor *__restrict__ fac) {
-  __shared__ float Hs[kWarps][256];
-  __shared__ float Lf[kWarps][256];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t blk = (int64_t)blockIdx.x * kWarps + warp;
-  if (blk >= nblocks) return;  // whole warps only
+  __shared__ float Hs[256];
+  __shared__ float Lf[256];
+  __shared__ double inv_d[16];
+  const int lane = threadIdx.x;
+  const int64_t blk = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;  // one warp per block of H
   const float *Hb = H + blk * 256;
-  for (int i = lane; i < 256; i += 32) Hs[warp][i] = Hb[i];
+  for (int i = lane; i < 256; i += 32) Hs[i] = Hb[i];
   __syncwarp();
-  cholesky16(Hs[warp], Lf[warp]);
+  cholesky16(Hs, Lf);
   __syncwarp();
   float m = 0.0f;
-  for (int i = lane; i < 256; i += 32) m = fmaxf(m, fabsf(Lf[warp][i]));
+  for (int i = lane; i < 256; i += 32) m = fmaxf(m, fabsf(Lf[i]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  const float lam = lambda_lower_bound(Lf[warp]);
+  const float lam = lambda_lower_bound(Lf, inv_d);
   int e = 0;
   frexpf(m, &e);  // m < 2^e
   const float sigma = m > 0.0f ? ldexpf(1.0f, 15 - e) : 1.0f;
@@ -366,7 +386,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int k0 = 2 * t + 8 * half;
-      const float x0 = Lf[warp][k0 * 16 + n] * sigma, x1 = Lf[warp][(k0 + 1) * 16 + n] * sigma;
+      const float x0 = Lf[k0 * 16 + n] * sigma, x1 = Lf[(k0 + 1) * 16 + n] * sigma;
       const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
       const __half l0 = __float2half_rn(x0 - __half2float(h0));
       const __half l1 = __float2half_rn(x1 - __half2float(h1));
@@ -471,6 +491,7 @@ __global__ void __launch_bounds__(kThreads)
       k2.r_hi = (float)rr;
       k2.r_lo = (float)(rr - (double)k2.r_hi);
       k2.end = by_class ? kClassBegin[threadIdx.x + 1] : (int)threadIdx.x + 1;
+      k2.certified = S >= 0x1p-100f && S < 0x1p100f && quotients_far_from_midpoints(S);
       cls[threadIdx.x] = k2;
     }
     if (threadIdx.x == 0) ncls_sh = ncls;
@@ -514,6 +535,7 @@ __global__ void __launch_bounds__(kThreads)
     }
   }
 
+  unsigned long long evals = 0;
   for (int tile = warp; tile < kRowsPerCta / kTileRows; tile += kWarps) {
     const uint32_t kg = keys[tile * kTileRows + g], kg8 = keys[tile * kTileRows + g + 8];
     const bool v0 = (kg >> 16) != 0xFFFFu, v1 = (kg8 >> 16) != 0xFFFFu;
@@ -527,6 +549,10 @@ __global__ void __launch_bounds__(kThreads)
       W1[0] = c0.x; W1[1] = c0.y; W1[2] = c0.z; W1[3] = c0.w;
       W1[4] = c1.x; W1[5] = c1.y; W1[6] = c1.z; W1[7] = c1.w;
     }
+    // rows of the tile that are not padding (each row sits in four lanes)
+    const uint32_t nvalid =
+        (__popc(__ballot_sync(0xFFFFFFFFu, v0)) + __popc(__ballot_sync(0xFFFFFFFFu, v1))) >> 2;
+    uint32_t ncand = 0;  // candidates evaluated for the tile
     // row amax (bf16 magnitude bits; 0 for padding) and the tile's largest
     const uint32_t am0 = v0 ? kg >> 16 : 0u, am1 = v1 ? kg8 >> 16 : 0u;
     const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(am0, am1));
@@ -610,11 +636,14 @@ __global__ void __launch_bounds__(kThreads)
       float tq[8], ta[8];
       bool near = false;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        tq[e] = fmaf(a[e], ci.r_hi, a[e] * ci.r_lo);
-        // t within two floats of a value whose low 21 mantissa bits are zero
-        // (every rounding midpoint times a power of two is one)
-        near = near || ((__float_as_uint(tq[e]) + 2u) & 0x1FFFFFu) <= 4u;
+      for (int e = 0; e < 8; ++e) tq[e] = fmaf(a[e], ci.r_hi, a[e] * ci.r_lo);
+      if (!ci.certified) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          // t within two floats of a value whose low 21 mantissa bits are
+          // zero (every rounding midpoint times a power of two is one)
+          near = near || ((__float_as_uint(tq[e]) + 2u) & 0x1FFFFFu) <= 4u;
+        }
       }
       const bool alt = !kAltSkip || __any_sync(0xFFFFFFFFu, near);
       if (alt) {
@@ -646,6 +675,7 @@ __global__ void __launch_bounds__(kThreads)
             alt ? candidate_objective<kLH, true>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper)
                 : candidate_objective<kLH, false>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
         track3(key_of(e0, c0.c), b1, b2, b3);
+        ++ncand;
       }
       // upwards from js + 1
       for (int j = js + 1; j < ci.end; ++j) {
@@ -670,9 +700,12 @@ __global__ void __launch_bounds__(kThreads)
             alt ? candidate_objective<kLH, true>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper)
                 : candidate_objective<kLH, false>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
         track3(key_of(e0, c0.c), b1, b2, b3);
+        ++ncand;
       }
       jbegin = ci.end;
     }
+
+    evals += (unsigned long long)ncand * nvalid;
 
     // lane t = 0 finishes row g, lane t = 2 row g + 8; near ties are
     // re-scored by the whole warp, one row at a time
@@ -708,9 +741,22 @@ __global__ void __launch_bounds__(kThreads)
       if (ob) ob[r * nb] = obj;
     }
   }
+  if (lane == 0 && evals) atomicAdd(&g_search_evals[kLH ? 1 : 0], evals);
 }
 
 }  // namespace
+
+cudaError_t read_search_evaluations(cudaStream_t st, unsigned long long out[2], bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_search_evals, sizeof(g_search_evals), 0,
+                                            cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess && reset) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_search_evals);
+    if (e == cudaSuccess) e = cudaMemsetAsync(p, 0, sizeof(g_search_evals), st);
+  }
+  const cudaError_t es = cudaStreamSynchronize(st);
+  return e != cudaSuccess ? e : es;
+}
 
 cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int64_t C,
                                 const float *s_g, const float *H, uint8_t *codes,
@@ -731,8 +777,7 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
   if (e != cudaSuccess) return e;
   uint4 *frag = static_cast<uint4 *>(scratch);
   Factor *fac = reinterpret_cast<Factor *>(static_cast<char *>(scratch) + frag_bytes);
-  factor_kernel<<<(unsigned)((nblocks + kWarps - 1) / kWarps), kThreads, 0, st>>>(H, nblocks,
-                                                                                  frag, fac);
+  factor_kernel<<<dim3((unsigned)(C / kBlock), (unsigned)batch), 32, 0, st>>>(H, frag, fac);
   e = cudaGetLastError();
   if (e == cudaSuccess) {
     search_kernel<true><<<grid, kThreads, 0, st>>>(w, R, C, s_g, H, frag, fac, codes, best_obj);

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
 STATUS = {
     0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_SHAPE", 3: "NVFP4_ERR_MISALIGNED",
     4: "NVFP4_ERR_NONFINITE", 5: "NVFP4_ERR_CUDA", 6: "NVFP4_ERR_NOT_IMPLEMENTED",
-    7: "NVFP4_ERR_TOO_LARGE",
+    7: "NVFP4_ERR_TOO_LARGE", 8: "NVFP4_ERR_DEVICE_TIMEOUT",
 }
 
 # C entry points and their argument types (mirrors include/nvfp4.h)
@@ -35,6 +35,7 @@ SIGNATURES = {
     "nvfp4_dequantize": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
     "nvfp4_fake_quant": [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp],
     "nvfp4_get_device_status": [_vp, _vp],
+    "nvfp4_search_evaluations": [_vp, ctypes.c_int, _vp],
 }
 
 
@@ -258,6 +259,15 @@ def get_device_status(stream=None):
     st = ctypes.c_int(0)
     _call("nvfp4_get_device_status", _stream(stream), ctypes.byref(st))
     return STATUS.get(st.value, str(st.value))
+
+
+def search_evaluations(reset=False, stream=None):
+    """(MSE, Local-Hessian) counts of (block, candidate) objective evaluations
+    made by the scale searches on the current device since the last reset;
+    synchronises the stream."""
+    out = (ctypes.c_uint64 * 2)()
+    _call("nvfp4_search_evaluations", _stream(stream), int(bool(reset)), out)
+    return int(out[0]), int(out[1])
 
 
 def status_string(code):

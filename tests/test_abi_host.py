@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in range(8):
+    for code in range(9):
         s = L.nvfp4_status_string(code).decode()
         assert s.startswith("NVFP4_")
     assert L.nvfp4_status_string(0).decode() == "NVFP4_OK"
@@ -90,6 +90,8 @@ def test_validation_rejects_before_launch(L):
     # sizes that overflow
     assert L.nvfp4_scale_search_max(P, 1, 1 << 40, 1 << 24, P, P, None) == SHAPE
     assert L.nvfp4_scale_search_max(P, 70000, 4, 16, P, P, None) == TOOLARGE
+    # the statistics call needs somewhere to write
+    assert L.nvfp4_search_evaluations(None, 0, None) == INVALID
 
 
 def test_binding_rejects_cpu_tensors():

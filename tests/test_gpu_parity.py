@@ -99,7 +99,12 @@ def test_max_rule_exact_midpoint_ties(nv):
 # ------------------------------------------------------------ E2M1 encode
 @pytest.mark.parametrize("s_g,code", [(1.0, 0x38), (1.0, 0x56), (2.0 ** -5, 0x7E),
                                       (0.0123456, 0x31), (3.3e-3, 0x01), (7.1e-4, 0x77),
-                                      (1.0, 0x07), (0.5, 0x00)])
+                                      (1.0, 0x07), (0.5, 0x00),
+                                      # scales next to the threshold of the kernels'
+                                      # "no quotient near a midpoint" certificate
+                                      # (1 + 9 ulp passes it, 1 + 8 ulp does not)
+                                      (1.0 + 9 * 2.0 ** -23, 0x38), (1.0 + 8 * 2.0 ** -23, 0x38),
+                                      (2.0 - 9 * 2.0 ** -23, 0x38), (1.0 + 9 * 2.0 ** -23, 0x3B)])
 def test_encode_every_bf16_pattern(nv, s_g, code):
     """All 65,536 bf16 bit patterns (NaN/Inf replaced by 0) through the
     packed encode at one block scale: bit-exact against the oracle."""
@@ -362,6 +367,26 @@ def test_search_ragged_rows_mixed_magnitudes(nv):
     rc, _ = oracle.scale_search_mse(wu, sg)
     check_search_codes(cm, rc, wu, sg)
     assert np.all(cm[7] == 1) and np.all(clh[300:310] == 1)
+
+
+def test_search_evaluation_counters(nv):
+    """The work statistic: between 1 and 126 evaluations per block searched,
+    counted per rule, and zeroed by a reset."""
+    W, X = _layer("tiny")
+    s_g = nv.global_scale(W)
+    H = torch.zeros(W.shape[1] // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate(X, H)
+    nv.search_evaluations(reset=True)
+    assert nv.search_evaluations() == (0, 0)
+    blocks = W.numel() // 16
+    nv.scale_search_mse(W, s_g)
+    m, l = nv.search_evaluations()
+    assert blocks <= m <= 126 * blocks and l == 0
+    nv.scale_search_local_hessian(W, s_g, H)
+    nv.scale_search_local_hessian(W, s_g, H)
+    m2, l2 = nv.search_evaluations(reset=True)
+    assert m2 == m and 2 * blocks <= l2 <= 2 * 126 * blocks and l2 % 2 == 0
+    assert nv.search_evaluations() == (0, 0)
 
 
 def test_dense_layer_sampled(nv):

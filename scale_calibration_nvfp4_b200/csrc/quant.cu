@@ -131,56 +131,32 @@ __device__ __forceinline__ float toward(float t, float rho) {
   return __int_as_float(__float_as_int(t) + (rb != 0 ? dir : 0));
 }
 
-// Low 21 mantissa bits of t within two floats of zero (a superset test).
-__device__ __forceinline__ uint32_t near_key(float t) {
-  return (__float_as_uint(t) + 2u) & 0x1FFFF8u;
+// Packed signed E2M1 codes of 8 consecutive elements (4 bf16 pairs) at scale
+// s > 0 with r_hi + r_lo = 1/s (r_lo >= 0).  Every element is rounded twice:
+// t (within one float of q = x / s) and its neighbour on the other side of q
+// (by the exact sign of the residual x - t s, one fma).  The two codes can
+// differ only when one of the floats is an E2M1 rounding midpoint, which it
+// then rounds to its even neighbour, while q lies strictly on the other
+// side: the correct code is the odd one of the two.  Branch-free: exact ties
+// (q on a midpoint) are common for bf16 data at round scales.
+__device__ __forceinline__ uint32_t encode_word(const uint32_t *w, float s, float r_hi,
+                                                float r_lo) {
+  float t[8], ta[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
+    t[e] = fmaf(x, r_hi, x * r_lo);
+    ta[e] = toward(t[e], fmaf(-t[e], s, x));
+  }
+  const uint32_t ct = cvt4_e2m1(t[1], t[0], t[3], t[2], t[5], t[4], t[7], t[6]);
+  const uint32_t ca = cvt4_e2m1(ta[1], ta[0], ta[3], ta[2], ta[5], ta[4], ta[7], ta[6]);
+  const uint32_t odd = (ct & 0x11111111u) * 15u;
+  return (ct & odd) | (ca & ~odd);
 }
 
-// Packed signed E2M1 codes of one block (two words, 16 codes) at scale s > 0
-// with r_hi + r_lo = 1/s (r_lo >= 0).
 __device__ __forceinline__ uint2 encode_block(const uint32_t w[8], float s, float r_hi,
                                               float r_lo) {
-  float t[16];
-  uint32_t nk = 0xFFFFFFFFu;
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
-    t[e] = fmaf(x, r_hi, x * r_lo);
-    nk = min(nk, near_key(t[e]));
-  }
-  uint2 c;
-  c.x = cvt4_e2m1(t[1], t[0], t[3], t[2], t[5], t[4], t[7], t[6]);
-  c.y = cvt4_e2m1(t[9], t[8], t[11], t[10], t[13], t[12], t[15], t[14]);
-  if (__any_sync(__activemask(), nk == 0u)) {
-    float ta[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
-      ta[e] = toward(t[e], fmaf(-t[e], s, x));
-    }
-    const uint32_t ax = cvt4_e2m1(ta[1], ta[0], ta[3], ta[2], ta[5], ta[4], ta[7], ta[6]);
-    const uint32_t ay = cvt4_e2m1(ta[9], ta[8], ta[11], ta[10], ta[13], ta[12], ta[15], ta[14]);
-    const uint32_t ox = (c.x & 0x11111111u) * 15u, oy = (c.y & 0x11111111u) * 15u;
-    c.x = (c.x & ox) | (ax & ~ox);
-    c.y = (c.y & oy) | (ay & ~oy);
-  }
-  return c;
-}
-
-// Packed codes with no midpoint test: only for scales certified by
-// quotients_far_from_midpoints.
-__device__ __forceinline__ uint2 encode_block_certified(const uint32_t w[8], float r_hi,
-                                                        float r_lo) {
-  float t[16];
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
-    t[e] = fmaf(x, r_hi, x * r_lo);
-  }
-  uint2 c;
-  c.x = cvt4_e2m1(t[1], t[0], t[3], t[2], t[5], t[4], t[7], t[6]);
-  c.y = cvt4_e2m1(t[9], t[8], t[11], t[10], t[13], t[12], t[15], t[14]);
-  return c;
+  return make_uint2(encode_word(w, s, r_hi, r_lo), encode_word(w + 4, s, r_hi, r_lo));
 }
 
 // Packed codes by the exact fp64 midpoint test (s = 0: signed zeros).
@@ -205,31 +181,28 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
 }
 
 // Everything a block's encode needs from its scale, computed once per code
-// and CTA: s_eff, its reciprocal split (r_hi rounded down, so r_lo >= 0 and
-// x = -0 keeps its sign in t) and which encode is exact for it.
-constexpr uint32_t kCertified = 0;  // plain rounding of t
-constexpr uint32_t kChecked = 1;    // per-element midpoint test, odd-code rule
-constexpr uint32_t kExact = 2;      // s < 2^-100 (reciprocal may overflow), 0 or NaN
+// and CTA: s_eff and its reciprocal split (r_hi rounded down, so r_lo >= 0 and
+// x = -0 keeps its sign in t), or 0 for scales below 2^-100 (where the
+// reciprocal may overflow), zero or NaN, which take the exact fp64 encode.
 struct ScaleEntry {
   float s, r_hi, r_lo;
-  uint32_t mode;
+  uint32_t exact64;
 };
 __device__ __forceinline__ ScaleEntry make_scale_entry(float s) {
   ScaleEntry e;
   e.s = s;
   e.r_hi = 0.0f;
   e.r_lo = 0.0f;
-  e.mode = kExact;
+  e.exact64 = 1u;
   if (s >= 0x1p-100f) {
     e.r_hi = __frcp_rd(s);
     e.r_lo = fmaf(-s, e.r_hi, 1.0f) * e.r_hi;
-    e.mode = quotients_far_from_midpoints(s) ? kCertified : kChecked;
+    e.exact64 = 0u;
   }
   return e;
 }
 __device__ __forceinline__ uint2 encode_block_entry(const uint32_t w[8], const ScaleEntry &e) {
-  if (e.mode == kCertified) return encode_block_certified(w, e.r_hi, e.r_lo);
-  if (e.mode == kChecked) return encode_block(w, e.s, e.r_hi, e.r_lo);
+  if (!e.exact64) return encode_block(w, e.s, e.r_hi, e.r_lo);
   return encode_block_exact(w, e.s);
 }
 
@@ -312,8 +285,6 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const uint16_t *__restri
                                                         const uint8_t *__restrict__ codes,
                                                         uint8_t *__restrict__ packed) {
   const int64_t b = blockIdx.y;
-  __shared__ ScaleEntry tab[256];
-  fill_scale_table(tab, s_g[b]);
   w += b * nblk * kBlock;
   codes += b * nblk;
   packed += b * nblk * (kBlock / 2);
@@ -325,6 +296,9 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const uint16_t *__restri
     load_block(w + i * kBlock, v);
     code = codes[i];
   }
+  // the table is built while the first block is in flight
+  __shared__ ScaleEntry tab[256];
+  fill_scale_table(tab, s_g[b]);
   for (; i < nblk; i += stride) {
     // issue the next block's loads before this block's arithmetic
     uint32_t nv[8];
@@ -369,14 +343,15 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__
                                                               uint16_t *__restrict__ out,
                                                               uint8_t *__restrict__ packed,
                                                               uint8_t *__restrict__ codes) {
-  const float sg = *s_g;
-  const MaxRule mr = make_max_rule(sg);
-  __shared__ ScaleEntry tab[256];
-  fill_scale_table(tab, sg);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   uint32_t v[8];
   if (i < nblk) load_block(x + i * kBlock, v);
+  // the table is built while the first block is in flight
+  const float sg = *s_g;
+  const MaxRule mr = make_max_rule(sg);
+  __shared__ ScaleEntry tab[256];
+  fill_scale_table(tab, sg);
   for (; i < nblk; i += stride) {
     // issue the next block's loads before this block's arithmetic
     uint32_t nv[8];

@@ -22,6 +22,7 @@ __device__ int g_device_status = 0;
 namespace {
 
 constexpr int kThreads = 256;
+
 constexpr uint32_t kMagMask = 0x7FFF7FFFu;
 
 // ---------------------------------------------------------------- amax
@@ -423,13 +424,14 @@ cudaError_t launch_scale_max(const uint16_t *w, int64_t batch, int64_t nblk, con
 cudaError_t launch_pack(const uint16_t *w, int64_t batch, int64_t nblk, const float *s_g,
                         const uint8_t *codes, uint8_t *packed, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
-  // at least four blocks per thread where there is enough work, so that the
-  // CTA's scale table is amortised, but enough CTAs to fill every SM across
-  // the batch
-  const int64_t need = grid_for(nblk, 16);
-  const int64_t want = (nblk + 4 * kThreads - 1) / (4 * kThreads);
-  const int64_t fill = ((int64_t)sm_count() * 4 + batch - 1) / batch;
-  const int gx = (int)std::min(need, std::max(want, fill));
+  // up to eight blocks per thread, so that each CTA's scale table is
+  // amortised, but never fewer than four waves of resident CTAs (five per
+  // SM) across the whole batch, which keeps the tail short
+  const int64_t need = (nblk + kThreads - 1) / kThreads;  // one block per thread
+  const int64_t by_work = (batch * nblk + 8 * kThreads - 1) / (8 * kThreads);
+  const int64_t by_waves = std::min(batch * need, (int64_t)sm_count() * 5 * 4);
+  const int64_t total = std::max(by_work, by_waves);
+  const int gx = (int)std::min(std::min(need, (total + batch - 1) / batch), (int64_t)1 << 30);
   pack_kernel<<<dim3(gx, (unsigned)batch), kThreads, 0, st>>>(w, nblk, s_g, codes, packed);
   return cudaGetLastError();
 }

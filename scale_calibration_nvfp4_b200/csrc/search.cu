@@ -32,7 +32,9 @@
 // 2^-p exactly.  Round-to-nearest-even of t and of t_alt (hardware e2m1x2
 // conversion) can only disagree when one of them is a rounding midpoint; q
 // then lies strictly on the other one's side and the correct code is the odd
-// one of the two (the tie went to the even one).
+// one of the two (the tie went to the even one).  Classes whose S passes
+// quotients_far_from_midpoints (no bf16 value comes near a midpoint) round t
+// alone.
 //
 // Winner: fp32 screen keeping the best three objectives; when the best two
 // are within 2^-12 (relative) or the best is numerically zero, the candidates
@@ -60,11 +62,7 @@ constexpr int kTileRows = 16;
 #ifndef NVFP4_SEARCH_TILES
 #define NVFP4_SEARCH_TILES 4
 #endif
-#ifndef NVFP4_SEARCH_ALT_SKIP
-#define NVFP4_SEARCH_ALT_SKIP 1
-#endif
 constexpr int kTilesPerWarp = NVFP4_SEARCH_TILES;
-constexpr bool kAltSkip = NVFP4_SEARCH_ALT_SKIP;
 constexpr int kRowsPerCta = kWarps * kTileRows * kTilesPerWarp;  // 256
 constexpr float kTieBand = 1.0f / 4096.0f;
 constexpr float kZeroFloor = 0x1p-40f;  // relative to ||p||^2
@@ -634,18 +632,12 @@ __global__ void __launch_bounds__(kThreads)
       const ClassInfo ci = cls[k];
       // class quotient t per element (within one float of q)
       float tq[8], ta[8];
-      bool near = false;
 #pragma unroll
       for (int e = 0; e < 8; ++e) tq[e] = fmaf(a[e], ci.r_hi, a[e] * ci.r_lo);
-      if (!ci.certified) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          // t within two floats of a value whose low 21 mantissa bits are
-          // zero (every rounding midpoint times a power of two is one)
-          near = near || ((__float_as_uint(tq[e]) + 2u) & 0x1FFFFFu) <= 4u;
-        }
-      }
-      const bool alt = !kAltSkip || __any_sync(0xFFFFFFFFu, near);
+      // uncertified classes take the neighbour rounding for every candidate:
+      // at the scales where the certificate fails, some element of most
+      // tiles does sit near a midpoint
+      const bool alt = !ci.certified;
       if (alt) {
         // the neighbouring float of t on the other side of q, by the exact
         // sign of the residual |w| - t S (t itself when exact)

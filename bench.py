@@ -574,9 +574,14 @@ def cpu_baseline(run, budget_s=15.0):
             oracle.fake_quant(fq)
         return time.perf_counter() - t0, x_rows
 
-    probe = min(R, 32)
-    t_probe, _ = path(probe)
-    rows = int(max(1, min(R, probe * budget_s / max(t_probe, 1e-3))))
+    # time = fixed part (tensor scale, thread start-up) + per-row part, fitted
+    # from two probes, then the sample sized to the budget
+    p1, p2 = min(R, 32), min(R, 128)
+    t1, _ = path(p1)
+    t2, _ = path(p2)
+    per_row = max((t2 - t1) / max(p2 - p1, 1), 1e-7)
+    fixed = max(t1 - p1 * per_row, 0.0)
+    rows = int(max(1, min(R, (budget_s - fixed) / per_row)))
     t, x_rows = path(rows)
     blocks = rows * C // 16
     return {"value": round(blocks / t, 2), "unit": UNIT, "cores": oracle.max_threads(),

@@ -233,6 +233,16 @@ nvfp4_status nvfp4_get_device_status(void *stream, nvfp4_status *out);
  */
 nvfp4_status nvfp4_search_evaluations(void *stream, int reset, uint64_t *out);
 
+/*
+ * Diagnostic of the failure path of the kernels that wait on their own tile
+ * copies (the pages have no counterpart): enqueues one warp that waits on an
+ * mbarrier nothing arrives on.  Its wait gives up after about one second and
+ * sets the device status to NVFP4_ERR_DEVICE_TIMEOUT, which the next
+ * nvfp4_get_device_status reports; the context stays usable.  No data is
+ * touched.
+ */
+nvfp4_status nvfp4_self_test_device_timeout(void *stream);
+
 /* Releases the library's memory pool on every device it touched.  No call
  * may be in flight. */
 void nvfp4_shutdown(void);

@@ -240,6 +240,10 @@ nvfp4_status nvfp4_search_evaluations(void *stream, int reset, uint64_t *out) {
   return NVFP4_OK;
 }
 
+nvfp4_status nvfp4_self_test_device_timeout(void *stream) {
+  return map_cuda(nvfp4::launch_wait_timeout_probe(as_stream(stream)));
+}
+
 void nvfp4_shutdown(void) { nvfp4::scratch_release_all(); }
 
 }  // extern "C"

@@ -242,6 +242,19 @@ __global__ void __launch_bounds__(kGramThreads)
   }
 }
 
+// Diagnostic: one warp waits on an mbarrier that nothing arrives on, so the
+// bounded wait runs out after kWaitLimitNs and the timeout status is set (no
+// copy is in flight).  Exercises the same wait and status path as
+// gram_partial_kernel.
+__global__ void wait_timeout_probe_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = (uint32_t)__cvta_generic_to_shared(&bar);
+  if (threadIdx.x == 0) mbar_init(b, 1);
+  __syncwarp();
+  const bool ok = mbar_wait_bounded(b, 0);
+  if (!ok && threadIdx.x == 0) atomicExch(&g_gram_status, (int)NVFP4_ERR_DEVICE_TIMEOUT);
+}
+
 // H[g][j][e] += sum of the partials of group g's items, in item order.
 __global__ void gram_reduce_kernel(const float *__restrict__ partial, int64_t nb, int64_t G,
                                    const int64_t *__restrict__ item_start, int64_t n_items_uniform,
@@ -471,6 +484,11 @@ cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, in
   }
   cudaError_t e2 = scratch_free(ws, st);
   return e != cudaSuccess ? e : e2;
+}
+
+cudaError_t launch_wait_timeout_probe(cudaStream_t st) {
+  wait_timeout_probe_kernel<<<1, 32, 0, st>>>();
+  return cudaGetLastError();
 }
 
 cudaError_t read_and_clear_gram_status(cudaStream_t st, int *out) {

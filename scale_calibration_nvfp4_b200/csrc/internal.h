@@ -42,6 +42,10 @@ int64_t gram_noalloc_max_channels();
 // `st`, and clears it.
 cudaError_t read_and_clear_gram_status(cudaStream_t st, int *out);
 
+// One warp whose bounded mbarrier wait runs out (about one second), setting
+// the device timeout status.
+cudaError_t launch_wait_timeout_probe(cudaStream_t st);
+
 // Stream-ordered scratch from the library's pool on the current device.
 cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t st);
 cudaError_t scratch_free(void *p, cudaStream_t st);

@@ -36,6 +36,7 @@ SIGNATURES = {
     "nvfp4_fake_quant": [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp],
     "nvfp4_get_device_status": [_vp, _vp],
     "nvfp4_search_evaluations": [_vp, ctypes.c_int, _vp],
+    "nvfp4_self_test_device_timeout": [_vp],
 }
 
 
@@ -268,6 +269,12 @@ def search_evaluations(reset=False, stream=None):
     out = (ctypes.c_uint64 * 2)()
     _call("nvfp4_search_evaluations", _stream(stream), int(bool(reset)), out)
     return int(out[0]), int(out[1])
+
+
+def self_test_device_timeout(stream=None):
+    """Enqueue the diagnostic wait that times out (about one second); the
+    next get_device_status() reports NVFP4_ERR_DEVICE_TIMEOUT."""
+    _call("nvfp4_self_test_device_timeout", _stream(stream))
 
 
 def status_string(code):

@@ -64,6 +64,20 @@ def test_global_scale_nonfinite_reports(nv):
     assert nv.get_device_status() == "NVFP4_OK"  # cleared by the read
 
 
+def test_bounded_wait_reports_timeout_and_context_survives(nv):
+    """A wait that nothing completes gives up (about one second), the host
+    reads NVFP4_ERR_DEVICE_TIMEOUT, and the context still runs kernels."""
+    assert nv.get_device_status() == "NVFP4_OK"
+    nv.self_test_device_timeout()
+    assert nv.get_device_status() == "NVFP4_ERR_DEVICE_TIMEOUT"
+    assert nv.get_device_status() == "NVFP4_OK"  # cleared by the read
+    x = rand_bf16((300, 64), 12)
+    H = torch.zeros(4, 16, 16, device="cuda")
+    nv.hessian_accumulate(x.cuda(), H)
+    assert rel_frobenius(H.cpu().numpy().astype(np.float64), oracle.gram(bf16_bits(x))) <= GRAM_REL
+    assert nv.get_device_status() == "NVFP4_OK"
+
+
 # ------------------------------------------------------------ max rule
 def test_max_rule_bitexact_with_edge_blocks(nv):
     x = rand_bf16((67, 176), 2, 0.02, 0.01, 20.0)

@@ -39,6 +39,8 @@ def lib():
         L.oracle_global_scale.argtypes = [vp, i64, vp]
         L.oracle_max_rule_code.argtypes = [vp, f32]
         L.oracle_scale_search_max.argtypes = [vp, i64, i64, f32, vp]
+        L.oracle_four_over_six_code.argtypes = [vp, f32]
+        L.oracle_scale_search_four_over_six.argtypes = [vp, i64, i64, f32, vp]
         L.oracle_block_mse.restype = f64
         L.oracle_block_mse.argtypes = [vp, f32, i32]
         L.oracle_block_lh.restype = f64
@@ -119,6 +121,24 @@ def scale_search_max(w_u16, s_g):
     codes = np.zeros((R, C // 16), np.uint8)
     _check(lib().oracle_scale_search_max(_ptr(w), R, C, float(s_g), _ptr(codes)))
     return codes
+
+
+def scale_search_four_over_six(w_u16, s_g):
+    w = _u16(w_u16)
+    R, C = w.shape
+    codes = np.zeros((R, C // 16), np.uint8)
+    _check(lib().oracle_scale_search_four_over_six(_ptr(w), R, C, float(s_g), _ptr(codes)))
+    return codes
+
+
+def block_mse(blk_u16, s_g, code):
+    b = _u16(blk_u16).reshape(16)
+    return lib().oracle_block_mse(_ptr(b), ctypes.c_float(float(s_g)), int(code))
+
+
+def four_over_six_code(blk_u16, s_g):
+    b = _u16(blk_u16).reshape(16)
+    return lib().oracle_four_over_six_code(_ptr(b), ctypes.c_float(float(s_g)))
 
 
 def scale_search_mse(w_u16, s_g):

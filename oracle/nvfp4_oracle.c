@@ -336,6 +336,44 @@ int oracle_scale_search_sampled(const uint16_t *w, int64_t C, float s_g, const d
     return ORACLE_OK;
 }
 
+/* ------------------------------------------------------- Four Over Six */
+
+/* Four Over Six ([LH] "The NVFP4 structure": it chooses one of two
+ * candidate scales).  The pages do not name the two; the reading here: the
+ * max-rule scale, which puts the block amax on E2M1's largest magnitude 6,
+ * and the scale that puts it on 4, E4M3(amax / (4 s_g)) -- whichever gives
+ * the smaller block MSE, the smaller code on a tie.  An all-zero block gets
+ * code 0. */
+int oracle_four_over_six_code(const uint16_t *blk, float s_g)
+{
+    double amax = 0.0;
+    for (int i = 0; i < 16; i++) {
+        double v = fabs(oracle_bf16_to_double(blk[i]));
+        if (v > amax)
+            amax = v;
+    }
+    if (amax == 0.0)
+        return 0;
+    int c6 = oracle_e4m3_round_quotient(amax, 6.0 * (double)s_g);
+    int c4 = oracle_e4m3_round_quotient(amax, 4.0 * (double)s_g);
+    int lo = c4 < c6 ? c4 : c6, hi = c4 < c6 ? c6 : c4;
+    double e_lo = oracle_block_mse(blk, s_g, lo), e_hi = oracle_block_mse(blk, s_g, hi);
+    return e_hi < e_lo ? hi : lo;
+}
+
+int oracle_scale_search_four_over_six(const uint16_t *w, int64_t R, int64_t C, float s_g,
+                                      uint8_t *codes)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    int64_t nb = C / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t b = 0; b < nb; b++)
+            codes[r * nb + b] = (uint8_t)oracle_four_over_six_code(w + r * C + b * 16, s_g);
+    return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------- Gram */
 
 /* Block-diagonal Gram accumulation: for every column block j,

@@ -404,8 +404,9 @@ __global__ void __launch_bounds__(32)
   }
 }
 
+// Local-Hessian: at most 72 registers, seven CTAs per SM; MSE nine.
 template <bool kLH>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     search_kernel(const uint16_t *__restrict__ w, int64_t R, int64_t C,
                   const float *__restrict__ s_g_arr, const float *__restrict__ H,
                   const uint4 *__restrict__ frag, const Factor *__restrict__ fac,

@@ -388,3 +388,84 @@ def test_sampled_search_equals_full_search(oracle_mod):
     assert np.array_equal(c, full[rows, blocks]) and np.array_equal(o, fobj[rows, blocks])
     c, o = oracle_mod.scale_search_sampled(W, s_g, None, rows, blocks)
     assert np.array_equal(c, mfull[rows, blocks]) and np.array_equal(o, mobj[rows, blocks])
+
+
+# ------------------------------------------------------------ Four Over Six
+def _exact_block_mse(vals, s):
+    """Exact rational sum of squared errors of a block at scale s (brute-force
+    E2M1 codes by enumeration)."""
+    e = Fraction(0)
+    for x in vals:
+        k = brute_e2m1(float(x), float(s)) & 7
+        v = E2M1_MAG[k] * Fraction(s)
+        e += (abs(Fraction(float(x))) - v) ** 2
+    return e
+
+
+def _brute_four_over_six(vals, s_g, table):
+    amax = max(abs(Fraction(float(x))) for x in vals)
+    if amax == 0:
+        return 0
+    sg = Fraction(float(np.float32(s_g)))
+    c6 = brute_e4m3(amax / (6 * sg), table)
+    c4 = brute_e4m3(amax / (4 * sg), table)
+    lo, hi = min(c4, c6), max(c4, c6)
+    s_lo = Fraction(float(np.float32(np.float32(s_g) * np.float32(float(table[lo])))))
+    s_hi = Fraction(float(np.float32(np.float32(s_g) * np.float32(float(table[hi])))))
+    return hi if _exact_block_mse(vals, s_hi) < _exact_block_mse(vals, s_lo) else lo
+
+
+def test_four_over_six_closed_form_blocks(oracle_mod):
+    """Two blocks with tensor scale 1 and amax 48: the candidate scales are
+    48/6 = 8 (code 0x50) and 48/4 = 12 (code 0x54).  A block on the grid of
+    12 (0, 6, 12, 18, 24, 36, 48) has zero error there and not at 8 (36/8 =
+    4.5 rounds to 4): 0x54 wins.  A block on the grid of 8 (0, 4, 8, 12,
+    16, 24, 32, 48) with 32 in it (32/12 = 2.67 -> 3) is exact at 8 only:
+    0x50 wins."""
+    assert oracle_mod.e4m3_value(0x50) == 8.0 and oracle_mod.e4m3_value(0x54) == 12.0
+    on12 = [48, 36, 24, 18, 12, 6, 0, -6, -12, -18, -24, -36, 6, 12, 24, 36]
+    on8 = [48, 32, 24, 16, 12, 8, 4, 0, -4, -8, -12, -16, -24, -32, 8, 4]
+    u12 = f32_to_bf16_bits(np.array(on12, np.float32))
+    u8 = f32_to_bf16_bits(np.array(on8, np.float32))
+    assert oracle_mod.block_mse(u12, 1.0, 0x54) == 0.0 < oracle_mod.block_mse(u12, 1.0, 0x50)
+    assert oracle_mod.block_mse(u8, 1.0, 0x50) == 0.0 < oracle_mod.block_mse(u8, 1.0, 0x54)
+    assert oracle_mod.four_over_six_code(u12, 1.0) == 0x54
+    assert oracle_mod.four_over_six_code(u8, 1.0) == 0x50
+    assert oracle_mod.four_over_six_code(np.zeros(16, np.uint16), 1.0) == 0
+
+
+def test_four_over_six_brute_force_exact_rationals(oracle_mod):
+    """Random blocks (several magnitudes, one saturating the E4M3 range):
+    the oracle's choice equals the exact-rational argmin over the two
+    candidates."""
+    table = e4m3_table()
+    rng = np.random.default_rng(21)
+    for trial in range(120):
+        scale = 10.0 ** rng.uniform(-3, 2)
+        vals = rng.standard_normal(16) * scale
+        if trial % 10 == 0:
+            vals[rng.integers(16)] *= 40
+        u = f32_to_bf16_bits(vals.astype(np.float32))
+        x = bits_to_f64(u)
+        s_g = float(np.float32(np.abs(x).max() * (2.0 if trial % 3 == 0 else 0.4) / 2688.0))
+        assert oracle_mod.four_over_six_code(u, s_g) == _brute_four_over_six(x, s_g, table), trial
+
+
+def test_four_over_six_invariants(oracle_mod):
+    """c_46 is the max-rule code or E4M3(amax / (4 s_g)); its MSE is at most
+    the max rule's and at least the exhaustive MSE search's."""
+    wu, _ = _tiny_layer(32, 128, 8, 5)
+    sg = oracle_mod.global_scale(wu)
+    c46 = oracle_mod.scale_search_four_over_six(wu, sg)
+    cmax = oracle_mod.scale_search_max(wu, sg)
+    cmse, emse = oracle_mod.scale_search_mse(wu, sg)
+    R, nb = c46.shape
+    for r in range(R):
+        for b in range(nb):
+            blk = wu[r, 16 * b:16 * b + 16]
+            amax = np.abs(bits_to_f64(blk)).max()
+            c4 = oracle_mod.e4m3_round_quotient(amax, 4.0 * float(np.float32(sg)))
+            assert c46[r, b] in (cmax[r, b], c4)
+            e46 = oracle_mod.block_mse(blk, sg, int(c46[r, b]))
+            assert e46 <= oracle_mod.block_mse(blk, sg, int(cmax[r, b]))
+            assert emse[r, b] <= e46 * (1 + 1e-12)

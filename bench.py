@@ -49,7 +49,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
-WORKLOAD_NAMES = ["dense", "tiny", "moe", "mlp_pair", "w4a4"]
+WORKLOAD_NAMES = ["dense", "tiny", "moe", "mlp_pair", "w4a4", "four_over_six"]
 
 # Local-Hessian search work per block, counted on the definition E = delta
 # H_b delta^T: per candidate 256 FMA for H_b delta and 16 FMA for the dot
@@ -81,6 +81,7 @@ class Layer:
         self.H = torch.zeros(B, C // 16, 16, 16, dtype=torch.float32, device=dev)
         self.c_max = torch.empty(B, R, C // 16, dtype=torch.uint8, device=dev)
         self.c_mse = torch.empty_like(self.c_max)
+        self.c_46 = torch.empty_like(self.c_max)
         self.c_lh = torch.empty_like(self.c_max)
         self.packed = torch.empty(B, R, C // 2, dtype=torch.uint8, device=dev)
         self.deq = torch.empty(B, R, C, dtype=torch.bfloat16, device=dev)
@@ -108,6 +109,14 @@ class Runner:
             self.desc = wl.BY_NAME[workload].description
             self.rules = ["max", "mse", "lh"]
             self.fq_input = X
+        elif workload == "four_over_six":
+            # the dense projection's weights under the Four Over Six rule
+            W, _ = wl.layer_inputs("dense", device)
+            self.layers = [Layer("dense", W, None)]
+            self.desc = ("Four Over Six on the dense projection's W 4096x4096: global scale, "
+                         "the rule, pack, dequantise")
+            self.rules = ["four_over_six"]
+            self.fq_input = None
         elif workload == "moe":
             W, X, offsets = wl.moe_inputs(device)
             self.layers = [Layer("experts", W, X, offsets=offsets.to(device))]
@@ -161,25 +170,33 @@ class Runner:
                 rows.append((pre + "gram",
                              lambda L=L: nv.hessian_accumulate_grouped(L.X, L.offsets, L.H),
                              2 * L.X.numel() + 2 * h, 3))
-            else:
+            elif L.X is not None:
                 rows.append((pre + "gram", lambda L=L: nv.hessian_accumulate(L.X, L.H[0]),
                              2 * L.X.numel() + 2 * h, 2))
             if "max" in self.rules:
                 rows.append((pre + "search_max",
                              lambda L=L: nv.scale_search_max(L.W, L.s_g, out=L.c_max),
                              2 * n_w + nb, 1))
+            if "four_over_six" in self.rules:
+                rows.append((pre + "search_four_over_six",
+                             lambda L=L: nv.scale_search_four_over_six(L.W, L.s_g, out=L.c_46),
+                             2 * n_w + nb, 1))
             if "mse" in self.rules:
                 rows.append((pre + "search_mse",
                              lambda L=L: nv.scale_search_mse(L.W, L.s_g, out=L.c_mse),
                              2 * n_w + nb, 1))
-            rows.append((pre + "search_lh",
-                         lambda L=L: nv.scale_search_local_hessian(L.W, L.s_g, L.H, out=L.c_lh),
-                         2 * n_w + nb + h, 2))  # factor_kernel + search_kernel
+            if "lh" in self.rules:
+                rows.append((pre + "search_lh",
+                             lambda L=L: nv.scale_search_local_hessian(L.W, L.s_g, L.H,
+                                                                       out=L.c_lh),
+                             2 * n_w + nb + h, 2))  # factor_kernel + search_kernel
+            # pack and dequantise with the codes of the workload's final rule
+            fin = L.c_lh if "lh" in self.rules else L.c_46
             rows.append((pre + "quantize_pack",
-                         lambda L=L: nv.quantize_pack(L.W, L.s_g, L.c_lh, out=L.packed),
+                         lambda L=L, c=fin: nv.quantize_pack(L.W, L.s_g, c, out=L.packed),
                          2 * n_w + nb + n_w // 2, 1))
             rows.append((pre + "dequantize",
-                         lambda L=L: nv.dequantize(L.packed, L.c_lh, L.s_g, out=L.deq),
+                         lambda L=L, c=fin: nv.dequantize(L.packed, c, L.s_g, out=L.deq),
                          n_w // 2 + nb + 2 * n_w, 1))
         if self.fq_input is not None:
             n_x = self.fq_input.numel()
@@ -220,7 +237,7 @@ class Runner:
     def results(self):
         out = []
         for L in self.layers:
-            out += [L.c_lh, L.packed]
+            out += [L.c_lh if "lh" in self.rules else L.c_46, L.packed]
         if self.workload == "w4a4":
             out += [self.fq_packed, self.fq_codes]
         return out
@@ -466,6 +483,18 @@ def make_roofline(run, kernels, pk, pk_kind, workload, lh_evals):
             "evaluated_per_block": round(lh_evals / run.blocks(), 2),
             "all_126_equivalent_TFLOP/s": round(brute, 2),
         }
+    if "search_four_over_six" in kernels:
+        # a streaming pass over W (2 B per value read, a code byte per 16
+        # written); the exact encode of its two candidates is what bounds it
+        ms = kernels["search_four_over_six"]["ms"]
+        n = run.blocks() * 16
+        achieved = (2 * n + n // 16) / (ms / 1e3) / 1e9
+        hbm = float(pk.get("hbm_gbs", FALLBACK_HBM_GBS))
+        return {"kernel": "four_over_six_kernel", "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                "traffic": None, "peak_kind": "%s HBM copy bandwidth" % pk_kind,
+                "bytes_per_element": 2 + 1 / 16,
+                "note": "issue-bound on the exact E2M1 encode of both candidates"}
     ms = kernels["fake_quant"]["ms"]
     n = run.fq_input.numel()
     achieved = FAKE_QUANT_BYTES_PER_ELEM * n / (ms / 1e3) / 1e9
@@ -550,24 +579,27 @@ def cpu_baseline(run, budget_s=15.0):
         X = L.X[int(L.offsets[0]):int(L.offsets[1])]
     else:
         X = L.X
-    n_tok_total = L.tokens() if L.offsets is None else X.shape[0]
+    n_tok_total = 0 if X is None else (L.tokens() if L.offsets is None else X.shape[0])
 
     def path(rows):
         frac = rows / R
-        x_rows = min(X.shape[0], max(16, int(n_tok_total * frac)))
-        xu = _bits(X[:x_rows])
+        x_rows = 0 if X is None else min(X.shape[0], max(16, int(n_tok_total * frac)))
+        xu = None if X is None else _bits(X[:x_rows])
         fq = None
         if run.fq_input is not None:
             fq = _bits(run.fq_input[:max(1, int(run.fq_input.shape[0] * frac))])
         t0 = time.perf_counter()
         sg = oracle.global_scale(wu_all)
-        H = oracle.gram(xu)
+        H = None if xu is None else oracle.gram(xu)
         wu = np.ascontiguousarray(wu_all[:rows])
         if "max" in run.rules:
             oracle.scale_search_max(wu, sg)
+        if "four_over_six" in run.rules:
+            codes = oracle.scale_search_four_over_six(wu, sg)
         if "mse" in run.rules:
             oracle.scale_search_mse(wu, sg)
-        codes, _ = oracle.scale_search_lh(wu, sg, H)
+        if "lh" in run.rules:
+            codes, _ = oracle.scale_search_lh(wu, sg, H)
         packed = oracle.quantize_pack(wu, sg, codes)
         oracle.dequantize(packed, codes, sg)
         if fq is not None:
@@ -595,7 +627,7 @@ def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
         return
-    small = args.workload in ("tiny", "dense", "w4a4")
+    small = args.workload in ("tiny", "dense", "w4a4", "four_over_six")
     dev = "cpu" if small or not torch.cuda.is_available() else "cuda"
     run = Runner(args.workload, dev)
     budget = args.cpu_seconds / max(1, args.steps)

@@ -152,6 +152,20 @@ nvfp4_status nvfp4_scale_search_max(const uint16_t *w, int64_t batch, int64_t R,
                                     const float *s_g, uint8_t *scale_codes, void *stream);
 
 /*
+ * Four Over Six ([LH] "The NVFP4 structure": the rule picks one of two
+ * candidate scales per block).  The two are not named on the pages; the
+ * reading: the max-rule code (block amax onto E2M1's 6) and the code of
+ * amax_b / (4 * s_g) (block amax onto 4), both rounded as the max rule
+ * rounds; the one with the smaller block MSE sum_i (w_i - v(q_i) s_eff)^2
+ * wins, the smaller code on a tie; an all-zero block gets code 0.  The two
+ * objectives are evaluated in fp64 with the definition's operations in its
+ * order, so the choice is exact.  Arguments as nvfp4_scale_search_max.
+ */
+nvfp4_status nvfp4_scale_search_four_over_six(const uint16_t *w, int64_t batch, int64_t R,
+                                              int64_t C, const float *s_g, uint8_t *scale_codes,
+                                              void *stream);
+
+/*
  * MSE rule ([LH] "The NVFP4 structure"): for every block, the code in
  * 1..126 minimising sum_i (w_i - v(q_i) s_eff)^2, q_i the E2M1 code of w_i at
  * s_eff; the smallest code wins a tie.  Candidates are screened in fp32 and

@@ -165,6 +165,15 @@ nvfp4_status nvfp4_scale_search_max(const uint16_t *w, int64_t batch, int64_t R,
                                           as_stream(stream)));
 }
 
+nvfp4_status nvfp4_scale_search_four_over_six(const uint16_t *w, int64_t batch, int64_t R,
+                                              int64_t C, const float *s_g, uint8_t *scale_codes,
+                                              void *stream) {
+  nvfp4_status st = check_weight_args(w, batch, R, C, s_g, scale_codes);
+  if (st != NVFP4_OK) return st;
+  return map_cuda(nvfp4::launch_four_over_six(w, batch, R * C / 16, s_g, scale_codes,
+                                              as_stream(stream)));
+}
+
 nvfp4_status nvfp4_scale_search_mse(const uint16_t *w, int64_t batch, int64_t R, int64_t C,
                                     const float *s_g, uint8_t *scale_codes, float *best_obj,
                                     void *stream) {

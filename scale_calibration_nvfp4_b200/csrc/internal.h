@@ -11,6 +11,8 @@ cudaError_t launch_global_scale(const uint16_t *x, int64_t batch, int64_t n_per_
                                 float *s_g, cudaStream_t st);
 cudaError_t launch_scale_max(const uint16_t *w, int64_t batch, int64_t nblk, const float *s_g,
                              uint8_t *codes, cudaStream_t st);
+cudaError_t launch_four_over_six(const uint16_t *w, int64_t batch, int64_t nblk,
+                                 const float *s_g, uint8_t *codes, cudaStream_t st);
 cudaError_t launch_pack(const uint16_t *w, int64_t batch, int64_t nblk, const float *s_g,
                         const uint8_t *codes, uint8_t *packed, cudaStream_t st);
 cudaError_t launch_dequant(const uint8_t *packed, const uint8_t *codes, const float *s_g,

@@ -215,17 +215,18 @@ __device__ __forceinline__ void fill_scale_table(ScaleEntry *tab, float sg) {
   __syncthreads();
 }
 
-// E4M3 code of amax / (6 s_g), exact (nearest even, saturating at 448), from
-// D = 6 s_g (exact in fp64) and R = 1/D split as r_hi + r_lo: t = amax R, the
+// E4M3 code of amax / (k s_g) (k = 6: the max rule; k = 4: the second
+// candidate of Four Over Six), exact (nearest even, saturating at 448), from
+// D = k s_g (exact in fp64) and R = 1/D split as r_hi + r_lo: t = amax R, the
 // residual amax - t D is exact in one fp64 fma, and the same odd-code rule
 // picks between the two e4m3x2 conversions.
 struct MaxRule {
   double D;
   float r_hi, r_lo;
 };
-__device__ __forceinline__ MaxRule make_max_rule(float s_g) {
+__device__ __forceinline__ MaxRule make_max_rule(float s_g, double k = 6.0) {
   MaxRule m;
-  m.D = 6.0 * (double)s_g;
+  m.D = k * (double)s_g;
   const double R = 1.0 / m.D;
   m.r_hi = (float)R;
   m.r_lo = (float)(R - (double)m.r_hi);
@@ -277,6 +278,91 @@ __global__ void __launch_bounds__(kThreads) max_rule_kernel(const uint16_t *__re
     load_block(w + i * kBlock, v);
     const float amax = __uint_as_float(amax_bits8(v) << 16);
     codes[i] = (uint8_t)max_rule_code_fast(amax, mr);
+  }
+}
+
+// Signed E2M1 value of code i of a packed block (fp32, exact).
+__device__ __forceinline__ float e2m1_code_value(uint2 q, int i) {
+  const uint32_t code = ((i < 8 ? q.x : q.y) >> (4 * (i & 7))) & 0xFu;
+  const uint32_t k = code & 7u;
+  const float mag = k < 2 ? 0.5f * k : (1.0f + 0.5f * (float)(k & 1u)) * (float)(1 << ((k >> 1) - 1));
+  return (code & 8u) ? -mag : mag;
+}
+
+// Block MSE at scale s in fp32 (a screen: every d_i is rounded once and the
+// 16 non-negative terms are summed with one rounding each, so the relative
+// error stays below 2^-20).  Codes back to values by the hardware e2m1x2 ->
+// f16x2 conversion (exact).
+__device__ __forceinline__ float block_mse32(const uint32_t w[8], uint2 q, float s) {
+  float e = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t byte = ((j < 4 ? q.x : q.y) >> (8 * (j & 3))) & 0xFFu;
+    const uint32_t h2 = cvt_f16x2_from_e2m1x2(byte);
+    const float d0 = fmaf(-f16_lo_to_float(h2), s, bf16_lo(w[j]));
+    const float d1 = fmaf(-f16_hi_to_float(h2), s, bf16_hi(w[j]));
+    e = fmaf(d0, d0, e);
+    e = fmaf(d1, d1, e);
+  }
+  return e;
+}
+
+// Block MSE at the table entry's scale in fp64, with the operations of the
+// definition in its order: d_i = w_i - v_i s, e += d_i^2, i = 0..15, each
+// product and sum rounded on its own (no fused multiply-add), so that two
+// candidates compare exactly as in the definition.
+__device__ __noinline__ double block_mse64(const uint32_t w[8], uint2 q, float sf) {
+  const double s = (double)sf;
+  double e = 0.0;
+#pragma unroll 1
+  for (int i = 0; i < 16; ++i) {
+    const double v = (double)e2m1_code_value(q, i);
+    const double x = (double)((i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]));
+    const double d = __dsub_rn(x, __dmul_rn(v, s));
+    e = __dadd_rn(e, __dmul_rn(d, d));
+  }
+  return e;
+}
+
+// Four Over Six (the Local-Hessian write-up, "The NVFP4 structure": one of
+// two candidate scales per block): the max-rule code and the code of
+// amax / (4 s_g), whichever block MSE is smaller, the smaller code on a tie;
+// an all-zero block gets code 0.
+__global__ void __launch_bounds__(kThreads) four_over_six_kernel(const uint16_t *__restrict__ w,
+                                                                 int64_t nblk,
+                                                                 const float *__restrict__ s_g,
+                                                                 uint8_t *__restrict__ codes) {
+  const int64_t b = blockIdx.y;
+  w += b * nblk * kBlock;
+  codes += b * nblk;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  uint32_t v[8];
+  if (i < nblk) load_block(w + i * kBlock, v);
+  // the table is built while the first block is in flight
+  const float sg = s_g[b];
+  const MaxRule m6 = make_max_rule(sg, 6.0), m4 = make_max_rule(sg, 4.0);
+  __shared__ ScaleEntry tab[256];
+  fill_scale_table(tab, sg);
+  for (; i < nblk; i += stride) {
+    uint32_t nv[8];
+    const int64_t n = i + stride;
+    if (n < nblk) load_block(w + n * kBlock, nv);
+    const float amax = __uint_as_float(amax_bits8(v) << 16);
+    const uint32_t c6 = max_rule_code_fast(amax, m6), c4 = max_rule_code_fast(amax, m4);
+    const uint32_t lo = min(c4, c6), hi = max(c4, c6);
+    uint32_t code = lo;
+    if (amax > 0.0f && hi != lo) {
+      // fp32 screen; the exact fp64 comparison only when the two are close
+      const ScaleEntry el = tab[lo], eh = tab[hi];
+      const uint2 ql = encode_block_entry(v, el), qh = encode_block_entry(v, eh);
+      const float fl = block_mse32(v, ql, el.s), fh = block_mse32(v, qh, eh.s);
+      if (fabsf(fh - fl) > 0x1p-16f * fmaxf(fh, fl)) code = fh < fl ? hi : lo;
+      else code = block_mse64(v, qh, eh.s) < block_mse64(v, ql, el.s) ? hi : lo;
+    }
+    codes[i] = (uint8_t)(amax > 0.0f ? code : 0u);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = nv[j];
   }
 }
 
@@ -418,6 +504,14 @@ cudaError_t launch_scale_max(const uint16_t *w, int64_t batch, int64_t nblk, con
   if (nblk == 0) return cudaSuccess;
   int gx = grid_for(nblk, 16);
   max_rule_kernel<<<dim3(gx, (unsigned)batch), kThreads, 0, st>>>(w, nblk, s_g, codes);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_four_over_six(const uint16_t *w, int64_t batch, int64_t nblk,
+                                 const float *s_g, uint8_t *codes, cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  const int gx = grid_for(nblk, 8);
+  four_over_six_kernel<<<dim3(gx, (unsigned)batch), kThreads, 0, st>>>(w, nblk, s_g, codes);
   return cudaGetLastError();
 }
 

@@ -29,6 +29,7 @@ SIGNATURES = {
     "nvfp4_hessian_accumulate_noalloc": [_vp, _i64, _i64, _vp, _vp],
     "nvfp4_hessian_accumulate_grouped": [_vp, _vp, _i64, _i64, _i64, _vp, _vp],
     "nvfp4_scale_search_max": [_vp, _i64, _i64, _i64, _vp, _vp, _vp],
+    "nvfp4_scale_search_four_over_six": [_vp, _i64, _i64, _i64, _vp, _vp, _vp],
     "nvfp4_scale_search_mse": [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp],
     "nvfp4_scale_search_local_hessian": [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp],
     "nvfp4_quantize_pack": [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp],
@@ -180,6 +181,15 @@ def scale_search_max(w, s_g, out=None, stream=None):
     B, R, C = _weight_shape(w)
     out = _codes_out(w, out)
     _call("nvfp4_scale_search_max", _p(w), B, R, C, _p(s_g), _p(out), _stream(stream))
+    return out
+
+
+def scale_search_four_over_six(w, s_g, out=None, stream=None):
+    _need(w, torch.bfloat16, "w")
+    _need(s_g, torch.float32, "s_g")
+    B, R, C = _weight_shape(w)
+    out = _codes_out(w, out)
+    _call("nvfp4_scale_search_four_over_six", _p(w), B, R, C, _p(s_g), _p(out), _stream(stream))
     return out
 
 

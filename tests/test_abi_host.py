@@ -61,6 +61,9 @@ BAD = 0x10001  # misaligned
 def test_validation_rejects_before_launch(L):
     # shape: C not a multiple of 16
     assert L.nvfp4_scale_search_max(P, 1, 4, 17, P, P, None) == SHAPE
+    assert L.nvfp4_scale_search_four_over_six(P, 1, 4, 17, P, P, None) == SHAPE
+    assert L.nvfp4_scale_search_four_over_six(BAD, 1, 4, 16, P, P, None) == MISALIGNED
+    assert L.nvfp4_scale_search_four_over_six(None, 1, 4, 16, P, P, None) == INVALID
     assert L.nvfp4_scale_search_mse(P, 1, 4, 24, P, P, None, None) == SHAPE
     assert L.nvfp4_scale_search_local_hessian(P, 1, 4, 40, P, P, P, None, None) == SHAPE
     assert L.nvfp4_quantize_pack(P, 1, 4, 8, P, P, P, None) == SHAPE

@@ -306,6 +306,32 @@ def test_tiny_layer_all_rules(nv):
     assert n_tie_mse + n_tie_lh < 10
 
 
+def test_four_over_six_bitexact(nv):
+    """Four Over Six on every block of the tiny layer, a batch of experts
+    with their own tensor scales, a ragged shape with zero, saturating,
+    on-grid and tiny blocks: equal to the oracle block by block."""
+    W, _ = _layer("tiny")
+    s_g = nv.global_scale(W)
+    c = nv.scale_search_four_over_six(W, s_g).cpu().numpy()
+    np.testing.assert_array_equal(c, oracle.scale_search_four_over_six(bf16_bits(W), s_g.item()))
+    Wb = rand_bf16((3, 40, 96), 17, 0.02, 0.02, 30.0)
+    sb = nv.global_scale(Wb.cuda(), batch=3)
+    cb = nv.scale_search_four_over_six(Wb.cuda(), sb).cpu().numpy()
+    for e in range(3):
+        np.testing.assert_array_equal(cb[e], oracle.scale_search_four_over_six(bf16_bits(Wb[e]), sb[e].item()))
+    x = rand_bf16((37, 80), 23, 0.5)
+    x[0, :16] = 0
+    x[1, 16:32] = x.abs().max()                     # saturating candidate(s)
+    x[2, 32:48] = 1e-6 * x[2, 32:48]                # tiny block (codes near 0)
+    grid = torch.tensor([48, 36, 24, 18, 12, 6, 0, -6, -12, -18, -24, -36, 6, 12, 24, 36.0])
+    x[3, :16] = (grid / 1024).to(torch.bfloat16)    # on the grid of the amax/4 scale
+    s = nv.global_scale(x.cuda())
+    cx = nv.scale_search_four_over_six(x.cuda(), s).cpu().numpy()
+    rx = oracle.scale_search_four_over_six(bf16_bits(x), s.item())
+    np.testing.assert_array_equal(cx, rx)
+    assert cx[0, 0] == 0
+
+
 def test_identity_hessian_gives_mse_on_gpu(nv):
     W, _ = _layer("tiny")
     s_g = nv.global_scale(W)
@@ -401,6 +427,15 @@ def test_search_evaluation_counters(nv):
     m2, l2 = nv.search_evaluations(reset=True)
     assert m2 == m and 2 * blocks <= l2 <= 2 * 126 * blocks and l2 % 2 == 0
     assert nv.search_evaluations() == (0, 0)
+
+
+def test_four_over_six_dense_layer_every_block(nv):
+    """Dense 4096x4096 workload, every block (the oracle's two-candidate
+    rule is cheap enough for the full layer)."""
+    W, _ = _layer("dense")
+    s_g = nv.global_scale(W)
+    c = nv.scale_search_four_over_six(W, s_g).cpu().numpy()
+    np.testing.assert_array_equal(c, oracle.scale_search_four_over_six(bf16_bits(W), s_g.item()))
 
 
 def test_dense_layer_sampled(nv):

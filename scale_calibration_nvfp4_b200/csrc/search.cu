@@ -682,12 +682,12 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
           if ((e & 2) == 0) ug = fmaf(v, v, ug);
           else ug8 = fmaf(v, v, ug8);
         }
-        ug += __shfl_xor_sync(0xFFFFFFFFu, ug, 1);
-        ug += __shfl_xor_sync(0xFFFFFFFFu, ug, 2);
-        ug8 += __shfl_xor_sync(0xFFFFFFFFu, ug8, 1);
-        ug8 += __shfl_xor_sync(0xFFFFFFFFu, ug8, 2);
+        // the same quad reduce-scatter as the objective: lanes t < 2 keep row g
+        float zero_sum = upper ? ug8 : ug;
+        zero_sum += __shfl_xor_sync(0xFFFFFFFFu, upper ? ug : ug8, 2);
+        zero_sum += __shfl_xor_sync(0xFFFFFFFFu, zero_sum, 1);
         const bool done = amax_row == 0.0f ||
-                          zl2 * (upper ? ug8 : ug) * (1.0f - 2.0f * kTieBand) > b1 + row_floor;
+                          zl2 * zero_sum * (1.0f - 2.0f * kTieBand) > b1 + row_floor;
         if (__all_sync(0xFFFFFFFFu, done)) break;
         const float e0 =
             alt ? candidate_objective<kLH, true>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper)

@@ -40,6 +40,7 @@ def lib():
         L.oracle_max_rule_code.argtypes = [vp, f32]
         L.oracle_scale_search_max.argtypes = [vp, i64, i64, f32, vp]
         L.oracle_four_over_six_code.argtypes = [vp, f32]
+        L.oracle_gemm_nvfp4.argtypes = [vp, vp, f32, vp, vp, f32, i64, i64, i64, vp, vp]
         L.oracle_scale_search_four_over_six.argtypes = [vp, i64, i64, f32, vp]
         L.oracle_block_mse.restype = f64
         L.oracle_block_mse.argtypes = [vp, f32, i32]
@@ -139,6 +140,22 @@ def block_mse(blk_u16, s_g, code):
 def four_over_six_code(blk_u16, s_g):
     b = _u16(blk_u16).reshape(16)
     return lib().oracle_four_over_six_code(_ptr(b), ctypes.c_float(float(s_g)))
+
+
+def gemm_nvfp4(a_packed, a_codes, a_sg, b_packed, b_codes, b_sg):
+    """Y = dequant(A) dequant(B)^T in fp64 (exact products), and the sum of
+    the terms' magnitudes; A [M, K], B [N, K] as packed codes [*, K/2] and
+    block codes [*, K/16]."""
+    ap = np.ascontiguousarray(a_packed, np.uint8)
+    ac = np.ascontiguousarray(a_codes, np.uint8)
+    bp = np.ascontiguousarray(b_packed, np.uint8)
+    bc = np.ascontiguousarray(b_codes, np.uint8)
+    M, N, K = ap.shape[0], bp.shape[0], ap.shape[1] * 2
+    Y = np.zeros((M, N), np.float64)
+    A = np.zeros((M, N), np.float64)
+    _check(lib().oracle_gemm_nvfp4(_ptr(ap), _ptr(ac), float(a_sg), _ptr(bp), _ptr(bc),
+                                   float(b_sg), M, N, K, _ptr(Y), _ptr(A)))
+    return Y, A
 
 
 def scale_search_mse(w_u16, s_g):

@@ -374,6 +374,48 @@ int oracle_scale_search_four_over_six(const uint16_t *w, int64_t R, int64_t C, f
     return ORACLE_OK;
 }
 
+/* ------------------------------------------------------ W4A4 GEMM */
+
+/* The matrix product both NVFP4 operands stand for: with A [M, K] and
+ * B [N, K] (row-major, K contiguous) given as packed E2M1 codes, one E4M3
+ * code per 16 consecutive values and an FP32 tensor scale each,
+ *   Y[m][n] = s_ga s_gb sum_k (v(a_mk) e4m3(ca_m,k/16)) (v(b_nk) e4m3(cb_n,k/16))
+ * in fp64 (every product is exact; the sum runs over k in order), and
+ * absY[m][n] = the same sum of the terms' magnitudes (for tolerances).
+ * [W4A4] (weights and activations both NVFP4); [BT] "Block scaling" (a value
+ * is its E2M1 code times its block scale times the tensor scale). */
+static double nvfp4_value(const uint8_t *packed, const uint8_t *codes, int64_t row, int64_t K,
+                          int64_t k)
+{
+    uint8_t byte = packed[row * (K / 2) + k / 2];
+    int q = (k & 1) ? (byte >> 4) : (byte & 15);
+    return oracle_e2m1_value(q) * oracle_e4m3_value(codes[row * (K / 16) + k / 16]);
+}
+
+int oracle_gemm_nvfp4(const uint8_t *a_packed, const uint8_t *a_codes, float a_sg,
+                      const uint8_t *b_packed, const uint8_t *b_codes, float b_sg, int64_t M,
+                      int64_t N, int64_t K, double *Y, double *absY)
+{
+    if (K % 16)
+        return ORACLE_ERR_SHAPE;
+    double g = (double)a_sg * (double)b_sg;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                double t = nvfp4_value(a_packed, a_codes, m, K, k) *
+                           nvfp4_value(b_packed, b_codes, n, K, k);
+                acc += t;
+                aacc += fabs(t);
+            }
+            Y[m * N + n] = acc * g;
+            if (absY)
+                absY[m * N + n] = aacc * fabs(g);
+        }
+    return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------- Gram */
 
 /* Block-diagonal Gram accumulation: for every column block j,

@@ -4,8 +4,10 @@
 
 Each ``csrc/*.cu`` file is compiled by nvcc for ``arch=compute_100a,
 code=sm_100a`` and linked into ``scale_calibration_nvfp4_b200/libnvfp4.so``
-with the static CUDA runtime.  Rebuilds only when a source or header is newer
-than the library.
+with the static CUDA runtime.  Objects are rebuilt only when their source, a
+shared header or this script is newer; the library is relinked when an object
+is.  Sources that instantiate CUTLASS/CuTe templates (the FP4 GEMM) get the
+header tree vendored in the environment's site-packages.
 """
 import glob
 import os
@@ -42,11 +44,47 @@ def _inputs():
     return files
 
 
+def _shared_inputs():
+    files = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
+    files += glob.glob(os.path.join(ROOT, "include", "*.h"))
+    files.append(os.path.abspath(__file__))
+    return files
+
+
+def cutlass_include():
+    """CUTLASS/CuTe headers vendored with flashinfer (header-only use)."""
+    import importlib.util
+    spec = importlib.util.find_spec("flashinfer")
+    for base in (spec.submodule_search_locations or []) if spec else []:
+        inc = os.path.join(base, "data", "cutlass", "include")
+        util = os.path.join(base, "data", "cutlass", "tools", "util", "include")
+        if os.path.isdir(os.path.join(inc, "cute")):
+            return [inc, util]
+    raise RuntimeError("CUTLASS/CuTe headers not found (expected under flashinfer/data/cutlass)")
+
+
+def _uses_cutlass(src):
+    with open(src) as f:
+        return "#include <cute/" in f.read()
+
+
+def _obj(src):
+    return os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
+
+
+def _stale(src, obj):
+    if not os.path.exists(obj):
+        return True
+    t = os.path.getmtime(obj)
+    return any(os.path.getmtime(f) > t for f in [src] + _shared_inputs())
+
+
 def up_to_date():
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(f) <= t for f in _inputs())
+    return all(os.path.getmtime(f) <= t for f in _inputs()) and \
+        all(os.path.exists(_obj(s)) and os.path.getmtime(_obj(s)) <= t for s in sources())
 
 
 def build(force=False, verbose=False, ptxas_info=False):
@@ -56,14 +94,20 @@ def build(force=False, verbose=False, ptxas_info=False):
     os.makedirs(BUILD_DIR, exist_ok=True)
     objs = []
     for src in sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
-        cmd = [nvcc] + ARCH + NVCC_FLAGS + ["-c", src, "-o", obj]
+        obj = _obj(src)
+        objs.append(obj)
+        if not (force or ptxas_info or _stale(src, obj)):
+            continue
+        cmd = [nvcc] + ARCH + NVCC_FLAGS
+        if _uses_cutlass(src):
+            cmd += ["--expt-relaxed-constexpr", "-Xcompiler", "-Wno-unused-parameter"]
+            cmd += ["-I" + d for d in cutlass_include()]
+        cmd += ["-c", src, "-o", obj]
         if ptxas_info:
             cmd += ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd))
         subprocess.run(cmd, check=True)
-        objs.append(obj)
     tmp = LIB + ".tmp.%d" % os.getpid()
     cmd = [nvcc] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
     if verbose:

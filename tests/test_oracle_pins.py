@@ -469,3 +469,43 @@ def test_four_over_six_invariants(oracle_mod):
             e46 = oracle_mod.block_mse(blk, sg, int(c46[r, b]))
             assert e46 <= oracle_mod.block_mse(blk, sg, int(cmax[r, b]))
             assert emse[r, b] <= e46 * (1 + 1e-12)
+
+
+# ------------------------------------------------------------ W4A4 GEMM
+def _decode_nvfp4(packed, codes):
+    """Exact values of packed NVFP4 rows, decoded without the oracle: the
+    E2M1 magnitudes listed on the pages and torch's float8_e4m3fn decode."""
+    lo, hi = packed & 15, packed >> 4
+    q = np.stack([lo, hi], -1).reshape(packed.shape[0], -1)
+    mag = np.array([float(v) for v in E2M1_MAG])[q & 7]
+    v = np.where(q & 8, -mag, mag)
+    sf = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return v * np.repeat(sf, 16, axis=1)
+
+
+def test_gemm_oracle_equals_library_matmul_of_decoded_operands(oracle_mod):
+    rng = np.random.default_rng(31)
+    M, N, K = 7, 5, 96
+    ap = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    bp = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    ac = rng.integers(0, 127, (M, K // 16), dtype=np.uint8)
+    bc = rng.integers(0, 127, (N, K // 16), dtype=np.uint8)
+    sa, sb = float(np.float32(0.0123)), float(np.float32(3.5))
+    Y, absY = oracle_mod.gemm_nvfp4(ap, ac, sa, bp, bc, sb)
+    A, B = _decode_nvfp4(ap, ac), _decode_nvfp4(bp, bc)
+    ref = (A @ B.T) * (sa * sb)
+    np.testing.assert_allclose(Y, ref, rtol=1e-13, atol=1e-300)
+    np.testing.assert_allclose(absY, (np.abs(A) @ np.abs(B).T) * abs(sa * sb), rtol=1e-13)
+
+
+def test_gemm_oracle_hand_case(oracle_mod):
+    """One row of A with codes 1.0 (0x2) everywhere at block scale 2 and one
+    row of B with 6.0 (0x7) at block scale 0.5 over K = 32: Y = 32 * 2 * 3."""
+    ap = np.full((1, 16), 0x22, np.uint8)
+    bp = np.full((1, 16), 0x77, np.uint8)
+    two = torch.tensor([2.0]).to(torch.float8_e4m3fn).view(torch.uint8).item()
+    half = torch.tensor([0.5]).to(torch.float8_e4m3fn).view(torch.uint8).item()
+    ac = np.full((1, 2), two, np.uint8)
+    bc = np.full((1, 2), half, np.uint8)
+    Y, _ = oracle_mod.gemm_nvfp4(ap, ac, 1.0, bp, bc, 1.0)
+    assert Y[0, 0] == 32 * (1.0 * 2.0) * (6.0 * 0.5)

@@ -49,7 +49,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
-WORKLOAD_NAMES = ["dense", "tiny", "moe", "mlp_pair", "w4a4", "four_over_six"]
+WORKLOAD_NAMES = ["dense", "tiny", "moe", "mlp_pair", "w4a4", "four_over_six", "w4a4_gemm"]
 
 # Local-Hessian search work per block, counted on the definition E = delta
 # H_b delta^T: per candidate 256 FMA for H_b delta and 16 FMA for the dot
@@ -132,6 +132,23 @@ class Runner:
             self.desc = wl.BY_NAME["mlp_pair"].description
             self.rules = ["lh"]
             self.fq_input = None
+        elif workload == "w4a4_gemm":
+            # the W4A4 activations times an 8192x8192 NVFP4 weight: per step the
+            # dynamic fake-quant of X (packed outputs) and the product
+            X = wl.w4a4_inputs(device)
+            self.layers = []
+            self.desc = ("W4A4 layer: X 32768x8192 dynamic NVFP4 (fake-quant with packed "
+                         "outputs) times W 8192x8192 NVFP4 (seed 9, N(0,0.02), quantised once)")
+            self.rules = []
+            self.fq_input = X
+            g = torch.Generator(device=X.device).manual_seed(9)
+            W = (torch.randn(8192, 8192, generator=g, device=X.device) * 0.02).to(torch.bfloat16)
+            self.gemm_w = W
+            if X.is_cuda:
+                self.gw_sg = nvfp4.global_scale(W)
+                self.gw_codes = nvfp4.scale_search_max(W, self.gw_sg)
+                self.gw_packed = nvfp4.quantize_pack(W, self.gw_sg, self.gw_codes)
+                self.gemm_out = torch.empty(X.shape[0], 8192, dtype=torch.bfloat16, device=X.device)
         elif workload == "w4a4":
             X = wl.w4a4_inputs(device)
             self.layers = []
@@ -200,7 +217,18 @@ class Runner:
                          n_w // 2 + nb + 2 * n_w, 1))
         if self.fq_input is not None:
             n_x = self.fq_input.numel()
-            if self.workload == "w4a4":
+            if self.workload == "w4a4_gemm":
+                X = self.fq_input
+                M, K, N = X.shape[0], X.shape[1], self.gemm_w.shape[0]
+                rows.append(("fake_quant", lambda: self._fq(True),
+                             FAKE_QUANT_BYTES_PER_ELEM * n_x, 3))
+                if X.is_cuda:
+                    rows.append(("gemm", lambda: nv.gemm(self.fq_packed, self.fq_codes, self.fq_sg,
+                                                          self.gw_packed, self.gw_codes,
+                                                          self.gw_sg,
+                                                          out=self.gemm_out),
+                                 M * K // 2 + N * K // 2 + M * N * 2, 7))
+            elif self.workload == "w4a4":
                 rows.append(("fake_quant", lambda: self._fq(True),
                              FAKE_QUANT_BYTES_PER_ELEM * n_x, 3))
             else:
@@ -240,6 +268,8 @@ class Runner:
             out += [L.c_lh if "lh" in self.rules else L.c_46, L.packed]
         if self.workload == "w4a4":
             out += [self.fq_packed, self.fq_codes]
+        if self.workload == "w4a4_gemm":
+            out += [self.gemm_out]
         return out
 
 
@@ -483,6 +513,18 @@ def make_roofline(run, kernels, pk, pk_kind, workload, lh_evals):
             "evaluated_per_block": round(lh_evals / run.blocks(), 2),
             "all_126_equivalent_TFLOP/s": round(brute, 2),
         }
+    if "gemm" in kernels:
+        X = run.fq_input
+        M, K, N = X.shape[0], X.shape[1], run.gw_packed.shape[0]
+        ms = kernels["gemm"]["ms"]
+        achieved = 2.0 * M * N * K / (ms / 1e3) / 1e12
+        bf16 = float(pk.get("bf16_tflops", 1595.8))
+        peak = 4.0 * bf16
+        return {"kernel": "NVFP4 GEMM (scale layout + block-scaled tcgen05 MMA)", "bound": "tensor",
+                "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "peak_kind": "%s bf16 GEMM burst x 4 (nominal dense FP4/BF16 ratio 9/2.25)" % pk_kind,
+                "flop_basis": "2 M N K, M=%d N=%d K=%d" % (M, N, K)}
     if "search_four_over_six" in kernels:
         # a streaming pass over W (2 B per value read, a code byte per 16
         # written); the exact encode of its two candidates is what bounds it
@@ -554,6 +596,30 @@ def cpu_baseline(run, budget_s=15.0):
     blocks/s over the sample."""
     import oracle
     oracle.lib()
+    if run.workload == "w4a4_gemm":
+        # the weight is quantised once (setup, not timed); the step is the
+        # activations' fake-quant and the product, on leading rows of X
+        wb = _bits(run.gemm_w)
+        wsg = oracle.global_scale(wb)
+        wc = oracle.scale_search_max(wb, wsg)
+        wp = oracle.quantize_pack(wb, wsg, wc)
+        X = run.fq_input
+
+        def step(n):
+            t0 = time.perf_counter()
+            _, ap, ac, asg = oracle.fake_quant(_bits(X[:n]))
+            oracle.gemm_nvfp4(ap, ac, asg, wp, wc, wsg)
+            return time.perf_counter() - t0
+        t1, t2 = step(4), step(16)
+        per_row = max((t2 - t1) / 12, 1e-6)
+        n = int(max(1, min(X.shape[0], (budget_s - max(t1 - 4 * per_row, 0.0)) / per_row)))
+        t = step(n)
+        blocks = n * X.shape[1] // 16
+        return {"value": round(blocks / t, 2), "unit": UNIT, "cores": oracle.max_threads(),
+                "kind": "oracle", "seconds": round(t, 3),
+                "sample": "fake-quant of %d of %d token rows and their product with the "
+                          "8192x8192 NVFP4 weight (%d activation blocks)"
+                          % (n, X.shape[0], blocks)}
     if not run.layers:  # activation-only workload: fake-quant on leading rows
         X = run.fq_input
         t0 = time.perf_counter()
@@ -627,7 +693,7 @@ def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
         return
-    small = args.workload in ("tiny", "dense", "w4a4", "four_over_six")
+    small = args.workload in ("tiny", "dense", "w4a4", "four_over_six", "w4a4_gemm")
     dev = "cpu" if small or not torch.cuda.is_available() else "cuda"
     run = Runner(args.workload, dev)
     budget = args.cpu_seconds / max(1, args.steps)

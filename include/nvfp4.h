@@ -234,6 +234,28 @@ nvfp4_status nvfp4_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16
 nvfp4_status nvfp4_get_device_status(void *stream, nvfp4_status *out);
 
 /*
+ * NVFP4 x NVFP4 matrix product on the tensor cores (W4A4: weights and
+ * activations both NVFP4 -- the consumer of nvfp4_quantize_pack /
+ * nvfp4_fake_quant outputs):
+ *   out[m][n] = bf16_rn(s_ga s_gb sum_k (v(a_mk) e4m3(ca_m,k/16))
+ *                                      (v(b_nk) e4m3(cb_n,k/16)))
+ * accumulated in fp32 (the tensor cores' block-scaled E2M1 MMA; the
+ * products are exact, the sum is fp32), s_ga s_gb rounded to fp32.
+ *   a_packed [M, K/2] uint8 and a_codes [M, K/16] uint8 (A row-major, K
+ *            contiguous: e.g. activations), a_sg DEVICE float [1]
+ *   b_packed [N, K/2], b_codes [N, K/16] (B row-major: e.g. weights
+ *            [out, in], so out = A B^T), b_sg DEVICE float [1]
+ *   out      [M, N] bf16, written (16-byte aligned)
+ * K must be a multiple of 32 and N of 8 (NVFP4_ERR_SHAPE); packed operands
+ * and out 16-byte aligned.  The block codes are copied into the scale layout
+ * the MMA reads (stream-ordered scratch from the library pool).  Returns
+ * NVFP4_ERR_NOT_IMPLEMENTED if the kernel cannot take the shape.
+ */
+nvfp4_status nvfp4_gemm(const uint8_t *a_packed, const uint8_t *a_codes, const float *a_sg,
+                        const uint8_t *b_packed, const uint8_t *b_codes, const float *b_sg,
+                        int64_t M, int64_t N, int64_t K, uint16_t *out, void *stream);
+
+/*
  * Work statistic of the scale searches (the pages have no counterpart; it
  * measures how much of the 126-candidate search the exact pruning leaves):
  * out[0] and out[1] receive the number of (block, candidate) objective

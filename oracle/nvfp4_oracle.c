@@ -399,7 +399,7 @@ int oracle_gemm_nvfp4(const uint8_t *a_packed, const uint8_t *a_codes, float a_s
     if (K % 16)
         return ORACLE_ERR_SHAPE;
     double g = (double)a_sg * (double)b_sg;
-#pragma omp parallel for schedule(dynamic, 4)
+#pragma omp parallel for collapse(2) schedule(dynamic, 64)
     for (int64_t m = 0; m < M; m++)
         for (int64_t n = 0; n < N; n++) {
             double acc = 0.0, aacc = 0.0;

@@ -100,7 +100,8 @@ def build(force=False, verbose=False, ptxas_info=False):
             continue
         cmd = [nvcc] + ARCH + NVCC_FLAGS
         if _uses_cutlass(src):
-            cmd += ["--expt-relaxed-constexpr", "-Xcompiler", "-Wno-unused-parameter"]
+            cmd += ["--expt-relaxed-constexpr", "-Xcompiler", "-Wno-unused-parameter",
+                    "-diag-suppress", "20012"]
             cmd += ["-I" + d for d in cutlass_include()]
         cmd += ["-c", src, "-o", obj]
         if ptxas_info:

@@ -249,6 +249,25 @@ nvfp4_status nvfp4_search_evaluations(void *stream, int reset, uint64_t *out) {
   return NVFP4_OK;
 }
 
+nvfp4_status nvfp4_gemm(const uint8_t *a_packed, const uint8_t *a_codes, const float *a_sg,
+                        const uint8_t *b_packed, const uint8_t *b_codes, const float *b_sg,
+                        int64_t M, int64_t N, int64_t K, uint16_t *out, void *stream) {
+  if (!a_packed || !a_codes || !a_sg || !b_packed || !b_codes || !b_sg || !out)
+    return NVFP4_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (K % 32 || N % 8) return NVFP4_ERR_SHAPE;
+  if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2 || !fits(M, K) || !fits(N, K) ||
+      !fits(M, N))
+    return NVFP4_ERR_TOO_LARGE;
+  if (!aligned(a_packed, 16) || !aligned(b_packed, 16) || !aligned(out, 16) ||
+      !aligned(a_sg, 4) || !aligned(b_sg, 4))
+    return NVFP4_ERR_MISALIGNED;
+  const cudaError_t e = nvfp4::launch_gemm_fp4(a_packed, a_codes, a_sg, b_packed, b_codes, b_sg,
+                                               M, N, K, out, as_stream(stream));
+  if (e == cudaErrorNotSupported) return NVFP4_ERR_NOT_IMPLEMENTED;
+  return map_cuda(e);
+}
+
 nvfp4_status nvfp4_self_test_device_timeout(void *stream) {
   return map_cuda(nvfp4::launch_wait_timeout_probe(as_stream(stream)));
 }

@@ -48,6 +48,12 @@ cudaError_t read_and_clear_gram_status(cudaStream_t st, int *out);
 // the device timeout status.
 cudaError_t launch_wait_timeout_probe(cudaStream_t st);
 
+// NVFP4 x NVFP4 product Y[M, N] (bf16) of A [M, K] and B [N, K] given as
+// packed codes, row-major block codes and device tensor scales.
+cudaError_t launch_gemm_fp4(const uint8_t *a_packed, const uint8_t *a_codes, const float *a_sg,
+                            const uint8_t *b_packed, const uint8_t *b_codes, const float *b_sg,
+                            int64_t M, int64_t N, int64_t K, uint16_t *out, cudaStream_t st);
+
 // Stream-ordered scratch from the library's pool on the current device.
 cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t st);
 cudaError_t scratch_free(void *p, cudaStream_t st);

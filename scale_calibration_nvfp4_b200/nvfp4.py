@@ -38,6 +38,7 @@ SIGNATURES = {
     "nvfp4_get_device_status": [_vp, _vp],
     "nvfp4_search_evaluations": [_vp, ctypes.c_int, _vp],
     "nvfp4_self_test_device_timeout": [_vp],
+    "nvfp4_gemm": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
 }
 
 
@@ -279,6 +280,25 @@ def search_evaluations(reset=False, stream=None):
     out = (ctypes.c_uint64 * 2)()
     _call("nvfp4_search_evaluations", _stream(stream), int(bool(reset)), out)
     return int(out[0]), int(out[1])
+
+
+def gemm(a_packed, a_codes, a_sg, b_packed, b_codes, b_sg, out=None, stream=None):
+    """out[M, N] (bf16) = A B^T for NVFP4 operands A [M, K] and B [N, K] given
+    as packed codes [*, K/2], block codes [*, K/16] and tensor scales [1]."""
+    for t, n in ((a_packed, "a_packed"), (a_codes, "a_codes"), (b_packed, "b_packed"),
+                 (b_codes, "b_codes")):
+        _need(t, torch.uint8, n)
+    _need(a_sg, torch.float32, "a_sg")
+    _need(b_sg, torch.float32, "b_sg")
+    M, N, K = a_packed.shape[0], b_packed.shape[0], a_packed.shape[1] * 2
+    if b_packed.shape[1] * 2 != K or a_codes.shape != (M, K // 16) or b_codes.shape != (N, K // 16):
+        raise ValueError("operand shapes do not match")
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=a_packed.device)
+    _need(out, torch.bfloat16, "out")
+    _call("nvfp4_gemm", _p(a_packed), _p(a_codes), _p(a_sg), _p(b_packed), _p(b_codes), _p(b_sg),
+          M, N, K, _p(out), _stream(stream))
+    return out
 
 
 def self_test_device_timeout(stream=None):

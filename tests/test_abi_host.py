@@ -93,6 +93,11 @@ def test_validation_rejects_before_launch(L):
     # sizes that overflow
     assert L.nvfp4_scale_search_max(P, 1, 1 << 40, 1 << 24, P, P, None) == SHAPE
     assert L.nvfp4_scale_search_max(P, 70000, 4, 16, P, P, None) == TOOLARGE
+    # the NVFP4 product: K a multiple of 32, N of 8, aligned operands
+    assert L.nvfp4_gemm(P, P, P, P, P, P, 128, 64, 48, P, None) == SHAPE
+    assert L.nvfp4_gemm(P, P, P, P, P, P, 128, 60, 64, P, None) == SHAPE
+    assert L.nvfp4_gemm(BAD, P, P, P, P, P, 128, 64, 64, P, None) == MISALIGNED
+    assert L.nvfp4_gemm(P, P, P, P, P, P, 128, 64, 64, None, None) == INVALID
     # the statistics call needs somewhere to write
     assert L.nvfp4_search_evaluations(None, 0, None) == INVALID
 

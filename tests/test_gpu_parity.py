@@ -505,3 +505,52 @@ def test_moe_experts_sampled(nv):
         blocks = rng.integers(0, nb, 400)
         rc, _ = oracle.scale_search_sampled(wu_all[e], sg, Hc[e], rows, blocks)
         check_search_codes(codes[e][rows, blocks], rc, wu_all[e], sg, Hc[e], rows, blocks)
+
+
+# ------------------------------------------------------------ NVFP4 GEMM
+def _gemm_operands(nv, X, W):
+    """Activations through the dynamic fake-quant (packed outputs), weights
+    through the global scale, the max rule and pack."""
+    _, ap, ac, asg = nv.fake_quant(X, want_packed=True)
+    wsg = nv.global_scale(W)
+    wc = nv.scale_search_max(W, wsg)
+    wp = nv.quantize_pack(W, wsg, wc)
+    return ap, ac, asg, wp, wc, wsg
+
+
+def _check_gemm(Y, ref, absref, K):
+    y = bits_to_f64(bf16_bits(Y))
+    # bf16 rounding of the result plus fp32 accumulation over K terms
+    tol = 2.0 ** -8 * np.abs(ref) + K * 2.0 ** -23 * absref + 1e-35
+    bad = np.argwhere(np.abs(y - ref) > tol)
+    assert bad.size == 0, (bad[:5], y[tuple(bad[0])], ref[tuple(bad[0])])
+
+
+@pytest.mark.parametrize("M,N,K", [(200, 136, 256), (128, 256, 96), (1, 8, 32), (333, 520, 1024)])
+def test_gemm_matches_oracle(nv, M, N, K):
+    X = rand_bf16((M, K), M + K, 1.0, 0.01, 30.0).cuda()
+    W = rand_bf16((N, K), N + K, 0.02, 0.005, 15.0).cuda()
+    ap, ac, asg, wp, wc, wsg = _gemm_operands(nv, X, W)
+    Y = nv.gemm(ap, ac, asg, wp, wc, wsg)
+    ref, absref = oracle.gemm_nvfp4(ap.cpu().numpy(), ac.cpu().numpy(), asg.item(),
+                                    wp.cpu().numpy(), wc.cpu().numpy(), wsg.item())
+    _check_gemm(Y, ref, absref, K)
+
+
+def test_gemm_w4a4_full_size_sampled(nv):
+    """The W4A4 activations (32768x8192, dynamic fake-quant with packed
+    outputs) times an 8192x8192 NVFP4 weight, in one call; 48 rows x 48
+    columns of the result against the oracle."""
+    from scale_calibration_nvfp4_b200 import workloads
+    X = workloads.w4a4_inputs("cuda")
+    g = torch.Generator(device="cuda").manual_seed(9)
+    W = (torch.randn(8192, 8192, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    ap, ac, asg, wp, wc, wsg = _gemm_operands(nv, X, W)
+    Y = nv.gemm(ap, ac, asg, wp, wc, wsg)
+    rng = np.random.default_rng(4)
+    rows = np.sort(rng.choice(X.shape[0], 48, replace=False)); rows[-1] = X.shape[0] - 1
+    cols = np.sort(rng.choice(W.shape[0], 48, replace=False)); cols[0] = 0
+    r_t, c_t = torch.from_numpy(rows).cuda(), torch.from_numpy(cols).cuda()
+    ref, absref = oracle.gemm_nvfp4(ap[r_t].cpu().numpy(), ac[r_t].cpu().numpy(), asg.item(),
+                                    wp[c_t].cpu().numpy(), wc[c_t].cpu().numpy(), wsg.item())
+    _check_gemm(Y[r_t][:, c_t].contiguous(), ref, absref, X.shape[1])

@@ -41,6 +41,13 @@ def lib():
         L.oracle_scale_search_max.argtypes = [vp, i64, i64, f32, vp]
         L.oracle_four_over_six_code.argtypes = [vp, f32]
         L.oracle_gemm_nvfp4.argtypes = [vp, vp, f32, vp, vp, f32, i64, i64, i64, vp, vp]
+        L.oracle_fake_quant_static.argtypes = [vp, i64, i64, f32, vp, vp, vp]
+        L.oracle_abs_histogram.argtypes = [vp, i64, vp]
+        L.oracle_quantile_magnitude.argtypes = [vp, f64, vp]
+        L.oracle_static_scale.restype = f32
+        L.oracle_static_scale.argtypes = [f64]
+        L.oracle_quant_error.restype = f64
+        L.oracle_quant_error.argtypes = [vp, i64, i64, f32]
         L.oracle_scale_search_four_over_six.argtypes = [vp, i64, i64, f32, vp]
         L.oracle_block_mse.restype = f64
         L.oracle_block_mse.argtypes = [vp, f32, i32]
@@ -244,6 +251,42 @@ def dequantize(packed, codes, s_g):
     out = np.zeros((R, C), np.uint16)
     _check(lib().oracle_dequantize(_ptr(packed), _ptr(codes), float(s_g), R, C, _ptr(out)))
     return out
+
+
+def fake_quant_static(x_u16, s_g, want_packed=True):
+    x = _u16(x_u16)
+    R, C = x.shape
+    out = np.zeros((R, C), np.uint16)
+    packed = np.zeros((R, C // 2), np.uint8) if want_packed else None
+    codes = np.zeros((R, C // 16), np.uint8) if want_packed else None
+    _check(lib().oracle_fake_quant_static(_ptr(x), R, C, float(s_g), _ptr(out), _ptr(packed),
+                                          _ptr(codes)))
+    return out, packed, codes
+
+
+def abs_histogram(x_u16, hist=None):
+    x = _u16(x_u16).reshape(-1)
+    if hist is None:
+        hist = np.zeros(32768, np.uint64)
+    lib().oracle_abs_histogram(_ptr(x), x.size, _ptr(hist))
+    return hist
+
+
+def quantile_magnitude(hist, p):
+    m = ctypes.c_double()
+    h = np.ascontiguousarray(hist, np.uint64)
+    _check(lib().oracle_quantile_magnitude(_ptr(h), float(p), ctypes.byref(m)))
+    return m.value
+
+
+def static_scale(clip):
+    return np.float32(lib().oracle_static_scale(float(clip)))
+
+
+def quant_error(x_u16, s_g):
+    x = _u16(x_u16)
+    R, C = x.shape
+    return lib().oracle_quant_error(_ptr(x), R, C, float(s_g))
 
 
 def fake_quant(x_u16, want_packed=True):

@@ -509,16 +509,14 @@ int oracle_dequantize(const uint8_t *packed, const uint8_t *codes, float s_g, in
  * use their absolute maximum; [QAD] section 3.2: reshape into blocks of 16,
  * scale by the block max over 6, quantise, dequantise).  packed and codes
  * may be NULL. */
-int oracle_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16_t *out,
-                      uint8_t *packed, uint8_t *codes, float *s_g_out)
+/* Fake-quant at a given tensor scale (a static, calibrated one): per block
+ * the max rule, E2M1 encode and dequantise; values beyond 6 * 448 * s_g
+ * saturate.  [BT] "Calibration" (block scales from the block maximum). */
+int oracle_fake_quant_static(const uint16_t *x, int64_t rows, int64_t C, float s_g,
+                             uint16_t *out, uint8_t *packed, uint8_t *codes)
 {
     if (C % 16)
         return ORACLE_ERR_SHAPE;
-    float s_g;
-    int st = oracle_global_scale(x, rows * C, &s_g);
-    if (st)
-        return st;
-    *s_g_out = s_g;
     int64_t nb = C / 16;
 #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; r++)
@@ -542,6 +540,92 @@ int oracle_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16_t *out,
             }
         }
     return ORACLE_OK;
+}
+
+int oracle_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16_t *out,
+                      uint8_t *packed, uint8_t *codes, float *s_g_out)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    float s_g;
+    int st = oracle_global_scale(x, rows * C, &s_g);
+    if (st)
+        return st;
+    *s_g_out = s_g;
+    return oracle_fake_quant_static(x, rows, C, s_g, out, packed, codes);
+}
+
+/* ------------------------------------------- activation-range calibration */
+
+/* [BT] "Calibration": the clipping range of an activation tensor comes from
+ * calibration data -- the maximum avoids clipping, but percentile-,
+ * histogram- and error-based ranges clip a few outliers so that the typical
+ * values are represented more finely.  Reading: the range sets the static
+ * tensor scale s_g = fl32(clip / 2688) of fake_quant_static (block scales
+ * still follow each block's maximum).
+ *
+ * Histogram of |x| over the 32768 bf16 magnitude patterns (exact counts,
+ * accumulated: call once per calibration chunk). */
+void oracle_abs_histogram(const uint16_t *x, int64_t n, uint64_t *hist)
+{
+    for (int64_t i = 0; i < n; i++)
+        hist[x[i] & 0x7FFF]++;
+}
+
+/* The p-quantile of |x| (0 < p <= 1): the smallest bf16 magnitude m with at
+ * least ceil(p * N) of the N counted values at or below it.  Non-finite
+ * magnitudes are counted but a quantile that lands on one is an error. */
+int oracle_quantile_magnitude(const uint64_t *hist, double p, double *m_out)
+{
+    uint64_t n = 0;
+    for (int k = 0; k < 32768; k++)
+        n += hist[k];
+    if (n == 0 || !(p > 0.0) || p > 1.0)
+        return ORACLE_ERR_SHAPE;
+    uint64_t need = (uint64_t)ceil(p * (double)n);
+    if (need < 1)
+        need = 1;
+    uint64_t acc = 0;
+    for (int k = 0; k < 32768; k++) {
+        acc += hist[k];
+        if (acc >= need) {
+            double m = oracle_bf16_to_double((uint16_t)k);
+            if (!isfinite(m))
+                return ORACLE_ERR_NONFINITE;
+            *m_out = m;
+            return ORACLE_OK;
+        }
+    }
+    return ORACLE_ERR_SHAPE;
+}
+
+/* Static tensor scale from a clipping range: fl32(clip / 2688), 1 for 0. */
+float oracle_static_scale(double clip)
+{
+    if (clip == 0.0)
+        return 1.0f;
+    return (float)clip / 2688.0f;  /* clip is a bf16 value: exact in float */
+}
+
+/* Quantisation error of fake_quant_static: sum over all values of
+ * (x - y)^2 with y the bf16 fake-quant output, in fp64 -- the measure the
+ * error-based range minimises over candidate clips. */
+double oracle_quant_error(const uint16_t *x, int64_t rows, int64_t C, float s_g)
+{
+    uint16_t *y = (uint16_t *)malloc(sizeof(uint16_t) * rows * C);
+    if (!y)
+        return NAN;
+    if (oracle_fake_quant_static(x, rows, C, s_g, y, NULL, NULL)) {
+        free(y);
+        return NAN;
+    }
+    double e = 0.0;
+    for (int64_t i = 0; i < rows * C; i++) {
+        double d = oracle_bf16_to_double(x[i]) - oracle_bf16_to_double(y[i]);
+        e += d * d;
+    }
+    free(y);
+    return e;
 }
 
 int oracle_max_threads(void)

@@ -509,3 +509,60 @@ def test_gemm_oracle_hand_case(oracle_mod):
     bc = np.full((1, 2), half, np.uint8)
     Y, _ = oracle_mod.gemm_nvfp4(ap, ac, 1.0, bp, bc, 1.0)
     assert Y[0, 0] == 32 * (1.0 * 2.0) * (6.0 * 0.5)
+
+
+# ------------------------------------------------ activation-range calibration
+def _act(seed, n_rows=64, C=256):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(n_rows, C, generator=g)
+    x[:, 7] *= 40.0
+    x[3, 11] = -900.0
+    return bf16_bits(x.to(torch.bfloat16))
+
+
+def test_abs_histogram_is_magnitude_bincount(oracle_mod):
+    x = _act(1)
+    h = oracle_mod.abs_histogram(x)
+    ref = np.bincount((x & 0x7FFF).astype(np.int64).ravel(), minlength=32768)
+    assert np.array_equal(h, ref.astype(np.uint64))
+    # accumulates across chunks
+    h2 = oracle_mod.abs_histogram(x[32:], oracle_mod.abs_histogram(x[:32]))
+    assert np.array_equal(h2, h)
+
+
+@pytest.mark.parametrize("p", [1.0, 0.9999, 0.999, 0.99, 0.5, 1e-9])
+def test_quantile_is_order_statistic(oracle_mod, p):
+    x = _act(2)
+    mags = np.sort(np.abs(bits_to_f64(x)).ravel())
+    k = max(1, math.ceil(p * mags.size))
+    assert oracle_mod.quantile_magnitude(oracle_mod.abs_histogram(x), p) == mags[k - 1]
+
+
+def test_static_scale_at_the_max_is_the_dynamic_scale(oracle_mod):
+    x = _act(3)
+    amax = np.abs(bits_to_f64(x)).max()
+    assert oracle_mod.static_scale(amax) == oracle_mod.global_scale(x)
+    y, p, c = oracle_mod.fake_quant_static(x, oracle_mod.global_scale(x))
+    ry, rp, rc, _ = oracle_mod.fake_quant(x)
+    assert np.array_equal(y, ry) and np.array_equal(p, rp) and np.array_equal(c, rc)
+
+
+def test_static_scale_clips_outliers(oracle_mod):
+    """s_g = 1/64: the largest block scale is 448/64 = 7 (code 0x7E), so a
+    value of 100 saturates to 6 * 7 = 42 while the block's small values are
+    encoded at scale 7."""
+    x = np.zeros((1, 16), np.float32)
+    x[0, :4] = [100.0, -3.5, 7.0, 0.0]
+    u = f32_to_bf16_bits(x)
+    y, p, c = oracle_mod.fake_quant_static(u, np.float32(1 / 64))
+    yv = bits_to_f64(y)[0]
+    assert c[0, 0] == 0x7E
+    assert yv[0] == 42.0 and yv[1] == -3.5 and yv[2] == 7.0 and yv[3] == 0.0
+
+
+def test_quant_error_is_sum_of_squared_differences(oracle_mod):
+    x = _act(4)
+    for s_g in (oracle_mod.global_scale(x), np.float32(oracle_mod.global_scale(x) / 8)):
+        y, _, _ = oracle_mod.fake_quant_static(x, s_g, want_packed=False)
+        ref = float(np.sum((bits_to_f64(x) - bits_to_f64(y)) ** 2))
+        assert math.isclose(oracle_mod.quant_error(x, s_g), ref, rel_tol=1e-12)

@@ -227,9 +227,53 @@ nvfp4_status nvfp4_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16
                               uint8_t *packed, uint8_t *scale_codes, float *s_g, void *stream);
 
 /*
+ * Activation-range calibration ([BT] "Calibration": the clipping range of an
+ * activation tensor comes from calibration data; the maximum avoids
+ * clipping, percentile-, histogram- and error-based ranges clip a few
+ * outliers so that typical values are represented more finely).  The range
+ * sets a static tensor scale s_g = fl32(clip / 2688) (1 for clip 0) used by
+ * nvfp4_fake_quant_static; block scales still follow each block's maximum,
+ * so values beyond 6 * 448 * s_g saturate.
+ *
+ * nvfp4_abs_histogram: hist[|x| bf16 magnitude pattern] += count, exact, over
+ * the 32768 patterns; call once per calibration chunk.
+ *   x     [n] bf16 (16-byte aligned);  hist  DEVICE uint64 [32768], accumulated
+ */
+nvfp4_status nvfp4_abs_histogram(const uint16_t *x, int64_t n, uint64_t *hist, void *stream);
+
+/*
+ * The p-quantile (0 < p <= 1) of the counted magnitudes -- the smallest
+ * bf16 magnitude m with at least ceil(p * N) of the N values at or below it
+ * (p = 1: the maximum) -- as the static tensor scale s_g = fl32(m / 2688).
+ * An empty histogram gives s_g = 1; a quantile on a non-finite pattern sets
+ * s_g to NaN and the device status to NVFP4_ERR_NONFINITE.
+ *   hist  DEVICE uint64 [32768];  s_g  DEVICE float [1], written
+ */
+nvfp4_status nvfp4_static_scale_from_histogram(const uint64_t *hist, double p, float *s_g,
+                                               void *stream);
+
+/*
+ * nvfp4_fake_quant with a given (static, calibrated) tensor scale instead of
+ * the tensor's own maximum.  Arguments as nvfp4_fake_quant; s_g is read.
+ */
+nvfp4_status nvfp4_fake_quant_static(const uint16_t *x, int64_t rows, int64_t C, const float *s_g,
+                                     uint16_t *out, uint8_t *packed, uint8_t *scale_codes,
+                                     void *stream);
+
+/*
+ * Quantisation error of nvfp4_fake_quant_static at s_g: sum over x of
+ * (x - y)^2, y the bf16 fake-quant output, in fp64 (per-CTA partials added
+ * in a fixed order: reproducible for a shape) -- the measure an error-based
+ * range minimises over candidate clips.
+ *   err  DEVICE double [1], written
+ */
+nvfp4_status nvfp4_quant_error(const uint16_t *x, int64_t rows, int64_t C, const float *s_g,
+                               double *err, void *stream);
+
+/*
  * Reads and clears the device-side status of the current device after
  * synchronising `stream`.  *out is NVFP4_OK, NVFP4_ERR_NONFINITE or
- * NVFP4_ERR_DEVICE_TIMEOUT (the first one set, if several are).
+ * NVFP4_ERR_DEVICE_TIMEOUT.
  */
 nvfp4_status nvfp4_get_device_status(void *stream, nvfp4_status *out);
 

@@ -230,6 +230,40 @@ nvfp4_status nvfp4_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16
                                            as_stream(stream)));
 }
 
+nvfp4_status nvfp4_abs_histogram(const uint16_t *x, int64_t n, uint64_t *hist, void *stream) {
+  if (!hist || n < 0 || (n > 0 && !x)) return NVFP4_ERR_INVALID_ARG;
+  if (!fits(n, 1)) return NVFP4_ERR_SHAPE;
+  if ((x && !aligned(x, 16)) || !aligned(hist, 8)) return NVFP4_ERR_MISALIGNED;
+  return map_cuda(nvfp4::launch_abs_histogram(x, n, hist, as_stream(stream)));
+}
+
+nvfp4_status nvfp4_static_scale_from_histogram(const uint64_t *hist, double p, float *s_g,
+                                               void *stream) {
+  if (!hist || !s_g || !(p > 0.0) || !(p <= 1.0)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(hist, 8) || !aligned(s_g, 4)) return NVFP4_ERR_MISALIGNED;
+  return map_cuda(nvfp4::launch_quantile_scale(hist, p, s_g, as_stream(stream)));
+}
+
+nvfp4_status nvfp4_fake_quant_static(const uint16_t *x, int64_t rows, int64_t C, const float *s_g,
+                                     uint16_t *out, uint8_t *packed, uint8_t *scale_codes,
+                                     void *stream) {
+  if (!x || !out || !s_g || rows < 0 || C < 0) return NVFP4_ERR_INVALID_ARG;
+  if (C % 16 || !fits(rows, C)) return NVFP4_ERR_SHAPE;
+  if (!aligned(x, 16) || !aligned(out, 16) || !aligned(s_g, 4) ||
+      (packed && !aligned(packed, 16)))
+    return NVFP4_ERR_MISALIGNED;
+  return map_cuda(nvfp4::launch_fake_quant_static(x, rows, C, s_g, out, packed, scale_codes,
+                                                  as_stream(stream)));
+}
+
+nvfp4_status nvfp4_quant_error(const uint16_t *x, int64_t rows, int64_t C, const float *s_g,
+                               double *err, void *stream) {
+  if (!x || !s_g || !err || rows < 0 || C < 0) return NVFP4_ERR_INVALID_ARG;
+  if (C % 16 || !fits(rows, C)) return NVFP4_ERR_SHAPE;
+  if (!aligned(x, 16) || !aligned(s_g, 4) || !aligned(err, 8)) return NVFP4_ERR_MISALIGNED;
+  return map_cuda(nvfp4::launch_quant_error(x, rows, C, s_g, err, as_stream(stream)));
+}
+
 nvfp4_status nvfp4_get_device_status(void *stream, nvfp4_status *out) {
   if (!out) return NVFP4_ERR_INVALID_ARG;
   int v = 0;

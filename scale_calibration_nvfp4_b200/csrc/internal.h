@@ -54,6 +54,18 @@ cudaError_t launch_gemm_fp4(const uint8_t *a_packed, const uint8_t *a_codes, con
                             const uint8_t *b_packed, const uint8_t *b_codes, const float *b_sg,
                             int64_t M, int64_t N, int64_t K, uint16_t *out, cudaStream_t st);
 
+// Activation-range calibration: exact |x| histogram (uint64 [32768],
+// accumulated), its p-quantile as a static tensor scale, fake-quant at a
+// given tensor scale, and the quantisation error at a given tensor scale.
+cudaError_t launch_abs_histogram(const uint16_t *x, int64_t n, uint64_t *hist, cudaStream_t st);
+cudaError_t launch_quantile_scale(const uint64_t *hist, double p, float *s_g, cudaStream_t st);
+cudaError_t launch_fake_quant_static(const uint16_t *x, int64_t rows, int64_t C, const float *s_g,
+                                     uint16_t *out, uint8_t *packed, uint8_t *codes,
+                                     cudaStream_t st);
+cudaError_t launch_quant_error(const uint16_t *x, int64_t rows, int64_t C, const float *s_g,
+                               double *err, cudaStream_t st);
+cudaError_t read_and_clear_calib_status(cudaStream_t st, int *out);
+
 // Stream-ordered scratch from the library's pool on the current device.
 cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t st);
 cudaError_t scratch_free(void *p, cudaStream_t st);

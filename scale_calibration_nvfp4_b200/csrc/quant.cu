@@ -459,6 +459,58 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__
   }
 }
 
+// Sum of (x - y)^2 over a tensor for its bf16 fake-quant output y at the
+// given tensor scale (the static-range fake-quant without its writes), in
+// fp64; one partial per CTA, in a fixed order within the CTA.
+__global__ void __launch_bounds__(kThreads) quant_error_kernel(const uint16_t *__restrict__ x,
+                                                               int64_t nblk,
+                                                               const float *__restrict__ s_g,
+                                                               double *__restrict__ partial) {
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  uint32_t v[8];
+  if (i < nblk) load_block(x + i * kBlock, v);
+  const float sg = *s_g;
+  const MaxRule mr = make_max_rule(sg);
+  __shared__ ScaleEntry tab[256];
+  fill_scale_table(tab, sg);
+  double acc = 0.0;
+  for (; i < nblk; i += stride) {
+    uint32_t nv[8];
+    const int64_t n = i + stride;
+    if (n < nblk) load_block(x + n * kBlock, nv);
+    const float amax = __uint_as_float(amax_bits8(v) << 16);
+    const ScaleEntry se = tab[max_rule_code_fast(amax, mr)];
+    const uint2 q = encode_block_entry(v, se);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t y = dequant_byte(((j < 4 ? q.x : q.y) >> (8 * (j & 3))) & 0xFFu, se.s);
+      const double d0 = (double)bf16_lo(v[j]) - (double)bf16_lo(y);
+      const double d1 = (double)bf16_hi(v[j]) - (double)bf16_hi(y);
+      acc += d0 * d0 + d1 * d1;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = nv[j];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  __shared__ double warp_sum[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) warp_sum[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < kThreads / 32; ++w) t += warp_sum[w];
+    partial[blockIdx.x] = t;
+  }
+}
+
+__global__ void error_reduce_kernel(const double *__restrict__ partial, int n,
+                                    double *__restrict__ out) {
+  double t = 0.0;
+  for (int i = 0; i < n; ++i) t += partial[i];
+  *out = t;
+}
+
 int g_sm_count = 0;
 
 int grid_for(int64_t work_items, int max_ctas_per_sm) {
@@ -550,6 +602,31 @@ cudaError_t launch_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16
   return cudaGetLastError();
 }
 
+cudaError_t launch_fake_quant_static(const uint16_t *x, int64_t rows, int64_t C, const float *s_g,
+                                     uint16_t *out, uint8_t *packed, uint8_t *codes,
+                                     cudaStream_t st) {
+  const int64_t nblk = rows * C / kBlock;
+  if (nblk == 0) return cudaSuccess;
+  const int gx = grid_for(nblk, 16);
+  fake_quant_kernel<<<gx, kThreads, 0, st>>>(x, nblk, s_g, out, packed, codes);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_error(const uint16_t *x, int64_t rows, int64_t C, const float *s_g,
+                               double *err, cudaStream_t st) {
+  const int64_t nblk = rows * C / kBlock;
+  if (nblk == 0) return cudaMemsetAsync(err, 0, sizeof(double), st);
+  const int gx = grid_for(nblk, 8);
+  double *partial = nullptr;
+  cudaError_t e = scratch_alloc(reinterpret_cast<void **>(&partial), sizeof(double) * gx, st);
+  if (e != cudaSuccess) return e;
+  quant_error_kernel<<<gx, kThreads, 0, st>>>(x, nblk, s_g, partial);
+  error_reduce_kernel<<<1, 1, 0, st>>>(partial, gx, err);
+  e = cudaGetLastError();
+  const cudaError_t ef = scratch_free(partial, st);
+  return e != cudaSuccess ? e : ef;
+}
+
 cudaError_t read_and_clear_device_status(cudaStream_t st, int *out) {
   int zero = 0;
   cudaError_t e = cudaStreamSynchronize(st);
@@ -558,10 +635,12 @@ cudaError_t read_and_clear_device_status(cudaStream_t st, int *out) {
   if (e != cudaSuccess) return e;
   e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
   if (e != cudaSuccess) return e;
-  // the Gram kernels keep their own flag (a timed-out wait)
-  int gram = 0;
+  // the Gram kernels keep their own flag (a timed-out wait), the
+  // calibration kernels theirs (a quantile on a non-finite value)
+  int gram = 0, calib = 0;
   e = read_and_clear_gram_status(st, &gram);
-  if (*out == 0) *out = gram;
+  if (e == cudaSuccess) e = read_and_clear_calib_status(st, &calib);
+  if (*out == 0) *out = gram ? gram : calib;
   return e;
 }
 

@@ -39,6 +39,10 @@ SIGNATURES = {
     "nvfp4_search_evaluations": [_vp, ctypes.c_int, _vp],
     "nvfp4_self_test_device_timeout": [_vp],
     "nvfp4_gemm": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
+    "nvfp4_abs_histogram": [_vp, _i64, _vp, _vp],
+    "nvfp4_static_scale_from_histogram": [_vp, ctypes.c_double, _vp, _vp],
+    "nvfp4_fake_quant_static": [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp],
+    "nvfp4_quant_error": [_vp, _i64, _i64, _vp, _vp, _vp],
 }
 
 
@@ -298,6 +302,51 @@ def gemm(a_packed, a_codes, a_sg, b_packed, b_codes, b_sg, out=None, stream=None
     _need(out, torch.bfloat16, "out")
     _call("nvfp4_gemm", _p(a_packed), _p(a_codes), _p(a_sg), _p(b_packed), _p(b_codes), _p(b_sg),
           M, N, K, _p(out), _stream(stream))
+    return out
+
+
+def abs_histogram(x, hist=None, stream=None):
+    """hist[32768] (uint64, CUDA) += counts of |x| by bf16 magnitude pattern."""
+    _need(x, torch.bfloat16, "x")
+    if hist is None:
+        hist = torch.zeros(32768, dtype=torch.int64, device=x.device)
+    if hist.dtype != torch.int64 or hist.numel() != 32768 or not hist.is_cuda:
+        raise ValueError("hist must be a CUDA int64 tensor of 32768 counts")
+    _call("nvfp4_abs_histogram", _p(x), x.numel(), _p(hist), _stream(stream))
+    return hist
+
+
+def static_scale_from_histogram(hist, p, out=None, stream=None):
+    """Static tensor scale fl32(m / 2688) from the p-quantile m of the counts."""
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=hist.device)
+    _call("nvfp4_static_scale_from_histogram", _p(hist), float(p), _p(out), _stream(stream))
+    return out
+
+
+def fake_quant_static(x, s_g, want_packed=False, stream=None):
+    """Fake-quant of x [rows, C] at the given tensor scale; returns
+    (out, packed, codes) (packed/codes None unless want_packed)."""
+    _need(x, torch.bfloat16, "x")
+    _need(s_g, torch.float32, "s_g")
+    rows, C = x.shape
+    out = torch.empty_like(x)
+    packed = torch.empty(rows, C // 2, dtype=torch.uint8, device=x.device) if want_packed else None
+    codes = torch.empty(rows, C // 16, dtype=torch.uint8, device=x.device) if want_packed else None
+    _call("nvfp4_fake_quant_static", _p(x), rows, C, _p(s_g), _p(out),
+          _p(packed) if packed is not None else None, _p(codes) if codes is not None else None,
+          _stream(stream))
+    return out, packed, codes
+
+
+def quant_error(x, s_g, out=None, stream=None):
+    """sum (x - fake_quant_static(x, s_g))^2 in fp64, as a CUDA float64 [1]."""
+    _need(x, torch.bfloat16, "x")
+    _need(s_g, torch.float32, "s_g")
+    rows, C = x.shape
+    if out is None:
+        out = torch.empty(1, dtype=torch.float64, device=x.device)
+    _call("nvfp4_quant_error", _p(x), rows, C, _p(s_g), _p(out), _stream(stream))
     return out
 
 

@@ -98,6 +98,12 @@ def test_validation_rejects_before_launch(L):
     assert L.nvfp4_gemm(P, P, P, P, P, P, 128, 60, 64, P, None) == SHAPE
     assert L.nvfp4_gemm(BAD, P, P, P, P, P, 128, 64, 64, P, None) == MISALIGNED
     assert L.nvfp4_gemm(P, P, P, P, P, P, 128, 64, 64, None, None) == INVALID
+    # activation-range calibration
+    assert L.nvfp4_abs_histogram(BAD, 64, P, None) == MISALIGNED
+    assert L.nvfp4_static_scale_from_histogram(P, ctypes.c_double(0.0), P, None) == INVALID
+    assert L.nvfp4_static_scale_from_histogram(P, ctypes.c_double(1.5), P, None) == INVALID
+    assert L.nvfp4_fake_quant_static(P, 4, 20, P, P, None, None, None) == SHAPE
+    assert L.nvfp4_quant_error(P, 4, 16, P, None, None) == INVALID
     # the statistics call needs somewhere to write
     assert L.nvfp4_search_evaluations(None, 0, None) == INVALID
 

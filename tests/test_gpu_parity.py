@@ -1,6 +1,8 @@
 """GPU parity: every C-ABI entry point against the CPU oracle, element by
 element, on seeded inputs (small cases that span many tiles with ragged
 tails, edge cases, and samples of the full-size workloads)."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -554,3 +556,61 @@ def test_gemm_w4a4_full_size_sampled(nv):
     ref, absref = oracle.gemm_nvfp4(ap[r_t].cpu().numpy(), ac[r_t].cpu().numpy(), asg.item(),
                                     wp[c_t].cpu().numpy(), wc[c_t].cpu().numpy(), wsg.item())
     _check_gemm(Y[r_t][:, c_t].contiguous(), ref, absref, X.shape[1])
+
+
+# ------------------------------------------------ activation-range calibration
+def test_abs_histogram_and_static_scales(nv):
+    x = rand_bf16((301, 96), 41, 1.0, 0.003, 60.0)
+    xu = bf16_bits(x)
+    flat = x.reshape(-1)
+    h = nv.abs_histogram(flat[:10001].contiguous().cuda())       # ragged length
+    h = nv.abs_histogram(flat[10001:].contiguous().cuda(), h)    # accumulates
+    ref = oracle.abs_histogram(xu)
+    assert np.array_equal(h.cpu().numpy().astype(np.uint64), ref)
+    for p in (1.0, 0.99999, 0.9999, 0.999, 0.5):
+        s = nv.static_scale_from_histogram(h, p).item()
+        assert s == oracle.static_scale(oracle.quantile_magnitude(ref, p)), p
+
+
+def test_fake_quant_static_and_error(nv):
+    x = rand_bf16((333, 96), 43, 1.0, 0.003, 60.0)
+    xu = bf16_bits(x)
+    sg_max = oracle.global_scale(xu)
+    for s in (sg_max, np.float32(sg_max / 16), np.float32(sg_max * 3)):
+        s_t = torch.tensor([s], dtype=torch.float32, device="cuda")
+        y, p, c = nv.fake_quant_static(x.cuda(), s_t, want_packed=True)
+        ry, rp, rc = oracle.fake_quant_static(xu, s)
+        assert np.array_equal(bf16_bits(y), ry) and np.array_equal(p.cpu().numpy(), rp) \
+            and np.array_equal(c.cpu().numpy(), rc)
+        e = nv.quant_error(x.cuda(), s_t).item()
+        assert math.isclose(e, oracle.quant_error(xu, s), rel_tol=1e-10)
+    assert nv.get_device_status() == "NVFP4_OK"
+
+
+def test_static_scale_on_nonfinite_reports(nv):
+    x = torch.ones(64, dtype=torch.bfloat16)
+    x[5] = float("inf")
+    h = nv.abs_histogram(x.cuda())
+    assert math.isnan(nv.static_scale_from_histogram(h, 1.0).item())
+    assert nv.get_device_status() == "NVFP4_ERR_NONFINITE"
+    assert nv.static_scale_from_histogram(h, 0.5).item() == oracle.static_scale(1.0)
+    assert nv.get_device_status() == "NVFP4_OK"
+
+
+def test_calibration_w4a4_full_size(nv):
+    """The W4A4 activations (268 M values): histogram bit-exact, the
+    99.99th-percentile static scale bit-exact, the error at it and at the
+    maximum within 1e-9 of the oracle."""
+    from scale_calibration_nvfp4_b200 import workloads
+    X = workloads.w4a4_inputs("cuda")
+    xu = bf16_bits(X)
+    h = nv.abs_histogram(X)
+    ref = oracle.abs_histogram(xu)
+    assert np.array_equal(h.cpu().numpy().astype(np.uint64), ref)
+    s_p = nv.static_scale_from_histogram(h, 0.9999)
+    assert s_p.item() == oracle.static_scale(oracle.quantile_magnitude(ref, 0.9999))
+    s_max = nv.static_scale_from_histogram(h, 1.0)
+    assert s_max.item() == oracle.global_scale(xu)
+    e_p, e_max = nv.quant_error(X, s_p).item(), nv.quant_error(X, s_max).item()
+    assert math.isclose(e_p, oracle.quant_error(xu, s_p.item()), rel_tol=1e-9)
+    assert math.isclose(e_max, oracle.quant_error(xu, s_max.item()), rel_tol=1e-9)

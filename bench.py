@@ -49,7 +49,8 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
-WORKLOAD_NAMES = ["dense", "tiny", "moe", "mlp_pair", "w4a4", "four_over_six", "w4a4_gemm"]
+WORKLOAD_NAMES = ["dense", "tiny", "moe", "mlp_pair", "w4a4", "four_over_six", "w4a4_gemm",
+                  "act_calib"]
 
 # Local-Hessian search work per block, counted on the definition E = delta
 # H_b delta^T: per candidate 256 FMA for H_b delta and 16 FMA for the dot
@@ -149,6 +150,18 @@ class Runner:
                 self.gw_codes = nvfp4.scale_search_max(W, self.gw_sg)
                 self.gw_packed = nvfp4.quantize_pack(W, self.gw_sg, self.gw_codes)
                 self.gemm_out = torch.empty(X.shape[0], 8192, dtype=torch.bfloat16, device=X.device)
+        elif workload == "act_calib":
+            # static activation range: the W4A4 activations as the calibration
+            # set; per step the |x| histogram, the 99.99th-percentile tensor
+            # scale and the static fake-quant with packed outputs
+            X = wl.w4a4_inputs(device)
+            self.layers = []
+            self.desc = ("static activation range on X 32768x8192 (the W4A4 activations): |x| "
+                         "histogram, 99.99th-percentile tensor scale, static fake-quant")
+            self.rules = []
+            self.fq_input = X
+            self.hist = torch.zeros(32768, dtype=torch.int64, device=X.device)
+            self.calib_sg = torch.empty(1, dtype=torch.float32, device=X.device)
         elif workload == "w4a4":
             X = wl.w4a4_inputs(device)
             self.layers = []
@@ -217,7 +230,18 @@ class Runner:
                          n_w // 2 + nb + 2 * n_w, 1))
         if self.fq_input is not None:
             n_x = self.fq_input.numel()
-            if self.workload == "w4a4_gemm":
+            if self.workload == "act_calib":
+                X = self.fq_input
+                rows.append(("abs_histogram",
+                             lambda: (self.hist.zero_(), nv.abs_histogram(X, self.hist)),
+                             2 * n_x, 1))  # (the zeroing is a torch fill)
+                rows.append(("static_scale",
+                             lambda: nv.static_scale_from_histogram(self.hist, 0.9999,
+                                                                    out=self.calib_sg),
+                             32768 * 8, 1))
+                rows.append(("fake_quant_static", lambda: self._fq_static(),
+                             (FAKE_QUANT_BYTES_PER_ELEM - 2) * n_x, 1))
+            elif self.workload == "w4a4_gemm":
                 X = self.fq_input
                 M, K, N = X.shape[0], X.shape[1], self.gemm_w.shape[0]
                 rows.append(("fake_quant", lambda: self._fq(True),
@@ -234,6 +258,12 @@ class Runner:
             else:
                 rows.append(("fake_quant", lambda: self._fq(False), 6 * n_x, 3))
         return rows
+
+    def _fq_static(self):
+        nv = self.nv
+        X = self.fq_input
+        nv._call("nvfp4_fake_quant_static", nv._p(X), X.shape[0], X.shape[1], nv._p(self.calib_sg),
+                 nv._p(self.fq_out), nv._p(self.fq_packed), nv._p(self.fq_codes), nv._stream())
 
     def _fq(self, packed):
         nv = self.nv
@@ -266,7 +296,7 @@ class Runner:
         out = []
         for L in self.layers:
             out += [L.c_lh if "lh" in self.rules else L.c_46, L.packed]
-        if self.workload == "w4a4":
+        if self.workload in ("w4a4", "act_calib"):
             out += [self.fq_packed, self.fq_codes]
         if self.workload == "w4a4_gemm":
             out += [self.gemm_out]
@@ -513,6 +543,16 @@ def make_roofline(run, kernels, pk, pk_kind, workload, lh_evals):
             "evaluated_per_block": round(lh_evals / run.blocks(), 2),
             "all_126_equivalent_TFLOP/s": round(brute, 2),
         }
+    if "fake_quant_static" in kernels:
+        ms = kernels["abs_histogram"]["ms"] + kernels["fake_quant_static"]["ms"]
+        n = run.fq_input.numel()
+        achieved = FAKE_QUANT_BYTES_PER_ELEM * n / (ms / 1e3) / 1e9
+        hbm = float(pk.get("hbm_gbs", FALLBACK_HBM_GBS))
+        return {"kernel": "abs_histogram + fake_quant_static", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": None,
+                "peak_kind": "%s HBM copy bandwidth" % pk_kind,
+                "bytes_per_element": FAKE_QUANT_BYTES_PER_ELEM}
     if "gemm" in kernels:
         X = run.fq_input
         M, K, N = X.shape[0], X.shape[1], run.gw_packed.shape[0]
@@ -620,6 +660,25 @@ def cpu_baseline(run, budget_s=15.0):
                 "sample": "fake-quant of %d of %d token rows and their product with the "
                           "8192x8192 NVFP4 weight (%d activation blocks)"
                           % (n, X.shape[0], blocks)}
+    if run.workload == "act_calib":
+        X = run.fq_input
+
+        def step(n):
+            xu = _bits(X[:n])
+            t0 = time.perf_counter()
+            h = oracle.abs_histogram(xu)
+            sg = oracle.static_scale(oracle.quantile_magnitude(h, 0.9999))
+            oracle.fake_quant_static(xu, sg)
+            return time.perf_counter() - t0
+        t1, t2 = step(64), step(256)
+        per_row = max((t2 - t1) / 192, 1e-7)
+        n = int(max(1, min(X.shape[0], (budget_s - max(t1 - 64 * per_row, 0.0)) / per_row)))
+        t = step(n)
+        blocks = n * X.shape[1] // 16
+        return {"value": round(blocks / t, 2), "unit": UNIT, "cores": oracle.max_threads(),
+                "kind": "oracle", "seconds": round(t, 3),
+                "sample": "histogram, 99.99th-percentile scale and static fake-quant of %d of "
+                          "%d token rows (%d blocks)" % (n, X.shape[0], blocks)}
     if not run.layers:  # activation-only workload: fake-quant on leading rows
         X = run.fq_input
         t0 = time.perf_counter()
@@ -693,7 +752,7 @@ def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
         return
-    small = args.workload in ("tiny", "dense", "w4a4", "four_over_six", "w4a4_gemm")
+    small = args.workload in ("tiny", "dense", "w4a4", "four_over_six", "w4a4_gemm", "act_calib")
     dev = "cpu" if small or not torch.cuda.is_available() else "cuda"
     run = Runner(args.workload, dev)
     budget = args.cpu_seconds / max(1, args.steps)

@@ -9,9 +9,10 @@
 //  - abs_histogram_kernel: exact counts of |x| over the 32768 bf16
 //    magnitude patterns (one CTA per SM, a 128 KiB shared-memory histogram,
 //    shared atomics, non-zero bins flushed to the global uint64 histogram);
-//  - quantile_scale_kernel: one CTA scans the histogram for the p-quantile
-//    magnitude (the smallest m with at least ceil(p N) values at or below
-//    it) and writes s_g;
+//  - quantile_scale_kernel: one CTA finds the p-quantile magnitude (the
+//    smallest m with at least ceil(p N) values at or below it) -- per-warp
+//    chunk totals read coalesced, then the one warp whose chunk holds it
+//    walks that chunk -- and writes s_g;
 //  - quant_error_kernel + error_reduce_kernel: the sum of (x - y)^2 over a
 //    tensor for the bf16 fake-quant output y at a given s_g, in fp64, per-CTA
 //    partials added in a fixed order (the measure an error-based range
@@ -62,52 +63,57 @@ __global__ void __launch_bounds__(kHistThreads)
                          (unsigned long long)sh[i]);
 }
 
-// One CTA of 1024 threads, 32 bins each.
+// One CTA of 32 warps; warp w owns bins [1024 w, 1024 w + 1024), read
+// coalesced (lane l takes bins 1024 w + 32 j + l).
 __global__ void __launch_bounds__(kHistThreads)
     quantile_scale_kernel(const uint64_t *__restrict__ hist, double p, float *__restrict__ s_g) {
-  constexpr int kPer = kBins / kHistThreads;
-  __shared__ unsigned long long part[kHistThreads];
-  __shared__ int found;
-  const int t = threadIdx.x;
-  unsigned long long local = 0;
-  for (int j = 0; j < kPer; ++j) local += hist[t * kPer + j];
-  part[t] = local;
-  if (t == 0) found = kBins;
+  constexpr int kWarpBins = kBins / (kHistThreads / 32);  // 1024
+  __shared__ unsigned long long warp_total[kHistThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint64_t *h = hist + (size_t)warp * kWarpBins;
+  unsigned long long sum = 0;
+#pragma unroll 8
+  for (int j = 0; j < kWarpBins / 32; ++j) sum += h[j * 32 + lane];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+  if (lane == 0) warp_total[warp] = sum;
   __syncthreads();
-  // inclusive scan of the per-thread sums (Hillis-Steele)
-  for (int o = 1; o < kHistThreads; o <<= 1) {
-    const unsigned long long v = t >= o ? part[t - o] : 0ull;
-    __syncthreads();
-    part[t] += v;
-    __syncthreads();
+  // totals before this warp's chunk, and over all chunks (fixed order)
+  unsigned long long before = 0, total = 0;
+  for (int w = 0; w < kHistThreads / 32; ++w) {
+    if (w < warp) before += warp_total[w];
+    total += warp_total[w];
   }
-  const unsigned long long total = part[kHistThreads - 1];
   unsigned long long need = (unsigned long long)ceil(p * (double)total);
   if (need < 1ull) need = 1ull;
-  const unsigned long long before = t ? part[t - 1] : 0ull;
-  if (total > 0 && before < need && part[t] >= need) {
+  // the warp whose chunk holds the quantile walks it again in bin order
+  if (total > 0 && before < need && before + warp_total[warp] >= need) {
     unsigned long long acc = before;
-    for (int j = 0; j < kPer; ++j) {
-      acc += hist[t * kPer + j];
-      if (acc >= need) {
-        found = t * kPer + j;
-        break;
+    int found = -1;
+#pragma unroll 1
+    for (int j = 0; j < kWarpBins / 32 && found < 0; ++j) {
+      // inclusive prefix over the 32 bins of step j (bin order = lane order)
+      unsigned long long v = h[j * 32 + lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, v, o);
+        if (lane >= o) v += u;
+      }
+      const uint32_t hit = __ballot_sync(0xFFFFFFFFu, acc + v >= need);
+      if (hit) found = j * 32 + __ffs(hit) - 1;
+      acc += __shfl_sync(0xFFFFFFFFu, v, 31);
+    }
+    if (lane == 0) {
+      const float m = __uint_as_float((uint32_t)(warp * kWarpBins + found) << 16);
+      if (!isfinite(m)) {
+        atomicExch(&g_calib_status, (int)NVFP4_ERR_NONFINITE);
+        *s_g = __int_as_float(0x7FC00000);
+      } else {
+        *s_g = m == 0.0f ? 1.0f : __fdiv_rn(m, 2688.0f);
       }
     }
-  }
-  __syncthreads();
-  if (t == 0) {
-    if (total == 0 || found >= kBins) {
-      *s_g = 1.0f;
-      return;
-    }
-    const float m = __uint_as_float((uint32_t)found << 16);
-    if (!isfinite(m)) {
-      atomicExch(&g_calib_status, (int)NVFP4_ERR_NONFINITE);
-      *s_g = __int_as_float(0x7FC00000);
-    } else {
-      *s_g = m == 0.0f ? 1.0f : __fdiv_rn(m, 2688.0f);
-    }
+  } else if (total == 0 && threadIdx.x == 0) {
+    *s_g = 1.0f;
   }
 }
 

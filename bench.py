@@ -251,7 +251,7 @@ class Runner:
                                                           self.gw_packed, self.gw_codes,
                                                           self.gw_sg,
                                                           out=self.gemm_out),
-                                 M * K // 2 + N * K // 2 + M * N * 2, 7))
+                                 M * K // 2 + N * K // 2 + M * N * 2, 4))  # 2 scale layouts, alpha, GEMM
             elif self.workload == "w4a4":
                 rows.append(("fake_quant", lambda: self._fq(True),
                              FAKE_QUANT_BYTES_PER_ELEM * n_x, 3))

@@ -98,15 +98,13 @@ __device__ __forceinline__ void load_block(const uint16_t *p, uint32_t w[8]) {
 
 // ------------------------------------------------------- exact block encode
 //
-// Rounding rule used below (both for E2M1 codes and for the E4M3 max-rule
-// code): t, an fp32 value within one ulp of the exact quotient q, and t_alt,
-// the neighbouring float on the other side of q (chosen by the exact sign of
-// a residual), are rounded to nearest-even by the hardware conversion.  They
-// can only disagree when one of them is a rounding midpoint; q then lies
-// strictly on the other one's side, so the correct code is the odd one of the
-// two (the tie went to the even one).  When neither t is within two floats of
-// a value with 21 zero low mantissa bits (every E2M1 midpoint times a power of
-// two is such a value), t alone rounds exactly.
+// Exact rounding of a quotient q by the hardware nearest-even conversions.
+// The E4M3 max-rule code rounds t (within one float of q) and t_alt, the
+// neighbouring float on the other side of q (chosen by the exact sign of a
+// residual); the two can only disagree when one of them is a rounding
+// midpoint, q then lies strictly on the other one's side, and the correct
+// code is the odd one of the two (the tie went to the even one).  The E2M1
+// encode below needs the residual only for a t that could be a midpoint.
 
 // Four e2m1x2 conversions into one word: byte i = (code(h_i) << 4) | code(l_i),
 // signed inputs give signed codes (a negative value rounding to 0 gives -0).
@@ -133,26 +131,38 @@ __device__ __forceinline__ float toward(float t, float rho) {
 }
 
 // Packed signed E2M1 codes of 8 consecutive elements (4 bf16 pairs) at scale
-// s > 0 with r_hi + r_lo = 1/s (r_lo >= 0).  Every element is rounded twice:
-// t (within one float of q = x / s) and its neighbour on the other side of q
-// (by the exact sign of the residual x - t s, one fma).  The two codes can
-// differ only when one of the floats is an E2M1 rounding midpoint, which it
-// then rounds to its even neighbour, while q lies strictly on the other
-// side: the correct code is the odd one of the two.  Branch-free: exact ties
-// (q on a midpoint) are common for bf16 data at round scales.
+// s > 0 with r_hi + r_lo = 1/s (r_lo >= 0).  t = x (r_hi + r_lo) rounds
+// once from a value within 2^-45 (relative) of q = x / s, so it is one of the
+// two floats around q, and no float lies strictly between t and q.  Every
+// rounding midpoint (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5) is a float, so
+// when t is not one of them, rounding t to nearest-even gives q's code.
+// Midpoints have at most 3 significant bits; only a t with 21 zero low
+// mantissa bits (rare: an exact or nearly exact quotient) is stepped to its
+// neighbour across q by the exact sign of the residual x - t s (one fma),
+// which is t itself when q == t.  That neighbour has 24 significant bits, so
+// it is no midpoint and rounds like q: to the odd code when t was a midpoint
+// and q lies off it, to the even one on an exact tie.
 __device__ __forceinline__ uint32_t encode_word(const uint32_t *w, float s, float r_hi,
                                                 float r_lo) {
-  float t[8], ta[8];
+  float t[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
     t[e] = fmaf(x, r_hi, x * r_lo);
-    ta[e] = toward(t[e], fmaf(-t[e], s, x));
   }
-  const uint32_t ct = cvt4_e2m1(t[1], t[0], t[3], t[2], t[5], t[4], t[7], t[6]);
-  const uint32_t ca = cvt4_e2m1(ta[1], ta[0], ta[3], ta[2], ta[5], ta[4], ta[7], ta[6]);
-  const uint32_t odd = (ct & 0x11111111u) * 15u;
-  return (ct & odd) | (ca & ~odd);
+#pragma unroll
+  for (int p = 0; p < 8; p += 2) {
+    const bool n0 = (__float_as_uint(t[p]) & 0x1FFFFFu) == 0u;
+    const bool n1 = (__float_as_uint(t[p + 1]) & 0x1FFFFFu) == 0u;
+    if (n0 || n1) {
+      const float x0 = bf16_lo(w[p >> 1]), x1 = bf16_hi(w[p >> 1]);
+      const float a0 = toward(t[p], fmaf(-t[p], s, x0));
+      const float a1 = toward(t[p + 1], fmaf(-t[p + 1], s, x1));
+      t[p] = n0 ? a0 : t[p];
+      t[p + 1] = n1 ? a1 : t[p + 1];
+    }
+  }
+  return cvt4_e2m1(t[1], t[0], t[3], t[2], t[5], t[4], t[7], t[6]);
 }
 
 __device__ __forceinline__ uint2 encode_block(const uint32_t w[8], float s, float r_hi,

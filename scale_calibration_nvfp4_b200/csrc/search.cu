@@ -25,16 +25,17 @@
 //
 // Exact E2M1 codes without a fallback branch.  Candidate values are o * 2^p
 // with odd o in {1, 3, ..., 15}, and s(c) = fl(s_g o) 2^p exactly, so for each
-// element and each odd part o the quotient q = |w| / fl(s_g o) is formed once:
-// t from a double-float reciprocal (within one ulp of q), and t_alt, the
-// neighbouring float on the other side of q, chosen by the exact sign of the
-// residual |w| - t fl(s_g o) (one fma).  Candidates of class o scale both by
-// 2^-p exactly.  Round-to-nearest-even of t and of t_alt (hardware e2m1x2
-// conversion) can only disagree when one of them is a rounding midpoint; q
-// then lies strictly on the other one's side and the correct code is the odd
-// one of the two (the tie went to the even one).  Classes whose S passes
-// quotients_far_from_midpoints (no bf16 value comes near a midpoint) round t
-// alone.
+// element and each odd part o the quotient q = |w| / fl(s_g o) is formed once,
+// as t from a double-float reciprocal: t is one of the two floats around q.
+// Candidates of class o scale t by 2^-p exactly.  Every rounding midpoint of
+// E2M1 is a float with at most 3 significant bits, so a t with more bits is
+// no midpoint at any scale of the class, and its hardware round-to-nearest-
+// even gives q's code.  A t with at most 3 significant bits is replaced once
+// per class by its neighbouring float across q (by the exact sign of the
+// residual |w| - t fl(s_g o), one fma; t itself when q == t), which has 24
+// significant bits and so rounds like q.  Classes whose S passes
+// quotients_far_from_midpoints (no bf16 value comes near a midpoint) skip
+// that step.
 //
 // Winner: fp32 screen keeping the best three objectives; when the best two
 // are within 2^-12 (relative) or the best is numerically zero, the candidates
@@ -64,6 +65,8 @@ constexpr int kTileRows = 16;
 #endif
 constexpr int kTilesPerWarp = NVFP4_SEARCH_TILES;
 constexpr int kRowsPerCta = kWarps * kTileRows * kTilesPerWarp;  // 256
+static_assert((kRowsPerCta & (kRowsPerCta - 1)) == 0 && kRowsPerCta <= 65536,
+              "the row sort needs a power-of-two row count below 2^16");
 constexpr float kTieBand = 1.0f / 4096.0f;
 constexpr float kZeroFloor = 0x1p-40f;  // relative to ||p||^2
 constexpr int kMaxClasses = kCandidates;
@@ -299,27 +302,19 @@ __device__ __forceinline__ uint32_t pick4(uint32_t w0, uint32_t w1, uint32_t w2,
   return t == 0 ? w0 : (t == 1 ? w1 : (t == 2 ? w2 : w3));
 }
 
-// One candidate: codes (with or without the neighbouring-float correction),
-// the tensor-core product u, z = p - s u, and the row objective after a quad
-// reduce-scatter (lanes t < 2: row g, t >= 2: row g + 8).
-template <bool kLH, bool kAlt>
-__device__ __forceinline__ float candidate_objective(const float tq[8], const float ta[8],
-                                                     float f, float sm, uint32_t sgn,
-                                                     const uint32_t bh[2][2],
+// One candidate: codes, the tensor-core product u, z = p - s u, and the row
+// objective after a quad reduce-scatter (lanes t < 2: row g, t >= 2: row
+// g + 8).  tq holds the class quotients (stepped where a midpoint could
+// occur), f scales them to this candidate exactly.
+template <bool kLH>
+__device__ __forceinline__ float candidate_objective(const float tq[8], float f, float sm,
+                                                     uint32_t sgn, const uint32_t bh[2][2],
                                                      const uint32_t bl[2][2],
                                                      const float pz[2][4], bool upper) {
   const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  uint32_t code;
-  const uint32_t ct = cvt4_e2m1x2(tq[1] * f, tq[0] * f, tq[3] * f, tq[2] * f, tq[5] * f,
-                                  tq[4] * f, tq[7] * f, tq[6] * f);
-  if (kAlt) {
-    const uint32_t ca = cvt4_e2m1x2(ta[1] * f, ta[0] * f, ta[3] * f, ta[2] * f, ta[5] * f,
-                                    ta[4] * f, ta[7] * f, ta[6] * f);
-    const uint32_t odd = (ct & 0x11111111u) * 15u;
-    code = ((ct & odd) | (ca & ~odd)) | sgn;
-  } else {
-    code = ct | sgn;
-  }
+  const uint32_t code = cvt4_e2m1x2(tq[1] * f, tq[0] * f, tq[3] * f, tq[2] * f, tq[5] * f,
+                                    tq[4] * f, tq[7] * f, tq[6] * f) |
+                        sgn;
   uint32_t A[4];
   cvt4_f16x2(code, A);
   float u0[4], u1[4];
@@ -519,16 +514,18 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     keys[i] = key;
   }
   __syncthreads();
-  // bitonic sort of the 256 keys, ascending; one compare-exchange per thread
-  // and step
+  // bitonic sort of the keys, ascending; pair p of a step compares keys i
+  // and i + stride with i = 2p - (p mod stride), p < kRowsPerCta / 2
   for (int size = 2; size <= kRowsPerCta; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const int i = 2 * threadIdx.x - (threadIdx.x & (stride - 1));
-      const int j = i + stride;
-      const uint32_t ki = keys[i], kj = keys[j];
-      if ((ki > kj) == ((i & size) == 0)) {
-        keys[i] = kj;
-        keys[j] = ki;
+      for (int p = threadIdx.x; p < kRowsPerCta / 2; p += kThreads) {
+        const int i = 2 * p - (p & (stride - 1));
+        const int j = i + stride;
+        const uint32_t ki = keys[i], kj = keys[j];
+        if ((ki > kj) == ((i & size) == 0)) {
+          keys[i] = kj;
+          keys[j] = ki;
+        }
       }
       __syncthreads();
     }
@@ -632,21 +629,21 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     for (int k = 0; k < ncls; ++k) {
       const ClassInfo ci = cls[k];
       // class quotient t per element (within one float of q)
-      float tq[8], ta[8];
+      float tq[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) tq[e] = fmaf(a[e], ci.r_hi, a[e] * ci.r_lo);
-      // uncertified classes take the neighbour rounding for every candidate:
-      // at the scales where the certificate fails, some element of most
-      // tiles does sit near a midpoint
-      const bool alt = !ci.certified;
-      if (alt) {
-        // the neighbouring float of t on the other side of q, by the exact
-        // sign of the residual |w| - t S (t itself when exact)
+      // uncertified classes: a quotient with at most 3 significant bits
+      // (every rounding midpoint is one, and so is every power-of-two
+      // multiple) steps to its neighbouring float across q, by the exact
+      // sign of the residual |w| - t S; t itself when q == t.  Every other
+      // t is not a midpoint at any scale of the class and rounds like q.
+      if (!ci.certified) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float rho = fmaf(-tq[e], ci.S, a[e]);
           const int step = (rho > 0.0f) - (rho < 0.0f);
-          ta[e] = __int_as_float(__float_as_int(tq[e]) + step);
+          const bool near = (__float_as_uint(tq[e]) & 0x1FFFFFu) == 0u;
+          tq[e] = near ? __int_as_float(__float_as_int(tq[e]) + step) : tq[e];
         }
       }
       // first candidate of the class at or above smax (scales ascend within a
@@ -664,9 +661,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
                             (d > 0.0f && zl2 * d * d * (1.0f - 2.0f * kTieBand) > b1 + row_floor);
           if (__all_sync(0xFFFFFFFFu, done)) break;
         }
-        const float e0 =
-            alt ? candidate_objective<kLH, true>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper)
-                : candidate_objective<kLH, false>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
+        const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
         track3(key_of(e0, c0.c), b1, b2, b3);
         ++ncand;
       }
@@ -689,9 +684,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         const bool done = amax_row == 0.0f ||
                           zl2 * zero_sum * (1.0f - 2.0f * kTieBand) > b1 + row_floor;
         if (__all_sync(0xFFFFFFFFu, done)) break;
-        const float e0 =
-            alt ? candidate_objective<kLH, true>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper)
-                : candidate_objective<kLH, false>(tq, ta, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
+        const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
         track3(key_of(e0, c0.c), b1, b2, b3);
         ++ncand;
       }

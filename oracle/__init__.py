@@ -63,6 +63,10 @@ def lib():
         L.oracle_dequantize.argtypes = [vp, vp, f32, i64, i64, vp]
         L.oracle_fake_quant.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.oracle_max_threads.restype = i32
+        L.oracle_gram_full.argtypes = [vp, i64, i64, vp]
+        L.oracle_gptq_factor.argtypes = [vp, i64, f64, vp]
+        L.oracle_gptq_rows.argtypes = [vp, i64, f32, vp, vp, vp, i64, vp, vp]
+        L.oracle_gptq.argtypes = [vp, i64, i64, f32, vp, vp, f64, vp]
     return _lib
 
 
@@ -299,3 +303,50 @@ def fake_quant(x_u16, want_packed=True):
     _check(lib().oracle_fake_quant(_ptr(x), R, C, _ptr(out), _ptr(packed), _ptr(codes),
                                    ctypes.byref(s_g)))
     return out, packed, codes, np.float32(s_g.value)
+
+
+# ------------------------------------------------------------ full Gram, GPTQ
+def gram_full(x_u16, H=None):
+    """H += X^T X over all channels (fp64 [C, C])."""
+    x = _u16(x_u16)
+    N, C = x.shape
+    if H is None:
+        H = np.zeros((C, C), np.float64)
+    H = np.ascontiguousarray(H, np.float64)
+    _check(lib().oracle_gram_full(_ptr(x), N, C, _ptr(H)))
+    return H
+
+
+def gptq_factor(H, damp=0.01):
+    """Upper Cholesky factor U of (H + damp mean(diag H) I)^-1."""
+    H = np.ascontiguousarray(H, np.float64)
+    C = H.shape[0]
+    U = np.zeros((C, C), np.float64)
+    _check(lib().oracle_gptq_factor(_ptr(H), C, float(damp), _ptr(U)))
+    return U
+
+
+def gptq_rows(w_u16, s_g, codes, U, rows):
+    """GPTQ codes of the listed rows: (packed [n, C/2], value at rounding [n, C])."""
+    w = _u16(w_u16)
+    C = w.shape[1]
+    codes = np.ascontiguousarray(codes, np.uint8)
+    U = np.ascontiguousarray(U, np.float64)
+    rows = np.ascontiguousarray(rows, np.int64)
+    packed = np.zeros((rows.size, C // 2), np.uint8)
+    wq = np.zeros((rows.size, C), np.float64)
+    _check(lib().oracle_gptq_rows(_ptr(w), C, float(s_g), _ptr(codes), _ptr(U), _ptr(rows),
+                                  rows.size, _ptr(packed), _ptr(wq)))
+    return packed, wq
+
+
+def gptq(w_u16, s_g, codes, H, damp=0.01):
+    """Packed GPTQ codes of W [R, C] at the given block codes."""
+    w = _u16(w_u16)
+    R, C = w.shape
+    codes = np.ascontiguousarray(codes, np.uint8)
+    H = np.ascontiguousarray(H, np.float64)
+    packed = np.zeros((R, C // 2), np.uint8)
+    _check(lib().oracle_gptq(_ptr(w), R, C, float(s_g), _ptr(codes), _ptr(H), float(damp),
+                             _ptr(packed)))
+    return packed

@@ -23,7 +23,12 @@
  *   [LH]    "4 比特量化到底让模型笨了多少？" (2kiu.com), a write-up of NVIDIA
  *           Model Optimizer's "Improving NVFP4 Accuracy with Local-Hessian
  *           Weight Scales"; sections "The NVFP4 structure" and "A different
- *           objective: output error as the ruler".
+ *           objective: output error as the ruler", "Trying it" (Local-Hessian
+ *           combined with GPTQ).
+ *   [GPTQ]  Frantar, Ashkboos, Hoefler, Alistarh, "GPTQ: Accurate
+ *           Post-Training Quantization for Generative Pre-trained
+ *           Transformers" (the paper [LH] links): dampening, the Cholesky
+ *           reformulation and the column-by-column rounding loop.
  *
  * Readings where the pages are silent (each is also listed in the design
  * notes): the tensor scale s_g = fl32(amax / (6*448)) (1 when amax = 0);
@@ -626,6 +631,180 @@ double oracle_quant_error(const uint16_t *x, int64_t rows, int64_t C, float s_g)
     }
     free(y);
     return e;
+}
+
+/* ----------------------------------------------------- full Gram, GPTQ */
+
+/* Full Gram accumulation H += X^T X over all C channels (C x C, row-major,
+ * fp64).  [LH] "A different objective": the output-error Hessian is X X^T;
+ * "Trying it": Local-Hessian can be combined with GPTQ, which needs the whole
+ * matrix, not only its 16x16 diagonal blocks. */
+int oracle_gram_full(const uint16_t *x, int64_t n_tok, int64_t C, double *H)
+{
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t a = 0; a < C; a++)
+        for (int64_t b = 0; b < C; b++) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < n_tok; t++)
+                acc += oracle_bf16_to_double(x[t * C + a]) * oracle_bf16_to_double(x[t * C + b]);
+            H[a * C + b] += acc;
+        }
+    return ORACLE_OK;
+}
+
+/* GPTQ (Frantar, Ashkboos, Hoefler, Alistarh, "GPTQ: Accurate Post-Training
+ * Quantization for Generative Pre-trained Transformers"), as [LH] "Trying it"
+ * combines it with Local-Hessian scales: the block scales are given (from any
+ * scale rule) and GPTQ changes only the rounding.  The paper quantises the
+ * columns of W one at a time, in order, and after column j moves the columns
+ * not yet quantised to compensate its error, through the inverse Hessian:
+ *   (dampening)  H <- H + lambda I, lambda = damp * mean(diag H)
+ *   (Cholesky reformulation)  U = the upper Cholesky factor of H^-1
+ *   for j = 0..C-1:  q_j = quant(w_j);  e = (w_j - q_j) / U_jj;
+ *                    w_k <- w_k - e U_jk  for every k > j.
+ * The factor step, once per Hessian: U (C x C upper, row-major) from H.
+ * Plain fp64: H + lambda I = L L^T, H^-1 = L^-T L^-1, H^-1 = U^T U.
+ * Returns ORACLE_ERR_NOT_SPD when a pivot is not positive. */
+#define ORACLE_ERR_NOT_SPD 9
+int oracle_gptq_factor(const double *H, int64_t C, double damp, double *U)
+{
+    double *L = (double *)calloc((size_t)(C * C), sizeof(double));
+    double *Li = (double *)calloc((size_t)(C * C), sizeof(double));
+    double *Hi = (double *)calloc((size_t)(C * C), sizeof(double));
+    if (!L || !Li || !Hi) {
+        free(L); free(Li); free(Hi);
+        return ORACLE_ERR_SHAPE;
+    }
+    int st = ORACLE_OK;
+    double mean = 0.0;
+    for (int64_t i = 0; i < C; i++)
+        mean += H[i * C + i];
+    mean /= (double)C;
+    double lambda = damp * mean;
+    /* H + lambda I = L L^T (lower, column by column) */
+    for (int64_t j = 0; j < C && st == ORACLE_OK; j++) {
+        double d = H[j * C + j] + lambda;
+        for (int64_t k = 0; k < j; k++)
+            d -= L[j * C + k] * L[j * C + k];
+        if (!(d > 0.0)) {
+            st = ORACLE_ERR_NOT_SPD;
+            break;
+        }
+        double ljj = sqrt(d);
+        L[j * C + j] = ljj;
+#pragma omp parallel for schedule(static)
+        for (int64_t i = j + 1; i < C; i++) {
+            double v = H[i * C + j];
+            for (int64_t k = 0; k < j; k++)
+                v -= L[i * C + k] * L[j * C + k];
+            L[i * C + j] = v / ljj;
+        }
+    }
+    if (st == ORACLE_OK) {
+        /* L^-1 (lower), one column per unit vector, forward substitution */
+#pragma omp parallel for schedule(dynamic, 8)
+        for (int64_t c = 0; c < C; c++)
+            for (int64_t i = c; i < C; i++) {
+                double v = (i == c) ? 1.0 : 0.0;
+                for (int64_t k = c; k < i; k++)
+                    v -= L[i * C + k] * Li[k * C + c];
+                Li[i * C + c] = v / L[i * C + i];
+            }
+        /* H^-1 = L^-T L^-1: entry (a, b) = sum over k >= max(a, b) */
+#pragma omp parallel for schedule(dynamic, 8)
+        for (int64_t a = 0; a < C; a++)
+            for (int64_t b = 0; b < C; b++) {
+                double v = 0.0;
+                for (int64_t k = (a > b ? a : b); k < C; k++)
+                    v += Li[k * C + a] * Li[k * C + b];
+                Hi[a * C + b] = v;
+            }
+        /* H^-1 = U^T U (upper, row by row) */
+        memset(U, 0, sizeof(double) * (size_t)(C * C));
+        for (int64_t i = 0; i < C && st == ORACLE_OK; i++) {
+            double d = Hi[i * C + i];
+            for (int64_t k = 0; k < i; k++)
+                d -= U[k * C + i] * U[k * C + i];
+            if (!(d > 0.0)) {
+                st = ORACLE_ERR_NOT_SPD;
+                break;
+            }
+            double uii = sqrt(d);
+            U[i * C + i] = uii;
+#pragma omp parallel for schedule(static)
+            for (int64_t j = i + 1; j < C; j++) {
+                double v = Hi[i * C + j];
+                for (int64_t k = 0; k < i; k++)
+                    v -= U[k * C + i] * U[k * C + j];
+                U[i * C + j] = v / uii;
+            }
+        }
+    }
+    free(L); free(Li); free(Hi);
+    return st;
+}
+
+/* The column loop for a list of rows (rows are independent given U): packed
+ * GPTQ codes of each listed row ([n_rows][C/2], nibble order of
+ * oracle_quantize_pack) and, when wq is not NULL, the value each element
+ * had when it was rounded ([n_rows][C]).  The quantised value q_j = v s_eff
+ * is exact in fp64, and so is the rounding decision (oracle_e2m1_encode). */
+int oracle_gptq_rows(const uint16_t *w, int64_t C, float s_g, const uint8_t *codes,
+                     const double *U, const int64_t *rows, int64_t n_rows, uint8_t *packed,
+                     double *wq)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    int64_t nb = C / 16;
+    int st = ORACLE_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < n_rows; n++) {
+        int64_t r = rows[n];
+        double *x = (double *)malloc(sizeof(double) * (size_t)C);
+        if (!x) {
+            st = ORACLE_ERR_SHAPE;
+            continue;
+        }
+        for (int64_t i = 0; i < C; i++)
+            x[i] = oracle_bf16_to_double(w[r * C + i]);
+        for (int64_t j = 0; j < C; j++) {
+            double s = (double)oracle_effective_scale(s_g, codes[r * nb + j / 16]);
+            int q = oracle_e2m1_encode(x[j], s);
+            if (wq)
+                wq[n * C + j] = x[j];
+            if (j & 1)
+                packed[n * (C / 2) + j / 2] |= (uint8_t)(q << 4);
+            else
+                packed[n * (C / 2) + j / 2] = (uint8_t)q;
+            double e = (x[j] - oracle_e2m1_value(q) * s) / U[j * C + j];
+            for (int64_t k = j + 1; k < C; k++)
+                x[k] -= e * U[j * C + k];
+        }
+        free(x);
+    }
+    return st;
+}
+
+/* Whole-matrix GPTQ rounding of W [R, C] with its Hessian H [C, C]. */
+int oracle_gptq(const uint16_t *w, int64_t R, int64_t C, float s_g, const uint8_t *codes,
+                const double *H, double damp, uint8_t *packed)
+{
+    if (C % 16)
+        return ORACLE_ERR_SHAPE;
+    double *U = (double *)malloc(sizeof(double) * (size_t)(C * C));
+    int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)(R > 0 ? R : 1));
+    if (!U || !rows) {
+        free(U); free(rows);
+        return ORACLE_ERR_SHAPE;
+    }
+    int st = oracle_gptq_factor(H, C, damp, U);
+    if (st == ORACLE_OK) {
+        for (int64_t r = 0; r < R; r++)
+            rows[r] = r;
+        st = oracle_gptq_rows(w, C, s_g, codes, U, rows, R, packed, NULL);
+    }
+    free(U); free(rows);
+    return st;
 }
 
 int oracle_max_threads(void)

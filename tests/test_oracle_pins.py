@@ -566,3 +566,117 @@ def test_quant_error_is_sum_of_squared_differences(oracle_mod):
         y, _, _ = oracle_mod.fake_quant_static(x, s_g, want_packed=False)
         ref = float(np.sum((bits_to_f64(x) - bits_to_f64(y)) ** 2))
         assert math.isclose(oracle_mod.quant_error(x, s_g), ref, rel_tol=1e-12)
+
+
+# ------------------------------------------------------------ full Gram, GPTQ
+def _np_e2m1_round(x, s):
+    """Independent E2M1 rounding of fp64 values at scale s > 0: nearest grid
+    magnitude, ties to the even magnitude index, saturating at 6; returns the
+    signed quantised value v(q) * s and the code."""
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    a = np.abs(x)
+    k = np.zeros(a.shape, np.int64)
+    for i in range(7):
+        thr = 0.5 * (grid[i] + grid[i + 1]) * s  # exact in fp64
+        up = (a > thr) if i % 2 == 0 else (a >= thr)
+        k = np.where(up, i + 1, k)
+    code = k | np.where(np.signbit(x), 8, 0)
+    return np.where(np.signbit(x), -1.0, 1.0) * grid[k] * s, code
+
+
+def _gptq_obs_reference(W, S, H, damp):
+    """GPTQ in its Optimal-Brain-Surgeon form (the GPTQ paper, before the
+    Cholesky reformulation): quantise column j, move the remaining weights by
+    -(w_j - q_j) / [H^-1]_jj * [H^-1]_{j,:}, then remove j from the inverse
+    Hessian by one step of Gaussian elimination.  S: per-element scales."""
+    C = H.shape[0]
+    Hd = H + damp * np.mean(np.diag(H)) * np.eye(C)
+    Hi = np.linalg.inv(Hd)
+    Wc = W.copy()
+    codes = np.zeros(W.shape, np.int64)
+    at = np.zeros(W.shape)
+    for j in range(C):
+        at[:, j] = Wc[:, j]
+        q, codes[:, j] = _np_e2m1_round(Wc[:, j], S[:, j])
+        d = (Wc[:, j] - q) / Hi[j, j]
+        Wc[:, j + 1:] -= np.outer(d, Hi[j, j + 1:])
+        Hi = Hi - np.outer(Hi[:, j], Hi[j, :]) / Hi[j, j]
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    return packed, at
+
+
+def _gptq_case(oracle_mod, R, C, N, seed):
+    W, X = _tiny_layer(R, C, N, seed)
+    s_g = oracle_mod.global_scale(W)
+    codes = oracle_mod.scale_search_max(W, s_g)
+    H = oracle_mod.gram_full(X)
+    S = np.repeat(np.array([[oracle_mod.effective_scale(s_g, c) for c in row] for row in codes],
+                           np.float64), 16, axis=1)
+    return W, X, s_g, codes, H, S
+
+
+def test_full_gram_is_library_product(oracle_mod):
+    W, X = _tiny_layer(4, 64, 40, 11)
+    H = oracle_mod.gram_full(X)
+    Xf = bits_to_f64(X)
+    np.testing.assert_allclose(H, Xf.T @ Xf, rtol=1e-14, atol=0)
+    # its 16x16 diagonal blocks are the block-diagonal Gram
+    Hb = oracle_mod.gram(X)
+    for j in range(4):
+        np.testing.assert_array_equal(H[16 * j:16 * j + 16, 16 * j:16 * j + 16], Hb[j])
+
+
+def test_gptq_factor_is_cholesky_of_inverse(oracle_mod):
+    _, X = _tiny_layer(2, 48, 64, 12)
+    H = oracle_mod.gram_full(X)
+    U = oracle_mod.gptq_factor(H, 0.01)
+    Hd = H + 0.01 * np.mean(np.diag(H)) * np.eye(48)
+    assert np.all(np.tril(U, -1) == 0) and np.all(np.diag(U) > 0)
+    np.testing.assert_allclose(U.T @ U, np.linalg.inv(Hd), rtol=1e-9,
+                               atol=1e-12 * np.abs(np.linalg.inv(Hd)).max())
+
+
+def test_gptq_with_diagonal_hessian_is_plain_rounding(oracle_mod):
+    W, X, s_g, codes, _, _ = _gptq_case(oracle_mod, 16, 64, 32, 13)
+    rng = np.random.default_rng(13)
+    H = np.diag(rng.uniform(0.5, 40.0, 64))
+    np.testing.assert_array_equal(oracle_mod.gptq(W, s_g, codes, H, 0.01),
+                                  oracle_mod.quantize_pack(W, s_g, codes))
+
+
+def test_gptq_two_coupled_columns_closed_form(oracle_mod):
+    # H couples only columns 0 and 1: after column 0 is rounded, the output
+    # error is least when w_1 moves by (w_0 - q_0) H01 / H11 (dampened H);
+    # every other column is rounded as it is
+    W, X, s_g, codes, _, S = _gptq_case(oracle_mod, 16, 32, 32, 14)
+    H = np.eye(32) * 3.0
+    H[0, 0], H[1, 1], H[0, 1], H[1, 0] = 5.0, 2.0, 1.5, 1.5
+    damp = 0.01
+    Hd = H + damp * np.mean(np.diag(H)) * np.eye(32)
+    U = oracle_mod.gptq_factor(H, damp)
+    packed, at = oracle_mod.gptq_rows(W, s_g, codes, U, np.arange(16))
+    Wf = bits_to_f64(W)
+    q0, _ = _np_e2m1_round(Wf[:, 0], S[:, 0])
+    np.testing.assert_allclose(at[:, 1], Wf[:, 1] + (Wf[:, 0] - q0) * Hd[0, 1] / Hd[1, 1],
+                               rtol=1e-12, atol=1e-15)
+    np.testing.assert_array_equal(at[:, 2:], Wf[:, 2:])
+    np.testing.assert_array_equal(at[:, 0], Wf[:, 0])
+
+
+@pytest.mark.parametrize("R,C,N,seed", [(12, 48, 80, 15), (7, 64, 30, 16)])
+def test_gptq_equals_obs_elimination_form(oracle_mod, R, C, N, seed):
+    W, X, s_g, codes, H, S = _gptq_case(oracle_mod, R, C, N, seed)
+    ref_packed, ref_at = _gptq_obs_reference(bits_to_f64(W), S, H, 0.01)
+    U = oracle_mod.gptq_factor(H, 0.01)
+    packed, at = oracle_mod.gptq_rows(W, s_g, codes, U, np.arange(R))
+    np.testing.assert_allclose(at, ref_at, rtol=1e-9, atol=1e-12)
+    np.testing.assert_array_equal(packed, ref_packed)
+    np.testing.assert_array_equal(oracle_mod.gptq(W, s_g, codes, H, 0.01), packed)
+
+
+def test_gptq_not_positive_definite_is_reported(oracle_mod):
+    W, X, s_g, codes, H, _ = _gptq_case(oracle_mod, 4, 32, 16, 17)
+    bad = np.eye(32)
+    bad[5, 5] = -4.0
+    with pytest.raises(Exception):
+        oracle_mod.gptq(W, s_g, codes, bad, 0.0)

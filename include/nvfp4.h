@@ -69,9 +69,12 @@ typedef enum nvfp4_status {
     NVFP4_ERR_CUDA = 5,            /* a CUDA runtime call or launch failed */
     NVFP4_ERR_NOT_IMPLEMENTED = 6,
     NVFP4_ERR_TOO_LARGE = 7,       /* request beyond a documented maximum */
-    NVFP4_ERR_DEVICE_TIMEOUT = 8   /* a kernel gave up waiting (one second) for its own
+    NVFP4_ERR_DEVICE_TIMEOUT = 8,  /* a kernel gave up waiting (one second) for its own
                                       tile copies; its output was not written
                                       (device-side report) */
+    NVFP4_ERR_NOT_POSITIVE_DEFINITE = 9 /* a dampened Hessian had a non-positive (or
+                                           non-finite) Cholesky pivot; the GPTQ output
+                                           is not usable (device-side report) */
 } nvfp4_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -272,8 +275,8 @@ nvfp4_status nvfp4_quant_error(const uint16_t *x, int64_t rows, int64_t C, const
 
 /*
  * Reads and clears the device-side status of the current device after
- * synchronising `stream`.  *out is NVFP4_OK, NVFP4_ERR_NONFINITE or
- * NVFP4_ERR_DEVICE_TIMEOUT.
+ * synchronising `stream`.  *out is NVFP4_OK, NVFP4_ERR_NONFINITE,
+ * NVFP4_ERR_DEVICE_TIMEOUT or NVFP4_ERR_NOT_POSITIVE_DEFINITE.
  */
 nvfp4_status nvfp4_get_device_status(void *stream, nvfp4_status *out);
 
@@ -298,6 +301,46 @@ nvfp4_status nvfp4_get_device_status(void *stream, nvfp4_status *out);
 nvfp4_status nvfp4_gemm(const uint8_t *a_packed, const uint8_t *a_codes, const float *a_sg,
                         const uint8_t *b_packed, const uint8_t *b_codes, const float *b_sg,
                         int64_t M, int64_t N, int64_t K, uint16_t *out, void *stream);
+
+/*
+ * Full Gram accumulation ([LH] "A different objective": the output-error
+ * Hessian is X X^T; "Trying it": GPTQ, combined there with Local-Hessian
+ * scales, needs all of it):
+ *   H[a][b] += sum_t x[t][a] x[t][b]   for all a, b < C
+ * on the tensor cores (bf16 products, fp32 accumulation and sum into H).
+ *   x  [n_tok, C] bf16 (tokens by channels), 16-byte aligned
+ *   H  [C, C] float, row-major, accumulated in place (16-byte aligned)
+ * C must be a multiple of 16 (NVFP4_ERR_SHAPE).  Workspace, if the kernel
+ * needs any, is stream-ordered scratch from the library pool.  Returns
+ * NVFP4_ERR_NOT_IMPLEMENTED if the kernel cannot take the shape.
+ */
+nvfp4_status nvfp4_hessian_full_accumulate(const uint16_t *x, int64_t n_tok, int64_t C, float *H,
+                                           void *stream);
+
+/*
+ * GPTQ rounding at given block scales (GPTQ: Frantar et al., "GPTQ: Accurate
+ * Post-Training Quantization for Generative Pre-trained Transformers";
+ * [LH] "Trying it": Local-Hessian chooses the scales, GPTQ the rounding).
+ * The columns of each row are rounded in order (E2M1 nearest-even at the
+ * block's s_eff, exact), and every column not yet rounded first moves by
+ * the rounding errors of the earlier ones so that ||(W - Q) X||^2 stays
+ * least, through the dampened Hessian H + lambda I, lambda = damp *
+ * mean(diag H).  All of it in fp64.
+ *   w            [batch, R, C] bf16 (16-byte aligned)
+ *   s_g          DEVICE [batch] float
+ *   scale_codes  [batch, R, C/16] uint8, E4M3 codes 0..126 (any scale rule)
+ *   H            [batch, C, C] float (e.g. from nvfp4_hessian_full_accumulate);
+ *                only its lower triangle is read
+ *   damp         >= 0 (the GPTQ paper uses 0.01)
+ *   packed       [batch, R, C/2] uint8, written (nibble order of
+ *                nvfp4_quantize_pack)
+ * Scratch (stream-ordered, library pool): batch (C^2 + R C) doubles.  A
+ * Hessian that is not positive definite after dampening sets the device
+ * status NVFP4_ERR_NOT_POSITIVE_DEFINITE (see nvfp4_get_device_status).
+ */
+nvfp4_status nvfp4_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, const float *s_g,
+                        const uint8_t *scale_codes, const float *H, double damp,
+                        uint8_t *packed, void *stream);
 
 /*
  * Work statistic of the scale searches (the pages have no counterpart; it

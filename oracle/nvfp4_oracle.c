@@ -701,44 +701,52 @@ int oracle_gptq_factor(const double *H, int64_t C, double damp, double *U)
         }
     }
     if (st == ORACLE_OK) {
-        /* L^-1 (lower), one column per unit vector, forward substitution */
+        /* L^-1 (lower), one column c per unit vector by forward substitution;
+         * stored transposed (Li[c][i] = (L^-1)[i][c]) so the sums run along
+         * rows */
 #pragma omp parallel for schedule(dynamic, 8)
         for (int64_t c = 0; c < C; c++)
             for (int64_t i = c; i < C; i++) {
                 double v = (i == c) ? 1.0 : 0.0;
                 for (int64_t k = c; k < i; k++)
-                    v -= L[i * C + k] * Li[k * C + c];
-                Li[i * C + c] = v / L[i * C + i];
+                    v -= L[i * C + k] * Li[c * C + k];
+                Li[c * C + i] = v / L[i * C + i];
             }
-        /* H^-1 = L^-T L^-1: entry (a, b) = sum over k >= max(a, b) */
+        /* H^-1 = L^-T L^-1: entry (a, b) = sum over k >= max(a, b) of
+         * (L^-1)[k][a] (L^-1)[k][b] */
 #pragma omp parallel for schedule(dynamic, 8)
         for (int64_t a = 0; a < C; a++)
             for (int64_t b = 0; b < C; b++) {
                 double v = 0.0;
                 for (int64_t k = (a > b ? a : b); k < C; k++)
-                    v += Li[k * C + a] * Li[k * C + b];
+                    v += Li[a * C + k] * Li[b * C + k];
                 Hi[a * C + b] = v;
             }
-        /* H^-1 = U^T U (upper, row by row) */
-        memset(U, 0, sizeof(double) * (size_t)(C * C));
+        /* H^-1 = U^T U (U upper), row i of U finished at step i; built as its
+         * transpose Ut (lower, Ut[j][i] = U[i][j]) so the sums run along rows */
+        double *Ut = L; /* L is no longer needed */
+        memset(Ut, 0, sizeof(double) * (size_t)(C * C));
         for (int64_t i = 0; i < C && st == ORACLE_OK; i++) {
             double d = Hi[i * C + i];
             for (int64_t k = 0; k < i; k++)
-                d -= U[k * C + i] * U[k * C + i];
+                d -= Ut[i * C + k] * Ut[i * C + k];
             if (!(d > 0.0)) {
                 st = ORACLE_ERR_NOT_SPD;
                 break;
             }
             double uii = sqrt(d);
-            U[i * C + i] = uii;
+            Ut[i * C + i] = uii;
 #pragma omp parallel for schedule(static)
             for (int64_t j = i + 1; j < C; j++) {
                 double v = Hi[i * C + j];
                 for (int64_t k = 0; k < i; k++)
-                    v -= U[k * C + i] * U[k * C + j];
-                U[i * C + j] = v / uii;
+                    v -= Ut[i * C + k] * Ut[j * C + k];
+                Ut[j * C + i] = v / uii;
             }
         }
+        for (int64_t i = 0; i < C; i++)
+            for (int64_t j = 0; j < C; j++)
+                U[i * C + j] = (j >= i) ? Ut[j * C + i] : 0.0;
     }
     free(L); free(Li); free(Hi);
     return st;

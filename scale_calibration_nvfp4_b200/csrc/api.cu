@@ -2,6 +2,7 @@
 // the host, then launches on the caller's stream.  Nothing here computes on
 // the data.
 #include <climits>
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -112,6 +113,7 @@ const char *nvfp4_status_string(nvfp4_status st) {
     case NVFP4_ERR_NOT_IMPLEMENTED: return "NVFP4_ERR_NOT_IMPLEMENTED";
     case NVFP4_ERR_TOO_LARGE: return "NVFP4_ERR_TOO_LARGE";
     case NVFP4_ERR_DEVICE_TIMEOUT: return "NVFP4_ERR_DEVICE_TIMEOUT";
+    case NVFP4_ERR_NOT_POSITIVE_DEFINITE: return "NVFP4_ERR_NOT_POSITIVE_DEFINITE";
   }
   return "NVFP4_ERR_UNKNOWN";
 }
@@ -133,6 +135,17 @@ nvfp4_status nvfp4_hessian_accumulate(const uint16_t *x, int64_t n_tok, int64_t 
   if (C / 16 > 8 * 65535) return NVFP4_ERR_TOO_LARGE;
   if ((x && !aligned(x, 16)) || !aligned(H, 4)) return NVFP4_ERR_MISALIGNED;
   return map_cuda(nvfp4::launch_gram(x, nullptr, 1, n_tok, C, H, as_stream(stream)));
+}
+
+nvfp4_status nvfp4_hessian_full_accumulate(const uint16_t *x, int64_t n_tok, int64_t C,
+                                           float *H, void *stream) {
+  if (n_tok < 0 || C < 0 || !H || (n_tok > 0 && !x)) return NVFP4_ERR_INVALID_ARG;
+  if (C % 16 || !fits(n_tok, C) || !fits(C, C)) return NVFP4_ERR_SHAPE;
+  if (C > INT32_MAX || n_tok > INT32_MAX) return NVFP4_ERR_TOO_LARGE;
+  if ((x && !aligned(x, 16)) || !aligned(H, 16)) return NVFP4_ERR_MISALIGNED;
+  const cudaError_t e = nvfp4::launch_gram_full(x, n_tok, C, H, as_stream(stream));
+  if (e == cudaErrorNotSupported) return NVFP4_ERR_NOT_IMPLEMENTED;
+  return map_cuda(e);
 }
 
 nvfp4_status nvfp4_hessian_accumulate_noalloc(const uint16_t *x, int64_t n_tok, int64_t C,
@@ -271,6 +284,19 @@ nvfp4_status nvfp4_get_device_status(void *stream, nvfp4_status *out) {
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   *out = (nvfp4_status)v;
   return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, const float *s_g,
+                        const uint8_t *scale_codes, const float *H, double damp,
+                        uint8_t *packed, void *stream) {
+  const nvfp4_status st = check_weight_args(w, batch, R, C, s_g, scale_codes);
+  if (st != NVFP4_OK) return st;
+  if (!H || !packed || !(damp >= 0.0) || !(damp < INFINITY)) return NVFP4_ERR_INVALID_ARG;
+  if (!fits(batch, C, C) || !fits(batch, R, C)) return NVFP4_ERR_SHAPE;
+  if ((R + 63) / 64 > 65535) return NVFP4_ERR_TOO_LARGE;
+  if (!aligned(H, 4)) return NVFP4_ERR_MISALIGNED;
+  return map_cuda(nvfp4::launch_gptq(w, batch, R, C, s_g, scale_codes, H, damp, packed,
+                                     as_stream(stream)));
 }
 
 nvfp4_status nvfp4_search_evaluations(void *stream, int reset, uint64_t *out) {

@@ -66,6 +66,17 @@ cudaError_t launch_quant_error(const uint16_t *x, int64_t rows, int64_t C, const
                                double *err, cudaStream_t st);
 cudaError_t read_and_clear_calib_status(cudaStream_t st, int *out);
 
+// Full Gram H [C, C] += X^T X on the tensor cores.
+cudaError_t launch_gram_full(const uint16_t *x, int64_t n_tok, int64_t C, float *H,
+                             cudaStream_t st);
+
+// GPTQ rounding of W [batch, R, C] at the given block codes with the
+// Hessians H [batch, C, C]; packed [batch, R, C/2].
+cudaError_t launch_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, const float *s_g,
+                        const uint8_t *codes, const float *H, double damp, uint8_t *packed,
+                        cudaStream_t st);
+cudaError_t read_and_clear_gptq_status(cudaStream_t st, int *out);
+
 // Stream-ordered scratch from the library's pool on the current device.
 cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t st);
 cudaError_t scratch_free(void *p, cudaStream_t st);

@@ -646,11 +646,13 @@ cudaError_t read_and_clear_device_status(cudaStream_t st, int *out) {
   e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
   if (e != cudaSuccess) return e;
   // the Gram kernels keep their own flag (a timed-out wait), the
-  // calibration kernels theirs (a quantile on a non-finite value)
-  int gram = 0, calib = 0;
+  // calibration kernels theirs (a quantile on a non-finite value), the GPTQ
+  // kernels theirs (a Hessian that is not positive definite)
+  int gram = 0, calib = 0, gptq = 0;
   e = read_and_clear_gram_status(st, &gram);
   if (e == cudaSuccess) e = read_and_clear_calib_status(st, &calib);
-  if (*out == 0) *out = gram ? gram : calib;
+  if (e == cudaSuccess) e = read_and_clear_gptq_status(st, &gptq);
+  if (*out == 0) *out = gram ? gram : (calib ? calib : gptq);
   return e;
 }
 

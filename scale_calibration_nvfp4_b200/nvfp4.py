@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
 STATUS = {
     0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_SHAPE", 3: "NVFP4_ERR_MISALIGNED",
     4: "NVFP4_ERR_NONFINITE", 5: "NVFP4_ERR_CUDA", 6: "NVFP4_ERR_NOT_IMPLEMENTED",
-    7: "NVFP4_ERR_TOO_LARGE", 8: "NVFP4_ERR_DEVICE_TIMEOUT",
+    7: "NVFP4_ERR_TOO_LARGE", 8: "NVFP4_ERR_DEVICE_TIMEOUT", 9: "NVFP4_ERR_NOT_POSITIVE_DEFINITE",
 }
 
 # C entry points and their argument types (mirrors include/nvfp4.h)
@@ -43,6 +43,8 @@ SIGNATURES = {
     "nvfp4_static_scale_from_histogram": [_vp, ctypes.c_double, _vp, _vp],
     "nvfp4_fake_quant_static": [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp],
     "nvfp4_quant_error": [_vp, _i64, _i64, _vp, _vp, _vp],
+    "nvfp4_hessian_full_accumulate": [_vp, _i64, _i64, _vp, _vp],
+    "nvfp4_gptq": [_vp, _i64, _i64, _i64, _vp, _vp, _vp, ctypes.c_double, _vp, _vp],
 }
 
 
@@ -132,6 +134,17 @@ def hessian_accumulate(x, H, stream=None):
     if H.numel() != (C // 16) * 256:
         raise ValueError("H must hold C/16 x 16 x 16 floats")
     _call("nvfp4_hessian_accumulate", _p(x), N, C, _p(H), _stream(stream))
+    return H
+
+
+def hessian_full_accumulate(x, H, stream=None):
+    """H[C, C] += x^T x over all channels (in place, tensor cores)."""
+    _need(x, torch.bfloat16, "x")
+    _need(H, torch.float32, "H")
+    N, C = x.shape
+    if H.numel() != C * C:
+        raise ValueError("H must hold C x C floats")
+    _call("nvfp4_hessian_full_accumulate", _p(x), N, C, _p(H), _stream(stream))
     return H
 
 
@@ -233,6 +246,25 @@ def quantize_pack(w, s_g, scale_codes, out=None, stream=None):
         out = torch.empty(shape, dtype=torch.uint8, device=w.device)
     _need(out, torch.uint8, "packed")
     _call("nvfp4_quantize_pack", _p(w), B, R, C, _p(s_g), _p(scale_codes), _p(out),
+          _stream(stream))
+    return out
+
+
+def gptq(w, s_g, scale_codes, H, damp=0.01, out=None, stream=None):
+    """Packed GPTQ codes of w ([R, C] or [batch, R, C]) at the given block
+    codes, with the full Hessian(s) H ([C, C] or [batch, C, C], float32)."""
+    _need(w, torch.bfloat16, "w")
+    _need(s_g, torch.float32, "s_g")
+    _need(scale_codes, torch.uint8, "scale_codes")
+    _need(H, torch.float32, "H")
+    B, R, C = _weight_shape(w)
+    if H.numel() != B * C * C:
+        raise ValueError("H must hold batch x C x C floats")
+    shape = (R, C // 2) if w.dim() == 2 else (B, R, C // 2)
+    if out is None:
+        out = torch.empty(shape, dtype=torch.uint8, device=w.device)
+    _need(out, torch.uint8, "packed")
+    _call("nvfp4_gptq", _p(w), B, R, C, _p(s_g), _p(scale_codes), _p(H), float(damp), _p(out),
           _stream(stream))
     return out
 

@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in range(9):
+    for code in range(10):
         s = L.nvfp4_status_string(code).decode()
         assert s.startswith("NVFP4_")
     assert L.nvfp4_status_string(0).decode() == "NVFP4_OK"
@@ -104,6 +104,18 @@ def test_validation_rejects_before_launch(L):
     assert L.nvfp4_static_scale_from_histogram(P, ctypes.c_double(1.5), P, None) == INVALID
     assert L.nvfp4_fake_quant_static(P, 4, 20, P, P, None, None, None) == SHAPE
     assert L.nvfp4_quant_error(P, 4, 16, P, None, None) == INVALID
+    # full Gram and GPTQ
+    assert L.nvfp4_hessian_full_accumulate(P, 10, 24, P, None) == SHAPE
+    assert L.nvfp4_hessian_full_accumulate(P, 10, 32, BAD, None) == MISALIGNED
+    assert L.nvfp4_hessian_full_accumulate(P, 10, 32, None, None) == INVALID
+    d = ctypes.c_double
+    assert L.nvfp4_gptq(P, 1, 4, 24, P, P, P, d(0.01), P, None) == SHAPE
+    assert L.nvfp4_gptq(P, 1, 4, 32, P, P, None, d(0.01), P, None) == INVALID
+    assert L.nvfp4_gptq(P, 1, 4, 32, P, P, P, d(-1.0), P, None) == INVALID
+    assert L.nvfp4_gptq(P, 1, 4, 32, P, P, P, d(float("nan")), P, None) == INVALID
+    assert L.nvfp4_gptq(BAD, 1, 4, 32, P, P, P, d(0.01), P, None) == MISALIGNED
+    assert L.nvfp4_gptq(P, 1, 4, 32, P, P, BAD, d(0.01), P, None) == MISALIGNED
+    assert L.nvfp4_gptq(P, 70000, 4, 32, P, P, P, d(0.01), P, None) == TOOLARGE
     # the statistics call needs somewhere to write
     assert L.nvfp4_search_evaluations(None, 0, None) == INVALID
 

@@ -20,17 +20,19 @@
 //  - gptq_lambda_kernel / gptq_prepare_kernel: lambda per Hessian, then
 //    Hd = J (H + lambda I) J in fp64 (J reverses the index order), whose
 //    lower Cholesky factor L gives T = J L J;
-//  - chol_diag_kernel, chol_panel_kernel and the fp64 GEMM: blocked
-//    right-looking Cholesky of Hd in place, 32-column panels (the diagonal
-//    block by one warp, the rows below it by triangular solves, the trailing
-//    matrix by a rank-32 update);
-//  - gptq_block_kernel: 32 columns at a time, one thread per row, the
-//    in-block part of the sum above from registers and the block of T from
-//    shared memory; rounding by the exact fp64 midpoint test; the errors
-//    w_j - q_j replace the consumed sums;
-//  - the fp64 GEMM again: the block's errors times the next rows of T, added
-//    to the running sums of every later column (lazy batch updates).
+//  - chol_block_kernel and the fp64 GEMM: blocked right-looking Cholesky of
+//    Hd in place, 128-column panels (the diagonal block factored and
+//    inverted by one CTA in shared memory, the rows below it solved by a
+//    GEMM with that inverse, the trailing matrix by a rank-128 update);
+//  - gptq_block_kernel: 128 columns at a time, one thread per row, the
+//    in-block part of the sum above from the block of T and the row's
+//    errors, both in shared memory; rounding by the exact fp64 midpoint
+//    test; the errors w_j - q_j replace the consumed sums;
+//  - the fp64 GEMM (fp64 tensor-core MMA) again: each block's errors times
+//    the next rows of T, added to the running sums of every later column
+//    (lazy batch updates, rank 128).
 #include <cmath>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -44,7 +46,6 @@ __device__ int g_gptq_status = 0;
 
 namespace {
 
-constexpr int kPanel = 32;  // columns per Cholesky panel and per GPTQ block
 
 // ----------------------------------------------------------------- fp64 GEMM
 // C[m][n] += alpha sum_k A[m][k] B[k][n] for m < M, n < N, with arbitrary
@@ -59,164 +60,324 @@ struct GemmF64 {
   int64_t sBk, sBn, bsB;
   double *C;
   int64_t sCm, sCn, bsC;
-  int lower;
+  int lower;      // skip tiles wholly above the diagonal
+  int overwrite;  // C = alpha A B (C is not read)
 };
 
-constexpr int kGM = 64, kGN = 64, kGK = 16, kGThreads = 256;
+// 128 x 128 output tile per CTA on the fp64 tensor-core instruction
+// (mma.sync m8n8k4 f64; tcgen05 has no f64 kind): eight warps of 64 x 32,
+// each an 8 x 4 grid of 8 x 8 accumulator tiles.  k-slabs of 16 are staged
+// in shared memory by a three-stage cp.async pipeline (8-byte copies, so any
+// stride works; the unit-stride dimension is copied fastest), both operands
+// stored [row][k] with a row stride of 20 doubles, which keeps the fragment
+// reads (8 rows x 4 consecutive k) free of bank conflicts.
+constexpr int kGM = 128, kGN = 128, kGK = 16, kGThreads = 256, kGStages = 3;
+constexpr int kGRow = kGK + 4;  // shared-memory row stride (doubles)
+constexpr int kGSmem = kGStages * (kGM + kGN) * kGRow * (int)sizeof(double);  // 120 KiB
 
-__global__ void __launch_bounds__(kGThreads) gemm_f64_kernel(const GemmF64 g) {
+__device__ __forceinline__ void cp_async8(double *smem, const double *gmem, bool pred) {
+  const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+  const int n = pred ? 8 : 0;  // 0: fill with zeros, read nothing
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(sa), "l"(gmem), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_1() {
+  asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+
+// D (8x8) += A (8x4, row) B (4x8, col).  Lane l holds A[l/4][l%4],
+// B[l%4][l/4] and D[l/4][2(l%4)], D[l/4][2(l%4)+1].
+__device__ __forceinline__ void dmma_8x8x4(double d[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d[0]), "+d"(d[1])
+               : "d"(a), "d"(b));
+}
+
+__global__ void __launch_bounds__(kGThreads, 1) gemm_f64_kernel(const GemmF64 g) {
   const int64_t m0 = (int64_t)blockIdx.y * kGM, n0 = (int64_t)blockIdx.x * kGN;
   if (g.lower && n0 > m0 + kGM - 1) return;
   const int64_t z = blockIdx.z;
   const double *A = g.A + z * g.bsA;
   const double *B = g.B + z * g.bsB;
   double *Cz = g.C + z * g.bsC;
-  __shared__ __align__(16) double As[kGK][kGM];
-  __shared__ __align__(16) double Bs[kGK][kGN];
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  // unit-stride dimension first in the tile loads (coalesced)
+  extern __shared__ __align__(16) double gsm[];
+  double *As = gsm;                            // [stage][m][k]
+  double *Bs = gsm + kGStages * kGM * kGRow;   // [stage][n][k]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wm = (warp >> 2) * 64, wn = (warp & 3) * 32;  // warp tile origin
+  const int gr = lane >> 2, gc = lane & 3;
+  // This thread's eight copies per operand and slab lie on one line: element
+  // e sits at (row0 + e drow, k0 + kk0 + e dk) with one of drow, dk zero
+  // (16 rows apart when k is the unit-stride dimension, else 2 k apart), so
+  // their addresses and bounds come from a base, two steps and a row mask.
   const bool a_k_fast = g.sAk == 1 || g.sAk == -1;
-  const bool b_n_fast = g.sBn == 1 || g.sBn == -1;
-  double acc[4][4];
+  const bool b_k_fast = g.sBk == 1 || g.sBk == -1;
+  const int a_r0 = a_k_fast ? tid >> 4 : tid & (kGM - 1), a_k0 = a_k_fast ? tid & 15 : tid >> 7;
+  const int a_dr = a_k_fast ? 16 : 0, a_dk = a_k_fast ? 0 : 2;
+  const int b_r0 = b_k_fast ? tid >> 4 : tid & (kGN - 1), b_k0 = b_k_fast ? tid & 15 : tid >> 7;
+  const int b_dr = b_k_fast ? 16 : 0, b_dk = b_k_fast ? 0 : 2;
+  const double *a_base = A + (m0 + a_r0) * g.sAm + a_k0 * g.sAk;
+  const double *b_base = B + (n0 + b_r0) * g.sBn + b_k0 * g.sBk;
+  const int64_t a_step = a_dr * g.sAm + a_dk * g.sAk, b_step = b_dr * g.sBn + b_dk * g.sBk;
+  const int64_t a_slab = kGK * g.sAk, b_slab = kGK * g.sBk;
+  const int a_soff = a_r0 * kGRow + a_k0, a_sstep = a_dr * kGRow + a_dk;
+  const int b_soff = b_r0 * kGRow + b_k0, b_sstep = b_dr * kGRow + b_dk;
+  uint32_t a_rows = 0, b_rows = 0;  // bit e: row of copy e in range
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-  for (int64_t k0 = 0; k0 < g.K; k0 += kGK) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int idx = tid + kGThreads * e;  // 0..1023
-      const int am = a_k_fast ? idx >> 4 : idx & 63, ak = a_k_fast ? idx & 15 : idx >> 6;
-      const int64_t gm = m0 + am, gk = k0 + ak;
-      As[ak][am] = (gm < g.M && gk < g.K) ? A[gm * g.sAm + gk * g.sAk] : 0.0;
-      const int bn = b_n_fast ? idx & 63 : idx >> 4, bk = b_n_fast ? idx >> 6 : idx & 15;
-      const int64_t gn = n0 + bn, gk2 = k0 + bk;
-      Bs[bk][bn] = (gn < g.N && gk2 < g.K) ? B[gk2 * g.sBk + gn * g.sBn] : 0.0;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < kGK; ++kk) {
-      const double2 a01 = *reinterpret_cast<const double2 *>(&As[kk][ty * 4]);
-      const double2 a23 = *reinterpret_cast<const double2 *>(&As[kk][ty * 4 + 2]);
-      const double2 b01 = *reinterpret_cast<const double2 *>(&Bs[kk][tx * 4]);
-      const double2 b23 = *reinterpret_cast<const double2 *>(&Bs[kk][tx * 4 + 2]);
-      const double a[4] = {a01.x, a01.y, a23.x, a23.y};
-      const double b[4] = {b01.x, b01.y, b23.x, b23.y};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
+  for (int e = 0; e < 8; ++e) {
+    a_rows |= (uint32_t)(m0 + a_r0 + e * a_dr < g.M) << e;
+    b_rows |= (uint32_t)(n0 + b_r0 + e * b_dr < g.N) << e;
   }
+  const int64_t nslab = (g.K + kGK - 1) / kGK;
+
+  auto issue = [&](int64_t t) {
+    if (t < nslab) {
+      const int st = (int)(t % kGStages);
+      const int64_t k0 = t * kGK;
+      double *as = As + st * kGM * kGRow + a_soff, *bs = Bs + st * kGN * kGRow + b_soff;
+      const double *pa = a_base + t * a_slab, *pb = b_base + t * b_slab;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t m = m0 + ty * 4 + i;
-    if (m >= g.M) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t n = n0 + tx * 4 + j;
-      if (n < g.N) {
-        double *c = Cz + m * g.sCm + n * g.sCn;
-        *c = fma(g.alpha, acc[i][j], *c);
+      for (int e = 0; e < 8; ++e) {
+        const bool oka = ((a_rows >> e) & 1u) && k0 + a_k0 + e * a_dk < g.K;
+        cp_async8(as + e * a_sstep, oka ? pa + e * a_step : A, oka);
+        const bool okb = ((b_rows >> e) & 1u) && k0 + b_k0 + e * b_dk < g.K;
+        cp_async8(bs + e * b_sstep, okb ? pb + e * b_step : B, okb);
       }
     }
+    cp_async_commit();  // possibly empty: keeps the group count uniform
+  };
+
+  double acc[8][4][2];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+  issue(0);
+  issue(1);
+  for (int64_t t = 0; t < nslab; ++t) {
+    cp_async_wait_1();  // slab t has landed (only slab t + 1 may be in flight)
+    __syncthreads();
+    issue(t + 2);  // into the stage read at step t - 1, finished by every thread
+    const int st = (int)(t % kGStages);
+    const double *as = As + st * kGM * kGRow + (wm + gr) * kGRow + gc;
+    const double *bs = Bs + st * kGN * kGRow + (wn + gr) * kGRow + gc;
+#pragma unroll
+    for (int k4 = 0; k4 < kGK; k4 += 4) {
+      double a[8], b[4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = as[i * 8 * kGRow + k4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = bs[j * 8 * kGRow + k4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[i][j], a[i], b[j]);
+    }
+  }
+  // C += alpha acc, one accumulator row (8 values) at a time: the loads of a
+  // row are issued before its stores (the compiler cannot tell that the
+  // addresses differ, so a load never passes an earlier store)
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t m = m0 + wm + i * 8 + gr;
+    double cv[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t n = n0 + wn + j * 8 + gc * 2 + h;
+        cv[j][h] = (m < g.M && n < g.N && !g.overwrite) ? Cz[m * g.sCm + n * g.sCn] : 0.0;
+      }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t n = n0 + wn + j * 8 + gc * 2 + h;
+        if (m < g.M && n < g.N) Cz[m * g.sCm + n * g.sCn] = fma(g.alpha, acc[i][j][h], cv[j][h]);
+      }
   }
 }
 
+std::mutex g_gemm_attr_mu;
+bool g_gemm_attr[64] = {};
+
 cudaError_t gemm_f64(const GemmF64 &g, int64_t batch, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lk(g_gemm_attr_mu);
+    if (!g_gemm_attr[dev]) {
+      e = cudaFuncSetAttribute(gemm_f64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kGSmem);
+      if (e != cudaSuccess) return e;
+      g_gemm_attr[dev] = true;
+    }
+  }
   const dim3 grid((unsigned)((g.N + kGN - 1) / kGN), (unsigned)((g.M + kGM - 1) / kGM),
                   (unsigned)batch);
-  gemm_f64_kernel<<<grid, kGThreads, 0, st>>>(g);
+  gemm_f64_kernel<<<grid, kGThreads, kGSmem, st>>>(g);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ Cholesky
-// The nw x nw diagonal block at (p0, p0) of every batch element's matrix,
-// factored in place by one warp (lane i holds row i; column k is finished at
-// step k and its rank-1 update applied to the later columns).  A pivot that
-// is not positive (or not finite) sets the status and makes the factor NaN.
-__global__ void __launch_bounds__(32) chol_diag_kernel(double *A, int64_t C, int64_t p0, int nw) {
-  const int lane = threadIdx.x;
-  double *Ab = A + (int64_t)blockIdx.x * C * C + p0 * C + p0;
-  double a[kPanel];
+// Blocked right-looking Cholesky of every batch element's matrix, in place
+// (lower triangle), 128-column panels:
+//  - chol_block_kernel: one CTA per batch element factors the panel's
+//    diagonal block in shared memory (column k's pivot, then the rank-1
+//    update of the later columns, the scaling of column k deferred to the
+//    end), writes the factor L_pp back and its inverse L_pp^-1 (formed in
+//    place, last column first) to a scratch block;
+//  - the rows below the block: X = A_panel L_pp^-T, one fp64 GEMM, in place;
+//  - the trailing matrix: -= X X^T, one fp64 GEMM on the lower triangle.
+// A pivot that is not positive (or not finite) sets the status and makes
+// the factor NaN.
+constexpr int kBig = 128;  // columns per Cholesky panel and per GPTQ block
+constexpr int kCholThreads = 256;
+constexpr int kSRow = kBig + 1;  // shared-memory row stride (doubles)
+constexpr int kCholSmem = (kBig * kSRow + 2 * kBig) * (int)sizeof(double);
+
+__global__ void __launch_bounds__(kCholThreads)
+    chol_block_kernel(double *A, int64_t C, int64_t P0, int nw, double *Linv) {
+  extern __shared__ double csm[];
+  double *S = csm;               // [kBig][kSRow]
+  double *piv = S + kBig * kSRow;  // 1 / L_kk
+  double *tmp = piv + kBig;        // one column of L
+  const int tid = threadIdx.x;
+  double *Ab = A + (int64_t)blockIdx.x * C * C + P0 * C + P0;
+  double *Lb = Linv + (int64_t)blockIdx.x * kBig * kBig;
+  // stage the lower triangle (asynchronous copies, all in flight at once)
+  for (int idx = tid; idx < nw * nw; idx += kCholThreads) {
+    const int r = idx / nw, c = idx - r * nw;
+    if (c <= r) cp_async8(S + r * kSRow + c, Ab + (int64_t)r * C + c, true);
+  }
+  cp_async_commit();
+  cp_async_wait_all();
+  __syncthreads();
+  for (int k = 0; k < nw; ++k) {
+    if (tid == 0) {
+      const double p = S[k * kSRow + k];
+      const bool ok = p > 0.0 && p < INFINITY;
+      if (!ok) atomicExch(&g_gptq_status, (int)NVFP4_ERR_NOT_POSITIVE_DEFINITE);
+      piv[k] = ok ? rsqrt(p) : __longlong_as_double(0x7FF8000000000000LL);
+    }
+    __syncthreads();
+    // S[r][c] -= L_rk L_ck = S[r][k] S[c][k] / p for k < c <= r; this thread
+    // takes columns k+1+(tid%16)+16j (their column-k entries read once) and
+    // rows k+1+(tid/16)+16i, eight independent updates per row
+    const double iv2 = piv[k] * piv[k];
+    const int c0 = k + 1 + (tid & 15);
+    double sc[8];
 #pragma unroll
-  for (int j = 0; j < kPanel; ++j)
-    a[j] = (lane < nw && j <= lane) ? Ab[(int64_t)lane * C + j] : 0.0;
+    for (int j = 0; j < 8; ++j) sc[j] = c0 + 16 * j < nw ? S[(c0 + 16 * j) * kSRow + k] : 0.0;
+    for (int r = k + 1 + (tid >> 4); r < nw; r += 16) {
+      const double lr = S[r * kSRow + k] * iv2;
+      double *Sr = S + r * kSRow;
 #pragma unroll
-  for (int k = 0; k < kPanel; ++k) {
-    if (k < nw) {
-      const double piv = __shfl_sync(0xFFFFFFFFu, a[k], k);
-      const bool ok = piv > 0.0 && piv < INFINITY;
-      if (!ok && lane == 0) atomicExch(&g_gptq_status, (int)NVFP4_ERR_NOT_POSITIVE_DEFINITE);
-      const double lkk = ok ? sqrt(piv) : __longlong_as_double(0x7FF8000000000000LL);
-      const double l = lane == k ? lkk : (lane > k ? a[k] / lkk : 0.0);
-      a[k] = l;
-#pragma unroll
-      for (int j = k + 1; j < kPanel; ++j) {
-        const double ljk = __shfl_sync(0xFFFFFFFFu, l, j);
-        if (lane >= j) a[j] = fma(-l, ljk, a[j]);
+      for (int j = 0; j < 8; ++j) {
+        const int c = c0 + 16 * j;
+        if (c <= r) Sr[c] = fma(-lr, sc[j], Sr[c]);
       }
     }
+    __syncthreads();
   }
-  if (lane < nw)
-#pragma unroll
-    for (int j = 0; j < kPanel; ++j)
-      if (j <= lane) Ab[(int64_t)lane * C + j] = a[j];
-}
-
-// Rows p0 + nw .. C-1 of the panel: x L_pp^T = a by forward substitution,
-// one thread per row, the factored diagonal block in shared memory.
-constexpr int kRowThreads = 128;
-
-__global__ void __launch_bounds__(kRowThreads)
-    chol_panel_kernel(double *A, int64_t C, int64_t p0, int nw) {
-  __shared__ double L[kPanel][kPanel + 1];
-  double *Ab = A + (int64_t)blockIdx.y * C * C;
-  for (int idx = threadIdx.x; idx < kPanel * kPanel; idx += kRowThreads) {
-    const int r = idx / kPanel, c = idx % kPanel;
-    L[r][c] = (r < nw && c <= r) ? Ab[(p0 + r) * C + p0 + c] : 0.0;
+  for (int idx = tid; idx < nw * nw; idx += kCholThreads) {
+    const int r = idx / nw, c = idx - r * nw;
+    if (c <= r) {
+      const double l = S[r * kSRow + c] * piv[c];
+      S[r * kSRow + c] = l;
+      Ab[(int64_t)r * C + c] = l;
+    }
   }
   __syncthreads();
-  const int64_t i = p0 + nw + (int64_t)blockIdx.x * kRowThreads + threadIdx.x;
-  if (i >= C) return;
-  double *row = Ab + i * C + p0;
-  double x[kPanel];
+  // L^-1 in place, last column first: column j below the diagonal is
+  // -(1 / L_jj) (L^-1)[j+1.., j+1..] L[j+1.., j]
+  for (int j = nw - 1; j >= 0; --j) {
+    for (int m = j + 1 + tid; m < nw; m += kCholThreads) tmp[m] = S[m * kSRow + j];
+    if (tid == 0) piv[j] = 1.0 / S[j * kSRow + j];
+    __syncthreads();
+    const double dj = piv[j];
+    for (int i = j + 1 + tid; i < nw; i += kCholThreads) {
+      const double *Si = S + i * kSRow;
+      double t[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+      int m = j + 1;
+      for (; m + 7 <= i; m += 8) {
 #pragma unroll
-  for (int k = 0; k < kPanel; ++k) {
-    if (k < nw) {
-      double v = row[k];
-#pragma unroll
-      for (int m = 0; m < k; ++m) v = fma(-x[m], L[k][m], v);
-      x[k] = v / L[k][k];
-      row[k] = x[k];
-    } else {
-      x[k] = 0.0;
+        for (int u = 0; u < 8; ++u) t[u] = fma(Si[m + u], tmp[m + u], t[u]);
+      }
+      for (; m <= i; ++m) t[0] = fma(Si[m], tmp[m], t[0]);
+      S[i * kSRow + j] = -dj * (((t[0] + t[1]) + (t[2] + t[3])) + ((t[4] + t[5]) + (t[6] + t[7])));
     }
+    if (tid == 0) S[j * kSRow + j] = dj;
+    __syncthreads();
+  }
+  for (int idx = tid; idx < kBig * kBig; idx += kCholThreads) {
+    const int r = idx / kBig, c = idx - r * kBig;
+    Lb[idx] = (r < nw && c <= r) ? S[r * kSRow + c] : 0.0;
   }
 }
 
-cudaError_t cholesky_in_place(double *A, int64_t C, int64_t batch, cudaStream_t st) {
-  for (int64_t p0 = 0; p0 < C; p0 += kPanel) {
-    const int nw = (int)(C - p0 < kPanel ? C - p0 : kPanel);
-    chol_diag_kernel<<<(unsigned)batch, 32, 0, st>>>(A, C, p0, nw);
-    const int64_t rest = C - p0 - nw;
-    if (rest > 0) {
-      const dim3 grid((unsigned)((rest + kRowThreads - 1) / kRowThreads), (unsigned)batch);
-      chol_panel_kernel<<<grid, kRowThreads, 0, st>>>(A, C, p0, nw);
-      // trailing block -= panel panel^T (lower triangle)
-      GemmF64 g;
-      g.M = rest; g.N = rest; g.K = nw; g.alpha = -1.0;
-      g.A = A + (p0 + nw) * C + p0; g.sAm = C; g.sAk = 1; g.bsA = C * C;
-      g.B = g.A; g.sBk = 1; g.sBn = C; g.bsB = C * C;
-      g.C = A + (p0 + nw) * C + p0 + nw; g.sCm = C; g.sCn = 1; g.bsC = C * C;
-      g.lower = 1;
-      cudaError_t e = gemm_f64(g, batch, st);
+std::mutex g_chol_attr_mu;
+bool g_chol_attr[64] = {};
+
+template <class K>
+cudaError_t ensure_smem_attr(K kernel, int bytes, std::mutex &mu, bool *flags) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!flags[dev]) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    flags[dev] = true;
+  }
+  return cudaSuccess;
+}
+
+// Linv: scratch [batch][128][128].
+cudaError_t cholesky_in_place(double *A, int64_t C, int64_t batch, double *Linv,
+                              cudaStream_t st) {
+  cudaError_t e = ensure_smem_attr(chol_block_kernel, kCholSmem, g_chol_attr_mu, g_chol_attr);
+  if (e != cudaSuccess) return e;
+  const int64_t CC = C * C;
+  for (int64_t P0 = 0; P0 < C; P0 += kBig) {
+    const int nw = (int)(C - P0 < kBig ? C - P0 : kBig);
+    chol_block_kernel<<<(unsigned)batch, kCholThreads, kCholSmem, st>>>(A, C, P0, nw, Linv);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t P1 = P0 + nw, rest = C - P1;
+    if (rest <= 0) break;
+    {
+      // rows below the block: X = A_panel L_pp^-T (in place: one CTA column)
+      GemmF64 g{};
+      g.M = rest; g.N = nw; g.K = nw; g.alpha = 1.0;
+      g.A = A + P1 * C + P0; g.sAm = C; g.sAk = 1; g.bsA = CC;
+      g.B = Linv; g.sBk = 1; g.sBn = kBig; g.bsB = (int64_t)kBig * kBig;
+      g.C = A + P1 * C + P0; g.sCm = C; g.sCn = 1; g.bsC = CC;
+      g.overwrite = 1;
+      e = gemm_f64(g, batch, st);
       if (e != cudaSuccess) return e;
     }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    {
+      // trailing block -= X X^T (lower triangle)
+      GemmF64 g{};
+      g.M = rest; g.N = rest; g.K = nw; g.alpha = -1.0;
+      g.A = A + P1 * C + P0; g.sAm = C; g.sAk = 1; g.bsA = CC;
+      g.B = g.A; g.sBk = 1; g.sBn = C; g.bsB = CC;
+      g.C = A + P1 * C + P1; g.sCm = C; g.sCn = 1; g.bsC = CC;
+      g.lower = 1;
+      e = gemm_f64(g, batch, st);
+      if (e != cudaSuccess) return e;
+    }
   }
   return cudaSuccess;
 }
@@ -264,55 +425,84 @@ __device__ __forceinline__ double e2m1_magnitude(int k) {
   return k < 2 ? 0.5 * k : (1.0 + 0.5 * (double)(k & 1)) * (double)(1 << ((k >> 1) - 1));
 }
 
-// Columns c0 .. c0+nw-1 of every row: the value at rounding, its code, and
-// the error w - q written over the consumed running sum.  L is the lower
-// Cholesky factor of the reversed Hessian: T[i][j] = L[C-1-i][C-1-j].
-__global__ void __launch_bounds__(kRowThreads)
+// Columns c0 .. c0+nw-1 (nw <= 128) of every row: the value at rounding,
+// its code, and the error w - q written over the consumed running sum.  L is
+// the lower Cholesky factor of the reversed Hessian: T[i][j] = L[C-1-i][C-1-j].
+// One thread per row; the block of T (upper triangle), the row's running
+// sums / errors and its weights sit in shared memory ([column][row], so a
+// warp reads consecutive words).
+constexpr int kRowsPerCta = 64;
+constexpr int kBlockSmem =
+    (kBig * kBig + kBig * kRowsPerCta + kBig) * (int)sizeof(double) +
+    kBig * kRowsPerCta * (int)sizeof(uint16_t);  // 214,016 B
+
+__global__ void __launch_bounds__(kRowsPerCta)
     gptq_block_kernel(const uint16_t *__restrict__ w, int64_t R, int64_t C,
                       const float *__restrict__ s_g, const uint8_t *__restrict__ codes,
                       const double *__restrict__ L, double *__restrict__ SD,
                       uint8_t *__restrict__ packed, int64_t c0, int nw) {
+  extern __shared__ double bsm[];
+  double *T = bsm;                          // [j][k], j <= k
+  double *Dsm = T + kBig * kBig;            // [k][row]
+  double *Tinv = Dsm + kBig * kRowsPerCta;  // 1 / T[k][k]
+  uint16_t *Wsm = reinterpret_cast<uint16_t *>(Tinv + kBig);  // [k][row]
   const int64_t b = blockIdx.y;
-  __shared__ double T[kPanel][kPanel + 1];  // T[c0 + j][c0 + k], j <= k
+  const int tid = threadIdx.x;
   const double *Lb = L + b * C * C;
-  for (int idx = threadIdx.x; idx < kPanel * kPanel; idx += kRowThreads) {
-    const int j = idx / kPanel, k = idx % kPanel;
-    T[j][k] = (j <= k && k < nw) ? Lb[(C - 1 - c0 - j) * C + (C - 1 - c0 - k)] : 0.0;
+  const int64_t r = (int64_t)blockIdx.x * kRowsPerCta + tid;
+  const bool live = r < R;
+  const int64_t row = b * R + (live ? r : 0);
+  const uint16_t *wr = w + row * C + c0;
+  double *sd = SD + row * C + c0;
+  // stage T (upper triangle, zeros elsewhere) and this thread's running sums
+  // with asynchronous copies, all in flight at once
+  for (int idx = tid; idx < kBig * kBig; idx += kRowsPerCta) {
+    const int j = idx / kBig, k = idx - j * kBig;
+    const bool in = j <= k && k < nw;
+    cp_async8(T + idx, in ? Lb + (C - 1 - c0 - j) * C + (C - 1 - c0 - k) : Lb, in);
   }
+  for (int k = 0; k < nw; ++k) cp_async8(Dsm + k * kRowsPerCta + tid, live ? sd + k : sd, live);
+  cp_async_commit();
+#pragma unroll 8
+  for (int k = 0; k < nw; ++k) Wsm[k * kRowsPerCta + tid] = live ? wr[k] : (uint16_t)0;
+  cp_async_wait_all();
   __syncthreads();
-  const int64_t r = (int64_t)blockIdx.x * kRowThreads + threadIdx.x;
-  if (r >= R) return;
+  for (int k = tid; k < kBig; k += kRowsPerCta) Tinv[k] = k < nw ? 1.0 / T[k * kBig + k] : 0.0;
+  __syncthreads();
+  if (!live) return;
   const float sg = s_g[b];
-  const int64_t row = b * R + r;
-  const uint16_t *wr = w + row * C;
-  double *sd = SD + row * C;
-  const uint8_t *cr = codes + row * (C / kBlock);
-  uint8_t *pr = packed + row * (C / 2);
-  double d[kPanel];
+  const uint8_t *cr = codes + row * (C / kBlock) + c0 / kBlock;
+  uint8_t *pr = packed + row * (C / 2) + c0 / 2;
+  double s = 0.0;
   uint32_t lo = 0;
+  for (int k = 0; k < nw; ++k) {
+    if ((k & (kBlock - 1)) == 0) s = (double)effective_scale(sg, cr[k / kBlock]);
+    // running sum of the earlier blocks plus this block's columns j < k
+    double a[8] = {Dsm[k * kRowsPerCta + tid], 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    int j = 0;
+    for (; j + 7 < k; j += 8) {
 #pragma unroll
-  for (int k = 0; k < kPanel; ++k) {
-    if (k < nw) {
-      const int64_t col = c0 + k;
-      double acc = sd[col];
-#pragma unroll
-      for (int j = 0; j < k; ++j) acc = fma(d[j], T[j][k], acc);
-      const double wk = (double)__uint_as_float((uint32_t)wr[col] << 16);
-      const double x = wk + acc / T[k][k];
-      const double s = (double)effective_scale(sg, cr[col / kBlock]);
-      const int kq = e2m1_index64(fabs(x), s);
-      const double q = e2m1_magnitude(kq) * s;
-      const bool neg = signbit(x);
-      d[k] = wk - (neg ? -q : q);
-      sd[col] = d[k];
-      const uint32_t code = (uint32_t)kq | (neg ? 8u : 0u);
-      if (k & 1) pr[col >> 1] = (uint8_t)(lo | (code << 4));
-      else lo = code;
-    } else {
-      d[k] = 0.0;
+      for (int u = 0; u < 8; ++u)
+        a[u] = fma(Dsm[(j + u) * kRowsPerCta + tid], T[(j + u) * kBig + k], a[u]);
     }
+    for (; j < k; ++j) a[0] = fma(Dsm[j * kRowsPerCta + tid], T[j * kBig + k], a[0]);
+    const double acc = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+    const double wk = (double)__uint_as_float((uint32_t)Wsm[k * kRowsPerCta + tid] << 16);
+    const double x = fma(acc, Tinv[k], wk);
+    const int kq = e2m1_index64(fabs(x), s);
+    const double q = e2m1_magnitude(kq) * s;
+    const bool neg = signbit(x);
+    const double d = wk - (neg ? -q : q);
+    Dsm[k * kRowsPerCta + tid] = d;
+    sd[k] = d;
+    const uint32_t code = (uint32_t)kq | (neg ? 8u : 0u);
+    if (k & 1) pr[k >> 1] = (uint8_t)(lo | (code << 4));
+    else lo = code;
   }
 }
+
+std::mutex g_block_attr_mu;
+bool g_block_attr[64] = {};
 
 }  // namespace
 
@@ -324,13 +514,15 @@ cudaError_t launch_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
   const size_t lam_bytes = ((size_t)batch * sizeof(double) + 255) / 256 * 256;
   const size_t hd_bytes = (size_t)batch * (size_t)C * (size_t)C * sizeof(double);
   const size_t sd_bytes = (size_t)batch * (size_t)R * (size_t)C * sizeof(double);
+  const size_t li_bytes = (size_t)batch * kBig * kBig * sizeof(double);
   unsigned char *scratch = nullptr;
-  cudaError_t e = scratch_alloc(reinterpret_cast<void **>(&scratch), lam_bytes + hd_bytes + sd_bytes,
-                                st);
+  cudaError_t e = scratch_alloc(reinterpret_cast<void **>(&scratch),
+                                lam_bytes + hd_bytes + sd_bytes + li_bytes, st);
   if (e != cudaSuccess) return e;
   double *lam = reinterpret_cast<double *>(scratch);
   double *Hd = reinterpret_cast<double *>(scratch + lam_bytes);
   double *SD = reinterpret_cast<double *>(scratch + lam_bytes + hd_bytes);
+  double *Linv = reinterpret_cast<double *>(scratch + lam_bytes + hd_bytes + sd_bytes);
   e = cudaMemsetAsync(SD, 0, sd_bytes, st);
   if (e == cudaSuccess) {
     gptq_lambda_kernel<<<(unsigned)batch, 32, 0, st>>>(H, C, damp, lam);
@@ -340,21 +532,26 @@ cudaError_t launch_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
     gptq_prepare_kernel<<<dim3((unsigned)gx, (unsigned)batch), 256, 0, st>>>(H, C, lam, Hd);
     e = cudaGetLastError();
   }
-  if (e == cudaSuccess) e = cholesky_in_place(Hd, C, batch, st);
-  for (int64_t c0 = 0; e == cudaSuccess && c0 < C; c0 += kPanel) {
-    const int nw = (int)(C - c0 < kPanel ? C - c0 : kPanel);
-    const dim3 grid((unsigned)((R + kRowThreads - 1) / kRowThreads), (unsigned)batch);
-    gptq_block_kernel<<<grid, kRowThreads, 0, st>>>(w, R, C, s_g, codes, Hd, SD, packed, c0, nw);
+  if (e == cudaSuccess) e = cholesky_in_place(Hd, C, batch, Linv, st);
+  // columns in blocks of 128: each block's rows one thread each, then the
+  // block's errors added to the running sums of every later column (rank-128)
+  if (e == cudaSuccess)
+    e = ensure_smem_attr(gptq_block_kernel, kBlockSmem, g_block_attr_mu, g_block_attr);
+  const int64_t RC = R * C, CC = C * C;
+  for (int64_t c0 = 0; e == cudaSuccess && c0 < C; c0 += kBig) {
+    const int nw = (int)(C - c0 < kBig ? C - c0 : kBig);
+    const dim3 grid((unsigned)((R + kRowsPerCta - 1) / kRowsPerCta), (unsigned)batch);
+    gptq_block_kernel<<<grid, kRowsPerCta, kBlockSmem, st>>>(w, R, C, s_g, codes, Hd, SD, packed,
+                                                              c0, nw);
     e = cudaGetLastError();
     const int64_t c1 = c0 + nw;
     if (e == cudaSuccess && c1 < C) {
-      // running sums of columns c1.. += errors of this block x rows c0.. of T
-      GemmF64 g;
+      // SD[:, c1:] += SD[:, c0:c1] T[c0:c1, c1:], T[i][j] = Hd[C-1-i][C-1-j]
+      GemmF64 g{};
       g.M = R; g.N = C - c1; g.K = nw; g.alpha = 1.0;
-      g.A = SD + c0; g.sAm = C; g.sAk = 1; g.bsA = R * C;
-      g.B = Hd + (C - 1 - c0) * C + (C - 1 - c1); g.sBk = -C; g.sBn = -1; g.bsB = C * C;
-      g.C = SD + c1; g.sCm = C; g.sCn = 1; g.bsC = R * C;
-      g.lower = 0;
+      g.A = SD + c0; g.sAm = C; g.sAk = 1; g.bsA = RC;
+      g.B = Hd + (C - 1 - c0) * C + (C - 1 - c1); g.sBk = -C; g.sBn = -1; g.bsB = CC;
+      g.C = SD + c1; g.sCm = C; g.sCn = 1; g.bsC = RC;
       e = gemm_f64(g, batch, st);
     }
   }

@@ -50,7 +50,9 @@ FALLBACK_HBM_GBS = 6650.0
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
 WORKLOAD_NAMES = ["dense", "tiny", "moe", "mlp_pair", "w4a4", "four_over_six", "w4a4_gemm",
-                  "act_calib"]
+                  "act_calib", "lh_gptq"]
+FP64_FMA_PER_SM = 64  # B200: 64 fp64 FMA per clock per SM (about 40 TFLOP/s at boost clock)
+GPTQ_DAMP = 0.01
 
 # Local-Hessian search work per block, counted on the definition E = delta
 # H_b delta^T: per candidate 256 FMA for H_b delta and 16 FMA for the dot
@@ -103,6 +105,7 @@ class Runner:
         from scale_calibration_nvfp4_b200 import nvfp4, workloads
         self.nv = nvfp4
         self.workload = workload
+        self.gptq = False
         wl = workloads
         if workload in ("tiny", "dense"):
             W, X = wl.layer_inputs(workload, device)
@@ -110,6 +113,20 @@ class Runner:
             self.desc = wl.BY_NAME[workload].description
             self.rules = ["max", "mse", "lh"]
             self.fq_input = X
+        elif workload == "lh_gptq":
+            # the dense projection under Local-Hessian scales and GPTQ rounding:
+            # the block-diagonal and the full Gram of its calibration tokens,
+            # the scale search, GPTQ (dampening 0.01), dequantise
+            W, X = wl.layer_inputs("dense", device)
+            L = Layer("dense", W, X)
+            L.Hf = torch.zeros(L.C, L.C, dtype=torch.float32, device=W.device)
+            self.layers = [L]
+            self.desc = ("Local-Hessian + GPTQ on the dense projection (W 4096x4096, X 2048x4096): "
+                         "global scale, block-diagonal and full Gram, scale search, GPTQ "
+                         "rounding (damp %.2f), dequantise" % GPTQ_DAMP)
+            self.rules = ["lh"]
+            self.gptq = True
+            self.fq_input = None
         elif workload == "four_over_six":
             # the dense projection's weights under the Four Over Six rule
             W, _ = wl.layer_inputs("dense", device)
@@ -203,6 +220,9 @@ class Runner:
             elif L.X is not None:
                 rows.append((pre + "gram", lambda L=L: nv.hessian_accumulate(L.X, L.H[0]),
                              2 * L.X.numel() + 2 * h, 2))
+            if self.gptq:
+                rows.append((pre + "gram_full", lambda L=L: nv.hessian_full_accumulate(L.X, L.Hf),
+                             2 * L.X.numel() + 8 * L.C * L.C, 1))
             if "max" in self.rules:
                 rows.append((pre + "search_max",
                              lambda L=L: nv.scale_search_max(L.W, L.s_g, out=L.c_max),
@@ -220,11 +240,19 @@ class Runner:
                              lambda L=L: nv.scale_search_local_hessian(L.W, L.s_g, L.H,
                                                                        out=L.c_lh),
                              2 * n_w + nb + h, 2))  # factor_kernel + search_kernel
-            # pack and dequantise with the codes of the workload's final rule
+            # pack (GPTQ rounding or plain) and dequantise with the codes of the
+            # workload's final rule
             fin = L.c_lh if "lh" in self.rules else L.c_46
-            rows.append((pre + "quantize_pack",
-                         lambda L=L, c=fin: nv.quantize_pack(L.W, L.s_g, c, out=L.packed),
-                         2 * n_w + nb + n_w // 2, 1))
+            if self.gptq:
+                npan = (L.C + 127) // 128
+                rows.append((pre + "gptq",
+                             lambda L=L, c=fin: nv.gptq(L.W[0], L.s_g, c[0], L.Hf, GPTQ_DAMP,
+                                                        out=L.packed[0]),
+                             2 * n_w + nb + 4 * L.C * L.C + n_w // 2, 5 * npan - 1))
+            else:
+                rows.append((pre + "quantize_pack",
+                             lambda L=L, c=fin: nv.quantize_pack(L.W, L.s_g, c, out=L.packed),
+                             2 * n_w + nb + n_w // 2, 1))
             rows.append((pre + "dequantize",
                          lambda L=L, c=fin: nv.dequantize(L.packed, c, L.s_g, out=L.deq),
                          n_w // 2 + nb + 2 * n_w, 1))
@@ -499,7 +527,8 @@ def run_gpu(args):
         out = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64" if run.gptq else "bf16",
             "data": "synthetic (seeded; no dataset or trained weights)",
             "config": {"workload": args.workload, "desc": run.desc, "blocks_per_step": blocks,
                        "rows": [r[0] for r in rows],
@@ -522,6 +551,22 @@ def run_gpu(args):
 
 
 def make_roofline(run, kernels, pk, pk_kind, workload, lh_evals):
+    if "gptq" in kernels:
+        # fp64 arithmetic of the definition: the column loop's update of the
+        # later columns (R C^2 / 2 FMA) and the Cholesky factor (C^3 / 6 FMA)
+        L = run.layers[0]
+        R, C = L.R, L.C
+        ms = kernels["gptq"]["ms"]
+        sm_mhz = float(pk.get("sm_max_mhz", 1965.0))
+        fp64_peak = SM_COUNT * FP64_FMA_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+        flop = R * C * C + C ** 3 / 3
+        achieved = flop / (ms / 1e3) / 1e12
+        return {"kernel": "gptq (Cholesky + column loop + lazy-batch fp64 MMA updates)",
+                "bound": "alu", "achieved": round(achieved, 2), "peak": round(fp64_peak, 2),
+                "unit": "TFLOP/s", "frac": round(achieved / fp64_peak, 4), "traffic": None,
+                "peak_kind": "derived: 148 SMs x 64 fp64 FMA x 2 flop x %.0f MHz (%s clocks)"
+                             % (sm_mhz, pk_kind),
+                "flop_basis": "R C^2 (column loop) + C^3/3 (Cholesky), R=%d C=%d" % (R, C)}
     lh_rows = [k for k in kernels if k.endswith("search_lh")]
     if lh_rows:
         lh_ms = sum(kernels[k]["ms"] for k in lh_rows)
@@ -716,6 +761,7 @@ def cpu_baseline(run, budget_s=15.0):
         t0 = time.perf_counter()
         sg = oracle.global_scale(wu_all)
         H = None if xu is None else oracle.gram(xu)
+        Hf = oracle.gram_full(xu) if run.gptq else None
         wu = np.ascontiguousarray(wu_all[:rows])
         if "max" in run.rules:
             oracle.scale_search_max(wu, sg)
@@ -725,7 +771,11 @@ def cpu_baseline(run, budget_s=15.0):
             oracle.scale_search_mse(wu, sg)
         if "lh" in run.rules:
             codes, _ = oracle.scale_search_lh(wu, sg, H)
-        packed = oracle.quantize_pack(wu, sg, codes)
+        if run.gptq:
+            U = oracle.gptq_factor(Hf, GPTQ_DAMP)
+            packed, _ = oracle.gptq_rows(wu, sg, codes, U, np.arange(rows))
+        else:
+            packed = oracle.quantize_pack(wu, sg, codes)
         oracle.dequantize(packed, codes, sg)
         if fq is not None:
             oracle.fake_quant(fq)
@@ -752,7 +802,8 @@ def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
         return
-    small = args.workload in ("tiny", "dense", "w4a4", "four_over_six", "w4a4_gemm", "act_calib")
+    small = args.workload in ("tiny", "dense", "w4a4", "four_over_six", "w4a4_gemm", "act_calib",
+                              "lh_gptq")
     dev = "cpu" if small or not torch.cuda.is_available() else "cuda"
     run = Runner(args.workload, dev)
     budget = args.cpu_seconds / max(1, args.steps)

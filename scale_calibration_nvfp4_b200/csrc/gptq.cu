@@ -24,10 +24,11 @@
 //    Hd in place, 128-column panels (the diagonal block factored and
 //    inverted by one CTA in shared memory, the rows below it solved by a
 //    GEMM with that inverse, the trailing matrix by a rank-128 update);
-//  - gptq_block_kernel: 128 columns at a time, one thread per row, the
-//    in-block part of the sum above from the block of T and the row's
-//    errors, both in shared memory; rounding by the exact fp64 midpoint
-//    test; the errors w_j - q_j replace the consumed sums;
+//  - gptq_block_kernel: 128 columns at a time, four lanes per row each
+//    holding 32 columns' running sums in registers; each column is rounded
+//    by its owner lane (exact fp64 midpoint test), its error shuffled to the
+//    quad and added times T to the later columns' sums; the errors w_j - q_j
+//    replace the consumed sums;
 //  - the fp64 GEMM (fp64 tensor-core MMA) again: each block's errors times
 //    the next rows of T, added to the running sums of every later column
 //    (lazy batch updates, rank 128).
@@ -232,97 +233,147 @@ cudaError_t gemm_f64(const GemmF64 &g, int64_t batch, cudaStream_t st) {
 // Blocked right-looking Cholesky of every batch element's matrix, in place
 // (lower triangle), 128-column panels:
 //  - chol_block_kernel: one CTA per batch element factors the panel's
-//    diagonal block in shared memory (column k's pivot, then the rank-1
-//    update of the later columns, the scaling of column k deferred to the
-//    end), writes the factor L_pp back and its inverse L_pp^-1 (formed in
-//    place, last column first) to a scratch block;
+//    diagonal block, writes the factor L_pp back and its inverse L_pp^-1 to
+//    a scratch block;
 //  - the rows below the block: X = A_panel L_pp^-T, one fp64 GEMM, in place;
 //  - the trailing matrix: -= X X^T, one fp64 GEMM on the lower triangle.
 // A pivot that is not positive (or not finite) sets the status and makes
 // the factor NaN.
+//
+// In chol_block_kernel each of the 256 threads keeps an 8 x 8 tile of the
+// block in registers: rows ty + 16 i, columns tx + 16 j (tx, ty = thread
+// index mod / div 16).  Factor step k: the owners of column k publish it to
+// a shared vector (double-buffered, one barrier per step), every thread
+// takes the pivot p = A_kk and applies A_rc -= A_rk A_ck / p to its entries
+// with k < c <= r (64 independent updates); column k is scaled by p^-1/2
+// at the end.  The inverse X = L^-1 is the same pattern on the identity:
+// step k finishes row k of X (scaled by 1 / L_kk) from the row's owners and
+// removes it from the later rows, X_rc -= L_rk X_kc.
 constexpr int kBig = 128;  // columns per Cholesky panel and per GPTQ block
 constexpr int kCholThreads = 256;
 constexpr int kSRow = kBig + 1;  // shared-memory row stride (doubles)
-constexpr int kCholSmem = (kBig * kSRow + 2 * kBig) * (int)sizeof(double);
+constexpr int kCholSmem = (kBig * kSRow + 4 * kBig) * (int)sizeof(double);  // 136,192 B
 
 __global__ void __launch_bounds__(kCholThreads)
     chol_block_kernel(double *A, int64_t C, int64_t P0, int nw, double *Linv) {
   extern __shared__ double csm[];
-  double *S = csm;               // [kBig][kSRow]
-  double *piv = S + kBig * kSRow;  // 1 / L_kk
-  double *tmp = piv + kBig;        // one column of L
-  const int tid = threadIdx.x;
+  double *Lsm = csm;                 // [kBig][kSRow], the factor
+  double *vec = Lsm + kBig * kSRow;  // [2][kBig] column (factor) / row (inverse) of step k
+  double *inv = vec + 2 * kBig;      // p_k^-1/2
+  double *dinv = inv + kBig;         // 1 / L_kk
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   double *Ab = A + (int64_t)blockIdx.x * C * C + P0 * C + P0;
   double *Lb = Linv + (int64_t)blockIdx.x * kBig * kBig;
-  // stage the lower triangle (asynchronous copies, all in flight at once)
-  for (int idx = tid; idx < nw * nw; idx += kCholThreads) {
-    const int r = idx / nw, c = idx - r * nw;
-    if (c <= r) cp_async8(S + r * kSRow + c, Ab + (int64_t)r * C + c, true);
-  }
-  cp_async_commit();
-  cp_async_wait_all();
-  __syncthreads();
-  for (int k = 0; k < nw; ++k) {
-    if (tid == 0) {
-      const double p = S[k * kSRow + k];
-      const bool ok = p > 0.0 && p < INFINITY;
-      if (!ok) atomicExch(&g_gptq_status, (int)NVFP4_ERR_NOT_POSITIVE_DEFINITE);
-      piv[k] = ok ? rsqrt(p) : __longlong_as_double(0x7FF8000000000000LL);
-    }
-    __syncthreads();
-    // S[r][c] -= L_rk L_ck = S[r][k] S[c][k] / p for k < c <= r; this thread
-    // takes columns k+1+(tid%16)+16j (their column-k entries read once) and
-    // rows k+1+(tid/16)+16i, eight independent updates per row
-    const double iv2 = piv[k] * piv[k];
-    const int c0 = k + 1 + (tid & 15);
-    double sc[8];
+  double a[8][8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) sc[j] = c0 + 16 * j < nw ? S[(c0 + 16 * j) * kSRow + k] : 0.0;
-    for (int r = k + 1 + (tid >> 4); r < nw; r += 16) {
-      const double lr = S[r * kSRow + k] * iv2;
-      double *Sr = S + r * kSRow;
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = ty + 16 * i, c = tx + 16 * j;
+      a[i][j] = (r < nw && c <= r) ? Ab[(int64_t)r * C + c] : 0.0;
+    }
+  // ---- factor
+#pragma unroll
+  for (int j0 = 0; j0 < 8; ++j0) {
+    for (int kk = 0; kk < 16; ++kk) {
+      const int k = 16 * j0 + kk;
+      if (k >= nw) break;
+      double *col = vec + (k & 1) * kBig;
+      if (tx == kk) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = ty + 16 * i;
+          if (r >= k) col[r] = a[i][j0];
+        }
+      }
+      __syncthreads();
+      const double p = col[k];
+      const bool ok = p > 0.0 && p < INFINITY;
+      const double iv = ok ? rsqrt(p) : __longlong_as_double(0x7FF8000000000000LL);
+      if (tid == 0) {
+        inv[k] = iv;
+        if (!ok) atomicExch(&g_gptq_status, (int)NVFP4_ERR_NOT_POSITIVE_DEFINITE);
+      }
+      const double iv2 = iv * iv;
+      double cr[8], cc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = ty + 16 * i, c = tx + 16 * i;
+        cr[i] = r > k && r < nw ? col[r] * iv2 : 0.0;
+        cc[i] = c > k && c < nw ? col[c] : 0.0;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int r = ty + 16 * i, c = tx + 16 * j;
+          if (c > k && c <= r) a[i][j] = fma(-cr[i], cc[j], a[i][j]);
+        }
+    }
+  }
+  __syncthreads();
+  // scale the columns, write the factor back and keep it in shared memory
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = ty + 16 * i, c = tx + 16 * j;
+      if (r < nw && c <= r) {
+        const double l = a[i][j] * inv[c];
+        Lsm[r * kSRow + c] = l;
+        Ab[(int64_t)r * C + c] = l;
+      }
+    }
+  __syncthreads();
+  for (int k = tid; k < nw; k += kCholThreads) dinv[k] = 1.0 / Lsm[k * kSRow + k];
+  // ---- inverse: identity in the registers, rows finished in order
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a[i][j] = (ty + 16 * i == tx + 16 * j) ? 1.0 : 0.0;
+  __syncthreads();
+#pragma unroll
+  for (int i0 = 0; i0 < 8; ++i0) {
+    for (int kk = 0; kk < 16; ++kk) {
+      const int k = 16 * i0 + kk;
+      if (k >= nw) break;
+      double *row = vec + (k & 1) * kBig;
+      if (ty == kk) {
+        const double d = dinv[k];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = tx + 16 * j;
+          if (c <= k) {
+            a[i0][j] *= d;
+            row[c] = a[i0][j];
+          }
+        }
+      }
+      __syncthreads();
+      double xr[8], lr[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int c = c0 + 16 * j;
-        if (c <= r) Sr[c] = fma(-lr, sc[j], Sr[c]);
+        const int c = tx + 16 * j;
+        xr[j] = c <= k ? row[c] : 0.0;
       }
-    }
-    __syncthreads();
-  }
-  for (int idx = tid; idx < nw * nw; idx += kCholThreads) {
-    const int r = idx / nw, c = idx - r * nw;
-    if (c <= r) {
-      const double l = S[r * kSRow + c] * piv[c];
-      S[r * kSRow + c] = l;
-      Ab[(int64_t)r * C + c] = l;
-    }
-  }
-  __syncthreads();
-  // L^-1 in place, last column first: column j below the diagonal is
-  // -(1 / L_jj) (L^-1)[j+1.., j+1..] L[j+1.., j]
-  for (int j = nw - 1; j >= 0; --j) {
-    for (int m = j + 1 + tid; m < nw; m += kCholThreads) tmp[m] = S[m * kSRow + j];
-    if (tid == 0) piv[j] = 1.0 / S[j * kSRow + j];
-    __syncthreads();
-    const double dj = piv[j];
-    for (int i = j + 1 + tid; i < nw; i += kCholThreads) {
-      const double *Si = S + i * kSRow;
-      double t[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-      int m = j + 1;
-      for (; m + 7 <= i; m += 8) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) t[u] = fma(Si[m + u], tmp[m + u], t[u]);
+      for (int i = 0; i < 8; ++i) {
+        const int r = ty + 16 * i;
+        lr[i] = r > k && r < nw ? Lsm[r * kSRow + k] : 0.0;
       }
-      for (; m <= i; ++m) t[0] = fma(Si[m], tmp[m], t[0]);
-      S[i * kSRow + j] = -dj * (((t[0] + t[1]) + (t[2] + t[3])) + ((t[4] + t[5]) + (t[6] + t[7])));
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a[i][j] = fma(-lr[i], xr[j], a[i][j]);
     }
-    if (tid == 0) S[j * kSRow + j] = dj;
-    __syncthreads();
   }
-  for (int idx = tid; idx < kBig * kBig; idx += kCholThreads) {
-    const int r = idx / kBig, c = idx - r * kBig;
-    Lb[idx] = (r < nw && c <= r) ? S[r * kSRow + c] : 0.0;
-  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = ty + 16 * i, c = tx + 16 * j;
+      Lb[r * kBig + c] = (r < nw && c <= r) ? a[i][j] : 0.0;
+    }
 }
 
 std::mutex g_chol_attr_mu;
@@ -428,77 +479,96 @@ __device__ __forceinline__ double e2m1_magnitude(int k) {
 // Columns c0 .. c0+nw-1 (nw <= 128) of every row: the value at rounding,
 // its code, and the error w - q written over the consumed running sum.  L is
 // the lower Cholesky factor of the reversed Hessian: T[i][j] = L[C-1-i][C-1-j].
-// One thread per row; the block of T (upper triangle), the row's running
-// sums / errors and its weights sit in shared memory ([column][row], so a
-// warp reads consecutive words).
-constexpr int kRowsPerCta = 64;
-constexpr int kBlockSmem =
-    (kBig * kBig + kBig * kRowsPerCta + kBig) * (int)sizeof(double) +
-    kBig * kRowsPerCta * (int)sizeof(uint16_t);  // 214,016 B
+// A quad of lanes takes one row, lane q the columns 32q .. 32q+31 of the
+// block with their running sums in registers.  Column k = 32 q0 + kk is
+// rounded by its owner lane, whose error goes to the quad by a shuffle; then
+// every lane adds error x T[k][m] to the running sums of its columns m > k
+// (independent updates: the dependent chain per column is one fma and the
+// rounding).  The block of T (upper triangle) sits in shared memory.
+constexpr int kRowsPerCta = 32;                  // 128 threads, four per row
+constexpr int kBlockThreads = 4 * kRowsPerCta;
+constexpr int kBlockSmem = (kBig * kBig + kBig) * (int)sizeof(double);  // 132,096 B
 
-__global__ void __launch_bounds__(kRowsPerCta)
+__global__ void __launch_bounds__(kBlockThreads)
     gptq_block_kernel(const uint16_t *__restrict__ w, int64_t R, int64_t C,
                       const float *__restrict__ s_g, const uint8_t *__restrict__ codes,
                       const double *__restrict__ L, double *__restrict__ SD,
                       uint8_t *__restrict__ packed, int64_t c0, int nw) {
   extern __shared__ double bsm[];
-  double *T = bsm;                          // [j][k], j <= k
-  double *Dsm = T + kBig * kBig;            // [k][row]
-  double *Tinv = Dsm + kBig * kRowsPerCta;  // 1 / T[k][k]
-  uint16_t *Wsm = reinterpret_cast<uint16_t *>(Tinv + kBig);  // [k][row]
+  double *T = bsm;              // [j][k], j <= k
+  double *Tinv = T + kBig * kBig;  // 1 / T[k][k]
   const int64_t b = blockIdx.y;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, q = lane & 3;
   const double *Lb = L + b * C * C;
-  const int64_t r = (int64_t)blockIdx.x * kRowsPerCta + tid;
-  const bool live = r < R;
-  const int64_t row = b * R + (live ? r : 0);
-  const uint16_t *wr = w + row * C + c0;
-  double *sd = SD + row * C + c0;
-  // stage T (upper triangle, zeros elsewhere) and this thread's running sums
-  // with asynchronous copies, all in flight at once
-  for (int idx = tid; idx < kBig * kBig; idx += kRowsPerCta) {
+  // stage T (upper triangle, zeros elsewhere) with asynchronous copies
+  for (int idx = tid; idx < kBig * kBig; idx += kBlockThreads) {
     const int j = idx / kBig, k = idx - j * kBig;
     const bool in = j <= k && k < nw;
     cp_async8(T + idx, in ? Lb + (C - 1 - c0 - j) * C + (C - 1 - c0 - k) : Lb, in);
   }
-  for (int k = 0; k < nw; ++k) cp_async8(Dsm + k * kRowsPerCta + tid, live ? sd + k : sd, live);
   cp_async_commit();
-#pragma unroll 8
-  for (int k = 0; k < nw; ++k) Wsm[k * kRowsPerCta + tid] = live ? wr[k] : (uint16_t)0;
+  const int64_t r = (int64_t)blockIdx.x * kRowsPerCta + (tid >> 2);
+  const bool live = r < R;
+  const int64_t row = b * R + (live ? r : 0);
+  const int cq = 32 * q;                  // first column of this lane
+  const int ncols = nw - cq;              // columns of this lane inside the block (<= 32)
+  double *sd = SD + row * C + c0 + cq;
+  const uint16_t *wr = w + row * C + c0 + cq;
+  double S[32];
+  uint32_t wv[16];  // the lane's 32 bf16 weights, two per word
+#pragma unroll
+  for (int m = 0; m < 32; ++m) S[m] = (live && m < ncols) ? sd[m] : 0.0;
+#pragma unroll
+  for (int m = 0; m < 16; ++m)
+    wv[m] = (live && 2 * m < ncols) ? *reinterpret_cast<const uint32_t *>(wr + 2 * m) : 0u;
+  const float sg = s_g[b];
+  const uint8_t *cr = codes + row * (C / kBlock) + (c0 + cq) / kBlock;
+  const double s_lo = (live && ncols > 0) ? (double)effective_scale(sg, cr[0]) : 0.0;
+  const double s_hi = (live && ncols > 16) ? (double)effective_scale(sg, cr[1]) : 0.0;
   cp_async_wait_all();
   __syncthreads();
-  for (int k = tid; k < kBig; k += kRowsPerCta) Tinv[k] = k < nw ? 1.0 / T[k * kBig + k] : 0.0;
+  for (int k = tid; k < kBig; k += kBlockThreads) Tinv[k] = k < nw ? 1.0 / T[k * kBig + k] : 0.0;
   __syncthreads();
-  if (!live) return;
-  const float sg = s_g[b];
-  const uint8_t *cr = codes + row * (C / kBlock) + c0 / kBlock;
-  uint8_t *pr = packed + row * (C / 2) + c0 / 2;
-  double s = 0.0;
-  uint32_t lo = 0;
-  for (int k = 0; k < nw; ++k) {
-    if ((k & (kBlock - 1)) == 0) s = (double)effective_scale(sg, cr[k / kBlock]);
-    // running sum of the earlier blocks plus this block's columns j < k
-    double a[8] = {Dsm[k * kRowsPerCta + tid], 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-    int j = 0;
-    for (; j + 7 < k; j += 8) {
+  uint32_t pk[4] = {0u, 0u, 0u, 0u};  // the lane's 32 codes
+  const int src = lane & ~3;
+  for (int q0 = 0; q0 < 4; ++q0) {
+    if (32 * q0 >= nw) break;
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        a[u] = fma(Dsm[(j + u) * kRowsPerCta + tid], T[(j + u) * kBig + k], a[u]);
+    for (int kk = 0; kk < 32; ++kk) {
+      const int k = 32 * q0 + kk;
+      const bool valid = k < nw;
+      // the owner lane rounds column k (every lane computes; only q == q0 keeps it)
+      const double wk = (double)__uint_as_float(
+          (kk & 1) ? (wv[kk >> 1] & 0xFFFF0000u) : (wv[kk >> 1] << 16));
+      const double x = fma(S[kk], valid ? Tinv[k] : 0.0, wk);
+      const double sc = kk < 16 ? s_lo : s_hi;
+      const int kq = e2m1_index64(fabs(x), sc);
+      const double qv = e2m1_magnitude(kq) * sc;
+      const bool neg = signbit(x);
+      const double d = wk - (neg ? -qv : qv);
+      if (q == q0) {
+        S[kk] = d;
+        pk[kk >> 3] |= ((uint32_t)kq | (neg ? 8u : 0u)) << (4 * (kk & 7));
+      }
+      const double e = valid ? __shfl_sync(0xFFFFFFFFu, d, src | q0) : 0.0;
+      // running sums of the later columns of the quad's row
+      const double *Tk = T + k * kBig + cq;
+#pragma unroll
+      for (int m = 0; m < 32; ++m) {
+        const bool later = q > q0 || (q == q0 && m > kk);
+        if (later) S[m] = fma(e, Tk[m], S[m]);
+      }
     }
-    for (; j < k; ++j) a[0] = fma(Dsm[j * kRowsPerCta + tid], T[j * kBig + k], a[0]);
-    const double acc = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
-    const double wk = (double)__uint_as_float((uint32_t)Wsm[k * kRowsPerCta + tid] << 16);
-    const double x = fma(acc, Tinv[k], wk);
-    const int kq = e2m1_index64(fabs(x), s);
-    const double q = e2m1_magnitude(kq) * s;
-    const bool neg = signbit(x);
-    const double d = wk - (neg ? -q : q);
-    Dsm[k * kRowsPerCta + tid] = d;
-    sd[k] = d;
-    const uint32_t code = (uint32_t)kq | (neg ? 8u : 0u);
-    if (k & 1) pr[k >> 1] = (uint8_t)(lo | (code << 4));
-    else lo = code;
   }
+  if (!live) return;
+#pragma unroll
+  for (int m = 0; m < 32; ++m)
+    if (m < ncols) sd[m] = S[m];
+  // byte stores: a row of packed codes starts on any 8-byte boundary
+  uint8_t *pr = packed + row * (C / 2) + (c0 + cq) / 2;
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    if (2 * i < ncols) pr[i] = (uint8_t)(pk[i >> 2] >> (8 * (i & 3)));
 }
 
 std::mutex g_block_attr_mu;
@@ -541,8 +611,8 @@ cudaError_t launch_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
   for (int64_t c0 = 0; e == cudaSuccess && c0 < C; c0 += kBig) {
     const int nw = (int)(C - c0 < kBig ? C - c0 : kBig);
     const dim3 grid((unsigned)((R + kRowsPerCta - 1) / kRowsPerCta), (unsigned)batch);
-    gptq_block_kernel<<<grid, kRowsPerCta, kBlockSmem, st>>>(w, R, C, s_g, codes, Hd, SD, packed,
-                                                              c0, nw);
+    gptq_block_kernel<<<grid, kBlockThreads, kBlockSmem, st>>>(w, R, C, s_g, codes, Hd, SD,
+                                                                packed, c0, nw);
     e = cudaGetLastError();
     const int64_t c1 = c0 + nw;
     if (e == cudaSuccess && c1 < C) {

@@ -317,6 +317,44 @@ __device__ __forceinline__ float block_mse32(const uint32_t w[8], uint2 q, float
   return e;
 }
 
+// The same fp32 block MSE at a table entry's scale, straight from the
+// values: each pair is rounded (the encode above, one conversion) and its
+// byte decoded by the hardware e2m1x2 -> f16x2 conversion in the same asm
+// block, then d_i = x_i - v_i s and e += d_i^2 in block_mse32's order, so
+// the result equals block_mse32 of the packed codes bit for bit, without
+// packing them.
+__device__ __forceinline__ uint32_t e2m1x2_round_decode(float hi, float lo) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 q;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, q;\n\t}"
+      : "=r"(h2)
+      : "f"(hi), "f"(lo));
+  return h2;
+}
+__device__ __forceinline__ float block_mse32_entry(const uint32_t w[8], const ScaleEntry &e) {
+  if (e.exact64) return block_mse32(w, encode_block_exact(w, e.s), e.s);
+  float acc = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float x0 = bf16_lo(w[j]), x1 = bf16_hi(w[j]);
+    float t0 = fmaf(x0, e.r_hi, x0 * e.r_lo), t1 = fmaf(x1, e.r_hi, x1 * e.r_lo);
+    const bool n0 = (__float_as_uint(t0) & 0x1FFFFFu) == 0u;
+    const bool n1 = (__float_as_uint(t1) & 0x1FFFFFu) == 0u;
+    if (n0 || n1) {
+      const float a0 = toward(t0, fmaf(-t0, e.s, x0)), a1 = toward(t1, fmaf(-t1, e.s, x1));
+      t0 = n0 ? a0 : t0;
+      t1 = n1 ? a1 : t1;
+    }
+    const uint32_t h2 = e2m1x2_round_decode(t1, t0);
+    const float d0 = fmaf(-f16_lo_to_float(h2), e.s, x0);
+    const float d1 = fmaf(-f16_hi_to_float(h2), e.s, x1);
+    acc = fmaf(d0, d0, acc);
+    acc = fmaf(d1, d1, acc);
+  }
+  return acc;
+}
+
 // Block MSE at the table entry's scale in fp64, with the operations of the
 // definition in its order: d_i = w_i - v_i s, e += d_i^2, i = 0..15, each
 // product and sum rounded on its own (no fused multiply-add), so that two
@@ -365,10 +403,13 @@ __global__ void __launch_bounds__(kThreads) four_over_six_kernel(const uint16_t 
     if (amax > 0.0f && hi != lo) {
       // fp32 screen; the exact fp64 comparison only when the two are close
       const ScaleEntry el = tab[lo], eh = tab[hi];
-      const uint2 ql = encode_block_entry(v, el), qh = encode_block_entry(v, eh);
-      const float fl = block_mse32(v, ql, el.s), fh = block_mse32(v, qh, eh.s);
-      if (fabsf(fh - fl) > 0x1p-16f * fmaxf(fh, fl)) code = fh < fl ? hi : lo;
-      else code = block_mse64(v, qh, eh.s) < block_mse64(v, ql, el.s) ? hi : lo;
+      const float fl = block_mse32_entry(v, el), fh = block_mse32_entry(v, eh);
+      if (fabsf(fh - fl) > 0x1p-16f * fmaxf(fh, fl)) {
+        code = fh < fl ? hi : lo;
+      } else {
+        const uint2 ql = encode_block_entry(v, el), qh = encode_block_entry(v, eh);
+        code = block_mse64(v, qh, eh.s) < block_mse64(v, ql, el.s) ? hi : lo;
+      }
     }
     codes[i] = (uint8_t)(amax > 0.0f ? code : 0u);
 #pragma unroll

@@ -60,13 +60,9 @@ namespace {
 constexpr int kThreads = 128;  // 4 warps
 constexpr int kWarps = kThreads / 32;
 constexpr int kTileRows = 16;
-#ifndef NVFP4_SEARCH_TILES
-#define NVFP4_SEARCH_TILES 4
-#endif
-constexpr int kTilesPerWarp = NVFP4_SEARCH_TILES;
-constexpr int kRowsPerCta = kWarps * kTileRows * kTilesPerWarp;  // 256
-static_assert((kRowsPerCta & (kRowsPerCta - 1)) == 0 && kRowsPerCta <= 65536,
-              "the row sort needs a power-of-two row count below 2^16");
+// Rows per CTA: 256 (four 16-row tiles per warp), or 128 when a problem has
+// few CTAs (the tail of the last wave then costs less).
+constexpr int kRowsLarge = kWarps * kTileRows * 4, kRowsSmall = kWarps * kTileRows * 2;
 constexpr float kTieBand = 1.0f / 4096.0f;
 constexpr float kZeroFloor = 0x1p-40f;  // relative to ||p||^2
 constexpr int kMaxClasses = kCandidates;
@@ -400,12 +396,15 @@ __global__ void __launch_bounds__(32)
 }
 
 // Local-Hessian: at most 72 registers, seven CTAs per SM; MSE nine.
-template <bool kLH>
+template <bool kLH, int kRowsPerCta>
 __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     search_kernel(const uint16_t *__restrict__ w, int64_t R, int64_t C,
                   const float *__restrict__ s_g_arr, const float *__restrict__ H,
                   const uint4 *__restrict__ frag, const Factor *__restrict__ fac,
                   uint8_t *__restrict__ codes, float *__restrict__ best_obj) {
+  static_assert((kRowsPerCta & (kRowsPerCta - 1)) == 0 && kRowsPerCta <= 65536 &&
+                    kRowsPerCta % (kWarps * kTileRows) == 0,
+                "the row sort needs a power-of-two row count below 2^16");
   const int64_t nb = C / kBlock;
   const int64_t b = blockIdx.y;
   const int64_t batch = blockIdx.z;
@@ -748,11 +747,22 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
                                 const float *s_g, const float *H, uint8_t *codes,
                                 float *best_obj, int local_hessian, cudaStream_t st) {
   if (R == 0 || C == 0) return cudaSuccess;
-  dim3 grid((unsigned)((R + kRowsPerCta - 1) / kRowsPerCta), (unsigned)(C / kBlock),
-            (unsigned)batch);
+  // Local-Hessian: 128-row CTAs when 256-row ones would fill fewer than six
+  // waves of the resident CTAs (dense 4096 x 4096: 4096 CTAs of 256 rows,
+  // about four waves; measured 2% faster there, 3.5% slower on the 128 MoE
+  // experts, which have 47 waves).  The MSE search measured slower with the
+  // smaller groups of rows sorted together and keeps 256.
+  const int64_t ctas_large = (R + kRowsLarge - 1) / kRowsLarge * (C / kBlock) * batch;
+  const bool small = local_hessian && ctas_large < (int64_t)sm_count() * 7 * 6;
+  const int rows = small ? kRowsSmall : kRowsLarge;
+  dim3 grid((unsigned)((R + rows - 1) / rows), (unsigned)(C / kBlock), (unsigned)batch);
   if (!local_hessian) {
-    search_kernel<false><<<grid, kThreads, 0, st>>>(w, R, C, s_g, nullptr, nullptr, nullptr,
-                                                    codes, best_obj);
+    if (small)
+      search_kernel<false, kRowsSmall><<<grid, kThreads, 0, st>>>(w, R, C, s_g, nullptr, nullptr,
+                                                                  nullptr, codes, best_obj);
+    else
+      search_kernel<false, kRowsLarge><<<grid, kThreads, 0, st>>>(w, R, C, s_g, nullptr, nullptr,
+                                                                  nullptr, codes, best_obj);
     return cudaGetLastError();
   }
   // factors of every H_b first (stream-ordered scratch, freed after the search)
@@ -766,7 +776,12 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
   factor_kernel<<<dim3((unsigned)(C / kBlock), (unsigned)batch), 32, 0, st>>>(H, frag, fac);
   e = cudaGetLastError();
   if (e == cudaSuccess) {
-    search_kernel<true><<<grid, kThreads, 0, st>>>(w, R, C, s_g, H, frag, fac, codes, best_obj);
+    if (small)
+      search_kernel<true, kRowsSmall><<<grid, kThreads, 0, st>>>(w, R, C, s_g, H, frag, fac,
+                                                                 codes, best_obj);
+    else
+      search_kernel<true, kRowsLarge><<<grid, kThreads, 0, st>>>(w, R, C, s_g, H, frag, fac,
+                                                                 codes, best_obj);
     e = cudaGetLastError();
   }
   const cudaError_t ef = scratch_free(scratch, st);

@@ -334,7 +334,7 @@ nvfp4_status nvfp4_hessian_full_accumulate(const uint16_t *x, int64_t n_tok, int
  *   damp         >= 0 (the GPTQ paper uses 0.01)
  *   packed       [batch, R, C/2] uint8, written (nibble order of
  *                nvfp4_quantize_pack)
- * Scratch (stream-ordered, library pool): batch (C^2 + R C) doubles.  A
+ * Scratch (stream-ordered, library pool): batch (C^2 + R C + 128^2) doubles.  A
  * Hessian that is not positive definite after dampening sets the device
  * status NVFP4_ERR_NOT_POSITIVE_DEFINITE (see nvfp4_get_device_status).
  */

@@ -47,7 +47,6 @@ __device__ int g_gptq_status = 0;
 
 namespace {
 
-
 // ----------------------------------------------------------------- fp64 GEMM
 // C[m][n] += alpha sum_k A[m][k] B[k][n] for m < M, n < N, with arbitrary
 // (also negative) element strides and a batch index in blockIdx.z.  `lower`:
@@ -605,7 +604,8 @@ cudaError_t launch_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
                         const uint8_t *codes, const float *H, double damp, uint8_t *packed,
                         cudaStream_t st) {
   if (R == 0 || C == 0) return cudaSuccess;
-  // scratch: lambda | Hd (-> its factor) | running sums / errors
+  // scratch: lambda | Hd (-> its factor) | running sums / errors | the
+  // inverse of the current 128-column diagonal block
   const size_t lam_bytes = ((size_t)batch * sizeof(double) + 255) / 256 * 256;
   const size_t hd_bytes = (size_t)batch * (size_t)C * (size_t)C * sizeof(double);
   const size_t sd_bytes = (size_t)batch * (size_t)R * (size_t)C * sizeof(double);
@@ -628,7 +628,7 @@ cudaError_t launch_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) e = cholesky_in_place(Hd, C, batch, Linv, st);
-  // columns in blocks of 128: each block's rows one thread each, then the
+  // columns in blocks of 128: each row of a block on a quad of lanes, then the
   // block's errors added to the running sums of every later column (rank-128)
   if (e == cudaSuccess)
     e = ensure_smem_attr(gptq_block_kernel, kBlockSmem, g_block_attr_mu, g_block_attr);

@@ -22,8 +22,9 @@
 //    lower Cholesky factor L gives T = J L J;
 //  - chol_block_kernel and the fp64 GEMM: blocked right-looking Cholesky of
 //    Hd in place, 128-column panels (the diagonal block factored and
-//    inverted by one CTA in shared memory, the rows below it solved by a
-//    GEMM with that inverse, the trailing matrix by a rank-128 update);
+//    inverted by one CTA, the rows below it solved by a GEMM with that
+//    inverse, the trailing matrix by a rank-128 update split so that most of
+//    it overlaps the next panel on a second stream);
 //  - gptq_block_kernel: 128 columns at a time, four lanes per row each
 //    holding 32 columns' running sums in registers; each column is rounded
 //    by its owner lane (exact fp64 midpoint test), its error shuffled to the
@@ -419,18 +420,39 @@ cudaError_t ensure_smem_attr(K kernel, int bytes, std::mutex &mu, bool *flags) {
 }
 
 // Linv: scratch [batch][128][128].
+// Look-ahead: each panel's trailing update is split into the next panel's
+// 128 columns, on the caller's stream, and the columns beyond, on a second
+// stream, where it overlaps the next panel's factor and solve.  The next
+// panel's own split update waits for it (both write the columns after the
+// next panel); everything else they touch is disjoint.
 cudaError_t cholesky_in_place(double *A, int64_t C, int64_t batch, double *Linv,
                               cudaStream_t st) {
   cudaError_t e = ensure_smem_attr(chol_block_kernel, kCholSmem, g_chol_attr_mu, g_chol_attr);
   if (e != cudaSuccess) return e;
   const int64_t CC = C * C;
-  for (int64_t P0 = 0; P0 < C; P0 += kBig) {
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_main = nullptr, ev_side = nullptr;
+  e = cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_main, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_side, cudaEventDisableTiming);
+  bool side_used = false;
+  // A[r0.., r0 .. r0+ncols) -= X X^T on the lower triangle, X = the panel's
+  // rows r0.. in its columns P0 .. P0+nw
+  auto trailing = [&](int64_t P0, int nw, int64_t r0, int64_t ncols, cudaStream_t s) {
+    GemmF64 g{};
+    g.M = C - r0; g.N = ncols; g.K = nw; g.alpha = -1.0;
+    g.A = A + r0 * C + P0; g.sAm = C; g.sAk = 1; g.bsA = CC;
+    g.B = g.A; g.sBk = 1; g.sBn = C; g.bsB = CC;
+    g.C = A + r0 * C + r0; g.sCm = C; g.sCn = 1; g.bsC = CC;
+    g.lower = 1;
+    return gemm_f64(g, batch, s);
+  };
+  for (int64_t P0 = 0; e == cudaSuccess && P0 < C; P0 += kBig) {
     const int nw = (int)(C - P0 < kBig ? C - P0 : kBig);
     chol_block_kernel<<<(unsigned)batch, kCholThreads, kCholSmem, st>>>(A, C, P0, nw, Linv);
     e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
     const int64_t P1 = P0 + nw, rest = C - P1;
-    if (rest <= 0) break;
+    if (e != cudaSuccess || rest <= 0) break;
     {
       // rows below the block: X = A_panel L_pp^-T (in place: one CTA column)
       GemmF64 g{};
@@ -440,21 +462,28 @@ cudaError_t cholesky_in_place(double *A, int64_t C, int64_t batch, double *Linv,
       g.C = A + P1 * C + P0; g.sCm = C; g.sCn = 1; g.bsC = CC;
       g.overwrite = 1;
       e = gemm_f64(g, batch, st);
-      if (e != cudaSuccess) return e;
     }
-    {
-      // trailing block -= X X^T (lower triangle)
-      GemmF64 g{};
-      g.M = rest; g.N = rest; g.K = nw; g.alpha = -1.0;
-      g.A = A + P1 * C + P0; g.sAm = C; g.sAk = 1; g.bsA = CC;
-      g.B = g.A; g.sBk = 1; g.sBn = C; g.bsB = CC;
-      g.C = A + P1 * C + P1; g.sCm = C; g.sCn = 1; g.bsC = CC;
-      g.lower = 1;
-      e = gemm_f64(g, batch, st);
-      if (e != cudaSuccess) return e;
+    // the next panel's columns, after the earlier panels' updates beyond them
+    if (e == cudaSuccess && side_used) e = cudaStreamWaitEvent(st, ev_side, 0);
+    const int64_t nw2 = rest < kBig ? rest : kBig, P2 = P1 + nw2;
+    if (e == cudaSuccess) e = trailing(P0, nw, P1, nw2, st);
+    if (e == cudaSuccess && C - P2 > 0) {
+      e = cudaEventRecord(ev_main, st);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev_main, 0);
+      if (e == cudaSuccess) e = trailing(P0, nw, P2, C - P2, side);
+      if (e == cudaSuccess) e = cudaEventRecord(ev_side, side);
+      side_used = side_used || e == cudaSuccess;
     }
   }
-  return cudaSuccess;
+  // join the second stream before anything reads the factor
+  if (side_used) {
+    const cudaError_t ej = cudaStreamWaitEvent(st, ev_side, 0);
+    if (e == cudaSuccess) e = ej;
+  }
+  if (ev_main) cudaEventDestroy(ev_main);
+  if (ev_side) cudaEventDestroy(ev_side);
+  if (side) cudaStreamDestroy(side);
+  return e;
 }
 
 // ---------------------------------------------------------------------- GPTQ

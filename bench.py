@@ -248,7 +248,7 @@ class Runner:
                 rows.append((pre + "gptq",
                              lambda L=L, c=fin: nv.gptq(L.W[0], L.s_g, c[0], L.Hf, GPTQ_DAMP,
                                                         out=L.packed[0]),
-                             2 * n_w + nb + 4 * L.C * L.C + n_w // 2, 5 * npan - 1))
+                             2 * n_w + nb + 4 * L.C * L.C + n_w // 2, gptq_launches(npan)))
             else:
                 rows.append((pre + "quantize_pack",
                              lambda L=L, c=fin: nv.quantize_pack(L.W, L.s_g, c, out=L.packed),
@@ -548,6 +548,15 @@ def run_gpu(args):
     if pg:
         pg.barrier()
         pg.destroy_process_group()
+
+
+def gptq_launches(npan):
+    """Kernels one GPTQ call launches for npan 128-column panels: lambda and
+    the reversed copy; per panel the diagonal block, and (but the last) the
+    panel solve and the next panel's update, the update beyond it (but the
+    last two); per column block the row kernel and (but the last) the
+    running-sum product."""
+    return (2 + npan + 2 * max(npan - 1, 0) + max(npan - 2, 0) + npan + max(npan - 1, 0))
 
 
 def make_roofline(run, kernels, pk, pk_kind, workload, lh_evals):

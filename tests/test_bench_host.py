@@ -58,3 +58,11 @@ def test_roofline_gptq_is_fp64_definition_flops():
     assert r["bound"] == "alu" and abs(r["peak"] - round(peak, 2)) < 1e-9
     assert abs(r["achieved"] - round(flop / 10e-3 / 1e12, 2)) < 1e-9
     assert r["traffic"] is None
+
+
+def test_gptq_launch_count_follows_the_panel_schedule():
+    import bench
+    # C = 128: lambda, copy, one diagonal block, one row kernel
+    # C = 256: + panel solve and next-panel update, a second block, one product
+    # C = 384: + one update beyond the next panel, a third panel and block
+    assert [bench.gptq_launches(n) for n in (1, 2, 3)] == [4, 9, 15]

@@ -411,6 +411,29 @@ def test_search_ragged_rows_mixed_magnitudes(nv):
     assert np.all(cm[7] == 1) and np.all(clh[300:310] == 1)
 
 
+@pytest.mark.parametrize("R,C", [(1, 16), (3, 32), (17, 48), (1, 48), (17, 16), (3, 16)])
+def test_search_rules_on_tiny_shapes(nv, R, C):
+    """Every scale rule on the smallest shapes (one to seventeen rows, one to
+    three column blocks): almost every row of a CTA is padding."""
+    W = rand_bf16((R, C), R * 100 + C, 0.02, 0.1, 20.0)
+    X = rand_bf16((50, C), R + C, 1.0)
+    wu = bf16_bits(W)
+    s_g = nv.global_scale(W.cuda())
+    sg = s_g.item()
+    assert sg == oracle.global_scale(wu)
+    H = torch.zeros(C // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate(X.cuda(), H)
+    H64 = H.cpu().numpy().astype(np.float64)
+    clh = nv.scale_search_local_hessian(W.cuda(), s_g, H).cpu().numpy()
+    check_search_codes(clh, oracle.scale_search_lh(wu, sg, H64)[0], wu, sg, H64)
+    cm = nv.scale_search_mse(W.cuda(), s_g).cpu().numpy()
+    check_search_codes(cm, oracle.scale_search_mse(wu, sg)[0], wu, sg)
+    np.testing.assert_array_equal(nv.scale_search_max(W.cuda(), s_g).cpu().numpy(),
+                                  oracle.scale_search_max(wu, sg))
+    np.testing.assert_array_equal(nv.scale_search_four_over_six(W.cuda(), s_g).cpu().numpy(),
+                                  oracle.scale_search_four_over_six(wu, sg))
+
+
 def test_search_evaluation_counters(nv):
     """The work statistic: between 1 and 126 evaluations per block searched,
     counted per rule, and zeroed by a reset."""

@@ -76,3 +76,83 @@ def test_look_ahead_split_of_the_trailing_update():
     split[P2:, P2:] -= X[P2:] @ X[P2:].T
     lower = np.tril(np.ones((C, C), bool))
     np.testing.assert_allclose(split[lower], full[lower], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------ E2M1 encode rule
+def _f32(v):
+    return np.asarray(v, np.longdouble).astype(np.float32)
+
+
+def _encode_rule(x, s, step=True):
+    """The kernel's encode of x at scale s > 0 (s >= 2^-100; both arrays of
+    one shape), emulated with exact intermediates and one rounding per fp32
+    operation: r_hi = 1/s rounded down, r_lo = fl(fl(1 - s r_hi) r_hi),
+    t = fl(x r_hi + fl(x r_lo)); a t with 21 zero low mantissa bits steps to
+    its neighbouring float across q = x / s by the sign of x - t s; then
+    nearest-even on the E2M1 grid with saturation, the sign from t."""
+    ld = np.longdouble
+    s = np.asarray(s, np.float32)
+    sl = s.astype(ld)
+    r = (ld(1) / sl).astype(np.float32)
+    r = np.where(r.astype(ld) * sl > 1, np.nextafter(r, np.float32(-np.inf)), r)
+    r_lo = _f32(_f32(ld(1) - sl * r.astype(ld)).astype(ld) * r.astype(ld))
+    xl = np.asarray(x, np.float64).astype(ld)
+    t = _f32(xl * r.astype(ld) + _f32(xl * r_lo.astype(ld)).astype(ld))
+    if step:
+        near = (t.view(np.uint32) & np.uint32(0x1FFFFF)) == 0
+        rho = xl - t.astype(ld) * sl
+        up = np.nextafter(t, np.float32(np.inf))
+        dn = np.nextafter(t, np.float32(-np.inf))
+        t = np.where(near, np.where(rho > 0, up, np.where(rho < 0, dn, t)), t)
+    a = np.abs(t.astype(np.float64))
+    k = np.zeros(a.shape, np.int64)
+    for i, m in enumerate(MIDS):
+        k += (a > m) if i % 2 == 0 else (a >= m)
+    return k | np.where(np.signbit(t), 8, 0)
+
+
+def _all_finite_bf16():
+    u = np.arange(1 << 16, dtype=np.uint32)
+    return bits_to_f64(u[((u >> 7) & 0xFF) != 0xFF].astype(np.uint16))
+
+
+def _oracle_codes(oracle_mod, x, s):
+    return np.array([oracle_mod.e2m1_encode(float(a), float(b)) for a, b in zip(x, s)])
+
+
+# power-of-two scales (exact quotients and ties), other round scales, and
+# tensor scales fl32(amax / 2688) times an E4M3 value
+ROUND_SCALES = [1.0, 14.0, 2.0 ** -5, 3 * 2.0 ** -7,
+                float(np.float32(84 / 2688)), float(np.float32(97 / 2688)),
+                float(np.float32(np.float32(252 / 2688) * np.float32(1.75))),
+                float(np.float32(np.float32(189 / 2688) * np.float32(1.5)))]
+
+
+@pytest.mark.parametrize("s", ROUND_SCALES + list(
+    np.random.default_rng(0).uniform(1e-4, 1e2, 3).astype(np.float32)))
+@pytest.mark.filterwarnings("ignore:overflow encountered in cast")
+def test_kernel_encode_rule_on_every_bf16(oracle_mod, s):
+    x = _all_finite_bf16()
+    sv = np.full(x.shape, s, np.float32)
+    assert np.array_equal(_encode_rule(x, sv), _oracle_codes(oracle_mod, x, sv))
+
+
+def test_kernel_encode_rule_near_midpoints(oracle_mod):
+    """Scales chosen so that x / s lies within an fp32 ulp of a rounding
+    midpoint m: s = fl32(x / m) and its two fp32 neighbours.  Here t often
+    lands on m while q does not; the residual step must decide those, and
+    the cases must include some that nearest-even on t alone gets wrong."""
+    rng = np.random.default_rng(7)
+    u = rng.integers(0, 1 << 15, 3000).astype(np.uint16)
+    x = bits_to_f64(u)
+    x = x[(np.abs(x) > 2.0 ** -90) & (np.abs(x) < 2.0 ** 90)]
+    xs, ss = [], []
+    for m in MIDS:
+        s0 = (x / m).astype(np.float32)
+        for s in (s0, np.nextafter(s0, np.float32(np.inf)), np.nextafter(s0, np.float32(0))):
+            xs.append(x)
+            ss.append(s)
+    xs, ss = np.concatenate(xs), np.concatenate(ss)
+    ref = _oracle_codes(oracle_mod, xs, ss)
+    assert np.array_equal(_encode_rule(xs, ss), ref)
+    assert np.sum(_encode_rule(xs, ss, step=False) != ref) > 0

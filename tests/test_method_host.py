@@ -156,3 +156,74 @@ def test_kernel_encode_rule_near_midpoints(oracle_mod):
     ref = _oracle_codes(oracle_mod, xs, ss)
     assert np.array_equal(_encode_rule(xs, ss), ref)
     assert np.sum(_encode_rule(xs, ss, step=False) != ref) > 0
+
+
+# ------------------------------------------------------ E4M3 scale code
+def _e4m3_rn_satfinite(t):
+    """Nearest-even E4M3 code of the magnitude of fp32 t (codes 0..0x7E; above
+    448 saturates to 0x7E).  Values: subnormals j 2^-9 (j < 8), then
+    (1 + m/8) 2^(e-7)."""
+    vals = np.array([j * 2.0 ** -9 if j < 8 else (1 + (j & 7) / 8) * 2.0 ** ((j >> 3) - 7)
+                     for j in range(0x7F)])
+    a = np.abs(np.asarray(t, np.float64))
+    hi = np.clip(np.searchsorted(vals, a), 1, 0x7E)
+    lo = hi - 1
+    dl, dh = a - vals[lo], vals[hi] - a
+    code = np.where(dl < dh, lo, np.where(dh < dl, hi, np.where(lo % 2 == 0, lo, hi)))
+    return np.where(a >= vals[0x7E], 0x7E, code)
+
+
+def _max_rule_code(amax, s_g, k):
+    """The kernel's E4M3 code of amax / (k s_g): D = k s_g exact in fp64,
+    R = fl64(1/D) split r_hi = fl32(R), r_lo = fl32(R - r_hi);
+    t = fl32(amax r_hi + fl32(amax r_lo)); ta = the float next to t across
+    the quotient (the sign of amax - t D); the code is RN(t) when RN(t) and
+    RN(ta) agree or RN(t) is odd, else RN(ta)."""
+    ld = np.longdouble
+    D = float(k) * float(np.float32(s_g))
+    R = 1.0 / D
+    r_hi = np.float32(R)
+    r_lo = np.float32(R - float(r_hi))
+    a = np.asarray(amax, np.float32).astype(ld)
+    t = _f32(a * ld(r_hi) + _f32(a * ld(r_lo)).astype(ld))
+    rho = a - t.astype(ld) * ld(D)
+    ta = np.where(rho > 0, np.nextafter(t, np.float32(np.inf)),
+                  np.where(rho < 0, np.nextafter(t, np.float32(-np.inf)), t))
+    ct, ca = _e4m3_rn_satfinite(t), _e4m3_rn_satfinite(ta)
+    return np.where(ct % 2 == 1, ct, ca)
+
+
+@pytest.mark.parametrize("k", [6, 4])
+@pytest.mark.parametrize("s_g", [float(np.float32(v / 2688)) for v in (1.0, 0.37, 12.5, 3e4)]
+                         + [2.0 ** -7, float(np.float32(1 / 3))])
+def test_kernel_scale_code_on_every_bf16_amax(oracle_mod, k, s_g):
+    """Every positive finite bf16 amax whose quotient amax / (k s_g) falls in
+    [2^-12, 512], so the sweep spans zero, the subnormal codes, every
+    binade, and saturation."""
+    u = np.arange(1, 0x7F80, dtype=np.uint32).astype(np.uint16)
+    amax = bits_to_f64(u)
+    q = amax / (k * s_g)
+    amax = amax[(q >= 2.0 ** -12) & (q <= 512)]
+    ref = np.array([oracle_mod.e4m3_round_quotient(a, k * float(np.float32(s_g))) for a in amax])
+    assert np.array_equal(_max_rule_code(amax, s_g, k), ref)
+
+
+def test_kernel_scale_code_near_midpoints(oracle_mod):
+    """s_g chosen so that amax / (6 s_g) lies within an fp32 ulp of an E4M3
+    rounding midpoint; the step across the quotient must decide those, and
+    some must come out wrong from RN(t) alone."""
+    vals = np.array([j * 2.0 ** -9 if j < 8 else (1 + (j & 7) / 8) * 2.0 ** ((j >> 3) - 7)
+                     for j in range(0x7F)])
+    mids = (vals[:-1] + vals[1:]) / 2
+    rng = np.random.default_rng(3)
+    amax = bits_to_f64(rng.integers(0x3000, 0x4F00, 40).astype(np.uint16))
+    bad = 0
+    for a in amax:
+        for m in mids[::3]:
+            s0 = np.float32(a / (6 * m))
+            for s in (s0, np.nextafter(s0, np.float32(np.inf)), np.nextafter(s0, np.float32(0))):
+                ref = oracle_mod.e4m3_round_quotient(a, 6 * float(s))
+                assert int(_max_rule_code(np.array([a]), s, 6)[0]) == ref, (a, float(s))
+                t = _f32(np.longdouble(a) / np.longdouble(6 * float(s)))
+                bad += int(_e4m3_rn_satfinite(t)[()] != ref)
+    assert bad > 0

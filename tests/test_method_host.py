@@ -227,3 +227,111 @@ def test_kernel_scale_code_near_midpoints(oracle_mod):
                 t = _f32(np.longdouble(a) / np.longdouble(6 * float(s)))
                 bad += int(_e4m3_rn_satfinite(t)[()] != ref)
     assert bad > 0
+
+
+# ------------------------------------------- class quotients of the search
+def _certified(S):
+    """The search kernel's certificate for fp32 scales S: for m = 1, 3, 5, 7
+    the bits of m S (exact in fp64) below its eighth significant bit stay
+    more than 2^-20 of the leading bit away from 0 and from 1."""
+    S = np.asarray(S, np.float32).astype(np.float64)
+    far = np.ones(S.shape, bool)
+    for m in (1, 3, 5, 7):
+        rem = (S * m).view(np.int64) & ((1 << 45) - 1)
+        far &= (rem > (1 << 32)) & (rem < (1 << 45) - (1 << 32))
+    return far
+
+
+def _min_rel_distance_to_midpoints(S):
+    """Brute force: the smallest relative distance between x / S, over every
+    bf16 significand x (8 bits; a power of two aside every bf16 is one) and
+    an E2M1 rounding midpoint m 2^k (m = 1, 3, 5, 7, any k)."""
+    S = np.asarray(S, np.float32).astype(np.float64)
+    sig = np.arange(128, 256, dtype=np.float64)
+    out = np.full(S.shape, np.inf)
+    for m in (1, 3, 5, 7):
+        r = sig[None, :] / (m * S[:, None])
+        frac = r / np.exp2(np.floor(np.log2(r)))
+        frac = np.where(frac < 1, frac * 2, np.where(frac >= 2, frac / 2, frac))
+        out = np.minimum(out, np.minimum(frac - 1, (2 - frac) / 2).min(axis=1))
+    return out
+
+
+def test_search_certificate_is_sound():
+    """A certified class scale keeps every bf16 quotient more than 2^-22
+    (relative; twice the distance one fp32 rounding can cross) away from
+    every midpoint, on random scales over the whole range and on scales
+    built to sit on or next to a midpoint ratio; and it certifies most
+    scales, so the per-class stepping stays rare."""
+    rng = np.random.default_rng(11)
+    S = (rng.integers(0x0D800000, 0x71800000, 40000).astype(np.uint32)).view(np.float32)
+    sig = rng.integers(128, 256, 4000).astype(np.float64)
+    m = rng.choice([1.0, 3.0, 5.0, 7.0], 4000)
+    Sb = (sig / m).astype(np.float32)
+    Sb = np.concatenate([Sb, np.nextafter(Sb, np.float32(np.inf)), np.nextafter(Sb, np.float32(0))])
+    for s in (S, Sb):
+        cert = _certified(s)
+        assert np.all(_min_rel_distance_to_midpoints(s[cert]) > 2.0 ** -22)
+    assert _certified(S).mean() > 0.99
+    assert not np.any(_certified(Sb[:4000]))  # exact ratios: never certified
+
+
+def _class_codes(a, s_g, o, p, step=True):
+    """E2M1 codes of magnitudes a at the candidate o 2^p, the search kernel's
+    way: S = fl32(s_g o), R = fl64(1/S) split r_hi = fl32(R),
+    r_lo = fl32(R - r_hi); t = fl32(a r_hi + fl32(a r_lo)); for an
+    uncertified S a t with 21 zero low mantissa bits steps across a / S;
+    then nearest-even of t 2^-p."""
+    ld = np.longdouble
+    S = np.float32(np.float32(s_g) * np.float32(o))
+    R = 1.0 / float(S)
+    r_hi = np.float32(R)
+    r_lo = np.float32(R - float(r_hi))
+    al = np.asarray(a, np.float64).astype(ld)
+    t = _f32(al * ld(r_hi) + _f32(al * ld(r_lo)).astype(ld))
+    if step and not _certified(S):
+        near = (t.view(np.uint32) & np.uint32(0x1FFFFF)) == 0
+        rho = al - t.astype(ld) * ld(S)
+        t = np.where(near & (rho > 0), np.nextafter(t, np.float32(np.inf)),
+                     np.where(near & (rho < 0), np.nextafter(t, np.float32(0)), t))
+    v = np.abs(t.astype(np.float64) * 2.0 ** -p)
+    k = np.zeros(v.shape, np.int64)
+    for i, mid in enumerate(MIDS):
+        k += (v > mid) if i % 2 == 0 else (v >= mid)
+    return k
+
+
+def _candidates():
+    """(code, odd part o, exponent p) of every nonzero E4M3 code: value o 2^p."""
+    out = []
+    for c in range(1, 0x7F):
+        M, E = (c, -9) if c < 8 else (8 + (c & 7), (c >> 3) - 10)
+        tz = (M & -M).bit_length() - 1
+        out.append((c, M >> tz, E + tz))
+    return out
+
+
+@pytest.mark.parametrize("s_g,near_ratio",
+                         [(float(np.float32(v / 2688)), False) for v in (1.0, 0.0731, 17.0)]
+                         + [(float(np.float32(v)), True) for v in (1 / 3, 1 / 5, 1 / 7, 3 / 7)]
+                         + [(2.0 ** -9, False)])
+@pytest.mark.filterwarnings("ignore:overflow encountered in cast")
+def test_search_class_codes_on_every_bf16(oracle_mod, s_g, near_ratio):
+    """Every candidate code (126) on every non-negative finite bf16
+    magnitude: the class-quotient codes equal the oracle's rounding at the
+    candidate's effective scale.  The scales 1/3, 1/5, 1/7, 3/7 make class
+    quotients land within a float of midpoints, and there plain
+    nearest-even of t without the step must fail somewhere."""
+    u = np.arange(0, 0x7F80, dtype=np.uint16)
+    a = bits_to_f64(u)
+    w = u.reshape(-1, 16)
+    wrong_without_step = 0
+    for c, o, p in _candidates():
+        codes = np.full((w.shape[0], 1), c, np.uint8)
+        packed = oracle_mod.quantize_pack(w, np.float32(s_g), codes).reshape(-1)
+        ref = np.empty(a.size, np.int64)
+        ref[0::2], ref[1::2] = packed & 0xF, packed >> 4
+        assert np.array_equal(_class_codes(a, s_g, o, p), ref), (c, o, p)
+        wrong_without_step += int(np.sum(_class_codes(a, s_g, o, p, step=False) != ref))
+    if near_ratio:
+        assert wrong_without_step > 0

@@ -335,3 +335,87 @@ def test_search_class_codes_on_every_bf16(oracle_mod, s_g, near_ratio):
         wrong_without_step += int(np.sum(_class_codes(a, s_g, o, p, step=False) != ref))
     if near_ratio:
         assert wrong_without_step > 0
+
+
+# ------------------------------------------- eigenvalue bound of the pruning
+def _cholesky16_drop(H):
+    """The search kernel's 16x16 factor: fp64 right-looking Cholesky of the
+    fp32 block, a pivot at or below 1e-12 of the largest diagonal (or not
+    finite) dropping its column; the factor stored in fp32."""
+    a = H.astype(np.float64).copy()
+    n = a.shape[0]
+    tol = 1e-12 * np.max(np.diag(a))
+    L = np.zeros((n, n))
+    for k in range(n):
+        akk = a[k, k]
+        if akk > tol and akk < 1e300:
+            piv = np.sqrt(akk)
+            L[k, k] = piv
+            L[k + 1:, k] = a[k + 1:, k] / piv
+        a[k + 1:, k + 1:] -= np.outer(L[k + 1:, k], L[k + 1:, k])
+    return L.astype(np.float32)
+
+
+def _lambda_bound(Lf):
+    """0.98 / ||(L L^T)^-1||_1 from the fp32 factor (fp64 triangular solves),
+    0 for a dropped pivot or when max diag(L L^T) ||(L L^T)^-1||_1 > 1e4."""
+    L = Lf.astype(np.float64)
+    if np.any(np.diag(L) == 0):
+        return 0.0
+    maxdiag = np.max(np.sum(L * L, axis=1))
+    Linv = np.linalg.solve(L, np.eye(L.shape[0]))
+    colsum = np.max(np.sum(np.abs(Linv.T @ Linv), axis=0))
+    if not (0 < colsum < 1e300) or maxdiag * colsum > 1e4:
+        return 0.0
+    return float(np.float32(0.98 / colsum))
+
+
+def _gram_blocks():
+    """16x16 fp32 Gram blocks of bf16 calibration tokens: token counts from
+    1 to 2048, outlier channels up to 100x, zero and duplicated channels,
+    correlated channels, and the all-zero block."""
+    rng = np.random.default_rng(21)
+    out = []
+    for i in range(600):
+        n = int(rng.choice([1, 3, 15, 16, 17, 40, 256, 2048]))
+        x = rng.standard_normal((n, 16))
+        kind = i % 6
+        if kind == 1:
+            x[:, rng.integers(0, 16, 2)] *= rng.uniform(10, 100)
+        elif kind == 2:
+            x[:, rng.integers(0, 16)] = 0.0
+        elif kind == 3:
+            j = rng.integers(0, 15)
+            x[:, j + 1] = x[:, j]
+        elif kind == 4:
+            x = x @ (np.eye(16) + 0.9 * rng.standard_normal((16, 16)) / 4)
+        elif kind == 5:
+            x *= rng.uniform(1e-6, 1e6)
+        xb = bits_to_f64(bf16_bits(torch.from_numpy(x).float().to(torch.bfloat16)))
+        out.append((xb.T @ xb).astype(np.float32))
+    out.append(np.zeros((16, 16), np.float32))
+    return out
+
+
+def test_pruning_eigenvalue_bound_is_a_lower_bound():
+    """The pruning bounds hold when lambda <= the smallest eigenvalue of the
+    matrix the screen scores with (L L^T, L the fp32 factor) and of H itself;
+    a nonzero lambda also stays within the 1-norm's factor 4 (n = 16) of
+    lambda_min, so the bound keeps its pruning power; well-conditioned
+    blocks get a nonzero bound."""
+    nonzero = 0
+    for H in _gram_blocks():
+        Lf = _cholesky16_drop(H)
+        lam = _lambda_bound(Lf)
+        Ld = Lf.astype(np.float64)
+        lmin_llt = np.linalg.eigvalsh(Ld @ Ld.T)[0]
+        lmin_h = np.linalg.eigvalsh(H.astype(np.float64))[0]
+        assert lam >= 0.0
+        if lam > 0:
+            nonzero += 1
+            assert lam <= lmin_llt and lam <= lmin_h, (lam, lmin_llt, lmin_h)
+            assert lam >= 0.98 / 4 * lmin_llt * (1 - 1e-6)
+        d = np.diag(H).astype(np.float64)
+        if d.max() > 0 and lmin_h > 1e-3 * d.max():
+            assert lam > 0
+    assert nonzero > 150

@@ -193,8 +193,9 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
 
 // Everything a block's encode needs from its scale, computed once per code
 // and CTA: s_eff and its reciprocal split (r_hi rounded down, so r_lo >= 0 and
-// x = -0 keeps its sign in t), or 0 for scales below 2^-100 (where the
-// reciprocal may overflow), zero or NaN, which take the exact fp64 encode.
+// x = -0 keeps its sign in t), or 0 for scales outside [2^-100, 2^100) (below,
+// the reciprocal may overflow; above, r_lo is subnormal and too coarse near
+// the top of the fp32 range), zero or NaN, which take the exact fp64 encode.
 struct ScaleEntry {
   float s, r_hi, r_lo;
   uint32_t exact64;
@@ -205,7 +206,7 @@ __device__ __forceinline__ ScaleEntry make_scale_entry(float s) {
   e.r_hi = 0.0f;
   e.r_lo = 0.0f;
   e.exact64 = 1u;
-  if (s >= 0x1p-100f) {
+  if (s >= 0x1p-100f && s < 0x1p100f) {
     e.r_hi = __frcp_rd(s);
     e.r_lo = fmaf(-s, e.r_hi, 1.0f) * e.r_hi;
     e.exact64 = 0u;
@@ -300,9 +301,10 @@ __device__ __forceinline__ float e2m1_code_value(uint2 q, int i) {
 }
 
 // Block MSE at scale s in fp32 (a screen: every d_i is rounded once and the
-// 16 non-negative terms are summed with one rounding each, so the relative
-// error stays below 2^-20).  Codes back to values by the hardware e2m1x2 ->
-// f16x2 conversion (exact).
+// 16 non-negative terms are summed with one rounding each, so the error
+// stays below 2^-20 relative plus, where terms or partial sums fall into the
+// subnormal range (tensor scales near 1e-20 and below), 2^-145 absolute).
+// Codes back to values by the hardware e2m1x2 -> f16x2 conversion (exact).
 __device__ __forceinline__ float block_mse32(const uint32_t w[8], uint2 q, float s) {
   float e = 0.0f;
 #pragma unroll
@@ -402,9 +404,10 @@ __global__ void __launch_bounds__(kThreads) four_over_six_kernel(const uint16_t 
     uint32_t code = lo;
     if (amax > 0.0f && hi != lo) {
       // fp32 screen; the exact fp64 comparison only when the two are close
+      // (relative 2^-16, or absolute 2^-130 for subnormal sums)
       const ScaleEntry el = tab[lo], eh = tab[hi];
       const float fl = block_mse32_entry(v, el), fh = block_mse32_entry(v, eh);
-      if (fabsf(fh - fl) > 0x1p-16f * fmaxf(fh, fl)) {
+      if (fabsf(fh - fl) > fmaf(0x1p-16f, fmaxf(fh, fl), 0x1p-130f)) {
         code = fh < fl ? hi : lo;
       } else {
         const uint2 ql = encode_block_entry(v, el), qh = encode_block_entry(v, eh);

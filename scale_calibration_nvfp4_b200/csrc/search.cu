@@ -38,7 +38,8 @@
 // that step.
 //
 // Winner: fp32 screen keeping the best three objectives; when the best two
-// are within 2^-12 (relative) or the best is numerically zero, the candidates
+// are within 2^-12 (relative, plus 2^-130 absolute for objectives in the
+// subnormal range) or the best is numerically zero, the candidates
 // in the band are re-scored in fp64 straight from the definition
 // (delta H_b delta^T with exact E2M1 codes, one element per lane, two
 // candidates per warp pass) and the first minimum in ascending code order
@@ -64,6 +65,11 @@ constexpr int kTileRows = 16;
 // few CTAs (the tail of the last wave then costs less).
 constexpr int kRowsLarge = kWarps * kTileRows * 4, kRowsSmall = kWarps * kTileRows * 2;
 constexpr float kTieBand = 1.0f / 4096.0f;
+// Absolute part of the band and of the pruning margins: where objectives,
+// terms or bounds fall into the fp32 subnormal range (a row far below its
+// tile's largest), each operation errs by up to 2^-150 and a key moves by up
+// to 127 * 2^-149, far below this; elsewhere it changes nothing.
+constexpr float kAbsBand = 0x1p-130f;
 constexpr float kZeroFloor = 0x1p-40f;  // relative to ||p||^2
 constexpr int kMaxClasses = kCandidates;
 
@@ -572,14 +578,20 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     // pz[nt][2..3] row g+8, same n.  Local-Hessian: from the tensor cores
     // with w scaled by 2^kw (exact; the tile maximum lands in [2^14, 2^15) in
     // f16), so pz and every z below carry the factor sigma_L 2^kw, removed
-    // from the reported objective at the end.  MSE: p = w.
+    // from the reported objective at the end.  MSE: p = 2^kw w.
     float pz[2][4];
-    float zscale = 1.0f;  // objectives carry zscale^2
+    // Both rules scale w by 2^kw (exact), putting the tile's largest |w| in
+    // [2^14, 2^15): objectives and bounds then stay in the normal fp32 range
+    // for tiny and for huge weights alike (at most 2^127: a tile whose largest
+    // |w| is below 2^-113 lands lower, its bf16 values still exact in f16).
+    // Objectives carry zscale^2 = (sigma 2^kw)^2, kept as its exponent: zscale
+    // itself can pass the fp32 range (sigma <= 2^90 for an fp32 H), and
+    // nothing below multiplies by it.
+    const int kw = m ? min(14 - ((int)(m >> 7) - 127), 127) : 0;
+    const float wsc = ldexpf(1.0f, kw);
+    int zexp = kw;
     if (kLH) {
-      const int emax = (int)(m >> 7) - 127;  // exponent of the tile's largest |w|
-      const int kw = m ? 14 - emax : 0;
-      const float wsc = ldexpf(1.0f, kw);
-      zscale = sigma * wsc;
+      zexp += (int)((__float_as_uint(sigma) >> 23) & 0xFFu) - 127;
       uint32_t Aw[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -590,11 +602,12 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       mma_f16_16816(pz[0], Aw, bl[0][0], bl[0][1], pz[0]);
       mma_f16_16816(pz[1], Aw, bl[1][0], bl[1][1], pz[1]);
     } else {
-      pz[0][0] = xs[0]; pz[0][1] = xs[1]; pz[0][2] = xs[2]; pz[0][3] = xs[3];
-      pz[1][0] = xs[4]; pz[1][1] = xs[5]; pz[1][2] = xs[6]; pz[1][3] = xs[7];
+      pz[0][0] = xs[0] * wsc; pz[0][1] = xs[1] * wsc; pz[0][2] = xs[2] * wsc;
+      pz[0][3] = xs[3] * wsc; pz[1][0] = xs[4] * wsc; pz[1][1] = xs[5] * wsc;
+      pz[1][2] = xs[6] * wsc; pz[1][3] = xs[7] * wsc;
     }
-    // multiplier of u in z: s for MSE; s 2^kw for Local-Hessian (u carries sigma_L)
-    const float umul = kLH ? zscale / sigma : 1.0f;
+    // multiplier of u in z: s 2^kw (for Local-Hessian u carries sigma_L)
+    const float umul = wsc;
     float pp0 = pz[0][0] * pz[0][0] + pz[0][1] * pz[0][1] + pz[1][0] * pz[1][0] +
                 pz[1][1] * pz[1][1];
     float pp1 = pz[0][2] * pz[0][2] + pz[0][3] * pz[0][3] + pz[1][2] * pz[1][2] +
@@ -606,9 +619,11 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     const float inf = __int_as_float(0x7F800000);
     float b1 = inf, b2 = inf, b3 = inf;
     // Pruning, with lambda a lower bound of the smallest eigenvalue of H_b
-    // (1 for MSE); both bounds are in the objective's units (zl^2 = zscale^2
-    // lambda) and a candidate is skipped only when its bound exceeds the best
-    // objective beyond the tie band, for every row of the warp.
+    // (1 for MSE); both bounds are in the objective's units (zscale^2 lambda
+    // = sl^2 2^2kw, with sl = sigma sqrt(lambda) <= 2^17 and the values scaled
+    // by 2^kw before squaring) and a candidate is skipped only when its bound
+    // exceeds the best objective beyond the tie band, for every row of the
+    // warp.
     //  - small scales: for s < amax_row / 6 the row's largest value
     //    saturates, |delta| >= amax_row - 6 s, so E >= lambda (amax_row -
     //    6 s)^2, growing as s falls;
@@ -619,8 +634,9 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     // largest amax / 6 downwards, then from there upwards.  Rows past the end
     // and all-zero rows never hold the warp back.
     const float amax_row = __uint_as_float((upper ? am1 : am0) << 16);
-    const float zl = zscale * sqrtf(lambda);
-    const float zl2 = zl * zl;
+    const float sl = sigma * sqrtf(lambda);
+    const float sl2 = sl * sl;
+    const float amax_w = amax_row * wsc, m6w = -6.0f * wsc;
     const float row_floor = kZeroFloor * (upper ? pp1 : pp0);
     const float smax = __uint_as_float(m << 16) * (1.0f / 6.0f);
 
@@ -655,9 +671,10 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         const CandInfo c0 = cand[j];
         if (j < js) {
           // saturation bound at this scale (every later one is smaller)
-          const float d = fmaf(-6.0f, c0.s, amax_row);
+          const float d = fmaf(m6w, c0.s, amax_w);  // (amax_row - 6 s) 2^kw
           const bool done = amax_row == 0.0f ||
-                            (d > 0.0f && zl2 * d * d * (1.0f - 2.0f * kTieBand) > b1 + row_floor);
+                            (d > 0.0f &&
+                             sl2 * d * d * (1.0f - 2.0f * kTieBand) > b1 + row_floor + kAbsBand);
           if (__all_sync(0xFFFFFFFFu, done)) break;
         }
         const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
@@ -672,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         float ug = 0.0f, ug8 = 0.0f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float v = a[e] <= q4 ? a[e] : 0.0f;
+          const float v = (a[e] <= q4 ? a[e] : 0.0f) * wsc;
           if ((e & 2) == 0) ug = fmaf(v, v, ug);
           else ug8 = fmaf(v, v, ug8);
         }
@@ -681,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         zero_sum += __shfl_xor_sync(0xFFFFFFFFu, upper ? ug : ug8, 2);
         zero_sum += __shfl_xor_sync(0xFFFFFFFFu, zero_sum, 1);
         const bool done = amax_row == 0.0f ||
-                          zl2 * zero_sum * (1.0f - 2.0f * kTieBand) > b1 + row_floor;
+                          sl2 * zero_sum * (1.0f - 2.0f * kTieBand) > b1 + row_floor + kAbsBand;
         if (__all_sync(0xFFFFFFFFu, done)) break;
         const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
         track3(key_of(e0, c0.c), b1, b2, b3);
@@ -697,15 +714,15 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     const int64_t r = row_base + (upper ? i1 : i0);
     const bool owner = (t & 1) == 0 && (upper ? v1 : v0);
     int code = code_of(b1);
-    float obj = b1 / (zscale * zscale);
+    float obj = ldexpf(b1, -2 * zexp);
     int need = 0;  // 1: re-score the best two, 2: re-score every candidate
     if (owner) {
       const float fl = kZeroFloor * (upper ? pp1 : pp0);
       if (amax_row == 0.0f) {  // all-zero row: every candidate scores exactly 0
         code = 1;
         obj = 0.0f;
-      } else if (b2 - b1 <= kTieBand * b2 || b1 <= fl) {
-        need = (b3 - b1 > kTieBand * b3 + fl) ? 1 : 2;
+      } else if (b2 - b1 <= kTieBand * b2 + kAbsBand || b1 <= fl) {
+        need = (b3 - b1 > kTieBand * b3 + fl + kAbsBand) ? 1 : 2;
       }
     }
     for (uint32_t pend = __ballot_sync(0xFFFFFFFFu, need != 0); pend; pend &= pend - 1) {

@@ -637,3 +637,46 @@ def test_calibration_w4a4_full_size(nv):
     e_p, e_max = nv.quant_error(X, s_p).item(), nv.quant_error(X, s_max).item()
     assert math.isclose(e_p, oracle.quant_error(xu, s_p.item()), rel_tol=1e-9)
     assert math.isclose(e_max, oracle.quant_error(xu, s_max.item()), rel_tol=1e-9)
+
+
+# ------------------------------------------- tiny and huge tensor scales
+@pytest.mark.parametrize("e", [-56, -62, -66, -70, 70, 100])
+def test_extreme_tensor_scales_every_rule(nv, e):
+    """Weights scaled by 2^e (tensor scale near 2^(e-9), between 2^-100 and
+    2^100).  Tiny: Four Over Six's fp32 block MSEs are subnormal, where the
+    screen's absolute margin hands the close calls to the exact fp64 path,
+    and unscaled search objectives and bounds would underflow or overflow.
+    Huge: unscaled MSE objectives would overflow fp32.  Every rule, pack,
+    dequant and fake-quant equal the oracle."""
+    W = (rand_bf16((70, 128), 60 - e, 1.0).float() * 2.0 ** e).to(torch.bfloat16)
+    X = rand_bf16((200, 128), 41, 1.0, 0.01, 20.0)
+    wu = bf16_bits(W)
+    Wd = W.cuda()
+    s_g = nv.global_scale(Wd)
+    sg = s_g.item()
+    assert sg == oracle.global_scale(wu) and 2.0 ** -100 <= sg < 2.0 ** 100
+    cmax = oracle.scale_search_max(wu, sg)
+    np.testing.assert_array_equal(nv.scale_search_max(Wd, s_g).cpu().numpy(), cmax)
+    np.testing.assert_array_equal(nv.scale_search_four_over_six(Wd, s_g).cpu().numpy(),
+                                  oracle.scale_search_four_over_six(wu, sg))
+    rc, _ = oracle.scale_search_mse(wu, sg)
+    n_tie = check_search_codes(nv.scale_search_mse(Wd, s_g).cpu().numpy(), rc, wu, sg)
+    H = torch.zeros(W.shape[1] // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate(X.cuda(), H)
+    H64 = H.cpu().numpy().astype(np.float64)
+    rc, _ = oracle.scale_search_lh(wu, sg, H64)
+    n_tie += check_search_codes(nv.scale_search_local_hessian(Wd, s_g, H).cpu().numpy(), rc,
+                                wu, sg, H64)
+    assert n_tie < 10
+    packed = nv.quantize_pack(Wd, s_g, torch.from_numpy(cmax).cuda())
+    ref_p = oracle.quantize_pack(wu, sg, cmax)
+    np.testing.assert_array_equal(packed.cpu().numpy(), ref_p)
+    y = nv.dequantize(packed, torch.from_numpy(cmax).cuda(), s_g)
+    np.testing.assert_array_equal(bf16_bits(y), oracle.dequantize(ref_p, cmax, sg))
+    yf, pf, cf, sf = nv.fake_quant(Wd, want_packed=True)
+    ry, rp, rcf, rs = oracle.fake_quant(wu)
+    assert sf.item() == rs
+    np.testing.assert_array_equal(cf.cpu().numpy(), rcf)
+    np.testing.assert_array_equal(pf.cpu().numpy(), rp)
+    np.testing.assert_array_equal(bf16_bits(yf), ry)
+    assert nv.get_device_status() == "NVFP4_OK"

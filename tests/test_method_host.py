@@ -100,7 +100,7 @@ def _encode_rule(x, s, step=True):
     t = _f32(xl * r.astype(ld) + _f32(xl * r_lo.astype(ld)).astype(ld))
     if step:
         near = (t.view(np.uint32) & np.uint32(0x1FFFFF)) == 0
-        rho = xl - t.astype(ld) * sl
+        rho = _f32(xl - t.astype(ld) * sl)  # one fma: exact, then one rounding
         up = np.nextafter(t, np.float32(np.inf))
         dn = np.nextafter(t, np.float32(-np.inf))
         t = np.where(near, np.where(rho > 0, up, np.where(rho < 0, dn, t)), t)
@@ -120,12 +120,14 @@ def _oracle_codes(oracle_mod, x, s):
     return np.array([oracle_mod.e2m1_encode(float(a), float(b)) for a, b in zip(x, s)])
 
 
-# power-of-two scales (exact quotients and ties), other round scales, and
-# tensor scales fl32(amax / 2688) times an E4M3 value
+# power-of-two scales (exact quotients and ties), other round scales,
+# tensor scales fl32(amax / 2688) times an E4M3 value, and tiny scales
 ROUND_SCALES = [1.0, 14.0, 2.0 ** -5, 3 * 2.0 ** -7,
                 float(np.float32(84 / 2688)), float(np.float32(97 / 2688)),
                 float(np.float32(np.float32(252 / 2688) * np.float32(1.75))),
-                float(np.float32(np.float32(189 / 2688) * np.float32(1.5)))]
+                float(np.float32(np.float32(189 / 2688) * np.float32(1.5))),
+                # tiny tensor scales, down to the smallest the split reciprocal takes
+                float(np.float32(1.37 * 2.0 ** -90)), float(np.float32(1.0001 * 2.0 ** -100))]
 
 
 @pytest.mark.parametrize("s", ROUND_SCALES + list(
@@ -291,7 +293,7 @@ def _class_codes(a, s_g, o, p, step=True):
     t = _f32(al * ld(r_hi) + _f32(al * ld(r_lo)).astype(ld))
     if step and not _certified(S):
         near = (t.view(np.uint32) & np.uint32(0x1FFFFF)) == 0
-        rho = al - t.astype(ld) * ld(S)
+        rho = _f32(al - t.astype(ld) * ld(S))
         t = np.where(near & (rho > 0), np.nextafter(t, np.float32(np.inf)),
                      np.where(near & (rho < 0), np.nextafter(t, np.float32(0)), t))
     v = np.abs(t.astype(np.float64) * 2.0 ** -p)
@@ -314,7 +316,7 @@ def _candidates():
 @pytest.mark.parametrize("s_g,near_ratio",
                          [(float(np.float32(v / 2688)), False) for v in (1.0, 0.0731, 17.0)]
                          + [(float(np.float32(v)), True) for v in (1 / 3, 1 / 5, 1 / 7, 3 / 7)]
-                         + [(2.0 ** -9, False)])
+                         + [(2.0 ** -9, False), (float(np.float32(1 / 3)) * 2.0 ** -80, True)])
 @pytest.mark.filterwarnings("ignore:overflow encountered in cast")
 def test_search_class_codes_on_every_bf16(oracle_mod, s_g, near_ratio):
     """Every candidate code (126) on every non-negative finite bf16
@@ -419,3 +421,74 @@ def test_pruning_eigenvalue_bound_is_a_lower_bound():
         if d.max() > 0 and lmin_h > 1e-3 * d.max():
             assert lam > 0
     assert nonzero > 150
+
+
+# ------------------------------------------------ Four Over Six fp32 screen
+def _rn32(q):
+    """Round the exact rational q to fp32, nearest-even, subnormals kept."""
+    from fractions import Fraction
+    if q == 0:
+        return Fraction(0)
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    quantum = Fraction(2) ** (max(e, -126) - 23)
+    n = a / quantum
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return (fl * quantum) * (1 if q > 0 else -1)
+
+
+def _mse32(oracle_mod, x, s):
+    """The kernel's fp32 block MSE: d_i = RN(x_i - v_i s), e = RN(d_i^2 + e)
+    in element order, every step rounded once from its exact value."""
+    from fractions import Fraction
+    S = Fraction(float(s))
+    e = Fraction(0)
+    for xi in x:
+        k = oracle_mod.e2m1_encode(float(xi), float(s))
+        v = Fraction(float(GRID[k & 7])) * (-1 if k & 8 else 1)
+        d = _rn32(Fraction(float(xi)) - v * S)
+        e = _rn32(d * d + e)
+    return e
+
+
+def test_four_over_six_screen_with_absolute_floor(oracle_mod):
+    """Blocks at tensor scales from 2^-95 to 2^-55 (the fp32 block MSEs are
+    subnormal there) and at ordinary scales: whenever the fp32 screen decides
+    (|fh - fl| > RN(2^-16 max(fh, fl) + 2^-130)) it picks the oracle's code;
+    without the absolute term it would overrule the oracle on some blocks."""
+    from fractions import Fraction
+    rng = np.random.default_rng(0)
+    wrong_new = wrong_old = decided = 0
+    for trial in range(2400):
+        ordinary = trial % 8 == 0
+        log2s = rng.uniform(-20, 0) if ordinary else rng.uniform(-95, -55)
+        s_g = np.float32(2.0 ** log2s * rng.uniform(1, 2))
+        x = rng.standard_normal(16) * float(s_g) * 2688 * rng.uniform(0.05, 1)
+        blk = bf16_bits(torch.from_numpy(x).float().to(torch.bfloat16))
+        xd = bits_to_f64(blk)
+        amax = float(np.max(np.abs(xd)))
+        c6 = oracle_mod.e4m3_round_quotient(amax, 6.0 * float(s_g))
+        c4 = oracle_mod.e4m3_round_quotient(amax, 4.0 * float(s_g))
+        lo, hi = min(c4, c6), max(c4, c6)
+        if amax == 0 or lo == hi:
+            continue
+        fl = _mse32(oracle_mod, xd, oracle_mod.effective_scale(s_g, lo))
+        fh = _mse32(oracle_mod, xd, oracle_mod.effective_scale(s_g, hi))
+        gap = abs(_rn32(fh - fl))
+        pick = hi if fh < fl else lo
+        ref = oracle_mod.four_over_six_code(blk, float(s_g))
+        if gap > _rn32(Fraction(2) ** -16 * max(fh, fl) + Fraction(2) ** -130):
+            decided += 1
+            wrong_new += pick != ref
+        if gap > _rn32(Fraction(2) ** -16 * max(fh, fl)):
+            wrong_old += pick != ref
+    assert decided > 300
+    assert wrong_new == 0
+    assert wrong_old > 0

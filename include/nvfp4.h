@@ -175,10 +175,9 @@ nvfp4_status nvfp4_scale_search_four_over_six(const uint16_t *w, int64_t batch, 
  * near-ties (best two within 2^-12 relative) are re-scored in fp64.  Range:
  * the screen works on each 16-row tile scaled by a power of two, so tiny and
  * huge weights alike stay in fp32's normal range; the codes follow the
- * definition for tensor scales s_g in [2^-100, 2^100) (tensor maxima from
- * about 2^-88.6 to 2^111.4).  Other s_g take a per-candidate path whose
- * split reciprocals lose precision at the extremes; its result there is not
- * specified.
+ * definition for every tensor scale s_g; outside [2^-100, 2^100) (tensor
+ * maxima below about 2^-88.6 or above 2^111.4) every block is re-scored in
+ * fp64 over all 126 candidates, which is exact but slower.
  *   best_obj     optional [batch, R, C/16] float, the winning objective
  *                (0 or inf where it leaves fp32's range).
  */

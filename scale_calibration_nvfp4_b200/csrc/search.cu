@@ -721,6 +721,11 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       if (amax_row == 0.0f) {  // all-zero row: every candidate scores exactly 0
         code = 1;
         obj = 0.0f;
+      } else if (!by_class) {
+        // s_g outside [2^-100, 2^100): the per-candidate fp32 reciprocals can
+        // leave the normal range, so the screen only orders; every candidate
+        // is re-scored in fp64
+        need = 2;
       } else if (b2 - b1 <= kTieBand * b2 + kAbsBand || b1 <= fl) {
         need = (b3 - b1 > kTieBand * b3 + fl + kAbsBand) ? 1 : 2;
       }

@@ -640,21 +640,24 @@ def test_calibration_w4a4_full_size(nv):
 
 
 # ------------------------------------------- tiny and huge tensor scales
-@pytest.mark.parametrize("e", [-56, -62, -66, -70, 70, 100])
+@pytest.mark.parametrize("e", [-56, -62, -66, -70, -95, 70, 100, 115])
 def test_extreme_tensor_scales_every_rule(nv, e):
-    """Weights scaled by 2^e (tensor scale near 2^(e-9), between 2^-100 and
-    2^100).  Tiny: Four Over Six's fp32 block MSEs are subnormal, where the
-    screen's absolute margin hands the close calls to the exact fp64 path,
-    and unscaled search objectives and bounds would underflow or overflow.
-    Huge: unscaled MSE objectives would overflow fp32.  Every rule, pack,
-    dequant and fake-quant equal the oracle."""
+    """Weights scaled by 2^e (tensor scale near 2^(e-9)).  Tiny: Four Over
+    Six's fp32 block MSEs are subnormal, where the screen's absolute margin
+    hands the close calls to the exact fp64 path, and unscaled search
+    objectives and bounds would underflow or overflow.  Huge: unscaled MSE
+    objectives would overflow fp32.  Beyond [2^-100, 2^100) (e = -95, 115)
+    the searches re-score every candidate in fp64 and the encodes take the
+    exact fp64 path.  Every rule, pack, dequant and fake-quant equal the
+    oracle."""
     W = (rand_bf16((70, 128), 60 - e, 1.0).float() * 2.0 ** e).to(torch.bfloat16)
     X = rand_bf16((200, 128), 41, 1.0, 0.01, 20.0)
     wu = bf16_bits(W)
     Wd = W.cuda()
     s_g = nv.global_scale(Wd)
     sg = s_g.item()
-    assert sg == oracle.global_scale(wu) and 2.0 ** -100 <= sg < 2.0 ** 100
+    assert sg == oracle.global_scale(wu)
+    assert (2.0 ** -100 <= sg < 2.0 ** 100) == (-90 < e < 110)
     cmax = oracle.scale_search_max(wu, sg)
     np.testing.assert_array_equal(nv.scale_search_max(Wd, s_g).cpu().numpy(), cmax)
     np.testing.assert_array_equal(nv.scale_search_four_over_six(Wd, s_g).cpu().numpy(),

@@ -471,6 +471,42 @@ def test_four_over_six_invariants(oracle_mod):
             assert emse[r, b] <= e46 * (1 + 1e-12)
 
 
+@pytest.mark.parametrize("e", [-60, -24, 24, 60])
+def test_every_rule_is_invariant_under_powers_of_two(oracle_mod, e):
+    """Scaling the weights by 2^e scales s_g = fl32(amax / 2688) and every
+    effective scale fl32(s_g e4m3(c)) by exactly 2^e (all stay normal here),
+    every quotient and code is unchanged and every objective scales by
+    2^(2e) exactly (fp64, no rounding moves): so every rule picks the same
+    codes, pack gives the same bytes, and dequant / fake-quant scale by
+    exactly 2^e.  An absolute epsilon or an unscaled tolerance anywhere in
+    the path would break this."""
+    wu, xu = _tiny_layer(24, 96, 64, 12)
+    ws = f32_to_bf16_bits(bits_to_f64(wu) * 2.0 ** e)
+    assert np.array_equal(bits_to_f64(ws), bits_to_f64(wu) * 2.0 ** e)
+    sg, sgs = oracle_mod.global_scale(wu), oracle_mod.global_scale(ws)
+    assert float(sgs) == float(sg) * 2.0 ** e
+    for rule in ("scale_search_max", "scale_search_four_over_six"):
+        assert np.array_equal(getattr(oracle_mod, rule)(ws, sgs), getattr(oracle_mod, rule)(wu, sg))
+    H = oracle_mod.gram(xu)
+    for args in ((), (H,)):
+        f = oracle_mod.scale_search_lh if args else oracle_mod.scale_search_mse
+        c, o = f(wu, sg, *args)
+        cs, os_ = f(ws, sgs, *args)
+        assert np.array_equal(c, cs)
+        assert np.array_equal(os_, o * 2.0 ** (2 * e))
+    codes = oracle_mod.scale_search_max(wu, sg)
+    p, ps = oracle_mod.quantize_pack(wu, sg, codes), oracle_mod.quantize_pack(ws, sgs, codes)
+    assert np.array_equal(p, ps)
+    y, ys = oracle_mod.dequantize(p, codes, sg), oracle_mod.dequantize(ps, codes, sgs)
+    assert np.array_equal(bits_to_f64(ys), bits_to_f64(y) * 2.0 ** e)
+    fy, fp_, fc, fs = oracle_mod.fake_quant(wu)
+    gy, gp, gc, gs = oracle_mod.fake_quant(ws)
+    assert np.array_equal(fc, gc) and np.array_equal(fp_, gp) and float(gs) == float(fs) * 2.0 ** e
+    assert np.array_equal(bits_to_f64(gy), bits_to_f64(fy) * 2.0 ** e)
+    Hf = oracle_mod.gram_full(xu)
+    assert np.array_equal(oracle_mod.gptq(ws, sgs, codes, Hf), oracle_mod.gptq(wu, sg, codes, Hf))
+
+
 # ------------------------------------------------------------ W4A4 GEMM
 def _decode_nvfp4(packed, codes):
     """Exact values of packed NVFP4 rows, decoded without the oracle: the

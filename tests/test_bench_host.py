@@ -1,5 +1,5 @@
-"""Host logic of bench.py (no GPU): the reference arm's JSON line and the
-roofline arithmetic."""
+"""Host logic of bench.py (no GPU): the reference arm's JSON line, the
+roofline arithmetic, the clock record and the traffic lookup."""
 import json
 import os
 import subprocess
@@ -66,3 +66,58 @@ def test_gptq_launch_count_follows_the_panel_schedule():
     # C = 256: + panel solve and next-panel update, a second block, one product
     # C = 384: + one update beyond the next panel, a third panel and block
     assert [bench.gptq_launches(n) for n in (1, 2, 3)] == [4, 9, 15]
+
+
+class _Done:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+    def join(self, timeout=None):
+        pass
+
+
+def test_clock_sampler_reads_nvidia_smi_lines():
+    """The clocks key: median SM clock under load, the largest max clock,
+    and every throttle reason seen Active; short or unparsable lines are
+    skipped."""
+    import bench
+    s = bench.ClockSampler(0)
+    s.proc, s.thread = _Done(), _Done()
+    na = "Not Active"
+    s.lines = [
+        "0, 1965, 1965, 812.3, 0x0, %s, %s, %s, %s" % (na, na, na, na),
+        "0, 1800, 1965, 990.1, 0x4, %s, %s, %s, Active" % (na, na, na),
+        "0, 1890, 1965, 950.0, 0x4, %s, %s, %s, Active" % (na, na, na),
+        "0, [N/A], 1965, 950.0, 0x0, %s, %s, %s, %s" % (na, na, na, na),
+        "garbage",
+        "",
+    ]
+    c = s.stop()
+    assert c == {"sm_mhz": 1890.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                 "samples": 3}
+    s.lines = ["0, 1200, 1965, 400, 0x8, Active, %s, Active, %s" % (na, na)]
+    assert s.stop()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    s.lines = ["nothing usable"]
+    assert s.stop() is None
+
+
+def test_recorded_traffic_needs_the_current_sources(tmp_path, monkeypatch):
+    """ncu traffic is reported only while the kernel's sources hash to the
+    value recorded with it; otherwise (or with no file) it reads null."""
+    import bench
+    f = tmp_path / "traffic.json"
+    f.write_text(json.dumps({
+        "gram": {"dense": {"source_hash": bench.kernel_source_hash("gram"),
+                           "dram_bytes_per_launch": 123456}},
+        "fake_quant": {"w4a4": {"source_hash": "0000000000000000",
+                                "dram_bytes_per_launch": 7}},
+    }))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.recorded_traffic("gram", "dense") == 123456
+    assert bench.recorded_traffic("gram", "moe") is None
+    assert bench.recorded_traffic("fake_quant", "w4a4") is None
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
+    assert bench.recorded_traffic("gram", "dense") is None

@@ -173,8 +173,8 @@ nvfp4_status nvfp4_scale_search_four_over_six(const uint16_t *w, int64_t batch, 
  * 1..126 minimising sum_i (w_i - v(q_i) s_eff)^2, q_i the E2M1 code of w_i at
  * s_eff; the smallest code wins a tie.  Candidates are screened in fp32 and
  * near-ties (best two within 2^-12 relative) are re-scored in fp64.  Range:
- * the screen works on each 16-row tile scaled by a power of two, so tiny and
- * huge weights alike stay in fp32's normal range; the codes follow the
+ * the screen works on each row scaled by a power of two, so tiny and huge
+ * weights alike stay in fp32's normal range; the codes follow the
  * definition for every tensor scale s_g; outside [2^-100, 2^100) (tensor
  * maxima below about 2^-88.6 or above 2^111.4) every block is re-scored in
  * fp64 over all 126 candidates, which is exact but slower.
@@ -193,12 +193,9 @@ nvfp4_status nvfp4_scale_search_mse(const uint16_t *w, int64_t batch, int64_t R,
  * factored once per column block (fp64 Cholesky, semidefinite pivots
  * dropped) and candidates are screened in fp32 as ||L^T delta||^2;
  * near-ties (best two within 2^-12 relative) are re-scored in fp64 from H.
- * Range as nvfp4_scale_search_mse.  One more limit: the tensor-core screen
- * holds each tile's 16 rows in f16 at one common power-of-two scale, so a row
- * whose largest |w| is below about 2^-20 of its tile's largest (rows are
- * sorted by magnitude within each group of 128 or 256 before tiling) is
- * screened with reduced precision (below about 2^-30 its values flush to
- * zero in f16) and may get a different code than the definition's.
+ * Range as nvfp4_scale_search_mse; the tensor-core screen holds each row in
+ * f16 at its own power-of-two scale, so a row keeps full precision whatever
+ * the other rows of its 16-row tile hold.
  *   H            [batch, C/16, 16, 16] float (e.g. from
  *                nvfp4_hessian_accumulate), symmetric positive semidefinite
  *   best_obj     optional [batch, R, C/16] float, the winning objective.

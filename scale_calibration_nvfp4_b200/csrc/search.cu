@@ -65,10 +65,11 @@ constexpr int kTileRows = 16;
 // few CTAs (the tail of the last wave then costs less).
 constexpr int kRowsLarge = kWarps * kTileRows * 4, kRowsSmall = kWarps * kTileRows * 2;
 constexpr float kTieBand = 1.0f / 4096.0f;
-// Absolute part of the band and of the pruning margins: where objectives,
-// terms or bounds fall into the fp32 subnormal range (a row far below its
-// tile's largest), each operation errs by up to 2^-150 and a key moves by up
-// to 127 * 2^-149, far below this; elsewhere it changes nothing.
+// Absolute part of the band and of the pruning margins: where terms or
+// partial sums fall into the fp32 subnormal range (elements far below their
+// row's largest; every row itself is scaled into [2^14, 2^15)), each
+// operation errs by up to 2^-150 and a key moves by up to 127 * 2^-149, far
+// below this; elsewhere it changes nothing.
 constexpr float kAbsBand = 0x1p-130f;
 constexpr float kZeroFloor = 0x1p-40f;  // relative to ||p||^2
 constexpr int kMaxClasses = kCandidates;
@@ -307,10 +308,13 @@ __device__ __forceinline__ uint32_t pick4(uint32_t w0, uint32_t w1, uint32_t w2,
 // One candidate: codes, the tensor-core product u, z = p - s u, and the row
 // objective after a quad reduce-scatter (lanes t < 2: row g, t >= 2: row
 // g + 8).  tq holds the class quotients (stepped where a midpoint could
-// occur), f scales them to this candidate exactly.
+// occur), f scales them to this candidate exactly; sm0 and sm1 multiply u in
+// rows g and g + 8 (accumulator elements 0, 1 and 2, 3 of both n-tiles),
+// each row carrying its own power-of-two scale.
 template <bool kLH>
-__device__ __forceinline__ float candidate_objective(const float tq[8], float f, float sm,
-                                                     uint32_t sgn, const uint32_t bh[2][2],
+__device__ __forceinline__ float candidate_objective(const float tq[8], float f, float sm0,
+                                                     float sm1, uint32_t sgn,
+                                                     const uint32_t bh[2][2],
                                                      const uint32_t bl[2][2],
                                                      const float pz[2][4], bool upper) {
   const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -326,10 +330,10 @@ __device__ __forceinline__ float candidate_objective(const float tq[8], float f,
     mma_f16_16816(u0, A, bl[0][0], bl[0][1], u0);
     mma_f16_16816(u1, A, bl[1][0], bl[1][1], u1);
   }
-  const float z00 = fmaf(-sm, u0[0], pz[0][0]), z01 = fmaf(-sm, u0[1], pz[0][1]);
-  const float z02 = fmaf(-sm, u0[2], pz[0][2]), z03 = fmaf(-sm, u0[3], pz[0][3]);
-  const float z10 = fmaf(-sm, u1[0], pz[1][0]), z11 = fmaf(-sm, u1[1], pz[1][1]);
-  const float z12 = fmaf(-sm, u1[2], pz[1][2]), z13 = fmaf(-sm, u1[3], pz[1][3]);
+  const float z00 = fmaf(-sm0, u0[0], pz[0][0]), z01 = fmaf(-sm0, u0[1], pz[0][1]);
+  const float z02 = fmaf(-sm1, u0[2], pz[0][2]), z03 = fmaf(-sm1, u0[3], pz[0][3]);
+  const float z10 = fmaf(-sm0, u1[0], pz[1][0]), z11 = fmaf(-sm0, u1[1], pz[1][1]);
+  const float z12 = fmaf(-sm1, u1[2], pz[1][2]), z13 = fmaf(-sm1, u1[3], pz[1][3]);
   const float e0 = fmaf(z00, z00, fmaf(z01, z01, fmaf(z10, z10, z11 * z11)));
   const float e1 = fmaf(z02, z02, fmaf(z03, z03, fmaf(z12, z12, z13 * z13)));
   // the same sums in the same order on both lanes of a pair
@@ -576,38 +580,44 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     }
     // p = L^T w at the C positions: pz[nt][0..1] row g, n = 8nt + 2t + {0,1};
     // pz[nt][2..3] row g+8, same n.  Local-Hessian: from the tensor cores
-    // with w scaled by 2^kw (exact; the tile maximum lands in [2^14, 2^15) in
-    // f16), so pz and every z below carry the factor sigma_L 2^kw, removed
-    // from the reported objective at the end.  MSE: p = 2^kw w.
+    // with each row's w scaled by its own 2^kw (exact; the row's largest |w|
+    // lands in [2^14, 2^15) in f16, so every row keeps f16's full precision
+    // whatever the other rows of the tile hold), so pz and every z below
+    // carry the factor sigma_L 2^kw of their row, removed from the reported
+    // objective at the end.  MSE: p = 2^kw w.
     float pz[2][4];
-    // Both rules scale w by 2^kw (exact), putting the tile's largest |w| in
-    // [2^14, 2^15): objectives and bounds then stay in the normal fp32 range
-    // for tiny and for huge weights alike (at most 2^127: a tile whose largest
-    // |w| is below 2^-113 lands lower, its bf16 values still exact in f16).
-    // Objectives carry zscale^2 = (sigma 2^kw)^2, kept as its exponent: zscale
-    // itself can pass the fp32 range (sigma <= 2^90 for an fp32 H), and
-    // nothing below multiplies by it.
-    const int kw = m ? min(14 - ((int)(m >> 7) - 127), 127) : 0;
-    const float wsc = ldexpf(1.0f, kw);
-    int zexp = kw;
+    // Both rules scale each row this way: objectives and bounds then stay in
+    // the normal fp32 range for tiny and for huge weights alike (2^kw at most
+    // 2^127: a row whose largest |w| is below 2^-113 lands lower, its bf16
+    // values still exact in f16).  Objectives carry zscale^2 = (sigma 2^kw)^2
+    // of the lane's row, kept as its exponent: zscale itself can pass the
+    // fp32 range (sigma <= 2^90 for an fp32 H), and nothing below multiplies
+    // by it.  Padding and all-zero rows take 2^0.
+    const int kw0 = am0 ? min(14 - ((int)(am0 >> 7) - 127), 127) : 0;
+    const int kw1 = am1 ? min(14 - ((int)(am1 >> 7) - 127), 127) : 0;
+    const float wsc0 = ldexpf(1.0f, kw0), wsc1 = ldexpf(1.0f, kw1);
+    const float wsc = upper ? wsc1 : wsc0;  // the lane's own row
+    int zexp = upper ? kw1 : kw0;
     if (kLH) {
       zexp += (int)((__float_as_uint(sigma) >> 23) & 0xFFu) - 127;
-      uint32_t Aw[4];
+      uint32_t Aw[4];  // pairs 0, 2: row g; 1, 3: row g + 8
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        Aw[i] = pack_half2(__float2half_rn(xs[2 * i] * wsc), __float2half_rn(xs[2 * i + 1] * wsc));
+      for (int i = 0; i < 4; ++i) {
+        const float ws = (i & 1) ? wsc1 : wsc0;
+        Aw[i] = pack_half2(__float2half_rn(xs[2 * i] * ws), __float2half_rn(xs[2 * i + 1] * ws));
+      }
       const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       mma_f16_16816(pz[0], Aw, bh[0][0], bh[0][1], zero4);
       mma_f16_16816(pz[1], Aw, bh[1][0], bh[1][1], zero4);
       mma_f16_16816(pz[0], Aw, bl[0][0], bl[0][1], pz[0]);
       mma_f16_16816(pz[1], Aw, bl[1][0], bl[1][1], pz[1]);
     } else {
-      pz[0][0] = xs[0] * wsc; pz[0][1] = xs[1] * wsc; pz[0][2] = xs[2] * wsc;
-      pz[0][3] = xs[3] * wsc; pz[1][0] = xs[4] * wsc; pz[1][1] = xs[5] * wsc;
-      pz[1][2] = xs[6] * wsc; pz[1][3] = xs[7] * wsc;
+      pz[0][0] = xs[0] * wsc0; pz[0][1] = xs[1] * wsc0; pz[0][2] = xs[2] * wsc1;
+      pz[0][3] = xs[3] * wsc1; pz[1][0] = xs[4] * wsc0; pz[1][1] = xs[5] * wsc0;
+      pz[1][2] = xs[6] * wsc1; pz[1][3] = xs[7] * wsc1;
     }
-    // multiplier of u in z: s 2^kw (for Local-Hessian u carries sigma_L)
-    const float umul = wsc;
+    // multiplier of u in z: s 2^kw of the row (for Local-Hessian u carries
+    // sigma_L), passed per candidate as s * wsc0 and s * wsc1
     float pp0 = pz[0][0] * pz[0][0] + pz[0][1] * pz[0][1] + pz[1][0] * pz[1][0] +
                 pz[1][1] * pz[1][1];
     float pp1 = pz[0][2] * pz[0][2] + pz[0][3] * pz[0][3] + pz[1][2] * pz[1][2] +
@@ -677,7 +687,8 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
                              sl2 * d * d * (1.0f - 2.0f * kTieBand) > b1 + row_floor + kAbsBand);
           if (__all_sync(0xFFFFFFFFu, done)) break;
         }
-        const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
+        const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * wsc0, c0.s * wsc1, sgn, bh,
+                                                  bl, pz, upper);
         track3(key_of(e0, c0.c), b1, b2, b3);
         ++ncand;
       }
@@ -689,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         float ug = 0.0f, ug8 = 0.0f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float v = (a[e] <= q4 ? a[e] : 0.0f) * wsc;
+          const float v = (a[e] <= q4 ? a[e] : 0.0f) * ((e & 2) ? wsc1 : wsc0);
           if ((e & 2) == 0) ug = fmaf(v, v, ug);
           else ug8 = fmaf(v, v, ug8);
         }
@@ -700,7 +711,8 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         const bool done = amax_row == 0.0f ||
                           sl2 * zero_sum * (1.0f - 2.0f * kTieBand) > b1 + row_floor + kAbsBand;
         if (__all_sync(0xFFFFFFFFu, done)) break;
-        const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * umul, sgn, bh, bl, pz, upper);
+        const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * wsc0, c0.s * wsc1, sgn, bh,
+                                                  bl, pz, upper);
         track3(key_of(e0, c0.c), b1, b2, b3);
         ++ncand;
       }

@@ -683,3 +683,31 @@ def test_extreme_tensor_scales_every_rule(nv, e):
     np.testing.assert_array_equal(pf.cpu().numpy(), rp)
     np.testing.assert_array_equal(bf16_bits(yf), ry)
     assert nv.get_device_status() == "NVFP4_OK"
+
+
+def test_rows_far_below_their_tile_every_search(nv):
+    """Rows scaled by 2^-10, 2^-14, 2^-16 (codes down in E4M3's subnormal
+    range) and 2^-40 (every candidate ties at zero) among ordinary rows:
+    sorted by magnitude they share the first 16-row tile with ordinary rows,
+    and each row's own power-of-two scale keeps its f16 operand and fp32
+    objectives at full precision.  MSE and Local-Hessian codes equal the
+    oracle."""
+    W = rand_bf16((70, 128), 77, 0.02).float()
+    for r, e in ((5, -10), (17, -14), (33, -16), (41, -16), (50, -40)):
+        W[r] *= 2.0 ** e
+    W = W.to(torch.bfloat16)
+    X = rand_bf16((300, 128), 78, 1.0, 0.01, 20.0)
+    wu = bf16_bits(W)
+    Wd = W.cuda()
+    s_g = nv.global_scale(Wd)
+    sg = s_g.item()
+    rc, _ = oracle.scale_search_mse(wu, sg)
+    n_tie = check_search_codes(nv.scale_search_mse(Wd, s_g).cpu().numpy(), rc, wu, sg)
+    H = torch.zeros(W.shape[1] // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate(X.cuda(), H)
+    H64 = H.cpu().numpy().astype(np.float64)
+    rc, _ = oracle.scale_search_lh(wu, sg, H64)
+    n_tie += check_search_codes(nv.scale_search_local_hessian(Wd, s_g, H).cpu().numpy(), rc,
+                                wu, sg, H64)
+    assert n_tie < 10
+    assert nv.get_device_status() == "NVFP4_OK"

@@ -230,21 +230,30 @@ __device__ __forceinline__ void fill_scale_table(ScaleEntry *tab, float sg) {
 // candidate of Four Over Six), exact (nearest even, saturating at 448), from
 // D = k s_g (exact in fp64) and R = 1/D split as r_hi + r_lo: t = amax R, the
 // residual amax - t D is exact in one fp64 fma, and the same odd-code rule
-// picks between the two e4m3x2 conversions.
+// picks between the two e4m3x2 conversions.  Where R passes 2^100 (s_g below
+// about 2^-102, tensor maxima below about 2^-91; R itself can pass the fp32
+// range) R 2^-64 is split instead and amax enters as amax 2^64 (exact: amax
+// is at most about 2688 s_g there).
 struct MaxRule {
   double D;
-  float r_hi, r_lo;
+  float r_hi, r_lo, pre;
 };
 __device__ __forceinline__ MaxRule make_max_rule(float s_g, double k = 6.0) {
   MaxRule m;
   m.D = k * (double)s_g;
-  const double R = 1.0 / m.D;
+  double R = 1.0 / m.D;
+  m.pre = 1.0f;
+  if (R > 0x1p100) {
+    R *= 0x1p-64;
+    m.pre = 0x1p64f;
+  }
   m.r_hi = (float)R;
   m.r_lo = (float)(R - (double)m.r_hi);
   return m;
 }
 __device__ __forceinline__ uint32_t max_rule_code_fast(float amax, const MaxRule &m) {
-  const float t = fmaf(amax, m.r_hi, amax * m.r_lo);
+  const float as = amax * m.pre;
+  const float t = fmaf(as, m.r_hi, as * m.r_lo);
   const double rho = fma(-(double)t, m.D, (double)amax);
   const float ta = __int_as_float(__float_as_int(t) + (rho > 0.0 ? 1 : (rho < 0.0 ? -1 : 0)));
   unsigned short pair;

@@ -640,16 +640,17 @@ def test_calibration_w4a4_full_size(nv):
 
 
 # ------------------------------------------- tiny and huge tensor scales
-@pytest.mark.parametrize("e", [-56, -62, -66, -70, -95, 70, 100, 115])
+@pytest.mark.parametrize("e", [-56, -62, -66, -70, -95, -128, 70, 100, 115])
 def test_extreme_tensor_scales_every_rule(nv, e):
     """Weights scaled by 2^e (tensor scale near 2^(e-9)).  Tiny: Four Over
     Six's fp32 block MSEs are subnormal, where the screen's absolute margin
     hands the close calls to the exact fp64 path, and unscaled search
     objectives and bounds would underflow or overflow.  Huge: unscaled MSE
-    objectives would overflow fp32.  Beyond [2^-100, 2^100) (e = -95, 115)
-    the searches re-score every candidate in fp64 and the encodes take the
-    exact fp64 path.  Every rule, pack, dequant and fake-quant equal the
-    oracle."""
+    objectives would overflow fp32.  Beyond [2^-100, 2^100) (e = -95, -128,
+    115) the searches re-score every candidate in fp64 and the encodes take
+    the exact fp64 path; at e = -128 s_g is a subnormal fp32 and the max
+    rule's reciprocal is pre-scaled.  Every rule, pack, dequant and
+    fake-quant equal the oracle."""
     W = (rand_bf16((70, 128), 60 - e, 1.0).float() * 2.0 ** e).to(torch.bfloat16)
     X = rand_bf16((200, 128), 41, 1.0, 0.01, 20.0)
     wu = bf16_bits(W)

@@ -177,18 +177,23 @@ def _e4m3_rn_satfinite(t):
 
 def _max_rule_code(amax, s_g, k):
     """The kernel's E4M3 code of amax / (k s_g): D = k s_g exact in fp64,
-    R = fl64(1/D) split r_hi = fl32(R), r_lo = fl32(R - r_hi);
-    t = fl32(amax r_hi + fl32(amax r_lo)); ta = the float next to t across
-    the quotient (the sign of amax - t D); the code is RN(t) when RN(t) and
+    R = fl64(1/D) (times 2^-64 where R > 2^100, amax then times 2^64) split
+    r_hi = fl32(R), r_lo = fl32(R - r_hi); t = fl32(a r_hi + fl32(a r_lo))
+    with a the (pre-scaled) amax; ta = the float next to t across the
+    quotient (the sign of amax - t D); the code is RN(t) when RN(t) and
     RN(ta) agree or RN(t) is odd, else RN(ta)."""
     ld = np.longdouble
     D = float(k) * float(np.float32(s_g))
     R = 1.0 / D
+    pre = 1.0
+    if R > 2.0 ** 100:
+        R *= 2.0 ** -64
+        pre = 2.0 ** 64
     r_hi = np.float32(R)
     r_lo = np.float32(R - float(r_hi))
-    a = np.asarray(amax, np.float32).astype(ld)
+    a = np.asarray(amax, np.float32).astype(ld) * ld(pre)
     t = _f32(a * ld(r_hi) + _f32(a * ld(r_lo)).astype(ld))
-    rho = a - t.astype(ld) * ld(D)
+    rho = np.asarray(amax, np.float32).astype(ld) - t.astype(ld) * ld(D)
     ta = np.where(rho > 0, np.nextafter(t, np.float32(np.inf)),
                   np.where(rho < 0, np.nextafter(t, np.float32(-np.inf)), t))
     ct, ca = _e4m3_rn_satfinite(t), _e4m3_rn_satfinite(ta)
@@ -197,7 +202,10 @@ def _max_rule_code(amax, s_g, k):
 
 @pytest.mark.parametrize("k", [6, 4])
 @pytest.mark.parametrize("s_g", [float(np.float32(v / 2688)) for v in (1.0, 0.37, 12.5, 3e4)]
-                         + [2.0 ** -7, float(np.float32(1 / 3))])
+                         + [2.0 ** -7, float(np.float32(1 / 3)),
+                            # tiny tensors: the pre-scaled reciprocal, and a
+                            # subnormal fp32 s_g
+                            float(np.float32(1.37 * 2.0 ** -120)), float(np.float32(2.0 ** -140))])
 def test_kernel_scale_code_on_every_bf16_amax(oracle_mod, k, s_g):
     """Every positive finite bf16 amax whose quotient amax / (k s_g) falls in
     [2^-12, 512], so the sweep spans zero, the subnormal codes, every

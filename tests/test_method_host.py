@@ -500,3 +500,75 @@ def test_four_over_six_screen_with_absolute_floor(oracle_mod):
     assert decided > 300
     assert wrong_new == 0
     assert wrong_old > 0
+
+
+# ---------------------------------------- pruning bounds at any magnitude
+def _screen_objectives(w, s_list, sigma, Lf, kw):
+    """Every candidate's screen objective for one row, in the kernel's units:
+    sigma^2 2^(2 kw) delta^T (L L^T) delta with L the fp32 factor (exact
+    fp64 arithmetic on the exact codes; the kernel's fp32 value lies within
+    its band of this)."""
+    Ld = Lf.astype(np.float64)
+    out = []
+    for s in s_list:
+        k = np.array([_round(x, s)[1] & 7 for x in w])
+        v = np.copysign(GRID[k], w) * s
+        z = Ld.T @ (w - v)
+        out.append(float(z @ z) * sigma ** 2 * 4.0 ** kw)
+    return np.array(out)
+
+
+@pytest.mark.parametrize("e", [-128, -70, -35, 0, 60, 115])
+@pytest.mark.filterwarnings("ignore:overflow encountered")
+def test_pruning_bounds_hold_at_any_magnitude(oracle_mod, e):
+    """The search's two pruning bounds in fp32, as the kernel forms them in
+    the row's scaled units (sl = sigma sqrt(lambda), 2^kw putting the row's
+    largest |w| in [2^14, 2^15)): saturation sl^2 ((amax - 6 s) 2^kw)^2 for
+    s < amax / 6 and zero-code sl^2 sum_{|w| <= s/4} (w 2^kw)^2, each times
+    (1 - 2^-11).  For rows of every magnitude from 2^-128 to 2^115 they stay
+    finite and never exceed the candidate's screen objective, for the MSE
+    rule (sigma = lambda = 1) and for Local-Hessian blocks."""
+    rng = np.random.default_rng(1000 + e)
+    band = np.float32(1 - 2.0 ** -11)
+    blocks = _gram_blocks()[::37]
+    checked = 0
+    for i in range(24):
+        x = rng.standard_normal(16) * rng.uniform(0.2, 1.0) * 2.0 ** e
+        w = bits_to_f64(bf16_bits(torch.from_numpy(x).float().to(torch.bfloat16)))
+        if not np.any(w):
+            continue
+        amax = float(np.max(np.abs(w)))
+        s_g = float(np.float32(amax * rng.uniform(1.0, 3.0) / 2688))
+        s_list = [float(np.float32(np.float32(s_g) * np.float32(oracle_mod.e4m3_value(c))))
+                  for c in range(1, 127)]
+        s_list = [s for s in s_list if s > 0]
+        ebits = int(np.frexp(np.float32(amax))[1]) - 1   # amax in [2^ebits, 2^(ebits+1))
+        kw = min(14 - ebits, 127)
+        wsc = np.float32(2.0 ** kw)
+        for H in (None, blocks[i % len(blocks)]):
+            if H is None:
+                sigma, lam, Lf = 1.0, 1.0, np.eye(16, dtype=np.float32)
+            else:
+                Lf = _cholesky16_drop(H)
+                lam = _lambda_bound(Lf)
+                m = float(np.max(np.abs(Lf)))
+                if m == 0 or lam == 0:
+                    continue
+                sigma = 2.0 ** (15 - np.frexp(np.float32(m))[1])
+            sl = np.float32(np.float32(sigma) * np.sqrt(np.float32(lam)))
+            sl2 = np.float32(sl * sl)
+            E = _screen_objectives(w, s_list, sigma, Lf, kw)
+            for s, Ej in zip(s_list, E):
+                if s < amax / 6:
+                    d = _f32(np.longdouble(amax) * np.longdouble(wsc)
+                             - np.longdouble(6.0) * np.longdouble(wsc) * np.longdouble(s))
+                    b = np.float32(np.float32(np.float32(sl2 * d) * d) * band)
+                    assert np.isfinite(b) and b <= Ej * (1 + 2.0 ** -20), (s, b, Ej)
+                zs = np.float32(0)
+                for xv in w:
+                    v = np.float32(abs(xv) * wsc) if abs(xv) <= s / 4 else np.float32(0)
+                    zs = _f32(np.longdouble(v) * np.longdouble(v) + np.longdouble(zs))
+                b = np.float32(np.float32(sl2 * zs) * band)
+                assert np.isfinite(b) and b <= Ej * (1 + 2.0 ** -20), (s, b, Ej)
+                checked += 1
+    assert checked > 2000

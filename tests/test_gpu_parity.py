@@ -712,3 +712,40 @@ def test_rows_far_below_their_tile_every_search(nv):
                                 wu, sg, H64)
     assert n_tie < 10
     assert nv.get_device_status() == "NVFP4_OK"
+
+
+@pytest.mark.parametrize("e", [-40, 37])
+def test_every_rule_is_invariant_under_powers_of_two_on_gpu(nv, e):
+    """W and W 2^e through every rule on the device: s_g scales by 2^e, each
+    row's f16 operand, class quotients and certificates are unchanged, and
+    every fp32 / fp64 value of the screens scales exactly, so the codes are
+    identical bit for bit (near-ties included; no tolerance) and the
+    objectives scale by exactly 2^(2e)."""
+    W = rand_bf16((130, 256), 91, 0.02, 0.01, 30.0)
+    Ws = (W.float() * 2.0 ** e).to(torch.bfloat16)
+    assert torch.equal(Ws.float(), W.float() * 2.0 ** e)
+    X = rand_bf16((300, 256), 92, 1.0, 0.01, 20.0)
+    H = torch.zeros(W.shape[1] // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate(X.cuda(), H)
+    Hf = torch.zeros(256, 256, device="cuda")
+    nv.hessian_full_accumulate(X.cuda(), Hf)
+    out = []
+    for w in (W.cuda(), Ws.cuda()):
+        s_g = nv.global_scale(w)
+        cm, om = nv.scale_search_mse(w, s_g, return_objective=True)
+        cl, ol = nv.scale_search_local_hessian(w, s_g, H, return_objective=True)
+        cmax = nv.scale_search_max(w, s_g)
+        out.append(dict(s_g=s_g.item(), cmax=cmax, cm=cm, om=om, cl=cl, ol=ol,
+                        c46=nv.scale_search_four_over_six(w, s_g),
+                        packed=nv.quantize_pack(w, s_g, cl),
+                        gptq=nv.gptq(w, s_g, cl, Hf, 0.01)))
+    a, b = out
+    assert b["s_g"] == a["s_g"] * 2.0 ** e
+    for k in ("cmax", "cm", "cl", "c46", "packed", "gptq"):
+        assert torch.equal(a[k], b[k]), k
+    for k in ("om", "ol"):
+        ref = a[k].double() * 4.0 ** e
+        ok = (a[k] > 2.0 ** -100) & (a[k] < 2.0 ** 100) & (ref.abs() > 2.0 ** -120)
+        ok &= ref.abs() < 2.0 ** 120
+        assert torch.equal(b[k].double()[ok], ref[ok]), k
+    assert nv.get_device_status() == "NVFP4_OK"

@@ -28,6 +28,17 @@ def test_reference_arm_prints_one_json_line():
     assert d["config"]["workload"] == "tiny"
 
 
+def test_reference_arm_other_ranks_exit_quietly():
+    """Under torchrun only rank 0 runs and prints the reference arm; the
+    other ranks exit 0 without output or work."""
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.strip() == ""
+
+
 def _run(R, C, blocks):
     L = types.SimpleNamespace(R=R, C=C)
     return types.SimpleNamespace(layers=[L], blocks=lambda: blocks)

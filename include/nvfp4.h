@@ -160,9 +160,12 @@ nvfp4_status nvfp4_scale_search_max(const uint16_t *w, int64_t batch, int64_t R,
  * reading: the max-rule code (block amax onto E2M1's 6) and the code of
  * amax_b / (4 * s_g) (block amax onto 4), both rounded as the max rule
  * rounds; the one with the smaller block MSE sum_i (w_i - v(q_i) s_eff)^2
- * wins, the smaller code on a tie; an all-zero block gets code 0.  The two
- * objectives are evaluated in fp64 with the definition's operations in its
- * order, so the choice is exact.  Arguments as nvfp4_scale_search_max.
+ * wins, the smaller code on a tie; an all-zero block gets code 0.  The
+ * choice is the one the two objectives give when evaluated in fp64 with the
+ * definition's operations in its order: an fp32 screen decides only when
+ * they differ by more than its error bound (2^-16 relative plus 2^-130),
+ * otherwise that fp64 comparison decides.  Arguments as
+ * nvfp4_scale_search_max.
  */
 nvfp4_status nvfp4_scale_search_four_over_six(const uint16_t *w, int64_t batch, int64_t R,
                                               int64_t C, const float *s_g, uint8_t *scale_codes,

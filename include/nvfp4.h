@@ -175,7 +175,8 @@ nvfp4_status nvfp4_scale_search_four_over_six(const uint16_t *w, int64_t batch, 
  * MSE rule ([LH] "The NVFP4 structure"): for every block, the code in
  * 1..126 minimising sum_i (w_i - v(q_i) s_eff)^2, q_i the E2M1 code of w_i at
  * s_eff; the smallest code wins a tie.  Candidates are screened in fp32 and
- * near-ties (best two within 2^-12 relative) are re-scored in fp64.  Range:
+ * near-ties (best two within 2^-12 relative plus 2^-130, in the screen's
+ * units) are re-scored in fp64.  Range:
  * the screen works on each row scaled by a power of two, so tiny and huge
  * weights alike stay in fp32's normal range; the codes follow the
  * definition for every tensor scale s_g; outside [2^-100, 2^100) (tensor
@@ -195,7 +196,8 @@ nvfp4_status nvfp4_scale_search_mse(const uint16_t *w, int64_t batch, int64_t R,
  * columns (shared by all rows); the smallest code wins a tie.  H_b is
  * factored once per column block (fp64 Cholesky, semidefinite pivots
  * dropped) and candidates are screened in fp32 as ||L^T delta||^2;
- * near-ties (best two within 2^-12 relative) are re-scored in fp64 from H.
+ * near-ties (best two within 2^-12 relative plus 2^-130) are re-scored in
+ * fp64 from H.
  * Range as nvfp4_scale_search_mse; the tensor-core screen holds each row in
  * f16 at its own power-of-two scale, so a row keeps full precision whatever
  * the other rows of its 16-row tile hold.

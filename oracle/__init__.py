@@ -36,6 +36,7 @@ def lib():
         L.oracle_effective_scale.argtypes = [f32, i32]
         L.oracle_float_to_bf16.restype = ctypes.c_uint16
         L.oracle_float_to_bf16.argtypes = [f32]
+        L.oracle_floats_to_bf16.argtypes = [vp, i64, vp]
         L.oracle_global_scale.argtypes = [vp, i64, vp]
         L.oracle_max_rule_code.argtypes = [vp, f32]
         L.oracle_scale_search_max.argtypes = [vp, i64, i64, f32, vp]
@@ -117,6 +118,14 @@ def effective_scale(s_g, code):
 
 def float_to_bf16(f):
     return lib().oracle_float_to_bf16(float(f))
+
+
+def floats_to_bf16(a):
+    """bf16 bit patterns (uint16) of an fp32 array, rounded by the oracle."""
+    a = np.ascontiguousarray(a, np.float32)
+    out = np.empty(a.shape, np.uint16)
+    lib().oracle_floats_to_bf16(_ptr(a), a.size, _ptr(out))
+    return out
 
 
 # ------------------------------------------------------------ tensor ops

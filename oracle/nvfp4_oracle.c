@@ -104,6 +104,13 @@ uint16_t oracle_float_to_bf16(float f)
     return (uint16_t)(bits >> 16);
 }
 
+/* The same rounding over an array (n values). */
+void oracle_floats_to_bf16(const float *f, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = oracle_float_to_bf16(f[i]);
+}
+
 /* Effective block scale: the FP8 block scale times the FP32 tensor scale,
  * formed as one fp32 multiply ([BT] "Why do we need scales?": NVFP4 has a
  * tensor-level FP32 scale on top of the block scale). */

@@ -327,6 +327,97 @@ def test_pack_nibble_order_and_dequant(oracle_mod):
     np.testing.assert_array_equal(deq.ravel(), vals.astype(np.float64))
 
 
+def _bf16_nearest_even_exact(f32):
+    """bf16 pattern nearest to the finite fp32 value f32, ties to an even bf16
+    mantissa, by exact rational distances to the two bf16 values around it
+    (overflow past the largest finite bf16 goes to infinity, as IEEE rounding
+    does)."""
+    b = int(np.float32(f32).view(np.uint32))
+    sign, mag = b & 0x80000000, b & 0x7FFFFFFF
+    lo = mag & 0xFFFF0000
+    if lo == mag:
+        return (sign | mag) >> 16
+    hi = lo + 0x10000
+
+    def val(bits):
+        if bits >= 0x7F800000:  # one step past the largest finite bf16
+            return Fraction(2) ** 128
+        return Fraction(float(np.uint32(bits).view(np.float32)))
+    x = Fraction(float(np.uint32(mag).view(np.float32)))
+    dl, dh = x - val(lo), val(hi) - x
+    pick = lo if dl < dh else hi if dh < dl else (lo if (lo >> 16) % 2 == 0 else hi)
+    return (sign | min(pick, 0x7F800000)) >> 16
+
+
+def test_bf16_rounding_equals_torch_on_random_patterns(oracle_mod):
+    """fp32 -> bf16 rounding of every dequantised and fake-quantised output:
+    equal to torch's float32 -> bfloat16 conversion (round to nearest even)
+    on 10^7 random bit patterns (every exponent, both signs, subnormals) and
+    on every pattern whose low half is a tie (0x8000) or one step either side
+    of it, for the upper halves 0x0000..0xFFFF; NaN stays NaN."""
+    rng = np.random.default_rng(2024)
+    bits = rng.integers(0, 2 ** 32, 10_000_000, dtype=np.uint64).astype(np.uint32)
+    hi = np.arange(1 << 16, dtype=np.uint32) << 16
+    ties = np.concatenate([hi | 0x8000, hi | 0x7FFF, hi | 0x8001, hi])
+    for b in (bits, ties):
+        f = b.view(np.float32)
+        ours = oracle_mod.floats_to_bf16(f)
+        ref = torch.from_numpy(f.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        nan = np.isnan(f)
+        np.testing.assert_array_equal(ours[~nan], ref[~nan])
+        assert np.all((ours[nan] & 0x7F80) == 0x7F80) and np.all((ours[nan] & 0x7F) != 0)
+
+
+def test_bf16_rounding_exact_rationals_on_edge_patterns(oracle_mod):
+    """The same rounding against the exact nearest-even bf16 (rational
+    arithmetic) on ties of both parities of bit 16, values next to the bf16
+    maximum and to the overflow threshold, the smallest subnormals, signed
+    zeros and random fp32 values; truncation or round-half-up would fail the
+    ties."""
+    rng = np.random.default_rng(7)
+    pats = [0x3F808000, 0x3F818000, 0xBF808000, 0xBF818000,   # ties, even / odd bit 16
+            0x00008000, 0x00018000, 0x80008000, 0x80018000,   # ties among subnormals
+            0x7F7F7FFF, 0x7F7F8000, 0x7F7EFFFF, 0x7F7E8000,   # around the largest finite
+            0xFF7F8000, 0x00000001, 0x80000001, 0x00007FFF,   # overflow, tiny subnormals
+            0x00000000, 0x80000000, 0x3F800000, 0x007F8000]
+    pats += list(rng.integers(0, 0x7F800000, 3000, dtype=np.int64) |
+                 (rng.integers(0, 2, 3000, dtype=np.int64) << 31))
+    f = np.array(pats, np.uint64).astype(np.uint32).view(np.float32)
+    ours = oracle_mod.floats_to_bf16(f)
+    for x, o in zip(f, ours):
+        assert int(o) == _bf16_nearest_even_exact(x), hex(int(np.float32(x).view(np.uint32)))
+    # the two ties round to the even neighbour: down for bit 16 = 0, up for 1
+    assert list(ours[:4]) == [0x3F80, 0x3F82, 0xBF80, 0xBF82]
+    assert ours[9] == 0x7F80 and ours[12] == 0xFF80      # past the overflow threshold
+    assert ours[16] == 0x0000 and ours[17] == 0x8000     # signed zeros kept
+
+
+def test_dequant_of_products_off_the_bf16_grid(oracle_mod):
+    """Dequantisation where v * s_eff is not a bf16 value ([QAD] 3.2, the
+    quantised value times its scale): every magnitude at tensor scales whose
+    fp32 products need rounding to bf16, among them exact ties, against the
+    IEEE fp32 product (numpy) rounded by the exact nearest-even rule."""
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    for sg_bits in (0x3EAAAAAB, 0x3F808000, 0x3F818000, 0x3DCCCCCD, 0x0071C71C, 0x42F6E979):
+        s_g = np.uint32(sg_bits).view(np.float32)
+        for code in (0x38, 0x39, 0x5B, 0x01, 0x7E):
+            s_eff = np.float32(s_g) * np.float32(oracle_mod.e4m3_value(code))
+            assert s_eff == oracle_mod.effective_scale(s_g, code)
+            q = np.arange(16, dtype=np.uint8)                 # every E2M1 code once
+            packed = (q[0::2] | (q[1::2] << 4)).astype(np.uint8).reshape(1, 8)
+            deq = oracle_mod.dequantize(packed, np.array([[code]], np.uint8), s_g).ravel()
+            for k in range(16):
+                v = mags[k & 7] * (np.float32(-1) if k & 8 else np.float32(1))
+                prod = np.float32(v) * np.float32(s_eff)      # one IEEE fp32 multiply
+                assert int(deq[k]) == _bf16_nearest_even_exact(prod), (hex(sg_bits), code, k)
+    # the tie cases of the fp32 -> bf16 step: s_eff = s_g (code 0x38 = 1.0), v = 1
+    for sg_bits, want in ((0x3F808000, 0x3F80), (0x3F818000, 0x3F82)):
+        s_g = np.uint32(sg_bits).view(np.float32)
+        packed = np.array([[0x22] * 8], np.uint8)             # every element v = 1
+        deq = oracle_mod.dequantize(packed, np.array([[0x38]], np.uint8), s_g).ravel()
+        assert np.all(deq == want), hex(sg_bits)
+
+
 def test_quantize_dequantize_idempotent(oracle_mod):
     W, _ = _tiny_layer(16, 64, 1, 19)
     s_g = oracle_mod.global_scale(W)

@@ -69,12 +69,20 @@ typedef enum nvfp4_status {
     NVFP4_ERR_CUDA = 5,            /* a CUDA runtime call or launch failed */
     NVFP4_ERR_NOT_IMPLEMENTED = 6,
     NVFP4_ERR_TOO_LARGE = 7,       /* request beyond a documented maximum */
-    NVFP4_ERR_DEVICE_TIMEOUT = 8,  /* a kernel gave up waiting (one second) for its own
-                                      tile copies; its output was not written
-                                      (device-side report) */
-    NVFP4_ERR_NOT_POSITIVE_DEFINITE = 9 /* a dampened Hessian had a non-positive (or
+    NVFP4_ERR_DEVICE_TIMEOUT = 8,  /* a Gram kernel gave up waiting (one second) for its
+                                      own tile copies (device-side report).  H is left
+                                      as it was by that call, and by every later Gram
+                                      call until nvfp4_get_device_status has read and
+                                      cleared this status */
+    NVFP4_ERR_NOT_POSITIVE_DEFINITE = 9, /* a dampened Hessian had a non-positive (or
                                            non-finite) Cholesky pivot; the GPTQ output
                                            is not usable (device-side report) */
+    NVFP4_ERR_DEVICE_UNDRAINED = 10 /* after such a timeout, copies still in flight did
+                                       not land within ten more seconds and the kernel
+                                       returned anyway: shared memory of its SM may
+                                       still receive them, so results of later kernels
+                                       are not trustworthy; end the process (device-side
+                                       report, as NVFP4_ERR_DEVICE_TIMEOUT otherwise) */
 } nvfp4_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -290,7 +298,8 @@ nvfp4_status nvfp4_quant_error(const uint16_t *x, int64_t rows, int64_t C, const
 /*
  * Reads and clears the device-side status of the current device after
  * synchronising `stream`.  *out is NVFP4_OK, NVFP4_ERR_NONFINITE,
- * NVFP4_ERR_DEVICE_TIMEOUT or NVFP4_ERR_NOT_POSITIVE_DEFINITE.
+ * NVFP4_ERR_DEVICE_TIMEOUT, NVFP4_ERR_DEVICE_UNDRAINED or
+ * NVFP4_ERR_NOT_POSITIVE_DEFINITE.
  */
 nvfp4_status nvfp4_get_device_status(void *stream, nvfp4_status *out);
 
@@ -376,7 +385,8 @@ nvfp4_status nvfp4_search_evaluations(void *stream, int reset, uint64_t *out);
  * mbarrier nothing arrives on.  Its wait gives up after about one second and
  * sets the device status to NVFP4_ERR_DEVICE_TIMEOUT, which the next
  * nvfp4_get_device_status reports; the context stays usable.  No data is
- * touched.
+ * touched, but until that status is read, Gram calls leave H unchanged (as
+ * after a real timeout).
  */
 nvfp4_status nvfp4_self_test_device_timeout(void *stream);
 

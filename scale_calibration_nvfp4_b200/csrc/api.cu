@@ -114,6 +114,7 @@ const char *nvfp4_status_string(nvfp4_status st) {
     case NVFP4_ERR_TOO_LARGE: return "NVFP4_ERR_TOO_LARGE";
     case NVFP4_ERR_DEVICE_TIMEOUT: return "NVFP4_ERR_DEVICE_TIMEOUT";
     case NVFP4_ERR_NOT_POSITIVE_DEFINITE: return "NVFP4_ERR_NOT_POSITIVE_DEFINITE";
+    case NVFP4_ERR_DEVICE_UNDRAINED: return "NVFP4_ERR_DEVICE_UNDRAINED";
   }
   return "NVFP4_ERR_UNKNOWN";
 }

@@ -19,8 +19,13 @@
 //
 // Every wait on an mbarrier is bounded (one second of %globaltimer): on
 // expiry the CTA records NVFP4_ERR_DEVICE_TIMEOUT in this file's device
-// status, waits (bounded again) for its own copies still in flight, writes
-// nothing and returns.
+// status, waits (bounded again, ten seconds in all) for its own copies still
+// in flight, writes nothing and returns.  The reduce kernel adds nothing to H
+// while that status is set, so a Gram call whose CTA gave up leaves H as it
+// was, and so do later Gram calls until the status is read and cleared.  If
+// the copies in flight do not land within the second bound either, the CTA
+// returns anyway and records NVFP4_ERR_DEVICE_UNDRAINED: shared memory of its
+// SM may then still receive those copies.
 #include <algorithm>
 #include <mutex>
 
@@ -32,8 +37,9 @@
 
 namespace nvfp4 {
 
-// Sticky device status of the Gram kernels (NVFP4_OK or
-// NVFP4_ERR_DEVICE_TIMEOUT), read and cleared with the library status.
+// Sticky device status of the Gram kernels (NVFP4_OK,
+// NVFP4_ERR_DEVICE_TIMEOUT or NVFP4_ERR_DEVICE_UNDRAINED, the larger code
+// kept), read and cleared with the library status.
 __device__ int g_gram_status = 0;
 
 namespace {
@@ -49,6 +55,7 @@ constexpr int kGramSmem = kStages * kStageBytes + 1024;  // + alignment slack
 constexpr int64_t kGroupedItemTokens = 2048;  // tokens per work item, grouped form
 constexpr int64_t kMaxTokensPerLaunch = (int64_t)1 << 30;  // tile row coordinates fit int32
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+constexpr unsigned long long kDrainLimitNs = 10000000000ull;  // after a timeout, for all stages
 
 struct ItemRange {
   int64_t group, t_begin, t_end;
@@ -219,11 +226,24 @@ __global__ void __launch_bounds__(kGramThreads)
   }
 
   if (timed_out) {
-    if (threadIdx.x == 0) atomicExch(&g_gram_status, (int)NVFP4_ERR_DEVICE_TIMEOUT);
+    if (threadIdx.x == 0) atomicMax(&g_gram_status, (int)NVFP4_ERR_DEVICE_TIMEOUT);
     // copies still in flight land in this CTA's shared memory: wait for them
-    // (bounded) before leaving
-    for (int u = tile; u < ntiles && u < tile + kStages; ++u)
-      mbar_wait_bounded(bar0 + 8u * (u % kStages), (uint32_t)(u / kStages) & 1u);
+    // before leaving, under one deadline for all stages
+    if (threadIdx.x == 0) {
+      const unsigned long long t0 = global_ns();
+      bool drained = true;
+      for (int u = tile; u < ntiles && u < tile + kStages && drained; ++u) {
+        const uint32_t bar = bar0 + 8u * (u % kStages), par = (uint32_t)(u / kStages) & 1u;
+        while (!mbar_test(bar, par)) {
+          if (global_ns() - t0 > kDrainLimitNs) {
+            drained = false;
+            break;
+          }
+        }
+      }
+      if (!drained) atomicMax(&g_gram_status, (int)NVFP4_ERR_DEVICE_UNDRAINED);
+    }
+    __syncthreads();
     return;
   }
 
@@ -252,16 +272,19 @@ __global__ void wait_timeout_probe_kernel() {
   if (threadIdx.x == 0) mbar_init(b, 1);
   __syncwarp();
   const bool ok = mbar_wait_bounded(b, 0);
-  if (!ok && threadIdx.x == 0) atomicExch(&g_gram_status, (int)NVFP4_ERR_DEVICE_TIMEOUT);
+  if (!ok && threadIdx.x == 0) atomicMax(&g_gram_status, (int)NVFP4_ERR_DEVICE_TIMEOUT);
 }
 
 // H[g][j][e] += sum of the partials of group g's items, in item order.
+// Nothing is added while a timed-out wait is on record (a partial of this
+// call may then be missing, and its slot holds stale data).
 __global__ void gram_reduce_kernel(const float *__restrict__ partial, int64_t nb, int64_t G,
                                    const int64_t *__restrict__ item_start, int64_t n_items_uniform,
                                    float *__restrict__ H) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over G * nb * 256
   const int64_t per_group = nb * 256;
   if (idx >= G * per_group) return;
+  if (*(volatile const int *)&g_gram_status != 0) return;
   const int64_t g = idx / per_group;
   const int64_t je = idx - g * per_group;
   int64_t i0 = 0, i1 = n_items_uniform;
@@ -522,8 +545,10 @@ cudaError_t read_and_clear_gram_status(cudaStream_t st, int *out) {
 // token ranges are used when C is large.  All calls on a device share the
 // array: calls that overlap on the GPU (different streams, or graphs replayed
 // concurrently) race on it and must be serialised by the caller.  Every
-// partial is written before it is read, so nothing needs clearing between
-// calls.  The first call on each device looks up the array's device address
+// partial a call reads it has written first, so nothing needs clearing
+// between calls; the one exception is a call whose CTA gave up waiting for
+// its tile copies, and there the reduce adds nothing to H (see the timeout
+// handling above).  The first call on each device looks up the array's device address
 // (cudaGetSymbolAddress, with that device current) and caches it; make that
 // first call before any stream capture.
 constexpr size_t kNoAllocPartialFloats = (size_t)4 << 20;  // 16 MiB

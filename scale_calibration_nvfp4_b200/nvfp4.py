@@ -19,6 +19,7 @@ STATUS = {
     0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_SHAPE", 3: "NVFP4_ERR_MISALIGNED",
     4: "NVFP4_ERR_NONFINITE", 5: "NVFP4_ERR_CUDA", 6: "NVFP4_ERR_NOT_IMPLEMENTED",
     7: "NVFP4_ERR_TOO_LARGE", 8: "NVFP4_ERR_DEVICE_TIMEOUT", 9: "NVFP4_ERR_NOT_POSITIVE_DEFINITE",
+    10: "NVFP4_ERR_DEVICE_UNDRAINED",
 }
 
 # C entry points and their argument types (mirrors include/nvfp4.h)

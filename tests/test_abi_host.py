@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in range(10):
+    for code in range(11):
         s = L.nvfp4_status_string(code).decode()
         assert s.startswith("NVFP4_")
     assert L.nvfp4_status_string(0).decode() == "NVFP4_OK"

@@ -68,12 +68,23 @@ def test_global_scale_nonfinite_reports(nv):
 
 def test_bounded_wait_reports_timeout_and_context_survives(nv):
     """A wait that nothing completes gives up (about one second), the host
-    reads NVFP4_ERR_DEVICE_TIMEOUT, and the context still runs kernels."""
+    reads NVFP4_ERR_DEVICE_TIMEOUT, and the context still runs kernels.
+    While the timeout is on record, Gram calls (pool and no-alloc forms,
+    plain and grouped) leave H exactly as it was; after the read clears it,
+    they accumulate again."""
     assert nv.get_device_status() == "NVFP4_OK"
+    x = rand_bf16((300, 64), 12)
+    H0 = torch.randn(4, 16, 16, generator=torch.Generator().manual_seed(3)).cuda()
     nv.self_test_device_timeout()
+    H = H0.clone()
+    nv.hessian_accumulate(x.cuda(), H)
+    nv.hessian_accumulate_noalloc(x.cuda(), H)
+    Hg = H0.clone().view(1, 4, 16, 16)
+    nv.hessian_accumulate_grouped(x.cuda(), torch.tensor([0, 300]).cuda(), Hg)
+    torch.cuda.synchronize()
+    assert torch.equal(H, H0) and torch.equal(Hg.view(4, 16, 16), H0)
     assert nv.get_device_status() == "NVFP4_ERR_DEVICE_TIMEOUT"
     assert nv.get_device_status() == "NVFP4_OK"  # cleared by the read
-    x = rand_bf16((300, 64), 12)
     H = torch.zeros(4, 16, 16, device="cuda")
     nv.hessian_accumulate(x.cuda(), H)
     assert rel_frobenius(H.cpu().numpy().astype(np.float64), oracle.gram(bf16_bits(x))) <= GRAM_REL

@@ -68,6 +68,28 @@ def test_noalloc_gram_accumulates_in_place(nv):
     assert rel_frobenius(H.cpu().numpy(), H_ref.cpu().numpy()) <= GRAM_REL
 
 
+def test_noalloc_gram_at_its_channel_limit(nv):
+    # C = 262,144: one token range fills the whole array (every partial slot
+    # in use, the reduce over a single item), twice in a row
+    C = 262144
+    for call, n_tok in enumerate((300, 77)):
+        x = _calib(n_tok, C, 40 + call)
+        xd = x.cuda()
+        H_ref = torch.zeros(C // 16, 16, 16, device="cuda")
+        nv.hessian_accumulate(xd, H_ref)
+        H_na = torch.zeros(C // 16, 16, 16, device="cuda")
+        nv.hessian_accumulate_noalloc(xd, H_na)
+        torch.cuda.synchronize()
+        a, r = H_na.cpu().numpy(), H_ref.cpu().numpy()
+        assert rel_frobenius(a, r) <= GRAM_REL, call
+        err = np.linalg.norm((a - r).reshape(C // 16, -1), axis=1)
+        assert np.all(err <= GRAM_REL * np.linalg.norm(r.reshape(C // 16, -1), axis=1)), call
+        xu = bf16_bits(x)
+        for j in (0, 1, C // 32, C // 16 - 1):
+            ref = oracle.gram(np.ascontiguousarray(xu[:, 16 * j:16 * j + 16]))[0]
+            assert rel_frobenius(a[j], ref) <= GRAM_REL, (call, j)
+
+
 def test_noalloc_gram_rejects_channels_beyond_its_array(nv):
     # checked on the host before anything is launched
     from scale_calibration_nvfp4_b200.nvfp4 import NVFP4Error

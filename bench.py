@@ -1,18 +1,21 @@
 """Benchmark of the NVFP4 calibration path on B200.
 
 One step = one pass of the whole path over one workload's inputs, which are
-resident in HBM when the timed region starts.  Default workload: the dense
-projection (W 4096x4096, X 2048x4096), whose step is
+resident in HBM when the timed region starts.  Default workload: the MoE
+experts (128 experts of 768x2048, 262,144 routed calibration tokens), the
+largest single-GPU configuration by blocks searched, whose step is
 
-    global scale(W) -> Gram(X) -> max rule -> MSE search -> Local-Hessian
-    search -> quantise+pack (Local-Hessian codes) -> dequantise ->
-    W4A4 fake-quant(X)
+    global scale(W, per expert) -> zero H -> grouped Gram(X) ->
+    Local-Hessian search -> quantise+pack -> dequantise
 
-Other workloads (--workload): tiny, moe (128 experts, grouped Gram over 262,144
-routed tokens, per-expert scales, Local-Hessian search, pack, dequantise),
-mlp_pair (up and down projections with the 16 calibration chunks of 65,536
-tokens each kept resident), w4a4 (activation fake-quant of 32768x8192 with
-packed outputs).
+Other workloads (--workload): dense (W 4096x4096, X 2048x4096: global scale,
+Gram, max rule, MSE and Local-Hessian search, pack, dequantise, W4A4
+fake-quant of X), tiny, mlp_pair (up and down projections with the 16
+calibration chunks of 65,536 tokens each kept resident), w4a4 (activation
+fake-quant of 32768x8192 with packed outputs), and the rows beyond the core
+path (four_over_six, w4a4_gemm, act_calib, lh_gptq).  H is zeroed at the start
+of every step (its own row, a memset), so every step's search sees the
+configuration's Gram.
 
 Metric: NVFP4 blocks per second through the step (weight blocks; activation
 blocks for w4a4).  The L2 cache is flushed (a 256 MiB write) before every
@@ -49,8 +52,10 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
-WORKLOAD_NAMES = ["dense", "tiny", "moe", "mlp_pair", "w4a4", "four_over_six", "w4a4_gemm",
+WORKLOAD_NAMES = ["moe", "dense", "tiny", "mlp_pair", "w4a4", "four_over_six", "w4a4_gemm",
                   "act_calib", "lh_gptq"]
+DEFAULT_WORKLOAD = "moe"
+ISSUE_SLOTS_PER_SM = 4  # one warp instruction per clock per SM sub-partition
 FP64_FMA_PER_SM = 64  # B200: 64 fp64 FMA per clock per SM (about 40 TFLOP/s at boost clock)
 GPTQ_DAMP = 0.01
 
@@ -207,6 +212,11 @@ class Runner:
             pre = L.name + "." if len(self.layers) > 1 else ""
             rows.append((pre + "global_scale",
                          lambda L=L: nv.global_scale(L.W, batch=L.B, out=L.s_g), 2 * n_w, 2))
+            if L.X is not None or L.chunks is not None:
+                # a fresh Gram every step (a torch memset, not one of ours)
+                rows.append((pre + "zero_H", lambda L=L: L.H.zero_(), h, 0))
+            if self.gptq:
+                rows.append((pre + "zero_H_full", lambda L=L: L.Hf.zero_(), 4 * L.C * L.C, 0))
             if L.chunks is not None:
                 def gram(L=L):
                     for ch in L.chunks:
@@ -321,11 +331,28 @@ class Runner:
         return t
 
     def results(self):
+        """Every output the step writes: tensor scales, Grams, the codes of
+        every rule, packed and dequantised weights, fake-quant outputs."""
         out = []
         for L in self.layers:
-            out += [L.c_lh if "lh" in self.rules else L.c_46, L.packed]
-        if self.workload in ("w4a4", "act_calib"):
-            out += [self.fq_packed, self.fq_codes]
+            out.append(L.s_g)
+            if L.X is not None or L.chunks is not None:
+                out.append(L.H)
+            if self.gptq:
+                out.append(L.Hf)
+            for rule, t in (("max", L.c_max), ("mse", L.c_mse), ("lh", L.c_lh),
+                            ("four_over_six", L.c_46)):
+                if rule in self.rules:
+                    out.append(t)
+            out += [L.packed, L.deq]
+        if self.fq_input is not None:
+            out.append(self.fq_out)
+            if self.workload != "act_calib":  # there the static scale is calib_sg
+                out.append(self.fq_sg)
+            if self.workload != "dense" and self.workload != "tiny":
+                out += [self.fq_packed, self.fq_codes]  # packed outputs requested there
+        if self.workload == "act_calib":
+            out += [self.hist, self.calib_sg]
         if self.workload == "w4a4_gemm":
             out += [self.gemm_out]
         return out
@@ -413,9 +440,10 @@ def kernel_source_hash(kernel):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel, workload):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current sources of that kernel."""
+def recorded_counters(kernel, workload):
+    """The ncu counters committed for a kernel on a workload (DRAM bytes and
+    warp instructions per call), if they were taken on the current sources
+    of that kernel; else None."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
@@ -424,7 +452,14 @@ def recorded_traffic(kernel, workload):
     ent = t.get(kernel, {}).get(workload)
     if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
-    return ent.get("dram_bytes_per_launch")
+    return ent
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current sources of that kernel."""
+    ent = recorded_counters(kernel, workload)
+    return None if ent is None else ent.get("dram_bytes_per_launch")
 
 
 def dist_env():
@@ -534,9 +569,13 @@ def run_gpu(args):
                        "rows": [r[0] for r in rows],
                        "parallelism": "replicas (one per GPU)" if world > 1 else "single GPU",
                        "cache": "L2 flushed (256 MiB write) before every timed step"},
-            "roofline": make_roofline(run, kernels, pk, pk_kind, args.workload, evals[1]),
+            "roofline": make_roofline(run, kernels, pk, pk_kind, args.workload, evals[1],
+                                      clk["sm_mhz"] if clk else None),
             "search_evaluated_per_block": {"mse": round(evals[0] / blocks, 2),
                                            "local_hessian": round(evals[1] / blocks, 2)},
+            "search_lh_blocks_per_s": search_blocks_per_s(run, kernels),
+            "hbm_rows_GB/s": {k: v["GB/s"] for k, v in kernels.items()
+                              if k.split(".")[-1] in HBM_ROWS},
             "kernels": kernels,
             "gpu_launches": args.steps * run.launches(),
             "clocks": clk,
@@ -550,6 +589,18 @@ def run_gpu(args):
         pg.destroy_process_group()
 
 
+# rows that stream HBM (their GB/s is the figure of merit)
+HBM_ROWS = ("global_scale", "gram", "search_max", "quantize_pack", "dequantize", "fake_quant",
+            "fake_quant_static", "abs_histogram")
+
+
+def search_blocks_per_s(run, kernels):
+    """Blocks per second of the Local-Hessian search call alone (None when
+    the workload has no Local-Hessian search)."""
+    ms = sum(v["ms"] for k, v in kernels.items() if k.endswith("search_lh"))
+    return round(run.blocks() / (ms / 1e3), 1) if ms > 0 else None
+
+
 def gptq_launches(npan):
     """Kernels one GPTQ call launches for npan 128-column panels: lambda and
     the reversed copy; per panel the diagonal block, and (but the last) the
@@ -559,7 +610,7 @@ def gptq_launches(npan):
     return (2 + npan + 2 * max(npan - 1, 0) + max(npan - 2, 0) + npan + max(npan - 1, 0))
 
 
-def make_roofline(run, kernels, pk, pk_kind, workload, lh_evals):
+def make_roofline(run, kernels, pk, pk_kind, workload, lh_evals, sm_mhz_live=None):
     if "gptq" in kernels:
         # fp64 arithmetic of the definition: the column loop's update of the
         # later columns (R C^2 / 2 FMA) and the Cholesky factor (C^3 / 6 FMA)
@@ -578,25 +629,8 @@ def make_roofline(run, kernels, pk, pk_kind, workload, lh_evals):
                 "flop_basis": "R C^2 (column loop) + C^3/3 (Cholesky), R=%d C=%d" % (R, C)}
     lh_rows = [k for k in kernels if k.endswith("search_lh")]
     if lh_rows:
-        lh_ms = sum(kernels[k]["ms"] for k in lh_rows)
-        sm_mhz = float(pk.get("sm_max_mhz", 1965.0))
-        fp32_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
-        # the definition's cost of every candidate the exact pruned walk
-        # evaluates (counted on the device); the skipped ones provably lose
-        achieved = LH_FLOP_PER_EVAL * lh_evals / (lh_ms / 1e3) / 1e12
-        brute = LH_FLOP_PER_EVAL * 126 * run.blocks() / (lh_ms / 1e3) / 1e12
-        return {
-            "kernel": "search_kernel<Local-Hessian>",
-            "bound": "alu", "achieved": round(achieved, 2), "peak": round(fp32_peak, 2),
-            "unit": "TFLOP/s", "frac": round(achieved / fp32_peak, 4),
-            "traffic": recorded_traffic("search_lh", workload),
-            "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 flop x %.0f MHz (%s clocks)"
-                         % (sm_mhz, pk_kind),
-            "flop_basis": "definition delta H_b delta^T, (256 + 16) FMA = 544 flop per "
-                          "(block, candidate) evaluated; evaluations counted on the device",
-            "evaluated_per_block": round(lh_evals / run.blocks(), 2),
-            "all_126_equivalent_TFLOP/s": round(brute, 2),
-        }
+        return search_roofline(run, kernels, lh_rows, pk, pk_kind, workload, lh_evals,
+                               sm_mhz_live)
     if "fake_quant_static" in kernels:
         ms = kernels["abs_histogram"]["ms"] + kernels["fake_quant_static"]["ms"]
         n = run.fq_input.numel()
@@ -641,6 +675,58 @@ def make_roofline(run, kernels, pk, pk_kind, workload, lh_evals):
             "traffic": recorded_traffic("fake_quant", workload),
             "peak_kind": "%s HBM copy bandwidth" % pk_kind,
             "bytes_per_element": FAKE_QUANT_BYTES_PER_ELEM}
+
+
+def search_roofline(run, kernels, lh_rows, pk, pk_kind, workload, lh_evals, sm_mhz_live=None):
+    """Roofline of the Local-Hessian search call (factor_kernel +
+    search_kernel).  The kernel is bound by instruction issue (the candidate
+    walk, the exact encode and the pruning bounds around a 16x16 tensor-core
+    product per candidate), so the roofline is issue slots: one warp
+    instruction per clock on each of the 4 sub-partitions of the 148 SMs, at
+    the SM clock sampled during the timed region.  `achieved` is the warp
+    instructions one call executes (ncu smsp__inst_executed.sum of both
+    kernels, committed with the hash of their sources; the walk is
+    deterministic for given inputs) over the call's live CUDA-event time.
+    Without a counter taken on the current sources, the definition-equivalent
+    arithmetic rate stands in, labelled as such."""
+    lh_ms = sum(kernels[k]["ms"] for k in lh_rows)
+    sm_mhz = float(sm_mhz_live or pk.get("sm_max_mhz", 1965.0))
+    blocks = run.blocks()
+    fp32_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+    definition = {
+        "note": "not a utilisation: the definition's 544 flop (delta H_b delta^T) per "
+                "(block, candidate) over the FP32 CUDA-core peak; the product itself runs "
+                "on the tensor cores and the pruned walk skips candidates that provably lose",
+        "TFLOP/s_on_evaluations_made": round(LH_FLOP_PER_EVAL * lh_evals / (lh_ms / 1e3) / 1e12, 2),
+        "TFLOP/s_all_126_equivalent": round(LH_FLOP_PER_EVAL * 126 * blocks / (lh_ms / 1e3) / 1e12,
+                                            2),
+        "fp32_peak_TFLOP/s": round(fp32_peak, 2),
+    }
+    rec = recorded_counters("search_lh", workload) or {}
+    inst = rec.get("warp_inst_per_launch")
+    out = {"kernel": "factor_kernel + search_kernel<Local-Hessian> (one call)",
+           "bound": "alu", "traffic": rec.get("dram_bytes_per_launch"),
+           "evaluated_per_block": round(lh_evals / blocks, 2),
+           "definition_equivalent": definition}
+    if inst:
+        peak = SM_COUNT * ISSUE_SLOTS_PER_SM * sm_mhz * 1e6 / 1e12
+        achieved = inst / (lh_ms / 1e3) / 1e12
+        out.update({"achieved": round(achieved, 4), "peak": round(peak, 4),
+                    "unit": "Twarp-instructions/s", "frac": round(achieved / peak, 4),
+                    "peak_kind": "derived: 148 SMs x 4 issue slots x %.0f MHz (SM clock %s)"
+                                 % (sm_mhz, "sampled under load" if sm_mhz_live else
+                                    "max, %s" % pk_kind),
+                    "basis": "warp instructions per call from ncu (smsp__inst_executed.sum, "
+                             "current sources) over the live call time",
+                    "warp_inst_per_call": inst, "pipes": rec.get("pipes")})
+    else:
+        out.update({"achieved": definition["TFLOP/s_on_evaluations_made"],
+                    "peak": definition["fp32_peak_TFLOP/s"], "unit": "TFLOP/s",
+                    "frac": round(definition["TFLOP/s_on_evaluations_made"] / fp32_peak, 4),
+                    "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 flop x %.0f MHz" % sm_mhz,
+                    "basis": "definition-equivalent (no instruction count recorded on the "
+                             "current sources): not a utilisation"})
+    return out
 
 
 def run_e2e(run, args, pg, world):
@@ -838,7 +924,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="dense", choices=WORKLOAD_NAMES)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WORKLOAD_NAMES)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

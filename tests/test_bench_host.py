@@ -44,18 +44,44 @@ def _run(R, C, blocks):
     return types.SimpleNamespace(layers=[L], blocks=lambda: blocks)
 
 
-def test_roofline_local_hessian_counts_the_evaluations_made():
+def test_roofline_local_hessian_without_counters_is_labelled_definition_equivalent(
+        tmp_path, monkeypatch):
     import bench
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
     pk = {"sm_max_mhz": 1965.0, "hbm_gbs": 6555.5}
     run = _run(4096, 4096, 1 << 20)
     evals = 30.0 * (1 << 20)
     r = bench.make_roofline(run, {"search_lh": {"ms": 0.5}}, pk, "measured", "dense", evals)
     peak = 148 * 128 * 2 * 1965e6 / 1e12
-    assert r["bound"] == "alu" and r["unit"] == "TFLOP/s"
+    assert r["bound"] == "alu" and r["unit"] == "TFLOP/s" and "not a utilisation" in r["basis"]
     assert abs(r["peak"] - round(peak, 2)) < 1e-9
     assert abs(r["achieved"] - round(544 * evals / 0.5e-3 / 1e12, 2)) < 1e-9
     assert abs(r["frac"] - round(r["achieved"] / r["peak"], 4)) < 2e-4
     assert r["evaluated_per_block"] == 30.0
+    d = r["definition_equivalent"]
+    assert abs(d["TFLOP/s_all_126_equivalent"] - round(544 * 126 * (1 << 20) / 0.5e-3 / 1e12, 2)) < 1e-9
+
+
+def test_roofline_local_hessian_is_issue_slots_from_recorded_instructions(tmp_path, monkeypatch):
+    """With an ncu instruction count taken on the current sources, the
+    search's roofline is warp instructions per call over the live call time
+    against 148 SMs x 4 issue slots at the sampled SM clock."""
+    import bench
+    f = tmp_path / "traffic.json"
+    f.write_text(json.dumps({"search_lh": {"moe": {
+        "source_hash": bench.kernel_source_hash("search_lh"),
+        "dram_bytes_per_launch": 4.5e8, "warp_inst_per_launch": 2.0e9}}}))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    run = _run(768, 2048, 12582912)
+    r = bench.make_roofline(run, {"search_lh": {"ms": 2.5}}, {"sm_max_mhz": 1965.0}, "measured",
+                            "moe", 18.0 * 12582912, sm_mhz_live=1900.0)
+    peak = 148 * 4 * 1900e6 / 1e12
+    assert r["bound"] == "alu" and r["unit"] == "Twarp-instructions/s"
+    assert abs(r["peak"] - round(peak, 4)) < 1e-12
+    assert abs(r["achieved"] - round(2.0e9 / 2.5e-3 / 1e12, 4)) < 1e-12
+    assert abs(r["frac"] - round(r["achieved"] / r["peak"], 4)) < 2e-4
+    assert r["traffic"] == 4.5e8 and r["warp_inst_per_call"] == 2.0e9
+    assert bench.search_blocks_per_s(run, {"search_lh": {"ms": 2.5}}) == round(12582912 / 2.5e-3, 1)
 
 
 def test_roofline_gptq_is_fp64_definition_flops():

@@ -55,8 +55,8 @@ def lib():
         L.oracle_block_lh.restype = f64
         L.oracle_block_lh.argtypes = [vp, f32, i32, vp]
         L.oracle_block_objectives.argtypes = [vp, f32, vp, vp]
-        L.oracle_scale_search_mse.argtypes = [vp, i64, i64, f32, vp, vp]
-        L.oracle_scale_search_lh.argtypes = [vp, i64, i64, f32, vp, vp, vp]
+        L.oracle_scale_search_mse.argtypes = [vp, i64, i64, f32, vp, vp, vp]
+        L.oracle_scale_search_lh.argtypes = [vp, i64, i64, f32, vp, vp, vp, vp]
         L.oracle_scale_search_sampled.argtypes = [vp, i64, f32, vp, vp, vp, i64, vp, vp]
         L.oracle_gram_accumulate.argtypes = [vp, i64, i64, vp]
         L.oracle_gram_accumulate_grouped.argtypes = [vp, vp, i64, i64, vp]
@@ -178,24 +178,29 @@ def gemm_nvfp4(a_packed, a_codes, a_sg, b_packed, b_codes, b_sg):
     return Y, A
 
 
-def scale_search_mse(w_u16, s_g):
+def scale_search_mse(w_u16, s_g, runner_up=False):
+    """(codes, best objectives[, runner-up objectives]) of every block."""
     w = _u16(w_u16)
     R, C = w.shape
     codes = np.zeros((R, C // 16), np.uint8)
     best = np.zeros((R, C // 16), np.float64)
-    _check(lib().oracle_scale_search_mse(_ptr(w), R, C, float(s_g), _ptr(codes), _ptr(best)))
-    return codes, best
+    second = np.zeros((R, C // 16), np.float64) if runner_up else None
+    _check(lib().oracle_scale_search_mse(_ptr(w), R, C, float(s_g), _ptr(codes), _ptr(best),
+                                         _ptr(second)))
+    return (codes, best, second) if runner_up else (codes, best)
 
 
-def scale_search_lh(w_u16, s_g, H):
+def scale_search_lh(w_u16, s_g, H, runner_up=False):
+    """(codes, best objectives[, runner-up objectives]) of every block."""
     w = _u16(w_u16)
     R, C = w.shape
     H = np.ascontiguousarray(H, dtype=np.float64).reshape(C // 16, 16, 16)
     codes = np.zeros((R, C // 16), np.uint8)
     best = np.zeros((R, C // 16), np.float64)
+    second = np.zeros((R, C // 16), np.float64) if runner_up else None
     _check(lib().oracle_scale_search_lh(_ptr(w), R, C, float(s_g), _ptr(H), _ptr(codes),
-                                        _ptr(best)))
-    return codes, best
+                                        _ptr(best), _ptr(second)))
+    return (codes, best, second) if runner_up else (codes, best)
 
 
 def scale_search_sampled(w_u16, s_g, H, rows, blocks):

@@ -269,20 +269,28 @@ double oracle_block_lh(const uint16_t *blk, float s_g, int c, const double *Hb)
 }
 
 /* Exhaustive search over codes 1..126; the first (smallest) code reaching
- * the minimum wins.  Hb == NULL selects the MSE objective. */
-static int search_block(const uint16_t *blk, float s_g, const double *Hb, double *best)
+ * the minimum wins.  Hb == NULL selects the MSE objective.  *second (if not
+ * NULL) receives the smallest objective among the other 125 codes, which
+ * tells a test whether the block is a near tie. */
+static int search_block(const uint16_t *blk, float s_g, const double *Hb, double *best,
+                        double *second)
 {
     int best_c = 1;
-    double best_e = INFINITY;
+    double best_e = INFINITY, second_e = INFINITY;
     for (int c = 1; c <= 126; c++) {
         double e = Hb ? oracle_block_lh(blk, s_g, c, Hb) : oracle_block_mse(blk, s_g, c);
         if (e < best_e) {
+            second_e = best_e;
             best_e = e;
             best_c = c;
+        } else if (e < second_e) {
+            second_e = e;
         }
     }
     if (best)
         *best = best_e;
+    if (second)
+        *second = second_e;
     return best_c;
 }
 
@@ -294,8 +302,9 @@ void oracle_block_objectives(const uint16_t *blk, float s_g, const double *Hb, d
         out126[c - 1] = Hb ? oracle_block_lh(blk, s_g, c, Hb) : oracle_block_mse(blk, s_g, c);
 }
 
+/* second_obj (nullable): the runner-up objective of every block. */
 int oracle_scale_search_mse(const uint16_t *w, int64_t R, int64_t C, float s_g,
-                            uint8_t *codes, double *best_obj)
+                            uint8_t *codes, double *best_obj, double *second_obj)
 {
     if (C % 16)
         return ORACLE_ERR_SHAPE;
@@ -303,17 +312,21 @@ int oracle_scale_search_mse(const uint16_t *w, int64_t R, int64_t C, float s_g,
 #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t r = 0; r < R; r++)
         for (int64_t b = 0; b < nb; b++) {
-            double e;
-            codes[r * nb + b] = (uint8_t)search_block(w + r * C + b * 16, s_g, NULL, &e);
+            double e, e2;
+            codes[r * nb + b] = (uint8_t)search_block(w + r * C + b * 16, s_g, NULL, &e, &e2);
             if (best_obj)
                 best_obj[r * nb + b] = e;
+            if (second_obj)
+                second_obj[r * nb + b] = e2;
         }
     return ORACLE_OK;
 }
 
-/* H: [C/16][16][16] (row-major 16x16 per column block), shared by all rows. */
+/* H: [C/16][16][16] (row-major 16x16 per column block), shared by all rows.
+ * second_obj (nullable): the runner-up objective of every block. */
 int oracle_scale_search_lh(const uint16_t *w, int64_t R, int64_t C, float s_g,
-                           const double *H, uint8_t *codes, double *best_obj)
+                           const double *H, uint8_t *codes, double *best_obj,
+                           double *second_obj)
 {
     if (C % 16)
         return ORACLE_ERR_SHAPE;
@@ -321,10 +334,13 @@ int oracle_scale_search_lh(const uint16_t *w, int64_t R, int64_t C, float s_g,
 #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t r = 0; r < R; r++)
         for (int64_t b = 0; b < nb; b++) {
-            double e;
-            codes[r * nb + b] = (uint8_t)search_block(w + r * C + b * 16, s_g, H + b * 256, &e);
+            double e, e2;
+            codes[r * nb + b] =
+                (uint8_t)search_block(w + r * C + b * 16, s_g, H + b * 256, &e, &e2);
             if (best_obj)
                 best_obj[r * nb + b] = e;
+            if (second_obj)
+                second_obj[r * nb + b] = e2;
         }
     return ORACLE_OK;
 }
@@ -341,7 +357,7 @@ int oracle_scale_search_sampled(const uint16_t *w, int64_t C, float s_g, const d
     for (int64_t i = 0; i < n; i++) {
         double e;
         const double *Hb = H ? H + blocks[i] * 256 : NULL;
-        codes[i] = (uint8_t)search_block(w + rows[i] * C + blocks[i] * 16, s_g, Hb, &e);
+        codes[i] = (uint8_t)search_block(w + rows[i] * C + blocks[i] * 16, s_g, Hb, &e, NULL);
         if (best_obj)
             best_obj[i] = e;
     }

@@ -13,6 +13,25 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+# Per-configuration statistics that parity tests record (near-tie counts,
+# tolerated code differences, Gram errors), printed after the run even under
+# -q, where passing tests' output is captured.
+PARITY_STATS = []
+
+
+def record_stat(config_name, **values):
+    PARITY_STATS.append((config_name, values))
+
+
+def pytest_terminal_summary(terminalreporter):
+    if not PARITY_STATS:
+        return
+    terminalreporter.write_sep("-", "parity statistics per configuration")
+    for name, values in PARITY_STATS:
+        terminalreporter.write_line(
+            "%s: %s" % (name, ", ".join("%s=%s" % kv for kv in values.items())))
+
+
 def bf16_bits(t):
     """uint16 numpy view of a bf16 torch tensor (any device)."""
     import torch

@@ -300,6 +300,27 @@ def test_search_invariants(oracle_mod):
             assert e_lh[c_lh[r, b] - 1] <= e_lh[c_mse[r, b] - 1]
 
 
+def test_runner_up_objective_is_the_second_smallest(oracle_mod):
+    """The searches' runner-up output (used to count near ties) is the second
+    smallest of the block's 126 objectives, ties included."""
+    W, X = _tiny_layer(6, 48, 40, 29)
+    s_g = oracle_mod.global_scale(W)
+    W[0, :16] = 0                          # every candidate scores 0: runner-up 0
+    H = oracle_mod.gram(X)
+    for Hs in (None, H):
+        if Hs is None:
+            c, b, s2 = oracle_mod.scale_search_mse(W, s_g, runner_up=True)
+        else:
+            c, b, s2 = oracle_mod.scale_search_lh(W, s_g, Hs, runner_up=True)
+        for r in range(6):
+            for k in range(3):
+                E = oracle_mod.block_objectives(W[r, 16 * k:16 * k + 16], s_g,
+                                                None if Hs is None else Hs[k])
+                o = np.sort(E)
+                assert b[r, k] == o[0] and s2[r, k] == o[1] and E[c[r, k] - 1] == o[0]
+        assert s2[0, 0] == 0.0 and c[0, 0] == 1
+
+
 def test_zero_block_and_zero_hessian(oracle_mod):
     W = np.zeros((2, 32), np.uint16)
     W[1, 16:] = f32_to_bf16_bits(np.linspace(-1, 1, 16, dtype=np.float32))

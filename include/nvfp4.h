@@ -203,9 +203,13 @@ nvfp4_status nvfp4_scale_search_mse(const uint16_t *w, int64_t batch, int64_t R,
  * delta_i = w_i - v(q_i) s_eff and H_b the 16x16 Gram block of the block's
  * columns (shared by all rows); the smallest code wins a tie.  H_b is
  * factored once per column block (fp64 Cholesky, semidefinite pivots
- * dropped) and candidates are screened in fp32 as ||L^T delta||^2;
- * near-ties (best two within 2^-12 relative plus 2^-130) are re-scored in
- * fp64 from H.
+ * dropped) and candidates are screened in fp32 as ||L^T delta||^2 with the
+ * 16x16 product on the tensor cores; every block whose best two the
+ * screen's error bound cannot separate -- 2^-12 relative plus an absolute
+ * term that grows with ||L^T w|| (the f16 split of L and the MMA's fp32
+ * accumulation, assumed to err by at most 2^-18 of the sum of its addends'
+ * magnitudes; see nvfp4_self_test_mma) and with any dropped pivot -- is
+ * re-scored in fp64 from H, so the codes are the definition's.
  * Range as nvfp4_scale_search_mse; the tensor-core screen holds each row in
  * f16 at its own power-of-two scale, so a row keeps full precision whatever
  * the other rows of its 16-row tile hold.
@@ -389,6 +393,21 @@ nvfp4_status nvfp4_search_evaluations(void *stream, int reset, uint64_t *out);
  * after a real timeout).
  */
 nvfp4_status nvfp4_self_test_device_timeout(void *stream);
+
+/*
+ * Diagnostic of the scale search's error bound (the pages have no
+ * counterpart): runs each tile through the same tensor-core instruction the
+ * Local-Hessian screen uses, a 16x8x16 MMA of f16 operands with fp32
+ * accumulation, so that a test can check on the device the accumulation
+ * error the screen's bound assumes (at most 2^-18 of the sum of the
+ * magnitudes of the products and of c).
+ *   a  [n_tiles, 16, 16] f16 bit patterns (rows m, columns k), 2-byte aligned
+ *   b  [n_tiles, 16, 8] f16 (rows k, columns n), 2-byte aligned
+ *   c  [n_tiles, 16, 8] float, read;  d  [n_tiles, 16, 8] float, written:
+ *      d = a b + c per tile
+ */
+nvfp4_status nvfp4_self_test_mma(const uint16_t *a, const uint16_t *b, const float *c, float *d,
+                                 int64_t n_tiles, void *stream);
 
 /* Releases the library's memory pool on every device it touched.  No call
  * may be in flight. */

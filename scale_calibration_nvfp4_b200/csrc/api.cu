@@ -333,6 +333,15 @@ nvfp4_status nvfp4_self_test_device_timeout(void *stream) {
   return map_cuda(nvfp4::launch_wait_timeout_probe(as_stream(stream)));
 }
 
+nvfp4_status nvfp4_self_test_mma(const uint16_t *a, const uint16_t *b, const float *c, float *d,
+                                 int64_t n_tiles, void *stream) {
+  if (n_tiles < 0 || (n_tiles > 0 && (!a || !b || !c || !d))) return NVFP4_ERR_INVALID_ARG;
+  if (n_tiles > ((int64_t)1 << 31) * 4 - 4) return NVFP4_ERR_TOO_LARGE;
+  if (!aligned(a, 2) || !aligned(b, 2) || !aligned(c, 4) || !aligned(d, 4))
+    return NVFP4_ERR_MISALIGNED;
+  return map_cuda(nvfp4::launch_mma_probe(a, b, c, d, n_tiles, as_stream(stream)));
+}
+
 void nvfp4_shutdown(void) { nvfp4::scratch_release_all(); }
 
 }  // extern "C"

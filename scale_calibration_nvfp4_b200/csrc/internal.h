@@ -29,6 +29,8 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
 // Copies the search's evaluation counters ([0] MSE, [1] Local-Hessian) to
 // the host after the work queued on `st`, optionally zeroing them.
 cudaError_t read_search_evaluations(cudaStream_t st, unsigned long long out[2], bool reset);
+cudaError_t launch_mma_probe(const uint16_t *a, const uint16_t *b, const float *c, float *d,
+                             int64_t n, cudaStream_t st);
 
 // Gram accumulation.  `offsets` == nullptr: one group of n_tok tokens.
 cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, int64_t n_tok,

@@ -39,6 +39,7 @@ SIGNATURES = {
     "nvfp4_get_device_status": [_vp, _vp],
     "nvfp4_search_evaluations": [_vp, ctypes.c_int, _vp],
     "nvfp4_self_test_device_timeout": [_vp],
+    "nvfp4_self_test_mma": [_vp, _vp, _vp, _vp, _i64, _vp],
     "nvfp4_gemm": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
     "nvfp4_abs_histogram": [_vp, _i64, _vp, _vp],
     "nvfp4_static_scale_from_histogram": [_vp, ctypes.c_double, _vp, _vp],
@@ -387,6 +388,20 @@ def self_test_device_timeout(stream=None):
     """Enqueue the diagnostic wait that times out (about one second); the
     next get_device_status() reports NVFP4_ERR_DEVICE_TIMEOUT."""
     _call("nvfp4_self_test_device_timeout", _stream(stream))
+
+
+def self_test_mma(a, b, c, stream=None):
+    """d = a b + c per tile through the screen's tensor-core instruction:
+    a [n, 16, 16] and b [n, 16, 8] float16, c [n, 16, 8] float32 (CUDA)."""
+    _need(a, torch.float16, "a")
+    _need(b, torch.float16, "b")
+    _need(c, torch.float32, "c")
+    n = a.shape[0]
+    if a.shape != (n, 16, 16) or b.shape != (n, 16, 8) or c.shape != (n, 16, 8):
+        raise ValueError("a [n,16,16], b [n,16,8], c [n,16,8]")
+    d = torch.empty_like(c)
+    _call("nvfp4_self_test_mma", _p(a), _p(b), _p(c), _p(d), n, _stream(stream))
+    return d
 
 
 def status_string(code):

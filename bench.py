@@ -835,6 +835,8 @@ def cpu_baseline(run, budget_s=15.0):
                 "sample": "fake-quant of %d of %d token rows (%d blocks)"
                           % (n, X.shape[0], blocks)}
     L = run.layers[0]
+    if L.B > 1 and L.offsets is not None:
+        return _cpu_baseline_experts(run, L, budget_s)
     W = L.W[0]
     R, C = W.shape
     wu_all = _bits(W)
@@ -891,6 +893,42 @@ def cpu_baseline(run, budget_s=15.0):
             "sample": "the step's rows on %d of %d weight rows (%d blocks) of %s with %d "
                       "calibration tokens (the same fraction); blocks/s over the sample"
                       % (rows, R, blocks, L.name, x_rows)}
+
+
+def _cpu_baseline_experts(run, L, budget_s):
+    """Batched experts: the step's rows (tensor scale, Gram of the expert's
+    routed tokens, the search, pack, dequantise) on whole experts 0, 1, ...
+    as many as the budget takes (expert 0 has the most tokens, so the probe
+    on it over-estimates the later ones); blocks/s over the sample."""
+    import oracle
+    off = [int(v) for v in L.offsets.cpu()]
+
+    def inputs(e):
+        return _bits(L.W[e]), _bits(L.X[off[e]:off[e + 1]])
+
+    def experts(data):
+        t0 = time.perf_counter()
+        for wu, xu in data:
+            sg = oracle.global_scale(wu)
+            H = oracle.gram(xu)
+            if "lh" in run.rules:
+                codes, _ = oracle.scale_search_lh(wu, sg, H)
+            else:
+                codes = oracle.scale_search_max(wu, sg)
+            packed = oracle.quantize_pack(wu, sg, codes)
+            oracle.dequantize(packed, codes, sg)
+        return time.perf_counter() - t0
+
+    t1 = experts([inputs(0)])
+    n = int(max(1, min(L.B, budget_s / max(t1, 1e-6))))
+    data = [inputs(e) for e in range(n)]
+    t = experts(data)
+    blocks = n * L.R * L.C // 16
+    tokens = off[n] - off[0]
+    return {"value": round(blocks / t, 2), "unit": UNIT, "cores": oracle.max_threads(),
+            "kind": "oracle", "seconds": round(t, 3),
+            "sample": "the step's rows on experts 0..%d of %d (%d blocks) with their %d routed "
+                      "calibration tokens; blocks/s over the sample" % (n - 1, L.B, blocks, tokens)}
 
 
 def run_reference(args):

@@ -133,11 +133,12 @@ class Runner:
             self.gptq = True
             self.fq_input = None
         elif workload == "four_over_six":
-            # the dense projection's weights under the Four Over Six rule
-            W, _ = wl.layer_inputs("dense", device)
-            self.layers = [Layer("dense", W, None)]
-            self.desc = ("Four Over Six on the dense projection's W 4096x4096: global scale, "
-                         "the rule, pack, dequantise")
+            # the MoE experts' weights (the largest weight tensor of the
+            # workloads, 403 MB) under the Four Over Six rule
+            W, _, _ = wl.moe_inputs(device)
+            self.layers = [Layer("experts", W, None)]
+            self.desc = ("Four Over Six on the MoE experts' weights (128 x 768x2048, per-expert "
+                         "tensor scales): global scale, the rule, pack, dequantise")
             self.rules = ["four_over_six"]
             self.fq_input = None
         elif workload == "moe":
@@ -835,7 +836,7 @@ def cpu_baseline(run, budget_s=15.0):
                 "sample": "fake-quant of %d of %d token rows (%d blocks)"
                           % (n, X.shape[0], blocks)}
     L = run.layers[0]
-    if L.B > 1 and L.offsets is not None:
+    if L.B > 1:
         return _cpu_baseline_experts(run, L, budget_s)
     W = L.W[0]
     R, C = W.shape
@@ -901,18 +902,19 @@ def _cpu_baseline_experts(run, L, budget_s):
     as many as the budget takes (expert 0 has the most tokens, so the probe
     on it over-estimates the later ones); blocks/s over the sample."""
     import oracle
-    off = [int(v) for v in L.offsets.cpu()]
+    off = None if L.offsets is None else [int(v) for v in L.offsets.cpu()]
 
     def inputs(e):
-        return _bits(L.W[e]), _bits(L.X[off[e]:off[e + 1]])
+        return _bits(L.W[e]), None if off is None else _bits(L.X[off[e]:off[e + 1]])
 
     def experts(data):
         t0 = time.perf_counter()
         for wu, xu in data:
             sg = oracle.global_scale(wu)
-            H = oracle.gram(xu)
             if "lh" in run.rules:
-                codes, _ = oracle.scale_search_lh(wu, sg, H)
+                codes, _ = oracle.scale_search_lh(wu, sg, oracle.gram(xu))
+            elif "four_over_six" in run.rules:
+                codes = oracle.scale_search_four_over_six(wu, sg)
             else:
                 codes = oracle.scale_search_max(wu, sg)
             packed = oracle.quantize_pack(wu, sg, codes)
@@ -924,19 +926,18 @@ def _cpu_baseline_experts(run, L, budget_s):
     data = [inputs(e) for e in range(n)]
     t = experts(data)
     blocks = n * L.R * L.C // 16
-    tokens = off[n] - off[0]
+    calib = "" if off is None else " with their %d routed calibration tokens" % (off[n] - off[0])
     return {"value": round(blocks / t, 2), "unit": UNIT, "cores": oracle.max_threads(),
             "kind": "oracle", "seconds": round(t, 3),
-            "sample": "the step's rows on experts 0..%d of %d (%d blocks) with their %d routed "
-                      "calibration tokens; blocks/s over the sample" % (n - 1, L.B, blocks, tokens)}
+            "sample": "the step's rows on experts 0..%d of %d (%d blocks)%s; blocks/s over the "
+                      "sample" % (n - 1, L.B, blocks, calib)}
 
 
 def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
         return
-    small = args.workload in ("tiny", "dense", "w4a4", "four_over_six", "w4a4_gemm", "act_calib",
-                              "lh_gptq")
+    small = args.workload in ("tiny", "dense", "w4a4", "w4a4_gemm", "act_calib", "lh_gptq")
     dev = "cpu" if small or not torch.cuda.is_available() else "cuda"
     run = Runner(args.workload, dev)
     budget = args.cpu_seconds / max(1, args.steps)

@@ -279,7 +279,7 @@ constexpr int kCholThreads = 256;
 constexpr int kSRow = kBig + 1;  // shared-memory row stride (doubles)
 constexpr int kCholSmem = (kBig * kSRow + 4 * kBig) * (int)sizeof(double);  // 136,192 B
 
-__global__ void __launch_bounds__(kCholThreads)
+__global__ void __launch_bounds__(kCholThreads, 1)
     chol_block_kernel(double *A, int64_t C, int64_t P0, int nw, double *Linv) {
   extern __shared__ double csm[];
   double *Lsm = csm;                 // [kBig][kSRow], the factor
@@ -297,7 +297,11 @@ __global__ void __launch_bounds__(kCholThreads)
       const int r = ty + 16 * i, c = tx + 16 * j;
       a[i][j] = (r < nw && c <= r) ? Ab[(int64_t)r * C + c] : 0.0;
     }
-  // ---- factor
+  // ---- factor.  At step k = 16 j0 + kk only rows and columns above k
+  // change: tile rows and columns i, j >= j0 (j0 is a compile-time constant
+  // of each unrolled copy), and within them the zeroed multipliers of rows
+  // and columns <= k leave entries as they are.  Entries above the diagonal
+  // take products too and are never read.
 #pragma unroll
   for (int j0 = 0; j0 < 8; ++j0) {
     for (int kk = 0; kk < 16; ++kk) {
@@ -306,7 +310,7 @@ __global__ void __launch_bounds__(kCholThreads)
       double *col = vec + (k & 1) * kBig;
       if (tx == kk) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = j0; i < 8; ++i) {
           const int r = ty + 16 * i;
           if (r >= k) col[r] = a[i][j0];
         }
@@ -322,18 +326,15 @@ __global__ void __launch_bounds__(kCholThreads)
       const double iv2 = iv * iv;
       double cr[8], cc[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = j0; i < 8; ++i) {
         const int r = ty + 16 * i, c = tx + 16 * i;
         cr[i] = r > k && r < nw ? col[r] * iv2 : 0.0;
         cc[i] = c > k && c < nw ? col[c] : 0.0;
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = j0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int r = ty + 16 * i, c = tx + 16 * j;
-          if (c > k && c <= r) a[i][j] = fma(-cr[i], cc[j], a[i][j]);
-        }
+        for (int j = j0; j < 8; ++j) a[i][j] = fma(-cr[i], cc[j], a[i][j]);
     }
   }
   __syncthreads();
@@ -357,6 +358,8 @@ __global__ void __launch_bounds__(kCholThreads)
 #pragma unroll
     for (int j = 0; j < 8; ++j) a[i][j] = (ty + 16 * i == tx + 16 * j) ? 1.0 : 0.0;
   __syncthreads();
+  // At step k = 16 i0 + kk only rows below k (tile rows i >= i0) take
+  // X_rc -= L_rk X_kc, and only in columns c <= k (tile columns j <= i0).
 #pragma unroll
   for (int i0 = 0; i0 < 8; ++i0) {
     for (int kk = 0; kk < 16; ++kk) {
@@ -366,7 +369,7 @@ __global__ void __launch_bounds__(kCholThreads)
       if (ty == kk) {
         const double d = dinv[k];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j <= i0; ++j) {
           const int c = tx + 16 * j;
           if (c <= k) {
             a[i0][j] *= d;
@@ -377,19 +380,19 @@ __global__ void __launch_bounds__(kCholThreads)
       __syncthreads();
       double xr[8], lr[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j <= i0; ++j) {
         const int c = tx + 16 * j;
         xr[j] = c <= k ? row[c] : 0.0;
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = i0; i < 8; ++i) {
         const int r = ty + 16 * i;
         lr[i] = r > k && r < nw ? Lsm[r * kSRow + k] : 0.0;
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = i0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) a[i][j] = fma(-lr[i], xr[j], a[i][j]);
+        for (int j = 0; j <= i0; ++j) a[i][j] = fma(-lr[i], xr[j], a[i][j]);
     }
   }
 #pragma unroll

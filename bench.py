@@ -536,7 +536,9 @@ def run_gpu(args):
     if pg:
         pg.barrier()
     clk = clocks.stop() if clocks else None
-    # (block, candidate) evaluations the searches made per step
+    # rows sent to the fp64 re-score, and (block, candidate) evaluations the
+    # searches made, per step (the second read resets both)
+    rescores = [v / args.steps for v in nvfp4.search_rescores()]
     evals = [v / args.steps for v in nvfp4.search_evaluations(reset=True)]
 
     per_row = {r[0]: [] for r in rows}
@@ -574,6 +576,11 @@ def run_gpu(args):
                                       clk["sm_mhz"] if clk else None),
             "search_evaluated_per_block": {"mse": round(evals[0] / blocks, 2),
                                            "local_hessian": round(evals[1] / blocks, 2)},
+            "search_rescored_per_block": {
+                "mse_best_two": round(rescores[0] / blocks, 5),
+                "mse_all_126": round(rescores[1] / blocks, 6),
+                "local_hessian_best_two": round(rescores[2] / blocks, 5),
+                "local_hessian_all_126": round(rescores[3] / blocks, 6)},
             "search_lh_blocks_per_s": search_blocks_per_s(run, kernels),
             "hbm_rows_GB/s": {k: v["GB/s"] for k, v in kernels.items()
                               if k.split(".")[-1] in HBM_ROWS},

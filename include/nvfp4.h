@@ -378,10 +378,22 @@ nvfp4_status nvfp4_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
  * reset (the fp64 re-scores of near ties are not counted); between 1 and 126
  * per block searched.  Synchronises `stream` first, so calls queued on it
  * are included; calls still running on other streams may be partly
- * included.  `reset` != 0 zeroes both counters afterwards.
+ * included.  `reset` != 0 zeroes every search statistic afterwards (these
+ * counters and those of nvfp4_search_rescores).
  *   out   [2] uint64, HOST, written
  */
 nvfp4_status nvfp4_search_evaluations(void *stream, int reset, uint64_t *out);
+
+/*
+ * Second statistic of the scale searches (no counterpart on the pages): how
+ * many rows the fp32 screen could not decide and sent to the fp64 re-score,
+ * since the last reset, on the current device: out[0] MSE rows re-scored over
+ * their best two candidates, out[1] MSE rows re-scored over all 126, out[2]
+ * and out[3] the same for nvfp4_scale_search_local_hessian.  Synchronises
+ * `stream` first; `reset` != 0 zeroes every search statistic afterwards.
+ *   out   [4] uint64, HOST, written
+ */
+nvfp4_status nvfp4_search_rescores(void *stream, int reset, uint64_t *out);
 
 /*
  * Diagnostic of the failure path of the kernels that wait on their own tile

@@ -302,11 +302,20 @@ nvfp4_status nvfp4_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
 
 nvfp4_status nvfp4_search_evaluations(void *stream, int reset, uint64_t *out) {
   if (!out) return NVFP4_ERR_INVALID_ARG;
-  unsigned long long v[2] = {0, 0};
+  unsigned long long v[6] = {0, 0, 0, 0, 0, 0};
   cudaError_t e = nvfp4::read_search_evaluations(as_stream(stream), v, reset != 0);
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   out[0] = v[0];
   out[1] = v[1];
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_search_rescores(void *stream, int reset, uint64_t *out) {
+  if (!out) return NVFP4_ERR_INVALID_ARG;
+  unsigned long long v[6] = {0, 0, 0, 0, 0, 0};
+  cudaError_t e = nvfp4::read_search_evaluations(as_stream(stream), v, reset != 0);
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  for (int i = 0; i < 4; ++i) out[i] = v[2 + i];
   return NVFP4_OK;
 }
 

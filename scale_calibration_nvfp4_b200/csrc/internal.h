@@ -28,7 +28,8 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
 
 // Copies the search's evaluation counters ([0] MSE, [1] Local-Hessian) to
 // the host after the work queued on `st`, optionally zeroing them.
-cudaError_t read_search_evaluations(cudaStream_t st, unsigned long long out[2], bool reset);
+// all six search statistics (see g_search_evals in search.cu)
+cudaError_t read_search_evaluations(cudaStream_t st, unsigned long long out[6], bool reset);
 cudaError_t launch_mma_probe(const uint16_t *a, const uint16_t *b, const float *c, float *d,
                              int64_t n, cudaStream_t st);
 

@@ -72,10 +72,12 @@
 
 namespace nvfp4 {
 
-// (block, candidate) objective evaluations of the fp32 screen since the last
-// reset: [0] MSE, [1] Local-Hessian.  A statistic of the work the pruned walk
-// does; nothing reads it on the device.
-__device__ unsigned long long g_search_evals[2];
+// Statistics of the work the searches do since the last reset; nothing reads
+// them on the device.  [0] MSE and [1] Local-Hessian (block, candidate)
+// objective evaluations of the fp32 screen; rows re-scored in fp64 over their
+// best two candidates ([2] MSE, [4] Local-Hessian) and over all 126 ([3] MSE,
+// [5] Local-Hessian).
+__device__ unsigned long long g_search_evals[6];
 
 namespace {
 
@@ -158,78 +160,80 @@ __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
   return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
 }
 
+// The factor kernel works on two 16x16 blocks per warp: the lanes of each
+// half (16 lanes) own one row each of their block, and every shuffle and
+// reduction below stays inside the half.
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
 // Cooperative Cholesky of the 16x16 block in Hs (fp32, row-major) by one
-// warp, lanes 0..15 owning one row each.  A pivot at or below 1e-12 of the
-// largest diagonal (or non-finite) drops its column, which keeps a positive
+// half-warp, lane r owning row r.  A pivot at or below 1e-12 of the largest
+// diagonal (or non-finite) drops its column, which keeps a positive
 // semidefinite H usable.  Writes the full lower-triangular factor (zeros above
 // the diagonal) to Lf (fp32) and Ld (fp64).
 __device__ void cholesky16(const float *Hs, float *Lf, double *Ld) {
-  const int lane = threadIdx.x & 31;
-  const bool own = lane < 16;
+  const int r = threadIdx.x & 15;
   double a[16];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) a[j] = own ? (double)Hs[lane * 16 + j] : 0.0;
+  for (int j = 0; j < 16; ++j) a[j] = (double)Hs[r * 16 + j];
   double diag = 0.0;
 #pragma unroll
   for (int j = 0; j < 16; ++j)
-    if (j == lane) diag = a[j];
+    if (j == r) diag = a[j];
   double maxdiag = diag;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1)
-    maxdiag = fmax(maxdiag, __shfl_xor_sync(0xFFFFFFFFu, maxdiag, o));
+  for (int o = 8; o > 0; o >>= 1) maxdiag = fmax(maxdiag, __shfl_xor_sync(kFull, maxdiag, o));
   const double tol = 1e-12 * maxdiag;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
-    const double akk = __shfl_sync(0xFFFFFFFFu, a[k], k);
+    const double akk = __shfl_sync(kFull, a[k], k, 16);
     const bool ok = (akk > tol) && (akk < 1e300);
     const double piv = ok ? sqrt(akk) : 0.0;
     double lik = 0.0;
-    if (lane == k) lik = piv;
-    else if (own && lane > k && ok) lik = a[k] / piv;
-    if (own) {
-      Lf[lane * 16 + k] = (float)lik;  // zero above the diagonal
-      Ld[lane * 16 + k] = lik;
-    }
+    if (r == k) lik = piv;
+    else if (r > k && ok) lik = a[k] / piv;
+    Lf[r * 16 + k] = (float)lik;  // zero above the diagonal
+    Ld[r * 16 + k] = lik;
 #pragma unroll
     for (int j = k + 1; j < 16; ++j) {
-      const double ljk = __shfl_sync(0xFFFFFFFFu, lik, j);
+      const double ljk = __shfl_sync(kFull, lik, j, 16);
       a[j] = fma(-lik, ljk, a[j]);
     }
   }
 }
 
-// Lower bound of the smallest eigenvalue of L L^T, computed by one warp and
-// returned to every lane: 0.98 / ||(L L^T)^-1||_1.  For a symmetric matrix the
-// column-sum norm bounds the 2-norm from above, so this bounds lambda_min from
-// below (with 2% to spare for rounding).  Lane i < 16 forms column i of the
-// inverse by a forward and a backward triangular solve in fp64.  A dropped
-// pivot (zero diagonal in L) makes the matrix singular: the bound is 0 (no
-// pruning).  So it is too when max diag(L L^T) ||(L L^T)^-1||_1 exceeds
-// 10^4: L L^T differs from H by at most 2^-23 trace(H) <= 2^-19 max diag(H)
-// (fp32 rounding of the factor), which then stays below 2% of lambda_min.
-__device__ __forceinline__ float lambda_lower_bound(const float *Lf, double *inv_d) {
-  const int lane = threadIdx.x & 31;
-  // 1 / L_kk and the largest diagonal entry of L L^T (lane k < 16: row k)
+// Lower bound of the smallest eigenvalue of L L^T, computed by one half-warp
+// and returned to each of its lanes: 0.98 / ||(L L^T)^-1||_1.  For a
+// symmetric matrix the column-sum norm bounds the 2-norm from above, so this
+// bounds lambda_min from below (with 2% to spare for rounding).  Lane r forms
+// column r of the inverse by a forward and a backward triangular solve in
+// fp64.  A dropped pivot (zero diagonal in L) makes the matrix singular: the
+// bound is 0 (no pruning).  So it is too when max diag(L L^T)
+// ||(L L^T)^-1||_1 exceeds 10^4: L L^T differs from H by at most 2^-23
+// trace(H) <= 2^-19 max diag(H) (fp32 rounding of the factor), which then
+// stays below 2% of lambda_min.  The same sweeps give the diagonal of the
+// inverse: cdiag[r] = 0.97 / ((L L^T)^-1)_rr (0 where lambda is), a lower
+// bound of min { x^T H x : x_r = 1 } = 1 / (H^-1)_rr under the same
+// condition (the diagonal entry moves by at most 1.9% relative).
+__device__ __forceinline__ float lambda_lower_bound(const float *Lf, double *inv_d,
+                                                   float *cdiag) {
+  const int lane = threadIdx.x & 31, r = lane & 15;
+  // 1 / L_kk and the largest diagonal entry of L L^T (lane r: row r)
   double maxdiag = 0.0;
-  int singular = 0;
-  if (lane < 16) {
-    const double d = (double)Lf[lane * 16 + lane];
-    singular = d == 0.0;
-    inv_d[lane] = 1.0 / d;
+  const double d = (double)Lf[r * 16 + r];
+  inv_d[r] = 1.0 / d;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) maxdiag = fma((double)Lf[lane * 16 + m], (double)Lf[lane * 16 + m], maxdiag);
-  }
-  singular = __any_sync(0xFFFFFFFFu, singular);
+  for (int m = 0; m < 16; ++m) maxdiag = fma((double)Lf[r * 16 + m], (double)Lf[r * 16 + m], maxdiag);
+  const bool singular = (__ballot_sync(kFull, d == 0.0) >> (lane & 16)) & 0xFFFFu;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) maxdiag = fmax(maxdiag, __shfl_xor_sync(0xFFFFFFFFu, maxdiag, o));
+  for (int o = 8; o > 0; o >>= 1) maxdiag = fmax(maxdiag, __shfl_xor_sync(kFull, maxdiag, o));
   __syncwarp();
-  double colsum = 0.0;
-  if (lane < 16 && !singular) {
-    // column sweeps: acc = e_lane, then L y = acc, then L^T z = y (in place;
+  double colsum = 0.0, dinv = 0.0;
+  if (!singular) {
+    // column sweeps: acc = e_r, then L y = acc, then L^T z = y (in place;
     // outer loops rolled, acc in local memory: once per block of H)
     double acc[16];
 #pragma unroll
-    for (int m = 0; m < 16; ++m) acc[m] = (m == lane) ? 1.0 : 0.0;
+    for (int m = 0; m < 16; ++m) acc[m] = (m == r) ? 1.0 : 0.0;
 #pragma unroll 1
     for (int k = 0; k < 16; ++k) {
       acc[k] *= inv_d[k];
@@ -243,11 +247,13 @@ __device__ __forceinline__ float lambda_lower_bound(const float *Lf, double *inv
 #pragma unroll
       for (int m = 0; m < k; ++m) acc[m] = fma(-(double)Lf[k * 16 + m], acc[k], acc[m]);
     }
+    dinv = acc[r];  // ((L L^T)^-1)_rr
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) colsum = fmax(colsum, __shfl_xor_sync(0xFFFFFFFFu, colsum, o));
-  if (singular || !(colsum > 0.0) || !(colsum < 1e300) || maxdiag * colsum > 1e4) return 0.0f;
-  return (float)(0.98 / colsum);
+  for (int o = 8; o > 0; o >>= 1) colsum = fmax(colsum, __shfl_xor_sync(kFull, colsum, o));
+  const bool valid = !singular && colsum > 0.0 && colsum < 1e300 && maxdiag * colsum <= 1e4;
+  cdiag[r] = valid && dinv > 0.0 ? (float)(0.97 / dinv) : 0.0f;
+  return valid ? (float)(0.98 / colsum) : 0.0f;
 }
 
 // fp64 objective of one candidate from the definition, computed by a
@@ -382,82 +388,97 @@ struct Factor {
   float lambda;  // lower bound of lambda_min(L L^T), 0 when unknown
   int zero;      // H_b == 0 (every candidate scores 0)
   float rho;     // sigma^2 ||H - L L^T||_inf (fp64 factor; dropped pivots), inf if unknown
+  float cdiag[16];  // lower bounds of 1 / (H^-1)_rr (0 when lambda is 0)
 };
 
-// ||H - Ld Ld^T||_inf by one warp (lanes < 16 sum one row each), plus
-// 2^-40 max diag(H) for the rounding of the fp64 factor and of this sum;
-// every lane returns it.  Zero unless pivots were dropped (up to rounding).
+// ||H - Ld Ld^T||_inf by one half-warp (lane r sums row r), plus 2^-40 max
+// diag(H) for the rounding of the fp64 factor and of this sum; each lane of
+// the half returns it.  Zero unless pivots were dropped (up to rounding).
 __device__ __forceinline__ double factor_residual(const float *Hs, const double *Ld) {
-  const int lane = threadIdx.x & 31;
-  double rs = 0.0, dg = 0.0;
-  if (lane < 16) {
-    dg = (double)Hs[lane * 16 + lane];
+  const int r = threadIdx.x & 15;
+  double rs = 0.0, dg = (double)Hs[r * 16 + r];
 #pragma unroll 1
-    for (int j = 0; j < 16; ++j) {
-      double r = (double)Hs[lane * 16 + j];
+  for (int j = 0; j < 16; ++j) {
+    double x = (double)Hs[r * 16 + j];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) r = fma(-Ld[lane * 16 + k], Ld[j * 16 + k], r);
-      rs += fabs(r);
-    }
+    for (int k = 0; k < 16; ++k) x = fma(-Ld[r * 16 + k], Ld[j * 16 + k], x);
+    rs += fabs(x);
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    rs = fmax(rs, __shfl_xor_sync(0xFFFFFFFFu, rs, o));
-    dg = fmax(dg, __shfl_xor_sync(0xFFFFFFFFu, dg, o));
+  for (int o = 8; o > 0; o >>= 1) {
+    rs = fmax(rs, __shfl_xor_sync(kFull, rs, o));
+    dg = fmax(dg, __shfl_xor_sync(kFull, dg, o));
   }
   return rs + 0x1p-40 * dg;
 }
 
+// Two column blocks of H per warp (half h of the lanes takes block 2 x + h of
+// batch element y; an odd last block leaves half 1 with zeros and nothing to
+// write).
 __global__ void __launch_bounds__(32)
-    factor_kernel(const float *__restrict__ H, uint4 *__restrict__ frag,
+    factor_kernel(const float *__restrict__ H, int64_t nb, uint4 *__restrict__ frag,
                   Factor *__restrict__ fac) {
-  __shared__ float Hs[256];
-  __shared__ float Lf[256];
-  __shared__ double Ld[256];
-  __shared__ double inv_d[16];
-  const int lane = threadIdx.x;
-  const int64_t blk = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;  // one warp per block of H
-  const float *Hb = H + blk * 256;
-  for (int i = lane; i < 256; i += 32) Hs[i] = Hb[i];
+  __shared__ float Hs[2][256];
+  __shared__ float Lf[2][256];
+  __shared__ double Ld[2][256];
+  __shared__ double inv_d[2][16];
+  __shared__ float cdiag[2][16];
+  const int lane = threadIdx.x, h = lane >> 4, r = lane & 15;
+  const int64_t j0 = (int64_t)blockIdx.x * 2;
+  const int64_t base = (int64_t)blockIdx.y * nb;  // first block of this batch element
+  const bool live = j0 + h < nb;
+  const float *Hb = H + (base + j0 + h) * 256;
+  for (int i = r; i < 256; i += 16) Hs[h][i] = live ? Hb[i] : 0.0f;
   __syncwarp();
-  cholesky16(Hs, Lf, Ld);
+  cholesky16(Hs[h], Lf[h], Ld[h]);
   __syncwarp();
-  const double resid = factor_residual(Hs, Ld);
+  const double resid = factor_residual(Hs[h], Ld[h]);
   float m = 0.0f;
-  for (int i = lane; i < 256; i += 32) m = fmaxf(m, fabsf(Lf[i]));
+  for (int i = r; i < 256; i += 16) m = fmaxf(m, fabsf(Lf[h][i]));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  const float lam = lambda_lower_bound(Lf, inv_d);
+  for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+  const float lam = lambda_lower_bound(Lf[h], inv_d[h], cdiag[h]);
+  __syncwarp();  // cdiag written by every lane of the half
   int e = 0;
   frexpf(m, &e);  // m < 2^e
   const float sigma = m > 0.0f ? ldexpf(1.0f, 15 - e) : 1.0f;
-  // this lane's fragments: B[k][n] = sigma L[k][n], n = 8 nt + g, k = 2t + 8 half + {0, 1}
-  const int g = lane >> 2, t = lane & 3;
-  uint32_t hi[4], lo[4];
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    const int n = nt * 8 + g;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int k0 = 2 * t + 8 * half;
-      const float x0 = Lf[k0 * 16 + n] * sigma, x1 = Lf[(k0 + 1) * 16 + n] * sigma;
-      const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
-      const __half l0 = __float2half_rn(x0 - __half2float(h0));
-      const __half l1 = __float2half_rn(x1 - __half2float(h1));
-      hi[nt * 2 + half] = pack_half2(h0, h1);
-      lo[nt * 2 + half] = pack_half2(l0, l1);
-    }
-  }
-  frag[(blk * 32 + lane) * 2] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-  frag[(blk * 32 + lane) * 2 + 1] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-  if (lane == 0) {
+  if (live && r == 0) {
     Factor f;
     f.sigma = sigma;
     f.lambda = lam;
     f.zero = !(m > 0.0f);
     const double rho = resid * (double)sigma * (double)sigma;  // below 2^40: no overflow
     f.rho = rho < 3.0e38 ? (float)rho : __int_as_float(0x7F800000);  // NaN -> inf too
-    fac[blk] = f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) f.cdiag[i] = cdiag[h][i];
+    fac[base + j0 + h] = f;
+  }
+  // every lane's fragments of both blocks: B[k][n] = sigma L[k][n], n = 8 nt
+  // + g, k = 2t + 8 half + {0, 1}
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int hb = 0; hb < 2; ++hb) {
+    const float sg = __shfl_sync(kFull, sigma, 16 * hb);
+    if (j0 + hb >= nb) break;
+    const float *L = Lf[hb];
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int n = nt * 8 + g;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int k0 = 2 * t + 8 * half;
+        const float x0 = L[k0 * 16 + n] * sg, x1 = L[(k0 + 1) * 16 + n] * sg;
+        const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+        const __half l0 = __float2half_rn(x0 - __half2float(h0));
+        const __half l1 = __float2half_rn(x1 - __half2float(h1));
+        hi[nt * 2 + half] = pack_half2(h0, h1);
+        lo[nt * 2 + half] = pack_half2(l0, l1);
+      }
+    }
+    const int64_t blk = base + j0 + hb;
+    frag[(blk * 32 + lane) * 2] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    frag[(blk * 32 + lane) * 2 + 1] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
 }
 
@@ -481,6 +502,8 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
 
   __shared__ ClassInfo cls[kMaxClasses];
   __shared__ CandInfo cand[kCandidates];
+  __shared__ float cdiag_sh[16];  // bounds of 1 / (H^-1)_rr of this column block
+  __shared__ float Hsh[kLH ? 256 : 1];  // H_b, for the fp64 re-scores
   __shared__ int ncls_sh;
   __shared__ uint4 Ws[kRowsPerCta][2];     // the CTA's 16-element row segments
   __shared__ uint32_t keys[kRowsPerCta];  // amax << 16 | local row, sorted
@@ -509,10 +532,13 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     sigma = f.sigma;
     lambda = f.lambda;
     rho = f.rho;
+    if (threadIdx.x < 16) cdiag_sh[threadIdx.x] = fac[blk].cdiag[threadIdx.x];
+    for (int i = threadIdx.x; i < 256; i += kThreads) Hsh[i] = Hb[i];
     const uint4 h = frag[(blk * 32 + lane) * 2], l = frag[(blk * 32 + lane) * 2 + 1];
     bh[0][0] = h.x; bh[0][1] = h.y; bh[1][0] = h.z; bh[1][1] = h.w;
     bl[0][0] = l.x; bl[0][1] = l.y; bl[1][0] = l.z; bl[1][1] = l.w;
   } else {
+    if (threadIdx.x < 16) cdiag_sh[threadIdx.x] = 1.0f;  // H = I
     // B = I: u = v exactly
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -598,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     }
   }
 
-  unsigned long long evals = 0;
+  unsigned long long evals = 0, rescored1 = 0, rescored2 = 0;
   for (int tile = warp; tile < kRowsPerCta / kTileRows; tile += kWarps) {
     const uint32_t kg = keys[tile * kTileRows + g], kg8 = keys[tile * kTileRows + g + 8];
     const bool v0 = (kg >> 16) != 0xFFFFu, v1 = (kg8 >> 16) != 0xFFFFu;
@@ -726,6 +752,28 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     const float amax_row = __uint_as_float((upper ? am1 : am0) << 16);
     const float sl = sigma * sqrtf(lambda);
     const float sl2 = sl * sl;
+    // saturation bound of the lane's row: its largest element (position i)
+    // alone forces E >= |delta_i|^2 / (H^-1)_ii; an element whose magnitude
+    // equals the row's amax, found in the quad (any one of equal maxima)
+    float ss2;
+    {
+      // every lane of the quad holds elements {2t, 2t+1, 2t+8, 2t+9} of both
+      // rows (pairs 0, 2: row g; 1, 3: row g + 8): search both, reduce over
+      // the quad, keep the lane's own row
+      auto find = [&](uint32_t pa, uint32_t pb, uint32_t am) {
+        int i = -1;
+        i = ((pb >> 16) & 0x7FFFu) == am ? 2 * t + 9 : i;
+        i = (pb & 0x7FFFu) == am ? 2 * t + 8 : i;
+        i = ((pa >> 16) & 0x7FFFu) == am ? 2 * t + 1 : i;
+        i = (pa & 0x7FFFu) == am ? 2 * t : i;
+        i = max(i, __shfl_xor_sync(0xFFFFFFFFu, i, 1));
+        return max(i, __shfl_xor_sync(0xFFFFFFFFu, i, 2));
+      };
+      const int i0 = find(pw[0], pw[2], am0), i1 = find(pw[1], pw[3], am1);
+      const int idx = upper ? i1 : i0;
+      const float si = sigma * sqrtf(idx >= 0 ? cdiag_sh[idx] : 0.0f);
+      ss2 = si * si;
+    }
     const float amax_w = amax_row * wsc, m6w = -6.0f * wsc;
     const float row_floor = kZeroFloor * (upper ? pp1 : pp0);
     // a candidate is skipped when its lower bound, less the bound's own
@@ -767,7 +815,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
           // saturation bound at this scale (every later one is smaller)
           const float d = fmaf(m6w, c0.s, amax_w);  // (amax_row - 6 s) 2^kw
           const bool done = amax_row == 0.0f ||
-                            (d > 0.0f && sl2 * d * d * (1.0f - 2.0f * kTieBand) >
+                            (d > 0.0f && ss2 * d * d * (1.0f - 2.0f * kTieBand) >
                                              fmaf(b1, 1.0f + 2.0f * kTieBand, prune_pad));
           if (__all_sync(0xFFFFFFFFu, done)) break;
         }
@@ -834,6 +882,8 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
                                                                                           : 2;
       }
     }
+    rescored1 += __popc(__ballot_sync(0xFFFFFFFFu, need == 1));
+    rescored2 += __popc(__ballot_sync(0xFFFFFFFFu, need == 2));
     for (uint32_t pend = __ballot_sync(0xFFFFFFFFu, need != 0); pend; pend &= pend - 1) {
       const int src = __ffs(pend) - 1;
       const int64_t rr = __shfl_sync(0xFFFFFFFFu, (long long)r, src);
@@ -841,7 +891,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       const int k1 = __shfl_sync(0xFFFFFFFFu, code_of(b1), src);
       const int k2 = __shfl_sync(0xFFFFFFFFu, code_of(b2), src);
       float o;
-      const int c = refine_block(wb + rr * C, s_g, Hb, k1, k2, n == 2, &o);
+      const int c = refine_block(wb + rr * C, s_g, kLH ? Hsh : nullptr, k1, k2, n == 2, &o);
       if (lane == src) {
         code = c;
         obj = o;
@@ -852,7 +902,11 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       if (ob) ob[r * nb] = obj;
     }
   }
-  if (lane == 0 && evals) atomicAdd(&g_search_evals[kLH ? 1 : 0], evals);
+  if (lane == 0) {
+    if (evals) atomicAdd(&g_search_evals[kLH ? 1 : 0], evals);
+    if (rescored1) atomicAdd(&g_search_evals[kLH ? 4 : 2], rescored1);
+    if (rescored2) atomicAdd(&g_search_evals[kLH ? 5 : 3], rescored2);
+  }
 }
 
 // Diagnostic of the screen's error model: tile i of a [n][16][16] (f16,
@@ -893,7 +947,7 @@ cudaError_t launch_mma_probe(const uint16_t *a, const uint16_t *b, const float *
   return cudaGetLastError();
 }
 
-cudaError_t read_search_evaluations(cudaStream_t st, unsigned long long out[2], bool reset) {
+cudaError_t read_search_evaluations(cudaStream_t st, unsigned long long out[6], bool reset) {
   cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_search_evals, sizeof(g_search_evals), 0,
                                             cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess && reset) {
@@ -935,7 +989,8 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
   if (e != cudaSuccess) return e;
   uint4 *frag = static_cast<uint4 *>(scratch);
   Factor *fac = reinterpret_cast<Factor *>(static_cast<char *>(scratch) + frag_bytes);
-  factor_kernel<<<dim3((unsigned)(C / kBlock), (unsigned)batch), 32, 0, st>>>(H, frag, fac);
+  const int64_t nb = C / kBlock;
+  factor_kernel<<<dim3((unsigned)((nb + 1) / 2), (unsigned)batch), 32, 0, st>>>(H, nb, frag, fac);
   e = cudaGetLastError();
   if (e == cudaSuccess) {
     if (small)

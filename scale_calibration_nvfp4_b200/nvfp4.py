@@ -38,6 +38,7 @@ SIGNATURES = {
     "nvfp4_fake_quant": [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp],
     "nvfp4_get_device_status": [_vp, _vp],
     "nvfp4_search_evaluations": [_vp, ctypes.c_int, _vp],
+    "nvfp4_search_rescores": [_vp, ctypes.c_int, _vp],
     "nvfp4_self_test_device_timeout": [_vp],
     "nvfp4_self_test_mma": [_vp, _vp, _vp, _vp, _i64, _vp],
     "nvfp4_gemm": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
@@ -318,6 +319,16 @@ def search_evaluations(reset=False, stream=None):
     out = (ctypes.c_uint64 * 2)()
     _call("nvfp4_search_evaluations", _stream(stream), int(bool(reset)), out)
     return int(out[0]), int(out[1])
+
+
+def search_rescores(reset=False, stream=None):
+    """Rows sent to the fp64 re-score since the last reset: (MSE over the
+    best two, MSE over all 126, Local-Hessian over the best two, Local-Hessian
+    over all 126); synchronises the stream.  A reset zeroes every search
+    statistic, the evaluation counts included."""
+    out = (ctypes.c_uint64 * 4)()
+    _call("nvfp4_search_rescores", _stream(stream), int(bool(reset)), out)
+    return tuple(int(v) for v in out)
 
 
 def gemm(a_packed, a_codes, a_sg, b_packed, b_codes, b_sg, out=None, stream=None):

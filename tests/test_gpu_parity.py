@@ -437,9 +437,13 @@ def test_search_evaluation_counters(nv):
     assert blocks <= m <= 126 * blocks and l == 0
     nv.scale_search_local_hessian(W, s_g, H)
     nv.scale_search_local_hessian(W, s_g, H)
+    r = nv.search_rescores()
     m2, l2 = nv.search_evaluations(reset=True)
     assert m2 == m and 2 * blocks <= l2 <= 2 * 126 * blocks and l2 % 2 == 0
-    assert nv.search_evaluations() == (0, 0)
+    assert nv.search_evaluations() == (0, 0) and nv.search_rescores() == (0, 0, 0, 0)
+    # re-scored rows: at most every block once per call; the tiny layer has
+    # near ties under both rules
+    assert 0 < r[0] + r[1] <= blocks and 0 < r[2] + r[3] <= 2 * blocks and r[2] % 2 == 0
 
 
 def test_four_over_six_dense_layer_every_block(nv):

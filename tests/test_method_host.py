@@ -380,6 +380,16 @@ def _lambda_bound(Lf):
     return float(np.float32(0.98 / colsum))
 
 
+def _cdiag_bound(Lf):
+    """The kernel's per-channel bounds 0.97 / ((L L^T)^-1)_rr (fp32 factor,
+    fp64 solves), all 0 where the eigenvalue bound is 0."""
+    if _lambda_bound(Lf) == 0.0:
+        return np.zeros(Lf.shape[0])
+    L = Lf.astype(np.float64)
+    Linv = np.linalg.solve(L, np.eye(L.shape[0]))
+    return (0.97 / np.diag(Linv.T @ Linv)).astype(np.float32).astype(np.float64)
+
+
 def _gram_blocks():
     """16x16 fp32 Gram blocks of bf16 calibration tokens: token counts from
     1 to 2048, outlier channels up to 100x, zero and duplicated channels,
@@ -421,6 +431,13 @@ def test_pruning_eigenvalue_bound_is_a_lower_bound():
         lmin_llt = np.linalg.eigvalsh(Ld @ Ld.T)[0]
         lmin_h = np.linalg.eigvalsh(H.astype(np.float64))[0]
         assert lam >= 0.0
+        # the per-channel saturation bounds: at most 1 / (A^-1)_rr for A = L L^T
+        # and for H (the least x^T A x with x_r = 1), and never below lambda
+        cd = _cdiag_bound(Lf)
+        if lam > 0:
+            for A in (Ld @ Ld.T, H.astype(np.float64)):
+                assert np.all(cd <= 1.0 / np.diag(np.linalg.inv(A))), (cd, lam)
+            assert np.all(cd >= lam * (1 - 1e-6))
         if lam > 0:
             nonzero += 1
             assert lam <= lmin_llt and lam <= lmin_h, (lam, lmin_llt, lmin_h)
@@ -523,8 +540,9 @@ def _screen_objectives(w, s_list, sigma, Lf, kw):
 def test_pruning_bounds_hold_at_any_magnitude(oracle_mod, e):
     """The search's two pruning bounds in fp32, as the kernel forms them in
     the row's scaled units (sl = sigma sqrt(lambda), 2^kw putting the row's
-    largest |w| in [2^14, 2^15)): saturation sl^2 ((amax - 6 s) 2^kw)^2 for
-    s < amax / 6 and zero-code sl^2 sum_{|w| <= s/4} (w 2^kw)^2, each times
+    largest |w| in [2^14, 2^15)): saturation si^2 ((amax - 6 s) 2^kw)^2 for
+    s < amax / 6, si = sigma sqrt(cdiag_i) at the row's largest element i,
+    and zero-code sl^2 sum_{|w| <= s/4} (w 2^kw)^2, each times
     (1 - 2^-11).  For rows of every magnitude from 2^-128 to 2^115 they stay
     finite and never exceed the candidate's screen objective, for the MSE
     rule (sigma = lambda = 1) and for Local-Hessian blocks."""
@@ -557,12 +575,15 @@ def test_pruning_bounds_hold_at_any_magnitude(oracle_mod, e):
                 sigma = 2.0 ** (15 - np.frexp(np.float32(m))[1])
             sl = np.float32(np.float32(sigma) * np.sqrt(np.float32(lam)))
             sl2 = np.float32(sl * sl)
+            cd = 1.0 if H is None else _cdiag_bound(Lf)[int(np.argmax(np.abs(w)))]
+            si = np.float32(np.float32(sigma) * np.sqrt(np.float32(cd)))
+            ss2 = np.float32(si * si)
             E = _screen_objectives(w, s_list, sigma, Lf, kw)
             for s, Ej in zip(s_list, E):
                 if s < amax / 6:
                     d = _f32(np.longdouble(amax) * np.longdouble(wsc)
                              - np.longdouble(6.0) * np.longdouble(wsc) * np.longdouble(s))
-                    b = np.float32(np.float32(np.float32(sl2 * d) * d) * band)
+                    b = np.float32(np.float32(np.float32(ss2 * d) * d) * band)
                     assert np.isfinite(b) and b <= Ej * (1 + 2.0 ** -20), (s, b, Ej)
                 zs = np.float32(0)
                 for xv in w:
@@ -671,8 +692,9 @@ def _screen(w, s_g, H, rng, q_on=True, favour=None, kappa=KAPPA):
         need = 1 if b3 - b1 > t3 else 2
     lam = _lambda_bound(Lf)
     pad = np.float32(np.float32(4102 * q) * q + np.float32(fl + ABS_BAND))
+    cd = _cdiag_bound(Lf)[int(np.argmax(np.abs(w)))]   # the row's largest element
     return dict(keys=keys, need=need, sigma=float(sigma), kw=kw, wsc=wsc, lam=lam, pad=pad,
-                svals=svals, amax=amax)
+                svals=svals, amax=amax, cd=cd)
 
 
 def _e4m3(c):
@@ -774,12 +796,14 @@ def _screen_violations(oracle_mod, q_on, n_rows=700, seed=5, adversarial=False, 
         if sc["lam"] > 0:
             sl = np.float32(np.float32(sc["sigma"]) * np.sqrt(np.float32(sc["lam"])))
             sl2 = np.float32(sl * sl)
+            si = np.float32(np.float32(sc["sigma"]) * np.sqrt(np.float32(sc["cd"])))
+            ss2 = np.float32(si * si)
             for c in range(1, 127):
                 s = sc["svals"][c - 1]
                 bounds = []
                 if s < sc["amax"] / 6:
                     d = np.float32(sc["amax"] * sc["wsc"] - 6.0 * sc["wsc"] * s)
-                    bounds.append(np.float32(sl2 * d * d * np.float32(1 - 2 * BAND)))
+                    bounds.append(np.float32(ss2 * d * d * np.float32(1 - 2 * BAND)))
                 zs = np.float32(np.sum((np.abs(w[np.abs(w) <= s / 4]) * sc["wsc"]) ** 2))
                 bounds.append(np.float32(sl2 * zs * np.float32(1 - 2 * BAND)))
                 lb = max(bounds)

@@ -51,14 +51,37 @@ def _shared_inputs():
     return files
 
 
+# The CUTLASS release the two template sources (gemm_fp4.cu, gram_full.cu) were
+# written and tested against; the header tree is taken from the environment,
+# so its version is checked rather than assumed.
+CUTLASS_VERSION = (4, 5, 0)
+
+
+def cutlass_version(include_dir):
+    """(major, minor, patch) from cutlass/version.h under include_dir."""
+    v = {}
+    with open(os.path.join(include_dir, "cutlass", "version.h")) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and parts[0] == "#define" and parts[1] in (
+                    "CUTLASS_MAJOR", "CUTLASS_MINOR", "CUTLASS_PATCH"):
+                v[parts[1]] = int(parts[2])
+    return v.get("CUTLASS_MAJOR"), v.get("CUTLASS_MINOR"), v.get("CUTLASS_PATCH")
+
+
 def cutlass_include():
-    """CUTLASS/CuTe headers vendored with flashinfer (header-only use)."""
+    """CUTLASS/CuTe headers vendored with flashinfer (header-only use), of
+    the release CUTLASS_VERSION names."""
     import importlib.util
     spec = importlib.util.find_spec("flashinfer")
     for base in (spec.submodule_search_locations or []) if spec else []:
         inc = os.path.join(base, "data", "cutlass", "include")
         util = os.path.join(base, "data", "cutlass", "tools", "util", "include")
         if os.path.isdir(os.path.join(inc, "cute")):
+            found = cutlass_version(inc)
+            if found != CUTLASS_VERSION:
+                raise RuntimeError("CUTLASS headers at %s are version %s; this library's "
+                                   "template sources need %s" % (inc, found, CUTLASS_VERSION))
             return [inc, util]
     raise RuntimeError("CUTLASS/CuTe headers not found (expected under flashinfer/data/cutlass)")
 

@@ -328,12 +328,15 @@ __device__ __forceinline__ float block_mse32(const uint32_t w[8], uint2 q, float
   return e;
 }
 
-// The same fp32 block MSE at a table entry's scale, straight from the
-// values: each pair is rounded (the encode above, one conversion) and its
-// byte decoded by the hardware e2m1x2 -> f16x2 conversion in the same asm
-// block, then d_i = x_i - v_i s and e += d_i^2 in block_mse32's order, so
-// the result equals block_mse32 of the packed codes bit for bit, without
-// packing them.
+// The fp32 block MSE at a table entry's scale, straight from the values:
+// each pair is rounded from t (one conversion) and its byte decoded by the
+// hardware e2m1x2 -> f16x2 conversion in the same asm block, then d_i = x_i -
+// v_i s and e += d_i^2 in block_mse32's order.  The codes are those of t, not
+// always of the exact quotient q: where t is a rounding midpoint and q lies
+// off it (t within one float of q), t may round to the other neighbour, and
+// then |d_i| moves by at most 2 ulp(t) s, i.e. d_i^2 by at most 2^-20 of
+// itself -- inside the screen's 2^-16 threshold; the exact comparison below
+// uses exact codes.
 __device__ __forceinline__ uint32_t e2m1x2_round_decode(float hi, float lo) {
   uint32_t h2;
   asm("{\n\t.reg .b8 q;\n\t"
@@ -349,14 +352,7 @@ __device__ __forceinline__ float block_mse32_entry(const uint32_t w[8], const Sc
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const float x0 = bf16_lo(w[j]), x1 = bf16_hi(w[j]);
-    float t0 = fmaf(x0, e.r_hi, x0 * e.r_lo), t1 = fmaf(x1, e.r_hi, x1 * e.r_lo);
-    const bool n0 = (__float_as_uint(t0) & 0x1FFFFFu) == 0u;
-    const bool n1 = (__float_as_uint(t1) & 0x1FFFFFu) == 0u;
-    if (n0 || n1) {
-      const float a0 = toward(t0, fmaf(-t0, e.s, x0)), a1 = toward(t1, fmaf(-t1, e.s, x1));
-      t0 = n0 ? a0 : t0;
-      t1 = n1 ? a1 : t1;
-    }
+    const float t0 = fmaf(x0, e.r_hi, x0 * e.r_lo), t1 = fmaf(x1, e.r_hi, x1 * e.r_lo);
     const uint32_t h2 = e2m1x2_round_decode(t1, t0);
     const float d0 = fmaf(-f16_lo_to_float(h2), e.s, x0);
     const float d1 = fmaf(-f16_hi_to_float(h2), e.s, x1);

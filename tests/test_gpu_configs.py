@@ -199,3 +199,22 @@ def test_w4a4_fake_quant_every_element(nv):
     np.testing.assert_array_equal(fp.cpu().numpy(), rp)
     np.testing.assert_array_equal(bf16_bits(fy), ry)
     record_stat("w4a4 32768x8192", blocks=X.numel() // 16, elements_bit_exact=X.numel())
+
+
+def test_four_over_six_moe_weights_every_block(nv):
+    """Four Over Six on the MoE experts' weights (128 x 768x2048, per-expert
+    tensor scales, the benchmark's Four Over Six workload): every block's
+    code against the oracle, and the packed bytes of every expert."""
+    from scale_calibration_nvfp4_b200 import workloads
+    W, _, _ = workloads.moe_inputs("cuda")
+    G = W.shape[0]
+    s_g = nv.global_scale(W, batch=G)
+    c = nv.scale_search_four_over_six(W, s_g)
+    packed = nv.quantize_pack(W, s_g, c).cpu().numpy()
+    c = c.cpu().numpy()
+    wu, sgs = bf16_bits(W), s_g.cpu().numpy()
+    for e in range(G):
+        ref = oracle.scale_search_four_over_six(wu[e], float(sgs[e]))
+        np.testing.assert_array_equal(c[e], ref, err_msg="expert %d" % e)
+        np.testing.assert_array_equal(packed[e], oracle.quantize_pack(wu[e], float(sgs[e]), ref))
+    record_stat("four_over_six moe 128x768x2048", blocks=W.numel() // 16, codes_differing=0)

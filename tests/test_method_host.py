@@ -469,16 +469,49 @@ def _rn32(q):
     return (fl * quantum) * (1 if q > 0 else -1)
 
 
-def _mse32(oracle_mod, x, s):
-    """The kernel's fp32 block MSE: d_i = RN(x_i - v_i s), e = RN(d_i^2 + e)
-    in element order, every step rounded once from its exact value."""
+def _rd32(q):
+    """Round the positive rational q down to fp32 (normal range)."""
     from fractions import Fraction
-    S = Fraction(float(s))
+    e = q.numerator.bit_length() - q.denominator.bit_length()
+    while Fraction(2) ** e > q:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= q:
+        e += 1
+    quantum = Fraction(2) ** (e - 23)
+    n = q / quantum
+    return (n.numerator // n.denominator) * quantum
+
+
+def _rne_e2m1(t):
+    """E2M1 code of the fp32 value t itself (nearest, ties to the even
+    magnitude index, saturating at 6), decided on t exactly."""
+    from fractions import Fraction
+    a = abs(Fraction(float(t)))
+    k = 0
+    for i, m in enumerate(MIDS):
+        M = Fraction(float(m))
+        k += int(a > M) if i % 2 == 0 else int(a >= M)
+    return k | (8 if np.signbit(t) else 0)
+
+
+def _mse32(oracle_mod, x, s):
+    """The kernel's fp32 block MSE screen: each value's code rounded from
+    t = RN(x r_hi + RN(x r_lo)) (r_hi = 1/s rounded down, r_lo its fp32
+    correction), not from the exact quotient; then d_i = RN(x_i - v_i s),
+    e = RN(d_i^2 + e) in element order, every step rounded once from its
+    exact value."""
+    from fractions import Fraction
+    s32 = np.float32(s)
+    S = Fraction(float(s32))
+    r_hi = _rd32(1 / S)                                  # the kernel's __frcp_rd
+    r_lo = _rn32(_rn32(1 - S * r_hi) * r_hi)             # fmaf(-s, r_hi, 1) * r_hi
     e = Fraction(0)
     for xi in x:
-        k = oracle_mod.e2m1_encode(float(xi), float(s))
+        X = Fraction(float(xi))
+        t = _rn32(X * r_hi + _rn32(X * r_lo))
+        k = _rne_e2m1(float(t) if t != 0 else (-0.0 if np.signbit(xi) else 0.0))
         v = Fraction(float(GRID[k & 7])) * (-1 if k & 8 else 1)
-        d = _rn32(Fraction(float(xi)) - v * S)
+        d = _rn32(X - v * S)
         e = _rn32(d * d + e)
     return e
 
@@ -842,3 +875,52 @@ def test_screen_error_bound_makes_every_decision_sound(oracle_mod):
     assert wrong == 0, wrong
     wrong_rel, _, _ = _screen_violations(oracle_mod, q_on=False, adversarial=True, rows=rows)
     assert wrong_rel > 5, wrong_rel
+
+
+def test_four_over_six_screen_tolerates_codes_of_t(oracle_mod):
+    """The Four Over Six screen rounds t, which lies within one float of the
+    exact quotient q, so where t is an E2M1 midpoint and q is not, its code
+    can differ from the exact one.  Blocks built for that: s_eff = fl32(x / M)
+    for a bf16 x and a midpoint M with odd part 3, 5 or 7 (so x / s_eff lies
+    within about 2^-24 of M without equalling it), the block maximum putting
+    the max-rule code on that scale.  The codes of t differ from the exact
+    ones on many of these elements, and still every choice the screen makes
+    (|fh - fl| > 2^-16 max(fh, fl) + 2^-130) is the oracle's."""
+    from fractions import Fraction
+    rng = np.random.default_rng(3)
+    mids = [0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    flips = decided = wrong = 0
+    for trial in range(900):
+        M = mids[trial % len(mids)]
+        xm = float(bits_to_f64(bf16_bits(torch.tensor([rng.uniform(1, 2) * 2.0 ** rng.integers(-20, 4)]).to(torch.bfloat16)))[0])
+        s = float(np.float32(xm / M))
+        s_g = np.float32(s)                        # code 0x38 (1.0): s_eff = s_g exactly
+        x = rng.standard_normal(16) * s * 1.5
+        x[0] = 6 * s * rng.uniform(0.985, 1.015)   # the maximum: max-rule code 0x38
+        x[1] = xm * rng.choice([-1.0, 1.0])
+        x[2] = xm * rng.choice([-1.0, 1.0])
+        blk = bf16_bits(torch.from_numpy(x).float().to(torch.bfloat16))
+        xd = bits_to_f64(blk)
+        amax = float(np.max(np.abs(xd)))
+        c6 = oracle_mod.e4m3_round_quotient(amax, 6.0 * float(s_g))
+        c4 = oracle_mod.e4m3_round_quotient(amax, 4.0 * float(s_g))
+        lo, hi = min(c4, c6), max(c4, c6)
+        if lo == hi:
+            continue
+        for c in (lo, hi):
+            se = oracle_mod.effective_scale(s_g, c)
+            S = Fraction(float(np.float32(se)))
+            r_hi = _rd32(1 / S)
+            r_lo = _rn32(_rn32(1 - S * r_hi) * r_hi)
+            for xi in xd:
+                X = Fraction(float(xi))
+                tt = _rn32(X * r_hi + _rn32(X * r_lo))
+                kt = _rne_e2m1(float(tt) if tt != 0 else (-0.0 if np.signbit(xi) else 0.0))
+                flips += kt != oracle_mod.e2m1_encode(float(xi), float(se))
+        fl = _mse32(oracle_mod, xd, oracle_mod.effective_scale(s_g, lo))
+        fh = _mse32(oracle_mod, xd, oracle_mod.effective_scale(s_g, hi))
+        if abs(_rn32(fh - fl)) > _rn32(Fraction(2) ** -16 * max(fh, fl) + Fraction(2) ** -130):
+            decided += 1
+            wrong += (hi if fh < fl else lo) != oracle_mod.four_over_six_code(blk, float(s_g))
+    assert flips > 100, flips
+    assert decided > 300 and wrong == 0, (decided, wrong)

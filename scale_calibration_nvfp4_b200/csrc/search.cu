@@ -287,6 +287,9 @@ __device__ __noinline__ double objective64_half(float x, float s_g, int c, const
 __device__ __noinline__ int refine_block(const uint16_t *wrow, float s_g, const float *Hs,
                                          int c1, int c2, bool full, float *obj) {
   const int lane = threadIdx.x & 31;
+  // the work statistic: one more row re-scored (over the best two or over
+  // every candidate), for this rule
+  if (lane == 0) atomicAdd(&g_search_evals[(Hs ? 4 : 2) + (full ? 1 : 0)], 1ull);
   const float x = __uint_as_float((uint32_t)wrow[lane & 15] << 16);
   double best = __longlong_as_double(0x7FF0000000000000LL);
   int best_c = 1;
@@ -317,6 +320,15 @@ __device__ __noinline__ int refine_block(const uint16_t *wrow, float s_g, const 
   }
   *obj = (float)best;
   return best_c;
+}
+
+// An upper bound of sqrt(x) for x >= 0 from the hardware approximation
+// (relative error far below 2^-16, so the 2^-16 inflation keeps it above the
+// exact root; only bounds are formed with it).
+__device__ __forceinline__ float sqrt_up(float x) {
+  float r;
+  asm("sqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r * (1.0f + 0x1p-16f);
 }
 
 // Objective and code in one sortable value: a non-negative float whose seven
@@ -385,24 +397,29 @@ __device__ __forceinline__ float candidate_objective(const float tq[8], float f,
 // its rows.
 struct Factor {
   float sigma;   // power of two putting max |L| in [2^14, 2^15)
-  float lambda;  // lower bound of lambda_min(L L^T), 0 when unknown
+  float sl2;     // sigma^2 lambda, lambda a lower bound of lambda_min(L L^T) (0 when unknown)
   int zero;      // H_b == 0 (every candidate scores 0)
-  float rho;     // sigma^2 ||H - L L^T||_inf (fp64 factor; dropped pivots), inf if unknown
-  float cdiag[16];  // lower bounds of 1 / (H^-1)_rr (0 when lambda is 0)
+  float rsq;     // 12 sqrt(sigma^2 ||H - L L^T||_inf), rounded up; inf if unknown
+  float cs[16];  // sigma^2 times lower bounds of 1 / (H^-1)_rr (0 where lambda is 0)
 };
 
-// ||H - Ld Ld^T||_inf by one half-warp (lane r sums row r), plus 2^-40 max
-// diag(H) for the rounding of the fp64 factor and of this sum; each lane of
-// the half returns it.  Zero unless pivots were dropped (up to rounding).
-__device__ __forceinline__ double factor_residual(const float *Hs, const double *Ld) {
+// A bound of ||H - Ld Ld^T||_inf by one half-warp, returned to each lane of
+// the half: 2^-40 max diag(H) covers the rounding of the fp64 factor (its
+// backward error is below 16 * 17 * 2^-53 max diag(H)) and of this sum;
+// where a pivot was dropped (`dropped`: the half's factor has a zero on the
+// diagonal) the residual itself is added, lane r summing row r.
+__device__ __forceinline__ double factor_residual(const float *Hs, const double *Ld,
+                                                  bool dropped) {
   const int r = threadIdx.x & 15;
   double rs = 0.0, dg = (double)Hs[r * 16 + r];
+  if (dropped) {
 #pragma unroll 1
-  for (int j = 0; j < 16; ++j) {
-    double x = (double)Hs[r * 16 + j];
+    for (int j = 0; j < 16; ++j) {
+      double x = (double)Hs[r * 16 + j];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) x = fma(-Ld[r * 16 + k], Ld[j * 16 + k], x);
-    rs += fabs(x);
+      for (int k = 0; k < 16; ++k) x = fma(-Ld[r * 16 + k], Ld[j * 16 + k], x);
+      rs += fabs(x);
+    }
   }
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) {
@@ -432,7 +449,8 @@ __global__ void __launch_bounds__(32)
   __syncwarp();
   cholesky16(Hs[h], Lf[h], Ld[h]);
   __syncwarp();
-  const double resid = factor_residual(Hs[h], Ld[h]);
+  const bool dropped = (__ballot_sync(kFull, Lf[h][r * 16 + r] == 0.0f) >> (lane & 16)) & 0xFFFFu;
+  const double resid = factor_residual(Hs[h], Ld[h], dropped);
   float m = 0.0f;
   for (int i = r; i < 256; i += 16) m = fmaxf(m, fabsf(Lf[h][i]));
 #pragma unroll
@@ -443,14 +461,17 @@ __global__ void __launch_bounds__(32)
   frexpf(m, &e);  // m < 2^e
   const float sigma = m > 0.0f ? ldexpf(1.0f, 15 - e) : 1.0f;
   if (live && r == 0) {
+    // the search's factors in its units (sigma^2 lambda and sigma^2 cdiag
+    // stay below 16 * 2^30: lambda, cdiag <= max diag(L L^T) <= 16 max |L|^2)
     Factor f;
+    const double s2 = (double)sigma * (double)sigma;
     f.sigma = sigma;
-    f.lambda = lam;
+    f.sl2 = __double2float_rd(s2 * (double)lam);
     f.zero = !(m > 0.0f);
-    const double rho = resid * (double)sigma * (double)sigma;  // below 2^40: no overflow
-    f.rho = rho < 3.0e38 ? (float)rho : __int_as_float(0x7F800000);  // NaN -> inf too
+    const double rsq = 12.0 * sqrt(resid * s2) * (1.0 + 0x1p-40);  // rounded up below
+    f.rsq = rsq < 3.0e38 ? __double2float_ru(rsq) : __int_as_float(0x7F800000);  // NaN too
 #pragma unroll
-    for (int i = 0; i < 16; ++i) f.cdiag[i] = cdiag[h][i];
+    for (int i = 0; i < 16; ++i) f.cs[i] = __double2float_rd(s2 * (double)cdiag[h][i]);
     fac[base + j0 + h] = f;
   }
   // every lane's fragments of both blocks: B[k][n] = sigma L[k][n], n = 8 nt
@@ -503,7 +524,6 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
   __shared__ ClassInfo cls[kMaxClasses];
   __shared__ CandInfo cand[kCandidates];
   __shared__ float cdiag_sh[16];  // bounds of 1 / (H^-1)_rr of this column block
-  __shared__ float Hsh[kLH ? 256 : 1];  // H_b, for the fp64 re-scores
   __shared__ int ncls_sh;
   __shared__ uint4 Ws[kRowsPerCta][2];     // the CTA's 16-element row segments
   __shared__ uint32_t keys[kRowsPerCta];  // amax << 16 | local row, sorted
@@ -516,8 +536,8 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
   // ---- factor of H_b (from factor_kernel) and the zero-H shortcut
   const int64_t blk = batch * nb + b;
   const float *Hb = kLH ? H + blk * 256 : nullptr;  // the definition, for re-scoring
-  float sigma = 1.0f, lambda = 1.0f;  // MSE: H = I
-  float rho = 0.0f;                    // sigma^2 ||H - L L^T||_inf (Local-Hessian)
+  float sigma = 1.0f, sl2 = 1.0f;  // MSE: H = I
+  float rsq = 0.0f;                // 12 sqrt(sigma^2 ||H - L L^T||_inf) (Local-Hessian)
   uint32_t bh[2][2], bl[2][2];
   if (kLH) {
     const Factor f = fac[blk];
@@ -530,10 +550,9 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       return;
     }
     sigma = f.sigma;
-    lambda = f.lambda;
-    rho = f.rho;
-    if (threadIdx.x < 16) cdiag_sh[threadIdx.x] = fac[blk].cdiag[threadIdx.x];
-    for (int i = threadIdx.x; i < 256; i += kThreads) Hsh[i] = Hb[i];
+    sl2 = f.sl2;
+    rsq = f.rsq;
+    if (threadIdx.x < 16) cdiag_sh[threadIdx.x] = fac[blk].cs[threadIdx.x];
     const uint4 h = frag[(blk * 32 + lane) * 2], l = frag[(blk * 32 + lane) * 2 + 1];
     bh[0][0] = h.x; bh[0][1] = h.y; bh[1][0] = h.z; bh[1][1] = h.w;
     bl[0][0] = l.x; bl[0][1] = l.y; bl[1][0] = l.z; bl[1][1] = l.w;
@@ -550,7 +569,6 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         bl[nt][half] = 0u;
       }
   }
-  const float sqrt_lambda = sqrtf(lambda);
 
   // ---- candidate tables (per CTA, from this batch element's s_g)
   const bool by_class = s_g >= 0x1p-100f && s_g < 0x1p100f;
@@ -624,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     }
   }
 
-  unsigned long long evals = 0, rescored1 = 0, rescored2 = 0;
+  unsigned long long evals = 0;
   for (int tile = warp; tile < kRowsPerCta / kTileRows; tile += kWarps) {
     const uint32_t kg = keys[tile * kTileRows + g], kg8 = keys[tile * kTileRows + g + 8];
     const bool v0 = (kg >> 16) != 0xFFFFu, v1 = (kg8 >> 16) != 0xFFFFu;
@@ -716,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       aa += __shfl_xor_sync(0xFFFFFFFFu, aa, 1);
       // dropped pivots: sqrt(F) <= 12 sqrt(rho) max|W| of the row
       const float wmax = __uint_as_float((upper ? am1 : am0) << 16) * wsc;
-      qerr = fmaf(kAccErr, sqrtf(aa), kAbsErr) + 12.0f * sqrtf(rho) * wmax;
+      qerr = fmaf(kAccErr, sqrt_up(aa), kAbsErr) + rsq * wmax;
     } else {
       pz[0][0] = xs[0] * wsc0; pz[0][1] = xs[1] * wsc0; pz[0][2] = xs[2] * wsc1;
       pz[0][3] = xs[3] * wsc1; pz[1][0] = xs[4] * wsc0; pz[1][1] = xs[5] * wsc0;
@@ -750,8 +768,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     // largest amax / 6 downwards, then from there upwards.  Rows past the end
     // and all-zero rows never hold the warp back.
     const float amax_row = __uint_as_float((upper ? am1 : am0) << 16);
-    const float sl = sigma * sqrtf(lambda);
-    const float sl2 = sl * sl;
+
     // saturation bound of the lane's row: its largest element (position i)
     // alone forces E >= |delta_i|^2 / (H^-1)_ii; an element whose magnitude
     // equals the row's amax, found in the quad (any one of equal maxima)
@@ -771,8 +788,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       };
       const int i0 = find(pw[0], pw[2], am0), i1 = find(pw[1], pw[3], am1);
       const int idx = upper ? i1 : i0;
-      const float si = sigma * sqrtf(idx >= 0 ? cdiag_sh[idx] : 0.0f);
-      ss2 = si * si;
+      ss2 = idx >= 0 ? cdiag_sh[idx] : 0.0f;
     }
     const float amax_w = amax_row * wsc, m6w = -6.0f * wsc;
     const float row_floor = kZeroFloor * (upper ? pp1 : pp0);
@@ -876,14 +892,12 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         // each (b3 may be infinite when pruning left two: then all 126)
         const float q4 = 4.0f * qerr, q12 = fmaf(12.0f * qerr, qerr, kAbsBand);
         const float big = 3.0e38f;
-        if (b2 - b1 <= fmaf(kTieBand, b2, fmaf(q4, sqrtf(fminf(b2, big)), q12)) ||
+        if (b2 - b1 <= fmaf(kTieBand, b2, fmaf(q4, sqrt_up(fminf(b2, big)), q12)) ||
             b1 <= fmaf(16.0f * qerr, qerr, fl))
-          need = (b3 - b1 > fmaf(kTieBand, b3, fmaf(q4, sqrtf(fminf(b3, big)), q12 + fl))) ? 1
+          need = (b3 - b1 > fmaf(kTieBand, b3, fmaf(q4, sqrt_up(fminf(b3, big)), q12 + fl))) ? 1
                                                                                           : 2;
       }
     }
-    rescored1 += __popc(__ballot_sync(0xFFFFFFFFu, need == 1));
-    rescored2 += __popc(__ballot_sync(0xFFFFFFFFu, need == 2));
     for (uint32_t pend = __ballot_sync(0xFFFFFFFFu, need != 0); pend; pend &= pend - 1) {
       const int src = __ffs(pend) - 1;
       const int64_t rr = __shfl_sync(0xFFFFFFFFu, (long long)r, src);
@@ -891,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       const int k1 = __shfl_sync(0xFFFFFFFFu, code_of(b1), src);
       const int k2 = __shfl_sync(0xFFFFFFFFu, code_of(b2), src);
       float o;
-      const int c = refine_block(wb + rr * C, s_g, kLH ? Hsh : nullptr, k1, k2, n == 2, &o);
+      const int c = refine_block(wb + rr * C, s_g, Hb, k1, k2, n == 2, &o);
       if (lane == src) {
         code = c;
         obj = o;
@@ -904,8 +918,6 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
   }
   if (lane == 0) {
     if (evals) atomicAdd(&g_search_evals[kLH ? 1 : 0], evals);
-    if (rescored1) atomicAdd(&g_search_evals[kLH ? 4 : 2], rescored1);
-    if (rescored2) atomicAdd(&g_search_evals[kLH ? 5 : 3], rescored2);
   }
 }
 

@@ -380,6 +380,12 @@ def _lambda_bound(Lf):
     return float(np.float32(0.98 / colsum))
 
 
+def _f32_down(x):
+    """x (a float64) rounded down to fp32."""
+    f = np.float32(x)
+    return np.nextafter(f, np.float32(-np.inf)) if float(f) > x else f
+
+
 def _cdiag_bound(Lf):
     """The kernel's per-channel bounds 0.97 / ((L L^T)^-1)_rr (fp32 factor,
     fp64 solves), all 0 where the eigenvalue bound is 0."""
@@ -606,11 +612,9 @@ def test_pruning_bounds_hold_at_any_magnitude(oracle_mod, e):
                 if m == 0 or lam == 0:
                     continue
                 sigma = 2.0 ** (15 - np.frexp(np.float32(m))[1])
-            sl = np.float32(np.float32(sigma) * np.sqrt(np.float32(lam)))
-            sl2 = np.float32(sl * sl)
+            sl2 = _f32_down(sigma ** 2 * lam)
             cd = 1.0 if H is None else _cdiag_bound(Lf)[int(np.argmax(np.abs(w)))]
-            si = np.float32(np.float32(sigma) * np.sqrt(np.float32(cd)))
-            ss2 = np.float32(si * si)
+            ss2 = _f32_down(sigma ** 2 * cd)
             E = _screen_objectives(w, s_list, sigma, Lf, kw)
             for s, Ej in zip(s_list, E):
                 if s < amax / 6:
@@ -827,10 +831,9 @@ def _screen_violations(oracle_mod, q_on, n_rows=700, seed=5, adversarial=False, 
             wrong += not ok(pick)
         # pruning: saturation and zero-code bounds against every evaluated key
         if sc["lam"] > 0:
-            sl = np.float32(np.float32(sc["sigma"]) * np.sqrt(np.float32(sc["lam"])))
-            sl2 = np.float32(sl * sl)
-            si = np.float32(np.float32(sc["sigma"]) * np.sqrt(np.float32(sc["cd"])))
-            ss2 = np.float32(si * si)
+            # the factor kernel's sigma^2 lambda and sigma^2 cdiag, rounded down
+            sl2 = _f32_down(sc["sigma"] ** 2 * sc["lam"])
+            ss2 = _f32_down(sc["sigma"] ** 2 * sc["cd"])
             for c in range(1, 127):
                 s = sc["svals"][c - 1]
                 bounds = []

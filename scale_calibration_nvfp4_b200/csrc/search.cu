@@ -510,9 +510,9 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
                   const float *__restrict__ s_g_arr, const float *__restrict__ H,
                   const uint4 *__restrict__ frag, const Factor *__restrict__ fac,
                   uint8_t *__restrict__ codes, float *__restrict__ best_obj) {
-  static_assert((kRowsPerCta & (kRowsPerCta - 1)) == 0 && kRowsPerCta <= 65536 &&
+  static_assert((kRowsPerCta & (kRowsPerCta - 1)) == 0 && kRowsPerCta <= 4096 &&
                     kRowsPerCta % (kWarps * kTileRows) == 0,
-                "the row sort needs a power-of-two row count below 2^16");
+                "the row sort needs a power-of-two row count up to 2^12");
   const int64_t nb = C / kBlock;
   const int64_t b = blockIdx.y;
   const int64_t batch = blockIdx.z;
@@ -607,8 +607,9 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
   // ---- the CTA's rows, staged in shared memory and ordered by amax so that
   // every warp tile holds rows of similar magnitude: the pruning bounds below
   // then stop the candidate walk at nearly the same point for all 16 rows.
-  // Sort key: amax (bf16 magnitude bits) above the local row index; rows past
-  // the end get magnitude 0xFFFF (zero data) and sort last.
+  // Sort key: amax (bf16 magnitude bits, bits 16..31), the position of the
+  // row's largest element (bits 12..15) and the local row index (bits
+  // 0..11); rows past the end get magnitude 0xFFFF (zero data) and sort last.
   for (int i = threadIdx.x; i < kRowsPerCta; i += kThreads) {
     const int64_t r = row_base + i;
     uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
@@ -618,7 +619,16 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       a0 = ld_stream_v4(q);
       a1 = ld_stream_v4(q + 1);
       const uint32_t w8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      key = (amax_bits8(w8) << 16) | (uint32_t)i;
+      // amax bits, then the position of an element that reaches it (for the
+      // row's saturation bound), then the local row
+      const uint32_t am = amax_bits8(w8);
+      uint32_t pos = 0;
+#pragma unroll
+      for (int e = 15; e >= 0; --e) {
+        const uint32_t mag = ((e & 1) ? (w8[e >> 1] >> 16) : w8[e >> 1]) & 0x7FFFu;
+        pos = mag == am ? (uint32_t)e : pos;
+      }
+      key = (am << 16) | (pos << 12) | (uint32_t)i;
     }
     Ws[i][0] = a0;
     Ws[i][1] = a1;
@@ -647,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     const uint32_t kg = keys[tile * kTileRows + g], kg8 = keys[tile * kTileRows + g + 8];
     const bool v0 = (kg >> 16) != 0xFFFFu, v1 = (kg8 >> 16) != 0xFFFFu;
     if (!__any_sync(0xFFFFFFFFu, v0 || v1)) break;  // only padding from here on
-    const int i0 = (int)(kg & 0xFFFFu), i1 = (int)(kg8 & 0xFFFFu);
+    const int i0 = (int)(kg & 0xFFFu), i1 = (int)(kg8 & 0xFFFu);
     uint32_t W0[8], W1[8];
     {
       const uint4 a0 = Ws[i0][0], a1 = Ws[i0][1], c0 = Ws[i1][0], c1 = Ws[i1][1];
@@ -769,27 +779,10 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     // and all-zero rows never hold the warp back.
     const float amax_row = __uint_as_float((upper ? am1 : am0) << 16);
 
-    // saturation bound of the lane's row: its largest element (position i)
-    // alone forces E >= |delta_i|^2 / (H^-1)_ii; an element whose magnitude
-    // equals the row's amax, found in the quad (any one of equal maxima)
-    float ss2;
-    {
-      // every lane of the quad holds elements {2t, 2t+1, 2t+8, 2t+9} of both
-      // rows (pairs 0, 2: row g; 1, 3: row g + 8): search both, reduce over
-      // the quad, keep the lane's own row
-      auto find = [&](uint32_t pa, uint32_t pb, uint32_t am) {
-        int i = -1;
-        i = ((pb >> 16) & 0x7FFFu) == am ? 2 * t + 9 : i;
-        i = (pb & 0x7FFFu) == am ? 2 * t + 8 : i;
-        i = ((pa >> 16) & 0x7FFFu) == am ? 2 * t + 1 : i;
-        i = (pa & 0x7FFFu) == am ? 2 * t : i;
-        i = max(i, __shfl_xor_sync(0xFFFFFFFFu, i, 1));
-        return max(i, __shfl_xor_sync(0xFFFFFFFFu, i, 2));
-      };
-      const int i0 = find(pw[0], pw[2], am0), i1 = find(pw[1], pw[3], am1);
-      const int idx = upper ? i1 : i0;
-      ss2 = idx >= 0 ? cdiag_sh[idx] : 0.0f;
-    }
+    // saturation bound of the lane's row: its largest element (position i,
+    // from the row's sort key; any one of equal maxima) alone forces
+    // E >= |delta_i|^2 / (H^-1)_ii
+    const float ss2 = cdiag_sh[((upper ? kg8 : kg) >> 12) & 0xFu];
     const float amax_w = amax_row * wsc, m6w = -6.0f * wsc;
     const float row_floor = kZeroFloor * (upper ? pp1 : pp0);
     // a candidate is skipped when its lower bound, less the bound's own

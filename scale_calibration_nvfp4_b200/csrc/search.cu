@@ -782,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     // saturation bound of the lane's row: its largest element (position i,
     // from the row's sort key; any one of equal maxima) alone forces
     // E >= |delta_i|^2 / (H^-1)_ii
-    const float ss2 = cdiag_sh[((upper ? kg8 : kg) >> 12) & 0xFu];
+    const float ss2 = kLH ? cdiag_sh[((upper ? kg8 : kg) >> 12) & 0xFu] : 1.0f;
     const float amax_w = amax_row * wsc, m6w = -6.0f * wsc;
     const float row_floor = kZeroFloor * (upper ? pp1 : pp0);
     // a candidate is skipped when its lower bound, less the bound's own
@@ -880,7 +880,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         // leave the normal range, so the screen only orders; every candidate
         // is re-scored in fp64
         need = 2;
-      } else {
+      } else if (kLH) {
         // both candidates' screen errors: kTieBand b + 2 Q sqrt(b) + 6 Q^2
         // each (b3 may be infinite when pruning left two: then all 126)
         const float q4 = 4.0f * qerr, q12 = fmaf(12.0f * qerr, qerr, kAbsBand);
@@ -889,6 +889,9 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
             b1 <= fmaf(16.0f * qerr, qerr, fl))
           need = (b3 - b1 > fmaf(kTieBand, b3, fmaf(q4, sqrt_up(fminf(b3, big)), q12 + fl))) ? 1
                                                                                           : 2;
+      } else if (b2 - b1 <= kTieBand * b2 + kAbsBand || b1 <= fl) {
+        // MSE: u = v and p = W exactly, Q = 0
+        need = (b3 - b1 > kTieBand * b3 + fl + kAbsBand) ? 1 : 2;
       }
     }
     for (uint32_t pend = __ballot_sync(0xFFFFFFFFu, need != 0); pend; pend &= pend - 1) {

@@ -329,14 +329,17 @@ __device__ __forceinline__ float block_mse32(const uint32_t w[8], uint2 q, float
 }
 
 // The fp32 block MSE at a table entry's scale, straight from the values:
-// each pair is rounded from t (one conversion) and its byte decoded by the
-// hardware e2m1x2 -> f16x2 conversion in the same asm block, then d_i = x_i -
-// v_i s and e += d_i^2 in block_mse32's order.  The codes are those of t, not
-// always of the exact quotient q: where t is a rounding midpoint and q lies
-// off it (t within one float of q), t may round to the other neighbour, and
-// then |d_i| moves by at most 2 ulp(t) s, i.e. d_i^2 by at most 2^-20 of
-// itself -- inside the screen's 2^-16 threshold; the exact comparison below
-// uses exact codes.
+// t = fl(x r_hi) (r_hi = 1/s rounded down: |t - q| <= 2^-23 |q| for the exact
+// quotient q), each pair rounded from t (one conversion) and its byte decoded
+// by the hardware e2m1x2 -> f16x2 conversion in the same asm block, then d_i =
+// x_i - v_i s and e += d_i^2 in block_mse32's order.  The codes are those of
+// t, not always of q: where a rounding midpoint M lies between q and t, t
+// takes the other neighbour, and |d_i| (about half a grid step times s either
+// way) moves by at most 2 |q - M| s <= 2^-22 |q| s, at most 2^-19.7 of itself
+// (the worst case M = 5 with a step of 2); d_i^2 then moves by at most
+// 2^-18.7, and with the roundings of the sums the screen stays within 2^-18.4
+// of the definition -- inside its 2^-16 threshold.  The exact comparison
+// below uses exact codes.
 __device__ __forceinline__ uint32_t e2m1x2_round_decode(float hi, float lo) {
   uint32_t h2;
   asm("{\n\t.reg .b8 q;\n\t"
@@ -352,7 +355,7 @@ __device__ __forceinline__ float block_mse32_entry(const uint32_t w[8], const Sc
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const float x0 = bf16_lo(w[j]), x1 = bf16_hi(w[j]);
-    const float t0 = fmaf(x0, e.r_hi, x0 * e.r_lo), t1 = fmaf(x1, e.r_hi, x1 * e.r_lo);
+    const float t0 = x0 * e.r_hi, t1 = x1 * e.r_hi;
     const uint32_t h2 = e2m1x2_round_decode(t1, t0);
     const float d0 = fmaf(-f16_lo_to_float(h2), e.s, x0);
     const float d1 = fmaf(-f16_hi_to_float(h2), e.s, x1);

@@ -230,24 +230,29 @@ __device__ __forceinline__ float lambda_lower_bound(const float *Lf, double *inv
   double colsum = 0.0, dinv = 0.0;
   if (!singular) {
     // column sweeps: acc = e_r, then L y = acc, then L^T z = y (in place;
-    // outer loops rolled, acc in local memory: once per block of H)
+    // fully unrolled, so acc stays in registers; the factor is read through a
+    // volatile pointer so its loads stay in program order and are not all
+    // hoisted into registers)
+    const volatile float *Lv = Lf;
     double acc[16];
 #pragma unroll
     for (int m = 0; m < 16; ++m) acc[m] = (m == r) ? 1.0 : 0.0;
-#pragma unroll 1
+#pragma unroll
     for (int k = 0; k < 16; ++k) {
       acc[k] *= inv_d[k];
 #pragma unroll
-      for (int m = k + 1; m < 16; ++m) acc[m] = fma(-(double)Lf[m * 16 + k], acc[k], acc[m]);
+      for (int m = k + 1; m < 16; ++m) acc[m] = fma(-(double)Lv[m * 16 + k], acc[k], acc[m]);
     }
-#pragma unroll 1
+#pragma unroll
     for (int k = 15; k >= 0; --k) {
       acc[k] *= inv_d[k];
       colsum += fabs(acc[k]);
 #pragma unroll
-      for (int m = 0; m < k; ++m) acc[m] = fma(-(double)Lf[k * 16 + m], acc[k], acc[m]);
+      for (int m = 0; m < k; ++m) acc[m] = fma(-(double)Lv[k * 16 + m], acc[k], acc[m]);
     }
-    dinv = acc[r];  // ((L L^T)^-1)_rr
+#pragma unroll
+    for (int m = 0; m < 16; ++m)
+      if (m == r) dinv = acc[m];  // ((L L^T)^-1)_rr
   }
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) colsum = fmax(colsum, __shfl_xor_sync(kFull, colsum, o));

@@ -502,19 +502,17 @@ def _rne_e2m1(t):
 
 def _mse32(oracle_mod, x, s):
     """The kernel's fp32 block MSE screen: each value's code rounded from
-    t = RN(x r_hi + RN(x r_lo)) (r_hi = 1/s rounded down, r_lo its fp32
-    correction), not from the exact quotient; then d_i = RN(x_i - v_i s),
-    e = RN(d_i^2 + e) in element order, every step rounded once from its
-    exact value."""
+    t = RN(x r_hi) (r_hi = 1/s rounded down), not from the exact quotient;
+    then d_i = RN(x_i - v_i s), e = RN(d_i^2 + e) in element order, every step
+    rounded once from its exact value."""
     from fractions import Fraction
     s32 = np.float32(s)
     S = Fraction(float(s32))
     r_hi = _rd32(1 / S)                                  # the kernel's __frcp_rd
-    r_lo = _rn32(_rn32(1 - S * r_hi) * r_hi)             # fmaf(-s, r_hi, 1) * r_hi
     e = Fraction(0)
     for xi in x:
         X = Fraction(float(xi))
-        t = _rn32(X * r_hi + _rn32(X * r_lo))
+        t = _rn32(X * r_hi)
         k = _rne_e2m1(float(t) if t != 0 else (-0.0 if np.signbit(xi) else 0.0))
         v = Fraction(float(GRID[k & 7])) * (-1 if k & 8 else 1)
         d = _rn32(X - v * S)
@@ -881,9 +879,9 @@ def test_screen_error_bound_makes_every_decision_sound(oracle_mod):
 
 
 def test_four_over_six_screen_tolerates_codes_of_t(oracle_mod):
-    """The Four Over Six screen rounds t, which lies within one float of the
-    exact quotient q, so where t is an E2M1 midpoint and q is not, its code
-    can differ from the exact one.  Blocks built for that: s_eff = fl32(x / M)
+    """The Four Over Six screen rounds t = fl(x r_hi), within 2^-23 of the
+    exact quotient q, so where a midpoint lies between q and t its code can
+    differ from the exact one.  Blocks built for that: s_eff = fl32(x / M)
     for a bf16 x and a midpoint M with odd part 3, 5 or 7 (so x / s_eff lies
     within about 2^-24 of M without equalling it), the block maximum putting
     the max-rule code on that scale.  The codes of t differ from the exact
@@ -914,10 +912,9 @@ def test_four_over_six_screen_tolerates_codes_of_t(oracle_mod):
             se = oracle_mod.effective_scale(s_g, c)
             S = Fraction(float(np.float32(se)))
             r_hi = _rd32(1 / S)
-            r_lo = _rn32(_rn32(1 - S * r_hi) * r_hi)
             for xi in xd:
                 X = Fraction(float(xi))
-                tt = _rn32(X * r_hi + _rn32(X * r_lo))
+                tt = _rn32(X * r_hi)
                 kt = _rne_e2m1(float(tt) if tt != 0 else (-0.0 if np.signbit(xi) else 0.0))
                 flips += kt != oracle_mod.e2m1_encode(float(xi), float(se))
         fl = _mse32(oracle_mod, xd, oracle_mod.effective_scale(s_g, lo))

@@ -119,34 +119,6 @@ struct CandInfo {
 };
 
 // ----------------------------------------------------------------- helpers
-// Four e2m1x2 conversions packed into one word: byte i holds
-// (code(hi_i) << 4) | code(lo_i).
-__device__ __forceinline__ uint32_t cvt4_e2m1x2(float h0, float l0, float h1, float l1,
-                                                float h2, float l2, float h3, float l3) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q0, %1, %2;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q1, %3, %4;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q2, %5, %6;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q3, %7, %8;\n\t"
-      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
-      : "=r"(r)
-      : "f"(h0), "f"(l0), "f"(h1), "f"(l1), "f"(h2), "f"(l2), "f"(h3), "f"(l3));
-  return r;
-}
-
-// Four code bytes -> four f16x2 registers (low nibble -> low half).
-__device__ __forceinline__ void cvt4_f16x2(uint32_t codes, uint32_t a[4]) {
-  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
-      "mov.b32 {q0, q1, q2, q3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, q2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, q3;\n\t}"
-      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
-      : "r"(codes));
-}
-
 __device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4], uint32_t b0,
                                               uint32_t b1, const float c[4]) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
@@ -351,6 +323,25 @@ __device__ __forceinline__ void track3(float key, float &b1, float &b2, float &b
   b1 = fminf(b1, key);
 }
 
+// Four signed pairs rounded to E2M1 (nearest even, saturating; a negative
+// value that rounds to zero gives -0) and decoded to f16x2 in one asm block:
+// A[i] holds (lo_i, hi_i), the MMA's A fragment, with no packing of the codes
+// in between.
+__device__ __forceinline__ void round_decode4(float h0, float l0, float h1, float l1, float h2,
+                                              float l2, float h3, float l3, uint32_t A[4]) {
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %4, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %6, %7;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %8, %9;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %10, %11;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, q2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, q3;\n\t}"
+      : "=r"(A[0]), "=r"(A[1]), "=r"(A[2]), "=r"(A[3])
+      : "f"(h0), "f"(l0), "f"(h1), "f"(l1), "f"(h2), "f"(l2), "f"(h3), "f"(l3));
+}
+
 // Select word t (0..3) of four without local memory.
 __device__ __forceinline__ uint32_t pick4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
                                           int t) {
@@ -359,22 +350,19 @@ __device__ __forceinline__ uint32_t pick4(uint32_t w0, uint32_t w1, uint32_t w2,
 
 // One candidate: codes, the tensor-core product u, z = p - s u, and the row
 // objective after a quad reduce-scatter (lanes t < 2: row g, t >= 2: row
-// g + 8).  tq holds the class quotients (stepped where a midpoint could
-// occur), f scales them to this candidate exactly; sm0 and sm1 multiply u in
-// rows g and g + 8 (accumulator elements 0, 1 and 2, 3 of both n-tiles),
+// g + 8).  tq holds the signed class quotients (stepped where a midpoint
+// could occur), f scales them to this candidate exactly; sm0 and sm1 multiply
+// u in rows g and g + 8 (accumulator elements 0, 1 and 2, 3 of both n-tiles),
 // each row carrying its own power-of-two scale.
 template <bool kLH>
 __device__ __forceinline__ float candidate_objective(const float tq[8], float f, float sm0,
-                                                     float sm1, uint32_t sgn,
-                                                     const uint32_t bh[2][2],
+                                                     float sm1, const uint32_t bh[2][2],
                                                      const uint32_t bl[2][2],
                                                      const float pz[2][4], bool upper) {
   const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  const uint32_t code = cvt4_e2m1x2(tq[1] * f, tq[0] * f, tq[3] * f, tq[2] * f, tq[5] * f,
-                                    tq[4] * f, tq[7] * f, tq[6] * f) |
-                        sgn;
   uint32_t A[4];
-  cvt4_f16x2(code, A);
+  round_decode4(tq[1] * f, tq[0] * f, tq[3] * f, tq[2] * f, tq[5] * f, tq[4] * f, tq[7] * f,
+                tq[6] * f, A);
   float u0[4], u1[4];
   mma_f16_16816(u0, A, bh[0][0], bh[0][1], zero4);
   mma_f16_16816(u1, A, bh[1][0], bh[1][1], zero4);
@@ -685,15 +673,11 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
                             pick4(W1[4], W1[5], W1[6], W1[7], t)};
     // element k of the lane in C order: 2i, 2i+1 = low, high half of pair i
     // (row g: elements 0, 1, 4, 5; row g + 8: 2, 3, 6, 7)
-    float xs[8], a[8];
-    uint32_t sgn = 0;
+    float xs[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       xs[2 * i] = bf16_lo(pw[i]);
       xs[2 * i + 1] = bf16_hi(pw[i]);
-      a[2 * i] = fabsf(xs[2 * i]);
-      a[2 * i + 1] = fabsf(xs[2 * i + 1]);
-      sgn |= (((pw[i] >> 12) & 0x8u) | ((pw[i] >> 24) & 0x80u)) << (8 * i);
     }
     // p = L^T w at the C positions: pz[nt][0..1] row g, n = 8nt + 2t + {0,1};
     // pz[nt][2..3] row g+8, same n.  Local-Hessian: from the tensor cores
@@ -802,19 +786,21 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       // class quotient t per element (within one float of q)
       float tq[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) tq[e] = fmaf(a[e], ci.r_hi, a[e] * ci.r_lo);
+      for (int e = 0; e < 8; ++e) tq[e] = fmaf(xs[e], ci.r_hi, xs[e] * ci.r_lo);
       // uncertified classes: a quotient with at most 3 significant bits
       // (every rounding midpoint is one, and so is every power-of-two
       // multiple) steps to its neighbouring float across q, by the exact
-      // sign of the residual |w| - t S; t itself when q == t.  Every other
-      // t is not a midpoint at any scale of the class and rounds like q.
+      // sign of the residual w - t S (away from zero when it has t's sign);
+      // t itself when q == t.  Every other t is not a midpoint at any scale of
+      // the class and rounds like q.
       if (!ci.certified) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float rho = fmaf(-tq[e], ci.S, a[e]);
-          const int step = (rho > 0.0f) - (rho < 0.0f);
-          const bool near = (__float_as_uint(tq[e]) & 0x1FFFFFu) == 0u;
-          tq[e] = near ? __int_as_float(__float_as_int(tq[e]) + step) : tq[e];
+          const float rho = fmaf(-tq[e], ci.S, xs[e]);
+          const int rb = __float_as_int(rho), tb = __float_as_int(tq[e]);
+          const int step = rb != 0 ? (((rb ^ tb) >> 31) | 1) : 0;
+          const bool near = (tb & 0x1FFFFF) == 0;
+          tq[e] = near ? __int_as_float(tb + step) : tq[e];
         }
       }
       // first candidate of the class at or above smax (scales ascend within a
@@ -833,7 +819,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
                                              fmaf(b1, 1.0f + 2.0f * kTieBand, prune_pad));
           if (__all_sync(0xFFFFFFFFu, done)) break;
         }
-        const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * wsc0, c0.s * wsc1, sgn, bh,
+        const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * wsc0, c0.s * wsc1, bh,
                                                   bl, pz, upper);
         track3(key_of(e0, c0.c), b1, b2, b3);
         ++ncand;
@@ -846,7 +832,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         float ug = 0.0f, ug8 = 0.0f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float v = (a[e] <= q4 ? a[e] : 0.0f) * ((e & 2) ? wsc1 : wsc0);
+          const float v = (fabsf(xs[e]) <= q4 ? xs[e] : 0.0f) * ((e & 2) ? wsc1 : wsc0);
           if ((e & 2) == 0) ug = fmaf(v, v, ug);
           else ug8 = fmaf(v, v, ug8);
         }
@@ -858,7 +844,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
                           sl2 * zero_sum * (1.0f - 2.0f * kTieBand) >
                               fmaf(b1, 1.0f + 2.0f * kTieBand, prune_pad);
         if (__all_sync(0xFFFFFFFFu, done)) break;
-        const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * wsc0, c0.s * wsc1, sgn, bh,
+        const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * wsc0, c0.s * wsc1, bh,
                                                   bl, pz, upper);
         track3(key_of(e0, c0.c), b1, b2, b3);
         ++ncand;
@@ -880,10 +866,12 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       if (amax_row == 0.0f) {  // all-zero row: every candidate scores exactly 0
         code = 1;
         obj = 0.0f;
-      } else if (!by_class) {
+      } else if (!by_class || __uint_as_float(m << 16) > 0x1p100f * s_g) {
         // s_g outside [2^-100, 2^100): the per-candidate fp32 reciprocals can
-        // leave the normal range, so the screen only orders; every candidate
-        // is re-scored in fp64
+        // leave the normal range; or a tile value above 2^100 s_g (a tensor
+        // scale far below the weights' own, amax / 2688): the class
+        // quotients w / S can overflow fp32.  The screen then only orders,
+        // and every candidate is re-scored in fp64.
         need = 2;
       } else if (kLH) {
         // both candidates' screen errors: kTieBand b + 2 Q sqrt(b) + 6 Q^2

@@ -609,6 +609,31 @@ def test_extreme_tensor_scales_every_rule(nv, e):
     assert nv.get_device_status() == "NVFP4_OK"
 
 
+def test_searches_with_a_tensor_scale_far_below_the_weights(nv):
+    """A caller-supplied tensor scale far below amax / 2688 (2^-99 for
+    weights up to 2^61): rows of ordinary size take the screen's class path,
+    rows whose values pass 2^100 s_g (their class quotients would overflow
+    fp32) send their tiles to the exact fp64 re-score.  Every block of both
+    searches against the oracle."""
+    g = torch.Generator().manual_seed(31)
+    R, C = 300, 64
+    W = torch.randn(R, C, generator=g) * 0.1         # below 2^100 s_g = 2: class path
+    big = torch.randperm(R, generator=g)[:70]
+    W[big] *= 2.0 ** 63
+    W = W.to(torch.bfloat16)
+    X = torch.randn(200, C, generator=g).to(torch.bfloat16)
+    wu = bf16_bits(W)
+    sg = 2.0 ** -99
+    s_g = torch.tensor([sg], dtype=torch.float32).cuda()
+    H = torch.zeros(C // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate(X.cuda(), H)
+    H64 = H.cpu().numpy().astype(np.float64)
+    clh = nv.scale_search_local_hessian(W.cuda(), s_g, H).cpu().numpy()
+    check_search_codes(clh, oracle.scale_search_lh(wu, sg, H64)[0], wu, sg, H64)
+    cm = nv.scale_search_mse(W.cuda(), s_g).cpu().numpy()
+    check_search_codes(cm, oracle.scale_search_mse(wu, sg)[0], wu, sg)
+
+
 def test_rows_far_below_their_tile_every_search(nv):
     """Rows scaled by 2^-10, 2^-14, 2^-16 (codes down in E4M3's subnormal
     range) and 2^-40 (every candidate ties at zero) among ordinary rows:

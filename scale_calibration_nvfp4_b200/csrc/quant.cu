@@ -595,6 +595,19 @@ int sm_count() {
   return g_sm_count;
 }
 
+// CTAs per batch element for a kernel whose CTAs pay a set-up (a scale
+// table, fp64 reciprocals) before their blocks: up to eight blocks per
+// thread, so that the set-up is amortised, but never fewer than four waves
+// of resident CTAs (`resident` per SM) across the whole batch, which keeps
+// the tail short.
+int amortised_grid(int64_t batch, int64_t nblk, int resident) {
+  const int64_t need = (nblk + kThreads - 1) / kThreads;  // one block per thread
+  const int64_t by_work = (batch * nblk + 8 * kThreads - 1) / (8 * kThreads);
+  const int64_t by_waves = std::min(batch * need, (int64_t)sm_count() * resident * 4);
+  const int64_t total = std::max(by_work, by_waves);
+  return (int)std::min(std::min(need, (total + batch - 1) / batch), (int64_t)1 << 30);
+}
+
 cudaError_t launch_global_scale(const uint16_t *x, int64_t batch, int64_t n_per_batch,
                                 float *s_g, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(s_g, 0, sizeof(float) * batch, st);
@@ -627,19 +640,6 @@ cudaError_t launch_four_over_six(const uint16_t *w, int64_t batch, int64_t nblk,
   const int gx = amortised_grid(batch, nblk, 3);  // 77 registers: three CTAs per SM
   four_over_six_kernel<<<dim3(gx, (unsigned)batch), kThreads, 0, st>>>(w, nblk, s_g, codes);
   return cudaGetLastError();
-}
-
-// CTAs per batch element for a kernel whose CTAs pay a set-up (a scale
-// table, fp64 reciprocals) before their blocks: up to eight blocks per
-// thread, so that the set-up is amortised, but never fewer than four waves
-// of resident CTAs (`resident` per SM) across the whole batch, which keeps
-// the tail short.
-int amortised_grid(int64_t batch, int64_t nblk, int resident) {
-  const int64_t need = (nblk + kThreads - 1) / kThreads;  // one block per thread
-  const int64_t by_work = (batch * nblk + 8 * kThreads - 1) / (8 * kThreads);
-  const int64_t by_waves = std::min(batch * need, (int64_t)sm_count() * resident * 4);
-  const int64_t total = std::max(by_work, by_waves);
-  return (int)std::min(std::min(need, (total + batch - 1) / batch), (int64_t)1 << 30);
 }
 
 cudaError_t launch_pack(const uint16_t *w, int64_t batch, int64_t nblk, const float *s_g,

@@ -364,6 +364,55 @@ def test_search_degenerate_blocks(nv):
     assert cm[0, 0] == 1
 
 
+def test_signed_zero_weights_every_rule(nv):
+    """Weights full of signed zeros (a dequantised or pruned layer holds -0
+    wherever a negative value rounded to zero): a quarter of the entries -0,
+    some +0, rows that are all -0 or -0 but for one value, under a Gram with
+    an outlier channel and dead channels.  Every block's max, Four Over Six,
+    MSE and Local-Hessian code against the oracle, and every packed byte and
+    dequantised value.  A -0 meets a class reciprocal whose low part is
+    negative on many candidates: its class quotient is +0 and the residual
+    -0, which must leave the quotient at zero."""
+    rng = np.random.default_rng(31)
+    R, C = 512, 256
+    u = f32_to_bf16_bits((rng.standard_normal((R, C)) * 0.02).astype(np.float32))
+    pick = rng.random((R, C))
+    u = np.where(pick < 0.25, np.uint16(0x8000), u)
+    u = np.where((pick >= 0.25) & (pick < 0.30), np.uint16(0), u)
+    u[3] = 0x8000
+    u[4] = 0x8000
+    u[4, 77] = f32_to_bf16_bits(np.array([-0.03], np.float32))[0]
+    u[5, 16:32] = 0x8000
+    u = np.ascontiguousarray(u.astype(np.uint16))
+    W = dev_bf16(u)
+    s_g = nv.global_scale(W)
+    sg = s_g.item()
+    assert sg == oracle.global_scale(u)
+    X = rand_bf16((300, C), 32)
+    X[:, 40] *= 30.0
+    X[:, 16:19] = 0                 # dead channels in block 1
+    H = torch.zeros(C // 16, 16, 16, device="cuda")
+    nv.hessian_accumulate(X.cuda(), H)
+    H64 = H.cpu().numpy().astype(np.float64)
+    np.testing.assert_array_equal(nv.scale_search_max(W, s_g).cpu().numpy(),
+                                  oracle.scale_search_max(u, sg))
+    np.testing.assert_array_equal(nv.scale_search_four_over_six(W, s_g).cpu().numpy(),
+                                  oracle.scale_search_four_over_six(u, sg))
+    cm = nv.scale_search_mse(W, s_g).cpu().numpy()
+    rc, _ = oracle.scale_search_mse(u, sg)
+    check_search_codes(cm, rc, u, sg)
+    clh_dev = nv.scale_search_local_hessian(W, s_g, H)
+    clh = clh_dev.cpu().numpy()
+    rc, _ = oracle.scale_search_lh(u, sg, H64)
+    check_search_codes(clh, rc, u, sg, H64)
+    assert np.all(clh[3] == 1) and np.all(cm[3] == 1)   # all-zero rows: the smallest code
+    packed = nv.quantize_pack(W, s_g, clh_dev)
+    rp = oracle.quantize_pack(u, sg, clh)
+    np.testing.assert_array_equal(packed.cpu().numpy(), rp)
+    y = nv.dequantize(packed, clh_dev, s_g)
+    np.testing.assert_array_equal(bf16_bits(y), oracle.dequantize(rp, clh, sg))
+
+
 def test_search_ragged_rows_mixed_magnitudes(nv):
     """Every block of a ragged 600-row weight (three row groups, the last one
     partly padding) whose rows differ in magnitude by up to 10^5, with zero

@@ -363,6 +363,37 @@ def test_search_class_codes_on_every_bf16(oracle_mod, s_g, near_ratio):
         assert wrong_without_step > 0
 
 
+def test_search_step_leaves_signed_zero_at_zero():
+    """-0 at a class whose reciprocal's low part is negative: the quotient
+    comes out as +0 and the residual w - t S as -0.  The step must treat a
+    zero residual of either sign as zero: stepping +0 one float towards
+    zero gives the bit pattern 0xFFFFFFFF, a NaN, which the saturating E2M1
+    conversion turns into a non-zero code.  The case exists at ordinary
+    tensor scales, and the kernel's rule keeps both zeros at magnitude 0."""
+    hits = 0
+    for s_g in (float(np.float32(1.0 / 2688)), float(np.float32(0.0731 / 2688)), 2.0 ** -9):
+        for c, o, p in _candidates():
+            S = np.float32(np.float32(s_g) * np.float32(o))
+            R = 1.0 / float(S)
+            r_hi = np.float32(R)
+            r_lo = np.float32(R - float(r_hi))
+            if r_lo >= 0 or _certified(S):
+                continue
+            # the kernel's arithmetic in fp32: t = fma(w, r_hi, w r_lo),
+            # rho = fma(-t, S, w), for w = -0
+            w = np.float32(-0.0)
+            t = np.float32(w * r_hi) + np.float32(w * r_lo)   # -0 + +0 = +0
+            rho = np.float32(-t * S) + w                       # -0 + -0 = -0
+            assert t == 0 and not np.signbit(t) and rho == 0 and np.signbit(rho)
+            hits += 1
+            codes = _class_codes(np.array([-0.0, 0.0]), s_g, o, p)
+            assert np.all((codes & 7) == 0), (s_g, c)
+            # the stepped pattern a sign-blind test would produce
+            stepped = np.array([t], np.float32).view(np.int32) - 1
+            assert np.isnan(stepped.view(np.float32)[0])
+    assert hits > 10
+
+
 # ------------------------------------------- eigenvalue bound of the pruning
 def _cholesky16_drop(H):
     """The search kernel's 16x16 factor: fp64 right-looking Cholesky of the

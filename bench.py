@@ -18,9 +18,12 @@ of every step (its own row, a memset), so every step's search sees the
 configuration's Gram.
 
 Metric: NVFP4 blocks per second through the step (weight blocks; activation
-blocks for w4a4).  The L2 cache is flushed (a 256 MiB write) before every
-timed step, outside the step's CUDA events.  Per-row times are CUDA events on
-the launching stream.
+blocks for w4a4).  The L2 cache is flushed before every timed step, outside
+the step's CUDA events: a 256 MiB write, then a read of the same buffer, so
+that the write's dirty lines are written back before the step rather than by
+its first kernels.  The value comes from K steps timed with CUDA events at the
+step boundaries only (the launches follow one another as in use); per-row
+times come from K further steps with an event between rows.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle on a bounded sample
@@ -212,7 +215,7 @@ class Runner:
             h = L.H.numel() * 4
             pre = L.name + "." if len(self.layers) > 1 else ""
             rows.append((pre + "global_scale",
-                         lambda L=L: nv.global_scale(L.W, batch=L.B, out=L.s_g), 2 * n_w, 2))
+                         lambda L=L: nv.global_scale(L.W, batch=L.B, out=L.s_g), 2 * n_w, 3))
             if L.X is not None or L.chunks is not None:
                 # a fresh Gram every step (a torch memset, not one of ours)
                 rows.append((pre + "zero_H", lambda L=L: L.H.zero_(), h, 0))
@@ -284,7 +287,7 @@ class Runner:
                 X = self.fq_input
                 M, K, N = X.shape[0], X.shape[1], self.gemm_w.shape[0]
                 rows.append(("fake_quant", lambda: self._fq(True),
-                             FAKE_QUANT_BYTES_PER_ELEM * n_x, 3))
+                             FAKE_QUANT_BYTES_PER_ELEM * n_x, 4))
                 if X.is_cuda:
                     rows.append(("gemm", lambda: nv.gemm(self.fq_packed, self.fq_codes, self.fq_sg,
                                                           self.gw_packed, self.gw_codes,
@@ -293,9 +296,9 @@ class Runner:
                                  M * K // 2 + N * K // 2 + M * N * 2, 4))  # 2 scale layouts, alpha, GEMM
             elif self.workload == "w4a4":
                 rows.append(("fake_quant", lambda: self._fq(True),
-                             FAKE_QUANT_BYTES_PER_ELEM * n_x, 3))
+                             FAKE_QUANT_BYTES_PER_ELEM * n_x, 4))
             else:
-                rows.append(("fake_quant", lambda: self._fq(False), 6 * n_x, 3))
+                rows.append(("fake_quant", lambda: self._fq(False), 6 * n_x, 4))
         return rows
 
     def _fq_static(self):
@@ -515,11 +518,23 @@ def run_gpu(args):
         if events is not None:
             events[-1].record(stream)
 
-    for _ in range(args.warmup):
+    def flush_l2():
+        # a 256 MiB write, then a read of it: the write's dirty lines are
+        # written back here, not by the step's first kernels
         flush.zero_()
+        flush.sum()
+
+    for _ in range(args.warmup):
+        flush_l2()
         step()
     torch.cuda.synchronize()
 
+    # timed pass: events at the step boundaries only, so that the step's
+    # launches follow one another as they would in use
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    # per-row pass (after the timed one, not part of the value): an event
+    # between rows
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(rows) + 1)]
           for _ in range(args.steps)]
     clocks = ClockSampler(local) if rank == 0 else None
@@ -530,23 +545,29 @@ def run_gpu(args):
         pg.barrier()
     nvfp4.search_evaluations(reset=True)  # synchronises
     for k in range(args.steps):
-        flush.zero_()
-        step(ev[k])
+        flush_l2()
+        ev_step[k][0].record(stream)
+        step()
+        ev_step[k][1].record(stream)
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
-    clk = clocks.stop() if clocks else None
     # rows sent to the fp64 re-score, and (block, candidate) evaluations the
     # searches made, per step (the second read resets both)
     rescores = [v / args.steps for v in nvfp4.search_rescores()]
     evals = [v / args.steps for v in nvfp4.search_evaluations(reset=True)]
+    for k in range(args.steps):
+        flush_l2()
+        step(ev[k])
+    torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else None
 
     per_row = {r[0]: [] for r in rows}
     step_ms = []
     for k in range(args.steps):
         for i, r in enumerate(rows):
             per_row[r[0]].append(ev[k][i].elapsed_time(ev[k][i + 1]))
-        step_ms.append(ev[k][0].elapsed_time(ev[k][-1]))
+        step_ms.append(ev_step[k][0].elapsed_time(ev_step[k][1]))
     ms_per_step = max_over_ranks(pg, sum(step_ms)) / args.steps
     blocks = run.blocks()
     value = job_value(world, blocks, ms_per_step)
@@ -571,7 +592,10 @@ def run_gpu(args):
             "config": {"workload": args.workload, "desc": run.desc, "blocks_per_step": blocks,
                        "rows": [r[0] for r in rows],
                        "parallelism": "replicas (one per GPU)" if world > 1 else "single GPU",
-                       "cache": "L2 flushed (256 MiB write) before every timed step"},
+                       "cache": "L2 flushed before every timed step: a 256 MiB write, then a read of it "
+                                "(its dirty lines written back outside the step)",
+                       "timing": "value from K steps with CUDA events at the step boundaries; "
+                                 "per-row times from K further steps with an event between rows"},
             "roofline": make_roofline(run, kernels, pk, pk_kind, args.workload, evals[1],
                                       clk["sm_mhz"] if clk else None),
             "search_evaluated_per_block": {"mse": round(evals[0] / blocks, 2),

@@ -20,6 +20,7 @@
 #include <cmath>
 #include <mutex>
 
+#include "chained.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "../../include/nvfp4.h"
@@ -41,6 +42,7 @@ __global__ void __launch_bounds__(kHistThreads)
   extern __shared__ uint32_t sh[];
   for (int i = threadIdx.x; i < kBins; i += kHistThreads) sh[i] = 0u;
   __syncthreads();
+  chained_entry(x);  // the shared histogram was cleared before the wait
   const int64_t nv = n / 8;  // whole 8-value vectors
   const uint4 *xv = reinterpret_cast<const uint4 *>(x);
   for (int64_t i = (int64_t)blockIdx.x * kHistThreads + threadIdx.x; i < nv;
@@ -67,6 +69,7 @@ __global__ void __launch_bounds__(kHistThreads)
 // coalesced (lane l takes bins 1024 w + 32 j + l).
 __global__ void __launch_bounds__(kHistThreads)
     quantile_scale_kernel(const uint64_t *__restrict__ hist, double p, float *__restrict__ s_g) {
+  chained_entry();
   constexpr int kWarpBins = kBins / (kHistThreads / 32);  // 1024
   __shared__ unsigned long long warp_total[kHistThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -144,13 +147,12 @@ cudaError_t launch_abs_histogram(const uint16_t *x, int64_t n, uint64_t *hist, c
   int64_t ctas = (n / 8 + kHistThreads - 1) / kHistThreads;
   if (ctas > sm_count()) ctas = sm_count();
   if (ctas < 1) ctas = 1;
-  abs_histogram_kernel<<<(unsigned)ctas, kHistThreads, kHistSmem, st>>>(x, n, hist);
-  return cudaGetLastError();
+  return launch_chained(abs_histogram_kernel, dim3((unsigned)ctas), dim3(kHistThreads), kHistSmem,
+                        st, x, n, hist);
 }
 
 cudaError_t launch_quantile_scale(const uint64_t *hist, double p, float *s_g, cudaStream_t st) {
-  quantile_scale_kernel<<<1, kHistThreads, 0, st>>>(hist, p, s_g);
-  return cudaGetLastError();
+  return launch_chained(quantile_scale_kernel, dim3(1), dim3(kHistThreads), 0, st, hist, p, s_g);
 }
 
 cudaError_t read_and_clear_calib_status(cudaStream_t st, int *out) {

@@ -23,6 +23,7 @@
 #include <cutlass/gemm/kernel/gemm_universal.hpp>
 #include <cutlass/util/packed_stride.hpp>
 
+#include "chained.cuh"
 #include "internal.h"
 
 namespace nvfp4 {
@@ -73,6 +74,7 @@ using ScaleConfig = typename CollectiveMainloop::Sm1xxBlkScaledConfig;
 template <class Layout>
 __global__ void scale_layout_kernel(const uint8_t *__restrict__ src, int64_t rows, int64_t kb,
                                     Layout layout, uint8_t *__restrict__ dst) {
+  chained_entry();
   const int64_t n = rows * kb;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -81,7 +83,10 @@ __global__ void scale_layout_kernel(const uint8_t *__restrict__ src, int64_t row
   }
 }
 
-__global__ void product_kernel(const float *a, const float *b, float *out) { *out = *a * *b; }
+__global__ void product_kernel(const float *a, const float *b, float *out) {
+  chained_entry();
+  *out = *a * *b;
+}
 
 int grid_for_elems(int64_t n) {
   const int64_t cap = (int64_t)sm_count() * 8;
@@ -126,12 +131,15 @@ cudaError_t launch_gemm_fp4(const uint8_t *a_packed, const uint8_t *a_codes, con
   // padding of the scale atoms must hold zero scales (never NaN codes)
   e = cudaMemsetAsync(sfa, 0, off_ws - off_sfa, st);
   if (e == cudaSuccess) {
-    scale_layout_kernel<<<grid_for_elems(M * (K / 16)), 256, 0, st>>>(a_codes, M, K / 16, lsfa,
-                                                                       sfa);
-    scale_layout_kernel<<<grid_for_elems(N * (K / 16)), 256, 0, st>>>(b_codes, N, K / 16, lsfb,
-                                                                       sfb);
-    product_kernel<<<1, 1, 0, st>>>(a_sg, b_sg, alpha);
-    e = cudaGetLastError();
+    // (the CUTLASS GEMM below is launched plainly: its own grid-dependency
+    // wait is compiled only where CUTLASS enables it)
+    e = launch_chained(scale_layout_kernel<LayoutSFA>, dim3(grid_for_elems(M * (K / 16))),
+                       dim3(256), 0, st, a_codes, M, K / 16, lsfa, sfa);
+    if (e == cudaSuccess)
+      e = launch_chained(scale_layout_kernel<LayoutSFB>, dim3(grid_for_elems(N * (K / 16))),
+                         dim3(256), 0, st, b_codes, N, K / 16, lsfb, sfb);
+    if (e == cudaSuccess)
+      e = launch_chained(product_kernel, dim3(1), dim3(1), 0, st, a_sg, b_sg, alpha);
   }
   if (e == cudaSuccess) {
     args.mainloop.ptr_SFA = reinterpret_cast<typename ElementA::ScaleFactorType const *>(sfa);

@@ -36,6 +36,7 @@
 #include <cmath>
 #include <mutex>
 
+#include "chained.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "../../include/nvfp4.h"
@@ -110,6 +111,9 @@ __global__ void __launch_bounds__(kGThreads, BN == 64 ? 2 : 1) gemm_f64_kernel(c
   constexpr int kBCopies = kGN * kGK / kGThreads;
   const int64_t m0 = (int64_t)blockIdx.y * kGM, n0 = (int64_t)blockIdx.x * kGN;
   if (g.lower && n0 > m0 + kGM - 1) return;
+  // operands arrive by cp.async (volatile asm, kept after the wait) and
+  // ordinary loads
+  chained_entry();
   const int64_t z = blockIdx.z;
   const double *A = g.A + z * g.bsA;
   const double *B = g.B + z * g.bsB;
@@ -221,8 +225,7 @@ template <int BN>
 cudaError_t gemm_launch(const GemmF64 &g, int64_t batch, cudaStream_t st) {
   const dim3 grid((unsigned)((g.N + BN - 1) / BN), (unsigned)((g.M + kGM - 1) / kGM),
                   (unsigned)batch);
-  gemm_f64_kernel<BN><<<grid, kGThreads, gemm_smem<BN>(), st>>>(g);
-  return cudaGetLastError();
+  return launch_chained(gemm_f64_kernel<BN>, grid, dim3(kGThreads), gemm_smem<BN>(), st, g);
 }
 
 // An in-place product (C aliasing A, `overwrite`) must run as one CTA column
@@ -281,6 +284,7 @@ constexpr int kCholSmem = (kBig * kSRow + 4 * kBig) * (int)sizeof(double);  // 1
 
 __global__ void __launch_bounds__(kCholThreads, 1)
     chol_block_kernel(double *A, int64_t C, int64_t P0, int nw, double *Linv) {
+  chained_entry();
   extern __shared__ double csm[];
   double *Lsm = csm;                 // [kBig][kSRow], the factor
   double *vec = Lsm + kBig * kSRow;  // [2][kBig] column (factor) / row (inverse) of step k
@@ -452,8 +456,8 @@ cudaError_t cholesky_in_place(double *A, int64_t C, int64_t batch, double *Linv,
   };
   for (int64_t P0 = 0; e == cudaSuccess && P0 < C; P0 += kBig) {
     const int nw = (int)(C - P0 < kBig ? C - P0 : kBig);
-    chol_block_kernel<<<(unsigned)batch, kCholThreads, kCholSmem, st>>>(A, C, P0, nw, Linv);
-    e = cudaGetLastError();
+    e = launch_chained(chol_block_kernel, dim3((unsigned)batch), dim3(kCholThreads), kCholSmem, st,
+                       A, C, P0, nw, Linv);
     const int64_t P1 = P0 + nw, rest = C - P1;
     if (e != cudaSuccess || rest <= 0) break;
     {
@@ -493,6 +497,7 @@ cudaError_t cholesky_in_place(double *A, int64_t C, int64_t batch, double *Linv,
 // lambda = damp * mean(diag H), the diagonal summed in a fixed order.
 __global__ void __launch_bounds__(32)
     gptq_lambda_kernel(const float *H, int64_t C, double damp, double *lam) {
+  chained_entry();
   const float *Hb = H + (int64_t)blockIdx.x * C * C;
   double s = 0.0;
   for (int64_t i = threadIdx.x; i < C; i += 32) s += (double)Hb[i * C + i];
@@ -504,6 +509,7 @@ __global__ void __launch_bounds__(32)
 // Hd[i][j] = H[C-1-i][C-1-j] + lambda [i == j], in fp64 (lower triangle).
 __global__ void __launch_bounds__(256)
     gptq_prepare_kernel(const float *H, int64_t C, const double *lam, double *Hd) {
+  chained_entry();
   const int64_t b = blockIdx.y;
   const float *Hb = H + b * C * C;
   double *Db = Hd + b * C * C;
@@ -550,6 +556,7 @@ __global__ void __launch_bounds__(kBlockThreads)
                       const float *__restrict__ s_g, const uint8_t *__restrict__ codes,
                       const double *__restrict__ L, double *__restrict__ SD,
                       uint8_t *__restrict__ packed, int64_t c0, int nw) {
+  chained_entry();
   extern __shared__ double bsm[];
   double *T = bsm;              // [j][k], j <= k
   double *Tinv = T + kBig * kBig;  // 1 / T[k][k]
@@ -652,12 +659,13 @@ cudaError_t launch_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
   double *Linv = reinterpret_cast<double *>(scratch + lam_bytes + hd_bytes + sd_bytes);
   e = cudaMemsetAsync(SD, 0, sd_bytes, st);
   if (e == cudaSuccess) {
-    gptq_lambda_kernel<<<(unsigned)batch, 32, 0, st>>>(H, C, damp, lam);
+    e = launch_chained(gptq_lambda_kernel, dim3((unsigned)batch), dim3(32), 0, st, H, C, damp, lam);
     const int64_t n = C * C;
     int64_t gx = (n + 255) / 256;
     if (gx > (int64_t)sm_count() * 8) gx = (int64_t)sm_count() * 8;
-    gptq_prepare_kernel<<<dim3((unsigned)gx, (unsigned)batch), 256, 0, st>>>(H, C, lam, Hd);
-    e = cudaGetLastError();
+    if (e == cudaSuccess)
+      e = launch_chained(gptq_prepare_kernel, dim3((unsigned)gx, (unsigned)batch), dim3(256), 0,
+                         st, H, C, static_cast<const double *>(lam), Hd);
   }
   if (e == cudaSuccess) e = cholesky_in_place(Hd, C, batch, Linv, st);
   // columns in blocks of 128: each row of a block on a quad of lanes, then the
@@ -668,9 +676,8 @@ cudaError_t launch_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
   for (int64_t c0 = 0; e == cudaSuccess && c0 < C; c0 += kBig) {
     const int nw = (int)(C - c0 < kBig ? C - c0 : kBig);
     const dim3 grid((unsigned)((R + kRowsPerCta - 1) / kRowsPerCta), (unsigned)batch);
-    gptq_block_kernel<<<grid, kBlockThreads, kBlockSmem, st>>>(w, R, C, s_g, codes, Hd, SD,
-                                                                packed, c0, nw);
-    e = cudaGetLastError();
+    e = launch_chained(gptq_block_kernel, grid, dim3(kBlockThreads), kBlockSmem, st, w, R, C, s_g,
+                       codes, static_cast<const double *>(Hd), SD, packed, c0, nw);
     const int64_t c1 = c0 + nw;
     if (e == cudaSuccess && c1 < C) {
       // SD[:, c1:] += SD[:, c0:c1] T[c0:c1, c1:], T[i][j] = Hd[C-1-i][C-1-j]

@@ -31,6 +31,7 @@
 
 #include <cuda.h>
 
+#include "chained.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "../../include/nvfp4.h"
@@ -151,6 +152,7 @@ __global__ void __launch_bounds__(kGramThreads)
     gram_partial_kernel(const __grid_constant__ CUtensorMap tmap, int64_t C,
                         const ItemRange *items, const int64_t *n_items_dev, int64_t n_tok,
                         int64_t per_item, float *__restrict__ partial) {
+  chained_entry();
   extern __shared__ unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t full[kStages];
   const int64_t nb = C / kBlock;
@@ -281,6 +283,7 @@ __global__ void wait_timeout_probe_kernel() {
 __global__ void gram_reduce_kernel(const float *__restrict__ partial, int64_t nb, int64_t G,
                                    const int64_t *__restrict__ item_start, int64_t n_items_uniform,
                                    float *__restrict__ H) {
+  chained_entry();
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over G * nb * 256
   const int64_t per_group = nb * 256;
   if (idx >= G * per_group) return;
@@ -303,6 +306,7 @@ __global__ void build_items_kernel(const int64_t *__restrict__ offsets, int64_t 
                                    int64_t per_item, int64_t max_items,
                                    int64_t *__restrict__ item_start, ItemRange *__restrict__ items,
                                    int64_t *__restrict__ n_items) {
+  chained_entry();
   __shared__ int64_t warp_sums[32];
   __shared__ int64_t carry;
   if (threadIdx.x == 0) carry = 0;
@@ -437,13 +441,13 @@ cudaError_t gram_uniform(const uint16_t *x, int64_t n_tok, int64_t C, float *H, 
   CUtensorMap tmap;
   cudaError_t e = make_x_tensor_map(x, n_tok, C, &tmap);
   if (e != cudaSuccess) return e;
-  gram_partial_kernel<<<dim3((unsigned)items, (unsigned)ngroups), kGramThreads, kGramSmem, st>>>(
-      tmap, C, nullptr, nullptr, n_tok, per_item, partial);
-  e = cudaGetLastError();
+  e = launch_chained(gram_partial_kernel, dim3((unsigned)items, (unsigned)ngroups),
+                     dim3(kGramThreads), kGramSmem, st, tmap, C, nullptr, nullptr, n_tok, per_item,
+                     partial);
   if (e != cudaSuccess) return e;
-  gram_reduce_kernel<<<(unsigned)((per_group + 255) / 256), 256, 0, st>>>(partial, nb, 1, nullptr,
-                                                                          items, H);
-  return cudaGetLastError();
+  return launch_chained(gram_reduce_kernel, dim3((unsigned)((per_group + 255) / 256)), dim3(256),
+                        0, st, static_cast<const float *>(partial), nb, (int64_t)1, nullptr, items,
+                        H);
 }
 
 }  // namespace
@@ -491,20 +495,17 @@ cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, in
   int64_t *n_items = item_start + G + 1;
   ItemRange *items = reinterpret_cast<ItemRange *>(ws + off_items);
   float *partial = reinterpret_cast<float *>(ws + off_part);
-  build_items_kernel<<<1, 1024, 0, st>>>(offsets, G, n_tok, per_item, max_items, item_start,
-                                         items, n_items);
-  e = cudaGetLastError();
-  if (e == cudaSuccess) {
-    gram_partial_kernel<<<dim3((unsigned)max_items, (unsigned)ngroups), kGramThreads, kGramSmem,
-                          st>>>(tmap, C, items, n_items, n_tok, per_item, partial);
-    e = cudaGetLastError();
-  }
-  if (e == cudaSuccess) {
-    const int64_t n = G * per_group;
-    gram_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, nb, G, item_start,
-                                                                    0, H);
-    e = cudaGetLastError();
-  }
+  e = launch_chained(build_items_kernel, dim3(1), dim3(1024), 0, st, offsets, G, n_tok, per_item,
+                     max_items, item_start, items, n_items);
+  if (e == cudaSuccess)
+    e = launch_chained(gram_partial_kernel, dim3((unsigned)max_items, (unsigned)ngroups),
+                       dim3(kGramThreads), kGramSmem, st, tmap, C,
+                       static_cast<const ItemRange *>(items), static_cast<const int64_t *>(n_items),
+                       n_tok, per_item, partial);
+  if (e == cudaSuccess)
+    e = launch_chained(gram_reduce_kernel, dim3((unsigned)((G * per_group + 255) / 256)),
+                       dim3(256), 0, st, static_cast<const float *>(partial), nb, G,
+                       static_cast<const int64_t *>(item_start), (int64_t)0, H);
   cudaError_t e2 = scratch_free(ws, st);
   return e != cudaSuccess ? e : e2;
 }

@@ -9,6 +9,7 @@
 // "為什么NVFP4推理精度會掉以及QAD到底在修什么" (2.1, 2.3, 3.2, 4.2).
 #include <algorithm>
 
+#include "chained.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "../../include/nvfp4.h"
@@ -32,6 +33,7 @@ constexpr uint32_t kMagMask = 0x7FFF7FFFu;
 __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t *__restrict__ x,
                                                         int64_t n_per_batch,
                                                         uint32_t *__restrict__ amax_bits) {
+  chained_entry(x);
   const int64_t b = blockIdx.y;
   const uint4 *xb = reinterpret_cast<const uint4 *>(x + b * n_per_batch);
   const int64_t nv = n_per_batch / 8;
@@ -70,9 +72,17 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t *__restri
   }
 }
 
+// n words set to zero
+__global__ void zero_words_kernel(uint32_t *p, int64_t n) {
+  chained_entry();
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = 0u;
+}
+
 // s_g = fl32(amax / 2688), 1 for amax = 0, NaN (and a NONFINITE report) when
 // the tensor held NaN/Inf.  The amax bits were accumulated in place.
 __global__ void global_scale_finish_kernel(float *s_g, int64_t batch) {
+  chained_entry();
   const int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= batch) return;
   const uint32_t bits = reinterpret_cast<const uint32_t *>(s_g)[b];
@@ -123,11 +133,12 @@ __device__ __forceinline__ uint32_t cvt4_e2m1(float h0, float l0, float h1, floa
 }
 
 // Adjacent float of t towards the side given by the residual (same sign as
-// q - t); t itself when the residual is zero (q == t exactly).
+// q - t); t itself when the residual is zero (q == t exactly), of either sign
+// (t = +0 with rho = -0 must not step towards zero into a NaN).
 __device__ __forceinline__ float toward(float t, float rho) {
   const int rb = __float_as_int(rho);
   const int dir = ((rb ^ __float_as_int(t)) >> 31) | 1;  // +1 away from 0, -1 towards
-  return __int_as_float(__float_as_int(t) + (rb != 0 ? dir : 0));
+  return __int_as_float(__float_as_int(t) + ((__float_as_uint(rho) << 1) != 0u ? dir : 0));
 }
 
 // Packed signed E2M1 codes of 8 consecutive elements (4 bf16 pairs) at scale
@@ -288,6 +299,7 @@ __global__ void __launch_bounds__(kThreads) max_rule_kernel(const uint16_t *__re
                                                             int64_t nblk,
                                                             const float *__restrict__ s_g,
                                                             uint8_t *__restrict__ codes) {
+  chained_entry(w);
   const int64_t b = blockIdx.y;
   const MaxRule mr = make_max_rule(s_g[b]);
   w += b * nblk * kBlock;
@@ -390,6 +402,7 @@ __global__ void __launch_bounds__(kThreads) four_over_six_kernel(const uint16_t 
                                                                  int64_t nblk,
                                                                  const float *__restrict__ s_g,
                                                                  uint8_t *__restrict__ codes) {
+  chained_entry(w);
   const int64_t b = blockIdx.y;
   w += b * nblk * kBlock;
   codes += b * nblk;
@@ -433,6 +446,7 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const uint16_t *__restri
                                                         const float *__restrict__ s_g,
                                                         const uint8_t *__restrict__ codes,
                                                         uint8_t *__restrict__ packed) {
+  chained_entry(w);
   const int64_t b = blockIdx.y;
   w += b * nblk * kBlock;
   codes += b * nblk;
@@ -469,6 +483,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t *__rest
                                                            const float *__restrict__ s_g,
                                                            int64_t nblk,
                                                            uint16_t *__restrict__ out) {
+  chained_entry(packed);
   const int64_t b = blockIdx.y;
   const float sg = s_g[b];
   packed += b * nblk * (kBlock / 2);
@@ -492,6 +507,7 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__
                                                               uint16_t *__restrict__ out,
                                                               uint8_t *__restrict__ packed,
                                                               uint8_t *__restrict__ codes) {
+  chained_entry(x);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   uint32_t v[8];
@@ -528,6 +544,7 @@ __global__ void __launch_bounds__(kThreads) quant_error_kernel(const uint16_t *_
                                                                int64_t nblk,
                                                                const float *__restrict__ s_g,
                                                                double *__restrict__ partial) {
+  chained_entry(x);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   uint32_t v[8];
@@ -568,6 +585,7 @@ __global__ void __launch_bounds__(kThreads) quant_error_kernel(const uint16_t *_
 
 __global__ void error_reduce_kernel(const double *__restrict__ partial, int n,
                                     double *__restrict__ out) {
+  chained_entry();
   double t = 0.0;
   for (int i = 0; i < n; ++i) t += partial[i];
   *out = t;
@@ -610,53 +628,54 @@ int amortised_grid(int64_t batch, int64_t nblk, int resident) {
 
 cudaError_t launch_global_scale(const uint16_t *x, int64_t batch, int64_t n_per_batch,
                                 float *s_g, cudaStream_t st) {
-  cudaError_t e = cudaMemsetAsync(s_g, 0, sizeof(float) * batch, st);
+  // the maxima are accumulated by atomicMax from zero (a kernel rather than a
+  // memset, so that the launches stay chained)
+  cudaError_t e = launch_chained(zero_words_kernel, dim3((unsigned)((batch + 127) / 128)),
+                                 dim3(128), 0, st, reinterpret_cast<uint32_t *>(s_g), batch);
   if (e != cudaSuccess) return e;
   if (n_per_batch > 0) {
     const int64_t nv = n_per_batch / 8;
     int gx = grid_for(nv / 4 + 1, 8);
     const int64_t per_batch_cap = ((int64_t)sm_count() * 8 + batch - 1) / batch;
     if (gx > per_batch_cap) gx = (int)(per_batch_cap > 0 ? per_batch_cap : 1);
-    amax_kernel<<<dim3(gx, (unsigned)batch), kThreads, 0, st>>>(
-        x, n_per_batch, reinterpret_cast<uint32_t *>(s_g));
-    e = cudaGetLastError();
+    e = launch_chained(amax_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st, x,
+                       n_per_batch, reinterpret_cast<uint32_t *>(s_g));
     if (e != cudaSuccess) return e;
   }
-  global_scale_finish_kernel<<<(unsigned)((batch + 127) / 128), 128, 0, st>>>(s_g, batch);
-  return cudaGetLastError();
+  return launch_chained(global_scale_finish_kernel, dim3((unsigned)((batch + 127) / 128)),
+                        dim3(128), 0, st, s_g, batch);
 }
 
 cudaError_t launch_scale_max(const uint16_t *w, int64_t batch, int64_t nblk, const float *s_g,
                              uint8_t *codes, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   int gx = grid_for(nblk, 16);
-  max_rule_kernel<<<dim3(gx, (unsigned)batch), kThreads, 0, st>>>(w, nblk, s_g, codes);
-  return cudaGetLastError();
+  return launch_chained(max_rule_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st, w,
+                        nblk, s_g, codes);
 }
 
 cudaError_t launch_four_over_six(const uint16_t *w, int64_t batch, int64_t nblk,
                                  const float *s_g, uint8_t *codes, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   const int gx = amortised_grid(batch, nblk, 3);  // 77 registers: three CTAs per SM
-  four_over_six_kernel<<<dim3(gx, (unsigned)batch), kThreads, 0, st>>>(w, nblk, s_g, codes);
-  return cudaGetLastError();
+  return launch_chained(four_over_six_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st,
+                        w, nblk, s_g, codes);
 }
 
 cudaError_t launch_pack(const uint16_t *w, int64_t batch, int64_t nblk, const float *s_g,
                         const uint8_t *codes, uint8_t *packed, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   const int gx = amortised_grid(batch, nblk, 5);
-  pack_kernel<<<dim3(gx, (unsigned)batch), kThreads, 0, st>>>(w, nblk, s_g, codes, packed);
-  return cudaGetLastError();
+  return launch_chained(pack_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st, w, nblk,
+                        s_g, codes, packed);
 }
 
 cudaError_t launch_dequant(const uint8_t *packed, const uint8_t *codes, const float *s_g,
                            int64_t batch, int64_t nblk, uint16_t *out, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   int gx = grid_for(nblk, 16);
-  dequant_kernel<<<dim3(gx, (unsigned)batch), kThreads, 0, st>>>(packed, codes, s_g, nblk,
-                                                                  out);
-  return cudaGetLastError();
+  return launch_chained(dequant_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st, packed,
+                        codes, s_g, nblk, out);
 }
 
 cudaError_t launch_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16_t *out,
@@ -666,8 +685,8 @@ cudaError_t launch_fake_quant(const uint16_t *x, int64_t rows, int64_t C, uint16
   if (e != cudaSuccess || n == 0) return e;
   const int64_t nblk = n / kBlock;
   int gx = grid_for(nblk, 16);
-  fake_quant_kernel<<<gx, kThreads, 0, st>>>(x, nblk, s_g, out, packed, codes);
-  return cudaGetLastError();
+  return launch_chained(fake_quant_kernel, dim3(gx), dim3(kThreads), 0, st, x, nblk,
+                        static_cast<const float *>(s_g), out, packed, codes);
 }
 
 cudaError_t launch_fake_quant_static(const uint16_t *x, int64_t rows, int64_t C, const float *s_g,
@@ -676,8 +695,8 @@ cudaError_t launch_fake_quant_static(const uint16_t *x, int64_t rows, int64_t C,
   const int64_t nblk = rows * C / kBlock;
   if (nblk == 0) return cudaSuccess;
   const int gx = grid_for(nblk, 16);
-  fake_quant_kernel<<<gx, kThreads, 0, st>>>(x, nblk, s_g, out, packed, codes);
-  return cudaGetLastError();
+  return launch_chained(fake_quant_kernel, dim3(gx), dim3(kThreads), 0, st, x, nblk, s_g, out,
+                        packed, codes);
 }
 
 cudaError_t launch_quant_error(const uint16_t *x, int64_t rows, int64_t C, const float *s_g,
@@ -688,9 +707,10 @@ cudaError_t launch_quant_error(const uint16_t *x, int64_t rows, int64_t C, const
   double *partial = nullptr;
   cudaError_t e = scratch_alloc(reinterpret_cast<void **>(&partial), sizeof(double) * gx, st);
   if (e != cudaSuccess) return e;
-  quant_error_kernel<<<gx, kThreads, 0, st>>>(x, nblk, s_g, partial);
-  error_reduce_kernel<<<1, 1, 0, st>>>(partial, gx, err);
-  e = cudaGetLastError();
+  e = launch_chained(quant_error_kernel, dim3(gx), dim3(kThreads), 0, st, x, nblk, s_g, partial);
+  if (e == cudaSuccess)
+    e = launch_chained(error_reduce_kernel, dim3(1), dim3(1), 0, st,
+                       static_cast<const double *>(partial), gx, err);
   const cudaError_t ef = scratch_free(partial, st);
   return e != cudaSuccess ? e : ef;
 }

@@ -67,6 +67,7 @@
 // and only the relative error of the sums is left (Q = 0).
 #include <cuda_fp16.h>
 
+#include "chained.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -428,6 +429,7 @@ __device__ __forceinline__ double factor_residual(const float *Hs, const double 
 __global__ void __launch_bounds__(32)
     factor_kernel(const float *__restrict__ H, int64_t nb, uint4 *__restrict__ frag,
                   Factor *__restrict__ fac) {
+  chained_entry();
   __shared__ float Hs[2][256];
   __shared__ float Lf[2][256];
   __shared__ double Ld[2][256];
@@ -521,35 +523,26 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
   __shared__ uint4 Ws[kRowsPerCta][2];     // the CTA's 16-element row segments
   __shared__ uint32_t keys[kRowsPerCta];  // amax << 16 | local row, sorted
 
+  // Chained launch.  MSE: wait for the previous kernel before anything.
+  // Local-Hessian: the previous kernel on the stream is always this call's
+  // factor kernel, which neither reads nor writes W, s_g, codes or best_obj
+  // and released its dependents only after its own wait (all earlier work
+  // on the stream has completed): the rows are loaded and sorted while it
+  // finishes, and the wait comes before the first read of its output.
+  if constexpr (!kLH) chained_entry(w);
   const float s_g = s_g_arr[batch];
   const uint16_t *wb = w + batch * R * C + b * kBlock;
   uint8_t *cb = codes + batch * R * nb + b;
   float *ob = best_obj ? best_obj + batch * R * nb + b : nullptr;
 
-  // ---- factor of H_b (from factor_kernel) and the zero-H shortcut
+  // ---- the product's B operand: B = I for MSE here; the Local-Hessian factor
+  // of H_b (from factor_kernel) and its zero-H shortcut come after the sort
   const int64_t blk = batch * nb + b;
-  const float *Hb = kLH ? H + blk * 256 : nullptr;  // the definition, for re-scoring
+  const float *Hb = nullptr;  // H_b, the definition, for re-scoring (Local-Hessian)
   float sigma = 1.0f, sl2 = 1.0f;  // MSE: H = I
   float rsq = 0.0f;                // 12 sqrt(sigma^2 ||H - L L^T||_inf) (Local-Hessian)
   uint32_t bh[2][2], bl[2][2];
-  if (kLH) {
-    const Factor f = fac[blk];
-    if (f.zero) {  // every candidate scores 0: the smallest code wins
-      const int64_t r_end = min(R, row_base + kRowsPerCta);
-      for (int64_t r = row_base + threadIdx.x; r < r_end; r += kThreads) {
-        cb[r * nb] = 1;
-        if (ob) ob[r * nb] = 0.0f;
-      }
-      return;
-    }
-    sigma = f.sigma;
-    sl2 = f.sl2;
-    rsq = f.rsq;
-    if (threadIdx.x < 16) cdiag_sh[threadIdx.x] = fac[blk].cs[threadIdx.x];
-    const uint4 h = frag[(blk * 32 + lane) * 2], l = frag[(blk * 32 + lane) * 2 + 1];
-    bh[0][0] = h.x; bh[0][1] = h.y; bh[1][0] = h.z; bh[1][1] = h.w;
-    bl[0][0] = l.x; bl[0][1] = l.y; bl[1][0] = l.z; bl[1][1] = l.w;
-  } else {
+  if (!kLH) {
     if (threadIdx.x < 16) cdiag_sh[threadIdx.x] = 1.0f;  // H = I
     // B = I: u = v exactly
 #pragma unroll
@@ -643,6 +636,28 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       }
       __syncthreads();
     }
+  }
+
+  if constexpr (kLH) {
+    chained_entry();
+    Hb = H + blk * 256;
+    const Factor f = fac[blk];
+    if (f.zero) {  // every candidate scores 0: the smallest code wins
+      const int64_t r_end = min(R, row_base + kRowsPerCta);
+      for (int64_t r = row_base + threadIdx.x; r < r_end; r += kThreads) {
+        cb[r * nb] = 1;
+        if (ob) ob[r * nb] = 0.0f;
+      }
+      return;
+    }
+    sigma = f.sigma;
+    sl2 = f.sl2;
+    rsq = f.rsq;
+    if (threadIdx.x < 16) cdiag_sh[threadIdx.x] = fac[blk].cs[threadIdx.x];
+    const uint4 h = frag[(blk * 32 + lane) * 2], l = frag[(blk * 32 + lane) * 2 + 1];
+    bh[0][0] = h.x; bh[0][1] = h.y; bh[1][0] = h.z; bh[1][1] = h.w;
+    bl[0][0] = l.x; bl[0][1] = l.y; bl[1][0] = l.z; bl[1][1] = l.w;
+    __syncthreads();  // cdiag_sh
   }
 
   unsigned long long evals = 0;
@@ -798,7 +813,10 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         for (int e = 0; e < 8; ++e) {
           const float rho = fmaf(-tq[e], ci.S, xs[e]);
           const int rb = __float_as_int(rho), tb = __float_as_int(tq[e]);
-          const int step = rb != 0 ? (((rb ^ tb) >> 31) | 1) : 0;
+          // no step for a zero residual of either sign: w = -0 with r_lo < 0
+          // gives t = +0 and rho = -0, and stepping +0 towards zero would
+          // make a NaN
+          const int step = (__float_as_uint(rho) << 1) != 0u ? (((rb ^ tb) >> 31) | 1) : 0;
           const bool near = (tb & 0x1FFFFF) == 0;
           tq[e] = near ? __int_as_float(tb + step) : tq[e];
         }
@@ -974,13 +992,10 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
   const int rows = small ? kRowsSmall : kRowsLarge;
   dim3 grid((unsigned)((R + rows - 1) / rows), (unsigned)(C / kBlock), (unsigned)batch);
   if (!local_hessian) {
-    if (small)
-      search_kernel<false, kRowsSmall><<<grid, kThreads, 0, st>>>(w, R, C, s_g, nullptr, nullptr,
-                                                                  nullptr, codes, best_obj);
-    else
-      search_kernel<false, kRowsLarge><<<grid, kThreads, 0, st>>>(w, R, C, s_g, nullptr, nullptr,
-                                                                  nullptr, codes, best_obj);
-    return cudaGetLastError();
+    return launch_chained(small ? search_kernel<false, kRowsSmall>
+                                : search_kernel<false, kRowsLarge>,
+                          grid, dim3(kThreads), 0, st, w, R, C, s_g, nullptr, nullptr, nullptr,
+                          codes, best_obj);
   }
   // factors of every H_b first (stream-ordered scratch, freed after the search)
   const int64_t nblocks = batch * (C / kBlock);
@@ -991,17 +1006,15 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
   uint4 *frag = static_cast<uint4 *>(scratch);
   Factor *fac = reinterpret_cast<Factor *>(static_cast<char *>(scratch) + frag_bytes);
   const int64_t nb = C / kBlock;
-  factor_kernel<<<dim3((unsigned)((nb + 1) / 2), (unsigned)batch), 32, 0, st>>>(H, nb, frag, fac);
-  e = cudaGetLastError();
-  if (e == cudaSuccess) {
-    if (small)
-      search_kernel<true, kRowsSmall><<<grid, kThreads, 0, st>>>(w, R, C, s_g, H, frag, fac,
-                                                                 codes, best_obj);
-    else
-      search_kernel<true, kRowsLarge><<<grid, kThreads, 0, st>>>(w, R, C, s_g, H, frag, fac,
-                                                                 codes, best_obj);
-    e = cudaGetLastError();
-  }
+  // the search kernel reads W and s_g before waiting for the factor kernel
+  // (see its prologue): nothing may come between the two launches
+  e = launch_chained(factor_kernel, dim3((unsigned)((nb + 1) / 2), (unsigned)batch), dim3(32), 0,
+                     st, H, nb, frag, fac);
+  if (e == cudaSuccess)
+    e = launch_chained(small ? search_kernel<true, kRowsSmall> : search_kernel<true, kRowsLarge>,
+                       grid, dim3(kThreads), 0, st, w, R, C, s_g, H,
+                       static_cast<const uint4 *>(frag), static_cast<const Factor *>(fac), codes,
+                       best_obj);
   const cudaError_t ef = scratch_free(scratch, st);
   return e != cudaSuccess ? e : ef;
 }

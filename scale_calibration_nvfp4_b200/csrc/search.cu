@@ -804,21 +804,21 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       for (int e = 0; e < 8; ++e) tq[e] = fmaf(xs[e], ci.r_hi, xs[e] * ci.r_lo);
       // uncertified classes: a quotient with at most 3 significant bits
       // (every rounding midpoint is one, and so is every power-of-two
-      // multiple) steps to its neighbouring float across q, by the exact
-      // sign of the residual w - t S (away from zero when it has t's sign);
-      // t itself when q == t.  Every other t is not a midpoint at any scale of
-      // the class and rounds like q.
+      // multiple) moves towards q = w / S: v = t + rho (16 / S), rounded
+      // once, with the exact residual rho = w - t S.  For such a t a non-zero
+      // residual lies between 2^-27 |q| S and one float of q times S (w has 8
+      // significant bits, t S at most 27), so v lands at least one float and
+      // at most 2^-19 |q| from t on q's side: off the midpoint, and short of
+      // any other rounding decision (at least 4% away).  A zero residual of
+      // either sign leaves t.  Every other t is not a midpoint at any scale
+      // of the class and rounds like q.
       if (!ci.certified) {
+        const float r16 = 16.0f * ci.r_hi;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float rho = fmaf(-tq[e], ci.S, xs[e]);
-          const int rb = __float_as_int(rho), tb = __float_as_int(tq[e]);
-          // no step for a zero residual of either sign: w = -0 with r_lo < 0
-          // gives t = +0 and rho = -0, and stepping +0 towards zero would
-          // make a NaN
-          const int step = (__float_as_uint(rho) << 1) != 0u ? (((rb ^ tb) >> 31) | 1) : 0;
-          const bool near = (tb & 0x1FFFFF) == 0;
-          tq[e] = near ? __int_as_float(tb + step) : tq[e];
+          const bool near = (__float_as_uint(tq[e]) & 0x1FFFFFu) == 0u;
+          tq[e] = near ? fmaf(rho, r16, tq[e]) : tq[e];
         }
       }
       // first candidate of the class at or above smax (scales ascend within a

@@ -291,10 +291,15 @@ def _class_codes(a, s_g, o, p, step=True):
     candidate o 2^p, the search kernel's way: S = fl32(s_g o), R = fl64(1/S)
     split r_hi = fl32(R), r_lo = fl32(R - r_hi); t = fl32(a r_hi + fl32(a
     r_lo)), signed; for an uncertified S a t with 21 zero low mantissa bits
-    steps across a / S (one float away from zero when the residual a - t S
-    has t's sign bit, towards zero when not, not at all when it is 0); then
-    nearest-even of t 2^-p, the sign kept (-0 for negative values that round
-    to zero)."""
+    moves towards a / S: v = fl32(t + rho 16 r_hi) with the residual rho =
+    fl32(a - t S) (zero of either sign leaves t); then nearest-even of t
+    2^-p, the sign kept (-0 for negative values that round to zero).
+
+    Where the step applies and rho is not zero, v must lie at least one float
+    and at most 2^-19 |q| from t on q's side (the kernel's argument: such a t
+    has at most 3 significant bits, so a non-zero residual is at least
+    2^-27 |q| S and at most one float of q times S); the emulation asserts
+    it."""
     ld = np.longdouble
     S = np.float32(np.float32(s_g) * np.float32(o))
     R = 1.0 / float(S)
@@ -305,10 +310,19 @@ def _class_codes(a, s_g, o, p, step=True):
     if step and not _certified(S):
         near = (t.view(np.uint32) & np.uint32(0x1FFFFF)) == 0
         rho = _f32(al - t.astype(ld) * ld(S))
-        same = np.signbit(rho) == np.signbit(t)
-        tb = t.view(np.int32).astype(np.int64)
-        tb = np.where(near & (rho != 0), tb + np.where(same, 1, -1), tb)
-        t = tb.astype(np.int32).view(np.float32)
+        r16 = np.float32(16.0) * r_hi
+        v = _f32(t.astype(ld) + rho.astype(ld) * ld(r16))
+        # (values beyond 2^100 s_g, whose quotients overflow, are re-scored
+        # in fp64 by the kernel and left out here)
+        moved = near & (rho != 0) & np.isfinite(t) & np.isfinite(v)
+        if np.any(moved):
+            q = (al / ld(S))[moved]
+            tm, vm = t[moved].astype(ld), v[moved].astype(ld)
+            assert np.all(np.sign(vm - tm) == np.sign(q - tm))
+            assert np.all(np.abs(vm - tm) <= ld(2.0 ** -19) * np.abs(q) * (1 + ld(2.0 ** -20)))
+            tb, vb = t[moved].view(np.int32), v[moved].view(np.int32)
+            assert np.all(tb != vb)            # at least one float away
+        t = np.where(near, v, t)
     v = np.abs(t.astype(np.float64) * 2.0 ** -p)
     k = np.zeros(v.shape, np.int64)
     for i, mid in enumerate(MIDS):

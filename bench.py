@@ -569,6 +569,7 @@ def run_gpu(args):
         for i, r in enumerate(rows):
             per_row[r[0]].append(ev[k][i].elapsed_time(ev[k][i + 1]))
         step_ms.append(ev_step[k][0].elapsed_time(ev_step[k][1]))
+    log("timed steps (ms):", " ".join("%.4f" % v for v in step_ms))
     ms_per_step = max_over_ranks(pg, sum(step_ms)) / args.steps
     blocks = run.blocks()
     value = job_value(world, blocks, ms_per_step)

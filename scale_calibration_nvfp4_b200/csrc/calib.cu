@@ -147,12 +147,12 @@ cudaError_t launch_abs_histogram(const uint16_t *x, int64_t n, uint64_t *hist, c
   int64_t ctas = (n / 8 + kHistThreads - 1) / kHistThreads;
   if (ctas > sm_count()) ctas = sm_count();
   if (ctas < 1) ctas = 1;
-  return launch_chained(abs_histogram_kernel, dim3((unsigned)ctas), dim3(kHistThreads), kHistSmem,
+  return launch_first(abs_histogram_kernel, dim3((unsigned)ctas), dim3(kHistThreads), kHistSmem,
                         st, x, n, hist);
 }
 
 cudaError_t launch_quantile_scale(const uint64_t *hist, double p, float *s_g, cudaStream_t st) {
-  return launch_chained(quantile_scale_kernel, dim3(1), dim3(kHistThreads), 0, st, hist, p, s_g);
+  return launch_first(quantile_scale_kernel, dim3(1), dim3(kHistThreads), 0, st, hist, p, s_g);
 }
 
 cudaError_t read_and_clear_calib_status(cudaStream_t st, int *out) {

@@ -133,7 +133,7 @@ cudaError_t launch_gemm_fp4(const uint8_t *a_packed, const uint8_t *a_codes, con
   if (e == cudaSuccess) {
     // (the CUTLASS GEMM below is launched plainly: its own grid-dependency
     // wait is compiled only where CUTLASS enables it)
-    e = launch_chained(scale_layout_kernel<LayoutSFA>, dim3(grid_for_elems(M * (K / 16))),
+    e = launch_first(scale_layout_kernel<LayoutSFA>, dim3(grid_for_elems(M * (K / 16))),
                        dim3(256), 0, st, a_codes, M, K / 16, lsfa, sfa);
     if (e == cudaSuccess)
       e = launch_chained(scale_layout_kernel<LayoutSFB>, dim3(grid_for_elems(N * (K / 16))),

@@ -659,7 +659,7 @@ cudaError_t launch_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
   double *Linv = reinterpret_cast<double *>(scratch + lam_bytes + hd_bytes + sd_bytes);
   e = cudaMemsetAsync(SD, 0, sd_bytes, st);
   if (e == cudaSuccess) {
-    e = launch_chained(gptq_lambda_kernel, dim3((unsigned)batch), dim3(32), 0, st, H, C, damp, lam);
+    e = launch_first(gptq_lambda_kernel, dim3((unsigned)batch), dim3(32), 0, st, H, C, damp, lam);
     const int64_t n = C * C;
     int64_t gx = (n + 255) / 256;
     if (gx > (int64_t)sm_count() * 8) gx = (int64_t)sm_count() * 8;

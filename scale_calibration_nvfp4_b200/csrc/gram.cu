@@ -441,7 +441,7 @@ cudaError_t gram_uniform(const uint16_t *x, int64_t n_tok, int64_t C, float *H, 
   CUtensorMap tmap;
   cudaError_t e = make_x_tensor_map(x, n_tok, C, &tmap);
   if (e != cudaSuccess) return e;
-  e = launch_chained(gram_partial_kernel, dim3((unsigned)items, (unsigned)ngroups),
+  e = launch_first(gram_partial_kernel, dim3((unsigned)items, (unsigned)ngroups),
                      dim3(kGramThreads), kGramSmem, st, tmap, C, nullptr, nullptr, n_tok, per_item,
                      partial);
   if (e != cudaSuccess) return e;
@@ -495,7 +495,7 @@ cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, in
   int64_t *n_items = item_start + G + 1;
   ItemRange *items = reinterpret_cast<ItemRange *>(ws + off_items);
   float *partial = reinterpret_cast<float *>(ws + off_part);
-  e = launch_chained(build_items_kernel, dim3(1), dim3(1024), 0, st, offsets, G, n_tok, per_item,
+  e = launch_first(build_items_kernel, dim3(1), dim3(1024), 0, st, offsets, G, n_tok, per_item,
                      max_items, item_start, items, n_items);
   if (e == cudaSuccess)
     e = launch_chained(gram_partial_kernel, dim3((unsigned)max_items, (unsigned)ngroups),

@@ -630,7 +630,7 @@ cudaError_t launch_global_scale(const uint16_t *x, int64_t batch, int64_t n_per_
                                 float *s_g, cudaStream_t st) {
   // the maxima are accumulated by atomicMax from zero (a kernel rather than a
   // memset, so that the launches stay chained)
-  cudaError_t e = launch_chained(zero_words_kernel, dim3((unsigned)((batch + 127) / 128)),
+  cudaError_t e = launch_first(zero_words_kernel, dim3((unsigned)((batch + 127) / 128)),
                                  dim3(128), 0, st, reinterpret_cast<uint32_t *>(s_g), batch);
   if (e != cudaSuccess) return e;
   if (n_per_batch > 0) {
@@ -650,7 +650,7 @@ cudaError_t launch_scale_max(const uint16_t *w, int64_t batch, int64_t nblk, con
                              uint8_t *codes, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   int gx = grid_for(nblk, 16);
-  return launch_chained(max_rule_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st, w,
+  return launch_first(max_rule_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st, w,
                         nblk, s_g, codes);
 }
 
@@ -658,7 +658,7 @@ cudaError_t launch_four_over_six(const uint16_t *w, int64_t batch, int64_t nblk,
                                  const float *s_g, uint8_t *codes, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   const int gx = amortised_grid(batch, nblk, 3);  // 77 registers: three CTAs per SM
-  return launch_chained(four_over_six_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st,
+  return launch_first(four_over_six_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st,
                         w, nblk, s_g, codes);
 }
 
@@ -666,7 +666,7 @@ cudaError_t launch_pack(const uint16_t *w, int64_t batch, int64_t nblk, const fl
                         const uint8_t *codes, uint8_t *packed, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   const int gx = amortised_grid(batch, nblk, 5);
-  return launch_chained(pack_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st, w, nblk,
+  return launch_first(pack_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st, w, nblk,
                         s_g, codes, packed);
 }
 
@@ -674,7 +674,7 @@ cudaError_t launch_dequant(const uint8_t *packed, const uint8_t *codes, const fl
                            int64_t batch, int64_t nblk, uint16_t *out, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   int gx = grid_for(nblk, 16);
-  return launch_chained(dequant_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st, packed,
+  return launch_first(dequant_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st, packed,
                         codes, s_g, nblk, out);
 }
 
@@ -695,7 +695,7 @@ cudaError_t launch_fake_quant_static(const uint16_t *x, int64_t rows, int64_t C,
   const int64_t nblk = rows * C / kBlock;
   if (nblk == 0) return cudaSuccess;
   const int gx = grid_for(nblk, 16);
-  return launch_chained(fake_quant_kernel, dim3(gx), dim3(kThreads), 0, st, x, nblk, s_g, out,
+  return launch_first(fake_quant_kernel, dim3(gx), dim3(kThreads), 0, st, x, nblk, s_g, out,
                         packed, codes);
 }
 
@@ -707,7 +707,7 @@ cudaError_t launch_quant_error(const uint16_t *x, int64_t rows, int64_t C, const
   double *partial = nullptr;
   cudaError_t e = scratch_alloc(reinterpret_cast<void **>(&partial), sizeof(double) * gx, st);
   if (e != cudaSuccess) return e;
-  e = launch_chained(quant_error_kernel, dim3(gx), dim3(kThreads), 0, st, x, nblk, s_g, partial);
+  e = launch_first(quant_error_kernel, dim3(gx), dim3(kThreads), 0, st, x, nblk, s_g, partial);
   if (e == cudaSuccess)
     e = launch_chained(error_reduce_kernel, dim3(1), dim3(1), 0, st,
                        static_cast<const double *>(partial), gx, err);

@@ -523,12 +523,11 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
   __shared__ uint4 Ws[kRowsPerCta][2];     // the CTA's 16-element row segments
   __shared__ uint32_t keys[kRowsPerCta];  // amax << 16 | local row, sorted
 
-  // Chained launch.  MSE: wait for the previous kernel before anything.
-  // Local-Hessian: the previous kernel on the stream is always this call's
-  // factor kernel, which neither reads nor writes W, s_g, codes or best_obj
-  // and released its dependents only after its own wait (all earlier work
-  // on the stream has completed): the rows are loaded and sorted while it
-  // finishes, and the wait comes before the first read of its output.
+  // MSE: the call's first kernel (its wait returns at once).  Local-Hessian:
+  // chained to this call's factor kernel, which started after all earlier
+  // work on the stream had completed and neither reads nor writes W, s_g,
+  // codes or best_obj: the rows are loaded and sorted while it finishes, and
+  // the wait comes before the first read of its output.
   if constexpr (!kLH) chained_entry(w);
   const float s_g = s_g_arr[batch];
   const uint16_t *wb = w + batch * R * C + b * kBlock;
@@ -992,7 +991,7 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
   const int rows = small ? kRowsSmall : kRowsLarge;
   dim3 grid((unsigned)((R + rows - 1) / rows), (unsigned)(C / kBlock), (unsigned)batch);
   if (!local_hessian) {
-    return launch_chained(small ? search_kernel<false, kRowsSmall>
+    return launch_first(small ? search_kernel<false, kRowsSmall>
                                 : search_kernel<false, kRowsLarge>,
                           grid, dim3(kThreads), 0, st, w, R, C, s_g, nullptr, nullptr, nullptr,
                           codes, best_obj);
@@ -1007,8 +1006,9 @@ cudaError_t launch_scale_search(const uint16_t *w, int64_t batch, int64_t R, int
   Factor *fac = reinterpret_cast<Factor *>(static_cast<char *>(scratch) + frag_bytes);
   const int64_t nb = C / kBlock;
   // the search kernel reads W and s_g before waiting for the factor kernel
-  // (see its prologue): nothing may come between the two launches
-  e = launch_chained(factor_kernel, dim3((unsigned)((nb + 1) / 2), (unsigned)batch), dim3(32), 0,
+  // (see its prologue): nothing may come between the two launches, and the
+  // factor kernel starts after all earlier work
+  e = launch_first(factor_kernel, dim3((unsigned)((nb + 1) / 2), (unsigned)batch), dim3(32), 0,
                      st, H, nb, frag, fac);
   if (e == cudaSuccess)
     e = launch_chained(small ? search_kernel<true, kRowsSmall> : search_kernel<true, kRowsLarge>,

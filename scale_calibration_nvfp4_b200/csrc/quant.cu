@@ -344,7 +344,8 @@ __device__ __forceinline__ float block_mse32(const uint32_t w[8], uint2 q, float
 // t = fl(x r_hi) (r_hi = 1/s rounded down: |t - q| <= 2^-23 |q| for the exact
 // quotient q), each pair rounded from t (one conversion) and its byte decoded
 // by the hardware e2m1x2 -> f16x2 conversion in the same asm block, then d_i =
-// x_i - v_i s and e += d_i^2 in block_mse32's order.  The codes are those of
+// x_i - v_i s and the d_i^2 summed by fma in two partial sums (even and odd
+// elements, each in element order), added at the end.  The codes are those of
 // t, not always of q: where a rounding midpoint M lies between q and t, t
 // takes the other neighbour, and |d_i| (about half a grid step times s either
 // way) moves by at most 2 |q - M| s <= 2^-22 |q| s, at most 2^-19.7 of itself
@@ -363,18 +364,19 @@ __device__ __forceinline__ uint32_t e2m1x2_round_decode(float hi, float lo) {
 }
 __device__ __forceinline__ float block_mse32_entry(const uint32_t w[8], const ScaleEntry &e) {
   if (e.exact64) return block_mse32(w, encode_block_exact(w, e.s), e.s);
-  float acc = 0.0f;
+  // paired fp32 arithmetic on each value pair (each lane rounded as its
+  // scalar form): even elements accumulate in .x, odd ones in .y
+  const float2 rh = make_float2(e.r_hi, e.r_hi), ns = make_float2(-e.s, -e.s);
+  float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    const float x0 = bf16_lo(w[j]), x1 = bf16_hi(w[j]);
-    const float t0 = x0 * e.r_hi, t1 = x1 * e.r_hi;
-    const uint32_t h2 = e2m1x2_round_decode(t1, t0);
-    const float d0 = fmaf(-f16_lo_to_float(h2), e.s, x0);
-    const float d1 = fmaf(-f16_hi_to_float(h2), e.s, x1);
-    acc = fmaf(d0, d0, acc);
-    acc = fmaf(d1, d1, acc);
+    const float2 x = make_float2(bf16_lo(w[j]), bf16_hi(w[j]));
+    const float2 t = __fmul2_rn(x, rh);
+    const uint32_t h2 = e2m1x2_round_decode(t.y, t.x);
+    const float2 d = __ffma2_rn(make_float2(f16_lo_to_float(h2), f16_hi_to_float(h2)), ns, x);
+    acc = __ffma2_rn(d, d, acc);
   }
-  return acc;
+  return acc.x + acc.y;
 }
 
 // Block MSE at the table entry's scale in fp64, with the operations of the

@@ -361,9 +361,15 @@ __device__ __forceinline__ float candidate_objective(const float tq[8], float f,
                                                      const uint32_t bl[2][2],
                                                      const float pz[2][4], bool upper) {
   const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  // paired fp32 arithmetic (two independent lanes per instruction, each
+  // rounded as its scalar form)
+  const float2 ff = make_float2(f, f);
+  const float2 q0 = __fmul2_rn(make_float2(tq[0], tq[1]), ff);
+  const float2 q1 = __fmul2_rn(make_float2(tq[2], tq[3]), ff);
+  const float2 q2 = __fmul2_rn(make_float2(tq[4], tq[5]), ff);
+  const float2 q3 = __fmul2_rn(make_float2(tq[6], tq[7]), ff);
   uint32_t A[4];
-  round_decode4(tq[1] * f, tq[0] * f, tq[3] * f, tq[2] * f, tq[5] * f, tq[4] * f, tq[7] * f,
-                tq[6] * f, A);
+  round_decode4(q0.y, q0.x, q1.y, q1.x, q2.y, q2.x, q3.y, q3.x, A);
   float u0[4], u1[4];
   mma_f16_16816(u0, A, bh[0][0], bh[0][1], zero4);
   mma_f16_16816(u1, A, bh[1][0], bh[1][1], zero4);
@@ -371,12 +377,15 @@ __device__ __forceinline__ float candidate_objective(const float tq[8], float f,
     mma_f16_16816(u0, A, bl[0][0], bl[0][1], u0);
     mma_f16_16816(u1, A, bl[1][0], bl[1][1], u1);
   }
-  const float z00 = fmaf(-sm0, u0[0], pz[0][0]), z01 = fmaf(-sm0, u0[1], pz[0][1]);
-  const float z02 = fmaf(-sm1, u0[2], pz[0][2]), z03 = fmaf(-sm1, u0[3], pz[0][3]);
-  const float z10 = fmaf(-sm0, u1[0], pz[1][0]), z11 = fmaf(-sm0, u1[1], pz[1][1]);
-  const float z12 = fmaf(-sm1, u1[2], pz[1][2]), z13 = fmaf(-sm1, u1[3], pz[1][3]);
-  const float e0 = fmaf(z00, z00, fmaf(z01, z01, fmaf(z10, z10, z11 * z11)));
-  const float e1 = fmaf(z02, z02, fmaf(z03, z03, fmaf(z12, z12, z13 * z13)));
+  // z = p - s u: row g in accumulator elements 0, 1, row g + 8 in 2, 3
+  const float2 n0 = make_float2(-sm0, -sm0), n1 = make_float2(-sm1, -sm1);
+  const float2 za = __ffma2_rn(make_float2(u0[0], u0[1]), n0, make_float2(pz[0][0], pz[0][1]));
+  const float2 zb = __ffma2_rn(make_float2(u0[2], u0[3]), n1, make_float2(pz[0][2], pz[0][3]));
+  const float2 zc = __ffma2_rn(make_float2(u1[0], u1[1]), n0, make_float2(pz[1][0], pz[1][1]));
+  const float2 zd = __ffma2_rn(make_float2(u1[2], u1[3]), n1, make_float2(pz[1][2], pz[1][3]));
+  const float2 ea = __ffma2_rn(zc, zc, __fmul2_rn(za, za));  // row g
+  const float2 eb = __ffma2_rn(zd, zd, __fmul2_rn(zb, zb));  // row g + 8
+  const float e0 = ea.x + ea.y, e1 = eb.x + eb.y;
   // the same sums in the same order on both lanes of a pair
   float mine = upper ? e1 : e0;
   const float other = upper ? e0 : e1;
@@ -791,7 +800,14 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     // a candidate is skipped when its lower bound, less the bound's own
     // rounding, exceeds what the best so far can be: b1 (1 + 2 kTieBand) +
     // 4102 Q^2 + the floors
-    const float prune_pad = fmaf(4102.0f * qerr, qerr, row_floor + kAbsBand);
+    // (rows past the end and all-zero rows take -inf, so that they never
+    // hold the warp back: every check runs after at least one evaluation,
+    // so b1 is finite there)
+    const float prune_pad =
+        amax_row == 0.0f ? -__int_as_float(0x7F800000)
+                         : fmaf(4102.0f * qerr, qerr, row_floor + kAbsBand);
+    // the bounds' factors with their rounding allowance
+    const float ss2t = ss2 * (1.0f - 2.0f * kTieBand), sl2t = sl2 * (1.0f - 2.0f * kTieBand);
     const float smax = __uint_as_float(m << 16) * (1.0f / 6.0f);
 
     int jbegin = 0;
@@ -799,8 +815,19 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       const ClassInfo ci = cls[k];
       // class quotient t per element (within one float of q)
       float tq[8];
+      if constexpr (kLH) {
+        const float2 rhi = make_float2(ci.r_hi, ci.r_hi), rlo = make_float2(ci.r_lo, ci.r_lo);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) tq[e] = fmaf(xs[e], ci.r_hi, xs[e] * ci.r_lo);
+        for (int e = 0; e < 8; e += 2) {
+          const float2 x2 = make_float2(xs[e], xs[e + 1]);
+          const float2 t2 = __ffma2_rn(x2, rhi, __fmul2_rn(x2, rlo));
+          tq[e] = t2.x;
+          tq[e + 1] = t2.y;
+        }
+      } else {  // (paired, the MSE kernel would pass its 56 registers)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) tq[e] = fmaf(xs[e], ci.r_hi, xs[e] * ci.r_lo);
+      }
       // uncertified classes: a quotient with at most 3 significant bits
       // (every rounding midpoint is one, and so is every power-of-two
       // multiple) moves towards q = w / S: v = t + rho (16 / S), rounded
@@ -812,12 +839,15 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       // either sign leaves t.  Every other t is not a midpoint at any scale
       // of the class and rounds like q.
       if (!ci.certified) {
-        const float r16 = 16.0f * ci.r_hi;
+        const float2 nS = make_float2(-ci.S, -ci.S);
+        const float2 r16 = make_float2(16.0f * ci.r_hi, 16.0f * ci.r_hi);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float rho = fmaf(-tq[e], ci.S, xs[e]);
-          const bool near = (__float_as_uint(tq[e]) & 0x1FFFFFu) == 0u;
-          tq[e] = near ? fmaf(rho, r16, tq[e]) : tq[e];
+        for (int e = 0; e < 8; e += 2) {
+          const float2 t2 = make_float2(tq[e], tq[e + 1]);
+          const float2 rho = __ffma2_rn(t2, nS, make_float2(xs[e], xs[e + 1]));
+          const float2 v2 = __ffma2_rn(rho, r16, t2);
+          tq[e] = (__float_as_uint(t2.x) & 0x1FFFFFu) == 0u ? v2.x : t2.x;
+          tq[e + 1] = (__float_as_uint(t2.y) & 0x1FFFFFu) == 0u ? v2.y : t2.y;
         }
       }
       // first candidate of the class at or above smax (scales ascend within a
@@ -830,10 +860,10 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         const CandInfo c0 = cand[j];
         if (j < js) {
           // saturation bound at this scale (every later one is smaller)
-          const float d = fmaf(m6w, c0.s, amax_w);  // (amax_row - 6 s) 2^kw
-          const bool done = amax_row == 0.0f ||
-                            (d > 0.0f && ss2 * d * d * (1.0f - 2.0f * kTieBand) >
-                                             fmaf(b1, 1.0f + 2.0f * kTieBand, prune_pad));
+          // (amax_row - 6 s) 2^kw where the row's largest value saturates,
+          // else 0 (no bound: the threshold is positive for real rows)
+          const float d = fmaxf(fmaf(m6w, c0.s, amax_w), 0.0f);
+          const bool done = ss2t * d * d > fmaf(b1, 1.0f + 2.0f * kTieBand, prune_pad);
           if (__all_sync(0xFFFFFFFFu, done)) break;
         }
         const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * wsc0, c0.s * wsc1, bh,
@@ -846,20 +876,23 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
         const CandInfo c0 = cand[j];
         // zero-code bound at this scale (every later one is larger)
         const float q4 = 0.25f * c0.s;
-        float ug = 0.0f, ug8 = 0.0f;
+        // pairs (e, e + 1) lie in one row: e = 0, 4 in row g, e = 2, 6 in g + 8
+        float2 ugp = make_float2(0.0f, 0.0f), ug8p = ugp;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float v = (fabsf(xs[e]) <= q4 ? xs[e] : 0.0f) * ((e & 2) ? wsc1 : wsc0);
-          if ((e & 2) == 0) ug = fmaf(v, v, ug);
-          else ug8 = fmaf(v, v, ug8);
+        for (int e = 0; e < 8; e += 2) {
+          const float2 x2 = make_float2(fabsf(xs[e]) <= q4 ? xs[e] : 0.0f,
+                                        fabsf(xs[e + 1]) <= q4 ? xs[e + 1] : 0.0f);
+          const float ws = (e & 2) ? wsc1 : wsc0;
+          const float2 v2 = __fmul2_rn(x2, make_float2(ws, ws));
+          if ((e & 2) == 0) ugp = __ffma2_rn(v2, v2, ugp);
+          else ug8p = __ffma2_rn(v2, v2, ug8p);
         }
+        const float ug = ugp.x + ugp.y, ug8 = ug8p.x + ug8p.y;
         // the same quad reduce-scatter as the objective: lanes t < 2 keep row g
         float zero_sum = upper ? ug8 : ug;
         zero_sum += __shfl_xor_sync(0xFFFFFFFFu, upper ? ug : ug8, 2);
         zero_sum += __shfl_xor_sync(0xFFFFFFFFu, zero_sum, 1);
-        const bool done = amax_row == 0.0f ||
-                          sl2 * zero_sum * (1.0f - 2.0f * kTieBand) >
-                              fmaf(b1, 1.0f + 2.0f * kTieBand, prune_pad);
+        const bool done = sl2t * zero_sum > fmaf(b1, 1.0f + 2.0f * kTieBand, prune_pad);
         if (__all_sync(0xFFFFFFFFu, done)) break;
         const float e0 = candidate_objective<kLH>(tq, c0.f, c0.s * wsc0, c0.s * wsc1, bh,
                                                   bl, pz, upper);

@@ -564,21 +564,23 @@ def _rne_e2m1(t):
 def _mse32(oracle_mod, x, s):
     """The kernel's fp32 block MSE screen: each value's code rounded from
     t = RN(x r_hi) (r_hi = 1/s rounded down), not from the exact quotient;
-    then d_i = RN(x_i - v_i s), e = RN(d_i^2 + e) in element order, every step
-    rounded once from its exact value."""
+    then d_i = RN(x_i - v_i s) and two partial sums by fma, e_p = RN(d_i^2 +
+    e_p) over the even (p = 0) and the odd (p = 1) elements in element
+    order, returned as RN(e_0 + e_1); every step rounded once from its exact
+    value."""
     from fractions import Fraction
     s32 = np.float32(s)
     S = Fraction(float(s32))
     r_hi = _rd32(1 / S)                                  # the kernel's __frcp_rd
-    e = Fraction(0)
-    for xi in x:
+    e = [Fraction(0), Fraction(0)]
+    for i, xi in enumerate(x):
         X = Fraction(float(xi))
         t = _rn32(X * r_hi)
         k = _rne_e2m1(float(t) if t != 0 else (-0.0 if np.signbit(xi) else 0.0))
         v = Fraction(float(GRID[k & 7])) * (-1 if k & 8 else 1)
         d = _rn32(X - v * S)
-        e = _rn32(d * d + e)
-    return e
+        e[i % 2] = _rn32(d * d + e[i % 2])
+    return _rn32(e[0] + e[1])
 
 
 def test_four_over_six_screen_with_absolute_floor(oracle_mod):

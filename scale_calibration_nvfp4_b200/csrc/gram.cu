@@ -295,8 +295,18 @@ __global__ void gram_reduce_kernel(const float *__restrict__ partial, int64_t nb
     i0 = item_start[g];
     i1 = item_start[g + 1];
   }
+  // eight loads in flight, then their sum in item order (the largest group
+  // of a routed batch can hold tens of items)
   float acc = 0.0f;
-  for (int64_t i = i0; i < i1; ++i) acc += partial[i * per_group + je];
+  int64_t i = i0;
+  for (; i + 8 <= i1; i += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = partial[(i + u) * per_group + je];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc += v[u];
+  }
+  for (; i < i1; ++i) acc += partial[i * per_group + je];
   H[idx] += acc;
 }
 

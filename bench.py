@@ -525,11 +525,6 @@ def run_gpu(args):
         flush.zero_()
         flush.sum()
 
-    for _ in range(args.warmup):
-        flush_l2()
-        step()
-    torch.cuda.synchronize()
-
     # timed pass: events at the step boundaries only, so that the step's
     # launches follow one another as they would in use
     ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -542,6 +537,12 @@ def run_gpu(args):
     if clocks:
         clocks.start()
         time.sleep(0.3)
+    # the warm-up steps come after the sampler's start-up pause, so that the
+    # timed steps follow them without the GPU idling in between
+    for _ in range(args.warmup):
+        flush_l2()
+        step()
+    torch.cuda.synchronize()
     if pg:
         pg.barrier()
     nvfp4.search_evaluations(reset=True)  # synchronises

@@ -768,36 +768,64 @@ def search_roofline(run, kernels, lh_rows, pk, pk_kind, workload, lh_evals, sm_m
 def run_e2e(run, args, pg, world):
     """Same metric through the public API with host buffers: every step copies
     the inputs from pinned host memory to the device, runs the path and reads
-    the results (codes and packed weights, or packed activations) back."""
+    the results (codes and packed weights, or packed activations) back.
+
+    The steps are pipelined the way a calibration loop streams its layers:
+    uploads on one stream, the path on another, downloads on a third.  Step
+    k + 1's uploads start once step k's path has read its inputs and run
+    while step k's results come back (the two copy directions use separate
+    copy engines); step k + 1's path starts once its inputs are in and step
+    k's results have left the output buffers.  Every step still moves all
+    of its inputs and results."""
     ins = [(t, t.cpu().pin_memory()) for t in run.inputs()]
     outs = [(t, torch.empty(t.shape, dtype=t.dtype).pin_memory()) for t in run.results()]
-    stream = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    s_c = torch.cuda.current_stream()
+    state = {"computed": None, "drained": None}
 
     def step():
-        for d, h in ins:
-            d.copy_(h, non_blocking=True)
+        up, done, down = (torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event())
+        with torch.cuda.stream(s_in):
+            if state["computed"] is not None:
+                s_in.wait_event(state["computed"])   # the inputs have been read
+            for d, h in ins:
+                d.copy_(h, non_blocking=True)
+            up.record(s_in)
+        s_c.wait_event(up)
+        if state["drained"] is not None:
+            s_c.wait_event(state["drained"])        # the outputs have left
         for r in run.rows:
             r[1]()
-        for d, h in outs:
-            h.copy_(d, non_blocking=True)
+        done.record(s_c)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done)
+            for d, h in outs:
+                h.copy_(d, non_blocking=True)
+            down.record(s_out)
+        state["computed"], state["drained"] = done, down
 
     for _ in range(max(1, args.warmup)):
         step()
+    s_c.wait_event(state["drained"])
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(s_c)
+    s_in.wait_event(e0)
     for _ in range(args.steps):
         step()
-    e1.record(stream)
+    s_c.wait_event(state["drained"])             # the last results are on the host
+    e1.record(s_c)
     torch.cuda.synchronize()
     ms_step = max_over_ranks(pg, e0.elapsed_time(e1)) / args.steps
     h2d = sum(h.numel() * h.element_size() for _, h in ins)
     d2h = sum(h.numel() * h.element_size() for _, h in outs)
     return {"value": round(job_value(world, run.blocks(), ms_step), 1), "unit": UNIT,
             "ms_per_step": round(ms_step, 5), "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h}
+            "d2h_bytes_per_step": d2h,
+            "overlap": "uploads of step k+1 with downloads of step k (separate streams and "
+                       "copy engines); each step's path after its own uploads"}
 
 
 # ------------------------------------------------------------------ CPU arm

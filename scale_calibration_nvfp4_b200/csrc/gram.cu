@@ -284,10 +284,15 @@ __global__ void gram_reduce_kernel(const float *__restrict__ partial, int64_t nb
                                    const int64_t *__restrict__ item_start, int64_t n_items_uniform,
                                    float *__restrict__ H) {
   chained_entry();
+  // the status once per CTA (a load of the one word by every thread queued
+  // millions of requests on one L2 slice)
+  __shared__ int status;
+  if (threadIdx.x == 0) status = *(volatile const int *)&g_gram_status;
+  __syncthreads();
+  if (status != 0) return;
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over G * nb * 256
   const int64_t per_group = nb * 256;
   if (idx >= G * per_group) return;
-  if (*(volatile const int *)&g_gram_status != 0) return;
   const int64_t g = idx / per_group;
   const int64_t je = idx - g * per_group;
   int64_t i0 = 0, i1 = n_items_uniform;

@@ -668,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     __syncthreads();  // cdiag_sh
   }
 
-  unsigned long long evals = 0;
+  uint32_t evals = 0;  // (at most 16 tiles x 126 candidates x 16 rows per warp)
   for (int tile = warp; tile < kRowsPerCta / kTileRows; tile += kWarps) {
     const uint32_t kg = keys[tile * kTileRows + g], kg8 = keys[tile * kTileRows + g + 8];
     const bool v0 = (kg >> 16) != 0xFFFFu, v1 = (kg8 >> 16) != 0xFFFFu;
@@ -797,6 +797,12 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     const float ss2 = kLH ? cdiag_sh[((upper ? kg8 : kg) >> 12) & 0xFu] : 1.0f;
     const float amax_w = amax_row * wsc, m6w = -6.0f * wsc;
     const float row_floor = kZeroFloor * (upper ? pp1 : pp0);
+    // what the tile's epilogue needs, formed here so that nothing else stays
+    // live across the candidate walk: the lane's row, whether it finishes
+    // it, and whether a tile value lies above 2^100 s_g
+    const int my_row = upper ? i1 : i0;
+    const bool owner = (t & 1) == 0 && (upper ? v1 : v0);
+    const bool tile_over = __uint_as_float(m << 16) > 0x1p100f * s_g;
     // a candidate is skipped when its lower bound, less the bound's own
     // rounding, exceeds what the best so far can be: b1 (1 + 2 kTieBand) +
     // 4102 Q^2 + the floors
@@ -902,21 +908,20 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
       jbegin = ci.end;
     }
 
-    evals += (unsigned long long)ncand * nvalid;
+    evals += ncand * nvalid;
 
     // lane t = 0 finishes row g, lane t = 2 row g + 8; near ties are
     // re-scored by the whole warp, one row at a time
-    const int64_t r = row_base + (upper ? i1 : i0);
-    const bool owner = (t & 1) == 0 && (upper ? v1 : v0);
+    const int64_t r = row_base + my_row;
     int code = code_of(b1);
     float obj = ldexpf(b1, -2 * zexp);
     int need = 0;  // 1: re-score the best two, 2: re-score every candidate
     if (owner) {
-      const float fl = kZeroFloor * (upper ? pp1 : pp0);
-      if (amax_row == 0.0f) {  // all-zero row: every candidate scores exactly 0
+      const float fl = row_floor;
+      if (amax_w == 0.0f) {  // all-zero row: every candidate scores exactly 0
         code = 1;
         obj = 0.0f;
-      } else if (!by_class || __uint_as_float(m << 16) > 0x1p100f * s_g) {
+      } else if (!by_class || tile_over) {
         // s_g outside [2^-100, 2^100): the per-candidate fp32 reciprocals can
         // leave the normal range; or a tile value above 2^100 s_g (a tensor
         // scale far below the weights' own, amax / 2688): the class
@@ -956,7 +961,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? 7 : 9)
     }
   }
   if (lane == 0) {
-    if (evals) atomicAdd(&g_search_evals[kLH ? 1 : 0], evals);
+    if (evals) atomicAdd(&g_search_evals[kLH ? 1 : 0], (unsigned long long)evals);
   }
 }
 

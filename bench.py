@@ -771,61 +771,70 @@ def run_e2e(run, args, pg, world):
     the results (codes and packed weights, or packed activations) back.
 
     The steps are pipelined the way a calibration loop streams its layers:
-    uploads on one stream, the path on another, downloads on a third.  Step
-    k + 1's uploads start once step k's path has read its inputs and run
-    while step k's results come back (the two copy directions use separate
-    copy engines); step k + 1's path starts once its inputs are in and step
-    k's results have left the output buffers.  Every step still moves all
-    of its inputs and results."""
-    ins = [(t, t.cpu().pin_memory()) for t in run.inputs()]
-    outs = [(t, torch.empty(t.shape, dtype=t.dtype).pin_memory()) for t in run.results()]
+    uploads on one stream, the path on another, downloads on a third, and
+    two sets of device buffers used in turn where the device has room for a
+    second (one set otherwise).  Step k + 1's uploads go to the other set and
+    run while step k's path runs and its results come back (the two copy
+    directions use separate copy engines); a set is refilled once the path
+    two steps back has read it, and its results are overwritten once they
+    have left.  Every step still moves all of its inputs and results."""
+    runs = [run]
+    free, _ = torch.cuda.mem_get_info()
+    if free > 1.5 * torch.cuda.memory_allocated():
+        runs.append(Runner(run.workload, "cuda"))
+    hosts = [h for h in (t.cpu().pin_memory() for t in run.inputs())]
+    outs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in run.results()]
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     s_c = torch.cuda.current_stream()
-    state = {"computed": None, "drained": None}
+    state = [{"computed": None, "drained": None} for _ in runs]
+    last = {"drained": None}
 
-    def step():
-        up, done, down = (torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event())
+    def step(k):
+        b = k % len(runs)
+        R, st = runs[b], state[b]
+        up, done, down = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
         with torch.cuda.stream(s_in):
-            if state["computed"] is not None:
-                s_in.wait_event(state["computed"])   # the inputs have been read
-            for d, h in ins:
+            if st["computed"] is not None:
+                s_in.wait_event(st["computed"])      # this set's inputs have been read
+            for d, h in zip(R.inputs(), hosts):
                 d.copy_(h, non_blocking=True)
             up.record(s_in)
         s_c.wait_event(up)
-        if state["drained"] is not None:
-            s_c.wait_event(state["drained"])        # the outputs have left
-        for r in run.rows:
+        if st["drained"] is not None:
+            s_c.wait_event(st["drained"])           # this set's results have left
+        for r in R.rows:
             r[1]()
         done.record(s_c)
         with torch.cuda.stream(s_out):
             s_out.wait_event(done)
-            for d, h in outs:
+            for d, h in zip(R.results(), outs):
                 h.copy_(d, non_blocking=True)
             down.record(s_out)
-        state["computed"], state["drained"] = done, down
+        st["computed"], st["drained"] = done, down
+        last["drained"] = down
 
-    for _ in range(max(1, args.warmup)):
-        step()
-    s_c.wait_event(state["drained"])
+    for k in range(max(len(runs), args.warmup)):
+        step(k)
+    s_c.wait_event(last["drained"])
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(s_c)
     s_in.wait_event(e0)
-    for _ in range(args.steps):
-        step()
-    s_c.wait_event(state["drained"])             # the last results are on the host
+    for k in range(args.steps):
+        step(k)
+    s_c.wait_event(last["drained"])                # the last results are on the host
     e1.record(s_c)
     torch.cuda.synchronize()
     ms_step = max_over_ranks(pg, e0.elapsed_time(e1)) / args.steps
-    h2d = sum(h.numel() * h.element_size() for _, h in ins)
-    d2h = sum(h.numel() * h.element_size() for _, h in outs)
+    h2d = sum(h.numel() * h.element_size() for h in hosts)
+    d2h = sum(h.numel() * h.element_size() for h in outs)
     return {"value": round(job_value(world, run.blocks(), ms_step), 1), "unit": UNIT,
             "ms_per_step": round(ms_step, 5), "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h,
-            "overlap": "uploads of step k+1 with downloads of step k (separate streams and "
-                       "copy engines); each step's path after its own uploads"}
+            "d2h_bytes_per_step": d2h, "device_buffer_sets": len(runs),
+            "overlap": "uploads of step k+1 (into the other buffer set) with the path and the "
+                       "downloads of step k; separate streams and copy engines"}
 
 
 # ------------------------------------------------------------------ CPU arm

@@ -277,12 +277,15 @@ __global__ void wait_timeout_probe_kernel() {
   if (!ok && threadIdx.x == 0) atomicMax(&g_gram_status, (int)NVFP4_ERR_DEVICE_TIMEOUT);
 }
 
-// H[g][j][e] += sum of the partials of group g's items, in item order.
+// H[g][e] += sum of the partials of group g's items, in item order, four
+// consecutive entries per thread (16-byte loads of the partials; the
+// partials are library scratch, 256-byte aligned, and a group is a multiple
+// of 256 floats), group g = blockIdx.y (grid-stride beyond 65,535 groups).
 // Nothing is added while a timed-out wait is on record (a partial of this
 // call may then be missing, and its slot holds stale data).
-__global__ void gram_reduce_kernel(const float *__restrict__ partial, int64_t nb, int64_t G,
-                                   const int64_t *__restrict__ item_start, int64_t n_items_uniform,
-                                   float *__restrict__ H) {
+__global__ void gram_reduce_kernel(const float *__restrict__ partial, int64_t per_group,
+                                   int64_t G, const int64_t *__restrict__ item_start,
+                                   int64_t n_items_uniform, float *__restrict__ H) {
   chained_entry();
   // the status once per CTA (a load of the one word by every thread queued
   // millions of requests on one L2 slice)
@@ -290,33 +293,47 @@ __global__ void gram_reduce_kernel(const float *__restrict__ partial, int64_t nb
   if (threadIdx.x == 0) status = *(volatile const int *)&g_gram_status;
   __syncthreads();
   if (status != 0) return;
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over G * nb * 256
-  const int64_t per_group = nb * 256;
-  if (idx >= G * per_group) return;
-  const int64_t g = idx / per_group;
-  const int64_t je = idx - g * per_group;
-  int64_t i0 = 0, i1 = n_items_uniform;
-  if (item_start) {
-    i0 = item_start[g];
-    i1 = item_start[g + 1];
-  }
-  // eight loads in flight, then their sum in item order (the largest group
-  // of a routed batch can hold tens of items)
-  float acc = 0.0f;
-  int64_t i = i0;
-  for (; i + 8 <= i1; i += 8) {
-    float v[8];
+  const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (e >= per_group) return;
+  const int64_t stride4 = per_group / 4;
+  for (int64_t g = blockIdx.y; g < G; g += gridDim.y) {
+    int64_t i0 = 0, i1 = n_items_uniform;
+    if (item_start) {
+      i0 = item_start[g];
+      i1 = item_start[g + 1];
+    }
+    const float4 *p4 = reinterpret_cast<const float4 *>(partial + e);
+    // eight loads in flight, then their sum in item order (the largest group
+    // of a routed batch can hold tens of items)
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    int64_t i = i0;
+    for (; i + 8 <= i1; i += 8) {
+      float4 v[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = partial[(i + u) * per_group + je];
+      for (int u = 0; u < 8; ++u) v[u] = p4[(i + u) * stride4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) acc += v[u];
+      for (int u = 0; u < 8; ++u) {
+        acc.x += v[u].x;
+        acc.y += v[u].y;
+        acc.z += v[u].z;
+        acc.w += v[u].w;
+      }
+    }
+    for (; i < i1; ++i) {
+      const float4 v = p4[i * stride4];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    float *h = H + g * per_group + e;  // 4-byte aligned: scalar updates
+    h[0] += acc.x;
+    h[1] += acc.y;
+    h[2] += acc.z;
+    h[3] += acc.w;
   }
-  for (; i < i1; ++i) acc += partial[i * per_group + je];
-  H[idx] += acc;
 }
 
-// Grouped form: per-group item counts, an exclusive scan (one CTA) and the
-// item table.  Offsets are clamped to [0, n_tok] and made non-decreasing.
 __global__ void build_items_kernel(const int64_t *__restrict__ offsets, int64_t G, int64_t n_tok,
                                    int64_t per_item, int64_t max_items,
                                    int64_t *__restrict__ item_start, ItemRange *__restrict__ items,
@@ -460,9 +477,9 @@ cudaError_t gram_uniform(const uint16_t *x, int64_t n_tok, int64_t C, float *H, 
                      dim3(kGramThreads), kGramSmem, st, tmap, C, nullptr, nullptr, n_tok, per_item,
                      partial);
   if (e != cudaSuccess) return e;
-  return launch_chained(gram_reduce_kernel, dim3((unsigned)((per_group + 255) / 256)), dim3(256),
-                        0, st, static_cast<const float *>(partial), nb, (int64_t)1, nullptr, items,
-                        H);
+  return launch_chained(gram_reduce_kernel, dim3((unsigned)((per_group / 4 + 255) / 256)),
+                        dim3(256), 0, st, static_cast<const float *>(partial), per_group,
+                        (int64_t)1, nullptr, items, H);
 }
 
 }  // namespace
@@ -518,8 +535,10 @@ cudaError_t launch_gram(const uint16_t *x, const int64_t *offsets, int64_t G, in
                        static_cast<const ItemRange *>(items), static_cast<const int64_t *>(n_items),
                        n_tok, per_item, partial);
   if (e == cudaSuccess)
-    e = launch_chained(gram_reduce_kernel, dim3((unsigned)((G * per_group + 255) / 256)),
-                       dim3(256), 0, st, static_cast<const float *>(partial), nb, G,
+    e = launch_chained(gram_reduce_kernel,
+                       dim3((unsigned)((per_group / 4 + 255) / 256),
+                            (unsigned)std::min<int64_t>(G, 65535)),
+                       dim3(256), 0, st, static_cast<const float *>(partial), per_group, G,
                        static_cast<const int64_t *>(item_start), (int64_t)0, H);
   cudaError_t e2 = scratch_free(ws, st);
   return e != cudaSuccess ? e : e2;

@@ -379,6 +379,32 @@ __device__ __forceinline__ float block_mse32_entry(const uint32_t w[8], const Sc
   return acc.x + acc.y;
 }
 
+// Both candidates' fp32 block MSEs in one pass over the values (each pair
+// unpacked once), each with exactly block_mse32_entry's arithmetic.
+__device__ __forceinline__ void block_mse32_two(const uint32_t w[8], const ScaleEntry &ea,
+                                                const ScaleEntry &eb, float &fa, float &fb) {
+  if (ea.exact64 || eb.exact64) {
+    fa = block_mse32_entry(w, ea);
+    fb = block_mse32_entry(w, eb);
+    return;
+  }
+  const float2 rha = make_float2(ea.r_hi, ea.r_hi), nsa = make_float2(-ea.s, -ea.s);
+  const float2 rhb = make_float2(eb.r_hi, eb.r_hi), nsb = make_float2(-eb.s, -eb.s);
+  float2 acca = make_float2(0.0f, 0.0f), accb = acca;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float2 x = make_float2(bf16_lo(w[j]), bf16_hi(w[j]));
+    const float2 ta = __fmul2_rn(x, rha), tb = __fmul2_rn(x, rhb);
+    const uint32_t ha = e2m1x2_round_decode(ta.y, ta.x), hb = e2m1x2_round_decode(tb.y, tb.x);
+    const float2 da = __ffma2_rn(make_float2(f16_lo_to_float(ha), f16_hi_to_float(ha)), nsa, x);
+    const float2 db = __ffma2_rn(make_float2(f16_lo_to_float(hb), f16_hi_to_float(hb)), nsb, x);
+    acca = __ffma2_rn(da, da, acca);
+    accb = __ffma2_rn(db, db, accb);
+  }
+  fa = acca.x + acca.y;
+  fb = accb.x + accb.y;
+}
+
 // Block MSE at the table entry's scale in fp64, with the operations of the
 // definition in its order: d_i = w_i - v_i s, e += d_i^2, i = 0..15, each
 // product and sum rounded on its own (no fused multiply-add), so that two
@@ -429,7 +455,8 @@ __global__ void __launch_bounds__(kThreads) four_over_six_kernel(const uint16_t 
       // fp32 screen; the exact fp64 comparison only when the two are close
       // (relative 2^-16, or absolute 2^-130 for subnormal sums)
       const ScaleEntry el = tab[lo], eh = tab[hi];
-      const float fl = block_mse32_entry(v, el), fh = block_mse32_entry(v, eh);
+      float fl, fh;
+      block_mse32_two(v, el, eh, fl, fh);
       if (fabsf(fh - fl) > fmaf(0x1p-16f, fmaxf(fh, fl), 0x1p-130f)) {
         code = fh < fl ? hi : lo;
       } else {

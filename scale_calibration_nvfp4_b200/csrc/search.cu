@@ -627,11 +627,13 @@ __global__ void __launch_bounds__(kThreads, kLH ? kLhCtasPerSm : kMseCtasPerSm)
       // amax bits, then the position of an element that reaches it (for the
       // row's saturation bound), then the local row
       const uint32_t am = amax_bits8(w8);
-      uint32_t pos = 0;
+      uint32_t pos = 0;  // (the MSE rule's saturation factor is 1 for every position)
+      if constexpr (kLH) {
 #pragma unroll
-      for (int e = 15; e >= 0; --e) {
-        const uint32_t mag = ((e & 1) ? (w8[e >> 1] >> 16) : w8[e >> 1]) & 0x7FFFu;
-        pos = mag == am ? (uint32_t)e : pos;
+        for (int e = 15; e >= 0; --e) {
+          const uint32_t mag = ((e & 1) ? (w8[e >> 1] >> 16) : w8[e >> 1]) & 0x7FFFu;
+          pos = mag == am ? (uint32_t)e : pos;
+        }
       }
       key = (am << 16) | (pos << 12) | (uint32_t)i;
     }

@@ -608,14 +608,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? kLhCtasPerSm : kMseCtasPerSm)
   // Sort key: amax (bf16 magnitude bits, bits 16..31), the position of the
   // row's largest element (bits 12..15) and the local row index (bits
   // 0..11); rows past the end get magnitude 0xFFFF (zero data) and sort last.
-  // (thread t stages rows t + u kThreads, u < kKeys, and holds their keys in
-  // kv[u] for the sort)
-  constexpr int kKeys = kRowsPerCta / kThreads;
-  static_assert(kKeys == 1 || kKeys == 2, "the register sort takes one or two keys per thread");
-  uint32_t kv[kKeys];
-#pragma unroll
-  for (int u = 0; u < kKeys; ++u) {
-    const int i = threadIdx.x + u * kThreads;
+  for (int i = threadIdx.x; i < kRowsPerCta; i += kThreads) {
     const int64_t r = row_base + i;
     uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
     uint32_t key = 0xFFFF0000u | (uint32_t)i;
@@ -639,53 +632,24 @@ __global__ void __launch_bounds__(kThreads, kLH ? kLhCtasPerSm : kMseCtasPerSm)
     }
     Ws[i][0] = a0;
     Ws[i][1] = a1;
-    kv[u] = key;
+    keys[i] = key;
   }
-  // bitonic sort of the keys, ascending, in registers: thread t holds the
-  // keys at positions t kKeys + u.  The compare-exchange of positions i and
-  // i ^ stride (the lower one takes the smaller key when (i & size) == 0) is
-  // inside the thread for stride < kKeys, between lanes of a warp (one
-  // shuffle per key) for stride < 32 kKeys, and through shared memory only
-  // beyond (three of the 36 steps for 256 rows).
-  {
-    const int t = threadIdx.x;
-    for (int size = 2; size <= kRowsPerCta; size <<= 1) {
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        if (stride < kKeys) {  // kKeys == 2, stride == 1: positions 2t, 2t + 1
-          if constexpr (kKeys == 2) {
-            const bool asc = ((2 * t) & size) == 0;
-            const uint32_t lo = min(kv[0], kv[1]), hi = max(kv[0], kv[1]);
-            kv[0] = asc ? lo : hi;
-            kv[1] = asc ? hi : lo;
-          }
-        } else if (stride < 32 * kKeys) {
-          const int d = stride / kKeys;  // lane distance
-          const bool lower = (t & d) == 0;
-#pragma unroll
-          for (int u = 0; u < kKeys; ++u) {
-            const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, kv[u], d);
-            const bool asc = ((t * kKeys + u) & size) == 0;
-            kv[u] = lower == asc ? min(kv[u], o) : max(kv[u], o);
-          }
-        } else {
-          __syncthreads();  // the previous exchange's reads are done
-#pragma unroll
-          for (int u = 0; u < kKeys; ++u) keys[t * kKeys + u] = kv[u];
-          __syncthreads();
-#pragma unroll
-          for (int u = 0; u < kKeys; ++u) {
-            const int i = t * kKeys + u;
-            const uint32_t o = keys[i ^ stride];
-            const bool asc = (i & size) == 0;
-            kv[u] = (i < (i ^ stride)) == asc ? min(kv[u], o) : max(kv[u], o);
-          }
+  __syncthreads();
+  // bitonic sort of the keys, ascending; pair p of a step compares keys i
+  // and i + stride with i = 2p - (p mod stride), p < kRowsPerCta / 2
+  for (int size = 2; size <= kRowsPerCta; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int p = threadIdx.x; p < kRowsPerCta / 2; p += kThreads) {
+        const int i = 2 * p - (p & (stride - 1));
+        const int j = i + stride;
+        const uint32_t ki = keys[i], kj = keys[j];
+        if ((ki > kj) == ((i & size) == 0)) {
+          keys[i] = kj;
+          keys[j] = ki;
         }
       }
+      __syncthreads();
     }
-    __syncthreads();  // the last exchange's reads are done
-#pragma unroll
-    for (int u = 0; u < kKeys; ++u) keys[t * kKeys + u] = kv[u];
-    __syncthreads();
   }
 
   if constexpr (kLH) {

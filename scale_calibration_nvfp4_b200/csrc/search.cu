@@ -15,7 +15,8 @@
 // of rows g and g+8.
 //
 // Per candidate scale s the objective is rewritten with H_b = L L^T (fp64
-// Cholesky once per CTA, semidefinite pivots dropped):
+// Cholesky once per column block, in factor_kernel; semidefinite pivots
+// dropped):
 //     E = ||L^T delta||^2,  delta = w - s v,   so   L^T delta = p - s u,
 // with p = L^T w fixed per row and u = L^T v.  The signed E2M1 values v are
 // exact in f16, so u comes from two f16 MMAs per 8 outputs against L split
@@ -25,17 +26,18 @@
 //
 // Exact E2M1 codes without a fallback branch.  Candidate values are o * 2^p
 // with odd o in {1, 3, ..., 15}, and s(c) = fl(s_g o) 2^p exactly, so for each
-// element and each odd part o the quotient q = |w| / fl(s_g o) is formed once,
-// as t from a double-float reciprocal: t is one of the two floats around q.
-// Candidates of class o scale t by 2^-p exactly.  Every rounding midpoint of
-// E2M1 is a float with at most 3 significant bits, so a t with more bits is
-// no midpoint at any scale of the class, and its hardware round-to-nearest-
-// even gives q's code.  A t with at most 3 significant bits is replaced once
-// per class by its neighbouring float across q (by the exact sign of the
-// residual |w| - t fl(s_g o), one fma; t itself when q == t), which has 24
-// significant bits and so rounds like q.  Classes whose S passes
-// quotients_far_from_midpoints (no bf16 value comes near a midpoint) skip
-// that step.
+// element and each odd part o the signed quotient q = w / fl(s_g o) is formed
+// once, as t from a double-float reciprocal: t is one of the two floats
+// around q.  Candidates of class o scale t by 2^-p exactly.  Every rounding
+// midpoint of E2M1 is a float with at most 3 significant bits, so a t with
+// more bits is no midpoint at any scale of the class, and its hardware
+// round-to-nearest-even gives q's code.  A t with at most 3 significant bits
+// moves once per class towards q by one fma, t + rho 16 / fl(s_g o) with the
+// exact residual rho = w - t fl(s_g o): a non-zero residual of such a t puts
+// the moved value between one float and 2^-19 |q| from t on q's side, off
+// the midpoint and short of any other decision; a zero residual (of either
+// sign) leaves t.  Classes whose S passes quotients_far_from_midpoints (no
+// bf16 value comes near a midpoint) skip that step.
 //
 // Winner: fp32 screen keeping the best three objectives; the candidates that
 // the screen's error bound cannot separate are re-scored in fp64 straight
@@ -351,8 +353,8 @@ __device__ __forceinline__ uint32_t pick4(uint32_t w0, uint32_t w1, uint32_t w2,
 
 // One candidate: codes, the tensor-core product u, z = p - s u, and the row
 // objective after a quad reduce-scatter (lanes t < 2: row g, t >= 2: row
-// g + 8).  tq holds the signed class quotients (stepped where a midpoint
-// could occur), f scales them to this candidate exactly; sm0 and sm1 multiply
+// g + 8).  tq holds the signed class quotients (moved off a possible
+// midpoint where one could occur), f scales them to this candidate exactly; sm0 and sm1 multiply
 // u in rows g and g + 8 (accumulator elements 0, 1 and 2, 3 of both n-tiles),
 // each row carrying its own power-of-two scale.
 template <bool kLH>
@@ -394,10 +396,9 @@ __device__ __forceinline__ float candidate_objective(const float tq[8], float f,
   return mine;
 }
 
-// Per column block (and batch element) of H: the f16 high/low B-operand
-// fragments of sigma L for every lane, sigma, the eigenvalue bound and the
-// zero-H flag.  One warp per block; the search kernel then starts straight on
-// its rows.
+// Per column block (and batch element) of H, from factor_kernel: the f16
+// high/low B-operand fragments of sigma L for every lane, sigma, the pruning
+// bounds' factors, the dropped-pivot residual and the zero-H flag.
 struct Factor {
   float sigma;   // power of two putting max |L| in [2^14, 2^15)
   float sl2;     // sigma^2 lambda, lambda a lower bound of lambda_min(L L^T) (0 when unknown)

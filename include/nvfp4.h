@@ -39,9 +39,15 @@
  *   - `batch` >= 1 stacks independent tensors (e.g. MoE experts) with a
  *     contiguous batch stride; each has its own FP32 scale s_g[batch].
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
- *     enqueue work on it and return without synchronising, except
- *     nvfp4_get_device_status and nvfp4_search_evaluations.  Argument errors are detected on the host
+ *     enqueue work on it and return without synchronising, except the status
+ *     and statistics reads (nvfp4_get_device_status, nvfp4_search_evaluations,
+ *     nvfp4_search_rescores).  Argument errors are detected on the host
  *     before anything is enqueued; a failed launch returns NVFP4_ERR_CUDA.
+ *   - Stream order holds between calls and with the caller's own work: a
+ *     call's first kernel starts after everything enqueued before it.  The
+ *     later kernels of a call are launched with programmatic stream
+ *     serialisation (their launch overlaps the previous kernel's tail; each
+ *     waits for it before touching memory).
  *   - A CUDA device must be current; all pointers must belong to it.
  *
  * Block-scale codes are E4M3 (FN variant) bit patterns, 0x00..0x7E.  The

@@ -354,9 +354,9 @@ __device__ __forceinline__ uint32_t pick4(uint32_t w0, uint32_t w1, uint32_t w2,
 // One candidate: codes, the tensor-core product u, z = p - s u, and the row
 // objective after a quad reduce-scatter (lanes t < 2: row g, t >= 2: row
 // g + 8).  tq holds the signed class quotients (moved off a possible
-// midpoint where one could occur), f scales them to this candidate exactly; sm0 and sm1 multiply
-// u in rows g and g + 8 (accumulator elements 0, 1 and 2, 3 of both n-tiles),
-// each row carrying its own power-of-two scale.
+// midpoint where one could occur), f scales them to this candidate exactly;
+// sm0 and sm1 multiply u in rows g and g + 8 (accumulator elements 0, 1 and
+// 2, 3 of both n-tiles), each row carrying its own power-of-two scale.
 template <bool kLH>
 __device__ __forceinline__ float candidate_objective(const float tq[8], float f, float sm0,
                                                      float sm1, const uint32_t bh[2][2],

@@ -273,6 +273,24 @@ __device__ __forceinline__ uint32_t max_rule_code_fast(float amax, const MaxRule
   return (ct & 1u) ? ct : ca;  // equal, or the odd one of two neighbours
 }
 
+// The same code with the fp64 residual only near a midpoint.  t as above is
+// within 2^-23.9 of q; fl(t (1 + 2^-22)) and fl(t (1 - 2^-22)) lie at least
+// 2^-22.4 t from t (the product's rounding takes at most 2^-24), so they
+// bracket q.  Where both round to the same code no E4M3 rounding midpoint lies
+// between them (nearest-even rounding is monotone, and a midpoint on an end
+// goes to that end's side, as q does), and that code is q's (saturation above
+// 448 included); otherwise, for a quotient within about 2^-22 of a midpoint,
+// the residual decides.
+__device__ __forceinline__ uint32_t max_rule_code_margin(float amax, const MaxRule &m) {
+  const float as = amax * m.pre;
+  const float t = fmaf(as, m.r_hi, as * m.r_lo);
+  const float2 b = __fmul2_rn(make_float2(t, t), make_float2(1.0f + 0x1p-22f, 1.0f - 0x1p-22f));
+  unsigned short pair;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(b.x), "f"(b.y));
+  const uint32_t cu = pair >> 8, cd = pair & 0xFFu;
+  return cu == cd ? cu : max_rule_code_fast(amax, m);
+}
+
 // bf16 pair of v(q) * s for one packed byte: fp32 product, then bf16 RN.
 __device__ __forceinline__ uint32_t dequant_byte(uint32_t byte, float s) {
   const uint32_t h2 = cvt_f16x2_from_e2m1x2(byte);
@@ -309,7 +327,7 @@ __global__ void __launch_bounds__(kThreads) max_rule_kernel(const uint16_t *__re
     uint32_t v[8];
     load_block(w + i * kBlock, v);
     const float amax = __uint_as_float(amax_bits8(v) << 16);
-    codes[i] = (uint8_t)max_rule_code_fast(amax, mr);
+    codes[i] = (uint8_t)max_rule_code_margin(amax, mr);
   }
 }
 
@@ -422,51 +440,85 @@ __device__ __noinline__ double block_mse64(const uint32_t w[8], uint2 q, float s
   return e;
 }
 
+// Per-CTA constants of Four Over Six: the two max rules (k = 6, 4).
+struct FourSixConsts {
+  MaxRule m6, m4;
+};
+
+// One block's Four Over Six code (see four_over_six_kernel).
+__device__ __forceinline__ uint32_t four_over_six_code(const uint32_t v[8],
+                                                       const ScaleEntry *tab,
+                                                       const FourSixConsts &cs, float2 pre,
+                                                       float2 r_hi, float2 r_lo) {
+  const float amax = __uint_as_float(amax_bits8(v) << 16);
+  // max_rule_code_margin for both codes at once: the quotients paired (each
+  // lane rounded as the scalar t), the brackets of both in two conversions
+  // (c4 in the upper byte), the residuals where either code is in doubt.
+  const float2 a = __fmul2_rn(make_float2(amax, amax), pre);
+  const float2 t = __ffma2_rn(a, r_hi, __fmul2_rn(a, r_lo));
+  const float2 tu = __fmul2_rn(t, make_float2(1.0f + 0x1p-22f, 1.0f + 0x1p-22f));
+  const float2 td = __fmul2_rn(t, make_float2(1.0f - 0x1p-22f, 1.0f - 0x1p-22f));
+  unsigned short pu, pd;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pu) : "f"(tu.y), "f"(tu.x));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pd) : "f"(td.y), "f"(td.x));
+  uint32_t c6 = pu & 0xFFu, c4 = pu >> 8;
+  if (pu != pd) {
+    c6 = max_rule_code_fast(amax, cs.m6);
+    c4 = max_rule_code_fast(amax, cs.m4);
+  }
+  const uint32_t lo = min(c4, c6), hi = max(c4, c6);
+  uint32_t code = lo;
+  if (amax > 0.0f && hi != lo) {
+    // fp32 screen; the exact fp64 comparison only when the two are close
+    // (relative 2^-16, or absolute 2^-130 for subnormal sums)
+    const ScaleEntry el = tab[lo], eh = tab[hi];
+    float fl, fh;
+    block_mse32_two(v, el, eh, fl, fh);
+    if (fabsf(fh - fl) > fmaf(0x1p-16f, fmaxf(fh, fl), 0x1p-130f)) {
+      code = fh < fl ? hi : lo;
+    } else {
+      const uint2 ql = encode_block_entry(v, el), qh = encode_block_entry(v, eh);
+      code = block_mse64(v, qh, eh.s) < block_mse64(v, ql, el.s) ? hi : lo;
+    }
+  }
+  return amax > 0.0f ? code : 0u;
+}
+
 // Four Over Six (the Local-Hessian write-up, "The NVFP4 structure": one of
 // two candidate scales per block): the max-rule code and the code of
 // amax / (4 s_g), whichever block MSE is smaller, the smaller code on a tie;
-// an all-zero block gets code 0.
-__global__ void __launch_bounds__(kThreads) four_over_six_kernel(const uint16_t *__restrict__ w,
-                                                                 int64_t nblk,
-                                                                 const float *__restrict__ s_g,
-                                                                 uint8_t *__restrict__ codes) {
+// an all-zero block gets code 0.  Blocks are taken two per loop pass, each
+// one's loads issued before the other's arithmetic.
+__global__ void __launch_bounds__(kThreads, 3)
+    four_over_six_kernel(const uint16_t *__restrict__ w, int64_t nblk,
+                         const float *__restrict__ s_g, uint8_t *__restrict__ codes) {
   chained_entry(w);
   const int64_t b = blockIdx.y;
   w += b * nblk * kBlock;
   codes += b * nblk;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  uint32_t v[8];
-  if (i < nblk) load_block(w + i * kBlock, v);
-  // the table is built while the first block is in flight
+  uint32_t va[8], vb[8];
+  if (i < nblk) load_block(w + i * kBlock, va);
+  // the max rules (by the first lane of each of two warps; the others read
+  // them) and the table are formed while the first block is in flight
   const float sg = s_g[b];
-  const MaxRule m6 = make_max_rule(sg, 6.0), m4 = make_max_rule(sg, 4.0);
+  __shared__ FourSixConsts cs;
   __shared__ ScaleEntry tab[256];
+  if (threadIdx.x == 0) cs.m6 = make_max_rule(sg, 6.0);
+  if (threadIdx.x == 32) cs.m4 = make_max_rule(sg, 4.0);
   fill_scale_table(tab, sg);
-  for (; i < nblk; i += stride) {
-    uint32_t nv[8];
+  const float2 pre = make_float2(cs.m6.pre, cs.m4.pre);
+  const float2 r_hi = make_float2(cs.m6.r_hi, cs.m4.r_hi);
+  const float2 r_lo = make_float2(cs.m6.r_lo, cs.m4.r_lo);
+  while (i < nblk) {
     const int64_t n = i + stride;
-    if (n < nblk) load_block(w + n * kBlock, nv);
-    const float amax = __uint_as_float(amax_bits8(v) << 16);
-    const uint32_t c6 = max_rule_code_fast(amax, m6), c4 = max_rule_code_fast(amax, m4);
-    const uint32_t lo = min(c4, c6), hi = max(c4, c6);
-    uint32_t code = lo;
-    if (amax > 0.0f && hi != lo) {
-      // fp32 screen; the exact fp64 comparison only when the two are close
-      // (relative 2^-16, or absolute 2^-130 for subnormal sums)
-      const ScaleEntry el = tab[lo], eh = tab[hi];
-      float fl, fh;
-      block_mse32_two(v, el, eh, fl, fh);
-      if (fabsf(fh - fl) > fmaf(0x1p-16f, fmaxf(fh, fl), 0x1p-130f)) {
-        code = fh < fl ? hi : lo;
-      } else {
-        const uint2 ql = encode_block_entry(v, el), qh = encode_block_entry(v, eh);
-        code = block_mse64(v, qh, eh.s) < block_mse64(v, ql, el.s) ? hi : lo;
-      }
-    }
-    codes[i] = (uint8_t)(amax > 0.0f ? code : 0u);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = nv[j];
+    if (n < nblk) load_block(w + n * kBlock, vb);
+    codes[i] = (uint8_t)four_over_six_code(va, tab, cs, pre, r_hi, r_lo);
+    if (n >= nblk) break;
+    i = n + stride;
+    if (i < nblk) load_block(w + i * kBlock, va);
+    codes[n] = (uint8_t)four_over_six_code(vb, tab, cs, pre, r_hi, r_lo);
   }
 }
 
@@ -528,8 +580,26 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t *__rest
   }
 }
 
+// One block of the fused fake-quant: max-rule code, exact E2M1 codes, the
+// dequantised bf16 values, and the optional packed codes and block code.
+__device__ __forceinline__ void fake_quant_block(const uint32_t v[8], int64_t i,
+                                                 const ScaleEntry *tab, const MaxRule &mr,
+                                                 uint16_t *out, uint8_t *packed,
+                                                 uint8_t *codes) {
+  const float amax = __uint_as_float(amax_bits8(v) << 16);
+  const uint32_t code = max_rule_code_margin(amax, mr);
+  const ScaleEntry se = tab[code];
+  const uint2 q = encode_block_entry(v, se);
+  const uint32_t bytes[8] = {q.x & 0xFFu, (q.x >> 8) & 0xFFu, (q.x >> 16) & 0xFFu, q.x >> 24,
+                             q.y & 0xFFu, (q.y >> 8) & 0xFFu, (q.y >> 16) & 0xFFu, q.y >> 24};
+  store_dequant(out + i * kBlock, bytes, se.s);
+  if (packed) st_stream_v2(packed + i * 8, q);
+  if (codes) codes[i] = (uint8_t)code;
+}
+
 // Fused fake-quant pass (after the tensor scale is known): max rule, encode,
-// dequantise; optional packed codes and block codes.
+// dequantise; optional packed codes and block codes.  Blocks are taken two
+// per loop pass, each one's loads issued before the other's arithmetic.
 __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__restrict__ x,
                                                               int64_t nblk,
                                                               const float *__restrict__ s_g,
@@ -539,30 +609,21 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__
   chained_entry(x);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  uint32_t v[8];
-  if (i < nblk) load_block(x + i * kBlock, v);
+  uint32_t va[8], vb[8];
+  if (i < nblk) load_block(x + i * kBlock, va);
   // the table is built while the first block is in flight
   const float sg = *s_g;
   const MaxRule mr = make_max_rule(sg);
   __shared__ ScaleEntry tab[256];
   fill_scale_table(tab, sg);
-  for (; i < nblk; i += stride) {
-    // issue the next block's loads before this block's arithmetic
-    uint32_t nv[8];
+  while (i < nblk) {
     const int64_t n = i + stride;
-    if (n < nblk) load_block(x + n * kBlock, nv);
-    const float amax = __uint_as_float(amax_bits8(v) << 16);
-    const uint32_t code = max_rule_code_fast(amax, mr);
-    const ScaleEntry se = tab[code];
-    const float s = se.s;
-    const uint2 q = encode_block_entry(v, se);
-    const uint32_t bytes[8] = {q.x & 0xFFu, (q.x >> 8) & 0xFFu, (q.x >> 16) & 0xFFu, q.x >> 24,
-                               q.y & 0xFFu, (q.y >> 8) & 0xFFu, (q.y >> 16) & 0xFFu, q.y >> 24};
-    store_dequant(out + i * kBlock, bytes, s);
-    if (packed) st_stream_v2(packed + i * 8, q);
-    if (codes) codes[i] = (uint8_t)code;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = nv[j];
+    if (n < nblk) load_block(x + n * kBlock, vb);
+    fake_quant_block(va, i, tab, mr, out, packed, codes);
+    if (n >= nblk) break;
+    i = n + stride;
+    if (i < nblk) load_block(x + i * kBlock, va);
+    fake_quant_block(vb, n, tab, mr, out, packed, codes);
   }
 }
 
@@ -686,7 +747,7 @@ cudaError_t launch_scale_max(const uint16_t *w, int64_t batch, int64_t nblk, con
 cudaError_t launch_four_over_six(const uint16_t *w, int64_t batch, int64_t nblk,
                                  const float *s_g, uint8_t *codes, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
-  const int gx = amortised_grid(batch, nblk, 3);  // 77 registers: three CTAs per SM
+  const int gx = amortised_grid(batch, nblk, 3);  // 78 registers: three CTAs per SM
   return launch_first(four_over_six_kernel, dim3(gx, (unsigned)batch), dim3(kThreads), 0, st,
                         w, nblk, s_g, codes);
 }

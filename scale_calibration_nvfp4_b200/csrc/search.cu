@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(32)
 
 // Resident CTAs per SM.  Local-Hessian eight (64 registers, 8 bytes of
 // spill; measured 1.9% faster on the MoE experts and 1.3% on the dense layer
-// than 66 registers at seven); MSE nine (56 registers).
+// than 66 registers at seven); MSE nine (53 registers).
 constexpr int kLhCtasPerSm = 8, kMseCtasPerSm = 9;
 
 template <bool kLH, int kRowsPerCta>
@@ -837,7 +837,7 @@ __global__ void __launch_bounds__(kThreads, kLH ? kLhCtasPerSm : kMseCtasPerSm)
           tq[e] = t2.x;
           tq[e + 1] = t2.y;
         }
-      } else {  // (paired, the MSE kernel would pass its 56 registers)
+      } else {  // unpaired: the paired form spilled at nine MSE CTAs per SM
 #pragma unroll
         for (int e = 0; e < 8; ++e) tq[e] = fmaf(xs[e], ci.r_hi, xs[e] * ci.r_lo);
       }

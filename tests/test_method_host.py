@@ -175,13 +175,14 @@ def _e4m3_rn_satfinite(t):
     return np.where(a >= vals[0x7E], 0x7E, code)
 
 
-def _max_rule_code(amax, s_g, k):
+def _max_rule_code(amax, s_g, k, fast=False):
     """The kernel's E4M3 code of amax / (k s_g): D = k s_g exact in fp64,
     R = fl64(1/D) (times 2^-64 where R > 2^100, amax then times 2^64) split
     r_hi = fl32(R), r_lo = fl32(R - r_hi); t = fl32(a r_hi + fl32(a r_lo))
     with a the (pre-scaled) amax; ta = the float next to t across the
     quotient (the sign of amax - t D); the code is RN(t) when RN(t) and
-    RN(ta) agree or RN(t) is odd, else RN(ta)."""
+    RN(ta) agree or RN(t) is odd, else RN(ta).  fast: RN(t) alone ("t": t
+    itself)."""
     ld = np.longdouble
     D = float(k) * float(np.float32(s_g))
     R = 1.0 / D
@@ -193,6 +194,10 @@ def _max_rule_code(amax, s_g, k):
     r_lo = np.float32(R - float(r_hi))
     a = np.asarray(amax, np.float32).astype(ld) * ld(pre)
     t = _f32(a * ld(r_hi) + _f32(a * ld(r_lo)).astype(ld))
+    if fast == "t":
+        return t
+    if fast:
+        return _e4m3_rn_satfinite(t)
     rho = np.asarray(amax, np.float32).astype(ld) - t.astype(ld) * ld(D)
     ta = np.where(rho > 0, np.nextafter(t, np.float32(np.inf)),
                   np.where(rho < 0, np.nextafter(t, np.float32(-np.inf)), t))
@@ -237,6 +242,63 @@ def test_kernel_scale_code_near_midpoints(oracle_mod):
                 t = _f32(np.longdouble(a) / np.longdouble(6 * float(s)))
                 bad += int(_e4m3_rn_satfinite(t)[()] != ref)
     assert bad > 0
+
+
+def _max_rule_t(amax, s_g, k):
+    return _max_rule_code(amax, s_g, k, fast="t")
+
+
+def _margin_max_code(amax, s_g, k):
+    """The streaming kernels' code of amax / (k s_g) (the max rule, k = 6;
+    Four Over Six's two codes, k = 6 and 4): t as in _max_rule_code, then
+    tu = fl32(t (1 + 2^-22)) and td = fl32(t (1 - 2^-22)); where RN(tu) ==
+    RN(td) that code, else the exact-residual code.  Returns the codes and
+    where the residual decided."""
+    tu = _f32(_max_rule_t(amax, s_g, k).astype(np.float64) * float(np.float32(1 + 2.0 ** -22)))
+    td = _f32(_max_rule_t(amax, s_g, k).astype(np.float64) * float(np.float32(1 - 2.0 ** -22)))
+    cu, cd = _e4m3_rn_satfinite(tu), _e4m3_rn_satfinite(td)
+    slow = cu != cd
+    return np.where(slow, _max_rule_code(amax, s_g, k), cu), slow
+
+
+def test_max_rule_code_margin_rule_is_exact(oracle_mod):
+    """Every positive finite bf16 amax whose quotient lies in [2^-12, 512], at
+    tensor scales fl32(a / 2688) (a bf16), at random fp32 scales, and at
+    scales built so that a quotient sits on, or one float off, an E4M3
+    midpoint: the margin rule gives the oracle's code.  On the built scales
+    the residual decides some blocks and RN(t) alone would be wrong on some.
+    On tensor scales it decides under 1% of the bf16 values: those a simple
+    ratio away from the tensor maximum (3/4, 1/2 ... of it; 2^-16 of it),
+    whose quotients lie within one rounding of s_g of a midpoint (21 2^j,
+    7 2^-10), since 6 s_g and 4 s_g are the maximum over 448 and 672."""
+    rng = np.random.default_rng(17)
+    a = bits_to_f64(rng.integers(0x3F80, 0x4000, 8).astype(np.uint16))
+    tensor = (a * np.exp2(rng.integers(-60, 60, a.size)) / 2688).astype(np.float32)
+    rand = (rng.integers(0x0D800000, 0x71800000, 6).astype(np.uint32)).view(np.float32)
+    u = np.arange(1, 0x7F80, dtype=np.uint32).astype(np.uint16)
+    allb = bits_to_f64(u)
+    n_slow = {"tensor": 0, "built": 0}
+    n_blocks = {"tensor": 0, "built": 0}
+    wrong_alone = 0
+    for k in (6, 4):
+        mids = np.array([o * 2.0 ** j for o in (1, 7, 17, 21, 31) for j in (-10, -3, 5)])
+        amx = bits_to_f64(rng.integers(0x3000, 0x4F00, mids.size).astype(np.uint16))
+        sb = (amx / (k * mids)).astype(np.float32)
+        built = np.concatenate([sb, np.nextafter(sb, np.float32(np.inf))])
+        for kind, scales in (("tensor", tensor), ("rand", rand), ("built", built)):
+            for s_g in scales:
+                Dk = k * float(s_g)
+                q = allb / Dk
+                amax = allb[(q >= 2.0 ** -12) & (q <= 512)]
+                ref = np.array([oracle_mod.e4m3_round_quotient(x, Dk) for x in amax])
+                code, slow = _margin_max_code(amax, s_g, k)
+                assert np.array_equal(code, ref), (k, kind, float(s_g))
+                wrong_alone += int(np.sum(_max_rule_code(amax, s_g, k, fast=True) != ref))
+                if kind in n_slow:
+                    n_slow[kind] += int(slow.sum())
+                    n_blocks[kind] += amax.size
+    assert n_slow["built"] > 0 and wrong_alone > 0
+    assert 0 < n_slow["tensor"] < 1e-2 * n_blocks["tensor"]
 
 
 # ------------------------------------------- class quotients of the search

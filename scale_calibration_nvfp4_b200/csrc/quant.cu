@@ -207,7 +207,7 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
 // x = -0 keeps its sign in t), or 0 for scales outside [2^-100, 2^100) (below,
 // the reciprocal may overflow; above, r_lo is subnormal and too coarse near
 // the top of the fp32 range), zero or NaN, which take the exact fp64 encode.
-struct ScaleEntry {
+struct __align__(16) ScaleEntry {  // one 128-bit shared-memory load
   float s, r_hi, r_lo;
   uint32_t exact64;
 };
@@ -445,16 +445,28 @@ struct FourSixConsts {
   MaxRule m6, m4;
 };
 
-// One block's Four Over Six code (see four_over_six_kernel).
+// The exact fp64 comparison of Four Over Six's two candidates (codes lo <
+// hi) for a block whose fp32 screen could not separate them; the block by
+// value, so that the caller keeps nothing in memory for this rare path.
+__device__ __noinline__ uint32_t four_over_six_exact(uint4 w0, uint4 w1, ScaleEntry el,
+                                                     ScaleEntry eh, uint32_t lo, uint32_t hi) {
+  const uint32_t v[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  const uint2 ql = encode_block_entry(v, el), qh = encode_block_entry(v, eh);
+  return block_mse64(v, qh, eh.s) < block_mse64(v, ql, el.s) ? hi : lo;
+}
+
+// One block's Four Over Six code (see four_over_six_kernel).  plain: neither
+// max rule pre-scales its quotient (so amax enters as it is).
 __device__ __forceinline__ uint32_t four_over_six_code(const uint32_t v[8],
                                                        const ScaleEntry *tab,
-                                                       const FourSixConsts &cs, float2 pre,
+                                                       const FourSixConsts &cs, bool plain,
                                                        float2 r_hi, float2 r_lo) {
   const float amax = __uint_as_float(amax_bits8(v) << 16);
   // max_rule_code_margin for both codes at once: the quotients paired (each
   // lane rounded as the scalar t), the brackets of both in two conversions
-  // (c4 in the upper byte), the residuals where either code is in doubt.
-  const float2 a = __fmul2_rn(make_float2(amax, amax), pre);
+  // (c4 in the upper byte), the residuals where either code is in doubt or a
+  // max rule pre-scales.
+  const float2 a = make_float2(amax, amax);
   const float2 t = __ffma2_rn(a, r_hi, __fmul2_rn(a, r_lo));
   const float2 tu = __fmul2_rn(t, make_float2(1.0f + 0x1p-22f, 1.0f + 0x1p-22f));
   const float2 td = __fmul2_rn(t, make_float2(1.0f - 0x1p-22f, 1.0f - 0x1p-22f));
@@ -462,9 +474,21 @@ __device__ __forceinline__ uint32_t four_over_six_code(const uint32_t v[8],
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pu) : "f"(tu.y), "f"(tu.x));
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pd) : "f"(td.y), "f"(td.x));
   uint32_t c6 = pu & 0xFFu, c4 = pu >> 8;
-  if (pu != pd) {
+  if (!plain) {
     c6 = max_rule_code_fast(amax, cs.m6);
     c4 = max_rule_code_fast(amax, cs.m4);
+  } else if (pu != pd) {
+    // max_rule_code_fast's residual step on the quotients already formed
+    const double A = (double)amax;
+    const double r6 = fma(-(double)t.x, cs.m6.D, A), r4 = fma(-(double)t.y, cs.m4.D, A);
+    const float a6 = __int_as_float(__float_as_int(t.x) + (r6 > 0.0 ? 1 : (r6 < 0.0 ? -1 : 0)));
+    const float a4 = __int_as_float(__float_as_int(t.y) + (r4 > 0.0 ? 1 : (r4 < 0.0 ? -1 : 0)));
+    unsigned short pt, pa;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pt) : "f"(t.y), "f"(t.x));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pa) : "f"(a4), "f"(a6));
+    const uint32_t t6 = pt & 0xFFu, t4 = pt >> 8;
+    c6 = (t6 & 1u) ? t6 : (pa & 0xFFu);  // equal, or the odd one of two neighbours
+    c4 = (t4 & 1u) ? t4 : (uint32_t)(pa >> 8);
   }
   const uint32_t lo = min(c4, c6), hi = max(c4, c6);
   uint32_t code = lo;
@@ -477,8 +501,8 @@ __device__ __forceinline__ uint32_t four_over_six_code(const uint32_t v[8],
     if (fabsf(fh - fl) > fmaf(0x1p-16f, fmaxf(fh, fl), 0x1p-130f)) {
       code = fh < fl ? hi : lo;
     } else {
-      const uint2 ql = encode_block_entry(v, el), qh = encode_block_entry(v, eh);
-      code = block_mse64(v, qh, eh.s) < block_mse64(v, ql, el.s) ? hi : lo;
+      code = four_over_six_exact(make_uint4(v[0], v[1], v[2], v[3]),
+                                 make_uint4(v[4], v[5], v[6], v[7]), el, eh, lo, hi);
     }
   }
   return amax > 0.0f ? code : 0u;
@@ -487,8 +511,7 @@ __device__ __forceinline__ uint32_t four_over_six_code(const uint32_t v[8],
 // Four Over Six (the Local-Hessian write-up, "The NVFP4 structure": one of
 // two candidate scales per block): the max-rule code and the code of
 // amax / (4 s_g), whichever block MSE is smaller, the smaller code on a tie;
-// an all-zero block gets code 0.  Blocks are taken two per loop pass, each
-// one's loads issued before the other's arithmetic.
+// an all-zero block gets code 0.
 __global__ void __launch_bounds__(kThreads, 3)
     four_over_six_kernel(const uint16_t *__restrict__ w, int64_t nblk,
                          const float *__restrict__ s_g, uint8_t *__restrict__ codes) {
@@ -498,8 +521,8 @@ __global__ void __launch_bounds__(kThreads, 3)
   codes += b * nblk;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  uint32_t va[8], vb[8];
-  if (i < nblk) load_block(w + i * kBlock, va);
+  uint32_t v[8];
+  if (i < nblk) load_block(w + i * kBlock, v);
   // the max rules (by the first lane of each of two warps; the others read
   // them) and the table are formed while the first block is in flight
   const float sg = s_g[b];
@@ -508,17 +531,17 @@ __global__ void __launch_bounds__(kThreads, 3)
   if (threadIdx.x == 0) cs.m6 = make_max_rule(sg, 6.0);
   if (threadIdx.x == 32) cs.m4 = make_max_rule(sg, 4.0);
   fill_scale_table(tab, sg);
-  const float2 pre = make_float2(cs.m6.pre, cs.m4.pre);
+  const bool plain = cs.m6.pre == 1.0f && cs.m4.pre == 1.0f;
   const float2 r_hi = make_float2(cs.m6.r_hi, cs.m4.r_hi);
   const float2 r_lo = make_float2(cs.m6.r_lo, cs.m4.r_lo);
-  while (i < nblk) {
+  for (; i < nblk; i += stride) {
+    // issue the next block's loads before this block's arithmetic
+    uint32_t nv[8];
     const int64_t n = i + stride;
-    if (n < nblk) load_block(w + n * kBlock, vb);
-    codes[i] = (uint8_t)four_over_six_code(va, tab, cs, pre, r_hi, r_lo);
-    if (n >= nblk) break;
-    i = n + stride;
-    if (i < nblk) load_block(w + i * kBlock, va);
-    codes[n] = (uint8_t)four_over_six_code(vb, tab, cs, pre, r_hi, r_lo);
+    if (n < nblk) load_block(w + n * kBlock, nv);
+    codes[i] = (uint8_t)four_over_six_code(v, tab, cs, plain, r_hi, r_lo);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = nv[j];
   }
 }
 
@@ -598,8 +621,7 @@ __device__ __forceinline__ void fake_quant_block(const uint32_t v[8], int64_t i,
 }
 
 // Fused fake-quant pass (after the tensor scale is known): max rule, encode,
-// dequantise; optional packed codes and block codes.  Blocks are taken two
-// per loop pass, each one's loads issued before the other's arithmetic.
+// dequantise; optional packed codes and block codes.
 __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__restrict__ x,
                                                               int64_t nblk,
                                                               const float *__restrict__ s_g,
@@ -609,21 +631,21 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__
   chained_entry(x);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  uint32_t va[8], vb[8];
-  if (i < nblk) load_block(x + i * kBlock, va);
+  uint32_t v[8];
+  if (i < nblk) load_block(x + i * kBlock, v);
   // the table is built while the first block is in flight
   const float sg = *s_g;
   const MaxRule mr = make_max_rule(sg);
   __shared__ ScaleEntry tab[256];
   fill_scale_table(tab, sg);
-  while (i < nblk) {
+  for (; i < nblk; i += stride) {
+    // issue the next block's loads before this block's arithmetic
+    uint32_t nv[8];
     const int64_t n = i + stride;
-    if (n < nblk) load_block(x + n * kBlock, vb);
-    fake_quant_block(va, i, tab, mr, out, packed, codes);
-    if (n >= nblk) break;
-    i = n + stride;
-    if (i < nblk) load_block(x + i * kBlock, va);
-    fake_quant_block(vb, n, tab, mr, out, packed, codes);
+    if (n < nblk) load_block(x + n * kBlock, nv);
+    fake_quant_block(v, i, tab, mr, out, packed, codes);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = nv[j];
   }
 }
 

@@ -603,23 +603,6 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t *__rest
   }
 }
 
-// One block of the fused fake-quant: max-rule code, exact E2M1 codes, the
-// dequantised bf16 values, and the optional packed codes and block code.
-__device__ __forceinline__ void fake_quant_block(const uint32_t v[8], int64_t i,
-                                                 const ScaleEntry *tab, const MaxRule &mr,
-                                                 uint16_t *out, uint8_t *packed,
-                                                 uint8_t *codes) {
-  const float amax = __uint_as_float(amax_bits8(v) << 16);
-  const uint32_t code = max_rule_code_margin(amax, mr);
-  const ScaleEntry se = tab[code];
-  const uint2 q = encode_block_entry(v, se);
-  const uint32_t bytes[8] = {q.x & 0xFFu, (q.x >> 8) & 0xFFu, (q.x >> 16) & 0xFFu, q.x >> 24,
-                             q.y & 0xFFu, (q.y >> 8) & 0xFFu, (q.y >> 16) & 0xFFu, q.y >> 24};
-  store_dequant(out + i * kBlock, bytes, se.s);
-  if (packed) st_stream_v2(packed + i * 8, q);
-  if (codes) codes[i] = (uint8_t)code;
-}
-
 // Fused fake-quant pass (after the tensor scale is known): max rule, encode,
 // dequantise; optional packed codes and block codes.
 __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__restrict__ x,
@@ -643,7 +626,16 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(const uint16_t *__
     uint32_t nv[8];
     const int64_t n = i + stride;
     if (n < nblk) load_block(x + n * kBlock, nv);
-    fake_quant_block(v, i, tab, mr, out, packed, codes);
+    const float amax = __uint_as_float(amax_bits8(v) << 16);
+    const uint32_t code = max_rule_code_fast(amax, mr);
+    const ScaleEntry se = tab[code];
+    const float s = se.s;
+    const uint2 q = encode_block_entry(v, se);
+    const uint32_t bytes[8] = {q.x & 0xFFu, (q.x >> 8) & 0xFFu, (q.x >> 16) & 0xFFu, q.x >> 24,
+                               q.y & 0xFFu, (q.y >> 8) & 0xFFu, (q.y >> 16) & 0xFFu, q.y >> 24};
+    store_dequant(out + i * kBlock, bytes, s);
+    if (packed) st_stream_v2(packed + i * 8, q);
+    if (codes) codes[i] = (uint8_t)code;
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = nv[j];
   }

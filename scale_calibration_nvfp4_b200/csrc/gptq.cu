@@ -24,7 +24,7 @@
 //    Hd in place, 128-column panels (the diagonal block factored and
 //    inverted by one CTA, the rows below it solved by a GEMM with that
 //    inverse, the trailing matrix by a rank-128 update split so that most of
-//    it overlaps the next panel on a second stream of lower priority);
+//    it overlaps the next panel on a second stream);
 //  - gptq_block_kernel: 128 columns at a time, four lanes per row each
 //    holding 32 columns' running sums in registers; each column is rounded
 //    by its owner lane (exact fp64 midpoint test), its error shuffled to the
@@ -32,9 +32,7 @@
 //    replace the consumed sums;
 //  - the fp64 GEMM (fp64 tensor-core MMA) again: each block's errors times
 //    the next rows of T, added to the running sums of every later column
-//    (lazy batch updates, rank 128), split like the Cholesky's: the next
-//    block's columns first, the columns beyond on the second stream, where
-//    they overlap the next block's column loop.
+//    (lazy batch updates, rank 128).
 #include <cmath>
 #include <mutex>
 
@@ -430,18 +428,20 @@ cudaError_t ensure_smem_attr(K kernel, int bytes, std::mutex &mu, bool *flags) {
 
 // Linv: scratch [batch][128][128].
 // Look-ahead: each panel's trailing update is split into the next panel's
-// 128 columns, on the main stream st, and the columns beyond, on the side
+// 128 columns, on the caller's stream, and the columns beyond, on a second
 // stream, where it overlaps the next panel's factor and solve.  The next
 // panel's own split update waits for it (both write the columns after the
-// next panel); everything else they touch is disjoint.  On return every
-// kernel of the factorisation is ordered before st's next work (the side
-// stream is joined); ev_main and ev_side are the caller's events.
+// next panel); everything else they touch is disjoint.
 cudaError_t cholesky_in_place(double *A, int64_t C, int64_t batch, double *Linv,
-                              cudaStream_t st, cudaStream_t side, cudaEvent_t ev_main,
-                              cudaEvent_t ev_side) {
+                              cudaStream_t st) {
   cudaError_t e = ensure_smem_attr(chol_block_kernel, kCholSmem, g_chol_attr_mu, g_chol_attr);
   if (e != cudaSuccess) return e;
   const int64_t CC = C * C;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_main = nullptr, ev_side = nullptr;
+  e = cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_main, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_side, cudaEventDisableTiming);
   bool side_used = false;
   // A[r0.., r0 .. r0+ncols) -= X X^T on the lower triangle, X = the panel's
   // rows r0.. in its columns P0 .. P0+nw
@@ -482,11 +482,14 @@ cudaError_t cholesky_in_place(double *A, int64_t C, int64_t batch, double *Linv,
       side_used = side_used || e == cudaSuccess;
     }
   }
-  // join the side stream before anything reads the factor
+  // join the second stream before anything reads the factor
   if (side_used) {
     const cudaError_t ej = cudaStreamWaitEvent(st, ev_side, 0);
     if (e == cudaSuccess) e = ej;
   }
+  if (ev_main) cudaEventDestroy(ev_main);
+  if (ev_side) cudaEventDestroy(ev_side);
+  if (side) cudaStreamDestroy(side);
   return e;
 }
 
@@ -664,79 +667,28 @@ cudaError_t launch_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
       e = launch_chained(gptq_prepare_kernel, dim3((unsigned)gx, (unsigned)batch), dim3(256), 0,
                          st, H, C, static_cast<const double *>(lam), Hd);
   }
-  // The factorisation and the column loop run on a stream of the highest
-  // priority (hs) and their large trailing updates on a side stream of the
-  // lowest: the factor and column-block kernels, one CTA per Hessian or per
-  // 32 rows on the critical path, take the first SM slots that free up while
-  // an update's CTAs fill the rest.  hs starts after the work above; st
-  // waits for both streams before the scratch is released.
-  cudaStream_t hs = nullptr, side = nullptr;
-  cudaEvent_t ev_start = nullptr, ev_main = nullptr, ev_side = nullptr, ev_done = nullptr;
-  int prio_least = 0, prio_greatest = 0;
-  if (e == cudaSuccess) e = cudaDeviceGetStreamPriorityRange(&prio_least, &prio_greatest);
-  if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&hs, cudaStreamNonBlocking, prio_greatest);
-  if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&side, cudaStreamNonBlocking, prio_least);
-  for (cudaEvent_t *ev : {&ev_start, &ev_main, &ev_side, &ev_done})
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
-  bool hs_used = false;
-  if (e == cudaSuccess) e = cudaEventRecord(ev_start, st);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(hs, ev_start, 0);
-  hs_used = e == cudaSuccess;
-  if (e == cudaSuccess) e = cholesky_in_place(Hd, C, batch, Linv, hs, side, ev_main, ev_side);
+  if (e == cudaSuccess) e = cholesky_in_place(Hd, C, batch, Linv, st);
   // columns in blocks of 128: each row of a block on a quad of lanes, then the
-  // block's errors added to the running sums of every later column (rank-128):
-  // the next block's columns on hs, the columns beyond on the side stream,
-  // where they overlap the next block.  Block k reads the updates of blocks
-  // k - 1 (hs, in order) and k - 2 and before (side: each small update waits
-  // for the side stream's previous update, which writes its columns too).
+  // block's errors added to the running sums of every later column (rank-128)
   if (e == cudaSuccess)
     e = ensure_smem_attr(gptq_block_kernel, kBlockSmem, g_block_attr_mu, g_block_attr);
   const int64_t RC = R * C, CC = C * C;
-  // SD[:, n0 : n0 + n] += SD[:, c0 : c0 + nw] T[c0 : c0 + nw, n0 : n0 + n],
-  // T[i][j] = Hd[C-1-i][C-1-j]
-  auto update = [&](int64_t c0, int nw, int64_t n0, int64_t n, cudaStream_t s) {
-    GemmF64 g{};
-    g.M = R; g.N = n; g.K = nw; g.alpha = 1.0;
-    g.A = SD + c0; g.sAm = C; g.sAk = 1; g.bsA = RC;
-    g.B = Hd + (C - 1 - c0) * C + (C - 1 - n0); g.sBk = -C; g.sBn = -1; g.bsB = CC;
-    g.C = SD + n0; g.sCm = C; g.sCn = 1; g.bsC = RC;
-    return gemm_f64(g, batch, s);
-  };
-  bool side_used = false;
   for (int64_t c0 = 0; e == cudaSuccess && c0 < C; c0 += kBig) {
     const int nw = (int)(C - c0 < kBig ? C - c0 : kBig);
     const dim3 grid((unsigned)((R + kRowsPerCta - 1) / kRowsPerCta), (unsigned)batch);
-    e = launch_chained(gptq_block_kernel, grid, dim3(kBlockThreads), kBlockSmem, hs, w, R, C, s_g,
+    e = launch_chained(gptq_block_kernel, grid, dim3(kBlockThreads), kBlockSmem, st, w, R, C, s_g,
                        codes, static_cast<const double *>(Hd), SD, packed, c0, nw);
     const int64_t c1 = c0 + nw;
-    if (e != cudaSuccess || c1 >= C) continue;
-    const int64_t nw2 = C - c1 < kBig ? C - c1 : kBig, c2 = c1 + nw2;
-    if (side_used) e = cudaStreamWaitEvent(hs, ev_side, 0);
-    if (e == cudaSuccess) e = update(c0, nw, c1, nw2, hs);
-    if (e == cudaSuccess && c2 < C) {
-      e = cudaEventRecord(ev_main, hs);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev_main, 0);
-      if (e == cudaSuccess) e = update(c0, nw, c2, C - c2, side);
-      if (e == cudaSuccess) e = cudaEventRecord(ev_side, side);
-      side_used = side_used || e == cudaSuccess;
+    if (e == cudaSuccess && c1 < C) {
+      // SD[:, c1:] += SD[:, c0:c1] T[c0:c1, c1:], T[i][j] = Hd[C-1-i][C-1-j]
+      GemmF64 g{};
+      g.M = R; g.N = C - c1; g.K = nw; g.alpha = 1.0;
+      g.A = SD + c0; g.sAm = C; g.sAk = 1; g.bsA = RC;
+      g.B = Hd + (C - 1 - c0) * C + (C - 1 - c1); g.sBk = -C; g.sBn = -1; g.bsB = CC;
+      g.C = SD + c1; g.sCm = C; g.sCn = 1; g.bsC = RC;
+      e = gemm_f64(g, batch, st);
     }
   }
-  // join: st after everything on hs and on the side stream (also on error,
-  // so that nothing still runs when the scratch is released)
-  if (hs_used) {
-    cudaError_t ej = side_used ? cudaStreamWaitEvent(hs, ev_side, 0) : cudaSuccess;
-    if (ej == cudaSuccess) ej = cudaEventRecord(ev_done, hs);
-    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(st, ev_done, 0);
-    if (ej != cudaSuccess) {  // st cannot be ordered after them: wait for them here
-      cudaStreamSynchronize(side);
-      cudaStreamSynchronize(hs);
-    }
-    if (e == cudaSuccess) e = ej;
-  }
-  for (cudaEvent_t ev : {ev_start, ev_main, ev_side, ev_done})
-    if (ev) cudaEventDestroy(ev);
-  if (hs) cudaStreamDestroy(hs);
-  if (side) cudaStreamDestroy(side);
   const cudaError_t ef = scratch_free(scratch, st);
   return e != cudaSuccess ? e : ef;
 }

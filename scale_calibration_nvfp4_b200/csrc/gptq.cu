@@ -25,11 +25,11 @@
 //    inverted by one CTA, the rows below it solved by a GEMM with that
 //    inverse, the trailing matrix by a rank-128 update split so that most of
 //    it overlaps the next panel on a second stream);
-//  - gptq_block_kernel: 128 columns at a time, four lanes per row each
-//    holding 32 columns' running sums in registers; each column is rounded
+//  - gptq_block_kernel: 128 columns at a time, sixteen lanes per row each
+//    holding 8 columns' running sums in registers; each column is rounded
 //    by its owner lane (exact fp64 midpoint test), its error shuffled to the
-//    quad and added times T to the later columns' sums; the errors w_j - q_j
-//    replace the consumed sums;
+//    row's lanes and added times T to the later columns' sums; the errors
+//    w_j - q_j replace the consumed sums;
 //  - the fp64 GEMM (fp64 tensor-core MMA) again: each block's errors times
 //    the next rows of T, added to the running sums of every later column
 //    (lazy batch updates, rank 128).
@@ -525,88 +525,120 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// E2M1 magnitude index of |x| / s for an fp64 x: the count of midpoints
-// mu_i s below |x| (ties to the even index), exact since mu_i s is exact in
-// fp64; 0 when s is not positive.
-__device__ __forceinline__ int e2m1_index64(double a, double s) {
-  if (!(s > 0.0)) return 0;
-  return (a > 0.25 * s) + (a >= 0.75 * s) + (a > 1.25 * s) + (a >= 1.75 * s) + (a > 2.5 * s) +
-         (a >= 3.5 * s) + (a > 5.0 * s);
-}
-
-__device__ __forceinline__ double e2m1_magnitude(int k) {
-  return k < 2 ? 0.5 * k : (1.0 + 0.5 * (double)(k & 1)) * (double)(1 << ((k >> 1) - 1));
-}
-
 // Columns c0 .. c0+nw-1 (nw <= 128) of every row: the value at rounding,
 // its code, and the error w - q written over the consumed running sum.  L is
 // the lower Cholesky factor of the reversed Hessian: T[i][j] = L[C-1-i][C-1-j].
-// A quad of lanes takes one row, lane q the columns 32q .. 32q+31 of the
-// block with their running sums in registers.  Column k = 32 q0 + kk is
-// rounded by its owner lane, whose error goes to the quad by a shuffle; then
-// every lane adds error x T[k][m] to the running sums of its columns m > k
-// (independent updates: the dependent chain per column is one fma and the
-// rounding).  The block of T (upper triangle) sits in shared memory.
-constexpr int kRowsPerCta = 32;                  // 128 threads, four per row
-constexpr int kBlockThreads = 4 * kRowsPerCta;
-constexpr int kBlockSmem = (kBig * kBig + kBig) * (int)sizeof(double);  // 132,096 B
+// kLanes lanes take one row, lane q the columns kCols q .. kCols q + kCols - 1
+// of the block (kCols = 128 / kLanes) with their running sums in registers.
+// Column k = kCols q0 + kk is rounded by its owner lane, whose error goes to
+// the row's lanes by a shuffle; then every lane adds error x T[k][m] to the
+// running sums of its columns m > k (independent updates: the dependent chain
+// per column is one fma and the rounding).  The block of T (upper triangle)
+// sits in shared memory, one copy per CTA of kRowsPerCta rows, each lane's
+// chunk of a row followed by one double of padding: at every step the lanes
+// of a row read one element of each chunk, kCols + 1 doubles apart, which
+// puts them in distinct banks (kCols apart they all shared one).
+constexpr int kRowsPerCta = 32;
+template <int kLanes>
+__host__ __device__ constexpr int block_row_stride() { return kBig + kLanes; }  // doubles
+template <int kLanes>
+constexpr int block_smem() {
+  return (kBig * block_row_stride<kLanes>() + kBig) * (int)sizeof(double);
+}
 
-__global__ void __launch_bounds__(kBlockThreads)
+template <int kLanes>
+__global__ void __launch_bounds__(kLanes * kRowsPerCta)
     gptq_block_kernel(const uint16_t *__restrict__ w, int64_t R, int64_t C,
                       const float *__restrict__ s_g, const uint8_t *__restrict__ codes,
                       const double *__restrict__ L, double *__restrict__ SD,
                       uint8_t *__restrict__ packed, int64_t c0, int nw) {
+  constexpr int kThreadsB = kLanes * kRowsPerCta;
+  constexpr int kCols = kBig / kLanes;  // columns per lane
+  constexpr int kTS = block_row_stride<kLanes>();
+  static_assert(kCols % 8 == 0, "a lane's columns are whole packed words");
   chained_entry();
   extern __shared__ double bsm[];
-  double *T = bsm;              // [j][k], j <= k
-  double *Tinv = T + kBig * kBig;  // 1 / T[k][k]
+  double *T = bsm;                // [j][k + k / kCols], j <= k
+  double *Tinv = T + kBig * kTS;  // 1 / T[k][k]
   const int64_t b = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, q = lane & 3;
+  const int tid = threadIdx.x, lane = tid & 31, q = lane & (kLanes - 1);
   const double *Lb = L + b * C * C;
   // stage T (upper triangle, zeros elsewhere) with asynchronous copies
-  for (int idx = tid; idx < kBig * kBig; idx += kBlockThreads) {
+  for (int idx = tid; idx < kBig * kBig; idx += kThreadsB) {
     const int j = idx / kBig, k = idx - j * kBig;
     const bool in = j <= k && k < nw;
-    cp_async8(T + idx, in ? Lb + (C - 1 - c0 - j) * C + (C - 1 - c0 - k) : Lb, in);
+    cp_async8(T + j * kTS + k + k / kCols, in ? Lb + (C - 1 - c0 - j) * C + (C - 1 - c0 - k) : Lb,
+              in);
   }
   cp_async_commit();
-  const int64_t r = (int64_t)blockIdx.x * kRowsPerCta + (tid >> 2);
+  const int64_t r = (int64_t)blockIdx.x * kRowsPerCta + tid / kLanes;
   const bool live = r < R;
   const int64_t row = b * R + (live ? r : 0);
-  const int cq = 32 * q;                  // first column of this lane
-  const int ncols = nw - cq;              // columns of this lane inside the block (<= 32)
+  const int cq = kCols * q;               // first column of this lane
+  const int ncols = nw - cq;              // columns of this lane inside the block
   double *sd = SD + row * C + c0 + cq;
   const uint16_t *wr = w + row * C + c0 + cq;
-  double S[32];
-  uint32_t wv[16];  // the lane's 32 bf16 weights, two per word
+  double S[kCols];
+  uint32_t wv[kCols / 2];  // the lane's bf16 weights, two per word
 #pragma unroll
-  for (int m = 0; m < 32; ++m) S[m] = (live && m < ncols) ? sd[m] : 0.0;
+  for (int m = 0; m < kCols; ++m) S[m] = (live && m < ncols) ? sd[m] : 0.0;
 #pragma unroll
-  for (int m = 0; m < 16; ++m)
+  for (int m = 0; m < kCols / 2; ++m)
     wv[m] = (live && 2 * m < ncols) ? *reinterpret_cast<const uint32_t *>(wr + 2 * m) : 0u;
   const float sg = s_g[b];
   const uint8_t *cr = codes + row * (C / kBlock) + (c0 + cq) / kBlock;
-  const double s_lo = (live && ncols > 0) ? (double)effective_scale(sg, cr[0]) : 0.0;
-  const double s_hi = (live && ncols > 16) ? (double)effective_scale(sg, cr[1]) : 0.0;
+  // the scales of the lane's columns (one per 16; one for kCols <= 16) and,
+  // per scale, the E2M1 rounding thresholds and grid values times it (exact
+  // in fp64), so that a column's rounding is seven compares and a select
+  // chain (the dependent chain from one column to the next is its fp64
+  // fmas, one compare, one subtraction and the shuffle)
+  constexpr int kScales = (kCols + kBlock - 1) / kBlock;
+  double thr[kScales][7], val[kScales][8];
+#pragma unroll
+  for (int i = 0; i < kScales; ++i) {
+    const double sc = (live && ncols > kBlock * i) ? (double)effective_scale(sg, cr[i]) : 0.0;
+    const double tf[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
+    const double vf[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    // no scale (s = 0, or not a number): every test fails, index 0
+    const double nan = __longlong_as_double(0x7FF8000000000000LL);
+#pragma unroll
+    for (int j = 0; j < 7; ++j) thr[i][j] = sc > 0.0 ? tf[j] * sc : nan;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) val[i][j] = vf[j] * sc;
+  }
   cp_async_wait_all();
   __syncthreads();
-  for (int k = tid; k < kBig; k += kBlockThreads) Tinv[k] = k < nw ? 1.0 / T[k * kBig + k] : 0.0;
+  for (int k = tid; k < kBig; k += kThreadsB)
+    Tinv[k] = k < nw ? 1.0 / T[k * kTS + k + k / kCols] : 0.0;
   __syncthreads();
-  uint32_t pk[4] = {0u, 0u, 0u, 0u};  // the lane's 32 codes
-  const int src = lane & ~3;
-  for (int q0 = 0; q0 < 4; ++q0) {
-    if (32 * q0 >= nw) break;
+  uint32_t pk[kCols / 8];  // the lane's codes
 #pragma unroll
-    for (int kk = 0; kk < 32; ++kk) {
-      const int k = 32 * q0 + kk;
+  for (int i = 0; i < kCols / 8; ++i) pk[i] = 0u;
+  const int src = lane & ~(kLanes - 1);
+  for (int q0 = 0; q0 < kLanes; ++q0) {
+    if (kCols * q0 >= nw) break;
+#pragma unroll
+    for (int kk = 0; kk < kCols; ++kk) {
+      const int k = kCols * q0 + kk;
       const bool valid = k < nw;
       // the owner lane rounds column k (every lane computes; only q == q0 keeps it)
       const double wk = (double)__uint_as_float(
           (kk & 1) ? (wv[kk >> 1] & 0xFFFF0000u) : (wv[kk >> 1] << 16));
       const double x = fma(S[kk], valid ? Tinv[k] : 0.0, wk);
-      const double sc = kk < 16 ? s_lo : s_hi;
-      const int kq = e2m1_index64(fabs(x), sc);
-      const double qv = e2m1_magnitude(kq) * sc;
+      // nearest-even E2M1 magnitude index of |x| / s (ties: 0.25, 1.25, 2.5
+      // and 5 go down, 0.75, 1.75 and 3.5 up; 0 where s = 0) and its value
+      const double a = fabs(x);
+      const double *th = thr[kk / kBlock], *vs = val[kk / kBlock];
+      const bool p0 = a > th[0], p1 = a >= th[1], p2 = a > th[2], p3 = a >= th[3];
+      const bool p4 = a > th[4], p5 = a >= th[5], p6 = a > th[6];
+      double qv = p0 ? vs[1] : vs[0];
+      qv = p1 ? vs[2] : qv;
+      qv = p2 ? vs[3] : qv;
+      qv = p3 ? vs[4] : qv;
+      qv = p4 ? vs[5] : qv;
+      qv = p5 ? vs[6] : qv;
+      qv = p6 ? vs[7] : qv;
+      const int kq = (int)p0 + (int)p1 + (int)p2 + (int)p3 + (int)p4 + (int)p5 + (int)p6;
       const bool neg = signbit(x);
       const double d = wk - (neg ? -qv : qv);
       if (q == q0) {
@@ -614,10 +646,10 @@ __global__ void __launch_bounds__(kBlockThreads)
         pk[kk >> 3] |= ((uint32_t)kq | (neg ? 8u : 0u)) << (4 * (kk & 7));
       }
       const double e = valid ? __shfl_sync(0xFFFFFFFFu, d, src | q0) : 0.0;
-      // running sums of the later columns of the quad's row
-      const double *Tk = T + k * kBig + cq;
+      // running sums of the later columns of the row
+      const double *Tk = T + k * kTS + cq + q;
 #pragma unroll
-      for (int m = 0; m < 32; ++m) {
+      for (int m = 0; m < kCols; ++m) {
         const bool later = q > q0 || (q == q0 && m > kk);
         if (later) S[m] = fma(e, Tk[m], S[m]);
       }
@@ -625,14 +657,21 @@ __global__ void __launch_bounds__(kBlockThreads)
   }
   if (!live) return;
 #pragma unroll
-  for (int m = 0; m < 32; ++m)
+  for (int m = 0; m < kCols; ++m)
     if (m < ncols) sd[m] = S[m];
   // byte stores: a row of packed codes starts on any 8-byte boundary
   uint8_t *pr = packed + row * (C / 2) + (c0 + cq) / 2;
 #pragma unroll
-  for (int i = 0; i < 16; ++i)
+  for (int i = 0; i < kCols / 2; ++i)
     if (2 * i < ncols) pr[i] = (uint8_t)(pk[i >> 2] >> (8 * (i & 3)));
 }
+
+// lanes per row of the column-block kernel: sixteen (eight columns each, 16
+// warps per SM) measured 4% faster on the dense layer's GPTQ than four (32
+// columns each, 4 warps per SM, latency-bound on each column's chain) and
+// eight, with the padded T rows; without the padding the lanes' reads of T
+// shared one bank and more lanes were slower
+constexpr int kBlockLanes = 16;
 
 std::mutex g_block_attr_mu;
 bool g_block_attr[64] = {};
@@ -668,16 +707,19 @@ cudaError_t launch_gptq(const uint16_t *w, int64_t batch, int64_t R, int64_t C, 
                          st, H, C, static_cast<const double *>(lam), Hd);
   }
   if (e == cudaSuccess) e = cholesky_in_place(Hd, C, batch, Linv, st);
-  // columns in blocks of 128: each row of a block on a quad of lanes, then the
+  // columns in blocks of 128: each row of a block on kBlockLanes lanes, then the
   // block's errors added to the running sums of every later column (rank-128)
   if (e == cudaSuccess)
-    e = ensure_smem_attr(gptq_block_kernel, kBlockSmem, g_block_attr_mu, g_block_attr);
+    e = ensure_smem_attr(gptq_block_kernel<kBlockLanes>, block_smem<kBlockLanes>(),
+                         g_block_attr_mu, g_block_attr);
   const int64_t RC = R * C, CC = C * C;
   for (int64_t c0 = 0; e == cudaSuccess && c0 < C; c0 += kBig) {
     const int nw = (int)(C - c0 < kBig ? C - c0 : kBig);
     const dim3 grid((unsigned)((R + kRowsPerCta - 1) / kRowsPerCta), (unsigned)batch);
-    e = launch_chained(gptq_block_kernel, grid, dim3(kBlockThreads), kBlockSmem, st, w, R, C, s_g,
-                       codes, static_cast<const double *>(Hd), SD, packed, c0, nw);
+    e = launch_chained(gptq_block_kernel<kBlockLanes>, grid, dim3(kBlockLanes * kRowsPerCta),
+                       block_smem<kBlockLanes>(), st, w, R, C, s_g, codes,
+                       static_cast<const double *>(Hd), SD,
+                       packed, c0, nw);
     const int64_t c1 = c0 + nw;
     if (e == cudaSuccess && c1 < C) {
       // SD[:, c1:] += SD[:, c0:c1] T[c0:c1, c1:], T[i][j] = Hd[C-1-i][C-1-j]

@@ -152,6 +152,33 @@ def test_gptq_diagonal_hessian_is_plain_rounding(nv):
     np.testing.assert_array_equal(out.cpu().numpy(), oracle.quantize_pack(wu, s_g, codes))
 
 
+def test_gptq_blocks_with_zero_scale(nv):
+    """Blocks whose scale code is 0: an all-zero block column, a zero row,
+    signed zeros, and blocks about 1e-7 of the tensor maximum, whose max-rule
+    code rounds to 0 although their values are not zero.  Every value there
+    gets magnitude index 0 with its sign, and all of it is the error carried
+    to the later columns; every row against the oracle."""
+    R, C = 64, 256
+    W = rand_bf16((R, C), 30, 0.02)
+    W[:, 16:32] = 0.0
+    W[5, :] = 0.0
+    W[7, 96:112] = -0.0
+    W[:, 64:80] = W[:, 64:80] * 1e-7
+    X = rand_bf16((300, C), 130, 1.0, outlier_cols=(C // 3,), factor=25.0)
+    wu = bf16_bits(W)
+    s_g = oracle.global_scale(wu)
+    Hf = oracle.gram_full(bf16_bits(X)).astype(np.float32)
+    codes = oracle.scale_search_max(wu, s_g)
+    assert np.all(codes[:, 1] == 0) and np.all(codes[:, 4] == 0)
+    assert np.count_nonzero(wu.reshape(R, C // 16, 16)[:, 4] & 0x7FFF) > R
+    out = nv.gptq(W.cuda(), torch.tensor([s_g]).cuda(), torch.from_numpy(codes).cuda(),
+                  torch.from_numpy(Hf).cuda(), 0.01)
+    U = oracle.gptq_factor(Hf.astype(np.float64), 0.01)
+    ref, wq = oracle.gptq_rows(wu, s_g, codes, U, np.arange(R))
+    compare_gptq(out.cpu().numpy(), ref, wq, scales_per_element(s_g, codes), max_near_frac=0.0)
+    assert nv.get_device_status() == "NVFP4_OK"
+
+
 def test_gptq_not_positive_definite_reports(nv):
     W, wu, s_g, codes, _ = _case(16, 32, 10, 21, "max")
     sg, cd = torch.tensor([s_g]).cuda(), torch.from_numpy(codes).cuda()

@@ -45,12 +45,15 @@ def scales_per_element(s_g, codes):
 
 
 def near_tie_rows(wq, S, rel=1e-9):
+    """Rows holding a value at rounding within rel of a midpoint times its
+    scale (past column 0).  A scale of 0 has no midpoint: every value
+    encodes to index 0 there, whatever it is."""
     a = np.abs(wq[:, 1:])
     S = S[:, 1:]
     near = np.zeros(wq.shape[0], bool)
     for m in MIDPOINTS:
         thr = m * S
-        near |= np.any(np.abs(a - thr) <= rel * thr, axis=1)
+        near |= np.any((np.abs(a - thr) <= rel * thr) & (S > 0), axis=1)
     return near
 
 

@@ -66,18 +66,19 @@ struct GemmF64 {
   int overwrite;  // C = alpha A B (C is not read)
 };
 
-// 128 x BN output tile per CTA (BN = 128 or 64) on the fp64 tensor-core
-// instruction (mma.sync m8n8k4 f64; tcgen05 has no f64 kind): eight warps,
-// each a grid of 8 x 8 accumulator tiles (64 x 32 per warp for BN = 128, one
-// CTA per SM; 32 x 32 for BN = 64, two CTAs per SM).  k-slabs of 16 are
+// BM x BN output tile per CTA (128 x 64 for out-of-place products, 64 x 128
+// for the in-place panel solve, which must be one CTA column) on the fp64
+// tensor-core instruction (mma.sync m8n8k4 f64; tcgen05 has no f64 kind):
+// eight warps, each a grid of 8 x 8 accumulator tiles (32 x 32 per warp, two
+// CTAs per SM).  k-slabs of 16 are
 // staged in shared memory by a three-stage cp.async pipeline (8-byte copies,
 // so any stride works; the unit-stride dimension is copied fastest), both
 // operands stored [row][k] with a row stride of 20 doubles, which keeps the
 // fragment reads (8 rows x 4 consecutive k) free of bank conflicts.
-constexpr int kGM = 128, kGK = 16, kGThreads = 256, kGStages = 3;
+constexpr int kGK = 16, kGThreads = 256, kGStages = 3;
 constexpr int kGRow = kGK + 4;  // shared-memory row stride (doubles)
-template <int BN>
-constexpr int gemm_smem() { return kGStages * (kGM + BN) * kGRow * (int)sizeof(double); }
+template <int BM, int BN>
+constexpr int gemm_smem() { return kGStages * (BM + BN) * kGRow * (int)sizeof(double); }
 
 __device__ __forceinline__ void cp_async8(double *smem, const double *gmem, bool pred) {
   const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
@@ -103,12 +104,13 @@ __device__ __forceinline__ void dmma_8x8x4(double d[2], double a, double b) {
                : "d"(a), "d"(b));
 }
 
-template <int BN>
-__global__ void __launch_bounds__(kGThreads, BN == 64 ? 2 : 1) gemm_f64_kernel(const GemmF64 g) {
-  constexpr int kGN = BN;
+template <int BM, int BN>
+__global__ void __launch_bounds__(kGThreads, BM * BN <= 8192 ? 2 : 1)
+    gemm_f64_kernel(const GemmF64 g) {
+  constexpr int kGM = BM, kGN = BN;
   constexpr int kWarpsN = BN / 32, kWarpsM = 8 / kWarpsN;
   constexpr int kTm = kGM / kWarpsM / 8, kTn = 4;  // 8x8 tiles per warp
-  constexpr int kBCopies = kGN * kGK / kGThreads;
+  constexpr int kACopies = kGM * kGK / kGThreads, kBCopies = kGN * kGK / kGThreads;
   const int64_t m0 = (int64_t)blockIdx.y * kGM, n0 = (int64_t)blockIdx.x * kGN;
   if (g.lower && n0 > m0 + kGM - 1) return;
   // operands arrive by cp.async (volatile asm, kept after the wait) and
@@ -130,8 +132,8 @@ __global__ void __launch_bounds__(kGThreads, BN == 64 ? 2 : 1) gemm_f64_kernel(c
   // their addresses and bounds come from a base, two steps and a row mask.
   const bool a_k_fast = g.sAk == 1 || g.sAk == -1;
   const bool b_k_fast = g.sBk == 1 || g.sBk == -1;
-  const int a_r0 = a_k_fast ? tid >> 4 : tid & (kGM - 1), a_k0 = a_k_fast ? tid & 15 : tid >> 7;
-  const int a_dr = a_k_fast ? 16 : 0, a_dk = a_k_fast ? 0 : 2;
+  const int a_r0 = a_k_fast ? tid >> 4 : tid & (kGM - 1), a_k0 = a_k_fast ? tid & 15 : tid / kGM;
+  const int a_dr = a_k_fast ? 16 : 0, a_dk = a_k_fast ? 0 : kGThreads / kGM;
   const int b_r0 = b_k_fast ? tid >> 4 : tid & (kGN - 1), b_k0 = b_k_fast ? tid & 15 : tid / kGN;
   const int b_dr = b_k_fast ? 16 : 0, b_dk = b_k_fast ? 0 : kGThreads / kGN;
   const double *a_base = A + (m0 + a_r0) * g.sAm + a_k0 * g.sAk;
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(kGThreads, BN == 64 ? 2 : 1) gemm_f64_kernel(c
   uint32_t a_rows = 0, b_rows = 0;  // bit e: row of copy e in range
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    a_rows |= (uint32_t)(m0 + a_r0 + e * a_dr < g.M) << e;
+    if (e < kACopies) a_rows |= (uint32_t)(m0 + a_r0 + e * a_dr < g.M) << e;
     if (e < kBCopies) b_rows |= (uint32_t)(n0 + b_r0 + e * b_dr < g.N) << e;
   }
   const int64_t nslab = (g.K + kGK - 1) / kGK;
@@ -156,8 +158,10 @@ __global__ void __launch_bounds__(kGThreads, BN == 64 ? 2 : 1) gemm_f64_kernel(c
       const double *pa = a_base + t * a_slab, *pb = b_base + t * b_slab;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const bool oka = ((a_rows >> e) & 1u) && k0 + a_k0 + e * a_dk < g.K;
-        cp_async8(as + e * a_sstep, oka ? pa + e * a_step : A, oka);
+        if (e < kACopies) {
+          const bool oka = ((a_rows >> e) & 1u) && k0 + a_k0 + e * a_dk < g.K;
+          cp_async8(as + e * a_sstep, oka ? pa + e * a_step : A, oka);
+        }
         if (e < kBCopies) {
           const bool okb = ((b_rows >> e) & 1u) && k0 + b_k0 + e * b_dk < g.K;
           cp_async8(bs + e * b_sstep, okb ? pb + e * b_step : B, okb);
@@ -221,16 +225,18 @@ __global__ void __launch_bounds__(kGThreads, BN == 64 ? 2 : 1) gemm_f64_kernel(c
 std::mutex g_gemm_attr_mu;
 bool g_gemm_attr[64] = {};
 
-template <int BN>
+template <int BM, int BN>
 cudaError_t gemm_launch(const GemmF64 &g, int64_t batch, cudaStream_t st) {
-  const dim3 grid((unsigned)((g.N + BN - 1) / BN), (unsigned)((g.M + kGM - 1) / kGM),
+  const dim3 grid((unsigned)((g.N + BN - 1) / BN), (unsigned)((g.M + BM - 1) / BM),
                   (unsigned)batch);
-  return launch_chained(gemm_f64_kernel<BN>, grid, dim3(kGThreads), gemm_smem<BN>(), st, g);
+  return launch_chained(gemm_f64_kernel<BM, BN>, grid, dim3(kGThreads), gemm_smem<BM, BN>(), st,
+                        g);
 }
 
 // An in-place product (C aliasing A, `overwrite`) must run as one CTA column
 // (N <= 128, 128-wide tiles): every CTA reads all of its rows' A before
-// writing them, and no other CTA touches those rows.
+// writing them, and no other CTA touches those rows.  Its tiles are 64 rows
+// high, so that the panel's rows spread over twice as many SMs.
 cudaError_t gemm_f64(const GemmF64 &g, int64_t batch, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return cudaSuccess;
   if (g.overwrite && g.N > 128) return cudaErrorInvalidValue;
@@ -241,11 +247,11 @@ cudaError_t gemm_f64(const GemmF64 &g, int64_t batch, cudaStream_t st) {
   {
     std::lock_guard<std::mutex> lk(g_gemm_attr_mu);
     if (!g_gemm_attr[dev]) {
-      e = cudaFuncSetAttribute(gemm_f64_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               gemm_smem<128>());
+      e = cudaFuncSetAttribute(gemm_f64_kernel<64, 128>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem<64, 128>());
       if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(gemm_f64_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gemm_smem<64>());
+        e = cudaFuncSetAttribute(gemm_f64_kernel<128, 64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem<128, 64>());
       if (e != cudaSuccess) return e;
       g_gemm_attr[dev] = true;
     }
@@ -253,8 +259,8 @@ cudaError_t gemm_f64(const GemmF64 &g, int64_t batch, cudaStream_t st) {
   // 128 x 64 tiles, two CTAs per SM, hide one tile's prologue and epilogue
   // behind the other's products (measured 8% faster on the dense layer's
   // GPTQ than 128 x 128 tiles, one CTA per SM)
-  if (g.overwrite) return gemm_launch<128>(g, batch, st);
-  return gemm_launch<64>(g, batch, st);
+  if (g.overwrite) return gemm_launch<64, 128>(g, batch, st);
+  return gemm_launch<128, 64>(g, batch, st);
 }
 
 // ------------------------------------------------------------------ Cholesky

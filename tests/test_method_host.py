@@ -160,6 +160,45 @@ def test_kernel_encode_rule_near_midpoints(oracle_mod):
     assert np.sum(_encode_rule(xs, ss, step=False) != ref) > 0
 
 
+def _gptq_select_round(x, s):
+    """The GPTQ column-block kernel's rounding of fp64 x at scale s: seven
+    compares of |x| against the midpoints times s (strict at 0.25, 1.25, 2.5,
+    5; inclusive at 0.75, 1.75, 3.5), NaN thresholds when s is 0 or not a
+    number, and a select chain over the grid values times s.  Returns the
+    signed code and the quantised value."""
+    tf = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+    vf = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+    thr = [t * s if s > 0.0 else float("nan") for t in tf]
+    val = [v * s for v in vf]
+    a = abs(x)
+    p = [a > thr[0], a >= thr[1], a > thr[2], a >= thr[3], a > thr[4], a >= thr[5], a > thr[6]]
+    qv = val[1] if p[0] else val[0]
+    for i in range(1, 7):
+        qv = val[i + 1] if p[i] else qv
+    k = sum(p)
+    neg = np.signbit(x)
+    return (8 if neg else 0) | k, (-qv if neg else qv)
+
+
+def test_gptq_select_rounding_equals_the_encode(oracle_mod):
+    """The select chain gives the oracle's E2M1 code, and the code's value
+    times s, on values at, one ulp either side of and between every
+    threshold at ordinary, tiny and huge scales, on signed zeros, on values
+    beyond saturation, and at a scale of 0 (index 0, the sign kept)."""
+    scales = [1.0, 0.0375, float(np.float32(3.1e-7)), 2.0 ** -120, 2.0 ** 100, 0.0]
+    mids = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+    for s in scales:
+        xs = [0.0, -0.0, 7.0 * max(s, 1.0), -6.5 * s, 0.1 * s, 1e30]
+        for m in mids:
+            t = m * s
+            xs += [t, np.nextafter(t, np.inf), np.nextafter(t, -np.inf), -t, t * 1.01, t * 0.99]
+        for x in xs:
+            code, qv = _gptq_select_round(float(x), s)
+            ref = oracle_mod.e2m1_encode(float(x), s)
+            assert code == ref, (x, s, code, ref)
+            assert qv == (-1.0 if ref & 8 else 1.0) * oracle_mod.e2m1_value(ref & 7) * s, (x, s)
+
+
 # ------------------------------------------------------ E4M3 scale code
 def _e4m3_rn_satfinite(t):
     """Nearest-even E4M3 code of the magnitude of fp32 t (codes 0..0x7E; above
